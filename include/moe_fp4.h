@@ -1,0 +1,180 @@
+/*
+ * moe_fp4.h -- C ABI of the NVFP4 sparse mixture-of-experts layer forward
+ * (libmoe_fp4.so, CUDA, sm_100a).
+ *
+ * The operation (one decoder layer's MoE block, forward only):
+ *   for each token t with activation x[t] (bf16, width d):
+ *     l[t,e]   = sum_i x[t,i] * Wr[e,i]                          fp32 router logits
+ *     S_t      = the top_k experts by l[t,:], ties to the lower index
+ *     w[t,j]   = softmax(l[t,:])[S_j] / sum_{S} softmax(l[t,:])  renormalised
+ *     out[t]   = bf16( sum_j w[t,j] * Wd[S_j] (SiLU(Wg[S_j] x) * (Wu[S_j] x)) )
+ *   with every expert matrix stored in NVFP4.
+ * Sources: "Optimizing Muse Spark Open on TPU v7 with SGLang-TorchTPU"
+ * (Background: 8 of 256 experts per token, NVFP4 experts with one scale per
+ * 16 values; section 5: the expert loop chosen by per-expert row count;
+ * section 8: gate/up, SwiGLU, down, a one-pass combine that writes every
+ * output row once) and "Optimizing Models to Be Fast at Codegen" (section 2:
+ * FP4 e2m1 weights with a per-16 block scale, unpacked in registers, a
+ * grouped GEMM over only the active experts).
+ *
+ * NVFP4 (canonical layout accepted by moe_fp4_load_experts), per expert and
+ * matrix, row-major:
+ *   q  uint8 [rows][K/2]  two e2m1 codes per byte, element 2i in the LOW nibble
+ *                         (bit 3 sign, bits 2-1 exponent with bias 1, bit 0 mantissa)
+ *   sf uint8 [rows][K/16] e4m3fn block scales, block i covers K elements 16i..16i+15
+ *   gs float              one fp32 tensor scale per (expert, matrix)
+ *   value[n][k] = e2m1(q[n][k]) * e4m3(sf[n][k/16]) * gs
+ *   gate, up: rows = f, K = d;   down: rows = d, K = f.
+ *
+ * Activation precision, chosen per expert by its row count n_e in the call:
+ *   n_e <  dense_threshold : x (bf16) and h = SiLU(g)*u stay unquantised
+ *                            (tensor-core inputs are fp16 after an exact
+ *                            power-of-two rescale of each x row);
+ *   n_e >= dense_threshold : x and h are quantised to NVFP4 along K with
+ *                            tensor scale 1.0 (sf = e4m3_rn(amax/6),
+ *                            q = e2m1_rn(v/sf), decisions in fp32) and the
+ *                            expert runs on block-scaled FP4 tensor cores.
+ *   The threshold defaults to 128 (environment MOE_FP4_DENSE_THRESHOLD at
+ *   create time, or moe_fp4_set_dense_threshold).
+ *
+ * Conventions
+ *   - Every call returns a moe_fp4_status and never aborts the process.
+ *   - Device pointers are plain CUDA device addresses of the current device;
+ *     the library never frees caller memory.  The handle owns all of its
+ *     own device memory (repacked experts + workspace) and frees it in
+ *     moe_fp4_destroy.
+ *   - A handle is bound to the device current at create time, is not
+ *     thread-safe, and must be used from one stream at a time.
+ *   - moe_fp4_forward is asynchronous on `stream`, performs no host
+ *     synchronisation, and allocates nothing once moe_fp4_reserve(max_T) has
+ *     sized the workspace for T <= max_T; under those conditions it can be
+ *     captured into a CUDA graph.  Results are deterministic: the same inputs
+ *     give bit-identical outputs.
+ *   - Kernel-side failures (an internal wait that exceeded its bound, a
+ *     numeric overflow of an fp16 intermediate, an unsupported expert class)
+ *     set a device error word; read it with moe_fp4_get_device_error after
+ *     synchronising the stream.
+ */
+#ifndef MOE_FP4_H
+#define MOE_FP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define MOE_FP4_API __attribute__((visibility("default")))
+#else
+#define MOE_FP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct moe_fp4 moe_fp4_t;
+
+typedef enum {
+  MOE_FP4_OK = 0,
+  MOE_FP4_ERR_INVALID_ARG = 1,    /* null pointer, negative T, aliasing, bad value */
+  MOE_FP4_ERR_UNSUPPORTED = 2,    /* shape outside the supported limits */
+  MOE_FP4_ERR_NOT_LOADED = 3,     /* forward before moe_fp4_load_experts */
+  MOE_FP4_ERR_CUDA = 4,           /* a CUDA runtime call failed */
+  MOE_FP4_ERR_OOM = 5,            /* device allocation failed */
+  MOE_FP4_ERR_DEVICE_TIMEOUT = 6, /* (device error word) a bounded wait expired */
+  MOE_FP4_ERR_NUMERIC = 7,        /* (device error word) fp16 intermediate overflowed */
+  MOE_FP4_ERR_CAPTURE = 8         /* workspace growth needed while the stream is capturing */
+} moe_fp4_status;
+
+/* Create a layer handle on the current device.
+ *   E       experts, 1..1024
+ *   top_k   experts per token, 1..min(E, 32)
+ *   d, f    model width and expert FFN width; multiples of 128, 128..16384
+ * On success *out receives the handle (caller destroys it). */
+MOE_FP4_API int moe_fp4_create(int E, int top_k, int d, int f, moe_fp4_t** out);
+
+/* Canonical NVFP4 expert weights (device pointers, caller-owned, read only
+ * during the call).  Layout as described at the top of this file:
+ *   gate_q, up_q   [E][f][d/2]     gate_sf, up_sf [E][f][d/16]   gate_gs, up_gs [E]
+ *   down_q         [E][d][f/2]     down_sf        [E][d][f/16]   down_gs        [E] */
+typedef struct {
+  const uint8_t* gate_q;
+  const uint8_t* gate_sf;
+  const float*   gate_gs;
+  const uint8_t* up_q;
+  const uint8_t* up_sf;
+  const float*   up_gs;
+  const uint8_t* down_q;
+  const uint8_t* down_sf;
+  const float*   down_gs;
+} moe_fp4_experts;
+
+/* Copy and repack the experts into library-owned device buffers (the
+ * register-dequant GEMV layout and the tensor-core block-scaled layout).
+ * Synchronous; may be called again to replace the weights. */
+MOE_FP4_API int moe_fp4_load_experts(moe_fp4_t* h, const moe_fp4_experts* w);
+
+/* Pre-size the workspace for up to max_T tokens per forward (allocates).
+ * After this, moe_fp4_forward with T <= max_T allocates nothing. */
+MOE_FP4_API int moe_fp4_reserve(moe_fp4_t* h, int max_T);
+
+/* The layer forward.
+ *   x_bf16    device, bf16 [T][d] row-major
+ *   T         tokens, >= 0 (T = 0 is a no-op)
+ *   router_w  device, fp32 [E][d] row-major
+ *   out_bf16  device, bf16 [T][d]; written completely, must not overlap x
+ *   stream    CUDA stream (0 = legacy default stream)
+ * Asynchronous on `stream`. */
+MOE_FP4_API int moe_fp4_forward(moe_fp4_t* h, const void* x_bf16, int T, const float* router_w,
+                    void* out_bf16, cudaStream_t stream);
+
+/* Intermediates of a forward, for layer-by-layer comparison.  Every member
+ * may be NULL; non-NULL members are device buffers the caller owns:
+ *   logits   fp32  [T][E]
+ *   topk_ids int32 [T][top_k]   listed by (logit desc, expert asc)
+ *   topk_w   fp32  [T][top_k]
+ *   counts   int32 [E]          pairs per expert
+ *   offsets  int32 [E+1]        exclusive scan of counts
+ *   perm     int32 [T*top_k]    perm[pos] = t*top_k + j, pairs sorted by (expert, t, j)
+ *   h        fp32  [T*top_k][f] SiLU(g)*u per pair, rows in perm order
+ *   partial  fp32  [T*top_k][d] w * (Wd h) per pair, rows in perm order
+ * Copies are enqueued on `stream` after the forward. */
+typedef struct {
+  float*   logits;
+  int32_t* topk_ids;
+  float*   topk_w;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* perm;
+  float*   h;
+  float*   partial;
+} moe_fp4_debug;
+
+MOE_FP4_API int moe_fp4_forward_ex(moe_fp4_t* h, const void* x_bf16, int T, const float* router_w,
+                       void* out_bf16, cudaStream_t stream, moe_fp4_debug* dbg);
+
+/* End-to-end variant taking HOST buffers: copies x (host bf16 [T][d]) to the
+ * device, runs the forward and copies the result back into out_host (host
+ * bf16 [T][d]), all on `stream`, then synchronises the stream.  Pinned host
+ * memory gives asynchronous copies; pageable memory works but is slower.
+ * router_w is a device pointer as in moe_fp4_forward. */
+MOE_FP4_API int moe_fp4_forward_host(moe_fp4_t* h, const void* x_host, int T, const float* router_w,
+                         void* out_host, cudaStream_t stream);
+
+/* Activation-precision threshold (see the top of this file); thr >= 1. */
+MOE_FP4_API int moe_fp4_set_dense_threshold(moe_fp4_t* h, int thr);
+
+/* Read and clear the device error word (synchronises the handle's device).
+ * *code receives MOE_FP4_OK or the first MOE_FP4_ERR_* a kernel recorded. */
+MOE_FP4_API int moe_fp4_get_device_error(moe_fp4_t* h, int* code);
+
+/* Static text for a status code. */
+MOE_FP4_API const char* moe_fp4_status_string(int status);
+
+/* Release every device buffer the handle owns; NULL is allowed. */
+MOE_FP4_API void moe_fp4_destroy(moe_fp4_t* h);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_FP4_H */

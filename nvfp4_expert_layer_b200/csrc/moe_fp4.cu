@@ -1,0 +1,454 @@
+// libmoe_fp4: C ABI of the NVFP4 sparse-MoE layer forward (see include/moe_fp4.h).
+//
+// Host side: argument checking, device buffers owned by the handle, and the
+// launch sequence of one forward:
+//   router (+ fp16 staging of x) -> top-k -> permutation / expert classes
+//   -> light gate/up + SwiGLU -> light down (x routing weight)
+//   -> [dense class on block-scaled FP4 tensor cores] -> combine / unpermute.
+// No host synchronisation happens inside moe_fp4_forward; the expert kernels
+// read the class lists the permutation kernel left on the device.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "moe_fp4.h"
+#include "ptx.cuh"
+#include "layout.cuh"
+#include "route.cuh"
+#include "light.cuh"
+#include "combine.cuh"
+
+namespace {
+
+constexpr int kSmallT = 256;          // router_small up to this many tokens
+constexpr int kLightRing = 6;         // bulk-copy stages per warp in the light kernel
+
+struct Workspace {
+  void* base = nullptr;
+  size_t bytes = 0;
+  int max_T = 0;
+  float* logits = nullptr;
+  int* ids = nullptr;
+  float* wts = nullptr;
+  int* counts = nullptr;
+  int* offsets = nullptr;
+  int* perm = nullptr;
+  int* inv = nullptr;
+  int4* light_jobs = nullptr;
+  int* n_light_jobs = nullptr;
+  int4* dense_list = nullptr;
+  int* n_dense = nullptr;
+  __half* x16 = nullptr;
+  float* xscale = nullptr;
+  float* h32 = nullptr;
+  __half* h16 = nullptr;
+  float* partial = nullptr;
+  uint16_t* xin = nullptr;     // host-API staging
+  uint16_t* xout = nullptr;
+};
+
+}  // namespace
+
+struct moe_fp4 {
+  int device = 0;
+  int E = 0, k = 0, d = 0, f = 0;
+  int thr = 128;
+  int sm_count = 0;
+  int light_blocks_per_sm = 1;
+  int64_t wait_timeout_ns = 2000000000LL;
+  bool loaded = false;
+  uint8_t* gu_frag = nullptr;     // gate/up fragment layout, all experts
+  uint8_t* dn_frag = nullptr;     // down fragment layout, all experts
+  float* gs = nullptr;            // [3][E]: gate, up, down
+  int* err = nullptr;             // device error word
+  Workspace ws;
+};
+
+namespace {
+
+#define MOE_CUDA(call)                                  \
+  do {                                                  \
+    cudaError_t e_ = (call);                            \
+    if (e_ != cudaSuccess) { (void)cudaGetLastError(); return MOE_FP4_ERR_CUDA; } \
+  } while (0)
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+template <typename T>
+T* carve(uint8_t*& cur, size_t count) {
+  T* p = reinterpret_cast<T*>(cur);
+  cur += align_up(count * sizeof(T), 256);
+  return p;
+}
+
+size_t workspace_bytes(const moe_fp4* h, int Tm) {
+  const size_t P = (size_t)Tm * h->k;
+  size_t b = 0;
+  auto add = [&](size_t n) { b += align_up(n, 256); };
+  add((size_t)Tm * h->E * 4);       // logits
+  add(P * 4);                       // ids
+  add(P * 4);                       // wts
+  add((size_t)h->E * 4);            // counts
+  add((size_t)(h->E + 1) * 4);      // offsets
+  add(P * 4);                       // perm
+  add(P * 4);                       // inv
+  add(((size_t)h->E + P / moe::kJobRows + 1) * 16);   // light jobs
+  add(4);
+  add((size_t)h->E * 16);           // dense list
+  add(4);
+  add((size_t)Tm * h->d * 2);       // x16
+  add((size_t)Tm * 4);              // xscale
+  add(P * h->f * 4);                // h32
+  add(P * h->f * 2);                // h16
+  add(P * h->d * 4);                // partial
+  add((size_t)Tm * h->d * 2);       // xin
+  add((size_t)Tm * h->d * 2);       // xout
+  return b;
+}
+
+int ensure_workspace(moe_fp4* h, int Tm, cudaStream_t stream) {
+  if (Tm <= h->ws.max_T && h->ws.base) return MOE_FP4_OK;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) == cudaSuccess && cs != cudaStreamCaptureStatusNone)
+    return MOE_FP4_ERR_CAPTURE;
+  if (h->ws.base) {
+    MOE_CUDA(cudaDeviceSynchronize());
+    cudaFree(h->ws.base);
+    h->ws = Workspace{};
+  }
+  const size_t bytes = workspace_bytes(h, Tm);
+  void* base = nullptr;
+  if (cudaMalloc(&base, bytes) != cudaSuccess) { (void)cudaGetLastError(); return MOE_FP4_ERR_OOM; }
+  Workspace w;
+  w.base = base;
+  w.bytes = bytes;
+  w.max_T = Tm;
+  const size_t P = (size_t)Tm * h->k;
+  uint8_t* cur = static_cast<uint8_t*>(base);
+  w.logits = carve<float>(cur, (size_t)Tm * h->E);
+  w.ids = carve<int>(cur, P);
+  w.wts = carve<float>(cur, P);
+  w.counts = carve<int>(cur, h->E);
+  w.offsets = carve<int>(cur, h->E + 1);
+  w.perm = carve<int>(cur, P);
+  w.inv = carve<int>(cur, P);
+  w.light_jobs = carve<int4>(cur, (size_t)h->E + P / moe::kJobRows + 1);
+  w.n_light_jobs = carve<int>(cur, 1);
+  w.dense_list = carve<int4>(cur, h->E);
+  w.n_dense = carve<int>(cur, 1);
+  w.x16 = carve<__half>(cur, (size_t)Tm * h->d);
+  w.xscale = carve<float>(cur, Tm);
+  w.h32 = carve<float>(cur, P * h->f);
+  w.h16 = carve<__half>(cur, P * h->f);
+  w.partial = carve<float>(cur, P * h->d);
+  w.xin = carve<uint16_t>(cur, (size_t)Tm * h->d);
+  w.xout = carve<uint16_t>(cur, (size_t)Tm * h->d);
+  h->ws = w;
+  return MOE_FP4_OK;
+}
+
+bool ranges_overlap(const void* a, size_t an, const void* b, size_t bn) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + bn && b0 < a0 + an;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                   bool pdl, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+size_t light_smem_bytes() {
+  return (size_t)moe::kLightWarps * kLightRing * moe::kStageBytes +
+         (size_t)moe::kLightWarps * kLightRing * 8 +
+         (size_t)moe::kLightWarps * moe::kLightNT * 32 * 4 * 4;
+}
+
+size_t permute_smem_bytes(int E) { return (size_t)(32 * E + 3 * E + 2) * 4; }
+
+int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cudaStream_t st) {
+  Workspace& w = h->ws;
+  const int E = h->E, k = h->k, d = h->d, f = h->f;
+  const uint16_t* xb = static_cast<const uint16_t*>(x);
+  // 1. router logits (+ fp16 staging of x)
+  if (T <= kSmallT) {
+    MOE_CUDA(launch(moe::router_small_kernel, dim3(E), dim3(256), (size_t)d * 4, st, false,
+                    xb, rw, T, d, E, w.logits, w.x16, w.xscale, h->err));
+  } else {
+    MOE_CUDA(launch(moe::router_tiled_kernel, dim3((T + 63) / 64, (E + 63) / 64), dim3(256), 0, st,
+                    false, xb, rw, T, d, E, w.logits));
+    MOE_CUDA(launch(moe::stage_x_kernel, dim3(std::min(T, 8 * h->sm_count)), dim3(256), 0, st, false,
+                    xb, T, d, w.x16, w.xscale, h->err));
+  }
+  // 2. top-k
+  MOE_CUDA(launch(moe::topk_kernel, dim3((T + 7) / 8), dim3(256), 0, st, false,
+                  (const float*)w.logits, T, E, k, w.ids, w.wts));
+  // 3. permutation and expert classes
+  moe::PermuteOut po{w.counts, w.offsets, w.perm, w.inv, w.light_jobs, w.n_light_jobs,
+                     w.dense_list, w.n_dense, h->err};
+  MOE_CUDA(launch(moe::permute_kernel, dim3(1), dim3(1024), permute_smem_bytes(E), st, false,
+                  (const int*)w.ids, T, k, E, h->thr, 0, po));
+  // 4. light gate/up + SwiGLU
+  const int grid = h->sm_count * h->light_blocks_per_sm;
+  moe::LightParams lp{};
+  lp.frag = h->gu_frag;
+  lp.tpe = f / 8;
+  lp.cpt = d / moe::kChunkK;
+  lp.jobs = w.light_jobs;
+  lp.njobs = w.n_light_jobs;
+  lp.perm = w.perm;
+  lp.topk = k;
+  lp.bsrc = w.x16;
+  lp.bk = d;
+  lp.xscale = w.xscale;
+  lp.gs0 = h->gs;
+  lp.gs1 = h->gs + E;
+  lp.wts = w.wts;
+  lp.h32 = w.h32;
+  lp.h16 = w.h16;
+  lp.f = f;
+  lp.partial = w.partial;
+  lp.d = d;
+  lp.err = h->err;
+  lp.wait_timeout_ns = h->wait_timeout_ns;
+  MOE_CUDA(launch(moe::light_expert_kernel<moe::kGateUp, kLightRing>, dim3(grid),
+                  dim3(moe::kLightThreads), light_smem_bytes(), st, true, lp));
+  // 5. light down (x routing weight)
+  moe::LightParams dp = lp;
+  dp.frag = h->dn_frag;
+  dp.tpe = d / 16;
+  dp.cpt = f / moe::kChunkK;
+  dp.bsrc = w.h16;
+  dp.bk = f;
+  dp.gs0 = h->gs + 2 * E;
+  dp.gs1 = nullptr;
+  MOE_CUDA(launch(moe::light_expert_kernel<moe::kDown, kLightRing>, dim3(grid),
+                  dim3(moe::kLightThreads), light_smem_bytes(), st, true, dp));
+  // 6. combine / unpermute
+  MOE_CUDA(launch(moe::combine_kernel, dim3((d + 1023) / 1024, T), dim3(128), 0, st, true,
+                  (const float*)w.partial, (const int*)w.inv, T, k, d,
+                  static_cast<uint16_t*>(out)));
+  return MOE_FP4_OK;
+}
+
+int check_forward_args(moe_fp4* h, const void* x, int T, const float* rw, const void* out) {
+  if (!h) return MOE_FP4_ERR_INVALID_ARG;
+  if (T < 0) return MOE_FP4_ERR_INVALID_ARG;
+  if (T == 0) return MOE_FP4_OK;
+  if (!x || !rw || !out) return MOE_FP4_ERR_INVALID_ARG;
+  if ((long long)T * h->k >= (1LL << 30)) return MOE_FP4_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(rw) |
+       reinterpret_cast<uintptr_t>(out)) & 15)
+    return MOE_FP4_ERR_INVALID_ARG;
+  const size_t xb = (size_t)T * h->d * 2;
+  if (ranges_overlap(x, xb, out, xb)) return MOE_FP4_ERR_INVALID_ARG;
+  if (!h->loaded) return MOE_FP4_ERR_NOT_LOADED;
+  return MOE_FP4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_fp4_status_string(int s) {
+  switch (s) {
+    case MOE_FP4_OK: return "ok";
+    case MOE_FP4_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_FP4_ERR_UNSUPPORTED: return "unsupported shape or expert class";
+    case MOE_FP4_ERR_NOT_LOADED: return "experts not loaded";
+    case MOE_FP4_ERR_CUDA: return "CUDA runtime error";
+    case MOE_FP4_ERR_OOM: return "device out of memory";
+    case MOE_FP4_ERR_DEVICE_TIMEOUT: return "device wait exceeded its bound";
+    case MOE_FP4_ERR_NUMERIC: return "fp16 intermediate overflow or non-finite input";
+    case MOE_FP4_ERR_CAPTURE: return "workspace growth needed during stream capture";
+    default: return "unknown status";
+  }
+}
+
+int moe_fp4_create(int E, int top_k, int d, int f, moe_fp4_t** out) {
+  if (!out) return MOE_FP4_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (E < 1 || E > 1024) return MOE_FP4_ERR_UNSUPPORTED;
+  if (top_k < 1 || top_k > std::min(E, 32)) return MOE_FP4_ERR_UNSUPPORTED;
+  if (d < 128 || f < 128 || d > 16384 || f > 16384 || d % 128 || f % 128)
+    return MOE_FP4_ERR_UNSUPPORTED;
+  moe_fp4* h = new (std::nothrow) moe_fp4();
+  if (!h) return MOE_FP4_ERR_OOM;
+  h->E = E; h->k = top_k; h->d = d; h->f = f;
+  if (const char* s = std::getenv("MOE_FP4_DENSE_THRESHOLD")) {
+    const int v = std::atoi(s);
+    if (v >= 1) h->thr = v;
+  }
+  if (const char* s = std::getenv("MOE_FP4_WAIT_TIMEOUT_MS")) {
+    const long long v = std::atoll(s);
+    if (v >= 1) h->wait_timeout_ns = v * 1000000LL;
+  }
+  int rc = MOE_FP4_OK;
+  do {
+    if (cudaGetDevice(&h->device) != cudaSuccess) { rc = MOE_FP4_ERR_CUDA; break; }
+    if (cudaDeviceGetAttribute(&h->sm_count, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess) {
+      rc = MOE_FP4_ERR_CUDA; break;
+    }
+    const size_t ls = light_smem_bytes();
+    if (cudaFuncSetAttribute(moe::light_expert_kernel<moe::kGateUp, kLightRing>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ls) != cudaSuccess ||
+        cudaFuncSetAttribute(moe::light_expert_kernel<moe::kDown, kLightRing>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ls) != cudaSuccess ||
+        cudaFuncSetAttribute(moe::router_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             d * 4) != cudaSuccess ||
+        cudaFuncSetAttribute(moe::permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)permute_smem_bytes(E)) != cudaSuccess) {
+      rc = MOE_FP4_ERR_CUDA; break;
+    }
+    int nb = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &nb, moe::light_expert_kernel<moe::kGateUp, kLightRing>, moe::kLightThreads, ls) != cudaSuccess) {
+      rc = MOE_FP4_ERR_CUDA; break;
+    }
+    h->light_blocks_per_sm = std::max(1, nb);
+    if (cudaMalloc(&h->err, sizeof(int)) != cudaSuccess) { rc = MOE_FP4_ERR_OOM; break; }
+    if (cudaMemset(h->err, 0, sizeof(int)) != cudaSuccess) { rc = MOE_FP4_ERR_CUDA; break; }
+    if (cudaMalloc(&h->gs, sizeof(float) * 3 * E) != cudaSuccess) { rc = MOE_FP4_ERR_OOM; break; }
+  } while (0);
+  if (rc != MOE_FP4_OK) {
+    (void)cudaGetLastError();
+    moe_fp4_destroy(h);
+    return rc;
+  }
+  *out = h;
+  return MOE_FP4_OK;
+}
+
+void moe_fp4_destroy(moe_fp4_t* h) {
+  if (!h) return;
+  cudaDeviceSynchronize();
+  cudaFree(h->gu_frag);
+  cudaFree(h->dn_frag);
+  cudaFree(h->gs);
+  cudaFree(h->err);
+  cudaFree(h->ws.base);
+  (void)cudaGetLastError();
+  delete h;
+}
+
+int moe_fp4_load_experts(moe_fp4_t* h, const moe_fp4_experts* w) {
+  if (!h || !w) return MOE_FP4_ERR_INVALID_ARG;
+  if (!w->gate_q || !w->gate_sf || !w->gate_gs || !w->up_q || !w->up_sf || !w->up_gs ||
+      !w->down_q || !w->down_sf || !w->down_gs)
+    return MOE_FP4_ERR_INVALID_ARG;
+  const int E = h->E, d = h->d, f = h->f;
+  const size_t gu_bytes = (size_t)E * (f / 8) * (d / moe::kChunkK) * moe::kChunkBytes;
+  const size_t dn_bytes = (size_t)E * (d / 16) * (f / moe::kChunkK) * moe::kChunkBytes;
+  if (!h->gu_frag) {
+    if (cudaMalloc(&h->gu_frag, gu_bytes) != cudaSuccess) { (void)cudaGetLastError(); return MOE_FP4_ERR_OOM; }
+  }
+  if (!h->dn_frag) {
+    if (cudaMalloc(&h->dn_frag, dn_bytes) != cudaSuccess) { (void)cudaGetLastError(); return MOE_FP4_ERR_OOM; }
+  }
+  h->loaded = false;
+  MOE_CUDA(cudaDeviceSynchronize());
+  {
+    const long long thr = (long long)E * (f / 8) * (d / moe::kChunkK) * 32;
+    const int blocks = (int)std::min<long long>((thr + 255) / 256, 65535LL * 16);
+    moe::repack_fragment_kernel<moe::kGateUp><<<blocks, 256>>>(w->gate_q, w->gate_sf, w->up_q, w->up_sf,
+                                                              E, f, d, h->gu_frag);
+    MOE_CUDA(cudaGetLastError());
+  }
+  {
+    const long long thr = (long long)E * (d / 16) * (f / moe::kChunkK) * 32;
+    const int blocks = (int)std::min<long long>((thr + 255) / 256, 65535LL * 16);
+    moe::repack_fragment_kernel<moe::kDown><<<blocks, 256>>>(w->down_q, w->down_sf, nullptr, nullptr,
+                                                            E, d, f, h->dn_frag);
+    MOE_CUDA(cudaGetLastError());
+  }
+  MOE_CUDA(cudaMemcpy(h->gs, w->gate_gs, sizeof(float) * E, cudaMemcpyDeviceToDevice));
+  MOE_CUDA(cudaMemcpy(h->gs + E, w->up_gs, sizeof(float) * E, cudaMemcpyDeviceToDevice));
+  MOE_CUDA(cudaMemcpy(h->gs + 2 * E, w->down_gs, sizeof(float) * E, cudaMemcpyDeviceToDevice));
+  MOE_CUDA(cudaDeviceSynchronize());
+  h->loaded = true;
+  return MOE_FP4_OK;
+}
+
+int moe_fp4_reserve(moe_fp4_t* h, int max_T) {
+  if (!h || max_T < 1) return MOE_FP4_ERR_INVALID_ARG;
+  if ((long long)max_T * h->k >= (1LL << 30)) return MOE_FP4_ERR_UNSUPPORTED;
+  return ensure_workspace(h, max_T, nullptr);
+}
+
+int moe_fp4_set_dense_threshold(moe_fp4_t* h, int thr) {
+  if (!h || thr < 1) return MOE_FP4_ERR_INVALID_ARG;
+  h->thr = thr;
+  return MOE_FP4_OK;
+}
+
+int moe_fp4_forward(moe_fp4_t* h, const void* x, int T, const float* rw, void* out,
+                    cudaStream_t stream) {
+  int rc = check_forward_args(h, x, T, rw, out);
+  if (rc != MOE_FP4_OK || T == 0) return rc;
+  rc = ensure_workspace(h, T, stream);
+  if (rc != MOE_FP4_OK) return rc;
+  return run_forward(h, x, T, rw, out, stream);
+}
+
+int moe_fp4_forward_ex(moe_fp4_t* h, const void* x, int T, const float* rw, void* out,
+                       cudaStream_t stream, moe_fp4_debug* dbg) {
+  int rc = moe_fp4_forward(h, x, T, rw, out, stream);
+  if (rc != MOE_FP4_OK || T == 0 || !dbg) return rc;
+  const Workspace& w = h->ws;
+  const size_t P = (size_t)T * h->k;
+  auto cp = [&](void* dst, const void* src, size_t bytes) -> int {
+    if (!dst) return MOE_FP4_OK;
+    MOE_CUDA(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, stream));
+    return MOE_FP4_OK;
+  };
+  if ((rc = cp(dbg->logits, w.logits, (size_t)T * h->E * 4))) return rc;
+  if ((rc = cp(dbg->topk_ids, w.ids, P * 4))) return rc;
+  if ((rc = cp(dbg->topk_w, w.wts, P * 4))) return rc;
+  if ((rc = cp(dbg->counts, w.counts, (size_t)h->E * 4))) return rc;
+  if ((rc = cp(dbg->offsets, w.offsets, (size_t)(h->E + 1) * 4))) return rc;
+  if ((rc = cp(dbg->perm, w.perm, P * 4))) return rc;
+  if ((rc = cp(dbg->h, w.h32, P * h->f * 4))) return rc;
+  if ((rc = cp(dbg->partial, w.partial, P * h->d * 4))) return rc;
+  return MOE_FP4_OK;
+}
+
+int moe_fp4_forward_host(moe_fp4_t* h, const void* x_host, int T, const float* rw, void* out_host,
+                         cudaStream_t stream) {
+  if (!h || T < 0) return MOE_FP4_ERR_INVALID_ARG;
+  if (T == 0) return MOE_FP4_OK;
+  if (!x_host || !out_host || !rw) return MOE_FP4_ERR_INVALID_ARG;
+  if (!h->loaded) return MOE_FP4_ERR_NOT_LOADED;
+  int rc = ensure_workspace(h, T, stream);
+  if (rc != MOE_FP4_OK) return rc;
+  const size_t bytes = (size_t)T * h->d * 2;
+  MOE_CUDA(cudaMemcpyAsync(h->ws.xin, x_host, bytes, cudaMemcpyHostToDevice, stream));
+  rc = moe_fp4_forward(h, h->ws.xin, T, rw, h->ws.xout, stream);
+  if (rc != MOE_FP4_OK) return rc;
+  MOE_CUDA(cudaMemcpyAsync(out_host, h->ws.xout, bytes, cudaMemcpyDeviceToHost, stream));
+  MOE_CUDA(cudaStreamSynchronize(stream));
+  return MOE_FP4_OK;
+}
+
+int moe_fp4_get_device_error(moe_fp4_t* h, int* code) {
+  if (!h || !code) return MOE_FP4_ERR_INVALID_ARG;
+  MOE_CUDA(cudaDeviceSynchronize());
+  MOE_CUDA(cudaMemcpy(code, h->err, sizeof(int), cudaMemcpyDeviceToHost));
+  MOE_CUDA(cudaMemset(h->err, 0, sizeof(int)));
+  return MOE_FP4_OK;
+}
+
+}  // extern "C"

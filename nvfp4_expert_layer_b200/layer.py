@@ -1,0 +1,124 @@
+"""Python binding of the NVFP4 sparse-MoE layer (argument marshalling only).
+
+PyTorch supplies device memory and the stream; every step of the forward runs
+in libmoe_fp4.so's CUDA kernels."""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+
+EXPERT_FIELDS = ("gate_q", "gate_sf", "gate_gs", "up_q", "up_sf", "up_gs",
+                 "down_q", "down_sf", "down_gs")
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class MoeFp4Layer:
+    """Handle of one layer: MoeFp4Layer(E, top_k, d, f) on the current device."""
+
+    def __init__(self, E: int, top_k: int, d: int, f: int):
+        self.lib = _lib.load()
+        self.E, self.k, self.d, self.f = E, top_k, d, f
+        h = ctypes.c_void_p()
+        _lib.check(self.lib.moe_fp4_create(E, top_k, d, f, ctypes.byref(h)), "moe_fp4_create")
+        self._h = h
+
+    # ------------------------------------------------------------------ setup
+    def load_experts(self, experts: dict) -> None:
+        """experts: canonical device tensors (uint8 q/sf, float32 gs), see moe_fp4.h."""
+        s = _lib.Experts()
+        for n in EXPERT_FIELDS:
+            t = experts[n]
+            if not t.is_cuda or not t.is_contiguous():
+                raise ValueError(f"{n} must be a contiguous CUDA tensor")
+            setattr(s, n, t.data_ptr())
+        _lib.check(self.lib.moe_fp4_load_experts(self._h, ctypes.byref(s)), "moe_fp4_load_experts")
+
+    def reserve(self, max_T: int) -> None:
+        _lib.check(self.lib.moe_fp4_reserve(self._h, max_T), "moe_fp4_reserve")
+
+    def set_dense_threshold(self, thr: int) -> None:
+        _lib.check(self.lib.moe_fp4_set_dense_threshold(self._h, thr), "moe_fp4_set_dense_threshold")
+
+    def device_error(self) -> int:
+        code = ctypes.c_int(0)
+        _lib.check(self.lib.moe_fp4_get_device_error(self._h, ctypes.byref(code)),
+                   "moe_fp4_get_device_error")
+        return code.value
+
+    # ---------------------------------------------------------------- forward
+    def _out(self, x, out):
+        if out is None:
+            out = torch.empty_like(x)
+        return out
+
+    def forward(self, x: torch.Tensor, router_w: torch.Tensor, out=None, stream=None):
+        out = self._out(x, out)
+        T = x.shape[0] if x.dim() == 2 else 0
+        _lib.check(self.lib.moe_fp4_forward(self._h, _ptr(x), T, _ptr(router_w), _ptr(out),
+                                            _stream_ptr(stream)), "moe_fp4_forward")
+        return out
+
+    __call__ = forward
+
+    def forward_ex(self, x: torch.Tensor, router_w: torch.Tensor, out=None, stream=None,
+                   want=("logits", "topk_ids", "topk_w", "counts", "offsets", "perm", "h",
+                         "partial")):
+        out = self._out(x, out)
+        T = x.shape[0]
+        P = T * self.k
+        dev = x.device
+        shapes = {"logits": ((T, self.E), torch.float32), "topk_ids": ((T, self.k), torch.int32),
+                  "topk_w": ((T, self.k), torch.float32), "counts": ((self.E,), torch.int32),
+                  "offsets": ((self.E + 1,), torch.int32), "perm": ((P,), torch.int32),
+                  "h": ((P, self.f), torch.float32), "partial": ((P, self.d), torch.float32)}
+        bufs = {n: torch.full(shapes[n][0], float("nan") if shapes[n][1] == torch.float32 else -1,
+                              dtype=shapes[n][1], device=dev) for n in want}
+        dbg = _lib.Debug()
+        for n, t in bufs.items():
+            setattr(dbg, n, t.data_ptr())
+        _lib.check(self.lib.moe_fp4_forward_ex(self._h, _ptr(x), T, _ptr(router_w), _ptr(out),
+                                               _stream_ptr(stream), ctypes.byref(dbg)),
+                   "moe_fp4_forward_ex")
+        return out, bufs
+
+    def forward_host(self, x_host: torch.Tensor, router_w: torch.Tensor, out_host=None,
+                     stream=None):
+        """x_host / out_host: CPU bf16 tensors (pinned for asynchronous copies)."""
+        if out_host is None:
+            out_host = torch.empty_like(x_host, pin_memory=x_host.is_pinned())
+        _lib.check(self.lib.moe_fp4_forward_host(self._h, _ptr(x_host), x_host.shape[0],
+                                                 _ptr(router_w), _ptr(out_host),
+                                                 _stream_ptr(stream)), "moe_fp4_forward_host")
+        return out_host
+
+    # -------------------------------------------------------------- lifetime
+    def close(self) -> None:
+        if getattr(self, "_h", None) is not None and self._h.value:
+            self.lib.moe_fp4_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def experts_to_device(ex, device="cuda") -> dict:
+    """Upload workloads.ExpertWeights (numpy) as canonical device tensors."""
+    out = {}
+    for n in EXPERT_FIELDS:
+        a = getattr(ex, n)
+        out[n] = torch.from_numpy(a).to(device)
+    return out

@@ -1,0 +1,133 @@
+"""GPU parity: the CUDA layer against the oracle on seeded inputs (B200)."""
+import numpy as np
+import pytest
+import torch
+
+from nvfp4_expert_layer_b200 import workloads as W
+from nvfp4_expert_layer_b200.layer import MoeFp4Layer, experts_to_device
+from oracle import moe_oracle as O
+from tests.parity import Case, to_dev_x, bf16_to_bits
+
+pytestmark = pytest.mark.gpu
+
+
+def test_tiny_layer_full_parity():
+    Case(W.CONFIGS["tiny"]).run_gpu().run_oracle().check_all()
+
+
+@pytest.mark.parametrize("T", [1, 3, 17, 40])
+def test_ragged_small_layers(T):
+    cfg = W.custom_config(T=T, d=256, E=16, k=4, f=128, seed=10 + T, router="unit")
+    Case(cfg).run_gpu().run_oracle().check_all()
+
+
+def test_job_split_boundaries():
+    # E=2, k=1, T=49: expert loads straddle the 16-row job size (16, 17, 32, 33 ...)
+    cfg = W.custom_config(T=49, d=256, E=2, k=1, f=256, seed=5, router="unit")
+    c = Case(cfg).run_gpu().run_oracle()
+    assert c.o["counts"].max() > 16
+    c.check_all()
+
+
+def test_single_expert_top1():
+    cfg = W.custom_config(T=5, d=128, E=1, k=1, f=128, seed=9)
+    Case(cfg).run_gpu().run_oracle().check_all()
+
+
+def test_all_experts_selected():
+    cfg = W.custom_config(T=6, d=256, E=4, k=4, f=128, seed=12)
+    Case(cfg).run_gpu().run_oracle().check_all()
+
+
+def test_tiled_router_path():
+    # T > 256 takes the tiled router + separate x staging
+    cfg = W.custom_config(T=300, d=256, E=32, k=2, f=128, seed=13, router="unit")
+    Case(cfg).run_gpu().run_oracle().check_all()
+
+
+def test_decode1_full_size():
+    cfg = W.CONFIGS["decode1"]
+    Case(cfg).run_gpu().run_oracle().check_all()
+
+
+def test_decode64_full_size():
+    cfg = W.CONFIGS["decode64"]
+    Case(cfg).run_gpu().run_oracle().check_all()
+
+
+def test_verify_sampled_tokens():
+    cfg = W.CONFIGS["verify"]
+    Case(cfg, token_subset=[0, 1, 2, 3, 61, 127]).run_gpu().run_oracle().check_all()
+
+
+def test_deterministic_repeat():
+    cfg = W.custom_config(T=33, d=512, E=8, k=2, f=256, seed=21, router="unit")
+    x, rw = W.gen_x_router(cfg)
+    ex = W.gen_experts(cfg)
+    layer = MoeFp4Layer(cfg.E, cfg.k, cfg.d, cfg.f)
+    layer.load_experts(experts_to_device(ex))
+    xd, rwd = to_dev_x(x), torch.from_numpy(rw).cuda()
+    a = bf16_to_bits(layer(xd, rwd))
+    b = bf16_to_bits(layer(xd, rwd))
+    assert np.array_equal(a, b)
+
+
+def test_zero_tokens_is_a_noop():
+    cfg = W.CONFIGS["tiny"]
+    layer = MoeFp4Layer(cfg.E, cfg.k, cfg.d, cfg.f)
+    x = torch.empty((0, cfg.d), dtype=torch.bfloat16, device="cuda")
+    out = layer(x, torch.zeros((cfg.E, cfg.d), device="cuda"))
+    assert out.shape == (0, cfg.d)
+
+
+def test_forward_before_load_and_bad_args():
+    from nvfp4_expert_layer_b200._lib import MoeFp4Error, STATUS_CODE
+    cfg = W.CONFIGS["tiny"]
+    layer = MoeFp4Layer(cfg.E, cfg.k, cfg.d, cfg.f)
+    x = torch.zeros((4, cfg.d), dtype=torch.bfloat16, device="cuda")
+    rw = torch.zeros((cfg.E, cfg.d), device="cuda")
+    with pytest.raises(MoeFp4Error) as ei:
+        layer(x, rw)
+    assert ei.value.status == STATUS_CODE["MOE_FP4_ERR_NOT_LOADED"]
+    layer.load_experts(experts_to_device(W.gen_experts(cfg)))
+    with pytest.raises(MoeFp4Error) as ei:
+        layer(x, rw, out=x)                       # out aliases x
+    assert ei.value.status == STATUS_CODE["MOE_FP4_ERR_INVALID_ARG"]
+    xs = torch.zeros((4 * cfg.d + 8,), dtype=torch.bfloat16, device="cuda")[4:4 + 4 * cfg.d]
+    with pytest.raises(MoeFp4Error) as ei:
+        layer(xs.view(4, cfg.d), rw)              # 8-byte offset: not 16-byte aligned
+    assert ei.value.status == STATUS_CODE["MOE_FP4_ERR_INVALID_ARG"]
+    with pytest.raises(MoeFp4Error):
+        layer.set_dense_threshold(0)
+
+
+def test_forward_host_matches_device_forward():
+    cfg = W.custom_config(T=9, d=512, E=8, k=2, f=256, seed=31, router="unit")
+    x, rw = W.gen_x_router(cfg)
+    layer = MoeFp4Layer(cfg.E, cfg.k, cfg.d, cfg.f)
+    layer.load_experts(experts_to_device(W.gen_experts(cfg)))
+    rwd = torch.from_numpy(rw).cuda()
+    dev = bf16_to_bits(layer(to_dev_x(x), rwd))
+    xh = torch.from_numpy(x.view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+    host = layer.forward_host(xh, rwd)
+    assert np.array_equal(host.view(torch.int16).numpy().view(np.uint16), dev)
+
+
+def test_graph_capture_after_reserve():
+    cfg = W.custom_config(T=12, d=512, E=8, k=2, f=256, seed=41, router="unit")
+    x, rw = W.gen_x_router(cfg)
+    layer = MoeFp4Layer(cfg.E, cfg.k, cfg.d, cfg.f)
+    layer.load_experts(experts_to_device(W.gen_experts(cfg)))
+    layer.reserve(cfg.T)
+    xd, rwd = to_dev_x(x), torch.from_numpy(rw).cuda()
+    ref = bf16_to_bits(layer(xd, rwd))
+    out = torch.empty_like(xd)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            layer(xd, rwd, out=out, stream=s)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    assert np.array_equal(bf16_to_bits(out), ref)
