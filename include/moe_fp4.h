@@ -164,6 +164,18 @@ MOE_FP4_API int moe_fp4_forward_host(moe_fp4_t* h, const void* x_host, int T, co
 /* Activation-precision threshold (see the top of this file); thr >= 1. */
 MOE_FP4_API int moe_fp4_set_dense_threshold(moe_fp4_t* h, int thr);
 
+/* Stage timing (profiling hook).  With n = 7, every later forward records
+ * events[0] before the router, events[1] after the router (and x staging),
+ * events[2] after top-k, events[3] after the permutation, events[4] after the
+ * gate/up + SwiGLU kernels, events[5] after the down kernels and events[6]
+ * after the combine, all on the forward's stream (as external event nodes
+ * when the stream is being captured into a CUDA graph).  The events must be
+ * created with timing enabled; the caller owns them.  n = 0 (events may be
+ * NULL) turns the hook off.  Any other n is MOE_FP4_ERR_INVALID_ARG.
+ * Recording between stages serialises kernels that would otherwise overlap
+ * through programmatic dependent launch. */
+MOE_FP4_API int moe_fp4_set_stage_events(moe_fp4_t* h, cudaEvent_t* events, int n);
+
 /* Read and clear the device error word (synchronises the handle's device).
  * *code receives MOE_FP4_OK or the first MOE_FP4_ERR_* a kernel recorded. */
 MOE_FP4_API int moe_fp4_get_device_error(moe_fp4_t* h, int* code);

@@ -19,12 +19,27 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
   const int col = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
   if (t < T && col < d) {
     float s[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int j = 0; j < k; ++j) {
-      const float* src = partial + (size_t)inv[(size_t)t * k + j] * d + col;
-      const float4 a = *reinterpret_cast<const float4*>(src);
-      const float4 b = *reinterpret_cast<const float4*>(src + 4);
-      s[0] += a.x; s[1] += a.y; s[2] += a.z; s[3] += a.w;
-      s[4] += b.x; s[5] += b.y; s[6] += b.z; s[7] += b.w;
+    // slots in groups of 8: all index loads, then all row loads, then the sums
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      int pos[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) pos[q] = j0 + q < k ? inv[(size_t)t * k + j0 + q] : -1;
+      float4 a[8], b[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (pos[q] >= 0) {
+          const float* src = partial + (size_t)pos[q] * d + col;
+          a[q] = *reinterpret_cast<const float4*>(src);
+          b[q] = *reinterpret_cast<const float4*>(src + 4);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (pos[q] >= 0) {
+          s[0] += a[q].x; s[1] += a[q].y; s[2] += a[q].z; s[3] += a[q].w;
+          s[4] += b[q].x; s[5] += b[q].y; s[6] += b[q].z; s[7] += b[q].w;
+        }
+      }
     }
     uint4 o;
     uint32_t* ow = reinterpret_cast<uint32_t*>(&o);

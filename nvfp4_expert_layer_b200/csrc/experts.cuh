@@ -1,0 +1,444 @@
+// Light-class expert phase as one persistent kernel: gate/up + SwiGLU, down
+// (x routing weight) and the combine / unpermute, for every job whose expert
+// received fewer rows than the dense threshold.
+//
+// The weights stay 4-bit in HBM and shared memory; each warp unpacks e2m1
+// codes and their e4m3 block scales in registers into exact fp16 MMA operands
+// ("Optimizing Models to Be Fast at Codegen", section 2: stream the packed
+// weights through TMA, unpack e2m1 and the per-16 block scale in registers, a
+// grouped GEMM over only the active experts, a persistent kernel so every SM
+// stays busy at batch 1, split-K to fill the machine) and multiplies them with
+// up to 16 token rows on m16n8k16 tensor-core MMAs.
+//
+// One uninterrupted weight stream ("Optimizing Muse Spark Open on TPU v7 with
+// SGLang-TorchTPU", section 1-2: a decode step should be one stream of weights
+// with every transfer in flight before it is needed): block b owns tiles
+// b, b + G, b + 2G, ... of one list that holds every gate/up tile followed by
+// every down tile.  A warp's bulk-copy ring therefore runs straight from its
+// gate/up tiles into its down tiles, so down weights are fetched while other
+// blocks finish gate/up.  A down tile waits (bounded) for the gate/up tiles of
+// its job through a per-job completion counter before it reads h.
+//
+// Tile = 16 weight rows of one job over the full K.  The 4 warps of a block
+// split K into quarters and meet in shared memory at the end of the tile
+// (split-K inside the block).  Gate/up tile t pairs gate rows f = 8t+g with up
+// rows 8t+g, so one accumulator holds g and u of the same f and the SwiGLU
+// epilogue stays in registers.
+//
+// Combine (section 8 of the Muse Spark page: a one-pass combine; every output
+// row written once, no zero fill): every down tile adds its row count to the
+// counter of its 16-row output slice; the block that completes a slice sums
+// the k partials of every token in slot order and writes bf16 once.
+//
+// Counters reset themselves: the combining block clears its slice counter and
+// the last block to leave clears the per-job counters, so a CUDA graph can
+// replay the kernel without a memset.  The permutation kernel guarantees that
+// every job has 1..16 rows.
+#pragma once
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include "ptx.cuh"
+#include "layout.cuh"
+
+namespace moe {
+
+constexpr int kExpWarps = 4;
+constexpr int kExpThreads = kExpWarps * 32;
+constexpr int kExpSC = 4;          // 64-wide K chunks per bulk-copy stage (2304 bytes)
+constexpr int kExpRing = 6;        // stages in flight per warp
+constexpr int kExpSB = kExpSC * kChunkBytes;
+
+struct ExpertParams {
+  const uint8_t* gu_frag;     // gate/up fragment layout [E][f/8 tiles][d/64 chunks]
+  const uint8_t* dn_frag;     // down fragment layout    [E][d/16 tiles][f/64 chunks]
+  int tpe_gu, cpt_gu;         // f/8, d/64
+  int tpe_dn, cpt_dn;         // d/16, f/64
+  const int4* jobs;           // {expert, row0, nrows, 0}, 1 <= nrows <= 16
+  const int* njobs;
+  const int* n_dense;         // dense experts present -> combine is left to a later kernel
+  const int* perm;            // pair index per permuted row
+  const int* inv;             // permuted row per pair
+  int topk, T, d, f, E;
+  const __half* x16;          // [T][d] B-fragment layout, x * 2^s
+  const float* xscale;        // [T] 2^-s
+  __half* h16;                // [P][f] B-fragment layout
+  float* h32;                 // [P][f]
+  const float* gs;            // [3][E] gate, up, down tensor scales
+  const float* wts;           // [P] routing weight per pair
+  float* partial;             // [P][d]
+  uint16_t* out;              // [T][d] bf16
+  int* gu_done;               // [max jobs] gate/up tiles finished per job
+  int* dn_done;               // [d/16] pairs finished per output slice
+  int* exit_cnt;              // blocks that left
+  int* err;
+  int64_t wait_timeout_ns;
+};
+
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint4 ldg_cg_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ float4 ldg_cg_f4(const float* p) {
+  float4 v;
+  asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p));
+  return v;
+}
+
+// Everything a warp needs to know about one tile of the list.
+struct TileInfo {
+  int down;       // 0 gate/up, 1 down
+  int job, t;     // job index, tile index within the expert
+  int e, row0, nrows;
+  int cpt;        // chunks per tile
+  int slo, nw;    // this warp's first stage and stage count
+  const uint8_t* base;
+};
+
+__device__ __forceinline__ TileInfo tile_info(const ExpertParams& p, int i, int ngu, int warp) {
+  TileInfo ti;
+  ti.down = i >= ngu;
+  const int tpe = ti.down ? p.tpe_dn : p.tpe_gu;
+  const int li = ti.down ? i - ngu : i;
+  ti.job = li / tpe;
+  ti.t = li - ti.job * tpe;
+  const int4 jb = p.jobs[ti.job];
+  ti.e = jb.x;
+  ti.row0 = jb.y;
+  ti.nrows = jb.z;
+  ti.cpt = ti.down ? p.cpt_dn : p.cpt_gu;
+  const int spt = (ti.cpt + kExpSC - 1) / kExpSC;
+  ti.slo = warp * spt / kExpWarps;
+  ti.nw = (warp + 1) * spt / kExpWarps - ti.slo;
+  ti.base = (ti.down ? p.dn_frag : p.gu_frag) + (size_t)((size_t)ti.e * tpe + ti.t) * ti.cpt * kChunkBytes;
+  return ti;
+}
+
+// Activation fragments of one stage for this lane (NT n-tiles x 4 chunks).
+template <int NT>
+struct BFrag {
+  uint4 v[NT][kExpSC][2];
+};
+
+template <int NT, bool COHERENT>
+__device__ __forceinline__ void load_bfrag(BFrag<NT>& b, const __half* const (&row)[2], int chunk0,
+                                           int nch, int c) {
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int ch = 0; ch < kExpSC; ++ch) {
+      if (row[nt] != nullptr && ch < nch) {
+        const __half* bp = row[nt] + (size_t)(chunk0 + ch) * kChunkK + c * 16;
+        b.v[nt][ch][0] = COHERENT ? ldg_cg_v4(bp) : ldg_nc_v4(bp);
+        b.v[nt][ch][1] = COHERENT ? ldg_cg_v4(bp + 8) : ldg_nc_v4(bp + 8);
+      } else {
+        b.v[nt][ch][0] = make_uint4(0, 0, 0, 0);
+        b.v[nt][ch][1] = make_uint4(0, 0, 0, 0);
+      }
+    }
+}
+
+// One stage of shared-memory weights times the lane's activation fragments.
+template <int NT>
+__device__ __forceinline__ void mma_stage(uint32_t st, int nch, int lane, int g, const BFrag<NT>& b,
+                                          int nrows, float (&acc)[4][2][4]) {
+#pragma unroll
+  for (int ch = 0; ch < kExpSC; ++ch) {
+    if (ch < nch) {
+      const uint4 codes = ld_shared_v4(st + ch * kChunkBytes + lane * 16);
+      const uint2 sc = ld_shared_v2(st + ch * kChunkBytes + kChunkCodeBytes + g * 8);
+      const uint32_t cw[4] = {codes.x, codes.y, codes.z, codes.w};
+      // scales: sc.x = row A(g) for K steps 0..3, sc.y = row B(g)
+      const uint32_t sa01 = e4m3x2_to_f16x2(sc.x & 0xffffu), sa23 = e4m3x2_to_f16x2(sc.x >> 16);
+      const uint32_t sb01 = e4m3x2_to_f16x2(sc.y & 0xffffu), sb23 = e4m3x2_to_f16x2(sc.y >> 16);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const uint32_t pa = ks < 2 ? sa01 : sa23, pb = ks < 2 ? sb01 : sb23;
+        const uint32_t sA = (ks & 1) ? dup_hi(pa) : dup_lo(pa);
+        const uint32_t sB = (ks & 1) ? dup_hi(pb) : dup_lo(pb);
+        uint32_t a[4];
+        e2m1x8_to_f16x2x4(cw[ks], a);
+        a[0] = hmul2_u32(a[0], sA);
+        a[1] = hmul2_u32(a[1], sB);
+        a[2] = hmul2_u32(a[2], sA);
+        a[3] = hmul2_u32(a[3], sB);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const uint4& lo = b.v[nt][ch][0];
+          const uint4& hi = b.v[nt][ch][1];
+          const uint32_t b0 = ks == 0 ? lo.x : ks == 1 ? lo.z : ks == 2 ? hi.x : hi.z;
+          const uint32_t b1 = ks == 0 ? lo.y : ks == 1 ? lo.w : ks == 2 ? hi.y : hi.w;
+          if (NT == 1 || nt * 8 < nrows) mma_16816_f16(acc[ks][nt], a, b0, b1);
+        }
+      }
+    }
+  }
+}
+
+
+__global__ void __launch_bounds__(kExpThreads, 1) expert_kernel(ExpertParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t* bars_all = reinterpret_cast<uint64_t*>(smem + kExpWarps * kExpRing * kExpSB);
+  float* red = reinterpret_cast<float*>(bars_all + kExpWarps * kExpRing);   // [4][2][32][4]
+  __shared__ int s_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const int G = (int)gridDim.x, b = (int)blockIdx.x;
+
+  pdl_wait();                                   // routing results of the previous kernel
+  const int njobs = *p.njobs;
+  const int ngu = njobs * p.tpe_gu;
+  const int ntot = ngu + njobs * p.tpe_dn;
+  const bool fuse_combine = *p.n_dense == 0;
+  const int P = p.T * p.topk;
+  const int my_tiles = b < ntot ? (ntot - 1 - b) / G + 1 : 0;
+  const uint64_t deadline = globaltimer_ns() + (uint64_t)p.wait_timeout_ns;
+
+  const uint32_t ring_s = smem_u32(smem + warp * kExpRing * kExpSB);
+  const uint32_t bars_s = smem_u32(bars_all + warp * kExpRing);
+  const uint64_t pol = policy_evict_first();
+  if (lane == 0) {
+    for (int i = 0; i < kExpRing; ++i) mbar_init(bars_s + 8 * i, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
+  // ---- producer state (lane 0 of each warp): walks this warp's stages in order
+  int c_it = 0, c_s = 0, issued = 0;
+  bool c_valid = false;
+  TileInfo c_ti{};
+  auto cursor_ready = [&]() -> bool {
+    while (true) {
+      if (!c_valid) {
+        if (c_it >= my_tiles) return false;
+        c_ti = tile_info(p, b + c_it * G, ngu, warp);
+        c_s = 0;
+        c_valid = true;
+      }
+      if (c_s < c_ti.nw) return true;
+      c_valid = false;
+      ++c_it;
+    }
+  };
+  auto produce = [&](int consumed) {          // keep kExpRing stages in flight
+    while (issued < consumed + kExpRing && cursor_ready()) {
+      const int s = c_ti.slo + c_s;
+      const int nch = min(kExpSC, c_ti.cpt - kExpSC * s);
+      const int slot = issued % kExpRing;
+      mbar_arrive_expect_tx(bars_s + 8 * slot, nch * kChunkBytes);
+      bulk_g2s(ring_s + slot * kExpSB, c_ti.base + (size_t)kExpSC * s * kChunkBytes, nch * kChunkBytes,
+               bars_s + 8 * slot, pol);
+      ++c_s;
+      ++issued;
+    }
+  };
+  if (lane == 0) produce(0);
+
+  bool failed = false;
+  int consumed = 0;
+  BFrag<1> b1cur, b1nxt;
+  BFrag<2> b2;
+
+  for (int it = 0; it < my_tiles; ++it) {
+    const TileInfo ti = tile_info(p, b + it * G, ngu, warp);
+    const int nt_used = (ti.nrows + 7) >> 3;
+    // B rows of this lane (row n = nt*8 + g of the job)
+    const __half* row[2] = {nullptr, nullptr};
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const int n = nt * 8 + g;
+      if (n < ti.nrows) {
+        const int r = ti.row0 + n;
+        row[nt] = ti.down ? p.h16 + (size_t)r * p.f : p.x16 + (size_t)(p.perm[r] / p.topk) * p.d;
+      }
+    }
+    if (ti.down && ti.nw > 0 && !failed) {      // h of this job must be complete
+      int ok = 1;
+      if (lane == 0) {
+        uint32_t n = 0;
+        while (ld_acquire(p.gu_done + ti.job) < p.tpe_gu) {
+          if ((++n & 63u) == 0 && globaltimer_ns() > deadline) { ok = 0; break; }
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) {
+        failed = true;
+        if (lane == 0) set_error(p.err, kErrTimeout);
+      }
+    }
+
+    float acc[4][2][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[a][nt][q] = 0.f;
+
+    if (nt_used == 1) {
+      if (ti.nw > 0) {
+        const int s0 = ti.slo;
+        if (ti.down) load_bfrag<1, true>(b1cur, row, kExpSC * s0, min(kExpSC, ti.cpt - kExpSC * s0), c);
+        else load_bfrag<1, false>(b1cur, row, kExpSC * s0, min(kExpSC, ti.cpt - kExpSC * s0), c);
+      }
+      for (int ss = 0; ss < ti.nw; ++ss) {
+        const int s = ti.slo + ss;
+        const int nch = min(kExpSC, ti.cpt - kExpSC * s);
+        if (ss + 1 < ti.nw) {
+          const int s1 = s + 1, n1 = min(kExpSC, ti.cpt - kExpSC * s1);
+          if (ti.down) load_bfrag<1, true>(b1nxt, row, kExpSC * s1, n1, c);
+          else load_bfrag<1, false>(b1nxt, row, kExpSC * s1, n1, c);
+        }
+        const int slot = consumed % kExpRing;
+        if (!failed && !mbar_wait_until(bars_s + 8 * slot, (consumed / kExpRing) & 1, deadline)) {
+          failed = true;
+          set_error(p.err, kErrTimeout);
+        }
+        if (!failed) mma_stage<1>(ring_s + slot * kExpSB, nch, lane, g, b1cur, ti.nrows, acc);
+        __syncwarp();
+        ++consumed;
+        if (lane == 0 && !failed) produce(consumed);
+        b1cur = b1nxt;
+      }
+    } else {
+      for (int ss = 0; ss < ti.nw; ++ss) {
+        const int s = ti.slo + ss;
+        const int nch = min(kExpSC, ti.cpt - kExpSC * s);
+        if (ti.down) load_bfrag<2, true>(b2, row, kExpSC * s, nch, c);
+        else load_bfrag<2, false>(b2, row, kExpSC * s, nch, c);
+        const int slot = consumed % kExpRing;
+        if (!failed && !mbar_wait_until(bars_s + 8 * slot, (consumed / kExpRing) & 1, deadline)) {
+          failed = true;
+          set_error(p.err, kErrTimeout);
+        }
+        if (!failed) mma_stage<2>(ring_s + slot * kExpSB, nch, lane, g, b2, ti.nrows, acc);
+        __syncwarp();
+        ++consumed;
+        if (lane == 0 && !failed) produce(consumed);
+      }
+    }
+
+    // ---- cross-warp reduction of the tile
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        red[((warp * 2 + nt) * 32 + lane) * 4 + q] =
+            (acc[0][nt][q] + acc[1][nt][q]) + (acc[2][nt][q] + acc[3][nt][q]);
+    __syncthreads();
+    if (warp < nt_used) {
+      const int nt = warp;
+      float v[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kExpWarps; ++w) sum += red[((w * 2 + nt) * 32 + lane) * 4 + q];
+        v[q] = sum;
+      }
+      if (!ti.down) {
+        const float gsg = p.gs[ti.e], gsu = p.gs[p.E + ti.e];
+        const int fidx = ti.t * 8 + g;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int n = nt * 8 + 2 * c + q;
+          if (n < ti.nrows) {
+            const int r = ti.row0 + n;
+            const float xs = p.xscale[p.perm[r] / p.topk];
+            const float gv = v[q] * gsg * xs;
+            const float uv = v[2 + q] * gsu * xs;
+            const float hv = gv / (1.f + expf(-gv)) * uv;
+            p.h32[(size_t)r * p.f + fidx] = hv;
+            if (!(fabsf(hv) <= 65504.f)) set_error(p.err, kErrNumeric);
+            p.h16[(size_t)r * p.f + bfrag_offset(fidx)] = __float2half_rn(hv);
+          }
+        }
+      } else {
+        const float gsd = p.gs[2 * p.E + ti.e];
+        const int drow = ti.t * 16 + g;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int n = nt * 8 + 2 * c + q;
+          if (n < ti.nrows) {
+            const int r = ti.row0 + n;
+            const float wv = p.wts[p.perm[r]] * gsd;
+            p.partial[(size_t)r * p.d + drow] = v[q] * wv;
+            p.partial[(size_t)r * p.d + drow + 8] = v[2 + q] * wv;
+          }
+        }
+      }
+    }
+    __syncthreads();
+    // ---- publish completion
+    if (threadIdx.x == 0) {
+      __threadfence();
+      if (!ti.down) {
+        atomicAdd(p.gu_done + ti.job, 1);
+        s_flag = 0;
+      } else if (fuse_combine) {
+        const int old = atomicAdd(p.dn_done + ti.t, ti.nrows);
+        s_flag = (old + ti.nrows == P) ? 1 : 0;
+        if (s_flag) __threadfence();
+      } else {
+        s_flag = 0;
+      }
+    }
+    __syncthreads();
+    if (ti.down && s_flag) {
+      // this block completed output slice t: combine rows [16t, 16t+16) of every token
+      const int col0 = ti.t * 16;
+      for (int task = threadIdx.x; task < p.T * 4; task += blockDim.x) {
+        const int tok = task >> 2, col = col0 + (task & 3) * 4;
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+        for (int j = 0; j < p.topk; ++j) {
+          const float4 v = ldg_cg_f4(p.partial + (size_t)p.inv[tok * p.topk + j] * p.d + col);
+          s0 += v.x; s1 += v.y; s2 += v.z; s3 += v.w;
+        }
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(s0, s1), hi = __floats2bfloat162_rn(s2, s3);
+        uint2 o;
+        o.x = *reinterpret_cast<const uint32_t*>(&lo);
+        o.y = *reinterpret_cast<const uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(p.out + (size_t)tok * p.d + col) = o;
+      }
+      if (threadIdx.x == 0) p.dn_done[ti.t] = 0;
+    }
+    __syncthreads();
+  }
+
+  // Drain: after a failed wait, give the copies already issued a bounded chance
+  // to land before the block's shared memory is released.
+  if (failed && lane == 0) {
+    const uint64_t drain = globaltimer_ns() + (uint64_t)p.wait_timeout_ns;
+    for (int jj = consumed; jj < issued; ++jj)
+      if (!mbar_wait_until(bars_s + 8 * (jj % kExpRing), (jj / kExpRing) & 1, drain)) break;
+  }
+  // ---- exit protocol: the last block clears the per-job counters
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const int old = atomicAdd(p.exit_cnt, 1);
+    if (old == G - 1) {
+      for (int jb = 0; jb < njobs; ++jb) p.gu_done[jb] = 0;
+      *p.exit_cnt = 0;
+      __threadfence();
+    }
+  }
+  pdl_launch_dependents();
+}
+
+constexpr size_t expert_smem_size() {
+  return (size_t)kExpWarps * kExpRing * kExpSB + (size_t)kExpWarps * kExpRing * 8 +
+         (size_t)kExpWarps * 2 * 32 * 4 * 4;
+}
+
+}  // namespace moe

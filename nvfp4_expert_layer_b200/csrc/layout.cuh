@@ -11,8 +11,8 @@
 //                      byte 4ks+2: row A(g),  K = 16ks + 8 + 2c, +1 (a4:a5)
 //                      byte 4ks+3: row B(g),  same K               (a6:a7)
 //                    (low nibble = lower K, as in the canonical layout)
-//   bytes [512, 576) 8 groups g x 8 B of e4m3 scales: byte 2ks = scale of row
-//                    A(g) for step ks, byte 2ks+1 = scale of row B(g).
+//   bytes [512, 576) 8 groups g x 8 B of e4m3 scales: bytes 0..3 = scales of
+//                    row A(g) for steps ks = 0..3, bytes 4..7 = row B(g).
 // Tile rows: gate/up tile t pairs gate rows f = 8t+g (A) with up rows 8t+g
 // (B), so one MMA accumulator holds g and u of the same f; down tile t holds
 // rows 16t+g (A) and 16t+8+g (B).

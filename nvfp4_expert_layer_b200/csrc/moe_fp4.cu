@@ -19,13 +19,14 @@
 #include "ptx.cuh"
 #include "layout.cuh"
 #include "route.cuh"
-#include "light.cuh"
+#include "repack.cuh"
+#include "experts.cuh"
 #include "combine.cuh"
 
 namespace {
 
-constexpr int kSmallT = 256;          // router_small up to this many tokens
-constexpr int kLightRing = 6;         // bulk-copy stages per warp in the light kernel
+constexpr int kSmallT = 256;          // fused routing kernel up to this many tokens
+constexpr size_t kExpSmem = moe::expert_smem_size();
 
 struct Workspace {
   void* base = nullptr;
@@ -38,8 +39,10 @@ struct Workspace {
   int* offsets = nullptr;
   int* perm = nullptr;
   int* inv = nullptr;
-  int4* light_jobs = nullptr;
-  int* n_light_jobs = nullptr;
+  int4* jobs = nullptr;
+  int* n_jobs = nullptr;
+  int* counters = nullptr;     // gu_done [max jobs] | dn_done [d/16] | exit | ticket
+  size_t counter_bytes = 0;
   int4* dense_list = nullptr;
   int* n_dense = nullptr;
   __half* x16 = nullptr;
@@ -58,13 +61,15 @@ struct moe_fp4 {
   int E = 0, k = 0, d = 0, f = 0;
   int thr = 128;
   int sm_count = 0;
-  int light_blocks_per_sm = 1;
+  int exp_bps = 1;                // resident blocks per SM of the expert kernel
   int64_t wait_timeout_ns = 2000000000LL;
   bool loaded = false;
   uint8_t* gu_frag = nullptr;     // gate/up fragment layout, all experts
   uint8_t* dn_frag = nullptr;     // down fragment layout, all experts
   float* gs = nullptr;            // [3][E]: gate, up, down
   int* err = nullptr;             // device error word
+  cudaEvent_t stage_ev[7] = {};   // optional stage-timing events (caller-owned)
+  bool stage_timing = false;
   Workspace ws;
 };
 
@@ -98,6 +103,7 @@ size_t workspace_bytes(const moe_fp4* h, int Tm) {
   add(P * 4);                       // inv
   add(((size_t)h->E + P / moe::kJobRows + 1) * 16);   // light jobs
   add(4);
+  add(((size_t)h->E + P / moe::kJobRows + 1 + h->d / 16 + 2) * 4);   // counters
   add((size_t)h->E * 16);           // dense list
   add(4);
   add((size_t)Tm * h->d * 2);       // x16
@@ -136,8 +142,10 @@ int ensure_workspace(moe_fp4* h, int Tm, cudaStream_t stream) {
   w.offsets = carve<int>(cur, h->E + 1);
   w.perm = carve<int>(cur, P);
   w.inv = carve<int>(cur, P);
-  w.light_jobs = carve<int4>(cur, (size_t)h->E + P / moe::kJobRows + 1);
-  w.n_light_jobs = carve<int>(cur, 1);
+  w.jobs = carve<int4>(cur, (size_t)h->E + P / moe::kJobRows + 1);
+  w.n_jobs = carve<int>(cur, 1);
+  w.counter_bytes = ((size_t)h->E + P / moe::kJobRows + 1 + h->d / 16 + 2) * 4;
+  w.counters = carve<int>(cur, w.counter_bytes / 4);
   w.dense_list = carve<int4>(cur, h->E);
   w.n_dense = carve<int>(cur, 1);
   w.x16 = carve<__half>(cur, (size_t)Tm * h->d);
@@ -147,6 +155,11 @@ int ensure_workspace(moe_fp4* h, int Tm, cudaStream_t stream) {
   w.partial = carve<float>(cur, P * h->d);
   w.xin = carve<uint16_t>(cur, (size_t)Tm * h->d);
   w.xout = carve<uint16_t>(cur, (size_t)Tm * h->d);
+  if (cudaMemset(w.counters, 0, w.counter_bytes) != cudaSuccess) {
+    (void)cudaGetLastError();
+    cudaFree(base);
+    return MOE_FP4_ERR_CUDA;
+  }
   h->ws = w;
   return MOE_FP4_OK;
 }
@@ -172,76 +185,90 @@ cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, c
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
-size_t light_smem_bytes() {
-  return (size_t)moe::kLightWarps * kLightRing * moe::kStageBytes +
-         (size_t)moe::kLightWarps * kLightRing * 8 +
-         (size_t)moe::kLightWarps * moe::kLightNT * 32 * 4 * 4;
+size_t permute_smem_bytes(int E) { return moe::permute_smem_ints(E) * 4; }
+
+size_t route_smem_bytes(int E, int d, int P) {
+  return std::max((size_t)d * 4, (moe::permute_smem_ints(E) + (size_t)P) * 4);
 }
 
-size_t permute_smem_bytes(int E) { return (size_t)(32 * E + 3 * E + 2) * 4; }
+cudaError_t mark(moe_fp4* h, int i, cudaStream_t st) {
+  if (!h->stage_timing) return cudaSuccess;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(st, &cs);
+  if (e != cudaSuccess) return e;
+  return cudaEventRecordWithFlags(h->stage_ev[i], st,
+                                  cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal
+                                                                      : cudaEventRecordDefault);
+}
 
 int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cudaStream_t st) {
   Workspace& w = h->ws;
   const int E = h->E, k = h->k, d = h->d, f = h->f;
   const uint16_t* xb = static_cast<const uint16_t*>(x);
-  // 1. router logits (+ fp16 staging of x)
+  const bool pdl = !h->stage_timing;
+  MOE_CUDA(mark(h, 0, st));
+  const size_t max_jobs = (size_t)E + (size_t)w.max_T * k / moe::kJobRows + 1;   // counter layout
+  int* gu_done = w.counters;
+  int* dn_done = gu_done + max_jobs;
+  int* exit_cnt = dn_done + d / 16;
+  int* ticket = exit_cnt + 1;
+  moe::PermuteOut po{w.counts, w.offsets, w.perm, w.inv, w.jobs, w.n_jobs, w.dense_list, w.n_dense,
+                     h->err};
   if (T <= kSmallT) {
-    MOE_CUDA(launch(moe::router_small_kernel, dim3(E), dim3(256), (size_t)d * 4, st, false,
-                    xb, rw, T, d, E, w.logits, w.x16, w.xscale, h->err));
+    // 1-3. router logits, x staging, top-k and permutation in one launch
+    MOE_CUDA(launch(moe::route_kernel, dim3(E), dim3(1024), route_smem_bytes(E, d, T * k), st, false,
+                    xb, rw, T, d, E, k, h->thr, 0, w.logits, w.x16, w.xscale, w.ids, w.wts, ticket, po));
+    MOE_CUDA(mark(h, 1, st));
+    MOE_CUDA(mark(h, 2, st));
   } else {
     MOE_CUDA(launch(moe::router_tiled_kernel, dim3((T + 63) / 64, (E + 63) / 64), dim3(256), 0, st,
                     false, xb, rw, T, d, E, w.logits));
     MOE_CUDA(launch(moe::stage_x_kernel, dim3(std::min(T, 8 * h->sm_count)), dim3(256), 0, st, false,
                     xb, T, d, w.x16, w.xscale, h->err));
+    MOE_CUDA(mark(h, 1, st));
+    MOE_CUDA(launch(moe::topk_kernel, dim3((T + 7) / 8), dim3(256), 0, st, false,
+                    (const float*)w.logits, T, E, k, w.ids, w.wts));
+    MOE_CUDA(mark(h, 2, st));
+    MOE_CUDA(launch(moe::permute_kernel, dim3(1), dim3(1024), permute_smem_bytes(E), st, false,
+                    (const int*)w.ids, T, k, E, h->thr, 0, po));
   }
-  // 2. top-k
-  MOE_CUDA(launch(moe::topk_kernel, dim3((T + 7) / 8), dim3(256), 0, st, false,
-                  (const float*)w.logits, T, E, k, w.ids, w.wts));
-  // 3. permutation and expert classes
-  moe::PermuteOut po{w.counts, w.offsets, w.perm, w.inv, w.light_jobs, w.n_light_jobs,
-                     w.dense_list, w.n_dense, h->err};
-  MOE_CUDA(launch(moe::permute_kernel, dim3(1), dim3(1024), permute_smem_bytes(E), st, false,
-                  (const int*)w.ids, T, k, E, h->thr, 0, po));
-  // 4. light gate/up + SwiGLU
-  const int grid = h->sm_count * h->light_blocks_per_sm;
-  moe::LightParams lp{};
-  lp.frag = h->gu_frag;
-  lp.tpe = f / 8;
-  lp.cpt = d / moe::kChunkK;
-  lp.jobs = w.light_jobs;
-  lp.njobs = w.n_light_jobs;
-  lp.perm = w.perm;
-  lp.topk = k;
-  lp.bsrc = w.x16;
-  lp.bk = d;
-  lp.xscale = w.xscale;
-  lp.gs0 = h->gs;
-  lp.gs1 = h->gs + E;
-  lp.wts = w.wts;
-  lp.h32 = w.h32;
-  lp.h16 = w.h16;
-  lp.f = f;
-  lp.partial = w.partial;
-  lp.d = d;
-  lp.err = h->err;
-  lp.wait_timeout_ns = h->wait_timeout_ns;
-  MOE_CUDA(launch(moe::light_expert_kernel<moe::kGateUp, kLightRing>, dim3(grid),
-                  dim3(moe::kLightThreads), light_smem_bytes(), st, true, lp));
-  // 5. light down (x routing weight)
-  moe::LightParams dp = lp;
-  dp.frag = h->dn_frag;
-  dp.tpe = d / 16;
-  dp.cpt = f / moe::kChunkK;
-  dp.bsrc = w.h16;
-  dp.bk = f;
-  dp.gs0 = h->gs + 2 * E;
-  dp.gs1 = nullptr;
-  MOE_CUDA(launch(moe::light_expert_kernel<moe::kDown, kLightRing>, dim3(grid),
-                  dim3(moe::kLightThreads), light_smem_bytes(), st, true, dp));
-  // 6. combine / unpermute
-  MOE_CUDA(launch(moe::combine_kernel, dim3((d + 1023) / 1024, T), dim3(128), 0, st, true,
-                  (const float*)w.partial, (const int*)w.inv, T, k, d,
-                  static_cast<uint16_t*>(out)));
+  MOE_CUDA(mark(h, 3, st));
+  // 4-6. light experts: gate/up + SwiGLU, down x routing weight, combine
+  moe::ExpertParams ep{};
+  ep.gu_frag = h->gu_frag;
+  ep.dn_frag = h->dn_frag;
+  ep.tpe_gu = f / 8;
+  ep.cpt_gu = d / moe::kChunkK;
+  ep.tpe_dn = d / 16;
+  ep.cpt_dn = f / moe::kChunkK;
+  ep.jobs = w.jobs;
+  ep.njobs = w.n_jobs;
+  ep.n_dense = w.n_dense;
+  ep.perm = w.perm;
+  ep.inv = w.inv;
+  ep.topk = k;
+  ep.T = T;
+  ep.d = d;
+  ep.f = f;
+  ep.E = E;
+  ep.x16 = w.x16;
+  ep.xscale = w.xscale;
+  ep.h16 = w.h16;
+  ep.h32 = w.h32;
+  ep.gs = h->gs;
+  ep.wts = w.wts;
+  ep.partial = w.partial;
+  ep.out = static_cast<uint16_t*>(out);
+  ep.gu_done = gu_done;
+  ep.dn_done = dn_done;
+  ep.exit_cnt = exit_cnt;
+  ep.err = h->err;
+  ep.wait_timeout_ns = h->wait_timeout_ns;
+  MOE_CUDA(launch(moe::expert_kernel, dim3(h->sm_count * h->exp_bps), dim3(moe::kExpThreads), kExpSmem,
+                  st, pdl, ep));
+  MOE_CUDA(mark(h, 4, st));
+  MOE_CUDA(mark(h, 5, st));
+  MOE_CUDA(mark(h, 6, st));
   return MOE_FP4_OK;
 }
 
@@ -303,23 +330,20 @@ int moe_fp4_create(int E, int top_k, int d, int f, moe_fp4_t** out) {
     if (cudaDeviceGetAttribute(&h->sm_count, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess) {
       rc = MOE_FP4_ERR_CUDA; break;
     }
-    const size_t ls = light_smem_bytes();
-    if (cudaFuncSetAttribute(moe::light_expert_kernel<moe::kGateUp, kLightRing>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ls) != cudaSuccess ||
-        cudaFuncSetAttribute(moe::light_expert_kernel<moe::kDown, kLightRing>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ls) != cudaSuccess ||
-        cudaFuncSetAttribute(moe::router_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             d * 4) != cudaSuccess ||
-        cudaFuncSetAttribute(moe::permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)permute_smem_bytes(E)) != cudaSuccess) {
+    auto smem_attr = [](const void* fn, size_t bytes) {
+      return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    };
+    if (smem_attr((const void*)moe::expert_kernel, kExpSmem) != cudaSuccess ||
+        smem_attr((const void*)moe::permute_kernel, permute_smem_bytes(E)) != cudaSuccess ||
+        smem_attr((const void*)moe::route_kernel, route_smem_bytes(E, d, kSmallT * top_k)) != cudaSuccess) {
       rc = MOE_FP4_ERR_CUDA; break;
     }
     int nb = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-            &nb, moe::light_expert_kernel<moe::kGateUp, kLightRing>, moe::kLightThreads, ls) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, moe::expert_kernel, moe::kExpThreads,
+                                                      kExpSmem) != cudaSuccess) {
       rc = MOE_FP4_ERR_CUDA; break;
     }
-    h->light_blocks_per_sm = std::max(1, nb);
+    h->exp_bps = std::max(1, nb);
     if (cudaMalloc(&h->err, sizeof(int)) != cudaSuccess) { rc = MOE_FP4_ERR_OOM; break; }
     if (cudaMemset(h->err, 0, sizeof(int)) != cudaSuccess) { rc = MOE_FP4_ERR_CUDA; break; }
     if (cudaMalloc(&h->gs, sizeof(float) * 3 * E) != cudaSuccess) { rc = MOE_FP4_ERR_OOM; break; }
@@ -443,11 +467,26 @@ int moe_fp4_forward_host(moe_fp4_t* h, const void* x_host, int T, const float* r
   return MOE_FP4_OK;
 }
 
+int moe_fp4_set_stage_events(moe_fp4_t* h, cudaEvent_t* events, int n) {
+  if (!h) return MOE_FP4_ERR_INVALID_ARG;
+  if (n == 0) { h->stage_timing = false; return MOE_FP4_OK; }
+  if (n != 7 || !events) return MOE_FP4_ERR_INVALID_ARG;
+  for (int i = 0; i < 7; ++i) {
+    if (!events[i]) return MOE_FP4_ERR_INVALID_ARG;
+    h->stage_ev[i] = events[i];
+  }
+  h->stage_timing = true;
+  return MOE_FP4_OK;
+}
+
 int moe_fp4_get_device_error(moe_fp4_t* h, int* code) {
   if (!h || !code) return MOE_FP4_ERR_INVALID_ARG;
   MOE_CUDA(cudaDeviceSynchronize());
   MOE_CUDA(cudaMemcpy(code, h->err, sizeof(int), cudaMemcpyDeviceToHost));
   MOE_CUDA(cudaMemset(h->err, 0, sizeof(int)));
+  // a forward that stopped on an error may leave its completion counters set
+  if (*code != MOE_FP4_OK && h->ws.counters)
+    MOE_CUDA(cudaMemset(h->ws.counters, 0, h->ws.counter_bytes));
   return MOE_FP4_OK;
 }
 

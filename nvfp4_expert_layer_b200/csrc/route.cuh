@@ -31,8 +31,23 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
 // ---------------------------------------------------------------------------
 __device__ void stage_x_row(const uint16_t* __restrict__ xrow, int d, __half* __restrict__ x16row,
                             float* __restrict__ xscale_out, int* err, float* red) {
+  // each thread owns up to 8 groups of 8 consecutive elements (d <= 16384)
+  constexpr int kMaxG = 8;
+  const int ngroups = d / 8;
+  uint4 v[kMaxG];
   float m = 0.f;
-  for (int i = threadIdx.x; i < d; i += blockDim.x) m = fmaxf(m, fabsf(bf16_bits_to_float(xrow[i])));
+#pragma unroll
+  for (int q = 0; q < kMaxG; ++q) {
+    const int gi = threadIdx.x + q * blockDim.x;
+    v[q] = gi < ngroups ? *reinterpret_cast<const uint4*>(xrow + 8 * gi) : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int q = 0; q < kMaxG; ++q) {
+    const uint32_t w[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      m = fmaxf(m, fmaxf(fabsf(__uint_as_float(w[i] << 16)), fabsf(__uint_as_float(w[i] & 0xffff0000u))));
+  }
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (lane == 0) red[warp] = m;
@@ -50,53 +65,26 @@ __device__ void stage_x_row(const uint16_t* __restrict__ xrow, int d, __half* __
   } else if (mx > 0.f) {
     int e;
     frexpf(mx, &e);                             // mx = m * 2^e, m in [0.5, 1)
-    s = 15 - e;
-    s = max(-120, min(120, s));
+    s = max(-120, min(120, 15 - e));
   }
   const float up = ldexpf(1.f, s);
-  for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    const float v = bf16_bits_to_float(xrow[i]) * up;
-    x16row[bfrag_offset(i)] = __float2half_rn(v);
+#pragma unroll
+  for (int q = 0; q < kMaxG; ++q) {
+    const int gi = threadIdx.x + q * blockDim.x;
+    if (gi < ngroups) {
+      // elements 8gi..8gi+7: same chunk, step and slot; c = 0..3, half = 0..1
+      const uint32_t w[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+      const int base = bfrag_offset(8 * gi);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __half2 h2 = __floats2half2_rn(__uint_as_float(w[i] << 16) * up,
+                                             __uint_as_float(w[i] & 0xffff0000u) * up);
+        *reinterpret_cast<__half2*>(x16row + base + 16 * i) = h2;
+      }
+    }
   }
   if (threadIdx.x == 0) *xscale_out = ldexpf(1.f, -s);
   __syncthreads();
-}
-
-// Small-T router: one block per expert e; each warp handles tokens
-// t = warp, warp + nwarps, ...  Block b < T also stages x row b (fp16).
-// Requires d % 256 == 0 handled by the host (d % 128 == 0 -> 4-wide loads).
-__global__ void __launch_bounds__(256) router_small_kernel(
-    const uint16_t* __restrict__ x, const float* __restrict__ rw, int T, int d, int E,
-    float* __restrict__ logits, __half* __restrict__ x16, float* __restrict__ xscale, int* err) {
-  extern __shared__ __align__(16) float s_w[];   // d floats
-  __shared__ float red[33];
-  const int e = blockIdx.x;
-  if (e < E) {
-    const float4* src = reinterpret_cast<const float4*>(rw + (size_t)e * d);
-    float4* dst = reinterpret_cast<float4*>(s_w);
-    for (int i = threadIdx.x; i < d / 4; i += blockDim.x) dst[i] = src[i];
-  }
-  __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  if (e < E) {
-    for (int t = warp; t < T; t += nwarps) {
-      const uint16_t* xr = x + (size_t)t * d;
-      float acc = 0.f;
-      // lane handles 4 consecutive elements per 128-wide step
-      for (int i = lane * 4; i < d; i += 128) {
-        const uint2 xv = *reinterpret_cast<const uint2*>(xr + i);
-        const float4 wv = *reinterpret_cast<const float4*>(s_w + i);
-        acc = fmaf(__uint_as_float(xv.x << 16), wv.x, acc);
-        acc = fmaf(__uint_as_float(xv.x & 0xffff0000u), wv.y, acc);
-        acc = fmaf(__uint_as_float(xv.y << 16), wv.z, acc);
-        acc = fmaf(__uint_as_float(xv.y & 0xffff0000u), wv.w, acc);
-      }
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) logits[(size_t)t * E + e] = acc;
-    }
-  }
-  for (int t = blockIdx.x; t < T; t += gridDim.x)
-    stage_x_row(x + (size_t)t * d, d, x16 + (size_t)t * d, xscale + t, err, red);
 }
 
 // Stage x rows (used with the tiled router for large T): one block per row.
@@ -151,22 +139,13 @@ __global__ void __launch_bounds__(256) router_tiled_kernel(
 // warp arg-max ordered by (logit desc, expert asc); weights are the softmax of
 // the selected logits (equal to the renormalised full softmax).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E,
-                                                   int k, int* __restrict__ ids,
-                                                   float* __restrict__ wts) {
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= T) return;
-  float v[32];
+// Warp top-k over v[i] = logit of expert lane + 32 i (-inf beyond E).
+// Lane j < k receives the j-th selected expert and its renormalised weight.
+__device__ __forceinline__ void topk_warp(const float (&v)[32], int E, int k, int lane, int& my_e,
+                                          float& my_w) {
   const int per = (E + 31) / 32;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const int e = lane + 32 * i;
-    v[i] = (i < per && e < E) ? logits[(size_t)t * E + e] : -INFINITY;
-  }
-  float sel_l0 = 0.f, sum = 0.f;
-  float my_l = 0.f;
-  int my_e = 0;
+  float sel_l0 = 0.f, sum = 0.f, my_p = 0.f;
+  my_e = 0;
   unsigned taken = 0u;            // bit i: element lane + 32 i already selected
   for (int j = 0; j < k; ++j) {
     float bv = -INFINITY;
@@ -189,54 +168,73 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
     if (j == 0) sel_l0 = bv;
     const float p = expf(bv - sel_l0);
     sum += p;
-    if (lane == j) { my_l = p; my_e = be; }
+    if (lane == j) { my_p = p; my_e = be; }
   }
+  my_w = my_p / sum;
+}
+
+// Top-k for large T: one warp per token over the full logits.
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E,
+                                                   int k, int* __restrict__ ids,
+                                                   float* __restrict__ wts) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = e < E ? logits[(size_t)t * E + e] : -INFINITY;
+  }
+  int my_e;
+  float my_w;
+  topk_warp(v, E, k, lane, my_e, my_w);
   if (lane < k) {
     ids[(size_t)t * k + lane] = my_e;
-    wts[(size_t)t * k + lane] = my_l / sum;
+    wts[(size_t)t * k + lane] = my_w;
   }
 }
 
 // ---------------------------------------------------------------------------
-// Permutation, single block of 1024 threads (32 warps).
+// Permutation, built by one block of 1024 threads (32 warps).
 // Pairs p = t*k + j in [0, P) are cut into 32 contiguous warp chunks.  Each
 // warp counts its chunk per expert (match_any groups equal experts inside a
 // 32-pair step, so no atomics), the counts are scanned, and a second walk
 // assigns positions in (expert, pair) order -- deterministic and stable.
-// Then experts are classed by row count: light (0 < n < thr) experts are
-// split into jobs of <= 16 rows, listed heavy-first; dense (n >= thr) experts
-// are listed by n descending.
-// Dynamic shared memory: 32*E + 3*E + 2 ints.
+// Then the active experts are classed by row count n:
+//   light (n < thr): cut into jobs of <= 16 rows, listed heavy expert first;
+//   dense (n >= thr): listed by n descending.
+// Shared memory (ints): 32*E (warp counts) + 4*E + 1 (counts, offsets,
+// active list) + 8 scalars.
 // ---------------------------------------------------------------------------
 struct PermuteOut {
-  int* counts;      // [E]
-  int* offsets;     // [E+1]
-  int* perm;        // [P]
-  int* inv;         // [P]
-  int4* light_jobs; // [E + P/16 + 1]  {expert, row0, nrows, 0}
-  int* n_light_jobs;
-  int4* dense_list; // [E]  {expert, row0, nrows, 0}
+  int* counts;       // [E]
+  int* offsets;      // [E+1]
+  int* perm;         // [P]
+  int* inv;          // [P]
+  int4* jobs;        // [E + P/16 + 1] {expert, row0, nrows, 0}, 1 <= nrows <= 16
+  int* n_jobs;
+  int4* dense_list;  // [E]            {expert, row0, nrows, 0}
   int* n_dense;
   int* err;
 };
 
-__global__ void __launch_bounds__(1024) permute_kernel(const int* __restrict__ ids, int T, int k,
-                                                       int E, int thr, int dense_supported,
-                                                       PermuteOut o) {
-  extern __shared__ int sm[];
+__host__ __device__ constexpr size_t permute_smem_ints(int E) { return (size_t)36 * E + 1 + 8; }
+
+__device__ void build_permutation(const int* ids, int T, int k, int E, int thr, int dense_supported,
+                                  const PermuteOut& o, int* sm) {
   int* wc = sm;                 // [32][E]
   int* cnt = wc + 32 * E;       // [E]
   int* off = cnt + E;           // [E+1]
-  int* jstart = off + E + 1;    // [E]
-  __shared__ int s_nlight, s_ndense;
+  int* act = off + E + 1;       // [E]  active experts, ascending
+  int* misc = act + E;          // [8]  0: n_active 1: n_jobs 3: n_dense
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const long long P = (long long)T * k;
   const long long c0 = P * warp / 32, c1 = P * (warp + 1) / 32;
   for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) wc[i] = 0;
-  if (threadIdx.x == 0) { s_nlight = 0; s_ndense = 0; }
+  if (threadIdx.x < 8) misc[threadIdx.x] = 0;
   __syncthreads();
-  // pass 1: per-warp counts
-  for (long long base = c0; base < c1; base += 32) {
+  for (long long base = c0; base < c1; base += 32) {          // pass 1: counts
     const long long idx = base + lane;
     const bool valid = idx < c1;
     const int e = valid ? ids[idx] : -1;
@@ -250,20 +248,23 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int* __restrict__ i
     cnt[e] = s;
   }
   __syncthreads();
-  if (warp == 0) {   // exclusive scan of cnt by one warp
-    int carry = 0;
+  if (warp == 0) {              // exclusive scan of the counts; compaction of active experts
+    int carry = 0, acarry = 0;
     for (int b = 0; b < E; b += 32) {
       const int e = b + lane;
-      int v = e < E ? cnt[e] : 0;
+      const int v = e < E ? cnt[e] : 0;
       int incl = v;
-      for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += n;
+      for (int d = 1; d < 32; d <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += n;
       }
       if (e < E) off[e] = carry + incl - v;
       carry += __shfl_sync(0xffffffffu, incl, 31);
+      const unsigned am = __ballot_sync(0xffffffffu, v > 0);
+      if (v > 0) act[acarry + __popc(am & ((1u << lane) - 1u))] = e;
+      acarry += __popc(am);
     }
-    if (lane == 0) off[E] = carry;
+    if (lane == 0) { off[E] = carry; misc[0] = acarry; }
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -278,33 +279,32 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int* __restrict__ i
   }
   if (threadIdx.x == 0) o.offsets[E] = off[E];
   __syncthreads();
-  // pass 2: positions
   const unsigned lt = (1u << lane) - 1u;
-  for (long long base = c0; base < c1; base += 32) {
+  for (long long base = c0; base < c1; base += 32) {          // pass 2: positions
     const long long idx = base + lane;
     const bool valid = idx < c1;
     const int e = valid ? ids[idx] : -1;
     const unsigned mask = __match_any_sync(0xffffffffu, e);
-    int pos = 0;
-    if (valid && e >= 0 && e < E) {
-      pos = wc[warp * E + e] + __popc(mask & lt);
+    const bool ok = valid && e >= 0 && e < E;
+    if (ok) {
+      const int pos = wc[warp * E + e] + __popc(mask & lt);
       o.perm[pos] = (int)idx;
       o.inv[idx] = pos;
     }
     __syncwarp();
-    if (valid && e >= 0 && e < E && lane == __ffs(mask) - 1) wc[warp * E + e] += __popc(mask);
+    if (ok && lane == __ffs(mask) - 1) wc[warp * E + e] += __popc(mask);
     __syncwarp();
   }
-  // classes and job lists
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+  // expert classes over the active experts only
+  const int A = misc[0];
+  for (int a = threadIdx.x; a < A; a += blockDim.x) {
+    const int e = act[a];
     const int n = cnt[e];
-    jstart[e] = 0;
-    if (n == 0) continue;
     const bool light = n < thr;
     int rank = 0, start = 0;
-    for (int e2 = 0; e2 < E; ++e2) {
-      const int n2 = cnt[e2];
-      if (n2 == 0 || (n2 < thr) != light) continue;
+    for (int b = 0; b < A; ++b) {
+      const int e2 = act[b], n2 = cnt[e2];
+      if ((n2 < thr) != light) continue;
       if (n2 > n || (n2 == n && e2 < e)) {
         ++rank;
         start += (n2 + kJobRows - 1) / kJobRows;
@@ -313,19 +313,101 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int* __restrict__ i
     if (light) {
       const int nj = (n + kJobRows - 1) / kJobRows;
       for (int q = 0; q < nj; ++q)
-        o.light_jobs[start + q] = make_int4(e, off[e] + q * kJobRows, min(kJobRows, n - q * kJobRows), 0);
-      atomicAdd(&s_nlight, nj);
+        o.jobs[start + q] = make_int4(e, off[e] + q * kJobRows, min(kJobRows, n - q * kJobRows), 0);
+      atomicAdd(&misc[1], nj);
     } else {
       o.dense_list[rank] = make_int4(e, off[e], n, 0);
-      atomicAdd(&s_ndense, 1);
+      atomicAdd(&misc[3], 1);
     }
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    *o.n_light_jobs = s_nlight;
-    *o.n_dense = s_ndense;
-    if (s_ndense > 0 && !dense_supported) set_error(o.err, kErrUnsupported);
+    *o.n_jobs = misc[1];
+    *o.n_dense = misc[3];
+    if (misc[3] > 0 && !dense_supported) set_error(o.err, kErrUnsupported);
   }
+}
+
+__global__ void __launch_bounds__(1024) permute_kernel(const int* __restrict__ ids, int T, int k,
+                                                       int E, int thr, int dense_supported,
+                                                       PermuteOut o) {
+  extern __shared__ int sm[];
+  build_permutation(ids, T, k, E, thr, dense_supported, o, sm);
+}
+
+// Small-T routing in one launch.  Block e (1024 threads) computes the fp32
+// logits of expert e for every token (its router row is staged in shared
+// memory, one warp per token) and stages x rows t = e, e + E, ... in fp16.
+// The last block to finish (an atomic ticket; no grid barrier) runs the
+// routing tail: top-k for every token (warp per token) and the permutation,
+// then clears the ticket for the next launch.  Dynamic shared memory:
+// max(d floats, permute_smem_ints(E) + T*k ints).
+__global__ void __launch_bounds__(1024) route_kernel(
+    const uint16_t* __restrict__ x, const float* __restrict__ rw, int T, int d, int E, int k,
+    int thr, int dense_supported, float* __restrict__ logits, __half* __restrict__ x16,
+    float* __restrict__ xscale, int* __restrict__ ids_out, float* __restrict__ wts,
+    int* __restrict__ ticket, PermuteOut o) {
+  extern __shared__ __align__(16) int sm[];
+  __shared__ float red[33];
+  __shared__ int s_last;
+  const int e = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float* s_w = reinterpret_cast<float*>(sm);
+  for (int i = threadIdx.x; i < d / 4; i += blockDim.x)
+    reinterpret_cast<float4*>(s_w)[i] = reinterpret_cast<const float4*>(rw + (size_t)e * d)[i];
+  __syncthreads();
+  for (int t = warp; t < T; t += 32) {
+    const uint16_t* xr = x + (size_t)t * d;
+    float acc = 0.f;
+    for (int kk = lane * 8; kk < d; kk += 256) {
+      const uint4 xv = *reinterpret_cast<const uint4*>(xr + kk);
+      const float4 a = *reinterpret_cast<const float4*>(s_w + kk);
+      const float4 bq = *reinterpret_cast<const float4*>(s_w + kk + 4);
+      acc = fmaf(__uint_as_float(xv.x << 16), a.x, acc);
+      acc = fmaf(__uint_as_float(xv.x & 0xffff0000u), a.y, acc);
+      acc = fmaf(__uint_as_float(xv.y << 16), a.z, acc);
+      acc = fmaf(__uint_as_float(xv.y & 0xffff0000u), a.w, acc);
+      acc = fmaf(__uint_as_float(xv.z << 16), bq.x, acc);
+      acc = fmaf(__uint_as_float(xv.z & 0xffff0000u), bq.y, acc);
+      acc = fmaf(__uint_as_float(xv.w << 16), bq.z, acc);
+      acc = fmaf(__uint_as_float(xv.w & 0xffff0000u), bq.w, acc);
+    }
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) logits[(size_t)t * E + e] = acc;
+  }
+  for (int t = e; t < T; t += gridDim.x)
+    stage_x_row(x + (size_t)t * d, d, x16 + (size_t)t * d, xscale + t, o.err, red);
+  // ---- last block: routing tail
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(ticket, 1) == (int)gridDim.x - 1;
+    if (s_last) __threadfence();
+  }
+  __syncthreads();
+  if (!s_last) return;
+  int* ids_s = sm + permute_smem_ints(E);
+  for (int t = warp; t < T; t += 32) {
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int ee = lane + 32 * i;
+      float l = -INFINITY;
+      if (ee < E) asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(l) : "l"(logits + (size_t)t * E + ee));
+      v[i] = l;
+    }
+    int my_e;
+    float my_w;
+    topk_warp(v, E, k, lane, my_e, my_w);
+    if (lane < k) {
+      ids_s[t * k + lane] = my_e;
+      ids_out[(size_t)t * k + lane] = my_e;
+      wts[(size_t)t * k + lane] = my_w;
+    }
+  }
+  __syncthreads();
+  build_permutation(ids_s, T, k, E, thr, dense_supported, o, sm);
+  if (threadIdx.x == 0) *ticket = 0;
 }
 
 }  // namespace moe

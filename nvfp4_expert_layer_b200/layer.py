@@ -50,6 +50,21 @@ class MoeFp4Layer:
     def set_dense_threshold(self, thr: int) -> None:
         _lib.check(self.lib.moe_fp4_set_dense_threshold(self._h, thr), "moe_fp4_set_dense_threshold")
 
+    STAGES = ("router", "topk", "permute", "gate_up", "down", "combine")
+
+    def set_stage_events(self, events) -> None:
+        """events: list of 7 torch.cuda.Event(enable_timing=True), or None to turn off."""
+        if events is None:
+            _lib.check(self.lib.moe_fp4_set_stage_events(self._h, None, 0), "moe_fp4_set_stage_events")
+            self._stage_events = None
+            return
+        for e in events:            # torch creates the CUDA event at its first record
+            if not e.cuda_event:
+                e.record()
+        arr = (ctypes.c_void_p * 7)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+        _lib.check(self.lib.moe_fp4_set_stage_events(self._h, arr, 7), "moe_fp4_set_stage_events")
+        self._stage_events = (events, arr)
+
     def device_error(self) -> int:
         code = ctypes.c_int(0)
         _lib.check(self.lib.moe_fp4_get_device_error(self._h, ctypes.byref(code)),

@@ -253,24 +253,32 @@ def silu(z: np.ndarray) -> np.ndarray:
 
 
 def expert_ffn(xrows: np.ndarray, Wg: np.ndarray, Wu: np.ndarray, Wd: np.ndarray,
-               quantized: bool):
+               quantized: bool, magnitudes: bool = False):
     """One expert on its rows.  Returns (h, y) in float64.
 
     quantized=False (R4, n_e < thr): h = SiLU(Wg x) * (Wu x); y = Wd h.
     quantized=True  (R4, n_e >= thr): x and h pass through quantize_act_nvfp4
     first; h is rounded to float32 before its quantiser (the kernel holds h
-    in float32)."""
+    in float32).
+    magnitudes=True also returns the absolute-value sums that bound rounding
+    errors element by element (|Wg||x|, |Wu||x|, |Wd||h|, and g, u)."""
     xin = quantize_act_nvfp4(xrows)[2] if quantized else xrows
     g = xin @ Wg.T
     u = xin @ Wu.T
     h = silu(g) * u
     hin = quantize_act_nvfp4(h.astype(np.float32))[2] if quantized else h
     y = hin @ Wd.T
-    return h, y
+    if not magnitudes:
+        return h, y
+    ax = np.abs(xin)
+    mag = dict(g=g, u=u, gabs=ax @ np.abs(Wg).T, uabs=ax @ np.abs(Wu).T,
+               yabs=np.abs(hin) @ np.abs(Wd).T)
+    return h, y, mag
 
 
 def forward(x_bits: np.ndarray, router_w: np.ndarray, experts, E: int, k: int,
-            thr: int = 128, token_subset=None, want_pairs: bool = True):
+            thr: int = 128, token_subset=None, want_pairs: bool = True,
+            magnitudes: bool = False):
     """The whole layer.  `experts.expert(e)` -> {0: (q,sf,gs) gate, 1: up, 2: down}.
 
     token_subset: if given, expert outputs are evaluated only for pairs of those
@@ -290,6 +298,7 @@ def forward(x_bits: np.ndarray, router_w: np.ndarray, experts, E: int, k: int,
     f = None
     h_all = partial_all = None
     out64 = np.zeros((T, d), dtype=np.float64)
+    mags = None
     for e in range(E):
         lo, hi = offsets[e], offsets[e + 1]
         if hi == lo:
@@ -310,7 +319,13 @@ def forward(x_bits: np.ndarray, router_w: np.ndarray, experts, E: int, k: int,
             if want_pairs:
                 h_all = np.full((P, f), np.nan)
                 partial_all = np.full((P, d), np.nan)
-        h, y = expert_ffn(x[toks], Wg, Wu, Wd, quantized=(hi - lo) >= thr)
+        res = expert_ffn(x[toks], Wg, Wu, Wd, quantized=(hi - lo) >= thr, magnitudes=magnitudes)
+        h, y = res[0], res[1]
+        if magnitudes:
+            if mags is None:
+                mags = {n: np.full((P, v.shape[1]), np.nan) for n, v in res[2].items()}
+            for n, v in res[2].items():
+                mags[n][pos] = v
         wj = w.reshape(-1)[pairs]
         contrib = wj[:, None] * y
         if want_pairs:
@@ -320,4 +335,4 @@ def forward(x_bits: np.ndarray, router_w: np.ndarray, experts, E: int, k: int,
     out_bits = f64_to_bf16_bits_rne(out64)
     return dict(logits=logits, ids=ids, w=w, gap=gap, counts=counts, offsets=offsets,
                 perm=perm, inv=inv, h=h_all, partial=partial_all, out64=out64,
-                out_bits=out_bits, tokens=tokens)
+                out_bits=out_bits, tokens=tokens, mags=mags)
