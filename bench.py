@@ -1,0 +1,447 @@
+"""Benchmark of the NVFP4 sparse-MoE layer forward on B200 (one JSON line).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--workload decode1|decode64|verify|tiny]
+
+A step is one forward of the layer (routing, permutation, gate/up + SwiGLU,
+down, combine) over one batch of synthetic tokens.  The default workload is
+batch-1 decode (T=1, d=7168, E=256, top-8, f=2048, NVFP4 experts).  Inputs
+are seeded and synthetic; every step takes the next x of a pool of 32
+distinct token batches whose routing touches different experts, so the
+weights a step streams were evicted from L2 by the steps in between.
+
+Timing: K steps replayed as one CUDA graph each, bracketed by a barrier and
+torch.cuda.synchronize on both sides, timed with CUDA events on the stream the
+kernels run on; the job time is the max over ranks.  With N > 1 (torchrun) the
+ranks run independent replicas of the layer (the path has no exchange step).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s; decode HBM GB/s and prefill FP4 TFLOP/s vs B200 roofline"
+EXPERT_BYTES = None   # set from the config: bytes of one expert (gate + up + down, NVFP4)
+POOL = 32
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="decode1")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def expert_bytes(cfg) -> int:
+    """Algorithmic bytes of one expert: 3 matrices of f x d NVFP4 values
+    (0.5 byte per value + one e4m3 byte per 16 values)."""
+    return 3 * cfg.f * cfg.d // 2 + 3 * cfg.f * cfg.d // 16
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            mp = json.load(fh)
+        return mp["hbm_gbs"], "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def source_digest() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "nvfp4_expert_layer_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, fn), "rb") as fh:
+            h.update(fn.encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None
+    when the kernel sources changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as fh:
+            rec = json.load(fh)
+    except Exception:
+        return None
+    ent = rec.get(kernel)
+    if not ent or ent.get("source_digest") != source_digest():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        load = [v for v in sm if smax and v > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing (one process per GPU; replicas of the layer)
+# ----------------------------------------------------------------------------
+
+def dist_setup(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=600))
+    return rank, world, local
+
+
+def allreduce_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------
+# CPU baseline: the oracle on a bounded sample of the same workload
+# ----------------------------------------------------------------------------
+
+def oracle_sample(cfg, x, rw, n_tokens: int):
+    """Time the fp64 oracle on the first n_tokens of x (routing over all
+    experts, the selected experts dequantised exactly and evaluated).  Expert
+    weights are generated before the clock starts.  Returns (seconds, result)."""
+    from nvfp4_expert_layer_b200 import workloads as W
+    from oracle import moe_oracle as O
+    lazy = W.LazyExperts(cfg)
+    ids, _, _ = O.route(O.router_logits(x[:n_tokens], rw), cfg.k)
+    for e in np.unique(ids):
+        lazy.expert(int(e))
+    t0 = time.perf_counter()
+    res = O.forward(x[:n_tokens], rw, lazy, cfg.E, cfg.k, thr=128)
+    return time.perf_counter() - t0, res
+
+
+REF_BLOCK = 128     # FFN channels per reference step
+
+
+def reference_unit(cfg, x, rw, lazy, step):
+    """One reference step: the oracle's arithmetic for one routed (token 0,
+    expert j) pair restricted to FFN channels [c0, c0 + 128): route the token,
+    dequantise those gate/up rows and the matching down columns, SwiGLU, and
+    the weighted contribution to the output.  1/(k * f/128) of a token."""
+    from oracle import moe_oracle as O
+    nblk = cfg.f // REF_BLOCK
+    j = step % cfg.k
+    c0 = ((step // cfg.k) % nblk) * REF_BLOCK
+    ids, w, _ = O.route(O.router_logits(x[:1], rw), cfg.k)
+    mats = lazy.expert(int(ids[0, j]))
+    rows = slice(c0, c0 + REF_BLOCK)
+    Wg = O.dequant_nvfp4(mats[0][0][rows], mats[0][1][rows], mats[0][2])
+    Wu = O.dequant_nvfp4(mats[1][0][rows], mats[1][1][rows], mats[1][2])
+    Wd = O.dequant_nvfp4(mats[2][0][:, c0 // 2:(c0 + REF_BLOCK) // 2],
+                         mats[2][1][:, c0 // 16:(c0 + REF_BLOCK) // 16], mats[2][2])
+    xf = O.bf16_bits_to_f64(x[:1])
+    g, u = xf @ Wg.T, xf @ Wu.T
+    return w[0, j] * ((O.silu(g) * u) @ Wd.T)
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------------------
+# native arm: the CUDA layer through its C ABI
+# ----------------------------------------------------------------------------
+
+def pool_inputs(cfg, n):
+    from nvfp4_expert_layer_b200 import workloads as W
+    _, rw = W.gen_x_router(cfg)
+    xs = []
+    for i in range(n):
+        ci = W.LayerConfig(cfg.name, cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.seed * 1000 + 17 + i,
+                           cfg.router, cfg.requests)
+        xs.append(W.gen_x_router(ci)[0] if i else W.gen_x_router(cfg)[0])
+    return xs, rw
+
+
+def run_native(args, rank, world, local):
+    import torch
+    from nvfp4_expert_layer_b200 import workloads as W
+    from nvfp4_expert_layer_b200.layer import MoeFp4Layer, experts_to_device
+    torch.cuda.set_device(local)
+    cfg = W.CONFIGS[args.workload]
+    ex = W.gen_experts(cfg)
+    layer = MoeFp4Layer(cfg.E, cfg.k, cfg.d, cfg.f)
+    dev = experts_to_device(ex)
+    layer.load_experts(dev)
+    del dev
+    torch.cuda.empty_cache()
+    layer.reserve(cfg.T)
+    xs_np, rw_np = pool_inputs(cfg, POOL)
+    xs = [torch.from_numpy(x.view(np.int16).copy()).cuda().view(torch.bfloat16) for x in xs_np]
+    rw = torch.from_numpy(rw_np).cuda()
+    out = torch.empty_like(xs[0])
+    # distinct experts each pool input routes to (units of work of one step), from the layer itself
+    experts_per_input = []
+    for x in xs:
+        _, dbg = layer.forward_ex(x, rw, want=("counts",))
+        experts_per_input.append(int((dbg["counts"] > 0).sum().item()))
+    stream = torch.cuda.Stream()
+    graphs = []
+    with torch.cuda.stream(stream):
+        for x in xs:                       # warm the path once per input before capture
+            layer(x, rw, out=out, stream=stream)
+        stream.synchronize()
+        for x in xs:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                layer(x, rw, out=out, stream=stream)
+            graphs.append(g)
+    torch.cuda.synchronize()
+    assert layer.device_error() == 0
+    cur = torch.cuda.current_stream()
+    for i in range(args.warmup):
+        graphs[i % POOL].replay()
+    torch.cuda.synchronize()
+    # ---- timed region (headline)
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(cur)
+    for i in range(args.steps):
+        graphs[i % POOL].replay()
+    e1.record(cur)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms = allreduce_max(e0.elapsed_time(e1), world)
+    err = layer.device_error()
+    # ---- per-stage pass: the same graphs with stage events (events between stages)
+    stage_ms = np.zeros(6)
+    sgraphs, sevents = [], []
+    with torch.cuda.stream(stream):
+        for x in xs:
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
+            layer.set_stage_events(evs)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                layer(x, rw, out=out, stream=stream)
+            sgraphs.append(g)
+            sevents.append(evs)
+        layer.set_stage_events(None)
+    torch.cuda.synchronize()
+    for i in range(POOL):
+        sgraphs[i].replay()
+    torch.cuda.synchronize()
+    dom_ms, dom_bytes, n = 0.0, 0.0, 0
+    for rep in range(max(1, args.steps // POOL)):
+        for i in range(POOL):
+            sgraphs[i].replay()
+        torch.cuda.synchronize()
+        for i in range(POOL):
+            d = [sevents[i][j].elapsed_time(sevents[i][j + 1]) for j in range(6)]
+            stage_ms += d
+            dom_ms += d[3]
+            dom_bytes += experts_per_input[i] * expert_bytes(cfg)
+            n += 1
+    stage_ms /= n
+    # ---- end to end through the C ABI with host buffers
+    xh = [torch.from_numpy(x.view(np.int16).copy()).view(torch.bfloat16).pin_memory() for x in xs_np]
+    oh = torch.empty_like(xh[0]).pin_memory()
+    for i in range(3):
+        layer.forward_host(xh[i % POOL], rw, out_host=oh, stream=stream)
+    barrier(world)
+    ee0, ee1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ee0.record(stream)
+    for i in range(args.steps):
+        layer.forward_host(xh[i % POOL], rw, out_host=oh, stream=stream)
+    ee1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = allreduce_max(ee0.elapsed_time(ee1), world)
+    gpu_out0 = None
+    layer(xs[0], rw, out=out)
+    torch.cuda.synchronize()
+    gpu_out0 = out.view(torch.int16).cpu().numpy().view(np.uint16).copy()
+    return dict(cfg=cfg, ms=ms, clk=clk, err=err, stage_ms=stage_ms, dom_ms=dom_ms / n,
+                dom_bytes=dom_bytes / n, e2e_ms=e2e_ms, xs_np=xs_np, rw_np=rw_np, gpu_out0=gpu_out0,
+                launches_per_step=(4 if cfg.T <= 256 else 6), stages=layer.STAGES)
+
+
+def parity_vs_oracle(res_oracle, gpu_bits, tol=1e-2):
+    """Output parity of one sampled token batch (bf16 output within 1e-2*rms
+    plus the final rounding's half ulp of the oracle's exact output)."""
+    from oracle import moe_oracle as O
+    toks = res_oracle["tokens"]
+    ov = res_oracle["out64"][toks]
+    gv = O.bf16_bits_to_f64(gpu_bits[toks])
+    rms = float(np.sqrt(np.mean(ov ** 2)))
+    half = np.exp2(np.floor(np.log2(np.maximum(np.abs(ov), 2.0 ** -126))) - 8)
+    ok = bool(np.all(np.abs(gv - ov) <= tol * rms + half)) and not bool(np.any(O.near_tie_flags(res_oracle["gap"])))
+    return ("pass" if ok else "fail"), float(np.abs(gv - ov).max() / rms)
+
+
+def cpu_baseline_sample(cfg, xs_np, rw_np):
+    """Oracle on a bounded sample: the first pool input (all of its tokens when
+    T <= 8, else its first 8 tokens)."""
+    n = min(cfg.T, 8)
+    secs, res = oracle_sample(cfg, xs_np[0], rw_np, n)
+    sample = (f"oracle on {n} token(s) of the {cfg.name} workload: routing over {cfg.E} experts, "
+              f"the selected experts dequantised exactly and evaluated in fp64")
+    return secs, n, res, sample
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_setup(args)
+    from nvfp4_expert_layer_b200 import workloads as W
+    cfg = W.CONFIGS[args.workload]
+    if args.impl == "reference":
+        # the reference arm is the oracle (plain fp64 CPU code) on bounded
+        # slices of the same workload; rank 0 only
+        if rank != 0:
+            return
+        xs_np, rw_np = pool_inputs(cfg, 1)
+        lazy = W.LazyExperts(cfg)
+        from oracle import moe_oracle as O
+        ids, _, _ = O.route(O.router_logits(xs_np[0][:1], rw_np), cfg.k)
+        for e in ids[0]:
+            lazy.expert(int(e))                     # generated before timing
+        for i in range(args.warmup):
+            reference_unit(cfg, xs_np[0], rw_np, lazy, i)
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            reference_unit(cfg, xs_np[0], rw_np, lazy, i)
+        secs = time.perf_counter() - t0
+        per_step_tokens = 1.0 / (cfg.k * (cfg.f // REF_BLOCK))
+        value = per_step_tokens * args.steps / secs
+        sample = (f"per step: one routed (token, expert) pair of the {cfg.name} workload restricted to "
+                  f"{REF_BLOCK} of the f={cfg.f} FFN channels ({per_step_tokens:.6f} token)")
+        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": f"{cfg.name}: T={cfg.T}, d={cfg.d}, E={cfg.E}, top-{cfg.k}, f={cfg.f}"},
+                "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+                                 "sample": sample},
+                "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    r = run_native(args, rank, world, local)
+    tokens = cfg.T * args.steps * world
+    value = tokens / (r["ms"] * 1e-3)
+    peak, peak_kind = measured_peaks()
+    achieved = r["dom_bytes"] / (r["dom_ms"] * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": r["ms"] / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic (seeded; NVFP4 experts from N(0,0.02), x ~ N(0,1) bf16)",
+        "config": {"workload": f"{cfg.name}: T={cfg.T} tokens, d={cfg.d}, E={cfg.E}, top-{cfg.k}, f={cfg.f}, "
+                               "NVFP4 experts (e2m1 + e4m3/16 + fp32 tensor scale)",
+                   "global_batch": cfg.T * world, "parallelism": f"replicas x{world}",
+                   "l2": f"inputs rotate over {POOL} token batches; their experts span "
+                         f"{cfg.E * expert_bytes(cfg) / 1e9:.2f} GB > 126 MB L2",
+                   "timing": "CUDA graph replay per step, CUDA events on the launch stream, max over ranks",
+                   "compute": "fp4 weights dequantised in registers to fp16, m16n8k16 MMA, fp32 accumulate"},
+        "roofline": {"bound": "hbm", "kernel": "expert_kernel (gate/up + SwiGLU + down, light class)",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_kind": peak_kind, "traffic": recorded_traffic("expert_kernel"),
+                     "algorithmic_bytes_per_launch": r["dom_bytes"], "avg_launch_ms": r["dom_ms"]},
+        "stage_us": {n: round(float(v) * 1e3, 2) for n, v in zip(r["stages"], r["stage_ms"])},
+        "clocks": r["clk"],
+        "e2e": {"value": tokens / (r["e2e_ms"] * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 2},
+        "gpu_launches": r["launches_per_step"] * args.steps,
+        "device_error": r["err"],
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        secs, n, res, sample = cpu_baseline_sample(cfg, r["xs_np"], r["rw_np"])
+        line["cpu_baseline"] = {"value": n / secs, "unit": "tokens/s", "cores": cpu_cores(),
+                                "kind": "oracle", "sample": sample}
+        line["parity"], line["parity_max_err_over_rms"] = parity_vs_oracle(res, r["gpu_out0"])
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -48,6 +48,7 @@ constexpr int kExpThreads = kExpWarps * 32;
 constexpr int kExpSC = 4;          // 64-wide K chunks per bulk-copy stage (2304 bytes)
 constexpr int kExpRing = 6;        // stages in flight per warp
 constexpr int kExpSB = kExpSC * kChunkBytes;
+constexpr int kExpSmemJobs = 512;  // job table copied to shared memory when it fits
 
 struct ExpertParams {
   const uint8_t* gu_frag;     // gate/up fragment layout [E][f/8 tiles][d/64 chunks]
@@ -81,6 +82,10 @@ __device__ __forceinline__ int ld_acquire(const int* p) {
   return v;
 }
 
+__device__ __forceinline__ void red_release_add(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ uint4 ldg_cg_v4(const void* p) {
   uint4 v;
   asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -105,14 +110,15 @@ struct TileInfo {
   const uint8_t* base;
 };
 
-__device__ __forceinline__ TileInfo tile_info(const ExpertParams& p, int i, int ngu, int warp) {
+__device__ __forceinline__ TileInfo tile_info(const ExpertParams& p, const int4* jobs, int i, int ngu,
+                                              int warp) {
   TileInfo ti;
   ti.down = i >= ngu;
   const int tpe = ti.down ? p.tpe_dn : p.tpe_gu;
   const int li = ti.down ? i - ngu : i;
   ti.job = li / tpe;
   ti.t = li - ti.job * tpe;
-  const int4 jb = p.jobs[ti.job];
+  const int4 jb = jobs[ti.job];
   ti.e = jb.x;
   ti.row0 = jb.y;
   ti.nrows = jb.z;
@@ -151,7 +157,7 @@ __device__ __forceinline__ void load_bfrag(BFrag<NT>& b, const __half* const (&r
 // One stage of shared-memory weights times the lane's activation fragments.
 template <int NT>
 __device__ __forceinline__ void mma_stage(uint32_t st, int nch, int lane, int g, const BFrag<NT>& b,
-                                          int nrows, float (&acc)[4][2][4]) {
+                                          int nrows, float (&acc)[4][NT][4]) {
 #pragma unroll
   for (int ch = 0; ch < kExpSC; ++ch) {
     if (ch < nch) {
@@ -186,11 +192,13 @@ __device__ __forceinline__ void mma_stage(uint32_t st, int nch, int lane, int g,
 }
 
 
-__global__ void __launch_bounds__(kExpThreads, 1) expert_kernel(ExpertParams p) {
+// NT = 8-wide n-tiles per job: expert_kernel<1> runs jobs of <= 8 rows,
+// expert_kernel<2> jobs of 9..16 rows; each has its own job list and counters.
+template <int NT>
+__global__ void __launch_bounds__(kExpThreads, 3) expert_kernel(ExpertParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* bars_all = reinterpret_cast<uint64_t*>(smem + kExpWarps * kExpRing * kExpSB);
-  float* red = reinterpret_cast<float*>(bars_all + kExpWarps * kExpRing);   // [4][2][32][4]
-  __shared__ int s_flag;
+  float* red_all = reinterpret_cast<float*>(bars_all + kExpWarps * kExpRing);   // [2][4][2][32][4]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
@@ -200,10 +208,15 @@ __global__ void __launch_bounds__(kExpThreads, 1) expert_kernel(ExpertParams p) 
   const int njobs = *p.njobs;
   const int ngu = njobs * p.tpe_gu;
   const int ntot = ngu + njobs * p.tpe_dn;
-  const bool fuse_combine = *p.n_dense == 0;
-  const int P = p.T * p.topk;
   const int my_tiles = b < ntot ? (ntot - 1 - b) / G + 1 : 0;
   const uint64_t deadline = globaltimer_ns() + (uint64_t)p.wait_timeout_ns;
+  __shared__ int4 s_jobs[kExpSmemJobs];
+  const int4* jobs = p.jobs;
+  if (njobs <= kExpSmemJobs) {
+    for (int i = threadIdx.x; i < njobs; i += blockDim.x) s_jobs[i] = p.jobs[i];
+    jobs = s_jobs;
+  }
+  __syncthreads();
 
   const uint32_t ring_s = smem_u32(smem + warp * kExpRing * kExpSB);
   const uint32_t bars_s = smem_u32(bars_all + warp * kExpRing);
@@ -222,7 +235,7 @@ __global__ void __launch_bounds__(kExpThreads, 1) expert_kernel(ExpertParams p) 
     while (true) {
       if (!c_valid) {
         if (c_it >= my_tiles) return false;
-        c_ti = tile_info(p, b + c_it * G, ngu, warp);
+        c_ti = tile_info(p, jobs, b + c_it * G, ngu, warp);
         c_s = 0;
         c_valid = true;
       }
@@ -250,25 +263,42 @@ __global__ void __launch_bounds__(kExpThreads, 1) expert_kernel(ExpertParams p) 
   BFrag<1> b1cur, b1nxt;
   BFrag<2> b2;
 
-  for (int it = 0; it < my_tiles; ++it) {
-    const TileInfo ti = tile_info(p, b + it * G, ngu, warp);
-    const int nt_used = (ti.nrows + 7) >> 3;
-    // B rows of this lane (row n = nt*8 + g of the job)
-    const __half* row[2] = {nullptr, nullptr};
+  // B rows of this lane (row n = nt*8 + g of the job), resolved one tile ahead
+  auto tile_rows = [&](const TileInfo& t, const __half* (&row)[2]) {
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
       const int n = nt * 8 + g;
-      if (n < ti.nrows) {
-        const int r = ti.row0 + n;
-        row[nt] = ti.down ? p.h16 + (size_t)r * p.f : p.x16 + (size_t)(p.perm[r] / p.topk) * p.d;
+      row[nt] = nullptr;
+      if (n < t.nrows) {
+        const int r = t.row0 + n;
+        row[nt] = t.down ? p.h16 + (size_t)r * p.f : p.x16 + (size_t)(p.perm[r] / p.topk) * p.d;
       }
+    }
+  };
+  TileInfo ti_next{};
+  const __half* row_next[2] = {nullptr, nullptr};
+  if (my_tiles > 0) {
+    ti_next = tile_info(p, jobs, b, ngu, warp);
+    tile_rows(ti_next, row_next);
+  }
+
+  for (int it = 0; it < my_tiles; ++it) {
+    const TileInfo ti = ti_next;
+    const int nt_used = (ti.nrows + 7) >> 3;
+    const __half* row[2] = {row_next[0], row_next[1]};
+    if (it + 1 < my_tiles) {
+      ti_next = tile_info(p, jobs, b + (it + 1) * G, ngu, warp);
+      tile_rows(ti_next, row_next);
     }
     if (ti.down && ti.nw > 0 && !failed) {      // h of this job must be complete
       int ok = 1;
       if (lane == 0) {
         uint32_t n = 0;
-        while (ld_acquire(p.gu_done + ti.job) < p.tpe_gu) {
-          if ((++n & 63u) == 0 && globaltimer_ns() > deadline) { ok = 0; break; }
+        // every gate/up tile of the job is published once per writer warp (n-tile)
+        const int target = p.tpe_gu * ((ti.nrows + 7) >> 3);
+        while (ld_acquire(p.gu_done + ti.job) < target) {
+          __nanosleep(128);
+          if ((++n & 15u) == 0 && globaltimer_ns() > deadline) { ok = 0; break; }
         }
       }
       if (!__shfl_sync(0xffffffffu, ok, 0)) {
@@ -277,40 +307,53 @@ __global__ void __launch_bounds__(kExpThreads, 1) expert_kernel(ExpertParams p) 
       }
     }
 
-    float acc[4][2][4];
+    float part[2][4];                    // this warp's partial sums of the tile, per n-tile
+    if constexpr (NT == 1) {
+      // one n-tile: activation fragments double-buffered one stage ahead
+      float acc[4][1][4];
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+      for (int a = 0; a < 4; ++a)
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[a][nt][q] = 0.f;
-
-    if (nt_used == 1) {
-      if (ti.nw > 0) {
-        const int s0 = ti.slo;
-        if (ti.down) load_bfrag<1, true>(b1cur, row, kExpSC * s0, min(kExpSC, ti.cpt - kExpSC * s0), c);
-        else load_bfrag<1, false>(b1cur, row, kExpSC * s0, min(kExpSC, ti.cpt - kExpSC * s0), c);
-      }
-      for (int ss = 0; ss < ti.nw; ++ss) {
-        const int s = ti.slo + ss;
+        for (int q = 0; q < 4; ++q) acc[a][0][q] = 0.f;
+      auto load1 = [&](BFrag<1>& bf, int s) {
+        const int n1 = min(kExpSC, ti.cpt - kExpSC * s);
+        if (ti.down) load_bfrag<1, true>(bf, row, kExpSC * s, n1, c);
+        else load_bfrag<1, false>(bf, row, kExpSC * s, n1, c);
+      };
+      auto step1 = [&](const BFrag<1>& bf, int s) {
         const int nch = min(kExpSC, ti.cpt - kExpSC * s);
-        if (ss + 1 < ti.nw) {
-          const int s1 = s + 1, n1 = min(kExpSC, ti.cpt - kExpSC * s1);
-          if (ti.down) load_bfrag<1, true>(b1nxt, row, kExpSC * s1, n1, c);
-          else load_bfrag<1, false>(b1nxt, row, kExpSC * s1, n1, c);
-        }
         const int slot = consumed % kExpRing;
         if (!failed && !mbar_wait_until(bars_s + 8 * slot, (consumed / kExpRing) & 1, deadline)) {
           failed = true;
           set_error(p.err, kErrTimeout);
         }
-        if (!failed) mma_stage<1>(ring_s + slot * kExpSB, nch, lane, g, b1cur, ti.nrows, acc);
+        if (!failed) mma_stage<1>(ring_s + slot * kExpSB, nch, lane, g, bf, ti.nrows, acc);
         __syncwarp();
         ++consumed;
         if (lane == 0 && !failed) produce(consumed);
-        b1cur = b1nxt;
+      };
+      if (ti.nw > 0) load1(b1cur, ti.slo);
+      int ss = 0;
+      for (; ss + 1 < ti.nw; ss += 2) {
+        load1(b1nxt, ti.slo + ss + 1);
+        step1(b1cur, ti.slo + ss);
+        if (ss + 2 < ti.nw) load1(b1cur, ti.slo + ss + 2);
+        step1(b1nxt, ti.slo + ss + 1);
+      }
+      if (ss < ti.nw) step1(b1cur, ti.slo + ss);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        part[0][q] = (acc[0][0][q] + acc[1][0][q]) + (acc[2][0][q] + acc[3][0][q]);
+        part[1][q] = 0.f;
       }
     } else {
+      float acc[4][2][4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc[a][nt][q] = 0.f;
       for (int ss = 0; ss < ti.nw; ++ss) {
         const int s = ti.slo + ss;
         const int nch = min(kExpSC, ti.cpt - kExpSC * s);
@@ -326,15 +369,20 @@ __global__ void __launch_bounds__(kExpThreads, 1) expert_kernel(ExpertParams p) 
         ++consumed;
         if (lane == 0 && !failed) produce(consumed);
       }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          part[nt][q] = (acc[0][nt][q] + acc[1][nt][q]) + (acc[2][nt][q] + acc[3][nt][q]);
     }
 
-    // ---- cross-warp reduction of the tile
+    // ---- cross-warp reduction of the tile (buffer alternates by tile parity)
+    float* red = red_all + (it & 1) * (kExpWarps * 2 * 32 * 4);
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        red[((warp * 2 + nt) * 32 + lane) * 4 + q] =
-            (acc[0][nt][q] + acc[1][nt][q]) + (acc[2][nt][q] + acc[3][nt][q]);
+        red[((warp * 2 + nt) * 32 + lane) * 4 + q] = part[nt][q];
     __syncthreads();
     if (warp < nt_used) {
       const int nt = warp;
@@ -377,42 +425,10 @@ __global__ void __launch_bounds__(kExpThreads, 1) expert_kernel(ExpertParams p) 
           }
         }
       }
+      // publish this n-tile of a gate/up tile (release, no round trip)
+      __syncwarp();
+      if (!ti.down && lane == 0) red_release_add(p.gu_done + ti.job, 1);
     }
-    __syncthreads();
-    // ---- publish completion
-    if (threadIdx.x == 0) {
-      __threadfence();
-      if (!ti.down) {
-        atomicAdd(p.gu_done + ti.job, 1);
-        s_flag = 0;
-      } else if (fuse_combine) {
-        const int old = atomicAdd(p.dn_done + ti.t, ti.nrows);
-        s_flag = (old + ti.nrows == P) ? 1 : 0;
-        if (s_flag) __threadfence();
-      } else {
-        s_flag = 0;
-      }
-    }
-    __syncthreads();
-    if (ti.down && s_flag) {
-      // this block completed output slice t: combine rows [16t, 16t+16) of every token
-      const int col0 = ti.t * 16;
-      for (int task = threadIdx.x; task < p.T * 4; task += blockDim.x) {
-        const int tok = task >> 2, col = col0 + (task & 3) * 4;
-        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-        for (int j = 0; j < p.topk; ++j) {
-          const float4 v = ldg_cg_f4(p.partial + (size_t)p.inv[tok * p.topk + j] * p.d + col);
-          s0 += v.x; s1 += v.y; s2 += v.z; s3 += v.w;
-        }
-        const __nv_bfloat162 lo = __floats2bfloat162_rn(s0, s1), hi = __floats2bfloat162_rn(s2, s3);
-        uint2 o;
-        o.x = *reinterpret_cast<const uint32_t*>(&lo);
-        o.y = *reinterpret_cast<const uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(p.out + (size_t)tok * p.d + col) = o;
-      }
-      if (threadIdx.x == 0) p.dn_done[ti.t] = 0;
-    }
-    __syncthreads();
   }
 
   // Drain: after a failed wait, give the copies already issued a bounded chance
@@ -438,7 +454,7 @@ __global__ void __launch_bounds__(kExpThreads, 1) expert_kernel(ExpertParams p) 
 
 constexpr size_t expert_smem_size() {
   return (size_t)kExpWarps * kExpRing * kExpSB + (size_t)kExpWarps * kExpRing * 8 +
-         (size_t)kExpWarps * 2 * 32 * 4 * 4;
+         (size_t)2 * kExpWarps * 2 * 32 * 4 * 4;
 }
 
 }  // namespace moe

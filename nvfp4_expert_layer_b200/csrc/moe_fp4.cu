@@ -39,8 +39,10 @@ struct Workspace {
   int* offsets = nullptr;
   int* perm = nullptr;
   int* inv = nullptr;
-  int4* jobs = nullptr;
-  int* n_jobs = nullptr;
+  int4* jobs1 = nullptr;
+  int* n_jobs1 = nullptr;
+  int4* jobs2 = nullptr;
+  int* n_jobs2 = nullptr;
   int* counters = nullptr;     // gu_done [max jobs] | dn_done [d/16] | exit | ticket
   size_t counter_bytes = 0;
   int4* dense_list = nullptr;
@@ -61,7 +63,7 @@ struct moe_fp4 {
   int E = 0, k = 0, d = 0, f = 0;
   int thr = 128;
   int sm_count = 0;
-  int exp_bps = 1;                // resident blocks per SM of the expert kernel
+  int exp_bps1 = 1, exp_bps2 = 1; // resident blocks per SM of the expert kernels
   int64_t wait_timeout_ns = 2000000000LL;
   bool loaded = false;
   uint8_t* gu_frag = nullptr;     // gate/up fragment layout, all experts
@@ -90,6 +92,12 @@ T* carve(uint8_t*& cur, size_t count) {
   return p;
 }
 
+// completion counters: gu_done of list 1 [E] | gu_done of list 2 [E + P/16 + 1] |
+// dn_done [d/16] | exit 1 | exit 2 | routing ticket
+size_t counter_ints(const moe_fp4* h, int Tm) {
+  return (size_t)h->E + ((size_t)h->E + (size_t)Tm * h->k / moe::kJobRows + 1) + h->d / 16 + 3;
+}
+
 size_t workspace_bytes(const moe_fp4* h, int Tm) {
   const size_t P = (size_t)Tm * h->k;
   size_t b = 0;
@@ -101,9 +109,11 @@ size_t workspace_bytes(const moe_fp4* h, int Tm) {
   add((size_t)(h->E + 1) * 4);      // offsets
   add(P * 4);                       // perm
   add(P * 4);                       // inv
-  add(((size_t)h->E + P / moe::kJobRows + 1) * 16);   // light jobs
+  add((size_t)h->E * 16);                              // light jobs, <= 8 rows
   add(4);
-  add(((size_t)h->E + P / moe::kJobRows + 1 + h->d / 16 + 2) * 4);   // counters
+  add(((size_t)h->E + P / moe::kJobRows + 1) * 16);   // light jobs, 9..16 rows
+  add(4);
+  add(counter_ints(h, Tm) * 4);                        // counters
   add((size_t)h->E * 16);           // dense list
   add(4);
   add((size_t)Tm * h->d * 2);       // x16
@@ -142,9 +152,11 @@ int ensure_workspace(moe_fp4* h, int Tm, cudaStream_t stream) {
   w.offsets = carve<int>(cur, h->E + 1);
   w.perm = carve<int>(cur, P);
   w.inv = carve<int>(cur, P);
-  w.jobs = carve<int4>(cur, (size_t)h->E + P / moe::kJobRows + 1);
-  w.n_jobs = carve<int>(cur, 1);
-  w.counter_bytes = ((size_t)h->E + P / moe::kJobRows + 1 + h->d / 16 + 2) * 4;
+  w.jobs1 = carve<int4>(cur, h->E);
+  w.n_jobs1 = carve<int>(cur, 1);
+  w.jobs2 = carve<int4>(cur, (size_t)h->E + P / moe::kJobRows + 1);
+  w.n_jobs2 = carve<int>(cur, 1);
+  w.counter_bytes = counter_ints(h, Tm) * 4;
   w.counters = carve<int>(cur, w.counter_bytes / 4);
   w.dense_list = carve<int4>(cur, h->E);
   w.n_dense = carve<int>(cur, 1);
@@ -188,7 +200,7 @@ cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, c
 size_t permute_smem_bytes(int E) { return moe::permute_smem_ints(E) * 4; }
 
 size_t route_smem_bytes(int E, int d, int P) {
-  return std::max((size_t)d * 4, (moe::permute_smem_ints(E) + (size_t)P) * 4);
+  return std::max((size_t)d * 4 + 32 * 32 * 4, (moe::permute_smem_ints(E) + (size_t)P) * 4);
 }
 
 cudaError_t mark(moe_fp4* h, int i, cudaStream_t st) {
@@ -207,13 +219,15 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
   const uint16_t* xb = static_cast<const uint16_t*>(x);
   const bool pdl = !h->stage_timing;
   MOE_CUDA(mark(h, 0, st));
-  const size_t max_jobs = (size_t)E + (size_t)w.max_T * k / moe::kJobRows + 1;   // counter layout
-  int* gu_done = w.counters;
-  int* dn_done = gu_done + max_jobs;
-  int* exit_cnt = dn_done + d / 16;
-  int* ticket = exit_cnt + 1;
-  moe::PermuteOut po{w.counts, w.offsets, w.perm, w.inv, w.jobs, w.n_jobs, w.dense_list, w.n_dense,
-                     h->err};
+  const size_t max_jobs2 = (size_t)E + (size_t)w.max_T * k / moe::kJobRows + 1;   // counter layout
+  int* gu_done1 = w.counters;
+  int* gu_done2 = gu_done1 + E;
+  int* dn_done = gu_done2 + max_jobs2;
+  int* exit1 = dn_done + d / 16;
+  int* exit2 = exit1 + 1;
+  int* ticket = exit2 + 1;
+  moe::PermuteOut po{w.counts, w.offsets, w.perm, w.inv, w.jobs1, w.n_jobs1, w.jobs2, w.n_jobs2,
+                     w.dense_list, w.n_dense, h->err};
   if (T <= kSmallT) {
     // 1-3. router logits, x staging, top-k and permutation in one launch
     MOE_CUDA(launch(moe::route_kernel, dim3(E), dim3(1024), route_smem_bytes(E, d, T * k), st, false,
@@ -241,8 +255,6 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
   ep.cpt_gu = d / moe::kChunkK;
   ep.tpe_dn = d / 16;
   ep.cpt_dn = f / moe::kChunkK;
-  ep.jobs = w.jobs;
-  ep.njobs = w.n_jobs;
   ep.n_dense = w.n_dense;
   ep.perm = w.perm;
   ep.inv = w.inv;
@@ -259,15 +271,21 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
   ep.wts = w.wts;
   ep.partial = w.partial;
   ep.out = static_cast<uint16_t*>(out);
-  ep.gu_done = gu_done;
   ep.dn_done = dn_done;
-  ep.exit_cnt = exit_cnt;
   ep.err = h->err;
   ep.wait_timeout_ns = h->wait_timeout_ns;
-  MOE_CUDA(launch(moe::expert_kernel, dim3(h->sm_count * h->exp_bps), dim3(moe::kExpThreads), kExpSmem,
-                  st, pdl, ep));
+  moe::ExpertParams ep1 = ep, ep2 = ep;
+  ep1.jobs = w.jobs1; ep1.njobs = w.n_jobs1; ep1.gu_done = gu_done1; ep1.exit_cnt = exit1;
+  ep2.jobs = w.jobs2; ep2.njobs = w.n_jobs2; ep2.gu_done = gu_done2; ep2.exit_cnt = exit2;
+  MOE_CUDA(launch(moe::expert_kernel<1>, dim3(h->sm_count * h->exp_bps1), dim3(moe::kExpThreads),
+                  kExpSmem, st, pdl, ep1));
+  MOE_CUDA(launch(moe::expert_kernel<2>, dim3(h->sm_count * h->exp_bps2), dim3(moe::kExpThreads),
+                  kExpSmem, st, pdl, ep2));
   MOE_CUDA(mark(h, 4, st));
   MOE_CUDA(mark(h, 5, st));
+  // 7. combine / unpermute: out[t] = bf16(sum_j partial[inv[t,j]])
+  MOE_CUDA(launch(moe::combine_kernel, dim3((d + 1023) / 1024, T), dim3(128), 0, st, pdl,
+                  (const float*)w.partial, (const int*)w.inv, T, k, d, static_cast<uint16_t*>(out)));
   MOE_CUDA(mark(h, 6, st));
   return MOE_FP4_OK;
 }
@@ -333,17 +351,21 @@ int moe_fp4_create(int E, int top_k, int d, int f, moe_fp4_t** out) {
     auto smem_attr = [](const void* fn, size_t bytes) {
       return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     };
-    if (smem_attr((const void*)moe::expert_kernel, kExpSmem) != cudaSuccess ||
+    if (smem_attr((const void*)moe::expert_kernel<1>, kExpSmem) != cudaSuccess ||
+        smem_attr((const void*)moe::expert_kernel<2>, kExpSmem) != cudaSuccess ||
         smem_attr((const void*)moe::permute_kernel, permute_smem_bytes(E)) != cudaSuccess ||
         smem_attr((const void*)moe::route_kernel, route_smem_bytes(E, d, kSmallT * top_k)) != cudaSuccess) {
       rc = MOE_FP4_ERR_CUDA; break;
     }
-    int nb = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, moe::expert_kernel, moe::kExpThreads,
+    int nb1 = 0, nb2 = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb1, moe::expert_kernel<1>, moe::kExpThreads,
+                                                      kExpSmem) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb2, moe::expert_kernel<2>, moe::kExpThreads,
                                                       kExpSmem) != cudaSuccess) {
       rc = MOE_FP4_ERR_CUDA; break;
     }
-    h->exp_bps = std::max(1, nb);
+    h->exp_bps1 = std::max(1, nb1);
+    h->exp_bps2 = std::max(1, nb2);
     if (cudaMalloc(&h->err, sizeof(int)) != cudaSuccess) { rc = MOE_FP4_ERR_OOM; break; }
     if (cudaMemset(h->err, 0, sizeof(int)) != cudaSuccess) { rc = MOE_FP4_ERR_CUDA; break; }
     if (cudaMalloc(&h->gs, sizeof(float) * 3 * E) != cudaSuccess) { rc = MOE_FP4_ERR_OOM; break; }

@@ -51,11 +51,24 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// try_wait with a suspend-time hint: the thread sleeps (up to hint_ns) until
+// the phase completes instead of spinning, leaving issue slots to the warps
+// that have data to work on.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t phase, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok) : "r"(bar), "r"(phase), "r"(hint_ns) : "memory");
+  return ok != 0;
+}
+
 // Bounded wait: returns false once the global timer passes `deadline_ns`.
 __device__ __forceinline__ bool mbar_wait_until(uint32_t bar, uint32_t phase, uint64_t deadline_ns) {
-  uint32_t n = 0;
-  while (!mbar_try_wait(bar, phase)) {
-    if ((++n & 255u) == 0 && globaltimer_ns() > deadline_ns) return false;
+  if (mbar_try_wait(bar, phase)) return true;
+  while (!mbar_try_wait_sleep(bar, phase, 200000u)) {
+    if (globaltimer_ns() > deadline_ns) return false;
   }
   return true;
 }

@@ -202,7 +202,9 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 // 32-pair step, so no atomics), the counts are scanned, and a second walk
 // assigns positions in (expert, pair) order -- deterministic and stable.
 // Then the active experts are classed by row count n:
-//   light (n < thr): cut into jobs of <= 16 rows, listed heavy expert first;
+//   light (n < thr): cut into jobs of 16 rows plus one remainder job; jobs of
+//     <= 8 rows go to list 1 (one 8-wide MMA n-tile), jobs of 9..16 rows to
+//     list 2 (two n-tiles); each list is ordered heavy expert first;
 //   dense (n >= thr): listed by n descending.
 // Shared memory (ints): 32*E (warp counts) + 4*E + 1 (counts, offsets,
 // active list) + 8 scalars.
@@ -212,8 +214,10 @@ struct PermuteOut {
   int* offsets;      // [E+1]
   int* perm;         // [P]
   int* inv;          // [P]
-  int4* jobs;        // [E + P/16 + 1] {expert, row0, nrows, 0}, 1 <= nrows <= 16
-  int* n_jobs;
+  int4* jobs1;       // [E]            {expert, row0, nrows, 0}, 1 <= nrows <= 8
+  int* n_jobs1;
+  int4* jobs2;       // [E + P/16 + 1] {expert, row0, nrows, 0}, 9 <= nrows <= 16
+  int* n_jobs2;
   int4* dense_list;  // [E]            {expert, row0, nrows, 0}
   int* n_dense;
   int* err;
@@ -227,7 +231,7 @@ __device__ void build_permutation(const int* ids, int T, int k, int E, int thr, 
   int* cnt = wc + 32 * E;       // [E]
   int* off = cnt + E;           // [E+1]
   int* act = off + E + 1;       // [E]  active experts, ascending
-  int* misc = act + E;          // [8]  0: n_active 1: n_jobs 3: n_dense
+  int* misc = act + E;          // [8]  0: n_active 1: n_jobs1 2: n_jobs2 3: n_dense
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const long long P = (long long)T * k;
   const long long c0 = P * warp / 32, c1 = P * (warp + 1) / 32;
@@ -301,20 +305,26 @@ __device__ void build_permutation(const int* ids, int T, int k, int E, int thr, 
     const int e = act[a];
     const int n = cnt[e];
     const bool light = n < thr;
-    int rank = 0, start = 0;
+    int rank = 0, s1 = 0, s2 = 0;
     for (int b = 0; b < A; ++b) {
       const int e2 = act[b], n2 = cnt[e2];
       if ((n2 < thr) != light) continue;
       if (n2 > n || (n2 == n && e2 < e)) {
         ++rank;
-        start += (n2 + kJobRows - 1) / kJobRows;
+        const int r2 = n2 % kJobRows;
+        s1 += (r2 > 0 && r2 <= 8) ? 1 : 0;
+        s2 += n2 / kJobRows + (r2 > 8 ? 1 : 0);
       }
     }
     if (light) {
-      const int nj = (n + kJobRows - 1) / kJobRows;
-      for (int q = 0; q < nj; ++q)
-        o.jobs[start + q] = make_int4(e, off[e] + q * kJobRows, min(kJobRows, n - q * kJobRows), 0);
-      atomicAdd(&misc[1], nj);
+      for (int r0 = 0; r0 < n; r0 += kJobRows) {
+        const int nr = min(kJobRows, n - r0);
+        const int4 jb = make_int4(e, off[e] + r0, nr, 0);
+        if (nr <= 8) o.jobs1[s1] = jb; else o.jobs2[s2++] = jb;
+      }
+      const int r = n % kJobRows;
+      atomicAdd(&misc[1], (r > 0 && r <= 8) ? 1 : 0);
+      atomicAdd(&misc[2], n / kJobRows + (r > 8 ? 1 : 0));
     } else {
       o.dense_list[rank] = make_int4(e, off[e], n, 0);
       atomicAdd(&misc[3], 1);
@@ -322,7 +332,8 @@ __device__ void build_permutation(const int* ids, int T, int k, int E, int thr, 
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    *o.n_jobs = misc[1];
+    *o.n_jobs1 = misc[1];
+    *o.n_jobs2 = misc[2];
     *o.n_dense = misc[3];
     if (misc[3] > 0 && !dense_supported) set_error(o.err, kErrUnsupported);
   }
@@ -353,27 +364,63 @@ __global__ void __launch_bounds__(1024) route_kernel(
   const int e = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   float* s_w = reinterpret_cast<float*>(sm);
-  for (int i = threadIdx.x; i < d / 4; i += blockDim.x)
-    reinterpret_cast<float4*>(s_w)[i] = reinterpret_cast<const float4*>(rw + (size_t)e * d)[i];
-  __syncthreads();
-  for (int t = warp; t < T; t += 32) {
-    const uint16_t* xr = x + (size_t)t * d;
-    float acc = 0.f;
-    for (int kk = lane * 8; kk < d; kk += 256) {
-      const uint4 xv = *reinterpret_cast<const uint4*>(xr + kk);
-      const float4 a = *reinterpret_cast<const float4*>(s_w + kk);
-      const float4 bq = *reinterpret_cast<const float4*>(s_w + kk + 4);
-      acc = fmaf(__uint_as_float(xv.x << 16), a.x, acc);
-      acc = fmaf(__uint_as_float(xv.x & 0xffff0000u), a.y, acc);
-      acc = fmaf(__uint_as_float(xv.y << 16), a.z, acc);
-      acc = fmaf(__uint_as_float(xv.y & 0xffff0000u), a.w, acc);
-      acc = fmaf(__uint_as_float(xv.z << 16), bq.x, acc);
-      acc = fmaf(__uint_as_float(xv.z & 0xffff0000u), bq.y, acc);
-      acc = fmaf(__uint_as_float(xv.w << 16), bq.z, acc);
-      acc = fmaf(__uint_as_float(xv.w & 0xffff0000u), bq.w, acc);
+  {
+    // d <= 16384: at most 4 float4 per thread, all loads issued before the stores
+    const float4* src = reinterpret_cast<const float4*>(rw + (size_t)e * d);
+    float4 v[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int i = threadIdx.x + q * blockDim.x;
+      if (i < d / 4) v[q] = src[i];
     }
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) logits[(size_t)t * E + e] = acc;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int i = threadIdx.x + q * blockDim.x;
+      if (i < d / 4) reinterpret_cast<float4*>(s_w)[i] = v[q];
+    }
+  }
+  __syncthreads();
+  // every thread owns up to 2 groups of 8 consecutive K (d <= 16384); per token
+  // the 32 warp sums meet in shared memory (tokens in batches of 32)
+  float* s_part = reinterpret_cast<float*>(sm) + d;     // [32 tokens][32 warps]
+  float4 wa[2], wb[2];
+  bool has[2];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const int kk = 8 * (threadIdx.x + q * blockDim.x);
+    has[q] = kk < d;
+    wa[q] = has[q] ? *reinterpret_cast<const float4*>(s_w + kk) : make_float4(0, 0, 0, 0);
+    wb[q] = has[q] ? *reinterpret_cast<const float4*>(s_w + kk + 4) : make_float4(0, 0, 0, 0);
+  }
+  for (int t0 = 0; t0 < T; t0 += 32) {
+    const int tn = min(32, T - t0);
+    for (int tt = 0; tt < tn; ++tt) {
+      const uint16_t* xr = x + (size_t)(t0 + tt) * d;
+      float acc = 0.f;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        if (has[q]) {
+          const uint4 xv = *reinterpret_cast<const uint4*>(xr + 8 * (threadIdx.x + q * blockDim.x));
+          acc = fmaf(__uint_as_float(xv.x << 16), wa[q].x, acc);
+          acc = fmaf(__uint_as_float(xv.x & 0xffff0000u), wa[q].y, acc);
+          acc = fmaf(__uint_as_float(xv.y << 16), wa[q].z, acc);
+          acc = fmaf(__uint_as_float(xv.y & 0xffff0000u), wa[q].w, acc);
+          acc = fmaf(__uint_as_float(xv.z << 16), wb[q].x, acc);
+          acc = fmaf(__uint_as_float(xv.z & 0xffff0000u), wb[q].y, acc);
+          acc = fmaf(__uint_as_float(xv.w << 16), wb[q].z, acc);
+          acc = fmaf(__uint_as_float(xv.w & 0xffff0000u), wb[q].w, acc);
+        }
+      }
+      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (lane == 0) s_part[tt * 32 + warp] = acc;
+    }
+    __syncthreads();
+    if (warp < tn) {                       // warp tt sums the 32 warp partials of token t0 + tt
+      float v = s_part[warp * 32 + lane];
+      for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+      if (lane == 0) logits[(size_t)(t0 + warp) * E + e] = v;
+    }
+    __syncthreads();
   }
   for (int t = e; t < T; t += gridDim.x)
     stage_x_row(x + (size_t)t * d, d, x16 + (size_t)t * d, xscale + t, o.err, red);
