@@ -180,6 +180,32 @@ MOE_FP4_API int moe_fp4_set_stage_events(moe_fp4_t* h, cudaEvent_t* events, int 
  * *code receives MOE_FP4_OK or the first MOE_FP4_ERR_* a kernel recorded. */
 MOE_FP4_API int moe_fp4_get_device_error(moe_fp4_t* h, int* code);
 
+/* Allocation-free routing: fp32 router logits, top-k (ties to the lower
+ * expert index) and the renormalised weights of every token, exactly the
+ * topk_ids / topk_w that moe_fp4_forward_ex reports, for callers that cannot
+ * call cudaMalloc: code that runs inside stream capture, under an external
+ * memory pool or allocator that owns all device memory, or in a process
+ * whose device memory budget is fixed in advance.  It needs no handle (a
+ * handle allocates) and allocates nothing: the logits live in a scratch
+ * array of MOE_FP4_STATIC_MAX_LOGITS floats (256 KB) that the library defines
+ * as a file-scope device array; every GPU that loads the library holds it
+ * until the process exits.  The pages this library follows have no
+ * counterpart of this call.
+ *   x_bf16    device, bf16 [T][d];   router_w device, fp32 [E][d]
+ *   topk_ids  device, int32 [T][top_k];   topk_w device, fp32 [T][top_k]
+ *   T >= 0 (0 is a no-op), T*E <= MOE_FP4_STATIC_MAX_LOGITS (else
+ *   MOE_FP4_ERR_UNSUPPORTED), E, top_k, d as in moe_fp4_create; pointers
+ *   16-byte aligned (else MOE_FP4_ERR_INVALID_ARG).
+ * The first call on each device looks the scratch array up on that device
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * Asynchronous on `stream`.  All calls share the one scratch array per
+ * device: calls whose executions overlap on the GPU (different streams
+ * without ordering) race and give undefined results. */
+#define MOE_FP4_STATIC_MAX_LOGITS 65536
+MOE_FP4_API int moe_fp4_route_topk_static(const void* x_bf16, int T, int d, const float* router_w,
+                                          int E, int top_k, int32_t* topk_ids, float* topk_w,
+                                          cudaStream_t stream);
+
 /* Static text for a status code. */
 MOE_FP4_API const char* moe_fp4_status_string(int status);
 

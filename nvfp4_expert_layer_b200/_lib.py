@@ -41,6 +41,7 @@ SIGNATURES = {
     "moe_fp4_set_dense_threshold": (_i, [_vp, _i]),
     "moe_fp4_get_device_error": (_i, [_vp, ctypes.POINTER(_i)]),
     "moe_fp4_set_stage_events": (_i, [_vp, ctypes.POINTER(_vp), _i]),
+    "moe_fp4_route_topk_static": (_i, [_vp, _i, _i, _vp, _i, _i, _vp, _vp, _vp]),
     "moe_fp4_status_string": (ctypes.c_char_p, [_i]),
     "moe_fp4_destroy": (None, [_vp]),
 }

@@ -13,6 +13,7 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include "moe_fp4.h"
@@ -513,3 +514,54 @@ int moe_fp4_get_device_error(moe_fp4_t* h, int* code) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free routing (moe_fp4_route_topk_static).
+// The logits scratch is a file-scope device array; host code cannot use the
+// symbol itself as a device address (in host code it names a host-side
+// stand-in), so its device address is looked up once per device, with that
+// device current, and passed to the kernels.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) float g_route_scratch[MOE_FP4_STATIC_MAX_LOGITS];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+float* g_scratch_ptr[kMaxDevices] = {};
+
+int route_scratch(float** out) {
+  int dev = 0;
+  MOE_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return MOE_FP4_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    MOE_CUDA(cudaGetSymbolAddress(&p, g_route_scratch));
+    g_scratch_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_scratch_ptr[dev];
+  return MOE_FP4_OK;
+}
+}  // namespace
+
+extern "C" int moe_fp4_route_topk_static(const void* x_bf16, int T, int d, const float* router_w,
+                                         int E, int top_k, int32_t* topk_ids, float* topk_w,
+                                         cudaStream_t stream) {
+  if (T < 0) return MOE_FP4_ERR_INVALID_ARG;
+  if (E < 1 || E > 1024 || top_k < 1 || top_k > std::min(E, 32) || d < 128 || d > 16384 || d % 128)
+    return MOE_FP4_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_FP4_OK;
+  if (!x_bf16 || !router_w || !topk_ids || !topk_w) return MOE_FP4_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x_bf16) | reinterpret_cast<uintptr_t>(router_w) |
+       reinterpret_cast<uintptr_t>(topk_ids) | reinterpret_cast<uintptr_t>(topk_w)) & 15)
+    return MOE_FP4_ERR_INVALID_ARG;
+  if ((long long)T * E > MOE_FP4_STATIC_MAX_LOGITS) return MOE_FP4_ERR_UNSUPPORTED;
+  float* logits = nullptr;
+  const int rc = route_scratch(&logits);
+  if (rc != MOE_FP4_OK) return rc;
+  MOE_CUDA(launch(moe::router_tiled_kernel, dim3((T + 63) / 64, (E + 63) / 64), dim3(256), 0, stream,
+                  false, static_cast<const uint16_t*>(x_bf16), router_w, T, d, E, logits));
+  MOE_CUDA(launch(moe::topk_kernel, dim3((T + 7) / 8), dim3(256), 0, stream, false,
+                  (const float*)logits, T, E, top_k, topk_ids, topk_w));
+  return MOE_FP4_OK;
+}
