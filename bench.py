@@ -1,14 +1,22 @@
 """Benchmark of the NVFP4 sparse-MoE layer forward on B200 (one JSON line).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
-                    [--workload decode1|decode64|verify|tiny]
+                    [--workload decode1|decode64|verify|prefill|tiny]
 
 A step is one forward of the layer (routing, permutation, gate/up + SwiGLU,
 down, combine) over one batch of synthetic tokens.  The default workload is
 batch-1 decode (T=1, d=7168, E=256, top-8, f=2048, NVFP4 experts).  Inputs
 are seeded and synthetic; every step takes the next x of a pool of 32
 distinct token batches whose routing touches different experts, so the
-weights a step streams were evicted from L2 by the steps in between.
+weights a step streams were evicted from L2 by the steps in between (the
+prefill workload, 16384 tokens, uses a pool of 2: one x alone is 235 MB,
+larger than L2, and every step touches all experts).
+
+Roofline of the dominant kernel: for decode shapes the light-class expert
+kernel against HBM bandwidth (algorithmic bytes = NVFP4 bytes of the experts
+the step routes to); for prefill the dense gate/up GEMM against the FP4
+tensor-core peak (algorithmic FLOPs = 2 * rows * d * 2f over the routed rows,
+padding excluded).
 
 Timing: K steps replayed as one CUDA graph each, bracketed by a barrier and
 torch.cuda.synchronize on both sides, timed with CUDA events on the stream the
@@ -35,6 +43,7 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE-layer tokens/s; decode HBM GB/s and prefill FP4 TFLOP/s vs B200 roofline"
 EXPERT_BYTES = None   # set from the config: bytes of one expert (gate + up + down, NVFP4)
 POOL = 32
+FP4_OVER_BF16 = 4.0   # nominal dense FP4 / BF16 tensor throughput ratio on B200 (9 / 2.25 PFLOP/s)
 
 
 def parse():
@@ -55,12 +64,19 @@ def expert_bytes(cfg) -> int:
 
 
 def measured_peaks():
+    """(HBM GB/s, dense FP4 TFLOP/s, kind).  FP4 = measured bf16 burst x 4."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
             mp = json.load(fh)
-        return mp["hbm_gbs"], "measured"
+        return mp["hbm_gbs"], mp["bf16_tflops"] * FP4_OVER_BF16, "measured"
     except Exception:
-        return 6650.0, "fallback"
+        return 6650.0, 1590.0 * FP4_OVER_BF16, "fallback"
+
+
+def is_dense(cfg, thr=128) -> bool:
+    """Whether the workload's experts run in the dense class (T >= thr and the
+    shapes the tensor-core path supports)."""
+    return cfg.T >= thr and cfg.d % 256 == 0 and cfg.f % 256 == 0
 
 
 def source_digest() -> str:
@@ -251,15 +267,20 @@ def run_native(args, rank, world, local):
     del dev
     torch.cuda.empty_cache()
     layer.reserve(cfg.T)
-    xs_np, rw_np = pool_inputs(cfg, POOL)
+    pool = 2 if cfg.T * cfg.d * 2 > 126e6 else POOL
+    xs_np, rw_np = pool_inputs(cfg, pool)
     xs = [torch.from_numpy(x.view(np.int16).copy()).cuda().view(torch.bfloat16) for x in xs_np]
     rw = torch.from_numpy(rw_np).cuda()
     out = torch.empty_like(xs[0])
-    # distinct experts each pool input routes to (units of work of one step), from the layer itself
-    experts_per_input = []
+    # units of work of one step, from the layer's own routing: distinct experts
+    # touched (decode bytes) and rows of dense-class experts (prefill FLOPs)
+    dense = is_dense(cfg)
+    experts_per_input, dense_rows = [], []
     for x in xs:
         _, dbg = layer.forward_ex(x, rw, want=("counts",))
-        experts_per_input.append(int((dbg["counts"] > 0).sum().item()))
+        c = dbg["counts"].cpu().numpy()
+        experts_per_input.append(int((c > 0).sum()))
+        dense_rows.append(int(c[c >= 128].sum()) if dense else 0)
     stream = torch.cuda.Stream()
     graphs = []
     with torch.cuda.stream(stream):
@@ -275,7 +296,7 @@ def run_native(args, rank, world, local):
     assert layer.device_error() == 0
     cur = torch.cuda.current_stream()
     for i in range(args.warmup):
-        graphs[i % POOL].replay()
+        graphs[i % pool].replay()
     torch.cuda.synchronize()
     # ---- timed region (headline)
     clocks = ClockSampler(local)
@@ -285,7 +306,7 @@ def run_native(args, rank, world, local):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(cur)
     for i in range(args.steps):
-        graphs[i % POOL].replay()
+        graphs[i % pool].replay()
     e1.record(cur)
     torch.cuda.synchronize()
     barrier(world)
@@ -293,11 +314,13 @@ def run_native(args, rank, world, local):
     ms = allreduce_max(e0.elapsed_time(e1), world)
     err = layer.device_error()
     # ---- per-stage pass: the same graphs with stage events (events between stages)
-    stage_ms = np.zeros(6)
+    nst = len(layer.STAGES)
+    dom = layer.STAGES.index("dense_gate_up" if dense else "light")
+    stage_ms = np.zeros(nst)
     sgraphs, sevents = [], []
     with torch.cuda.stream(stream):
         for x in xs:
-            evs = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)]
             layer.set_stage_events(evs)
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
@@ -306,31 +329,34 @@ def run_native(args, rank, world, local):
             sevents.append(evs)
         layer.set_stage_events(None)
     torch.cuda.synchronize()
-    for i in range(POOL):
+    for i in range(pool):
         sgraphs[i].replay()
     torch.cuda.synchronize()
-    dom_ms, dom_bytes, n = 0.0, 0.0, 0
-    for rep in range(max(1, args.steps // POOL)):
-        for i in range(POOL):
+    dom_ms, dom_work, n = 0.0, 0.0, 0
+    for rep in range(max(1, args.steps // pool)):
+        for i in range(pool):
             sgraphs[i].replay()
         torch.cuda.synchronize()
-        for i in range(POOL):
-            d = [sevents[i][j].elapsed_time(sevents[i][j + 1]) for j in range(6)]
+        for i in range(pool):
+            d = [sevents[i][j].elapsed_time(sevents[i][j + 1]) for j in range(nst)]
             stage_ms += d
-            dom_ms += d[3]
-            dom_bytes += experts_per_input[i] * expert_bytes(cfg)
+            dom_ms += d[dom]
+            if dense:   # gate and up GEMMs over the routed rows: 2 * rows * d * 2f
+                dom_work += 2.0 * dense_rows[i] * cfg.d * 2 * cfg.f
+            else:
+                dom_work += experts_per_input[i] * expert_bytes(cfg)
             n += 1
     stage_ms /= n
     # ---- end to end through the C ABI with host buffers
     xh = [torch.from_numpy(x.view(np.int16).copy()).view(torch.bfloat16).pin_memory() for x in xs_np]
     oh = torch.empty_like(xh[0]).pin_memory()
     for i in range(3):
-        layer.forward_host(xh[i % POOL], rw, out_host=oh, stream=stream)
+        layer.forward_host(xh[i % pool], rw, out_host=oh, stream=stream)
     barrier(world)
     ee0, ee1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ee0.record(stream)
     for i in range(args.steps):
-        layer.forward_host(xh[i % POOL], rw, out_host=oh, stream=stream)
+        layer.forward_host(xh[i % pool], rw, out_host=oh, stream=stream)
     ee1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = allreduce_max(ee0.elapsed_time(ee1), world)
@@ -338,9 +364,14 @@ def run_native(args, rank, world, local):
     layer(xs[0], rw, out=out)
     torch.cuda.synchronize()
     gpu_out0 = out.view(torch.int16).cpu().numpy().view(np.uint16).copy()
+    # kernels per step: routing (1 fused launch up to 256 tokens, else router,
+    # x staging, top-k, permutation), the dense class (quantiser + 2 GEMMs)
+    # when T >= thr, the two light-class expert kernels and the combine
+    launches = (1 if cfg.T <= 256 else 4) + (3 if cfg.T >= 128 else 0) + 3
     return dict(cfg=cfg, ms=ms, clk=clk, err=err, stage_ms=stage_ms, dom_ms=dom_ms / n,
-                dom_bytes=dom_bytes / n, e2e_ms=e2e_ms, xs_np=xs_np, rw_np=rw_np, gpu_out0=gpu_out0,
-                launches_per_step=(4 if cfg.T <= 256 else 6), stages=layer.STAGES)
+                dom_work=dom_work / n, dense=dense, e2e_ms=e2e_ms, xs_np=xs_np, rw_np=rw_np,
+                gpu_out0=gpu_out0, launches_per_step=launches, stages=layer.STAGES,
+                dense_rows=float(np.mean(dense_rows)), pool=pool)
 
 
 def parity_vs_oracle(res_oracle, gpu_bits, tol=1e-2):
@@ -352,13 +383,31 @@ def parity_vs_oracle(res_oracle, gpu_bits, tol=1e-2):
     gv = O.bf16_bits_to_f64(gpu_bits[toks])
     rms = float(np.sqrt(np.mean(ov ** 2)))
     half = np.exp2(np.floor(np.log2(np.maximum(np.abs(ov), 2.0 ** -126))) - 8)
-    ok = bool(np.all(np.abs(gv - ov) <= tol * rms + half)) and not bool(np.any(O.near_tie_flags(res_oracle["gap"])))
+    ties = bool(np.any(O.near_tie_flags(res_oracle["gap"])[toks]))
+    ok = bool(np.all(np.abs(gv - ov) <= tol * rms + half)) and not ties
     return ("pass" if ok else "fail"), float(np.abs(gv - ov).max() / rms)
 
 
 def cpu_baseline_sample(cfg, xs_np, rw_np):
-    """Oracle on a bounded sample: the first pool input (all of its tokens when
-    T <= 8, else its first 8 tokens)."""
+    """Oracle on a bounded sample of the first pool input: all of its tokens
+    when T <= 8, else its first 8 tokens as a batch of their own.  When the
+    workload's experts run in the dense class, the sample keeps the whole
+    batch's routing (which decides the class) and evaluates the experts of
+    its first token only."""
+    if is_dense(cfg):
+        from nvfp4_expert_layer_b200 import workloads as W
+        from oracle import moe_oracle as O
+        lazy = W.LazyExperts(cfg)
+        ids, _, _ = O.route(O.router_logits(xs_np[0][:1], rw_np), cfg.k)
+        for e in np.unique(ids):
+            lazy.expert(int(e))
+        t0 = time.perf_counter()
+        res = O.forward(xs_np[0], rw_np, lazy, cfg.E, cfg.k, thr=128, token_subset=[0])
+        secs = time.perf_counter() - t0
+        sample = (f"oracle on the {cfg.name} workload: routing and permutation of all {cfg.T} tokens "
+                  f"(fp64 logits), then the {cfg.k} experts of token 0 in the dense class (NVFP4 "
+                  f"activations) dequantised exactly and evaluated in fp64; value = 1 token / time")
+        return secs, 1, res, sample
     n = min(cfg.T, 8)
     secs, res = oracle_sample(cfg, xs_np[0], rw_np, n)
     sample = (f"oracle on {n} token(s) of the {cfg.name} workload: routing over {cfg.E} experts, "
@@ -406,24 +455,36 @@ def main():
     r = run_native(args, rank, world, local)
     tokens = cfg.T * args.steps * world
     value = tokens / (r["ms"] * 1e-3)
-    peak, peak_kind = measured_peaks()
-    achieved = r["dom_bytes"] / (r["dom_ms"] * 1e-3) / 1e9
+    hbm_peak, fp4_peak, peak_kind = measured_peaks()
+    if r["dense"]:
+        achieved = r["dom_work"] / (r["dom_ms"] * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "kernel": "dense_gemm_kernel<gate/up> (tcgen05 NVFP4, dense class)",
+                    "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s", "frac": achieved / fp4_peak,
+                    "peak_kind": f"{peak_kind} bf16 burst x {FP4_OVER_BF16:g} (nominal FP4/BF16 ratio)",
+                    "traffic": recorded_traffic("dense_gemm_kernel_gate_up"),
+                    "algorithmic_flops_per_launch": r["dom_work"], "avg_launch_ms": r["dom_ms"]}
+        compute = ("x and h quantised to NVFP4 (e4m3 scale per 16), tcgen05 block-scaled FP4 MMA, "
+                   "fp32 accumulate in TMEM")
+    else:
+        achieved = r["dom_work"] / (r["dom_ms"] * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "kernel": "expert_kernel (gate/up + SwiGLU + down, light class)",
+                    "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+                    "peak_kind": peak_kind, "traffic": recorded_traffic("expert_kernel"),
+                    "algorithmic_bytes_per_launch": r["dom_work"], "avg_launch_ms": r["dom_ms"]}
+        compute = "fp4 weights dequantised in registers to fp16, m16n8k16 MMA, fp32 accumulate"
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": r["ms"] / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp4" if r["dense"] else "f16",
         "data": "synthetic (seeded; NVFP4 experts from N(0,0.02), x ~ N(0,1) bf16)",
         "config": {"workload": f"{cfg.name}: T={cfg.T} tokens, d={cfg.d}, E={cfg.E}, top-{cfg.k}, f={cfg.f}, "
                                "NVFP4 experts (e2m1 + e4m3/16 + fp32 tensor scale)",
                    "global_batch": cfg.T * world, "parallelism": f"replicas x{world}",
-                   "l2": f"inputs rotate over {POOL} token batches; their experts span "
-                         f"{cfg.E * expert_bytes(cfg) / 1e9:.2f} GB > 126 MB L2",
+                   "l2": f"inputs rotate over {r['pool']} token batches of {cfg.T * cfg.d * 2 / 1e6:.1f} MB; "
+                         f"their experts span {cfg.E * expert_bytes(cfg) / 1e9:.2f} GB > 126 MB L2",
                    "timing": "CUDA graph replay per step, CUDA events on the launch stream, max over ranks",
-                   "compute": "fp4 weights dequantised in registers to fp16, m16n8k16 MMA, fp32 accumulate"},
-        "roofline": {"bound": "hbm", "kernel": "expert_kernel (gate/up + SwiGLU + down, light class)",
-                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_kind": peak_kind, "traffic": recorded_traffic("expert_kernel"),
-                     "algorithmic_bytes_per_launch": r["dom_bytes"], "avg_launch_ms": r["dom_ms"]},
+                   "compute": compute},
+        "roofline": roofline,
         "stage_us": {n: round(float(v) * 1e3, 2) for n, v in zip(r["stages"], r["stage_ms"])},
         "clocks": r["clk"],
         "e2e": {"value": tokens / (r["e2e_ms"] * 1e-3), "unit": "tokens/s",

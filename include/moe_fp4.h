@@ -35,7 +35,10 @@
  *                            q = e2m1_rn(v/sf), decisions in fp32) and the
  *                            expert runs on block-scaled FP4 tensor cores.
  *   The threshold defaults to 128 (environment MOE_FP4_DENSE_THRESHOLD at
- *   create time, or moe_fp4_set_dense_threshold).
+ *   create time, or moe_fp4_set_dense_threshold).  The dense class needs d
+ *   and f to be multiples of 256 (one 256-element K stage of the tensor-core
+ *   pipeline); for other shapes, or if the driver's tensor-map encoder is not
+ *   available, every expert runs in the light class whatever its row count.
  *
  * Conventions
  *   - Every call returns a moe_fp4_status and never aborts the process.
@@ -164,16 +167,18 @@ MOE_FP4_API int moe_fp4_forward_host(moe_fp4_t* h, const void* x_host, int T, co
 /* Activation-precision threshold (see the top of this file); thr >= 1. */
 MOE_FP4_API int moe_fp4_set_dense_threshold(moe_fp4_t* h, int thr);
 
-/* Stage timing (profiling hook).  With n = 7, every later forward records
- * events[0] before the router, events[1] after the router (and x staging),
- * events[2] after top-k, events[3] after the permutation, events[4] after the
- * gate/up + SwiGLU kernels, events[5] after the down kernels and events[6]
- * after the combine, all on the forward's stream (as external event nodes
- * when the stream is being captured into a CUDA graph).  The events must be
- * created with timing enabled; the caller owns them.  n = 0 (events may be
- * NULL) turns the hook off.  Any other n is MOE_FP4_ERR_INVALID_ARG.
- * Recording between stages serialises kernels that would otherwise overlap
- * through programmatic dependent launch. */
+/* Stage timing (profiling hook).  With n = 9, every later forward records,
+ * on the forward's stream, events[0] before the router, events[1] after the
+ * router (and x staging), events[2] after top-k, events[3] after the
+ * permutation, events[4] after the dense-class activation quantiser,
+ * events[5] after the dense gate/up + SwiGLU GEMM, events[6] after the dense
+ * down GEMM (4-6 follow 3 directly when T < thr and no expert can be dense),
+ * events[7] after the light-class expert kernels and events[8] after the
+ * combine (as external event nodes when the stream is being captured into a
+ * CUDA graph).  The events must be created with timing enabled; the caller
+ * owns them.  n = 0 (events may be NULL) turns the hook off.  Any other n is
+ * MOE_FP4_ERR_INVALID_ARG.  Recording between stages serialises kernels that
+ * would otherwise overlap through programmatic dependent launch. */
 MOE_FP4_API int moe_fp4_set_stage_events(moe_fp4_t* h, cudaEvent_t* events, int n);
 
 /* Read and clear the device error word (synchronises the handle's device).

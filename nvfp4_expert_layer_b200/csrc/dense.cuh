@@ -1,0 +1,400 @@
+// Dense expert class: experts that received at least `thr` rows run as
+// grouped block-scaled NVFP4 GEMMs on the tcgen05 tensor cores, accumulating
+// in TMEM ("Optimizing Models to Be Fast at Codegen", section 2: keep the
+// weights 4-bit all the way to the tensor core and feed Blackwell's FP4
+// tensor cores from shared memory; "Optimizing Muse Spark Open on TPU v7 with
+// SGLang-TorchTPU", section 8: the fused MoE prefill kernel streams one
+// expert's weights while the next prefetches, then gate/up, SwiGLU and down).
+//
+// Activations of the dense class are NVFP4 too (e2m1 values, one e4m3 scale
+// per 16 along K, tensor scale 1): sf = e4m3_rn(amax / 6), q = e2m1_rn(v / sf),
+// both decided in IEEE fp32.  Rows of every dense expert are padded to a
+// multiple of 128 so each 128-token MMA tile starts on a scale-atom boundary.
+//
+// GEMM 1 (kDenseGateUp): D[128 rows = 64 gate + 64 up rows of W][128 tokens]
+//   over K = d; the epilogue forms h = SiLU(g) * u, quantises it along f and
+//   writes the B operand of GEMM 2.
+// GEMM 2 (kDenseDown):   D[128 rows of Wd][128 tokens] over K = f; the
+//   epilogue writes w * gs * D as fp32 partials (rows in permutation order).
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include "ptx.cuh"
+#include "tc.cuh"
+
+namespace moe {
+
+constexpr int kDenseThreads = 192;        // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kDenseStages = 4;
+constexpr int kDenseTileBytes = 128 * 128; // 128 rows x 128 bytes (256 fp4 along K)
+constexpr int kDenseSfBytes = 4 * 512;     // 4 scale atoms (K = 256) per operand per stage
+constexpr int kDenseStageBytes = 2 * kDenseTileBytes + 2 * kDenseSfBytes;
+constexpr uint32_t kDenseTmemCols = 512;
+constexpr int kDenseBarBytes = (2 * kDenseStages + 6) * 8;   // mbarriers, padded to 16 bytes
+
+enum DenseMode { kDenseGateUp = 0, kDenseDown = 1 };
+
+// Dense list entry: {expert, row0 (permutation rows), rows, padded row0}.
+struct DenseParams {
+  CUtensorMap tmA0;      // gate/up: gate copy, box 128 B x 64 rows; down: down copy, box 128 B x 128 rows
+  CUtensorMap tmA1;      // gate/up: up copy, box 128 B x 64 rows
+  CUtensorMap tmB;       // activations (NVFP4, padded permutation order), box 128 B x 128 rows
+  const uint8_t* sfA;    // weight scale atoms
+  const uint8_t* sfB;    // activation scale atoms
+  const int4* dense;     // dense list, ranked by rows descending
+  const int* n_dense;
+  const int* ntoff;      // [E+1] exclusive prefix of ceil(rows / 128) over the dense list
+  int mt_per_expert;     // gate/up: f / 64; down: d / 128
+  int rows_per_expert;   // gate/up: f; down: d (rows of the weight copy per expert)
+  int kstages;           // K / 256
+  int kb64;              // K / 64
+  int d, f, topk;
+  const float* gs;       // [3][E]
+  int E;
+  const int* perm;
+  const float* wts;
+  // gate/up outputs
+  uint8_t* hq;           // [P_pad][f/2]
+  uint8_t* hsf;          // scale atoms of hq
+  float* h32;            // [P][f] or null
+  // down output
+  float* partial;        // [P][d]
+  int* err;
+  int64_t wait_timeout_ns;
+};
+
+// ---------------------------------------------------------------------------
+// Activation quantiser: one warp per padded row of the dense class.
+// src row (bf16) of token perm[row0 + i] / topk; rows past the expert's count
+// are written as zeros.  Output: codes [rows][K/2], scales in atom layout.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int dense_rank_of_padrow(const int4* dense, int nd, int prow) {
+  int lo = 0, hi = nd - 1;                       // pad0 increases with rank
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (dense[mid].w <= prow) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__global__ void __launch_bounds__(256) quant_x_dense_kernel(
+    const uint16_t* __restrict__ x, const int4* __restrict__ dense, const int* __restrict__ n_dense,
+    const int* __restrict__ pad_total, const int* __restrict__ perm, int topk, int d,
+    uint8_t* __restrict__ xq, uint8_t* __restrict__ xsf) {
+  pdl_wait();
+  const int nd = *n_dense;
+  if (nd == 0) { pdl_launch_dependents(); return; }
+  const int total = *pad_total;
+  const int lane = threadIdx.x & 31;
+  const int nblk = d / 16;
+  for (int prow = blockIdx.x * 8 + (threadIdx.x >> 5); prow < total; prow += gridDim.x * 8) {
+    const int j = dense_rank_of_padrow(dense, nd, prow);
+    const int4 de = dense[j];
+    const int i = prow - de.w;
+    const bool valid = i < de.z;
+    const uint16_t* src = valid ? x + (size_t)(perm[de.y + i] / topk) * d : nullptr;
+    for (int blk = lane; blk < nblk; blk += 32) {
+      uint2 codes = make_uint2(0, 0);
+      uint32_t sfbyte = 0;
+      if (valid) {
+        const uint4 a = *reinterpret_cast<const uint4*>(src + blk * 16);
+        const uint4 b = *reinterpret_cast<const uint4*>(src + blk * 16 + 8);
+        const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        float v[16];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          v[2 * q] = __uint_as_float(wv[q] << 16);
+          v[2 * q + 1] = __uint_as_float(wv[q] & 0xffff0000u);
+        }
+        float amax = 0.f;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) amax = fmaxf(amax, fabsf(v[q]));
+        sfbyte = f32x2_to_e4m3x2(0.f, amax / 6.0f) & 0xffu;
+        const float sf = e4m3_to_f32(sfbyte);
+        if (sf > 0.f) {
+          uint32_t c[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) c[q] = f32x2_to_e2m1x2(v[2 * q + 1] / sf, v[2 * q] / sf);
+          codes.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
+          codes.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
+        }
+      }
+      *reinterpret_cast<uint2*>(xq + (size_t)prow * (d / 2) + blk * 8) = codes;
+      xsf[sf_atom_offset(prow, blk, d / 64)] = (uint8_t)sfbyte;
+    }
+  }
+  pdl_launch_dependents();
+}
+
+
+// ---------------------------------------------------------------------------
+// Grouped block-scaled NVFP4 GEMM on tcgen05 (persistent, one block per SM).
+// Tiles are (dense rank j, M tile mt, token tile nt) with nt fastest, so
+// neighbouring blocks share the same weight tile through L2.
+// ---------------------------------------------------------------------------
+struct DenseTile {
+  int j, mt, nt;
+  int4 de;      // {expert, row0, rows, padded row0}
+};
+
+__device__ __forceinline__ DenseTile dense_tile(const int4* sd, const int* sntoff, int nd, int mtpe, int i) {
+  // find rank j with mtpe * ntoff[j] <= i < mtpe * ntoff[j+1]
+  int lo = 0, hi = nd - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (mtpe * sntoff[mid] <= i) lo = mid; else hi = mid - 1;
+  }
+  DenseTile t;
+  t.j = lo;
+  t.de = sd[lo];
+  const int ntj = sntoff[lo + 1] - sntoff[lo];
+  const int local = i - mtpe * sntoff[lo];
+  t.mt = local / ntj;
+  t.nt = local - t.mt * ntj;
+  return t;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(n) : "memory");
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __grid_constant__ DenseParams p) {
+  extern __shared__ __align__(1024) uint8_t dsm_raw[];
+  // 1024-byte alignment (shared-window offset) for the 128-byte-swizzled tiles
+  uint8_t* dsm = dsm_raw + ((1024u - (smem_u32(dsm_raw) & 1023u)) & 1023u);
+  uint8_t* meta = dsm + kDenseStages * kDenseStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(meta);                 // full[S] empty[S] accf[2] acce[2] done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(meta + kDenseBarBytes);
+  int* svote = reinterpret_cast<int*>(meta + kDenseBarBytes + 16);    // [4] epilogue wait outcomes
+  int4* sd = reinterpret_cast<int4*>(meta + kDenseBarBytes + 32);     // dense list (<= E entries)
+  int* sntoff = reinterpret_cast<int*>(sd + p.E);                     // [E+1]
+  float* ubuf = reinterpret_cast<float*>(sntoff + ((p.E + 4) & ~3));  // gate/up: [2][32][129]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();
+  const int nd = *p.n_dense;
+  if (nd == 0) { pdl_launch_dependents(); return; }
+  for (int i = threadIdx.x; i < nd; i += blockDim.x) sd[i] = p.dense[i];
+  for (int i = threadIdx.x; i <= nd; i += blockDim.x) sntoff[i] = p.ntoff[i];
+  const uint32_t bars_s = smem_u32(bars);
+  auto full_b = [&](int s) { return bars_s + 8 * s; };
+  auto empty_b = [&](int s) { return bars_s + 8 * (kDenseStages + s); };
+  auto accf_b = [&](int a) { return bars_s + 8 * (2 * kDenseStages + a); };
+  auto acce_b = [&](int a) { return bars_s + 8 * (2 * kDenseStages + 2 + a); };
+  const uint32_t done_b = bars_s + 8 * (2 * kDenseStages + 4);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDenseStages; ++s) { mbar_init(full_b(s), 1); mbar_init(empty_b(s), 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(accf_b(a), 1); mbar_init(acce_b(a), 4); }
+    mbar_init(done_b, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kDenseTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t acc_t0 = tmem, sfa_t = tmem + 256, sfb_t = tmem + 272;
+
+  const int ntiles = p.mt_per_expert * sntoff[nd];
+  const int G = gridDim.x, b = blockIdx.x;
+  const int my_tiles = b < ntiles ? (ntiles - 1 - b) / G + 1 : 0;
+  const uint64_t deadline = globaltimer_ns() + (uint64_t)p.wait_timeout_ns;
+  const uint32_t stage0 = smem_u32(dsm);
+  bool failed = false;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first(), pol_a = policy_evict_last();
+      tma_prefetch_desc(&p.tmA0);
+      if (MODE == kDenseGateUp) tma_prefetch_desc(&p.tmA1);
+      tma_prefetch_desc(&p.tmB);
+      int k = 0;
+      for (int it = 0; it < my_tiles && !failed; ++it) {
+        const DenseTile tl = dense_tile(sd, sntoff, nd, p.mt_per_expert, b + it * G);
+        const int e = tl.de.x;
+        const int brow = tl.de.w + tl.nt * 128;              // padded activation row
+        for (int ks = 0; ks < p.kstages; ++ks, ++k) {
+          const int s = k % kDenseStages;
+          if (!mbar_wait_until(empty_b(s), ((k / kDenseStages) & 1) ^ 1, deadline)) {
+            failed = true; set_error(p.err, kErrTimeout); break;
+          }
+          const uint32_t st = stage0 + s * kDenseStageBytes;
+          mbar_arrive_expect_tx(full_b(s), kDenseStageBytes);
+          if (MODE == kDenseGateUp) {
+            const int wrow = e * p.rows_per_expert + tl.mt * 64;
+            tma_load_2d(st, &p.tmA0, ks * 128, wrow, full_b(s), pol_w);
+            tma_load_2d(st + kDenseTileBytes / 2, &p.tmA1, ks * 128, wrow, full_b(s), pol_w);
+          } else {
+            tma_load_2d(st, &p.tmA0, ks * 128, e * p.rows_per_expert + tl.mt * 128, full_b(s), pol_w);
+          }
+          tma_load_2d(st + kDenseTileBytes, &p.tmB, ks * 128, brow, full_b(s), pol_a);
+          const uint8_t* sfa = p.sfA + ((size_t)(e * p.mt_per_expert + tl.mt) * p.kb64 + 4 * ks) * 512;
+          const uint8_t* sfb = p.sfB + ((size_t)(brow >> 7) * p.kb64 + 4 * ks) * 512;
+          bulk_g2s(st + 2 * kDenseTileBytes, sfa, kDenseSfBytes, full_b(s), pol_w);
+          bulk_g2s(st + 2 * kDenseTileBytes + kDenseSfBytes, sfb, kDenseSfBytes, full_b(s), pol_a);
+        }
+      }
+      // drain: every issued stage must land before the block exits
+      for (int kk = max(0, k - kDenseStages); kk < k; ++kk)
+        mbar_wait_until(full_b(kk % kDenseStages), (kk / kDenseStages) & 1,
+                        globaltimer_ns() + (uint64_t)p.wait_timeout_ns);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_nvf4(128);
+      int k = 0;
+      bool issued_any = false;
+      for (int it = 0; it < my_tiles && !failed; ++it) {
+        const int ab = it & 1;
+        if (!mbar_wait_until(acce_b(ab), ((it >> 1) & 1) ^ 1, deadline)) {
+          failed = true; set_error(p.err, kErrTimeout); break;
+        }
+        tc_fence_after();
+        const uint32_t acc = acc_t0 + ab * 128;
+        for (int ks = 0; ks < p.kstages; ++ks, ++k) {
+          const int s = k % kDenseStages;
+          if (!mbar_wait_until(full_b(s), (k / kDenseStages) & 1, deadline)) {
+            failed = true; set_error(p.err, kErrTimeout); break;
+          }
+          tc_fence_after();
+          const uint32_t st = stage0 + s * kDenseStageBytes;
+          const uint32_t sfa_s = st + 2 * kDenseTileBytes, sfb_s = sfa_s + kDenseSfBytes;
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) {
+            tc_cp_32x128b_x4(sfa_t + 4 * kb, smem_desc_sf(sfa_s + 512 * kb));
+            tc_cp_32x128b_x4(sfb_t + 4 * kb, smem_desc_sf(sfb_s + 512 * kb));
+          }
+          const uint64_t adesc = smem_desc_sw128(st), bdesc = smem_desc_sw128(st + kDenseTileBytes);
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb)
+            tc_mma_nvf4(acc, adesc + 2 * kb, bdesc + 2 * kb, idesc, sfa_t + 4 * kb, sfb_t + 4 * kb,
+                        (ks > 0 || kb > 0) ? 1u : 0u);
+          tc_commit(empty_b(s));
+          issued_any = true;
+        }
+        if (failed) break;
+        tc_commit(accf_b(ab));
+      }
+      // every MMA issued must complete before TMEM is released
+      if (issued_any) {
+        tc_commit(done_b);
+        mbar_wait_until(done_b, 0, globaltimer_ns() + (uint64_t)p.wait_timeout_ns);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;                              // TMEM lane quarter of this warp
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    for (int it = 0; it < my_tiles && !failed; ++it) {
+      const int ab = it & 1;
+      const DenseTile tl = dense_tile(sd, sntoff, nd, p.mt_per_expert, b + it * G);
+      // all epilogue warps take the same decision: each records whether its
+      // bounded wait succeeded, then they meet at a barrier every warp reaches
+      const bool ok = mbar_wait_until(accf_b(ab), (it >> 1) & 1, deadline);
+      if (lane == 0) svote[q] = ok ? 1 : 0;
+      named_bar_sync(2, 128);
+      const bool all_ok = svote[0] && svote[1] && svote[2] && svote[3];
+      named_bar_sync(2, 128);
+      if (!all_ok) {
+        failed = true;
+        if (lane == 0) set_error(p.err, kErrTimeout);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t acc = acc_t0 + ab * 128 + lane_base;
+      const int e = tl.de.x, ncols = min(128, tl.de.z - tl.nt * 128);
+      const int prow0 = tl.de.y + tl.nt * 128;           // permutation row of column 0
+      const int hrow0 = tl.de.w + tl.nt * 128;           // padded row of column 0
+      if (MODE == kDenseDown) {
+        const float gsd = p.gs[2 * p.E + e];
+        const int drow = tl.mt * 128 + q * 32 + lane;
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(acc + c0, r);
+          tmem_ld_wait();
+#pragma unroll 4
+          for (int c = 0; c < 32; ++c) {
+            const int n = c0 + c;
+            if (n < ncols) {
+              const float wv = p.wts[p.perm[prow0 + n]] * gsd;
+              p.partial[(size_t)(prow0 + n) * p.d + drow] = __uint_as_float(r[c]) * wv;
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acce_b(ab));
+      } else {
+        // quarters 2, 3 hold up rows; 0, 1 gate rows of the same 64 channels
+        float* ub = ubuf + (size_t)((q & 1) * 32 + lane) * 129;
+        if (q >= 2) {
+          for (int c0 = 0; c0 < 128; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(acc + c0, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) ub[c0 + c] = __uint_as_float(r[c]);
+          }
+        }
+        named_bar_sync(1, 128);                           // up values staged
+        if (q < 2) {
+          const float gsg = p.gs[e], gsu = p.gs[p.E + e];
+          const int fidx = tl.mt * 64 + q * 32 + lane;
+          for (int c0 = 0; c0 < 128; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(acc + c0, r);
+            tmem_ld_wait();
+            for (int c = 0; c < 32; ++c) {
+              const int n = c0 + c;
+              if (n >= ncols) break;                      // warp-uniform
+              const float gv = __uint_as_float(r[c]) * gsg;
+              const float uv = ub[n] * gsu;
+              const float hv = gv / (1.f + expf(-gv)) * uv;
+              if (p.h32) p.h32[(size_t)(prow0 + n) * p.f + fidx] = hv;
+              // NVFP4 along f: 16 lanes form one block
+              float am = fabsf(hv);
+#pragma unroll
+              for (int o = 8; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+              const uint32_t sfbyte = f32x2_to_e4m3x2(0.f, am / 6.0f) & 0xffu;
+              const float sf = e4m3_to_f32(sfbyte);
+              const uint32_t code = sf > 0.f ? (f32x2_to_e2m1x2(0.f, hv / sf) & 0xfu) : 0u;
+              const uint32_t hi = __shfl_down_sync(0xffffffffu, code, 1);
+              const int hr = hrow0 + n;
+              if ((lane & 1) == 0) p.hq[(size_t)hr * (p.f / 2) + (fidx >> 1)] = (uint8_t)(code | (hi << 4));
+              if ((lane & 15) == 0) p.hsf[sf_atom_offset(hr, fidx >> 4, p.f / 64)] = (uint8_t)sfbyte;
+            }
+          }
+        }
+        tc_fence_before();
+        named_bar_sync(1, 128);                           // up values consumed
+        if (lane == 0) mbar_arrive(acce_b(ab));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kDenseTmemCols);
+  }
+  pdl_launch_dependents();
+}
+
+template <int MODE>
+constexpr size_t dense_smem_size(int E) {
+  return 1024 + (size_t)kDenseStages * kDenseStageBytes + kDenseBarBytes + 32 + (size_t)E * 16 +
+         (size_t)((E + 4) & ~3) * 4 + (MODE == kDenseGateUp ? 2 * 32 * 129 * 4 : 0);
+}
+
+}  // namespace moe

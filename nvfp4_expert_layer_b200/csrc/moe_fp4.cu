@@ -7,10 +7,12 @@
 //   -> [dense class on block-scaled FP4 tensor cores] -> combine / unpermute.
 // No host synchronisation happens inside moe_fp4_forward; the expert kernels
 // read the class lists the permutation kernel left on the device.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
 #include <cstdint>
+#include <climits>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -23,11 +25,14 @@
 #include "repack.cuh"
 #include "experts.cuh"
 #include "combine.cuh"
+#include "dense.cuh"
 
 namespace {
 
 constexpr int kSmallT = 256;          // fused routing kernel up to this many tokens
 constexpr size_t kExpSmem = moe::expert_smem_size();
+constexpr int kDenseGridPerSm = 1;
+constexpr int kStageEvents = 9;
 
 struct Workspace {
   void* base = nullptr;
@@ -48,6 +53,14 @@ struct Workspace {
   size_t counter_bytes = 0;
   int4* dense_list = nullptr;
   int* n_dense = nullptr;
+  int* dense_ntoff = nullptr;    // [E+1]
+  int* dense_pad_total = nullptr;
+  uint8_t* xq = nullptr;         // dense class: NVFP4 activations [pad_rows][d/2]
+  uint8_t* xsf = nullptr;        //   and their scale atoms
+  uint8_t* hq = nullptr;         // [pad_rows][f/2]
+  uint8_t* hsf = nullptr;
+  size_t pad_rows = 0;
+  CUtensorMap tm_x{}, tm_h{};    // B operands of the dense GEMMs
   __half* x16 = nullptr;
   float* xscale = nullptr;
   float* h32 = nullptr;
@@ -70,8 +83,16 @@ struct moe_fp4 {
   uint8_t* gu_frag = nullptr;     // gate/up fragment layout, all experts
   uint8_t* dn_frag = nullptr;     // down fragment layout, all experts
   float* gs = nullptr;            // [3][E]: gate, up, down
+  uint8_t* dq_gate = nullptr;     // dense class: canonical codes with signs folded [E*f][d/2]
+  uint8_t* dq_up = nullptr;
+  uint8_t* dq_down = nullptr;     // [E*d][f/2]
+  uint8_t* dsf_gu = nullptr;      // scale atoms [E][f/64][d/64][512]
+  uint8_t* dsf_dn = nullptr;      // scale atoms [E][d/128][f/64][512]
+  CUtensorMap tm_gate{}, tm_up{}, tm_down{};
+  bool dense_ok = false;          // d, f multiples of 256 and tensor maps available
+  bool dense_h32 = false;         // write fp32 h of the dense class (debug copies)
   int* err = nullptr;             // device error word
-  cudaEvent_t stage_ev[7] = {};   // optional stage-timing events (caller-owned)
+  cudaEvent_t stage_ev[kStageEvents] = {};   // optional stage-timing events (caller-owned)
   bool stage_timing = false;
   Workspace ws;
 };
@@ -99,6 +120,45 @@ size_t counter_ints(const moe_fp4* h, int Tm) {
   return (size_t)h->E + ((size_t)h->E + (size_t)Tm * h->k / moe::kJobRows + 1) + h->d / 16 + 3;
 }
 
+// rows of the dense-class operand buffers: every pair plus up to 127 padding
+// rows per dense expert, in whole 128-row tiles
+size_t dense_pad_rows(const moe_fp4* h, int Tm) {
+  const size_t P = (size_t)Tm * h->k;
+  return (P + 128 * std::min<size_t>(h->E, P) + 127) / 128 * 128;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    else
+      (void)cudaGetLastError();
+  }
+  return fn;
+}
+
+// 2-D byte tensor [rows][row_bytes], 128-byte rows boxes with 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {row_bytes, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 size_t workspace_bytes(const moe_fp4* h, int Tm) {
   const size_t P = (size_t)Tm * h->k;
   size_t b = 0;
@@ -115,6 +175,13 @@ size_t workspace_bytes(const moe_fp4* h, int Tm) {
   add(((size_t)h->E + P / moe::kJobRows + 1) * 16);   // light jobs, 9..16 rows
   add(4);
   add(counter_ints(h, Tm) * 4);                        // counters
+  add(((size_t)h->E + 1) * 4);                         // dense n-tile prefix
+  add(4);                                              // dense padded rows
+  const size_t pr = dense_pad_rows(h, Tm);
+  add(pr * h->d / 2);                                  // xq
+  add(pr / 128 * (h->d / 64) * 512);                   // xsf
+  add(pr * h->f / 2);                                  // hq
+  add(pr / 128 * (h->f / 64) * 512);                   // hsf
   add((size_t)h->E * 16);           // dense list
   add(4);
   add((size_t)Tm * h->d * 2);       // x16
@@ -168,6 +235,15 @@ int ensure_workspace(moe_fp4* h, int Tm, cudaStream_t stream) {
   w.partial = carve<float>(cur, P * h->d);
   w.xin = carve<uint16_t>(cur, (size_t)Tm * h->d);
   w.xout = carve<uint16_t>(cur, (size_t)Tm * h->d);
+  w.dense_ntoff = carve<int>(cur, h->E + 1);
+  w.dense_pad_total = carve<int>(cur, 1);
+  w.pad_rows = dense_pad_rows(h, Tm);
+  w.xq = carve<uint8_t>(cur, w.pad_rows * h->d / 2);
+  w.xsf = carve<uint8_t>(cur, w.pad_rows / 128 * (h->d / 64) * 512);
+  w.hq = carve<uint8_t>(cur, w.pad_rows * h->f / 2);
+  w.hsf = carve<uint8_t>(cur, w.pad_rows / 128 * (h->f / 64) * 512);
+  if (!make_map(&w.tm_x, w.xq, h->d / 2, w.pad_rows, 128) || !make_map(&w.tm_h, w.hq, h->f / 2, w.pad_rows, 128))
+    h->dense_ok = false;
   if (cudaMemset(w.counters, 0, w.counter_bytes) != cudaSuccess) {
     (void)cudaGetLastError();
     cudaFree(base);
@@ -228,11 +304,17 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
   int* exit2 = exit1 + 1;
   int* ticket = exit2 + 1;
   moe::PermuteOut po{w.counts, w.offsets, w.perm, w.inv, w.jobs1, w.n_jobs1, w.jobs2, w.n_jobs2,
-                     w.dense_list, w.n_dense, h->err};
+                     w.dense_list, w.n_dense, w.dense_ntoff, w.dense_pad_total, h->err};
+  // Without the dense class (shape or tensor-map support missing) every
+  // expert runs in the light class.  An expert holds at most T rows (one per
+  // token), so below T = thr no expert can be dense and its kernels are skipped.
+  const int dense_ok = h->dense_ok ? 1 : 0;
+  const int thr = h->dense_ok ? h->thr : INT_MAX;
+  const bool run_dense = h->dense_ok && T >= h->thr;
   if (T <= kSmallT) {
     // 1-3. router logits, x staging, top-k and permutation in one launch
     MOE_CUDA(launch(moe::route_kernel, dim3(E), dim3(1024), route_smem_bytes(E, d, T * k), st, false,
-                    xb, rw, T, d, E, k, h->thr, 0, w.logits, w.x16, w.xscale, w.ids, w.wts, ticket, po));
+                    xb, rw, T, d, E, k, thr, dense_ok, w.logits, w.x16, w.xscale, w.ids, w.wts, ticket, po));
     MOE_CUDA(mark(h, 1, st));
     MOE_CUDA(mark(h, 2, st));
   } else {
@@ -245,9 +327,60 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
                     (const float*)w.logits, T, E, k, w.ids, w.wts));
     MOE_CUDA(mark(h, 2, st));
     MOE_CUDA(launch(moe::permute_kernel, dim3(1), dim3(1024), permute_smem_bytes(E), st, false,
-                    (const int*)w.ids, T, k, E, h->thr, 0, po));
+                    (const int*)w.ids, T, k, E, thr, dense_ok, po));
   }
   MOE_CUDA(mark(h, 3, st));
+  // 4-5 (dense class). NVFP4 activations, then the two tensor-core GEMMs
+  if (run_dense) {
+    MOE_CUDA(launch(moe::quant_x_dense_kernel, dim3(8 * h->sm_count), dim3(256), 0, st, pdl,
+                    xb, (const int4*)w.dense_list, (const int*)w.n_dense, (const int*)w.dense_pad_total,
+                    (const int*)w.perm, k, d, w.xq, w.xsf));
+    MOE_CUDA(mark(h, 4, st));
+    moe::DenseParams dp{};
+    dp.tmA0 = h->tm_gate;
+    dp.tmA1 = h->tm_up;
+    dp.tmB = w.tm_x;
+    dp.sfA = h->dsf_gu;
+    dp.sfB = w.xsf;
+    dp.dense = w.dense_list;
+    dp.n_dense = w.n_dense;
+    dp.ntoff = w.dense_ntoff;
+    dp.mt_per_expert = f / 64;
+    dp.rows_per_expert = f;
+    dp.kstages = d / 256;
+    dp.kb64 = d / 64;
+    dp.d = d;
+    dp.f = f;
+    dp.topk = k;
+    dp.gs = h->gs;
+    dp.E = E;
+    dp.perm = w.perm;
+    dp.wts = w.wts;
+    dp.hq = w.hq;
+    dp.hsf = w.hsf;
+    dp.h32 = h->dense_h32 ? w.h32 : nullptr;
+    dp.partial = w.partial;
+    dp.err = h->err;
+    dp.wait_timeout_ns = h->wait_timeout_ns;
+    MOE_CUDA(launch(moe::dense_gemm_kernel<moe::kDenseGateUp>, dim3(h->sm_count * kDenseGridPerSm),
+                    dim3(moe::kDenseThreads), moe::dense_smem_size<moe::kDenseGateUp>(E), st, pdl, dp));
+    MOE_CUDA(mark(h, 5, st));
+    moe::DenseParams dp2 = dp;
+    dp2.tmA0 = h->tm_down;
+    dp2.tmB = w.tm_h;
+    dp2.sfA = h->dsf_dn;
+    dp2.sfB = w.hsf;
+    dp2.mt_per_expert = d / 128;
+    dp2.rows_per_expert = d;
+    dp2.kstages = f / 256;
+    dp2.kb64 = f / 64;
+    MOE_CUDA(launch(moe::dense_gemm_kernel<moe::kDenseDown>, dim3(h->sm_count * kDenseGridPerSm),
+                    dim3(moe::kDenseThreads), moe::dense_smem_size<moe::kDenseDown>(E), st, pdl, dp2));
+  } else {
+    MOE_CUDA(mark(h, 4, st));
+    MOE_CUDA(mark(h, 5, st));
+  }
+  MOE_CUDA(mark(h, 6, st));
   // 4-6. light experts: gate/up + SwiGLU, down x routing weight, combine
   moe::ExpertParams ep{};
   ep.gu_frag = h->gu_frag;
@@ -282,12 +415,11 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
                   kExpSmem, st, pdl, ep1));
   MOE_CUDA(launch(moe::expert_kernel<2>, dim3(h->sm_count * h->exp_bps2), dim3(moe::kExpThreads),
                   kExpSmem, st, pdl, ep2));
-  MOE_CUDA(mark(h, 4, st));
-  MOE_CUDA(mark(h, 5, st));
+  MOE_CUDA(mark(h, 7, st));
   // 7. combine / unpermute: out[t] = bf16(sum_j partial[inv[t,j]])
   MOE_CUDA(launch(moe::combine_kernel, dim3((d + 1023) / 1024, T), dim3(128), 0, st, pdl,
                   (const float*)w.partial, (const int*)w.inv, T, k, d, static_cast<uint16_t*>(out)));
-  MOE_CUDA(mark(h, 6, st));
+  MOE_CUDA(mark(h, 8, st));
   return MOE_FP4_OK;
 }
 
@@ -355,7 +487,11 @@ int moe_fp4_create(int E, int top_k, int d, int f, moe_fp4_t** out) {
     if (smem_attr((const void*)moe::expert_kernel<1>, kExpSmem) != cudaSuccess ||
         smem_attr((const void*)moe::expert_kernel<2>, kExpSmem) != cudaSuccess ||
         smem_attr((const void*)moe::permute_kernel, permute_smem_bytes(E)) != cudaSuccess ||
-        smem_attr((const void*)moe::route_kernel, route_smem_bytes(E, d, kSmallT * top_k)) != cudaSuccess) {
+        smem_attr((const void*)moe::route_kernel, route_smem_bytes(E, d, kSmallT * top_k)) != cudaSuccess ||
+        smem_attr((const void*)moe::dense_gemm_kernel<moe::kDenseGateUp>,
+                  moe::dense_smem_size<moe::kDenseGateUp>(E)) != cudaSuccess ||
+        smem_attr((const void*)moe::dense_gemm_kernel<moe::kDenseDown>,
+                  moe::dense_smem_size<moe::kDenseDown>(E)) != cudaSuccess) {
       rc = MOE_FP4_ERR_CUDA; break;
     }
     int nb1 = 0, nb2 = 0;
@@ -386,6 +522,11 @@ void moe_fp4_destroy(moe_fp4_t* h) {
   cudaFree(h->gu_frag);
   cudaFree(h->dn_frag);
   cudaFree(h->gs);
+  cudaFree(h->dq_gate);
+  cudaFree(h->dq_up);
+  cudaFree(h->dq_down);
+  cudaFree(h->dsf_gu);
+  cudaFree(h->dsf_dn);
   cudaFree(h->err);
   cudaFree(h->ws.base);
   (void)cudaGetLastError();
@@ -422,6 +563,34 @@ int moe_fp4_load_experts(moe_fp4_t* h, const moe_fp4_experts* w) {
                                                             E, d, f, h->dn_frag);
     MOE_CUDA(cudaGetLastError());
   }
+  // dense class: codes with block-scale signs folded, scale atoms, tensor maps
+  {
+    const size_t gu_codes = (size_t)E * f * d / 2, dn_codes = (size_t)E * d * f / 2;
+    const size_t gu_atoms = (size_t)E * (f / 64) * (d / 64) * 512;
+    const size_t dn_atoms = (size_t)E * (d / 128) * (f / 64) * 512;
+    auto alloc = [](uint8_t** p, size_t n) {
+      if (*p) return true;
+      if (cudaMalloc(p, n) != cudaSuccess) { (void)cudaGetLastError(); *p = nullptr; return false; }
+      return true;
+    };
+    if (!alloc(&h->dq_gate, gu_codes) || !alloc(&h->dq_up, gu_codes) || !alloc(&h->dq_down, dn_codes) ||
+        !alloc(&h->dsf_gu, gu_atoms) || !alloc(&h->dsf_dn, dn_atoms))
+      return MOE_FP4_ERR_OOM;
+    const int blocks = h->sm_count * 8;
+    moe::dense_codes_kernel<<<blocks, 256>>>(w->gate_q, w->gate_sf, (long long)E * f, d, h->dq_gate);
+    moe::dense_codes_kernel<<<blocks, 256>>>(w->up_q, w->up_sf, (long long)E * f, d, h->dq_up);
+    moe::dense_codes_kernel<<<blocks, 256>>>(w->down_q, w->down_sf, (long long)E * d, f, h->dq_down);
+    moe::dense_sf_atoms_kernel<moe::kGateUp><<<blocks, 256>>>(w->gate_sf, w->up_sf, E, f, d, h->dsf_gu);
+    moe::dense_sf_atoms_kernel<moe::kDown><<<blocks, 256>>>(w->down_sf, nullptr, E, d, f, h->dsf_dn);
+    MOE_CUDA(cudaGetLastError());
+    h->dense_ok = (d % 256 == 0) && (f % 256 == 0) &&
+                  make_map(&h->tm_gate, h->dq_gate, d / 2, (uint64_t)E * f, 64) &&
+                  make_map(&h->tm_up, h->dq_up, d / 2, (uint64_t)E * f, 64) &&
+                  make_map(&h->tm_down, h->dq_down, f / 2, (uint64_t)E * d, 128);
+    if (h->ws.base && (!make_map(&h->ws.tm_x, h->ws.xq, d / 2, h->ws.pad_rows, 128) ||
+                       !make_map(&h->ws.tm_h, h->ws.hq, f / 2, h->ws.pad_rows, 128)))
+      h->dense_ok = false;
+  }
   MOE_CUDA(cudaMemcpy(h->gs, w->gate_gs, sizeof(float) * E, cudaMemcpyDeviceToDevice));
   MOE_CUDA(cudaMemcpy(h->gs + E, w->up_gs, sizeof(float) * E, cudaMemcpyDeviceToDevice));
   MOE_CUDA(cudaMemcpy(h->gs + 2 * E, w->down_gs, sizeof(float) * E, cudaMemcpyDeviceToDevice));
@@ -453,7 +622,9 @@ int moe_fp4_forward(moe_fp4_t* h, const void* x, int T, const float* rw, void* o
 
 int moe_fp4_forward_ex(moe_fp4_t* h, const void* x, int T, const float* rw, void* out,
                        cudaStream_t stream, moe_fp4_debug* dbg) {
+  if (h) h->dense_h32 = dbg && dbg->h;
   int rc = moe_fp4_forward(h, x, T, rw, out, stream);
+  if (h) h->dense_h32 = false;
   if (rc != MOE_FP4_OK || T == 0 || !dbg) return rc;
   const Workspace& w = h->ws;
   const size_t P = (size_t)T * h->k;
@@ -493,8 +664,8 @@ int moe_fp4_forward_host(moe_fp4_t* h, const void* x_host, int T, const float* r
 int moe_fp4_set_stage_events(moe_fp4_t* h, cudaEvent_t* events, int n) {
   if (!h) return MOE_FP4_ERR_INVALID_ARG;
   if (n == 0) { h->stage_timing = false; return MOE_FP4_OK; }
-  if (n != 7 || !events) return MOE_FP4_ERR_INVALID_ARG;
-  for (int i = 0; i < 7; ++i) {
+  if (n != kStageEvents || !events) return MOE_FP4_ERR_INVALID_ARG;
+  for (int i = 0; i < kStageEvents; ++i) {
     if (!events[i]) return MOE_FP4_ERR_INVALID_ARG;
     h->stage_ev[i] = events[i];
   }

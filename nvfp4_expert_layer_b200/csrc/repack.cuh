@@ -69,4 +69,60 @@ __global__ void repack_fragment_kernel(const uint8_t* __restrict__ qa, const uin
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Dense-class weight copies for the tensor cores.  The block-scaled MMA reads
+// unsigned e4m3 scales, so a negative block scale is folded into the codes:
+// the 16 codes of that block change sign and the scale's sign bit is cleared
+// (exact).  One thread per (row, 16-value block).
+// q: [rows][K/2] canonical codes, sf: [rows][K/16]; writes qd (same layout).
+// ---------------------------------------------------------------------------
+__global__ void dense_codes_kernel(const uint8_t* __restrict__ q, const uint8_t* __restrict__ sf,
+                                   long long rows, int K, uint8_t* __restrict__ qd) {
+  const int nb = K / 16;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < rows * nb;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long r = i / nb;
+    const int blk = (int)(i - r * nb);
+    uint2 v = *reinterpret_cast<const uint2*>(q + r * (K / 2) + blk * 8);
+    if (sf[i] & 0x80u) { v.x ^= 0x88888888u; v.y ^= 0x88888888u; }
+    *reinterpret_cast<uint2*>(qd + r * (K / 2) + blk * 8) = v;
+  }
+}
+
+// Scale atoms of the dense weights, one thread per atom byte.
+// MODE kGateUp: M tile mt of expert e = gate rows 64mt..64mt+63 (atom rows
+// 0..63) and up rows 64mt..64mt+63 (atom rows 64..127); K = d.
+// MODE kDown: M tile mt = down rows 128mt..128mt+127; K = f.
+// Atom (e, mt, kb64) holds byte (r % 32) * 16 + (r / 32) * 4 + kb4 = scale of
+// atom row r for K block 4 * kb64 + kb4, sign bit cleared.
+template <int MODE>
+__global__ void dense_sf_atoms_kernel(const uint8_t* __restrict__ sfa, const uint8_t* __restrict__ sfb,
+                                      int E, int rows, int K, uint8_t* __restrict__ out) {
+  const int kb64n = K / 64;
+  const int mtpe = (MODE == kGateUp) ? rows / 64 : rows / 128;
+  const long long total = (long long)E * mtpe * kb64n * 512;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int byte = (int)(i & 511);
+    const long long atom = i >> 9;
+    const int kb64 = (int)(atom % kb64n);
+    const long long em = atom / kb64n;
+    const int mt = (int)(em % mtpe);
+    const int e = (int)(em / mtpe);
+    const int r0 = byte >> 4, r1 = (byte >> 2) & 3, kb4 = byte & 3;
+    const int r = r1 * 32 + r0;
+    const uint8_t* src;
+    long long row;
+    if (MODE == kGateUp) {
+      src = r < 64 ? sfa : sfb;
+      row = (long long)e * rows + mt * 64 + (r & 63);
+    } else {
+      src = sfa;
+      row = (long long)e * rows + mt * 128 + r;
+    }
+    out[i] = src[row * (K / 16) + kb64 * 4 + kb4] & 0x7Fu;
+  }
+}
+
 }  // namespace moe

@@ -218,8 +218,10 @@ struct PermuteOut {
   int* n_jobs1;
   int4* jobs2;       // [E + P/16 + 1] {expert, row0, nrows, 0}, 9 <= nrows <= 16
   int* n_jobs2;
-  int4* dense_list;  // [E]            {expert, row0, nrows, 0}
+  int4* dense_list;  // [E]            {expert, row0, nrows, padded row0}
   int* n_dense;
+  int* dense_ntoff;  // [E+1]          exclusive prefix of ceil(nrows / 128) over the dense list
+  int* dense_pad_total;  // padded rows of the dense class (each expert rounded up to 128)
   int* err;
 };
 
@@ -305,7 +307,7 @@ __device__ void build_permutation(const int* ids, int T, int k, int E, int thr, 
     const int e = act[a];
     const int n = cnt[e];
     const bool light = n < thr;
-    int rank = 0, s1 = 0, s2 = 0;
+    int rank = 0, s1 = 0, s2 = 0, pad0 = 0, nt0 = 0;
     for (int b = 0; b < A; ++b) {
       const int e2 = act[b], n2 = cnt[e2];
       if ((n2 < thr) != light) continue;
@@ -314,6 +316,8 @@ __device__ void build_permutation(const int* ids, int T, int k, int E, int thr, 
         const int r2 = n2 % kJobRows;
         s1 += (r2 > 0 && r2 <= 8) ? 1 : 0;
         s2 += n2 / kJobRows + (r2 > 8 ? 1 : 0);
+        pad0 += (n2 + 127) & ~127;
+        nt0 += (n2 + 127) >> 7;
       }
     }
     if (light) {
@@ -326,8 +330,11 @@ __device__ void build_permutation(const int* ids, int T, int k, int E, int thr, 
       atomicAdd(&misc[1], (r > 0 && r <= 8) ? 1 : 0);
       atomicAdd(&misc[2], n / kJobRows + (r > 8 ? 1 : 0));
     } else {
-      o.dense_list[rank] = make_int4(e, off[e], n, 0);
+      o.dense_list[rank] = make_int4(e, off[e], n, pad0);
+      o.dense_ntoff[rank] = nt0;
       atomicAdd(&misc[3], 1);
+      atomicAdd(&misc[4], (n + 127) >> 7);
+      atomicAdd(&misc[5], (n + 127) & ~127);
     }
   }
   __syncthreads();
@@ -335,6 +342,8 @@ __device__ void build_permutation(const int* ids, int T, int k, int E, int thr, 
     *o.n_jobs1 = misc[1];
     *o.n_jobs2 = misc[2];
     *o.n_dense = misc[3];
+    o.dense_ntoff[misc[3]] = misc[4];
+    *o.dense_pad_total = misc[5];
     if (misc[3] > 0 && !dense_supported) set_error(o.err, kErrUnsupported);
   }
 }

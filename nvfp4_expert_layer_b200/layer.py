@@ -50,10 +50,10 @@ class MoeFp4Layer:
     def set_dense_threshold(self, thr: int) -> None:
         _lib.check(self.lib.moe_fp4_set_dense_threshold(self._h, thr), "moe_fp4_set_dense_threshold")
 
-    STAGES = ("router", "topk", "permute", "gate_up", "down", "combine")
+    STAGES = ("router", "topk", "permute", "dense_quant", "dense_gate_up", "dense_down", "light", "combine")
 
     def set_stage_events(self, events) -> None:
-        """events: list of 7 torch.cuda.Event(enable_timing=True), or None to turn off."""
+        """events: list of len(STAGES) + 1 torch.cuda.Event(enable_timing=True), or None to turn off."""
         if events is None:
             _lib.check(self.lib.moe_fp4_set_stage_events(self._h, None, 0), "moe_fp4_set_stage_events")
             self._stage_events = None
@@ -61,8 +61,11 @@ class MoeFp4Layer:
         for e in events:            # torch creates the CUDA event at its first record
             if not e.cuda_event:
                 e.record()
-        arr = (ctypes.c_void_p * 7)(*[ctypes.c_void_p(e.cuda_event) for e in events])
-        _lib.check(self.lib.moe_fp4_set_stage_events(self._h, arr, 7), "moe_fp4_set_stage_events")
+        n = len(self.STAGES) + 1
+        if len(events) != n:
+            raise ValueError(f"set_stage_events needs {n} events")
+        arr = (ctypes.c_void_p * n)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+        _lib.check(self.lib.moe_fp4_set_stage_events(self._h, arr, n), "moe_fp4_set_stage_events")
         self._stage_events = (events, arr)
 
     def device_error(self) -> int:

@@ -1,0 +1,100 @@
+"""GPU parity of the dense expert class (tcgen05 block-scaled NVFP4 GEMMs).
+
+Experts that receive at least `thr` rows quantise x and h to NVFP4 and run on
+the FP4 tensor cores; the oracle applies the same activation quantiser
+(reading R4) and the parity helpers bound the effect of quantiser decisions
+that may round the other way when h moves inside its accumulation bound."""
+import numpy as np
+import pytest
+import torch
+
+from nvfp4_expert_layer_b200 import workloads as W
+from nvfp4_expert_layer_b200.layer import MoeFp4Layer, experts_to_device
+from tests.parity import Case, bf16_to_bits, to_dev_x
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(cfg, thr, **kw):
+    c = Case(cfg, thr=thr, **kw).run_gpu().run_oracle()
+    c.check_all()
+    return c
+
+
+def test_dense_tiny_every_expert_dense():
+    # thr = 1: every active expert is dense; each holds <= 4 rows of a 128-row tile
+    c = _run(W.CONFIGS["tiny"], thr=1)
+    assert c.n_dense_rows == c.cfg.T * c.cfg.k
+
+
+def test_dense_ragged_multi_tile_experts():
+    # ~175 rows per expert: two 128-token tiles, the second ragged
+    cfg = W.custom_config(T=700, d=512, E=8, k=2, f=512, seed=51, router="unit")
+    c = _run(cfg, thr=64)
+    counts = c.o["counts"]
+    assert np.any((counts > 128) & (counts % 128 != 0))
+    assert c.n_dense_rows > 0
+
+
+def test_dense_and_light_classes_in_one_call():
+    cfg = W.custom_config(T=600, d=1024, E=16, k=4, f=768, seed=52, router="unit")
+    c = Case(cfg, thr=150).run_gpu().run_oracle()
+    counts = c.o["counts"]
+    assert np.any(counts >= 150) and np.any((counts > 0) & (counts < 150)), counts
+    c.check_all()
+    assert 0 < c.n_dense_rows < cfg.T * cfg.k
+
+
+def test_dense_threshold_is_inclusive():
+    cfg = W.custom_config(T=300, d=512, E=8, k=2, f=256, seed=53, router="unit")
+    x, rw = W.gen_x_router(cfg)
+    ex = W.gen_experts(cfg)
+    probe = Case(cfg, thr=1 << 30, experts=ex, x=x, rw=rw).run_oracle()
+    counts = np.sort(probe.o["counts"][probe.o["counts"] > 0])
+    thr = int(counts[len(counts) // 2])          # one expert sits exactly at thr
+    c = _run(cfg, thr=thr, experts=ex, x=x, rw=rw)
+    assert np.any(c.o["counts"] == thr)
+    # compared rows of experts at or above thr are exactly the dense rows
+    ro = c._rows()[:, 1]
+    e_of = np.searchsorted(c.o["offsets"], ro, side="right") - 1
+    assert c.n_dense_rows == int(np.sum(c.o["counts"][e_of] >= thr)) > 0
+
+
+def test_dense_unsupported_shape_runs_light():
+    # d = 384 is not a multiple of 256: every expert stays in the light class
+    cfg = W.custom_config(T=40, d=384, E=4, k=2, f=256, seed=54, router="unit")
+    c = _run(cfg, thr=1)
+    assert c.n_dense_rows == 0
+
+
+def test_dense_deterministic_and_graph_replay():
+    cfg = W.custom_config(T=400, d=512, E=8, k=2, f=256, seed=55, router="unit")
+    x, rw = W.gen_x_router(cfg)
+    layer = MoeFp4Layer(cfg.E, cfg.k, cfg.d, cfg.f)
+    layer.load_experts(experts_to_device(W.gen_experts(cfg)))
+    layer.set_dense_threshold(32)
+    layer.reserve(cfg.T)
+    xd, rwd = to_dev_x(x), torch.from_numpy(rw).cuda()
+    a = bf16_to_bits(layer(xd, rwd))
+    b = bf16_to_bits(layer(xd, rwd))
+    assert np.array_equal(a, b)
+    out = torch.empty_like(xd)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            layer(xd, rwd, out=out, stream=s)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    assert layer.device_error() == 0
+    assert np.array_equal(bf16_to_bits(out), a)
+
+
+def test_prefill_full_size_sampled_tokens():
+    # 8 x 2048 tokens, d = 7168, E = 256, k = 8, f = 2048: every expert dense
+    cfg = W.CONFIGS["prefill"]
+    c = Case(cfg, token_subset=[0, 8191, 16383]).run_gpu().run_oracle()
+    assert np.all(c.o["counts"] >= 128)
+    c.check_all()
+    assert c.n_dense_rows == len(c._rows()) > 0
