@@ -54,7 +54,21 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="decode1")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shape", default="",
+                    help="profiling sizes over the workload's recipe, e.g. T=4096,E=32 "
+                         "(the JSON line then names the changed sizes)")
     return ap.parse_args()
+
+
+def workload_config(args):
+    from nvfp4_expert_layer_b200 import workloads as W
+    cfg = W.CONFIGS[args.workload]
+    if args.shape:
+        kw = {k: int(v) for k, v in (item.split("=") for item in args.shape.split(","))}
+        cfg = W.LayerConfig(f"{cfg.name}[{args.shape}]", kw.get("T", cfg.T), kw.get("d", cfg.d),
+                            kw.get("E", cfg.E), kw.get("k", cfg.k), kw.get("f", cfg.f), cfg.seed,
+                            cfg.router, cfg.requests)
+    return cfg
 
 
 def expert_bytes(cfg) -> int:
@@ -259,7 +273,7 @@ def run_native(args, rank, world, local):
     from nvfp4_expert_layer_b200 import workloads as W
     from nvfp4_expert_layer_b200.layer import MoeFp4Layer, experts_to_device
     torch.cuda.set_device(local)
-    cfg = W.CONFIGS[args.workload]
+    cfg = workload_config(args)
     ex = W.gen_experts(cfg)
     layer = MoeFp4Layer(cfg.E, cfg.k, cfg.d, cfg.f)
     dev = experts_to_device(ex)
@@ -419,7 +433,7 @@ def main():
     args = parse()
     rank, world, local = dist_setup(args)
     from nvfp4_expert_layer_b200 import workloads as W
-    cfg = W.CONFIGS[args.workload]
+    cfg = workload_config(args)
     if args.impl == "reference":
         # the reference arm is the oracle (plain fp64 CPU code) on bounded
         # slices of the same workload; rank 0 only

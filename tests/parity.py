@@ -77,9 +77,8 @@ def quant_deviation(h, hb):
     i_lo = np.searchsorted(grid, s_lo)
     i_hi = np.searchsorted(grid, s_hi)
     assert np.all(grid[i_lo] == s_lo) and np.all(grid[i_hi] == s_hi)
-    assert np.all(i_hi - i_lo <= 3), "h bound too wide for a useful quantiser bound"
     dev = np.zeros_like(h)
-    for j in range(4):
+    for j in range(int((i_hi - i_lo).max()) + 1):
         sf = grid[np.minimum(i_lo + j, i_hi)]
         sfe = np.repeat(sf, 16, axis=-1)
         sf32 = sfe.astype(np.float32)
