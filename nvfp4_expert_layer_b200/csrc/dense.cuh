@@ -11,9 +11,12 @@
 // both decided in IEEE fp32.  Rows of every dense expert are padded to a
 // multiple of 128 so each 128-token MMA tile starts on a scale-atom boundary.
 //
-// GEMM 1 (kDenseGateUp): D[128 rows = 64 gate + 64 up rows of W][128 tokens]
-//   over K = d; the epilogue forms h = SiLU(g) * u, quantises it along f and
-//   writes the B operand of GEMM 2.
+// GEMM 1 (kDenseGateUp): D[128 rows of the combined gate/up matrix][128 tokens]
+//   over K = d.  Gate and up rows are interleaved in groups of 16 channels, so
+//   each 32-lane TMEM quarter holds gate (lanes 0-15) and up (lanes 16-31) of
+//   the same 16 channels -- one NVFP4 block of h.  The epilogue exchanges the
+//   halves with one shuffle, forms h = SiLU(g) * u, quantises each 16-channel
+//   block with warp shuffles and writes the B operand of GEMM 2.
 // GEMM 2 (kDenseDown):   D[128 rows of Wd][128 tokens] over K = f; the
 //   epilogue writes w * gs * D as fp32 partials (rows in permutation order).
 #pragma once
@@ -37,8 +40,7 @@ enum DenseMode { kDenseGateUp = 0, kDenseDown = 1 };
 
 // Dense list entry: {expert, row0 (permutation rows), rows, padded row0}.
 struct DenseParams {
-  CUtensorMap tmA0;      // gate/up: gate copy, box 128 B x 64 rows; down: down copy, box 128 B x 128 rows
-  CUtensorMap tmA1;      // gate/up: up copy, box 128 B x 64 rows
+  CUtensorMap tmA;       // weights: combined gate/up rows [E][2f] or down rows [E][d]; box 128 B x 128 rows
   CUtensorMap tmB;       // activations (NVFP4, padded permutation order), box 128 B x 128 rows
   const uint8_t* sfA;    // weight scale atoms
   const uint8_t* sfB;    // activation scale atoms
@@ -46,7 +48,7 @@ struct DenseParams {
   const int* n_dense;
   const int* ntoff;      // [E+1] exclusive prefix of ceil(rows / 128) over the dense list
   int mt_per_expert;     // gate/up: f / 64; down: d / 128
-  int rows_per_expert;   // gate/up: f; down: d (rows of the weight copy per expert)
+  int rows_per_expert;   // gate/up: 2f; down: d (rows of the weight copy per expert)
   int kstages;           // K / 256
   int kb64;              // K / 64
   int d, f, topk;
@@ -174,7 +176,6 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
   int* svote = reinterpret_cast<int*>(meta + kDenseBarBytes + 16);    // [4] epilogue wait outcomes
   int4* sd = reinterpret_cast<int4*>(meta + kDenseBarBytes + 32);     // dense list (<= E entries)
   int* sntoff = reinterpret_cast<int*>(sd + p.E);                     // [E+1]
-  float* ubuf = reinterpret_cast<float*>(sntoff + ((p.E + 4) & ~3));  // gate/up: [2][32][129]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_wait();
@@ -215,8 +216,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint64_t pol_w = policy_evict_first(), pol_a = policy_evict_last();
-      tma_prefetch_desc(&p.tmA0);
-      if (MODE == kDenseGateUp) tma_prefetch_desc(&p.tmA1);
+      tma_prefetch_desc(&p.tmA);
       tma_prefetch_desc(&p.tmB);
       int k = 0;
       for (int it = 0; it < my_tiles && !failed; ++it) {
@@ -230,13 +230,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
           }
           const uint32_t st = stage0 + s * kDenseStageBytes;
           mbar_arrive_expect_tx(full_b(s), kDenseStageBytes);
-          if (MODE == kDenseGateUp) {
-            const int wrow = e * p.rows_per_expert + tl.mt * 64;
-            tma_load_2d(st, &p.tmA0, ks * 128, wrow, full_b(s), pol_w);
-            tma_load_2d(st + kDenseTileBytes / 2, &p.tmA1, ks * 128, wrow, full_b(s), pol_w);
-          } else {
-            tma_load_2d(st, &p.tmA0, ks * 128, e * p.rows_per_expert + tl.mt * 128, full_b(s), pol_w);
-          }
+          tma_load_2d(st, &p.tmA, ks * 128, e * p.rows_per_expert + tl.mt * 128, full_b(s), pol_w);
           tma_load_2d(st + kDenseTileBytes, &p.tmB, ks * 128, brow, full_b(s), pol_a);
           const uint8_t* sfa = p.sfA + ((size_t)(e * p.mt_per_expert + tl.mt) * p.kb64 + 4 * ks) * 512;
           const uint8_t* sfb = p.sfB + ((size_t)(brow >> 7) * p.kb64 + 4 * ks) * 512;
@@ -319,67 +313,62 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
       if (MODE == kDenseDown) {
         const float gsd = p.gs[2 * p.E + e];
         const int drow = tl.mt * 128 + q * 32 + lane;
-        for (int c0 = 0; c0 < 128; c0 += 32) {
+        for (int c0 = 0; c0 < ncols; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(acc + c0, r);
+          // routing weight x tensor scale of column c0 + lane, broadcast below
+          const float wl = c0 + lane < ncols ? p.wts[p.perm[prow0 + c0 + lane]] * gsd : 0.f;
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float wv = __shfl_sync(0xffffffffu, wl, c);
+            if (c0 + c < ncols) p.partial[(size_t)(prow0 + c0 + c) * p.d + drow] = __uint_as_float(r[c]) * wv;
+          }
+        }
+      } else {
+        // lanes 0-15: gate rows, lanes 16-31: up rows of channels ch0 .. ch0 + 15
+        const bool upper = lane >= 16;
+        const float gsg = p.gs[e], gsu = p.gs[p.E + e];
+        const int ch0 = tl.mt * 64 + q * 16;
+        const int ch = ch0 + (lane & 15);
+        for (int c0 = 0; c0 < ncols; c0 += 32) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(acc + c0, r);
           tmem_ld_wait();
-#pragma unroll 4
-          for (int c = 0; c < 32; ++c) {
-            const int n = c0 + c;
-            if (n < ncols) {
-              const float wv = p.wts[p.perm[prow0 + n]] * gsd;
-              p.partial[(size_t)(prow0 + n) * p.d + drow] = __uint_as_float(r[c]) * wv;
-            }
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(acce_b(ab));
-      } else {
-        // quarters 2, 3 hold up rows; 0, 1 gate rows of the same 64 channels
-        float* ub = ubuf + (size_t)((q & 1) * 32 + lane) * 129;
-        if (q >= 2) {
-          for (int c0 = 0; c0 < 128; c0 += 32) {
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(acc + c0, r);
-            tmem_ld_wait();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) ub[c0 + c] = __uint_as_float(r[c]);
-          }
-        }
-        named_bar_sync(1, 128);                           // up values staged
-        if (q < 2) {
-          const float gsg = p.gs[e], gsu = p.gs[p.E + e];
-          const int fidx = tl.mt * 64 + q * 32 + lane;
-          for (int c0 = 0; c0 < 128; c0 += 32) {
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(acc + c0, r);
-            tmem_ld_wait();
-            for (int c = 0; c < 32; ++c) {
-              const int n = c0 + c;
-              if (n >= ncols) break;                      // warp-uniform
-              const float gv = __uint_as_float(r[c]) * gsg;
-              const float uv = ub[n] * gsu;
-              const float hv = gv / (1.f + expf(-gv)) * uv;
-              if (p.h32) p.h32[(size_t)(prow0 + n) * p.f + fidx] = hv;
-              // NVFP4 along f: 16 lanes form one block
-              float am = fabsf(hv);
+          for (int j = 0; j < 16; ++j) {
+            // lower lanes take column c0 + j, upper lanes column c0 + 16 + j
+            const float send = __uint_as_float(upper ? r[j] : r[16 + j]);
+            const float other = __shfl_xor_sync(0xffffffffu, send, 16);
+            const float gv = (upper ? other : __uint_as_float(r[j])) * gsg;
+            const float uv = (upper ? __uint_as_float(r[16 + j]) : other) * gsu;
+            const float hv = gv / (1.f + expf(-gv)) * uv;
+            const int n = c0 + j + (upper ? 16 : 0);
+            if (p.h32 && n < ncols) p.h32[(size_t)(prow0 + n) * p.f + ch] = hv;
+            // NVFP4 block of 16 channels = one half-warp
+            float am = fabsf(hv);
 #pragma unroll
-              for (int o = 8; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-              const uint32_t sfbyte = f32x2_to_e4m3x2(0.f, am / 6.0f) & 0xffu;
-              const float sf = e4m3_to_f32(sfbyte);
-              const uint32_t code = sf > 0.f ? (f32x2_to_e2m1x2(0.f, hv / sf) & 0xfu) : 0u;
-              const uint32_t hi = __shfl_down_sync(0xffffffffu, code, 1);
+            for (int o = 8; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+            const uint32_t sfbyte = f32x2_to_e4m3x2(0.f, am / 6.0f) & 0xffu;
+            const float sf = e4m3_to_f32(sfbyte);
+            const uint32_t code = sf > 0.f ? (f32x2_to_e2m1x2(0.f, hv / sf) & 0xfu) : 0u;
+            // channel c of the block -> nibble c % 8 of word c / 8 (element 2i in the low nibble)
+            uint32_t word = code << (4 * (lane & 7));
+            word |= __shfl_xor_sync(0xffffffffu, word, 1);
+            word |= __shfl_xor_sync(0xffffffffu, word, 2);
+            word |= __shfl_xor_sync(0xffffffffu, word, 4);
+            const uint32_t word_hi = __shfl_down_sync(0xffffffffu, word, 8);
+            if ((lane & 15) == 0) {
               const int hr = hrow0 + n;
-              if ((lane & 1) == 0) p.hq[(size_t)hr * (p.f / 2) + (fidx >> 1)] = (uint8_t)(code | (hi << 4));
-              if ((lane & 15) == 0) p.hsf[sf_atom_offset(hr, fidx >> 4, p.f / 64)] = (uint8_t)sfbyte;
+              *reinterpret_cast<uint2*>(p.hq + (size_t)hr * (p.f / 2) + (ch0 >> 1)) = make_uint2(word, word_hi);
+              p.hsf[sf_atom_offset(hr, ch0 >> 4, p.f / 64)] = (uint8_t)sfbyte;
             }
           }
         }
-        tc_fence_before();
-        named_bar_sync(1, 128);                           // up values consumed
-        if (lane == 0) mbar_arrive(acce_b(ab));
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce_b(ab));
     }
   }
   tc_fence_before();
@@ -394,7 +383,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
 template <int MODE>
 constexpr size_t dense_smem_size(int E) {
   return 1024 + (size_t)kDenseStages * kDenseStageBytes + kDenseBarBytes + 32 + (size_t)E * 16 +
-         (size_t)((E + 4) & ~3) * 4 + (MODE == kDenseGateUp ? 2 * 32 * 129 * 4 : 0);
+         (size_t)(E + 1) * 4;
 }
 
 }  // namespace moe

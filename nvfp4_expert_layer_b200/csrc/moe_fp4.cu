@@ -83,12 +83,11 @@ struct moe_fp4 {
   uint8_t* gu_frag = nullptr;     // gate/up fragment layout, all experts
   uint8_t* dn_frag = nullptr;     // down fragment layout, all experts
   float* gs = nullptr;            // [3][E]: gate, up, down
-  uint8_t* dq_gate = nullptr;     // dense class: canonical codes with signs folded [E*f][d/2]
-  uint8_t* dq_up = nullptr;
+  uint8_t* dq_gu = nullptr;       // dense class: gate/up codes, rows interleaved by 16, signs folded [E*2f][d/2]
   uint8_t* dq_down = nullptr;     // [E*d][f/2]
   uint8_t* dsf_gu = nullptr;      // scale atoms [E][f/64][d/64][512]
   uint8_t* dsf_dn = nullptr;      // scale atoms [E][d/128][f/64][512]
-  CUtensorMap tm_gate{}, tm_up{}, tm_down{};
+  CUtensorMap tm_gu{}, tm_down{};
   bool dense_ok = false;          // d, f multiples of 256 and tensor maps available
   bool dense_h32 = false;         // write fp32 h of the dense class (debug copies)
   int* err = nullptr;             // device error word
@@ -337,8 +336,7 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
                     (const int*)w.perm, k, d, w.xq, w.xsf));
     MOE_CUDA(mark(h, 4, st));
     moe::DenseParams dp{};
-    dp.tmA0 = h->tm_gate;
-    dp.tmA1 = h->tm_up;
+    dp.tmA = h->tm_gu;
     dp.tmB = w.tm_x;
     dp.sfA = h->dsf_gu;
     dp.sfB = w.xsf;
@@ -346,7 +344,7 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
     dp.n_dense = w.n_dense;
     dp.ntoff = w.dense_ntoff;
     dp.mt_per_expert = f / 64;
-    dp.rows_per_expert = f;
+    dp.rows_per_expert = 2 * f;
     dp.kstages = d / 256;
     dp.kb64 = d / 64;
     dp.d = d;
@@ -366,7 +364,7 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
                     dim3(moe::kDenseThreads), moe::dense_smem_size<moe::kDenseGateUp>(E), st, pdl, dp));
     MOE_CUDA(mark(h, 5, st));
     moe::DenseParams dp2 = dp;
-    dp2.tmA0 = h->tm_down;
+    dp2.tmA = h->tm_down;
     dp2.tmB = w.tm_h;
     dp2.sfA = h->dsf_dn;
     dp2.sfB = w.hsf;
@@ -522,8 +520,7 @@ void moe_fp4_destroy(moe_fp4_t* h) {
   cudaFree(h->gu_frag);
   cudaFree(h->dn_frag);
   cudaFree(h->gs);
-  cudaFree(h->dq_gate);
-  cudaFree(h->dq_up);
+  cudaFree(h->dq_gu);
   cudaFree(h->dq_down);
   cudaFree(h->dsf_gu);
   cudaFree(h->dsf_dn);
@@ -573,19 +570,17 @@ int moe_fp4_load_experts(moe_fp4_t* h, const moe_fp4_experts* w) {
       if (cudaMalloc(p, n) != cudaSuccess) { (void)cudaGetLastError(); *p = nullptr; return false; }
       return true;
     };
-    if (!alloc(&h->dq_gate, gu_codes) || !alloc(&h->dq_up, gu_codes) || !alloc(&h->dq_down, dn_codes) ||
+    if (!alloc(&h->dq_gu, 2 * gu_codes) || !alloc(&h->dq_down, dn_codes) ||
         !alloc(&h->dsf_gu, gu_atoms) || !alloc(&h->dsf_dn, dn_atoms))
       return MOE_FP4_ERR_OOM;
     const int blocks = h->sm_count * 8;
-    moe::dense_codes_kernel<<<blocks, 256>>>(w->gate_q, w->gate_sf, (long long)E * f, d, h->dq_gate);
-    moe::dense_codes_kernel<<<blocks, 256>>>(w->up_q, w->up_sf, (long long)E * f, d, h->dq_up);
+    moe::dense_gu_codes_kernel<<<blocks, 256>>>(w->gate_q, w->gate_sf, w->up_q, w->up_sf, E, f, d, h->dq_gu);
     moe::dense_codes_kernel<<<blocks, 256>>>(w->down_q, w->down_sf, (long long)E * d, f, h->dq_down);
     moe::dense_sf_atoms_kernel<moe::kGateUp><<<blocks, 256>>>(w->gate_sf, w->up_sf, E, f, d, h->dsf_gu);
     moe::dense_sf_atoms_kernel<moe::kDown><<<blocks, 256>>>(w->down_sf, nullptr, E, d, f, h->dsf_dn);
     MOE_CUDA(cudaGetLastError());
     h->dense_ok = (d % 256 == 0) && (f % 256 == 0) &&
-                  make_map(&h->tm_gate, h->dq_gate, d / 2, (uint64_t)E * f, 64) &&
-                  make_map(&h->tm_up, h->dq_up, d / 2, (uint64_t)E * f, 64) &&
+                  make_map(&h->tm_gu, h->dq_gu, d / 2, (uint64_t)E * 2 * f, 128) &&
                   make_map(&h->tm_down, h->dq_down, f / 2, (uint64_t)E * d, 128);
     if (h->ws.base && (!make_map(&h->ws.tm_x, h->ws.xq, d / 2, h->ws.pad_rows, 128) ||
                        !make_map(&h->ws.tm_h, h->ws.hq, f / 2, h->ws.pad_rows, 128)))

@@ -90,9 +90,38 @@ __global__ void dense_codes_kernel(const uint8_t* __restrict__ q, const uint8_t*
   }
 }
 
+// Gate/up rows of the dense class are interleaved in groups of 32 so that one
+// 32-lane TMEM quarter of a 128-row accumulator tile holds the gate rows
+// (lanes 0-15) and the up rows (lanes 16-31) of the same 16 FFN channels:
+// combined row rr of an expert (0 <= rr < 2f) is gate (rr & 16 == 0) or up
+// row 16 * (rr / 32) + rr % 16.
+__host__ __device__ __forceinline__ int gu_channel(int rr) { return 16 * (rr >> 5) + (rr & 15); }
+__host__ __device__ __forceinline__ bool gu_is_up(int rr) { return (rr & 16) != 0; }
+
+// Combined gate/up codes [E][2f][d/2] in the interleaved row order, signs of
+// negative block scales folded into the codes.  One thread per (row, block).
+__global__ void dense_gu_codes_kernel(const uint8_t* __restrict__ gq, const uint8_t* __restrict__ gsf,
+                                      const uint8_t* __restrict__ uq, const uint8_t* __restrict__ usf,
+                                      int E, int f, int d, uint8_t* __restrict__ qd) {
+  const int nb = d / 16;
+  const long long rows = (long long)E * 2 * f;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < rows * nb;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long R = i / nb;
+    const int blk = (int)(i - R * nb);
+    const int e = (int)(R / (2 * f)), rr = (int)(R % (2 * f));
+    const long long src = (long long)e * f + gu_channel(rr);
+    const uint8_t* q = gu_is_up(rr) ? uq : gq;
+    const uint8_t* sf = gu_is_up(rr) ? usf : gsf;
+    uint2 v = *reinterpret_cast<const uint2*>(q + src * (d / 2) + blk * 8);
+    if (sf[src * nb + blk] & 0x80u) { v.x ^= 0x88888888u; v.y ^= 0x88888888u; }
+    *reinterpret_cast<uint2*>(qd + R * (d / 2) + blk * 8) = v;
+  }
+}
+
 // Scale atoms of the dense weights, one thread per atom byte.
-// MODE kGateUp: M tile mt of expert e = gate rows 64mt..64mt+63 (atom rows
-// 0..63) and up rows 64mt..64mt+63 (atom rows 64..127); K = d.
+// MODE kGateUp: M tile mt of expert e = combined (interleaved) gate/up rows
+// 128mt..128mt+127, i.e. FFN channels 64mt..64mt+63; K = d.
 // MODE kDown: M tile mt = down rows 128mt..128mt+127; K = f.
 // Atom (e, mt, kb64) holds byte (r % 32) * 16 + (r / 32) * 4 + kb4 = scale of
 // atom row r for K block 4 * kb64 + kb4, sign bit cleared.
@@ -115,8 +144,9 @@ __global__ void dense_sf_atoms_kernel(const uint8_t* __restrict__ sfa, const uin
     const uint8_t* src;
     long long row;
     if (MODE == kGateUp) {
-      src = r < 64 ? sfa : sfb;
-      row = (long long)e * rows + mt * 64 + (r & 63);
+      const int rr = mt * 128 + r;
+      src = gu_is_up(rr) ? sfb : sfa;
+      row = (long long)e * rows + gu_channel(rr);
     } else {
       src = sfa;
       row = (long long)e * rows + mt * 128 + r;
