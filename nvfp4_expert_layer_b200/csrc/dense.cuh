@@ -157,14 +157,6 @@ __device__ __forceinline__ DenseTile dense_tile(const int4* sd, const int* sntof
   return t;
 }
 
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
-}
-
-__device__ __forceinline__ void named_bar_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(n) : "memory");
-}
-
 template <int MODE>
 __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __grid_constant__ DenseParams p) {
   extern __shared__ __align__(1024) uint8_t dsm_raw[];
@@ -215,7 +207,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first(), pol_a = policy_evict_last();
+      const uint64_t pol_w = policy_evict_normal(), pol_a = policy_evict_last();
       tma_prefetch_desc(&p.tmA);
       tma_prefetch_desc(&p.tmB);
       int k = 0;
@@ -225,7 +217,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
         const int brow = tl.de.w + tl.nt * 128;              // padded activation row
         for (int ks = 0; ks < p.kstages; ++ks, ++k) {
           const int s = k % kDenseStages;
-          if (!mbar_wait_until(empty_b(s), ((k / kDenseStages) & 1) ^ 1, deadline)) {
+          if (!mbar_wait_spin(empty_b(s), ((k / kDenseStages) & 1) ^ 1, deadline)) {
             failed = true; set_error(p.err, kErrTimeout); break;
           }
           const uint32_t st = stage0 + s * kDenseStageBytes;
@@ -240,7 +232,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
       }
       // drain: every issued stage must land before the block exits
       for (int kk = max(0, k - kDenseStages); kk < k; ++kk)
-        mbar_wait_until(full_b(kk % kDenseStages), (kk / kDenseStages) & 1,
+        mbar_wait_spin(full_b(kk % kDenseStages), (kk / kDenseStages) & 1,
                         globaltimer_ns() + (uint64_t)p.wait_timeout_ns);
     }
   } else if (warp == 1) {
@@ -251,14 +243,14 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
       bool issued_any = false;
       for (int it = 0; it < my_tiles && !failed; ++it) {
         const int ab = it & 1;
-        if (!mbar_wait_until(acce_b(ab), ((it >> 1) & 1) ^ 1, deadline)) {
+        if (!mbar_wait_spin(acce_b(ab), ((it >> 1) & 1) ^ 1, deadline)) {
           failed = true; set_error(p.err, kErrTimeout); break;
         }
         tc_fence_after();
         const uint32_t acc = acc_t0 + ab * 128;
         for (int ks = 0; ks < p.kstages; ++ks, ++k) {
           const int s = k % kDenseStages;
-          if (!mbar_wait_until(full_b(s), (k / kDenseStages) & 1, deadline)) {
+          if (!mbar_wait_spin(full_b(s), (k / kDenseStages) & 1, deadline)) {
             failed = true; set_error(p.err, kErrTimeout); break;
           }
           tc_fence_after();
@@ -283,7 +275,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
       // every MMA issued must complete before TMEM is released
       if (issued_any) {
         tc_commit(done_b);
-        mbar_wait_until(done_b, 0, globaltimer_ns() + (uint64_t)p.wait_timeout_ns);
+        mbar_wait_spin(done_b, 0, globaltimer_ns() + (uint64_t)p.wait_timeout_ns);
       }
     }
   } else {
@@ -295,7 +287,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
       const DenseTile tl = dense_tile(sd, sntoff, nd, p.mt_per_expert, b + it * G);
       // all epilogue warps take the same decision: each records whether its
       // bounded wait succeeded, then they meet at a barrier every warp reaches
-      const bool ok = mbar_wait_until(accf_b(ab), (it >> 1) & 1, deadline);
+      const bool ok = mbar_wait_spin(accf_b(ab), (it >> 1) & 1, deadline);
       if (lane == 0) svote[q] = ok ? 1 : 0;
       named_bar_sync(2, 128);
       const bool all_ok = svote[0] && svote[1] && svote[2] && svote[3];

@@ -26,6 +26,7 @@
 #include "experts.cuh"
 #include "combine.cuh"
 #include "dense.cuh"
+#include "router_tc.cuh"
 
 namespace {
 
@@ -61,6 +62,9 @@ struct Workspace {
   uint8_t* hsf = nullptr;
   size_t pad_rows = 0;
   CUtensorMap tm_x{}, tm_h{};    // B operands of the dense GEMMs
+  __nv_bfloat16* rw3 = nullptr;  // router weights split into three exact bf16 parts [3][E][d]
+  CUtensorMap tm_rw3{};
+  bool tc_router = false;        // tensor-core router available (tensor maps encoded)
   __half* x16 = nullptr;
   float* xscale = nullptr;
   float* h32 = nullptr;
@@ -145,17 +149,24 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D byte tensor [rows][row_bytes], 128-byte rows boxes with 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows, uint32_t box_rows) {
+// 2-D row-major tensor [rows][row_bytes]; boxes of 128 bytes x box_rows with
+// the 128-byte swizzle the tcgen05 K-major shared-memory descriptors expect.
+// Rows past `rows` read as zeros.
+bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint32_t elem_bytes,
+                 uint64_t row_bytes, uint64_t rows, uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  const cuuint64_t dims[2] = {row_bytes, rows};
+  const cuuint64_t dims[2] = {row_bytes / elem_bytes, rows};
   const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t box[2] = {128 / elem_bytes, box_rows};
   const cuuint32_t es[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows, uint32_t box_rows) {
+  return make_map_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, row_bytes, rows, box_rows);
 }
 
 size_t workspace_bytes(const moe_fp4* h, int Tm) {
@@ -163,6 +174,7 @@ size_t workspace_bytes(const moe_fp4* h, int Tm) {
   size_t b = 0;
   auto add = [&](size_t n) { b += align_up(n, 256); };
   add((size_t)Tm * h->E * 4);       // logits
+  add((size_t)3 * h->E * h->d * 2); // router weights, three bf16 parts
   add(P * 4);                       // ids
   add(P * 4);                       // wts
   add((size_t)h->E * 4);            // counts
@@ -213,6 +225,9 @@ int ensure_workspace(moe_fp4* h, int Tm, cudaStream_t stream) {
   const size_t P = (size_t)Tm * h->k;
   uint8_t* cur = static_cast<uint8_t*>(base);
   w.logits = carve<float>(cur, (size_t)Tm * h->E);
+  w.rw3 = carve<__nv_bfloat16>(cur, (size_t)3 * h->E * h->d);
+  w.tc_router = make_map_2d(&w.tm_rw3, w.rw3, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)h->d * 2,
+                            (uint64_t)3 * h->E, 128);
   w.ids = carve<int>(cur, P);
   w.wts = carve<float>(cur, P);
   w.counts = carve<int>(cur, h->E);
@@ -317,8 +332,26 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
     MOE_CUDA(mark(h, 1, st));
     MOE_CUDA(mark(h, 2, st));
   } else {
-    MOE_CUDA(launch(moe::router_tiled_kernel, dim3((T + 63) / 64, (E + 63) / 64), dim3(256), 0, st,
-                    false, xb, rw, T, d, E, w.logits));
+    // 1. router logits: fp32 weights split into three exact bf16 parts, then
+    // the tensor-core GEMM (x bf16 exact products, fp32 accumulation)
+    moe::RouterParams rp{};
+    const bool tc = w.tc_router && make_map_2d(&rp.tmX, xb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                                               (uint64_t)d * 2, (uint64_t)T, 128);
+    if (tc) {
+      MOE_CUDA(launch(moe::router_split_kernel, dim3(4 * h->sm_count), dim3(256), 0, st, false,
+                      rw, (long long)E * d, w.rw3));
+      rp.tmW = w.tm_rw3;
+      rp.T = T; rp.d = d; rp.E = E;
+      rp.logits = w.logits;
+      rp.err = h->err;
+      rp.wait_timeout_ns = h->wait_timeout_ns;
+      const int tiles = ((E + 127) / 128) * ((T + 127) / 128);
+      MOE_CUDA(launch(moe::router_tc_kernel, dim3(std::min(tiles, h->sm_count)), dim3(moe::kRtThreads),
+                      moe::router_tc_smem_size(), st, pdl, rp));
+    } else {
+      MOE_CUDA(launch(moe::router_tiled_kernel, dim3((T + 63) / 64, (E + 63) / 64), dim3(256), 0, st,
+                      false, xb, rw, T, d, E, w.logits));
+    }
     MOE_CUDA(launch(moe::stage_x_kernel, dim3(std::min(T, 8 * h->sm_count)), dim3(256), 0, st, false,
                     xb, T, d, w.x16, w.xscale, h->err));
     MOE_CUDA(mark(h, 1, st));
@@ -489,7 +522,8 @@ int moe_fp4_create(int E, int top_k, int d, int f, moe_fp4_t** out) {
         smem_attr((const void*)moe::dense_gemm_kernel<moe::kDenseGateUp>,
                   moe::dense_smem_size<moe::kDenseGateUp>(E)) != cudaSuccess ||
         smem_attr((const void*)moe::dense_gemm_kernel<moe::kDenseDown>,
-                  moe::dense_smem_size<moe::kDenseDown>(E)) != cudaSuccess) {
+                  moe::dense_smem_size<moe::kDenseDown>(E)) != cudaSuccess ||
+        smem_attr((const void*)moe::router_tc_kernel, moe::router_tc_smem_size()) != cudaSuccess) {
       rc = MOE_FP4_ERR_CUDA; break;
     }
     int nb1 = 0, nb2 = 0;

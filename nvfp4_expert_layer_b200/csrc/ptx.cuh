@@ -73,6 +73,16 @@ __device__ __forceinline__ bool mbar_wait_until(uint32_t bar, uint32_t phase, ui
   return true;
 }
 
+// Bounded wait for latency-critical pipeline hand-offs (TMA -> MMA -> TMA):
+// plain try_wait polls, no suspend-time hint, so the waiter resumes as soon
+// as the phase completes; the global timer is read every 64 polls.
+__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t phase, uint64_t deadline_ns) {
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, phase)) return true;
+    if ((i & 63u) == 0 && globaltimer_ns() > deadline_ns) return false;
+  }
+}
+
 // ---------------------------------------------------------------- bulk copy
 // Untiled TMA bulk copy global -> shared, completion signalled on `bar`.
 // src, dst 16-byte aligned; bytes a multiple of 16.
@@ -87,6 +97,12 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ uint64_t policy_evict_normal() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
 

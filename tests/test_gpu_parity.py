@@ -131,3 +131,12 @@ def test_graph_capture_after_reserve():
         g.replay()
     torch.cuda.synchronize()
     assert np.array_equal(bf16_to_bits(out), ref)
+
+
+@pytest.mark.parametrize("T,E,k,d", [(257, 130, 3, 384), (300, 1, 1, 256), (1000, 256, 8, 1024)])
+def test_tensor_core_router_shapes(T, E, k, d):
+    # T > 256 routes through the tensor-core router (fp32 weights split into
+    # three exact bf16 parts): ragged token tiles, expert counts that are not
+    # a multiple of 128, a single expert
+    cfg = W.custom_config(T=T, d=d, E=E, k=k, f=128, seed=60 + E, router="unit")
+    Case(cfg).run_gpu().run_oracle().check_all()
