@@ -14,9 +14,10 @@
 // GEMM 1 (kDenseGateUp): D[128 rows of the combined gate/up matrix][128 tokens]
 //   over K = d.  Gate and up rows are interleaved in groups of 16 channels, so
 //   each 32-lane TMEM quarter holds gate (lanes 0-15) and up (lanes 16-31) of
-//   the same 16 channels -- one NVFP4 block of h.  The epilogue exchanges the
-//   halves with one shuffle, forms h = SiLU(g) * u, quantises each 16-channel
-//   block with warp shuffles and writes the B operand of GEMM 2.
+//   the same 16 channels -- one NVFP4 block of h.  The epilogue transposes
+//   each 32 x 32 chunk through shared memory so that one lane holds the 16
+//   gate and 16 up values of one token, forms h = SiLU(g) * u, quantises the
+//   block in registers and writes the B operand of GEMM 2.
 // GEMM 2 (kDenseDown):   D[128 rows of Wd][128 tokens] over K = f; the
 //   epilogue writes w * gs * D as fp32 partials (rows in permutation order).
 #pragma once
@@ -34,6 +35,7 @@ constexpr int kDenseTileBytes = 128 * 128; // 128 rows x 128 bytes (256 fp4 alon
 constexpr int kDenseSfBytes = 4 * 512;     // 4 scale atoms (K = 256) per operand per stage
 constexpr int kDenseStageBytes = 2 * kDenseTileBytes + 2 * kDenseSfBytes;
 constexpr uint32_t kDenseTmemCols = 512;
+static_assert(256 + 32 * kDenseStages <= kDenseTmemCols, "accumulators + per-stage scale factors exceed TMEM");
 constexpr int kDenseBarBytes = (2 * kDenseStages + 6) * 8;   // mbarriers, padded to 16 bytes
 
 enum DenseMode { kDenseGateUp = 0, kDenseDown = 1 };
@@ -168,6 +170,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
   int* svote = reinterpret_cast<int*>(meta + kDenseBarBytes + 16);    // [4] epilogue wait outcomes
   int4* sd = reinterpret_cast<int4*>(meta + kDenseBarBytes + 32);     // dense list (<= E entries)
   int* sntoff = reinterpret_cast<int*>(sd + p.E);                     // [E+1]
+  float* tbuf = reinterpret_cast<float*>(sntoff + ((p.E + 4) & ~3));  // gate/up: [4 warps][32][33]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_wait();
@@ -195,7 +198,9 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t acc_t0 = tmem, sfa_t = tmem + 256, sfb_t = tmem + 272;
+  // TMEM columns: accumulators 0-255 (two buffers of 128), then one set of
+  // scale factors per shared-memory stage (16 columns for A, 16 for B).
+  const uint32_t acc_t0 = tmem, sf_t0 = tmem + 256;
 
   const int ntiles = p.mt_per_expert * sntoff[nd];
   const int G = gridDim.x, b = blockIdx.x;
@@ -256,6 +261,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
           tc_fence_after();
           const uint32_t st = stage0 + s * kDenseStageBytes;
           const uint32_t sfa_s = st + 2 * kDenseTileBytes, sfb_s = sfa_s + kDenseSfBytes;
+          const uint32_t sfa_t = sf_t0 + 32 * s, sfb_t = sfa_t + 16;
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb) {
             tc_cp_32x128b_x4(sfa_t + 4 * kb, smem_desc_sf(sfa_s + 512 * kb));
@@ -318,44 +324,49 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
           }
         }
       } else {
-        // lanes 0-15: gate rows, lanes 16-31: up rows of channels ch0 .. ch0 + 15
-        const bool upper = lane >= 16;
+        // Lanes 0-15 hold the gate rows and lanes 16-31 the up rows of channels
+        // ch0 .. ch0 + 15.  Each 32-column chunk is transposed through shared
+        // memory so that lane L owns token column c0 + L: its 16 h values, their
+        // NVFP4 block scale and 8 bytes of codes then need no cross-lane traffic.
         const float gsg = p.gs[e], gsu = p.gs[p.E + e];
         const int ch0 = tl.mt * 64 + q * 16;
-        const int ch = ch0 + (lane & 15);
+        float* tb = tbuf + q * (32 * 33);
         for (int c0 = 0; c0 < ncols; c0 += 32) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(acc + c0, r);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            // lower lanes take column c0 + j, upper lanes column c0 + 16 + j
-            const float send = __uint_as_float(upper ? r[j] : r[16 + j]);
-            const float other = __shfl_xor_sync(0xffffffffu, send, 16);
-            const float gv = (upper ? other : __uint_as_float(r[j])) * gsg;
-            const float uv = (upper ? __uint_as_float(r[16 + j]) : other) * gsu;
-            const float hv = gv / (1.f + expf(-gv)) * uv;
-            const int n = c0 + j + (upper ? 16 : 0);
-            if (p.h32 && n < ncols) p.h32[(size_t)(prow0 + n) * p.f + ch] = hv;
-            // NVFP4 block of 16 channels = one half-warp
-            float am = fabsf(hv);
+          for (int c = 0; c < 32; ++c) tb[lane * 33 + c] = __uint_as_float(r[c]);
+          __syncwarp();
+          float hv[16];
+          float am = 0.f;
 #pragma unroll
-            for (int o = 8; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-            const uint32_t sfbyte = f32x2_to_e4m3x2(0.f, am / 6.0f) & 0xffu;
-            const float sf = e4m3_to_f32(sfbyte);
-            const uint32_t code = sf > 0.f ? (f32x2_to_e2m1x2(0.f, hv / sf) & 0xfu) : 0u;
-            // channel c of the block -> nibble c % 8 of word c / 8 (element 2i in the low nibble)
-            uint32_t word = code << (4 * (lane & 7));
-            word |= __shfl_xor_sync(0xffffffffu, word, 1);
-            word |= __shfl_xor_sync(0xffffffffu, word, 2);
-            word |= __shfl_xor_sync(0xffffffffu, word, 4);
-            const uint32_t word_hi = __shfl_down_sync(0xffffffffu, word, 8);
-            if ((lane & 15) == 0) {
-              const int hr = hrow0 + n;
-              *reinterpret_cast<uint2*>(p.hq + (size_t)hr * (p.f / 2) + (ch0 >> 1)) = make_uint2(word, word_hi);
-              p.hsf[sf_atom_offset(hr, ch0 >> 4, p.f / 64)] = (uint8_t)sfbyte;
+          for (int i = 0; i < 16; ++i) {
+            const float gv = tb[i * 33 + lane] * gsg;
+            const float uv = tb[(16 + i) * 33 + lane] * gsu;
+            hv[i] = gv / (1.f + expf(-gv)) * uv;
+            am = fmaxf(am, fabsf(hv[i]));
+          }
+          __syncwarp();                                   // tb is rewritten by the next chunk
+          const int n = c0 + lane;                        // < 128: inside the expert's padded rows
+          if (p.h32 && n < ncols) {
+            float4* dst = reinterpret_cast<float4*>(p.h32 + (size_t)(prow0 + n) * p.f + ch0);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_float4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
+          }
+          const uint32_t sfbyte = f32x2_to_e4m3x2(0.f, am / 6.0f) & 0xffu;
+          const float sf = e4m3_to_f32(sfbyte);
+          uint32_t w0 = 0u, w1 = 0u;                      // channel i -> nibble i % 8 of word i / 8
+          if (sf > 0.f) {
+#pragma unroll
+            for (int i = 0; i < 8; i += 2) {
+              w0 |= f32x2_to_e2m1x2(hv[i + 1] / sf, hv[i] / sf) << (4 * i);
+              w1 |= f32x2_to_e2m1x2(hv[i + 9] / sf, hv[i + 8] / sf) << (4 * i);
             }
           }
+          const int hr = hrow0 + n;
+          *reinterpret_cast<uint2*>(p.hq + (size_t)hr * (p.f / 2) + (ch0 >> 1)) = make_uint2(w0, w1);
+          p.hsf[sf_atom_offset(hr, ch0 >> 4, p.f / 64)] = (uint8_t)sfbyte;
         }
       }
       tc_fence_before();
@@ -375,7 +386,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
 template <int MODE>
 constexpr size_t dense_smem_size(int E) {
   return 1024 + (size_t)kDenseStages * kDenseStageBytes + kDenseBarBytes + 32 + (size_t)E * 16 +
-         (size_t)(E + 1) * 4;
+         (size_t)((E + 4) & ~3) * 4 + (MODE == kDenseGateUp ? 4 * 32 * 33 * 4 : 0);
 }
 
 }  // namespace moe
