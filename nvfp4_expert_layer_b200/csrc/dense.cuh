@@ -29,10 +29,11 @@
 
 namespace moe {
 
-constexpr int kDenseThreads = 192;        // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
-constexpr int kDenseStages = 4;
+constexpr int kDenseEpiWarps = 8;         // two per TMEM lane quarter, each on half of the columns
+constexpr int kDenseThreads = 64 + 32 * kDenseEpiWarps;   // warp 0 TMA, warp 1 MMA, warps 2.. epilogue
+constexpr int kDenseStages = 3;
 constexpr int kDenseTileBytes = 128 * 128; // 128 rows x 128 bytes (256 fp4 along K)
-constexpr int kDenseSfBytes = 4 * 512;     // 4 scale atoms (K = 256) per operand per stage
+constexpr int kDenseSfBytes = 2 * 4096;    // per operand per stage: 2 scale pair units (K = 256)
 constexpr int kDenseStageBytes = 2 * kDenseTileBytes + 2 * kDenseSfBytes;
 constexpr uint32_t kDenseTmemCols = 512;
 static_assert(256 + 32 * kDenseStages <= kDenseTmemCols, "accumulators + per-stage scale factors exceed TMEM");
@@ -125,7 +126,9 @@ __global__ void __launch_bounds__(256) quant_x_dense_kernel(
         }
       }
       *reinterpret_cast<uint2*>(xq + (size_t)prow * (d / 2) + blk * 8) = codes;
-      xsf[sf_atom_offset(prow, blk, d / 64)] = (uint8_t)sfbyte;
+      const size_t so = sf_pair_offset(prow, blk, d / 64);
+#pragma unroll
+      for (int c = 0; c < kSfReplicas; ++c) xsf[so + 1024 * c] = (uint8_t)sfbyte;
     }
   }
   pdl_launch_dependents();
@@ -167,10 +170,10 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
   uint8_t* meta = dsm + kDenseStages * kDenseStageBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(meta);                 // full[S] empty[S] accf[2] acce[2] done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(meta + kDenseBarBytes);
-  int* svote = reinterpret_cast<int*>(meta + kDenseBarBytes + 16);    // [4] epilogue wait outcomes
-  int4* sd = reinterpret_cast<int4*>(meta + kDenseBarBytes + 32);     // dense list (<= E entries)
+  int* svote = reinterpret_cast<int*>(meta + kDenseBarBytes + 16);    // [8] epilogue wait outcomes
+  int4* sd = reinterpret_cast<int4*>(meta + kDenseBarBytes + 48);     // dense list (<= E entries)
   int* sntoff = reinterpret_cast<int*>(sd + p.E);                     // [E+1]
-  float* tbuf = reinterpret_cast<float*>(sntoff + ((p.E + 4) & ~3));  // gate/up: [4 warps][32][33]
+  float* tbuf = reinterpret_cast<float*>(sntoff + ((p.E + 4) & ~3));  // gate/up: [epilogue warps][32][33]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_wait();
@@ -186,7 +189,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
   const uint32_t done_b = bars_s + 8 * (2 * kDenseStages + 4);
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDenseStages; ++s) { mbar_init(full_b(s), 1); mbar_init(empty_b(s), 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(accf_b(a), 1); mbar_init(acce_b(a), 4); }
+    for (int a = 0; a < 2; ++a) { mbar_init(accf_b(a), 1); mbar_init(acce_b(a), kDenseEpiWarps); }
     mbar_init(done_b, 1);
     fence_mbar_init();
   }
@@ -229,8 +232,9 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
           mbar_arrive_expect_tx(full_b(s), kDenseStageBytes);
           tma_load_2d(st, &p.tmA, ks * 128, e * p.rows_per_expert + tl.mt * 128, full_b(s), pol_w);
           tma_load_2d(st + kDenseTileBytes, &p.tmB, ks * 128, brow, full_b(s), pol_a);
-          const uint8_t* sfa = p.sfA + ((size_t)(e * p.mt_per_expert + tl.mt) * p.kb64 + 4 * ks) * 512;
-          const uint8_t* sfb = p.sfB + ((size_t)(brow >> 7) * p.kb64 + 4 * ks) * 512;
+          // scales: the two 4 KB pair units of this K stage (see sf_pair_offset)
+          const uint8_t* sfa = p.sfA + ((size_t)(e * p.mt_per_expert + tl.mt) * (p.kb64 >> 1) + 2 * ks) * 4096;
+          const uint8_t* sfb = p.sfB + ((size_t)(brow >> 7) * (p.kb64 >> 1) + 2 * ks) * 4096;
           bulk_g2s(st + 2 * kDenseTileBytes, sfa, kDenseSfBytes, full_b(s), pol_w);
           bulk_g2s(st + 2 * kDenseTileBytes + kDenseSfBytes, sfb, kDenseSfBytes, full_b(s), pol_a);
         }
@@ -263,9 +267,9 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
           const uint32_t sfa_s = st + 2 * kDenseTileBytes, sfb_s = sfa_s + kDenseSfBytes;
           const uint32_t sfa_t = sf_t0 + 32 * s, sfb_t = sfa_t + 16;
 #pragma unroll
-          for (int kb = 0; kb < 4; ++kb) {
-            tc_cp_32x128b_x4(sfa_t + 4 * kb, smem_desc_sf(sfa_s + 512 * kb));
-            tc_cp_32x128b_x4(sfb_t + 4 * kb, smem_desc_sf(sfb_s + 512 * kb));
+          for (int pr = 0; pr < 2; ++pr) {                // one copy per pair of MMAs and operand
+            tc_cp_128x256b(sfa_t + 8 * pr, smem_desc_sf256(sfa_s + 4096 * pr));
+            tc_cp_128x256b(sfb_t + 8 * pr, smem_desc_sf256(sfb_s + 4096 * pr));
           }
           const uint64_t adesc = smem_desc_sw128(st), bdesc = smem_desc_sw128(st + kDenseTileBytes);
 #pragma unroll
@@ -285,8 +289,10 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2..5)
+    // ------------------------------------------------------------ epilogue (warps 2..)
     const int q = warp & 3;                              // TMEM lane quarter of this warp
+    const int ew = warp - 2;                             // epilogue warp index
+    const int chalf = (ew >> 2) * 32;                    // first 32-column chunk of this warp
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     for (int it = 0; it < my_tiles && !failed; ++it) {
       const int ab = it & 1;
@@ -294,10 +300,12 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
       // all epilogue warps take the same decision: each records whether its
       // bounded wait succeeded, then they meet at a barrier every warp reaches
       const bool ok = mbar_wait_spin(accf_b(ab), (it >> 1) & 1, deadline);
-      if (lane == 0) svote[q] = ok ? 1 : 0;
-      named_bar_sync(2, 128);
-      const bool all_ok = svote[0] && svote[1] && svote[2] && svote[3];
-      named_bar_sync(2, 128);
+      if (lane == 0) svote[ew] = ok ? 1 : 0;
+      named_bar_sync(2, 32 * kDenseEpiWarps);
+      bool all_ok = true;
+#pragma unroll
+      for (int i = 0; i < kDenseEpiWarps; ++i) all_ok = all_ok && svote[i];
+      named_bar_sync(2, 32 * kDenseEpiWarps);
       if (!all_ok) {
         failed = true;
         if (lane == 0) set_error(p.err, kErrTimeout);
@@ -311,7 +319,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
       if (MODE == kDenseDown) {
         const float gsd = p.gs[2 * p.E + e];
         const int drow = tl.mt * 128 + q * 32 + lane;
-        for (int c0 = 0; c0 < ncols; c0 += 32) {
+        for (int c0 = chalf; c0 < ncols; c0 += 64) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(acc + c0, r);
           // routing weight x tensor scale of column c0 + lane, broadcast below
@@ -330,8 +338,8 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
         // NVFP4 block scale and 8 bytes of codes then need no cross-lane traffic.
         const float gsg = p.gs[e], gsu = p.gs[p.E + e];
         const int ch0 = tl.mt * 64 + q * 16;
-        float* tb = tbuf + q * (32 * 33);
-        for (int c0 = 0; c0 < ncols; c0 += 32) {
+        float* tb = tbuf + ew * (32 * 33);
+        for (int c0 = chalf; c0 < ncols; c0 += 64) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(acc + c0, r);
           tmem_ld_wait();
@@ -366,7 +374,9 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
           }
           const int hr = hrow0 + n;
           *reinterpret_cast<uint2*>(p.hq + (size_t)hr * (p.f / 2) + (ch0 >> 1)) = make_uint2(w0, w1);
-          p.hsf[sf_atom_offset(hr, ch0 >> 4, p.f / 64)] = (uint8_t)sfbyte;
+          const size_t so = sf_pair_offset(hr, ch0 >> 4, p.f / 64);
+#pragma unroll
+          for (int c = 0; c < kSfReplicas; ++c) p.hsf[so + 1024 * c] = (uint8_t)sfbyte;
         }
       }
       tc_fence_before();
@@ -385,8 +395,8 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
 
 template <int MODE>
 constexpr size_t dense_smem_size(int E) {
-  return 1024 + (size_t)kDenseStages * kDenseStageBytes + kDenseBarBytes + 32 + (size_t)E * 16 +
-         (size_t)((E + 4) & ~3) * 4 + (MODE == kDenseGateUp ? 4 * 32 * 33 * 4 : 0);
+  return 1024 + (size_t)kDenseStages * kDenseStageBytes + kDenseBarBytes + 48 + (size_t)E * 16 +
+         (size_t)((E + 4) & ~3) * 4 + (MODE == kDenseGateUp ? kDenseEpiWarps * 32 * 33 * 4 : 0);
 }
 
 }  // namespace moe

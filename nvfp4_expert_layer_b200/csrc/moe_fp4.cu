@@ -89,8 +89,8 @@ struct moe_fp4 {
   float* gs = nullptr;            // [3][E]: gate, up, down
   uint8_t* dq_gu = nullptr;       // dense class: gate/up codes, rows interleaved by 16, signs folded [E*2f][d/2]
   uint8_t* dq_down = nullptr;     // [E*d][f/2]
-  uint8_t* dsf_gu = nullptr;      // scale atoms [E][f/64][d/64][512]
-  uint8_t* dsf_dn = nullptr;      // scale atoms [E][d/128][f/64][512]
+  uint8_t* dsf_gu = nullptr;      // scales, tensor-core layout (sf_pair_offset), rows E*2f, K = d
+  uint8_t* dsf_dn = nullptr;      // rows E*d, K = f
   CUtensorMap tm_gu{}, tm_down{};
   bool dense_ok = false;          // d, f multiples of 256 and tensor maps available
   bool dense_h32 = false;         // write fp32 h of the dense class (debug copies)
@@ -190,9 +190,9 @@ size_t workspace_bytes(const moe_fp4* h, int Tm) {
   add(4);                                              // dense padded rows
   const size_t pr = dense_pad_rows(h, Tm);
   add(pr * h->d / 2);                                  // xq
-  add(pr / 128 * (h->d / 64) * 512);                   // xsf
+  add(moe::sf_pair_bytes(pr, h->d));                   // xsf
   add(pr * h->f / 2);                                  // hq
-  add(pr / 128 * (h->f / 64) * 512);                   // hsf
+  add(moe::sf_pair_bytes(pr, h->f));                   // hsf
   add((size_t)h->E * 16);           // dense list
   add(4);
   add((size_t)Tm * h->d * 2);       // x16
@@ -253,9 +253,9 @@ int ensure_workspace(moe_fp4* h, int Tm, cudaStream_t stream) {
   w.dense_pad_total = carve<int>(cur, 1);
   w.pad_rows = dense_pad_rows(h, Tm);
   w.xq = carve<uint8_t>(cur, w.pad_rows * h->d / 2);
-  w.xsf = carve<uint8_t>(cur, w.pad_rows / 128 * (h->d / 64) * 512);
+  w.xsf = carve<uint8_t>(cur, moe::sf_pair_bytes(w.pad_rows, h->d));
   w.hq = carve<uint8_t>(cur, w.pad_rows * h->f / 2);
-  w.hsf = carve<uint8_t>(cur, w.pad_rows / 128 * (h->f / 64) * 512);
+  w.hsf = carve<uint8_t>(cur, moe::sf_pair_bytes(w.pad_rows, h->f));
   if (!make_map(&w.tm_x, w.xq, h->d / 2, w.pad_rows, 128) || !make_map(&w.tm_h, w.hq, h->f / 2, w.pad_rows, 128))
     h->dense_ok = false;
   if (cudaMemset(w.counters, 0, w.counter_bytes) != cudaSuccess) {
@@ -597,8 +597,8 @@ int moe_fp4_load_experts(moe_fp4_t* h, const moe_fp4_experts* w) {
   // dense class: codes with block-scale signs folded, scale atoms, tensor maps
   {
     const size_t gu_codes = (size_t)E * f * d / 2, dn_codes = (size_t)E * d * f / 2;
-    const size_t gu_atoms = (size_t)E * (f / 64) * (d / 64) * 512;
-    const size_t dn_atoms = (size_t)E * (d / 128) * (f / 64) * 512;
+    const size_t gu_atoms = moe::sf_pair_bytes((long long)E * 2 * f, d);
+    const size_t dn_atoms = moe::sf_pair_bytes((long long)E * d, f);
     auto alloc = [](uint8_t** p, size_t n) {
       if (*p) return true;
       if (cudaMalloc(p, n) != cudaSuccess) { (void)cudaGetLastError(); *p = nullptr; return false; }

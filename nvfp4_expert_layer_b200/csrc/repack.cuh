@@ -3,6 +3,7 @@
 #pragma once
 #include <cstdint>
 #include "layout.cuh"
+#include "tc.cuh"
 
 namespace moe {
 
@@ -119,39 +120,31 @@ __global__ void dense_gu_codes_kernel(const uint8_t* __restrict__ gq, const uint
   }
 }
 
-// Scale atoms of the dense weights, one thread per atom byte.
-// MODE kGateUp: M tile mt of expert e = combined (interleaved) gate/up rows
-// 128mt..128mt+127, i.e. FFN channels 64mt..64mt+63; K = d.
-// MODE kDown: M tile mt = down rows 128mt..128mt+127; K = f.
-// Atom (e, mt, kb64) holds byte (r % 32) * 16 + (r / 32) * 4 + kb4 = scale of
-// atom row r for K block 4 * kb64 + kb4, sign bit cleared.
+// Scales of the dense weights in the tensor-core layout (sf_pair_offset),
+// sign bit cleared.  One thread per (combined row, 16-block).
+// MODE kGateUp: combined (interleaved) gate/up rows, rows = f per matrix, K = d.
+// MODE kDown: down rows, rows = d, K = f.
 template <int MODE>
 __global__ void dense_sf_atoms_kernel(const uint8_t* __restrict__ sfa, const uint8_t* __restrict__ sfb,
                                       int E, int rows, int K, uint8_t* __restrict__ out) {
-  const int kb64n = K / 64;
-  const int mtpe = (MODE == kGateUp) ? rows / 64 : rows / 128;
-  const long long total = (long long)E * mtpe * kb64n * 512;
+  const int nb = K / 16;
+  const int crows = (MODE == kGateUp) ? 2 * rows : rows;     // combined rows per expert
+  const long long total = (long long)E * crows * nb;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (long long)gridDim.x * blockDim.x) {
-    const int byte = (int)(i & 511);
-    const long long atom = i >> 9;
-    const int kb64 = (int)(atom % kb64n);
-    const long long em = atom / kb64n;
-    const int mt = (int)(em % mtpe);
-    const int e = (int)(em / mtpe);
-    const int r0 = byte >> 4, r1 = (byte >> 2) & 3, kb4 = byte & 3;
-    const int r = r1 * 32 + r0;
-    const uint8_t* src;
-    long long row;
+    const long long R = i / nb;
+    const int kb = (int)(i - R * nb);
+    const int e = (int)(R / crows), rr = (int)(R % crows);
+    const uint8_t* src = sfa;
+    long long row = (long long)e * rows + rr;
     if (MODE == kGateUp) {
-      const int rr = mt * 128 + r;
       src = gu_is_up(rr) ? sfb : sfa;
       row = (long long)e * rows + gu_channel(rr);
-    } else {
-      src = sfa;
-      row = (long long)e * rows + mt * 128 + r;
     }
-    out[i] = src[row * (K / 16) + kb64 * 4 + kb4] & 0x7Fu;
+    const uint8_t v = src[row * nb + kb] & 0x7Fu;
+    const size_t o = sf_pair_offset(R, kb, K / 64);
+#pragma unroll
+    for (int c = 0; c < kSfReplicas; ++c) out[o + 1024 * c] = v;
   }
 }
 

@@ -28,9 +28,10 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                :: "r"(bar) : "memory");
 }
-// Shared memory (descriptor) -> TMEM: 32 lanes x 128 bits, broadcast to the 4 lane quarters.
-__device__ __forceinline__ void tc_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(sdesc) : "memory");
+// Shared memory (descriptor) -> TMEM: 128 lanes x 256 bits (8 columns), lane L
+// from source row L.
+__device__ __forceinline__ void tc_cp_128x256b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" :: "r"(taddr), "l"(sdesc) : "memory");
 }
 // D[128 x N] (+)= A[128 x 64] * B[N x 64]^T, NVFP4 operands with e4m3 scales per 16 (in TMEM).
 __device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -72,12 +73,14 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
   d |= (uint64_t)2 << 61;                           // layout: SWIZZLE_128B
   return d;
 }
-// Scale-factor atom (32 rows x 16 bytes, contiguous, no swizzle) as tcgen05.cp source.
-__device__ __forceinline__ uint64_t smem_desc_sf(uint32_t saddr) {
+// Scale-factor copy source: 128 rows x 32 bytes, no swizzle, as core matrices
+// of 8 rows x 16 bytes; the two 16-byte halves of a row group are 128 bytes
+// apart (leading byte offset), row groups 256 bytes apart (stride byte offset).
+__device__ __forceinline__ uint64_t smem_desc_sf256(uint32_t saddr) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFF);
-  d |= (uint64_t)1 << 16;                           // leading byte offset (single core matrix along K)
-  d |= (uint64_t)(128 >> 4) << 32;                  // stride byte offset: 8 rows x 16 bytes
+  d |= (uint64_t)(128 >> 4) << 16;
+  d |= (uint64_t)(256 >> 4) << 32;
   d |= (uint64_t)1 << 46;
   return d;                                         // layout: SWIZZLE_NONE
 }
@@ -115,14 +118,26 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
   return __half2float(__ushort_as_half((unsigned short)(h2 & 0xffffu)));
 }
 
-// Byte offset of the scale of (row r, K block kb of 16) inside the scale-atom
-// layout of a matrix whose rows are grouped by 128: atoms of 128 rows x 4
-// blocks (512 bytes), ordered (row group, K group of 64) with K fastest;
-// inside an atom byte (r % 32) * 16 + ((r % 128) / 32) * 4 + kb % 4.
-__host__ __device__ __forceinline__ size_t sf_atom_offset(long long r, int kb, int kblocks64) {
+// Byte offset of the scale of (row r, K block kb of 16) in the scale layout of
+// the tensor-core operands.  Rows are grouped by 128 (one MMA tile) and K by
+// pairs of 64-wide groups (two MMAs); each (row tile, pair) is a 4 KB unit:
+// four identical 1 KB replicas, each holding 32 row slots l = r % 32 as 8-row
+// core matrices at
+//   (l / 8) * 256 + h * 128 + (l % 8) * 16 + (r % 128 / 32) * 4 + kb % 4,
+// h = which 64-group of the pair.  The unit is the 128-row source of one
+// tcgen05.cp .128x256b, which gives every TMEM lane quarter the same 32 x 8
+// columns: column 4h + (r % 128) / 32 of lane r % 32 holds the four scales of
+// row r for the MMA of 64-group h.  Writers store the byte at this offset and
+// at +1024, +2048, +3072.  Size: rows / 128 * (K / 128) * 4096 bytes.
+constexpr int kSfReplicas = 4;
+__host__ __device__ __forceinline__ size_t sf_pair_offset(long long r, int kb, int kblocks64) {
   const long long tile = r >> 7;
-  const int rr = (int)(r & 127);
-  return ((size_t)tile * kblocks64 + (kb >> 2)) * 512 + (size_t)((rr & 31) * 16 + (rr >> 5) * 4 + (kb & 3));
+  const int rr = (int)(r & 127), l = rr & 31, kg = kb >> 2;
+  return ((size_t)tile * (kblocks64 >> 1) + (kg >> 1)) * (1024 * kSfReplicas) +
+         (size_t)((l >> 3) * 256 + (kg & 1) * 128 + (l & 7) * 16 + (rr >> 5) * 4 + (kb & 3));
+}
+__host__ __device__ constexpr size_t sf_pair_bytes(long long rows, int K) {
+  return (size_t)(rows / 128) * (K / 128) * 1024 * kSfReplicas;
 }
 
 }  // namespace moe
