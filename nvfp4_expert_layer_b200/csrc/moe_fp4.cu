@@ -89,7 +89,7 @@ struct moe_fp4 {
   float* gs = nullptr;            // [3][E]: gate, up, down
   uint8_t* dq_gu = nullptr;       // dense class: gate/up codes, rows interleaved by 16, signs folded [E*2f][d/2]
   uint8_t* dq_down = nullptr;     // [E*d][f/2]
-  uint8_t* dsf_gu = nullptr;      // scales, tensor-core layout (sf_pair_offset), rows E*2f, K = d
+  uint8_t* dsf_gu = nullptr;      // weight scales, 256-row tile layout (sf_rowpair_offset), rows E*2f, K = d
   uint8_t* dsf_dn = nullptr;      // rows E*d, K = f
   CUtensorMap tm_gu{}, tm_down{};
   bool dense_ok = false;          // d, f multiples of 256 and tensor maps available
@@ -369,14 +369,14 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
                     (const int*)w.perm, k, d, w.xq, w.xsf));
     MOE_CUDA(mark(h, 4, st));
     moe::DenseParams dp{};
-    dp.tmA = h->tm_gu;
-    dp.tmB = w.tm_x;
-    dp.sfA = h->dsf_gu;
-    dp.sfB = w.xsf;
+    dp.tmA = w.tm_x;           // tokens: the M side of the MMA
+    dp.tmB = h->tm_gu;         // weights: 256-row N tiles
+    dp.sfA = w.xsf;
+    dp.sfB = h->dsf_gu;
     dp.dense = w.dense_list;
     dp.n_dense = w.n_dense;
     dp.ntoff = w.dense_ntoff;
-    dp.mt_per_expert = f / 64;
+    dp.wt_per_expert = 2 * f / moe::kDenseN;
     dp.rows_per_expert = 2 * f;
     dp.kstages = d / 256;
     dp.kb64 = d / 64;
@@ -397,11 +397,11 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
                     dim3(moe::kDenseThreads), moe::dense_smem_size<moe::kDenseGateUp>(E), st, pdl, dp));
     MOE_CUDA(mark(h, 5, st));
     moe::DenseParams dp2 = dp;
-    dp2.tmA = h->tm_down;
-    dp2.tmB = w.tm_h;
-    dp2.sfA = h->dsf_dn;
-    dp2.sfB = w.hsf;
-    dp2.mt_per_expert = d / 128;
+    dp2.tmA = w.tm_h;
+    dp2.tmB = h->tm_down;
+    dp2.sfA = w.hsf;
+    dp2.sfB = h->dsf_dn;
+    dp2.wt_per_expert = d / moe::kDenseN;
     dp2.rows_per_expert = d;
     dp2.kstages = f / 256;
     dp2.kb64 = f / 64;
@@ -597,8 +597,8 @@ int moe_fp4_load_experts(moe_fp4_t* h, const moe_fp4_experts* w) {
   // dense class: codes with block-scale signs folded, scale atoms, tensor maps
   {
     const size_t gu_codes = (size_t)E * f * d / 2, dn_codes = (size_t)E * d * f / 2;
-    const size_t gu_atoms = moe::sf_pair_bytes((long long)E * 2 * f, d);
-    const size_t dn_atoms = moe::sf_pair_bytes((long long)E * d, f);
+    const size_t gu_atoms = moe::sf_rowpair_bytes((long long)E * 2 * f, d);
+    const size_t dn_atoms = moe::sf_rowpair_bytes((long long)E * d, f);
     auto alloc = [](uint8_t** p, size_t n) {
       if (*p) return true;
       if (cudaMalloc(p, n) != cudaSuccess) { (void)cudaGetLastError(); *p = nullptr; return false; }
@@ -614,8 +614,8 @@ int moe_fp4_load_experts(moe_fp4_t* h, const moe_fp4_experts* w) {
     moe::dense_sf_atoms_kernel<moe::kDown><<<blocks, 256>>>(w->down_sf, nullptr, E, d, f, h->dsf_dn);
     MOE_CUDA(cudaGetLastError());
     h->dense_ok = (d % 256 == 0) && (f % 256 == 0) &&
-                  make_map(&h->tm_gu, h->dq_gu, d / 2, (uint64_t)E * 2 * f, 128) &&
-                  make_map(&h->tm_down, h->dq_down, f / 2, (uint64_t)E * d, 128);
+                  make_map(&h->tm_gu, h->dq_gu, d / 2, (uint64_t)E * 2 * f, moe::kDenseN) &&
+                  make_map(&h->tm_down, h->dq_down, f / 2, (uint64_t)E * d, moe::kDenseN);
     if (h->ws.base && (!make_map(&h->ws.tm_x, h->ws.xq, d / 2, h->ws.pad_rows, 128) ||
                        !make_map(&h->ws.tm_h, h->ws.hq, f / 2, h->ws.pad_rows, 128)))
       h->dense_ok = false;

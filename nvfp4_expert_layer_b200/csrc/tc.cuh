@@ -140,4 +140,21 @@ __host__ __device__ constexpr size_t sf_pair_bytes(long long rows, int K) {
   return (size_t)(rows / 128) * (K / 128) * 1024 * kSfReplicas;
 }
 
+// Scale layout of an operand read as 256-row MMA tiles (N = 256): 4 KB units
+// per (256-row group, 64-wide K group), four identical 1 KB replicas with 32
+// row slots l = r % 32 as core matrices at
+//   (l / 8) * 256 + h * 128 + (l % 8) * 16 + (r % 128 / 32) * 4 + kb % 4,
+// h = (r % 256) / 128.  One tcgen05.cp .128x256b of a unit fills the 8 scale
+// columns one N = 256 MMA reads: column (r % 256) / 32 of lane r % 32, in
+// every lane quarter.  Size: rows / 256 * (K / 64) * 4096 bytes.
+__host__ __device__ __forceinline__ size_t sf_rowpair_offset(long long r, int kb, int kblocks64) {
+  const long long g = r >> 8;
+  const int rr = (int)(r & 255), h = rr >> 7, r128 = rr & 127, l = r128 & 31;
+  return ((size_t)g * kblocks64 + (kb >> 2)) * (1024 * kSfReplicas) +
+         (size_t)((l >> 3) * 256 + h * 128 + (l & 7) * 16 + (r128 >> 5) * 4 + (kb & 3));
+}
+__host__ __device__ constexpr size_t sf_rowpair_bytes(long long rows, int K) {
+  return (size_t)(rows / 256) * (K / 64) * 1024 * kSfReplicas;
+}
+
 }  // namespace moe
