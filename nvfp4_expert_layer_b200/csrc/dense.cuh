@@ -11,16 +11,20 @@
 // both decided in IEEE fp32.  Rows of every dense expert are padded to a
 // multiple of 128 so each 128-token tile starts on a scale-unit boundary.
 //
-// Each MMA is D[128 tokens][256 weight rows] += X[128][64] * W[256][64]^T
-// (kind::mxf4nvf4, scale vector 16): tokens are the M side, so one TMEM lane
-// holds one token and its accumulator row runs along the weight rows.
-// GEMM 1 (kDenseGateUp): the weight rows are the combined gate/up matrix, gate
-//   and up interleaved in groups of 16 channels, so a lane's 32 consecutive
-//   columns are the gate and the up values of one 16-channel NVFP4 block of
-//   h: the epilogue forms h = SiLU(g) * u, the block scale and the codes in
-//   registers and writes 32 bytes of the B operand of GEMM 2 per block pair.
-// GEMM 2 (kDenseDown): the weight rows are Wd; the epilogue writes w * gs * D
-//   as fp32 partials (rows in permutation order), 512 contiguous bytes per lane.
+// Each MMA is D[128][N] += A[128][64] * B[N][64]^T (kind::mxf4nvf4, scale
+// vector 16, N = 256, or 128 for a short last token tile of GEMM 2).
+// GEMM 1 (kDenseGateUp): A = 128 tokens, B = 256 rows of the combined gate/up
+//   matrix, gate and up interleaved in groups of 16 channels.  One TMEM lane
+//   holds one token, and its 32 consecutive columns are the gate and the up
+//   values of one 16-channel NVFP4 block of h: the epilogue forms
+//   h = SiLU(g) * u, the block scale and the codes in registers and writes
+//   the B operand of GEMM 2.
+// GEMM 2 (kDenseDown): A = 128 rows of Wd, B = 256 tokens.  One TMEM lane
+//   holds one output dimension, so for each token the 32 lanes of a warp write
+//   128 contiguous bytes of the fp32 partial w * gs * D (permutation order).
+// The A side is read as 128-row tiles with scales in the sf_pair_offset
+// layout, the B side as 256-row tiles with scales in the sf_rowpair_offset
+// layout; dense experts are padded to 256 rows.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -48,14 +52,15 @@ enum DenseMode { kDenseGateUp = 0, kDenseDown = 1 };
 
 // Dense list entry: {expert, row0 (permutation rows), rows, padded row0}.
 struct DenseParams {
-  CUtensorMap tmA;       // activations (NVFP4, padded permutation order) [rows][K/2]; box 128 B x 128 rows
-  CUtensorMap tmB;       // weights: combined gate/up rows [E*2f] or down rows [E*d]; box 128 B x 256 rows
-  const uint8_t* sfA;    // activation scales (sf_pair_offset layout)
-  const uint8_t* sfB;    // weight scales (sf_rowpair_offset layout)
+  CUtensorMap tmA;       // M side, box 128 B x 128 rows: gate/up x codes [pad rows][d/2]; down Wd [E*d][f/2]
+  CUtensorMap tmB;       // N side, box 128 B x 256 rows: gate/up combined W [E*2f][d/2]; down h codes [pad rows][f/2]
+  const uint8_t* sfA;    // M-side scales (sf_pair_offset layout)
+  const uint8_t* sfB;    // N-side scales (sf_rowpair_offset layout)
   const int4* dense;     // dense list, ranked by rows descending
   const int* n_dense;
-  const int* ntoff;      // [E+1] exclusive prefix of ceil(rows / 128) over the dense list
-  int wt_per_expert;     // 256-row weight tiles per expert: gate/up 2f / 256, down d / 256
+  const int* ntoff;      // [E+1] exclusive prefix over the dense list of the token tiles per expert
+                         // (gate/up: ceil(rows / 128); down: ceil(rows / 256))
+  int wt_per_expert;     // weight tiles per expert: gate/up 2f / 256, down d / 128
   int rows_per_expert;   // gate/up: 2f; down: d (rows of the weight copy per expert)
   int kstages;           // K / 256
   int kb64;              // K / 64
@@ -66,7 +71,7 @@ struct DenseParams {
   const float* wts;
   // gate/up outputs
   uint8_t* hq;           // [P_pad][f/2]
-  uint8_t* hsf;          // scales of hq (sf_pair_offset layout, K = f)
+  uint8_t* hsf;          // scales of hq (sf_rowpair_offset layout, K = f)
   float* h32;            // [P][f] or null
   // down output
   float* partial;        // [P][d]
@@ -223,8 +228,10 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
       int k = 0;
       for (int it = 0; it < my_tiles && !failed; ++it) {
         const DenseTile tl = dense_tile(p.dense, p.ntoff, nd, p.wt_per_expert, b + it * G);
-        const int arow = tl.de.w + tl.tt * 128;                             // padded token row
-        const int brow = tl.de.x * p.rows_per_expert + tl.wt * kDenseN;     // weight row
+        const int wrow = tl.de.x * p.rows_per_expert + tl.wt * (MODE == kDenseGateUp ? kDenseN : 128);
+        const int trow = tl.de.w + tl.tt * (MODE == kDenseGateUp ? 128 : kDenseN);   // padded token row
+        const int arow = MODE == kDenseGateUp ? trow : wrow;
+        const int brow = MODE == kDenseGateUp ? wrow : trow;
         const uint8_t* sfa = p.sfA + (size_t)(arow >> 7) * (p.kb64 >> 1) * 4096;
         const uint8_t* sfb = p.sfB + (size_t)(brow >> 8) * p.kb64 * 4096;
         for (int ks = 0; ks < p.kstages; ++ks, ++k) {
@@ -250,10 +257,15 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_nvf4(kDenseN);
       int k = 0;
       bool issued_any = false;
       for (int it = 0; it < my_tiles && !failed; ++it) {
+        // N = 256, or 128 when the down GEMM's token tile holds at most 128 rows
+        uint32_t idesc = idesc_nvf4(kDenseN);
+        if (MODE == kDenseDown) {
+          const DenseTile tl = dense_tile(p.dense, p.ntoff, nd, p.wt_per_expert, b + it * G);
+          if (tl.de.z - tl.tt * kDenseN <= 128) idesc = idesc_nvf4(128);
+        }
         // the epilogue has drained the previous tile's accumulator
         if (!mbar_wait_spin(acce_b, (it & 1) ^ 1, deadline)) {
           failed = true; set_error(p.err, kErrTimeout); break;
@@ -324,22 +336,31 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
       __syncwarp();
       if (lane == 0) mbar_arrive(acce_b);
       const int e = tl.de.x;
-      const int tok = q * 32 + lane;                     // token of this lane within the tile
-      const bool valid = tl.tt * 128 + tok < tl.de.z;
-      const int prow = tl.de.y + tl.tt * 128 + tok;      // permutation row
-      const int hrow = tl.de.w + tl.tt * 128 + tok;      // padded row
       if (MODE == kDenseDown) {
-        if (valid) {
-          const float wv = p.wts[p.perm[prow]] * p.gs[2 * p.E + e];
-          float4* dst = reinterpret_cast<float4*>(p.partial + (size_t)prow * p.d + tl.wt * kDenseN + hf * 128);
+        // lane = output dimension drow; columns = tokens 128 hf .. 128 hf + 127 of the tile
+        const int drow = tl.wt * 128 + q * 32 + lane;
+        const int nrows = min(kDenseN, tl.de.z - tl.tt * kDenseN) - hf * 128;
+        const int prow0 = tl.de.y + tl.tt * kDenseN + hf * 128;      // permutation row of column 0
+        const float gsd = p.gs[2 * p.E + e];
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            dst[i] = make_float4(__uint_as_float(r[4 * i]) * wv, __uint_as_float(r[4 * i + 1]) * wv,
-                                 __uint_as_float(r[4 * i + 2]) * wv, __uint_as_float(r[4 * i + 3]) * wv);
+        for (int c32 = 0; c32 < 4; ++c32) {
+          if (32 * c32 >= nrows) break;                              // warp-uniform
+          // routing weight x tensor scale of column 32 c32 + lane, broadcast below
+          const float wl = 32 * c32 + lane < nrows ? p.wts[p.perm[prow0 + 32 * c32 + lane]] * gsd : 0.f;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float wv = __shfl_sync(0xffffffffu, wl, c);
+            if (32 * c32 + c < nrows)
+              p.partial[(size_t)(prow0 + 32 * c32 + c) * p.d + drow] = __uint_as_float(r[32 * c32 + c]) * wv;
+          }
         }
       } else {
         // columns 32 bl .. 32 bl + 31: gate (first 16) and up (last 16) of the
         // channels chb + 16 bl .. chb + 16 bl + 15, one NVFP4 block of h each
+        const int tok = q * 32 + lane;                   // token of this lane within the tile
+        const bool valid = tl.tt * 128 + tok < tl.de.z;
+        const int prow = tl.de.y + tl.tt * 128 + tok;    // permutation row
+        const int hrow = tl.de.w + tl.tt * 128 + tok;    // padded row
         const float gsg = p.gs[e], gsu = p.gs[p.E + e];
         const int chb = tl.wt * (kDenseN / 2) + hf * 64;
         uint32_t codes[8];
@@ -379,7 +400,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
         dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
         dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
         // the four blocks share one 64-wide K group: four consecutive scale bytes
-        const size_t so = sf_pair_offset(hrow, chb >> 4, p.f / 64);
+        const size_t so = sf_rowpair_offset(hrow, chb >> 4, p.f / 64);
 #pragma unroll
         for (int c = 0; c < kSfReplicas; ++c) *reinterpret_cast<uint32_t*>(p.hsf + so + 1024 * c) = sfw;
       }

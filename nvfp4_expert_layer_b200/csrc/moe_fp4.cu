@@ -54,7 +54,7 @@ struct Workspace {
   size_t counter_bytes = 0;
   int4* dense_list = nullptr;
   int* n_dense = nullptr;
-  int* dense_ntoff = nullptr;    // [E+1]
+  int* dense_ntoff = nullptr;    // [2][E+1]: 128-row and 256-row tile prefixes
   int* dense_pad_total = nullptr;
   uint8_t* xq = nullptr;         // dense class: NVFP4 activations [pad_rows][d/2]
   uint8_t* xsf = nullptr;        //   and their scale atoms
@@ -90,7 +90,7 @@ struct moe_fp4 {
   uint8_t* dq_gu = nullptr;       // dense class: gate/up codes, rows interleaved by 16, signs folded [E*2f][d/2]
   uint8_t* dq_down = nullptr;     // [E*d][f/2]
   uint8_t* dsf_gu = nullptr;      // weight scales, 256-row tile layout (sf_rowpair_offset), rows E*2f, K = d
-  uint8_t* dsf_dn = nullptr;      // rows E*d, K = f
+  uint8_t* dsf_dn = nullptr;      // 128-row tile layout (sf_pair_offset), rows E*d, K = f
   CUtensorMap tm_gu{}, tm_down{};
   bool dense_ok = false;          // d, f multiples of 256 and tensor maps available
   bool dense_h32 = false;         // write fp32 h of the dense class (debug copies)
@@ -127,7 +127,7 @@ size_t counter_ints(const moe_fp4* h, int Tm) {
 // rows per dense expert, in whole 128-row tiles
 size_t dense_pad_rows(const moe_fp4* h, int Tm) {
   const size_t P = (size_t)Tm * h->k;
-  return (P + 128 * std::min<size_t>(h->E, P) + 127) / 128 * 128;
+  return (P + 256 * std::min<size_t>(h->E, P) + 255) / 256 * 256;
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -186,13 +186,13 @@ size_t workspace_bytes(const moe_fp4* h, int Tm) {
   add(((size_t)h->E + P / moe::kJobRows + 1) * 16);   // light jobs, 9..16 rows
   add(4);
   add(counter_ints(h, Tm) * 4);                        // counters
-  add(((size_t)h->E + 1) * 4);                         // dense n-tile prefix
+  add(((size_t)h->E + 1) * 8);                         // dense 128- and 256-row tile prefixes
   add(4);                                              // dense padded rows
   const size_t pr = dense_pad_rows(h, Tm);
   add(pr * h->d / 2);                                  // xq
   add(moe::sf_pair_bytes(pr, h->d));                   // xsf
   add(pr * h->f / 2);                                  // hq
-  add(moe::sf_pair_bytes(pr, h->f));                   // hsf
+  add(moe::sf_rowpair_bytes(pr, h->f));                // hsf
   add((size_t)h->E * 16);           // dense list
   add(4);
   add((size_t)Tm * h->d * 2);       // x16
@@ -249,14 +249,14 @@ int ensure_workspace(moe_fp4* h, int Tm, cudaStream_t stream) {
   w.partial = carve<float>(cur, P * h->d);
   w.xin = carve<uint16_t>(cur, (size_t)Tm * h->d);
   w.xout = carve<uint16_t>(cur, (size_t)Tm * h->d);
-  w.dense_ntoff = carve<int>(cur, h->E + 1);
+  w.dense_ntoff = carve<int>(cur, 2 * (h->E + 1));
   w.dense_pad_total = carve<int>(cur, 1);
   w.pad_rows = dense_pad_rows(h, Tm);
   w.xq = carve<uint8_t>(cur, w.pad_rows * h->d / 2);
   w.xsf = carve<uint8_t>(cur, moe::sf_pair_bytes(w.pad_rows, h->d));
   w.hq = carve<uint8_t>(cur, w.pad_rows * h->f / 2);
-  w.hsf = carve<uint8_t>(cur, moe::sf_pair_bytes(w.pad_rows, h->f));
-  if (!make_map(&w.tm_x, w.xq, h->d / 2, w.pad_rows, 128) || !make_map(&w.tm_h, w.hq, h->f / 2, w.pad_rows, 128))
+  w.hsf = carve<uint8_t>(cur, moe::sf_rowpair_bytes(w.pad_rows, h->f));
+  if (!make_map(&w.tm_x, w.xq, h->d / 2, w.pad_rows, 128) || !make_map(&w.tm_h, w.hq, h->f / 2, w.pad_rows, 256))
     h->dense_ok = false;
   if (cudaMemset(w.counters, 0, w.counter_bytes) != cudaSuccess) {
     (void)cudaGetLastError();
@@ -397,11 +397,12 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
                     dim3(moe::kDenseThreads), moe::dense_smem_size<moe::kDenseGateUp>(E), st, pdl, dp));
     MOE_CUDA(mark(h, 5, st));
     moe::DenseParams dp2 = dp;
-    dp2.tmA = w.tm_h;
-    dp2.tmB = h->tm_down;
-    dp2.sfA = w.hsf;
-    dp2.sfB = h->dsf_dn;
-    dp2.wt_per_expert = d / moe::kDenseN;
+    dp2.tmA = h->tm_down;       // weights: 128-row M tiles
+    dp2.tmB = w.tm_h;           // tokens: 256-row N tiles
+    dp2.sfA = h->dsf_dn;
+    dp2.sfB = w.hsf;
+    dp2.ntoff = w.dense_ntoff + (E + 1);
+    dp2.wt_per_expert = d / 128;
     dp2.rows_per_expert = d;
     dp2.kstages = f / 256;
     dp2.kb64 = f / 64;
@@ -598,7 +599,7 @@ int moe_fp4_load_experts(moe_fp4_t* h, const moe_fp4_experts* w) {
   {
     const size_t gu_codes = (size_t)E * f * d / 2, dn_codes = (size_t)E * d * f / 2;
     const size_t gu_atoms = moe::sf_rowpair_bytes((long long)E * 2 * f, d);
-    const size_t dn_atoms = moe::sf_rowpair_bytes((long long)E * d, f);
+    const size_t dn_atoms = moe::sf_pair_bytes((long long)E * d, f);
     auto alloc = [](uint8_t** p, size_t n) {
       if (*p) return true;
       if (cudaMalloc(p, n) != cudaSuccess) { (void)cudaGetLastError(); *p = nullptr; return false; }
@@ -615,9 +616,9 @@ int moe_fp4_load_experts(moe_fp4_t* h, const moe_fp4_experts* w) {
     MOE_CUDA(cudaGetLastError());
     h->dense_ok = (d % 256 == 0) && (f % 256 == 0) &&
                   make_map(&h->tm_gu, h->dq_gu, d / 2, (uint64_t)E * 2 * f, moe::kDenseN) &&
-                  make_map(&h->tm_down, h->dq_down, f / 2, (uint64_t)E * d, moe::kDenseN);
+                  make_map(&h->tm_down, h->dq_down, f / 2, (uint64_t)E * d, 128);
     if (h->ws.base && (!make_map(&h->ws.tm_x, h->ws.xq, d / 2, h->ws.pad_rows, 128) ||
-                       !make_map(&h->ws.tm_h, h->ws.hq, f / 2, h->ws.pad_rows, 128)))
+                       !make_map(&h->ws.tm_h, h->ws.hq, f / 2, h->ws.pad_rows, 256)))
       h->dense_ok = false;
   }
   MOE_CUDA(cudaMemcpy(h->gs, w->gate_gs, sizeof(float) * E, cudaMemcpyDeviceToDevice));

@@ -120,8 +120,9 @@ __global__ void dense_gu_codes_kernel(const uint8_t* __restrict__ gq, const uint
   }
 }
 
-// Scales of the dense weights in the layout of 256-row MMA operands
-// (sf_rowpair_offset), sign bit cleared.  One thread per (combined row, 16-block).
+// Scales of the dense weights in the tensor-core layouts (gate/up:
+// sf_rowpair_offset, 256-row N tiles; down: sf_pair_offset, 128-row M tiles),
+// sign bit cleared.  One thread per (combined row, 16-block).
 // MODE kGateUp: combined (interleaved) gate/up rows, rows = f per matrix, K = d.
 // MODE kDown: down rows, rows = d, K = f.
 template <int MODE>
@@ -142,7 +143,8 @@ __global__ void dense_sf_atoms_kernel(const uint8_t* __restrict__ sfa, const uin
       row = (long long)e * rows + gu_channel(rr);
     }
     const uint8_t v = src[row * nb + kb] & 0x7Fu;
-    const size_t o = sf_rowpair_offset(R, kb, K / 64);
+    // gate/up weights are the N = 256 operand, down weights the M = 128 one
+    const size_t o = MODE == kGateUp ? sf_rowpair_offset(R, kb, K / 64) : sf_pair_offset(R, kb, K / 64);
 #pragma unroll
     for (int c = 0; c < kSfReplicas; ++c) out[o + 1024 * c] = v;
   }

@@ -220,8 +220,9 @@ struct PermuteOut {
   int* n_jobs2;
   int4* dense_list;  // [E]            {expert, row0, nrows, padded row0}
   int* n_dense;
-  int* dense_ntoff;  // [E+1]          exclusive prefix of ceil(nrows / 128) over the dense list
-  int* dense_pad_total;  // padded rows of the dense class (each expert rounded up to 128)
+  int* dense_ntoff;  // [2][E+1]       exclusive prefixes of ceil(nrows / 128) and ceil(nrows / 256)
+                     //                over the dense list
+  int* dense_pad_total;  // padded rows of the dense class (each expert rounded up to 256)
   int* err;
 };
 
@@ -307,7 +308,7 @@ __device__ void build_permutation(const int* ids, int T, int k, int E, int thr, 
     const int e = act[a];
     const int n = cnt[e];
     const bool light = n < thr;
-    int rank = 0, s1 = 0, s2 = 0, pad0 = 0, nt0 = 0;
+    int rank = 0, s1 = 0, s2 = 0, pad0 = 0, nt0 = 0, nt1 = 0;
     for (int b = 0; b < A; ++b) {
       const int e2 = act[b], n2 = cnt[e2];
       if ((n2 < thr) != light) continue;
@@ -316,8 +317,9 @@ __device__ void build_permutation(const int* ids, int T, int k, int E, int thr, 
         const int r2 = n2 % kJobRows;
         s1 += (r2 > 0 && r2 <= 8) ? 1 : 0;
         s2 += n2 / kJobRows + (r2 > 8 ? 1 : 0);
-        pad0 += (n2 + 127) & ~127;
+        pad0 += (n2 + 255) & ~255;
         nt0 += (n2 + 127) >> 7;
+        nt1 += (n2 + 255) >> 8;
       }
     }
     if (light) {
@@ -332,9 +334,11 @@ __device__ void build_permutation(const int* ids, int T, int k, int E, int thr, 
     } else {
       o.dense_list[rank] = make_int4(e, off[e], n, pad0);
       o.dense_ntoff[rank] = nt0;
+      o.dense_ntoff[E + 1 + rank] = nt1;
       atomicAdd(&misc[3], 1);
       atomicAdd(&misc[4], (n + 127) >> 7);
-      atomicAdd(&misc[5], (n + 127) & ~127);
+      atomicAdd(&misc[5], (n + 255) & ~255);
+      atomicAdd(&misc[6], (n + 255) >> 8);
     }
   }
   __syncthreads();
@@ -343,6 +347,7 @@ __device__ void build_permutation(const int* ids, int T, int k, int E, int thr, 
     *o.n_jobs2 = misc[2];
     *o.n_dense = misc[3];
     o.dense_ntoff[misc[3]] = misc[4];
+    o.dense_ntoff[E + 1 + misc[3]] = misc[6];
     *o.dense_pad_total = misc[5];
     if (misc[3] > 0 && !dense_supported) set_error(o.err, kErrUnsupported);
   }
