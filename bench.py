@@ -386,7 +386,7 @@ def run_native(args, rank, world, local):
     # kernels per step: routing (1 fused launch up to 256 tokens, else router,
     # x staging, top-k, permutation), the dense class (quantiser + 2 GEMMs)
     # when T >= thr, the two light-class expert kernels and the combine
-    launches = (1 if cfg.T <= 256 else 4) + (3 if cfg.T >= 128 else 0) + 3
+    launches = (1 if cfg.T <= 256 else 5) + (4 if cfg.T >= 128 else 0) + 3
     return dict(cfg=cfg, ms=ms, clk=clk, err=err, stage_ms=stage_ms, dom_ms=dom_ms / n,
                 dom_work=dom_work / n, dense=dense, e2e_ms=e2e_ms, xs_np=xs_np, rw_np=rw_np,
                 gpu_out0=gpu_out0, launches_per_step=launches, stages=layer.STAGES,

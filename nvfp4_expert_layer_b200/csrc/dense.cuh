@@ -80,10 +80,16 @@ struct DenseParams {
 };
 
 // ---------------------------------------------------------------------------
-// Activation quantiser: one warp per padded row of the dense class.
-// src row (bf16) of token perm[row0 + i] / topk; rows past the expert's count
-// are written as zeros.  Output: codes [rows][K/2], scales in the
-// sf_pair_offset layout (four replicas).
+// Activation quantiser of the dense class, in two passes.
+// quant_tok_kernel: one warp per token: the bf16 row -> NVFP4 codes
+//   [T][d/2] and one e4m3 scale byte per 16 values [T][d/16] (plain layout).
+// gather_x_dense_kernel: one block per 128-row tile of the padded dense
+//   rows: the codes and scales of token perm[row0 + i] / topk copied into the
+//   padded permutation order (scales assembled into whole sf_pair_offset
+//   units, written as four replicas with coalesced 16-byte stores).
+//   Rows past an expert's count up to its next multiple of 128 -- the rows a
+//   128-token tile reads -- are zeros; rows beyond are never read.
+// Each token is quantised once, however many dense experts it is routed to.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ int dense_rank_of_padrow(const int4* dense, int nd, int prow) {
   int lo = 0, hi = nd - 1;                       // pad0 increases with rank
@@ -94,57 +100,96 @@ __device__ __forceinline__ int dense_rank_of_padrow(const int4* dense, int nd, i
   return lo;
 }
 
-__global__ void __launch_bounds__(256) quant_x_dense_kernel(
-    const uint16_t* __restrict__ x, const int4* __restrict__ dense, const int* __restrict__ n_dense,
-    const int* __restrict__ pad_total, const int* __restrict__ perm, int topk, int d,
-    uint8_t* __restrict__ xq, uint8_t* __restrict__ xsf) {
+__global__ void __launch_bounds__(256) quant_tok_kernel(const uint16_t* __restrict__ x, int T, int d,
+                                                        const int* __restrict__ n_dense,
+                                                        uint8_t* __restrict__ xq, uint8_t* __restrict__ xsf) {
   pdl_wait();
-  const int nd = *n_dense;
-  if (nd == 0) { pdl_launch_dependents(); return; }
-  const int total = *pad_total;
+  if (*n_dense == 0) { pdl_launch_dependents(); return; }
   const int lane = threadIdx.x & 31;
   const int nblk = d / 16;
-  for (int prow = blockIdx.x * 8 + (threadIdx.x >> 5); prow < total; prow += gridDim.x * 8) {
-    const int j = dense_rank_of_padrow(dense, nd, prow);
-    const int4 de = dense[j];
-    const int i = prow - de.w;
-    const bool valid = i < de.z;
-    const uint16_t* src = valid ? x + (size_t)(perm[de.y + i] / topk) * d : nullptr;
+  for (int t = blockIdx.x * 8 + (threadIdx.x >> 5); t < T; t += gridDim.x * 8) {
+    const uint16_t* src = x + (size_t)t * d;
     for (int blk = lane; blk < nblk; blk += 32) {
-      uint2 codes = make_uint2(0, 0);
-      uint32_t sfbyte = 0;
-      if (valid) {
-        const uint4 a = *reinterpret_cast<const uint4*>(src + blk * 16);
-        const uint4 b = *reinterpret_cast<const uint4*>(src + blk * 16 + 8);
-        const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-        float v[16];
+      const uint4 a = *reinterpret_cast<const uint4*>(src + blk * 16);
+      const uint4 b = *reinterpret_cast<const uint4*>(src + blk * 16 + 8);
+      const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      float v[16];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          v[2 * q] = __uint_as_float(wv[q] << 16);
-          v[2 * q + 1] = __uint_as_float(wv[q] & 0xffff0000u);
-        }
-        float amax = 0.f;
-#pragma unroll
-        for (int q = 0; q < 16; ++q) amax = fmaxf(amax, fabsf(v[q]));
-        sfbyte = f32x2_to_e4m3x2(0.f, amax / 6.0f) & 0xffu;
-        const float sf = e4m3_to_f32(sfbyte);
-        if (sf > 0.f) {
-          uint32_t c[8];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) c[q] = f32x2_to_e2m1x2(v[2 * q + 1] / sf, v[2 * q] / sf);
-          codes.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-          codes.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
-        }
+      for (int q = 0; q < 8; ++q) {
+        v[2 * q] = __uint_as_float(wv[q] << 16);
+        v[2 * q + 1] = __uint_as_float(wv[q] & 0xffff0000u);
       }
-      *reinterpret_cast<uint2*>(xq + (size_t)prow * (d / 2) + blk * 8) = codes;
-      const size_t so = sf_pair_offset(prow, blk, d / 64);
+      float amax = 0.f;
 #pragma unroll
-      for (int c = 0; c < kSfReplicas; ++c) xsf[so + 1024 * c] = (uint8_t)sfbyte;
+      for (int q = 0; q < 16; ++q) amax = fmaxf(amax, fabsf(v[q]));
+      const uint32_t sfbyte = f32x2_to_e4m3x2(0.f, amax / 6.0f) & 0xffu;
+      const float sf = e4m3_to_f32(sfbyte);
+      uint2 codes = make_uint2(0, 0);
+      if (sf > 0.f) {
+        uint32_t c[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) c[q] = f32x2_to_e2m1x2(v[2 * q + 1] / sf, v[2 * q] / sf);
+        codes.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
+        codes.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
+      }
+      *reinterpret_cast<uint2*>(xq + (size_t)t * (d / 2) + blk * 8) = codes;
+      xsf[(size_t)t * nblk + blk] = (uint8_t)sfbyte;
     }
   }
   pdl_launch_dependents();
 }
 
+__global__ void __launch_bounds__(256) gather_x_dense_kernel(
+    const uint8_t* __restrict__ xq_tok, const uint8_t* __restrict__ xsf_tok, const int4* __restrict__ dense,
+    const int* __restrict__ n_dense, const int* __restrict__ pad_total, const int* __restrict__ perm, int topk,
+    int d, uint8_t* __restrict__ xq, uint8_t* __restrict__ xsf) {
+  __shared__ int s_tok[128];                     // token of each row of the tile, -1 for padding
+  pdl_wait();
+  const int nd = *n_dense;
+  if (nd == 0) { pdl_launch_dependents(); return; }
+  const int ntile = *pad_total / 128;
+  const int n16 = d / 32;                        // 16-byte chunks of a code row
+  const int npairs = d / 128;                    // scale units per 128-row tile
+  for (int tile = blockIdx.x; tile < ntile; tile += gridDim.x) {
+    // a 128-row tile lies inside one expert: padding is to 256 rows
+    const int4 de = dense[dense_rank_of_padrow(dense, nd, tile * 128)];
+    const int i0 = tile * 128 - de.w;
+    if (i0 >= ((de.z + 127) & ~127)) continue;   // beyond the last 128-token tile: never read
+    __syncthreads();                             // s_tok of the previous tile consumed
+    if (threadIdx.x < 128) {
+      const int i = i0 + threadIdx.x;
+      s_tok[threadIdx.x] = i < de.z ? perm[de.y + i] / topk : -1;
+    }
+    __syncthreads();
+    // codes: one 16-byte chunk per thread and step, rows in order
+    for (int c = threadIdx.x; c < 128 * n16; c += blockDim.x) {
+      const int r = c / n16, ch = c - r * n16;
+      const int t = s_tok[r];
+      const uint4 v = t >= 0 ? reinterpret_cast<const uint4*>(xq_tok + (size_t)t * (d / 2))[ch]
+                             : make_uint4(0, 0, 0, 0);
+      reinterpret_cast<uint4*>(xq + (size_t)(tile * 128 + r) * (d / 2))[ch] = v;
+    }
+    // scales: 16-byte chunk q of unit p holds, for row slot l and 64-group
+    // 2p + h, the 4 scale bytes of rows l, l + 32, l + 64, l + 96 (see
+    // sf_pair_offset); consecutive threads write consecutive chunks
+    for (int c = threadIdx.x; c < npairs * 64; c += blockDim.x) {
+      const int pr = c >> 6, q = c & 63;
+      const int l = (q >> 4) * 8 + (q & 7), h = (q >> 3) & 1;
+      const int g = 2 * pr + h;                  // 64-wide K group
+      uint32_t w[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int t = s_tok[l + 32 * m];
+        w[m] = t >= 0 ? reinterpret_cast<const uint32_t*>(xsf_tok + (size_t)t * (d / 16))[g] : 0u;
+      }
+      const uint4 v = make_uint4(w[0], w[1], w[2], w[3]);
+      uint8_t* unit = xsf + ((size_t)tile * npairs + pr) * (1024 * kSfReplicas);
+#pragma unroll
+      for (int rep = 0; rep < kSfReplicas; ++rep) reinterpret_cast<uint4*>(unit + 1024 * rep)[q] = v;
+    }
+  }
+  pdl_launch_dependents();
+}
 
 // ---------------------------------------------------------------------------
 // Grouped block-scaled NVFP4 GEMM on tcgen05 (persistent, one block per SM).

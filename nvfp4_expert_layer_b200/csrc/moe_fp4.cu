@@ -56,6 +56,8 @@ struct Workspace {
   int* n_dense = nullptr;
   int* dense_ntoff = nullptr;    // [2][E+1]: 128-row and 256-row tile prefixes
   int* dense_pad_total = nullptr;
+  uint8_t* xq_tok = nullptr;     // dense class: NVFP4 x per token [T][d/2] and scales [T][d/16]
+  uint8_t* xsf_tok = nullptr;
   uint8_t* xq = nullptr;         // dense class: NVFP4 activations [pad_rows][d/2]
   uint8_t* xsf = nullptr;        //   and their scale atoms
   uint8_t* hq = nullptr;         // [pad_rows][f/2]
@@ -189,6 +191,8 @@ size_t workspace_bytes(const moe_fp4* h, int Tm) {
   add(((size_t)h->E + 1) * 8);                         // dense 128- and 256-row tile prefixes
   add(4);                                              // dense padded rows
   const size_t pr = dense_pad_rows(h, Tm);
+  add((size_t)Tm * h->d / 2);                          // xq_tok
+  add((size_t)Tm * h->d / 16);                         // xsf_tok
   add(pr * h->d / 2);                                  // xq
   add(moe::sf_pair_bytes(pr, h->d));                   // xsf
   add(pr * h->f / 2);                                  // hq
@@ -252,6 +256,8 @@ int ensure_workspace(moe_fp4* h, int Tm, cudaStream_t stream) {
   w.dense_ntoff = carve<int>(cur, 2 * (h->E + 1));
   w.dense_pad_total = carve<int>(cur, 1);
   w.pad_rows = dense_pad_rows(h, Tm);
+  w.xq_tok = carve<uint8_t>(cur, (size_t)Tm * h->d / 2);
+  w.xsf_tok = carve<uint8_t>(cur, (size_t)Tm * h->d / 16);
   w.xq = carve<uint8_t>(cur, w.pad_rows * h->d / 2);
   w.xsf = carve<uint8_t>(cur, moe::sf_pair_bytes(w.pad_rows, h->d));
   w.hq = carve<uint8_t>(cur, w.pad_rows * h->f / 2);
@@ -364,9 +370,11 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
   MOE_CUDA(mark(h, 3, st));
   // 4-5 (dense class). NVFP4 activations, then the two tensor-core GEMMs
   if (run_dense) {
-    MOE_CUDA(launch(moe::quant_x_dense_kernel, dim3(8 * h->sm_count), dim3(256), 0, st, pdl,
-                    xb, (const int4*)w.dense_list, (const int*)w.n_dense, (const int*)w.dense_pad_total,
-                    (const int*)w.perm, k, d, w.xq, w.xsf));
+    MOE_CUDA(launch(moe::quant_tok_kernel, dim3(std::min((T + 7) / 8, 8 * h->sm_count)), dim3(256), 0, st,
+                    pdl, xb, T, d, (const int*)w.n_dense, w.xq_tok, w.xsf_tok));
+    MOE_CUDA(launch(moe::gather_x_dense_kernel, dim3(8 * h->sm_count), dim3(256), 0, st, pdl,
+                    (const uint8_t*)w.xq_tok, (const uint8_t*)w.xsf_tok, (const int4*)w.dense_list,
+                    (const int*)w.n_dense, (const int*)w.dense_pad_total, (const int*)w.perm, k, d, w.xq, w.xsf));
     MOE_CUDA(mark(h, 4, st));
     moe::DenseParams dp{};
     dp.tmA = w.tm_x;           // tokens: the M side of the MMA
