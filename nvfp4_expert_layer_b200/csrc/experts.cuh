@@ -154,6 +154,16 @@ __device__ __forceinline__ void load_bfrag(BFrag<NT>& b, const __half* const (&r
     }
 }
 
+// {s, s} * 2^-8 as f16x2 for the non-negative e4m3 byte k of `four`, on the
+// integer pipes: the byte's 7 bits placed at f16 bit 7 give 2^(E-15) (1 + M/8)
+// for exponent field E >= 1 and 2^-14 M/8 for E = 0, i.e. exactly 2^-8 times
+// the e4m3 value in both cases (f16 subnormals cover the e4m3 subnormals).
+// The 2^-8 is undone on the fp32 accumulators.
+__device__ __forceinline__ uint32_t e4m3_dup_f16x2(uint32_t four, int k) {
+  return __byte_perm(four, 0u, 0x4440u + k) * 0x00800080u;
+}
+constexpr float kScaleUndo = 256.f;
+
 // One stage of shared-memory weights times the lane's activation fragments.
 template <int NT>
 __device__ __forceinline__ void mma_stage(uint32_t st, int nch, int lane, int g, const BFrag<NT>& b,
@@ -164,14 +174,12 @@ __device__ __forceinline__ void mma_stage(uint32_t st, int nch, int lane, int g,
       const uint4 codes = ld_shared_v4(st + ch * kChunkBytes + lane * 16);
       const uint2 sc = ld_shared_v2(st + ch * kChunkBytes + kChunkCodeBytes + g * 8);
       const uint32_t cw[4] = {codes.x, codes.y, codes.z, codes.w};
-      // scales: sc.x = row A(g) for K steps 0..3, sc.y = row B(g)
-      const uint32_t sa01 = e4m3x2_to_f16x2(sc.x & 0xffffu), sa23 = e4m3x2_to_f16x2(sc.x >> 16);
-      const uint32_t sb01 = e4m3x2_to_f16x2(sc.y & 0xffffu), sb23 = e4m3x2_to_f16x2(sc.y >> 16);
+      // scales: sc.x = row A(g) for K steps 0..3, sc.y = row B(g); non-negative
+      // e4m3 bytes (signs are folded into the codes), see e4m3_dup_f16x2
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
-        const uint32_t pa = ks < 2 ? sa01 : sa23, pb = ks < 2 ? sb01 : sb23;
-        const uint32_t sA = (ks & 1) ? dup_hi(pa) : dup_lo(pa);
-        const uint32_t sB = (ks & 1) ? dup_hi(pb) : dup_lo(pb);
+        const uint32_t sA = e4m3_dup_f16x2(sc.x, ks);
+        const uint32_t sB = e4m3_dup_f16x2(sc.y, ks);
         uint32_t a[4];
         e2m1x8_to_f16x2x4(cw[ks], a);
         a[0] = hmul2_u32(a[0], sA);
@@ -395,7 +403,7 @@ __global__ void __launch_bounds__(kExpThreads, 3) expert_kernel(ExpertParams p) 
         v[q] = sum;
       }
       if (!ti.down) {
-        const float gsg = p.gs[ti.e], gsu = p.gs[p.E + ti.e];
+        const float gsg = p.gs[ti.e] * kScaleUndo, gsu = p.gs[p.E + ti.e] * kScaleUndo;
         const int fidx = ti.t * 8 + g;
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
@@ -419,7 +427,7 @@ __global__ void __launch_bounds__(kExpThreads, 3) expert_kernel(ExpertParams p) 
           const int n = nt * 8 + 2 * c + q;
           if (n < ti.nrows) {
             const int r = ti.row0 + n;
-            const float wv = p.wts[p.perm[r]] * gsd;
+            const float wv = p.wts[p.perm[r]] * gsd * kScaleUndo;
             p.partial[(size_t)r * p.d + drow] = v[q] * wv;
             p.partial[(size_t)r * p.d + drow + 8] = v[2 + q] * wv;
           }

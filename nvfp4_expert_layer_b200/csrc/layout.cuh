@@ -10,9 +10,12 @@
 //                      byte 4ks+1: row B(g),  same K               (a2:a3)
 //                      byte 4ks+2: row A(g),  K = 16ks + 8 + 2c, +1 (a4:a5)
 //                      byte 4ks+3: row B(g),  same K               (a6:a7)
-//                    (low nibble = lower K, as in the canonical layout)
-//   bytes [512, 576) 8 groups g x 8 B of e4m3 scales: bytes 0..3 = scales of
-//                    row A(g) for steps ks = 0..3, bytes 4..7 = row B(g).
+//                    (low nibble = lower K, as in the canonical layout; the
+//                    codes of a block whose scale is negative have their
+//                    signs flipped, which is exact)
+//   bytes [512, 576) 8 groups g x 8 B of e4m3 scales with the sign bit
+//                    cleared: bytes 0..3 = scales of row A(g) for steps
+//                    ks = 0..3, bytes 4..7 = row B(g).
 // Tile rows: gate/up tile t pairs gate rows f = 8t+g (A) with up rows 8t+g
 // (B), so one MMA accumulator holds g and u of the same f; down tile t holds
 // rows 16t+g (A) and 16t+8+g (B).

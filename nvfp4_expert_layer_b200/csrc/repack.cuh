@@ -45,13 +45,18 @@ __global__ void repack_fragment_kernel(const uint8_t* __restrict__ qa, const uin
     const uint8_t* ra = qA + (mat + rowA) * (K / 2);
     const uint8_t* rb = qB + (mat + rowB) * (K / 2);
     uint8_t* dst = out + ((size_t)((size_t)e * tpe + t) * cpt + ch) * kChunkBytes;
+    const uint8_t* fa = sA + (mat + rowA) * (K / 16);
+    const uint8_t* fb = sB + (mat + rowB) * (K / 16);
     uint8_t b[16];
     for (int ks = 0; ks < 4; ++ks) {
       const int k0 = ch * kChunkK + ks * 16;
-      b[4 * ks + 0] = ra[k0 / 2 + c];
-      b[4 * ks + 1] = rb[k0 / 2 + c];
-      b[4 * ks + 2] = ra[(k0 + 8) / 2 + c];
-      b[4 * ks + 3] = rb[(k0 + 8) / 2 + c];
+      // a negative block scale is folded into its codes (sign flip, exact)
+      const uint8_t xa = (fa[ch * 4 + ks] & 0x80u) ? 0x88u : 0u;
+      const uint8_t xb = (fb[ch * 4 + ks] & 0x80u) ? 0x88u : 0u;
+      b[4 * ks + 0] = ra[k0 / 2 + c] ^ xa;
+      b[4 * ks + 1] = rb[k0 / 2 + c] ^ xb;
+      b[4 * ks + 2] = ra[(k0 + 8) / 2 + c] ^ xa;
+      b[4 * ks + 3] = rb[(k0 + 8) / 2 + c] ^ xb;
     }
     uint4 v;
     v.x = b[0] | (b[1] << 8) | (b[2] << 16) | ((uint32_t)b[3] << 24);
@@ -60,11 +65,9 @@ __global__ void repack_fragment_kernel(const uint8_t* __restrict__ qa, const uin
     v.w = b[12] | (b[13] << 8) | (b[14] << 16) | ((uint32_t)b[15] << 24);
     *reinterpret_cast<uint4*>(dst + lane * 16) = v;
     if (c == 0) {
-      const uint8_t* fa = sA + (mat + rowA) * (K / 16);
-      const uint8_t* fb = sB + (mat + rowB) * (K / 16);
       for (int ks = 0; ks < 4; ++ks) {
-        dst[kChunkCodeBytes + g * 8 + ks] = fa[ch * 4 + ks];
-        dst[kChunkCodeBytes + g * 8 + 4 + ks] = fb[ch * 4 + ks];
+        dst[kChunkCodeBytes + g * 8 + ks] = fa[ch * 4 + ks] & 0x7Fu;
+        dst[kChunkCodeBytes + g * 8 + 4 + ks] = fb[ch * 4 + ks] & 0x7Fu;
       }
     }
   }
