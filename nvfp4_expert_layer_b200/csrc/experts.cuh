@@ -110,14 +110,18 @@ struct TileInfo {
   const uint8_t* base;
 };
 
+// RT = 16-row tiles of the fragment layout per work tile (consecutive tiles
+// t, t + 1 of one expert matrix); ti.t is the first of them.
+template <int RT>
 __device__ __forceinline__ TileInfo tile_info(const ExpertParams& p, const int4* jobs, int i, int ngu,
                                               int warp) {
   TileInfo ti;
   ti.down = i >= ngu;
   const int tpe = ti.down ? p.tpe_dn : p.tpe_gu;
+  const int wtpe = tpe / RT;
   const int li = ti.down ? i - ngu : i;
-  ti.job = li / tpe;
-  ti.t = li - ti.job * tpe;
+  ti.job = li / wtpe;
+  ti.t = (li - ti.job * wtpe) * RT;
   const int4 jb = jobs[ti.job];
   ti.e = jb.x;
   ti.row0 = jb.y;
@@ -165,14 +169,17 @@ __device__ __forceinline__ uint32_t e4m3_dup_f16x2(uint32_t four, int k) {
 constexpr float kScaleUndo = 256.f;
 
 // One stage of shared-memory weights times the lane's activation fragments.
-template <int NT>
+template <int NT, int RT>
 __device__ __forceinline__ void mma_stage(uint32_t st, int nch, int lane, int g, const BFrag<NT>& b,
-                                          int nrows, float (&acc)[4][NT][4]) {
+                                          int nrows, float (&acc)[RT][4][NT][4]) {
 #pragma unroll
   for (int ch = 0; ch < kExpSC; ++ch) {
+#pragma unroll
+    for (int rt = 0; rt < RT; ++rt)
     if (ch < nch) {
-      const uint4 codes = ld_shared_v4(st + ch * kChunkBytes + lane * 16);
-      const uint2 sc = ld_shared_v2(st + ch * kChunkBytes + kChunkCodeBytes + g * 8);
+      const uint32_t sr = st + rt * kExpSB;
+      const uint4 codes = ld_shared_v4(sr + ch * kChunkBytes + lane * 16);
+      const uint2 sc = ld_shared_v2(sr + ch * kChunkBytes + kChunkCodeBytes + g * 8);
       const uint32_t cw[4] = {codes.x, codes.y, codes.z, codes.w};
       // scales: sc.x = row A(g) for K steps 0..3, sc.y = row B(g); non-negative
       // e4m3 bytes (signs are folded into the codes), see e4m3_dup_f16x2
@@ -192,7 +199,7 @@ __device__ __forceinline__ void mma_stage(uint32_t st, int nch, int lane, int g,
           const uint4& hi = b.v[nt][ch][1];
           const uint32_t b0 = ks == 0 ? lo.x : ks == 1 ? lo.z : ks == 2 ? hi.x : hi.z;
           const uint32_t b1 = ks == 0 ? lo.y : ks == 1 ? lo.w : ks == 2 ? hi.y : hi.w;
-          if (NT == 1 || nt * 8 < nrows) mma_16816_f16(acc[ks][nt], a, b0, b1);
+          if (NT == 1 || nt * 8 < nrows) mma_16816_f16(acc[rt][ks][nt], a, b0, b1);
         }
       }
     }
@@ -202,11 +209,16 @@ __device__ __forceinline__ void mma_stage(uint32_t st, int nch, int lane, int g,
 
 // NT = 8-wide n-tiles per job: expert_kernel<1> runs jobs of <= 8 rows,
 // expert_kernel<2> jobs of 9..16 rows; each has its own job list and counters.
+// With one n-tile a work tile is two 16-row tiles (RT = 2) that share the
+// activation fragments, the loop control and the epilogue barrier.
 template <int NT>
 __global__ void __launch_bounds__(kExpThreads, 3) expert_kernel(ExpertParams p) {
+  constexpr int RT = NT == 1 ? 2 : 1;
+  constexpr int RING = kExpRing / RT;          // stages in flight per warp (same bytes)
+  constexpr int SLOT = RT * kExpSB;
   extern __shared__ __align__(128) uint8_t smem[];
-  uint64_t* bars_all = reinterpret_cast<uint64_t*>(smem + kExpWarps * kExpRing * kExpSB);
-  float* red_all = reinterpret_cast<float*>(bars_all + kExpWarps * kExpRing);   // [2][4][2][32][4]
+  uint64_t* bars_all = reinterpret_cast<uint64_t*>(smem + kExpWarps * RING * SLOT);
+  float* red_all = reinterpret_cast<float*>(bars_all + kExpWarps * RING);   // [2][4][2][32][4]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
@@ -214,8 +226,8 @@ __global__ void __launch_bounds__(kExpThreads, 3) expert_kernel(ExpertParams p) 
 
   pdl_wait();                                   // routing results of the previous kernel
   const int njobs = *p.njobs;
-  const int ngu = njobs * p.tpe_gu;
-  const int ntot = ngu + njobs * p.tpe_dn;
+  const int ngu = njobs * (p.tpe_gu / RT);
+  const int ntot = ngu + njobs * (p.tpe_dn / RT);
   const int my_tiles = b < ntot ? (ntot - 1 - b) / G + 1 : 0;
   const uint64_t deadline = globaltimer_ns() + (uint64_t)p.wait_timeout_ns;
   __shared__ int4 s_jobs[kExpSmemJobs];
@@ -226,11 +238,11 @@ __global__ void __launch_bounds__(kExpThreads, 3) expert_kernel(ExpertParams p) 
   }
   __syncthreads();
 
-  const uint32_t ring_s = smem_u32(smem + warp * kExpRing * kExpSB);
-  const uint32_t bars_s = smem_u32(bars_all + warp * kExpRing);
+  const uint32_t ring_s = smem_u32(smem + warp * RING * SLOT);
+  const uint32_t bars_s = smem_u32(bars_all + warp * RING);
   const uint64_t pol = policy_evict_first();
   if (lane == 0) {
-    for (int i = 0; i < kExpRing; ++i) mbar_init(bars_s + 8 * i, 1);
+    for (int i = 0; i < RING; ++i) mbar_init(bars_s + 8 * i, 1);
     fence_mbar_init();
   }
   __syncwarp();
@@ -243,7 +255,7 @@ __global__ void __launch_bounds__(kExpThreads, 3) expert_kernel(ExpertParams p) 
     while (true) {
       if (!c_valid) {
         if (c_it >= my_tiles) return false;
-        c_ti = tile_info(p, jobs, b + c_it * G, ngu, warp);
+        c_ti = tile_info<RT>(p, jobs, b + c_it * G, ngu, warp);
         c_s = 0;
         c_valid = true;
       }
@@ -252,14 +264,17 @@ __global__ void __launch_bounds__(kExpThreads, 3) expert_kernel(ExpertParams p) 
       ++c_it;
     }
   };
-  auto produce = [&](int consumed) {          // keep kExpRing stages in flight
-    while (issued < consumed + kExpRing && cursor_ready()) {
+  auto produce = [&](int consumed) {          // keep RING stages in flight
+    while (issued < consumed + RING && cursor_ready()) {
       const int s = c_ti.slo + c_s;
       const int nch = min(kExpSC, c_ti.cpt - kExpSC * s);
-      const int slot = issued % kExpRing;
-      mbar_arrive_expect_tx(bars_s + 8 * slot, nch * kChunkBytes);
-      bulk_g2s(ring_s + slot * kExpSB, c_ti.base + (size_t)kExpSC * s * kChunkBytes, nch * kChunkBytes,
-               bars_s + 8 * slot, pol);
+      const int slot = issued % RING;
+      mbar_arrive_expect_tx(bars_s + 8 * slot, RT * nch * kChunkBytes);
+#pragma unroll
+      for (int rt = 0; rt < RT; ++rt)
+        bulk_g2s(ring_s + slot * SLOT + rt * kExpSB,
+                 c_ti.base + ((size_t)rt * c_ti.cpt + (size_t)kExpSC * s) * kChunkBytes, nch * kChunkBytes,
+                 bars_s + 8 * slot, pol);
       ++c_s;
       ++issued;
     }
@@ -286,7 +301,7 @@ __global__ void __launch_bounds__(kExpThreads, 3) expert_kernel(ExpertParams p) 
   TileInfo ti_next{};
   const __half* row_next[2] = {nullptr, nullptr};
   if (my_tiles > 0) {
-    ti_next = tile_info(p, jobs, b, ngu, warp);
+    ti_next = tile_info<RT>(p, jobs, b, ngu, warp);
     tile_rows(ti_next, row_next);
   }
 
@@ -295,7 +310,7 @@ __global__ void __launch_bounds__(kExpThreads, 3) expert_kernel(ExpertParams p) 
     const int nt_used = (ti.nrows + 7) >> 3;
     const __half* row[2] = {row_next[0], row_next[1]};
     if (it + 1 < my_tiles) {
-      ti_next = tile_info(p, jobs, b + (it + 1) * G, ngu, warp);
+      ti_next = tile_info<RT>(p, jobs, b + (it + 1) * G, ngu, warp);
       tile_rows(ti_next, row_next);
     }
     if (ti.down && ti.nw > 0 && !failed) {      // h of this job must be complete
@@ -315,14 +330,16 @@ __global__ void __launch_bounds__(kExpThreads, 3) expert_kernel(ExpertParams p) 
       }
     }
 
-    float part[2][4];                    // this warp's partial sums of the tile, per n-tile
+    float part[2][4];                    // this warp's partial sums, per unit u = rt * NT + nt
     if constexpr (NT == 1) {
-      // one n-tile: activation fragments double-buffered one stage ahead
-      float acc[4][1][4];
+      // one n-tile, two row tiles: activation fragments double-buffered one stage ahead
+      float acc[RT][4][1][4];
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+      for (int rt = 0; rt < RT; ++rt)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) acc[a][0][q] = 0.f;
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc[rt][a][0][q] = 0.f;
       auto load1 = [&](BFrag<1>& bf, int s) {
         const int n1 = min(kExpSC, ti.cpt - kExpSC * s);
         if (ti.down) load_bfrag<1, true>(bf, row, kExpSC * s, n1, c);
@@ -330,12 +347,12 @@ __global__ void __launch_bounds__(kExpThreads, 3) expert_kernel(ExpertParams p) 
       };
       auto step1 = [&](const BFrag<1>& bf, int s) {
         const int nch = min(kExpSC, ti.cpt - kExpSC * s);
-        const int slot = consumed % kExpRing;
-        if (!failed && !mbar_wait_until(bars_s + 8 * slot, (consumed / kExpRing) & 1, deadline)) {
+        const int slot = consumed % RING;
+        if (!failed && !mbar_wait_until(bars_s + 8 * slot, (consumed / RING) & 1, deadline)) {
           failed = true;
           set_error(p.err, kErrTimeout);
         }
-        if (!failed) mma_stage<1>(ring_s + slot * kExpSB, nch, lane, g, bf, ti.nrows, acc);
+        if (!failed) mma_stage<1, RT>(ring_s + slot * SLOT, nch, lane, g, bf, ti.nrows, acc);
         __syncwarp();
         ++consumed;
         if (lane == 0 && !failed) produce(consumed);
@@ -350,29 +367,29 @@ __global__ void __launch_bounds__(kExpThreads, 3) expert_kernel(ExpertParams p) 
       }
       if (ss < ti.nw) step1(b1cur, ti.slo + ss);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        part[0][q] = (acc[0][0][q] + acc[1][0][q]) + (acc[2][0][q] + acc[3][0][q]);
-        part[1][q] = 0.f;
-      }
+      for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          part[rt][q] = (acc[rt][0][0][q] + acc[rt][1][0][q]) + (acc[rt][2][0][q] + acc[rt][3][0][q]);
     } else {
-      float acc[4][2][4];
+      float acc[1][4][2][4];
 #pragma unroll
       for (int a = 0; a < 4; ++a)
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-          for (int q = 0; q < 4; ++q) acc[a][nt][q] = 0.f;
+          for (int q = 0; q < 4; ++q) acc[0][a][nt][q] = 0.f;
       for (int ss = 0; ss < ti.nw; ++ss) {
         const int s = ti.slo + ss;
         const int nch = min(kExpSC, ti.cpt - kExpSC * s);
         if (ti.down) load_bfrag<2, true>(b2, row, kExpSC * s, nch, c);
         else load_bfrag<2, false>(b2, row, kExpSC * s, nch, c);
-        const int slot = consumed % kExpRing;
-        if (!failed && !mbar_wait_until(bars_s + 8 * slot, (consumed / kExpRing) & 1, deadline)) {
+        const int slot = consumed % RING;
+        if (!failed && !mbar_wait_until(bars_s + 8 * slot, (consumed / RING) & 1, deadline)) {
           failed = true;
           set_error(p.err, kErrTimeout);
         }
-        if (!failed) mma_stage<2>(ring_s + slot * kExpSB, nch, lane, g, b2, ti.nrows, acc);
+        if (!failed) mma_stage<2, 1>(ring_s + slot * SLOT, nch, lane, g, b2, ti.nrows, acc);
         __syncwarp();
         ++consumed;
         if (lane == 0 && !failed) produce(consumed);
@@ -381,7 +398,7 @@ __global__ void __launch_bounds__(kExpThreads, 3) expert_kernel(ExpertParams p) 
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          part[nt][q] = (acc[0][nt][q] + acc[1][nt][q]) + (acc[2][nt][q] + acc[3][nt][q]);
+          part[nt][q] = (acc[0][0][nt][q] + acc[0][1][nt][q]) + (acc[0][2][nt][q] + acc[0][3][nt][q]);
     }
 
     // ---- cross-warp reduction of the tile (buffer alternates by tile parity)
@@ -392,19 +409,22 @@ __global__ void __launch_bounds__(kExpThreads, 3) expert_kernel(ExpertParams p) 
       for (int q = 0; q < 4; ++q)
         red[((warp * 2 + nt) * 32 + lane) * 4 + q] = part[nt][q];
     __syncthreads();
-    if (warp < nt_used) {
-      const int nt = warp;
+    const int units_used = RT * nt_used;
+    if (warp < units_used) {
+      const int nt = NT == 1 ? 0 : warp;           // unit u = warp: row tile rt, n-tile nt
+      const int rt = NT == 1 ? warp : 0;
+      const int red_u = warp;
       float v[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         float sum = 0.f;
 #pragma unroll
-        for (int w = 0; w < kExpWarps; ++w) sum += red[((w * 2 + nt) * 32 + lane) * 4 + q];
+        for (int w = 0; w < kExpWarps; ++w) sum += red[((w * 2 + red_u) * 32 + lane) * 4 + q];
         v[q] = sum;
       }
       if (!ti.down) {
         const float gsg = p.gs[ti.e] * kScaleUndo, gsu = p.gs[p.E + ti.e] * kScaleUndo;
-        const int fidx = ti.t * 8 + g;
+        const int fidx = (ti.t + rt) * 8 + g;
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           const int n = nt * 8 + 2 * c + q;
@@ -421,7 +441,7 @@ __global__ void __launch_bounds__(kExpThreads, 3) expert_kernel(ExpertParams p) 
         }
       } else {
         const float gsd = p.gs[2 * p.E + ti.e];
-        const int drow = ti.t * 16 + g;
+        const int drow = (ti.t + rt) * 16 + g;
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           const int n = nt * 8 + 2 * c + q;
@@ -433,7 +453,7 @@ __global__ void __launch_bounds__(kExpThreads, 3) expert_kernel(ExpertParams p) 
           }
         }
       }
-      // publish this n-tile of a gate/up tile (release, no round trip)
+      // publish this (row tile, n-tile) of a gate/up work tile (release, no round trip)
       __syncwarp();
       if (!ti.down && lane == 0) red_release_add(p.gu_done + ti.job, 1);
     }
@@ -444,7 +464,7 @@ __global__ void __launch_bounds__(kExpThreads, 3) expert_kernel(ExpertParams p) 
   if (failed && lane == 0) {
     const uint64_t drain = globaltimer_ns() + (uint64_t)p.wait_timeout_ns;
     for (int jj = consumed; jj < issued; ++jj)
-      if (!mbar_wait_until(bars_s + 8 * (jj % kExpRing), (jj / kExpRing) & 1, drain)) break;
+      if (!mbar_wait_until(bars_s + 8 * (jj % RING), (jj / RING) & 1, drain)) break;
   }
   // ---- exit protocol: the last block clears the per-job counters
   __syncthreads();
