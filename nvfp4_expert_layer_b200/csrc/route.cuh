@@ -141,21 +141,32 @@ __global__ void __launch_bounds__(256) router_tiled_kernel(
 // ---------------------------------------------------------------------------
 // Warp top-k over v[i] = logit of expert lane + 32 i (-inf beyond E).
 // Lane j < k receives the j-th selected expert and its renormalised weight.
-__device__ __forceinline__ void topk_warp(const float (&v)[32], int E, int k, int lane, int& my_e,
-                                          float& my_w) {
-  const int per = (E + 31) / 32;
+// PER = logits per lane rounded up to a power of two.  Each lane keeps its
+// best untaken (logit, expert); a round takes the warp arg-max and only the
+// winning lane rescans its PER values.  Within a lane experts increase with
+// i, so a strict comparison keeps the lower expert on ties.
+template <int PER>
+__device__ __forceinline__ void topk_warp_t(const float (&v)[32], int E, int k, int lane, int& my_e,
+                                            float& my_w) {
   float sel_l0 = 0.f, sum = 0.f, my_p = 0.f;
   my_e = 0;
   unsigned taken = 0u;            // bit i: element lane + 32 i already selected
-  for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
+  float lv = -INFINITY;
+  int le = 0x7fffffff;
+  auto lane_best = [&]() {
+    lv = -INFINITY;
+    le = 0x7fffffff;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int i = 0; i < PER; ++i) {
       const int e = lane + 32 * i;
-      const bool cand = i < per && e < E && !((taken >> i) & 1u);
-      if (cand && (be == 0x7fffffff || v[i] > bv || (v[i] == bv && e < be))) { bv = v[i]; be = e; }
+      const bool cand = e < E && !((taken >> i) & 1u);
+      if (cand && (le == 0x7fffffff || v[i] > lv)) { lv = v[i]; le = e; }
     }
+  };
+  lane_best();
+  for (int j = 0; j < k; ++j) {
+    float bv = lv;
+    int be = le;
     for (int o = 16; o > 0; o >>= 1) {
       const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
       const int oe = __shfl_xor_sync(0xffffffffu, be, o);
@@ -164,13 +175,27 @@ __device__ __forceinline__ void topk_warp(const float (&v)[32], int E, int k, in
       if (better) { bv = ov; be = oe; }
     }
     if (be == 0x7fffffff) be = 0;       // unreachable for k <= E
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    if ((be & 31) == lane) {
+      taken |= 1u << (be >> 5);
+      lane_best();
+    }
     if (j == 0) sel_l0 = bv;
     const float p = expf(bv - sel_l0);
     sum += p;
     if (lane == j) { my_p = p; my_e = be; }
   }
   my_w = my_p / sum;
+}
+
+__device__ __forceinline__ void topk_warp(const float (&v)[32], int E, int k, int lane, int& my_e,
+                                          float& my_w) {
+  const int per = (E + 31) / 32;
+  if (per <= 1) topk_warp_t<1>(v, E, k, lane, my_e, my_w);
+  else if (per <= 2) topk_warp_t<2>(v, E, k, lane, my_e, my_w);
+  else if (per <= 4) topk_warp_t<4>(v, E, k, lane, my_e, my_w);
+  else if (per <= 8) topk_warp_t<8>(v, E, k, lane, my_e, my_w);
+  else if (per <= 16) topk_warp_t<16>(v, E, k, lane, my_e, my_w);
+  else topk_warp_t<32>(v, E, k, lane, my_e, my_w);
 }
 
 // Top-k for large T: one warp per token over the full logits.
@@ -238,6 +263,52 @@ __device__ void build_permutation(const int* ids, int T, int k, int E, int thr, 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const long long P = (long long)T * k;
   const long long c0 = P * warp / 32, c1 = P * (warp + 1) / 32;
+  if (P <= 32) {
+    // Small batches (decode): one warp ranks the <= 32 pairs by (expert, pair);
+    // every thread derives count and offset of its experts from the pair list.
+    int* pe = wc;                                   // [32] expert of each pair, -1 if none
+    if (threadIdx.x < 32) {
+      const int e = threadIdx.x < P ? ids[threadIdx.x] : -1;
+      pe[threadIdx.x] = (e >= 0 && e < E) ? e : -1;
+    }
+    if (threadIdx.x < 8) misc[threadIdx.x] = 0;
+    __syncthreads();
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+      int cn = 0, before = 0;
+      for (int q = 0; q < (int)P; ++q) {
+        const int pq = pe[q];
+        cn += pq == e;
+        before += pq >= 0 && pq < e;
+      }
+      if (e < E) { cnt[e] = cn; o.counts[e] = cn; }
+      off[e] = before;
+      o.offsets[e] = before;
+    }
+    if (warp == 0) {
+      const int e = pe[lane];
+      const bool ok = e >= 0;
+      int rank = 0, arank = 0;
+      bool first = ok;
+      for (int m = 0; m < 32; ++m) {
+        const int em = pe[m];
+        rank += em >= 0 && (em < e || (em == e && m < lane));
+        if (m < lane && em == e) first = false;
+      }
+      for (int m = 0; m < 32; ++m) {
+        const bool fm = __shfl_sync(0xffffffffu, first, m);
+        const int em = __shfl_sync(0xffffffffu, e, m);
+        arank += fm && em < e;
+      }
+      if (ok) {
+        o.perm[rank] = lane;
+        o.inv[lane] = rank;
+      }
+      if (first) act[arank] = e;
+      const int A = __popc(__ballot_sync(0xffffffffu, first));
+      if (lane == 0) misc[0] = A;
+    }
+    __syncthreads();
+  } else {
   for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) wc[i] = 0;
   if (threadIdx.x < 8) misc[threadIdx.x] = 0;
   __syncthreads();
@@ -301,6 +372,7 @@ __device__ void build_permutation(const int* ids, int T, int k, int E, int thr, 
     __syncwarp();
     if (ok && lane == __ffs(mask) - 1) wc[warp * E + e] += __popc(mask);
     __syncwarp();
+  }
   }
   // expert classes over the active experts only
   const int A = misc[0];
