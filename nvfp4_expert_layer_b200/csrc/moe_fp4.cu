@@ -453,8 +453,10 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
   ep2.jobs = w.jobs2; ep2.njobs = w.n_jobs2; ep2.gu_done = gu_done2; ep2.exit_cnt = exit2;
   MOE_CUDA(launch(moe::expert_kernel<1>, dim3(h->sm_count * h->exp_bps1), dim3(moe::kExpThreads),
                   kExpSmem, st, pdl, ep1));
-  MOE_CUDA(launch(moe::expert_kernel<2>, dim3(h->sm_count * h->exp_bps2), dim3(moe::kExpThreads),
-                  kExpSmem, st, pdl, ep2));
+  // jobs of 9..16 rows need an expert with at least 9 rows, i.e. T >= 9
+  if (T >= 9)
+    MOE_CUDA(launch(moe::expert_kernel<2>, dim3(h->sm_count * h->exp_bps2), dim3(moe::kExpThreads),
+                    kExpSmem, st, pdl, ep2));
   MOE_CUDA(mark(h, 7, st));
   // 7. combine / unpermute: out[t] = bf16(sum_j partial[inv[t,j]])
   MOE_CUDA(launch(moe::combine_kernel, dim3((d + 1023) / 1024, T), dim3(128), 0, st, pdl,
