@@ -384,10 +384,10 @@ def run_native(args, rank, world, local):
     torch.cuda.synchronize()
     gpu_out0 = out.view(torch.int16).cpu().numpy().view(np.uint16).copy()
     # kernels per step: routing (1 fused launch up to 256 tokens, else the
-    # weight split, router, x staging, top-k, permutation), the dense class
+    # weight split, router, x staging, top-k, 3 permutation kernels), the dense class
     # (quantiser, gather, 2 GEMMs) when T >= thr, the light-class expert
     # kernels (the 9..16-row one only when T >= 9) and the combine
-    launches = (1 if cfg.T <= 256 else 5) + (4 if cfg.T >= 128 else 0) + (2 if cfg.T >= 9 else 1) + 1
+    launches = (1 if cfg.T <= 256 else 7) + (4 if cfg.T >= 128 else 0) + (2 if cfg.T >= 9 else 1) + 1
     return dict(cfg=cfg, ms=ms, clk=clk, err=err, stage_ms=stage_ms, dom_ms=dom_ms / n,
                 dom_work=dom_work / n, dense=dense, e2e_ms=e2e_ms, xs_np=xs_np, rw_np=rw_np,
                 gpu_out0=gpu_out0, launches_per_step=launches, stages=layer.STAGES,

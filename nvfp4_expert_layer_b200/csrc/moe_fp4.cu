@@ -34,6 +34,7 @@ constexpr int kSmallT = 256;          // fused routing kernel up to this many to
 constexpr size_t kExpSmem = moe::expert_smem_size();
 constexpr int kDenseGridPerSm = 1;
 constexpr int kStageEvents = 9;
+constexpr int kPermMaxBlocks = 296;       // blocks of the large-batch permutation
 
 struct Workspace {
   void* base = nullptr;
@@ -55,6 +56,7 @@ struct Workspace {
   int4* dense_list = nullptr;
   int* n_dense = nullptr;
   int* dense_ntoff = nullptr;    // [2][E+1]: 128-row and 256-row tile prefixes
+  int* perm_bcnt = nullptr;      // [kPermMaxBlocks][E] per-block expert counts / bases
   int* dense_pad_total = nullptr;
   uint8_t* xq_tok = nullptr;     // dense class: NVFP4 x per token [T][d/2] and scales [T][d/16]
   uint8_t* xsf_tok = nullptr;
@@ -189,6 +191,7 @@ size_t workspace_bytes(const moe_fp4* h, int Tm) {
   add(4);
   add(counter_ints(h, Tm) * 4);                        // counters
   add(((size_t)h->E + 1) * 8);                         // dense 128- and 256-row tile prefixes
+  add((size_t)kPermMaxBlocks * h->E * 4);              // permutation block counts
   add(4);                                              // dense padded rows
   const size_t pr = dense_pad_rows(h, Tm);
   add((size_t)Tm * h->d / 2);                          // xq_tok
@@ -254,6 +257,7 @@ int ensure_workspace(moe_fp4* h, int Tm, cudaStream_t stream) {
   w.xin = carve<uint16_t>(cur, (size_t)Tm * h->d);
   w.xout = carve<uint16_t>(cur, (size_t)Tm * h->d);
   w.dense_ntoff = carve<int>(cur, 2 * (h->E + 1));
+  w.perm_bcnt = carve<int>(cur, (size_t)kPermMaxBlocks * h->E);
   w.dense_pad_total = carve<int>(cur, 1);
   w.pad_rows = dense_pad_rows(h, Tm);
   w.xq_tok = carve<uint8_t>(cur, (size_t)Tm * h->d / 2);
@@ -364,8 +368,15 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
     MOE_CUDA(launch(moe::topk_kernel, dim3((T + 7) / 8), dim3(256), 0, st, false,
                     (const float*)w.logits, T, E, k, w.ids, w.wts));
     MOE_CUDA(mark(h, 2, st));
-    MOE_CUDA(launch(moe::permute_kernel, dim3(1), dim3(1024), permute_smem_bytes(E), st, false,
-                    (const int*)w.ids, T, k, E, thr, dense_ok, po));
+    // 3. permutation: per-block counts, one-block scan and classes, placement
+    const long long P = (long long)T * k;
+    const int nb = (int)std::min<long long>(kPermMaxBlocks, std::max<long long>(1, (P + 1023) / 1024));
+    MOE_CUDA(launch(moe::perm_hist_kernel, dim3(nb), dim3(1024), (size_t)E * 4, st, false,
+                    (const int*)w.ids, P, E, w.perm_bcnt));
+    MOE_CUDA(launch(moe::perm_scan_kernel, dim3(1), dim3(1024), permute_smem_bytes(E), st, false,
+                    w.perm_bcnt, nb, E, thr, dense_ok, po));
+    MOE_CUDA(launch(moe::perm_place_kernel, dim3(nb), dim3(1024), (size_t)32 * E * 4, st, false,
+                    (const int*)w.ids, P, E, (const int*)w.perm_bcnt, po));
   }
   MOE_CUDA(mark(h, 3, st));
   // 4-5 (dense class). NVFP4 activations, then the two tensor-core GEMMs
@@ -528,7 +539,8 @@ int moe_fp4_create(int E, int top_k, int d, int f, moe_fp4_t** out) {
     };
     if (smem_attr((const void*)moe::expert_kernel<1>, kExpSmem) != cudaSuccess ||
         smem_attr((const void*)moe::expert_kernel<2>, kExpSmem) != cudaSuccess ||
-        smem_attr((const void*)moe::permute_kernel, permute_smem_bytes(E)) != cudaSuccess ||
+        smem_attr((const void*)moe::perm_scan_kernel, permute_smem_bytes(E)) != cudaSuccess ||
+        smem_attr((const void*)moe::perm_place_kernel, (size_t)32 * E * 4) != cudaSuccess ||
         smem_attr((const void*)moe::route_kernel, route_smem_bytes(E, d, kSmallT * top_k)) != cudaSuccess ||
         smem_attr((const void*)moe::dense_gemm_kernel<moe::kDenseGateUp>,
                   moe::dense_smem_size<moe::kDenseGateUp>(E)) != cudaSuccess ||

@@ -253,6 +253,65 @@ struct PermuteOut {
 
 __host__ __device__ constexpr size_t permute_smem_ints(int E) { return (size_t)36 * E + 1 + 8; }
 
+// Expert classes over the active experts (light jobs, dense list) from the
+// counts, offsets and active list in shared memory (layout of
+// build_permutation); writes the job lists, the dense list and the scalars.
+__device__ void perm_classes(int E, int thr, int dense_supported, const PermuteOut& o, int* sm) {
+  int* cnt = sm + 32 * E;
+  int* off = cnt + E;
+  int* act = off + E + 1;
+  int* misc = act + E;
+  // expert classes over the active experts only
+  const int A = misc[0];
+  for (int a = threadIdx.x; a < A; a += blockDim.x) {
+    const int e = act[a];
+    const int n = cnt[e];
+    const bool light = n < thr;
+    int rank = 0, s1 = 0, s2 = 0, pad0 = 0, nt0 = 0, nt1 = 0;
+    for (int b = 0; b < A; ++b) {
+      const int e2 = act[b], n2 = cnt[e2];
+      if ((n2 < thr) != light) continue;
+      if (n2 > n || (n2 == n && e2 < e)) {
+        ++rank;
+        const int r2 = n2 % kJobRows;
+        s1 += (r2 > 0 && r2 <= 8) ? 1 : 0;
+        s2 += n2 / kJobRows + (r2 > 8 ? 1 : 0);
+        pad0 += (n2 + 255) & ~255;
+        nt0 += (n2 + 127) >> 7;
+        nt1 += (n2 + 255) >> 8;
+      }
+    }
+    if (light) {
+      for (int r0 = 0; r0 < n; r0 += kJobRows) {
+        const int nr = min(kJobRows, n - r0);
+        const int4 jb = make_int4(e, off[e] + r0, nr, 0);
+        if (nr <= 8) o.jobs1[s1] = jb; else o.jobs2[s2++] = jb;
+      }
+      const int r = n % kJobRows;
+      atomicAdd(&misc[1], (r > 0 && r <= 8) ? 1 : 0);
+      atomicAdd(&misc[2], n / kJobRows + (r > 8 ? 1 : 0));
+    } else {
+      o.dense_list[rank] = make_int4(e, off[e], n, pad0);
+      o.dense_ntoff[rank] = nt0;
+      o.dense_ntoff[E + 1 + rank] = nt1;
+      atomicAdd(&misc[3], 1);
+      atomicAdd(&misc[4], (n + 127) >> 7);
+      atomicAdd(&misc[5], (n + 255) & ~255);
+      atomicAdd(&misc[6], (n + 255) >> 8);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    *o.n_jobs1 = misc[1];
+    *o.n_jobs2 = misc[2];
+    *o.n_dense = misc[3];
+    o.dense_ntoff[misc[3]] = misc[4];
+    o.dense_ntoff[E + 1 + misc[3]] = misc[6];
+    *o.dense_pad_total = misc[5];
+    if (misc[3] > 0 && !dense_supported) set_error(o.err, kErrUnsupported);
+  }
+}
+
 __device__ void build_permutation(const int* ids, int T, int k, int E, int thr, int dense_supported,
                                   const PermuteOut& o, int* sm) {
   int* wc = sm;                 // [32][E]
@@ -374,62 +433,125 @@ __device__ void build_permutation(const int* ids, int T, int k, int E, int thr, 
     __syncwarp();
   }
   }
-  // expert classes over the active experts only
-  const int A = misc[0];
-  for (int a = threadIdx.x; a < A; a += blockDim.x) {
-    const int e = act[a];
-    const int n = cnt[e];
-    const bool light = n < thr;
-    int rank = 0, s1 = 0, s2 = 0, pad0 = 0, nt0 = 0, nt1 = 0;
-    for (int b = 0; b < A; ++b) {
-      const int e2 = act[b], n2 = cnt[e2];
-      if ((n2 < thr) != light) continue;
-      if (n2 > n || (n2 == n && e2 < e)) {
-        ++rank;
-        const int r2 = n2 % kJobRows;
-        s1 += (r2 > 0 && r2 <= 8) ? 1 : 0;
-        s2 += n2 / kJobRows + (r2 > 8 ? 1 : 0);
-        pad0 += (n2 + 255) & ~255;
-        nt0 += (n2 + 127) >> 7;
-        nt1 += (n2 + 255) >> 8;
+  perm_classes(E, thr, dense_supported, o, sm);
+}
+
+// ---------------------------------------------------------------------------
+// The same permutation for large batches in three launches.  Block b of nb
+// owns the contiguous pairs [P b / nb, P (b + 1) / nb):
+//   perm_hist_kernel:  per-block expert counts bcnt[b][e];
+//   perm_scan_kernel:  one block: counts, offsets, the active list and the
+//                      classes, and bcnt turned into per-block bases
+//                      off[e] + sum over earlier blocks;
+//   perm_place_kernel: per block, per-warp counts on top of the block base,
+//                      then positions in (expert, pair) order as in
+//                      build_permutation -- the same stable order.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) perm_hist_kernel(const int* __restrict__ ids, long long P, int E,
+                                                         int* __restrict__ bcnt) {
+  extern __shared__ int hist[];
+  const int b = blockIdx.x, nb = gridDim.x;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const long long c0 = P * b / nb, c1 = P * (b + 1) / nb;
+  for (long long i = c0 + threadIdx.x; i < c1; i += blockDim.x) {
+    const int e = ids[i];
+    if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) bcnt[(size_t)b * E + e] = hist[e];
+}
+
+__global__ void __launch_bounds__(1024) perm_scan_kernel(int* __restrict__ bcnt, int nb, int E, int thr,
+                                                         int dense_supported, PermuteOut o) {
+  extern __shared__ int sm[];
+  int* cnt = sm + 32 * E;
+  int* off = cnt + E;
+  int* act = off + E + 1;
+  int* misc = act + E;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x < 8) misc[threadIdx.x] = 0;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int s = 0;
+    for (int b = 0; b < nb; ++b) s += bcnt[(size_t)b * E + e];
+    cnt[e] = s;
+  }
+  __syncthreads();
+  if (warp == 0) {              // exclusive scan of the counts; compaction of active experts
+    int carry = 0, acarry = 0;
+    for (int b = 0; b < E; b += 32) {
+      const int e = b + lane;
+      const int v = e < E ? cnt[e] : 0;
+      int incl = v;
+      for (int dd = 1; dd < 32; dd <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, dd);
+        if (lane >= dd) incl += n;
       }
+      if (e < E) off[e] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+      const unsigned am = __ballot_sync(0xffffffffu, v > 0);
+      if (v > 0) act[acarry + __popc(am & ((1u << lane) - 1u))] = e;
+      acarry += __popc(am);
     }
-    if (light) {
-      for (int r0 = 0; r0 < n; r0 += kJobRows) {
-        const int nr = min(kJobRows, n - r0);
-        const int4 jb = make_int4(e, off[e] + r0, nr, 0);
-        if (nr <= 8) o.jobs1[s1] = jb; else o.jobs2[s2++] = jb;
-      }
-      const int r = n % kJobRows;
-      atomicAdd(&misc[1], (r > 0 && r <= 8) ? 1 : 0);
-      atomicAdd(&misc[2], n / kJobRows + (r > 8 ? 1 : 0));
-    } else {
-      o.dense_list[rank] = make_int4(e, off[e], n, pad0);
-      o.dense_ntoff[rank] = nt0;
-      o.dense_ntoff[E + 1 + rank] = nt1;
-      atomicAdd(&misc[3], 1);
-      atomicAdd(&misc[4], (n + 127) >> 7);
-      atomicAdd(&misc[5], (n + 255) & ~255);
-      atomicAdd(&misc[6], (n + 255) >> 8);
+    if (lane == 0) { off[E] = carry; misc[0] = acarry; }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = off[e];
+    for (int b = 0; b < nb; ++b) {
+      const int c = bcnt[(size_t)b * E + e];
+      bcnt[(size_t)b * E + e] = run;
+      run += c;
+    }
+    o.counts[e] = cnt[e];
+    o.offsets[e] = off[e];
+  }
+  if (threadIdx.x == 0) o.offsets[E] = off[E];
+  perm_classes(E, thr, dense_supported, o, sm);
+}
+
+__global__ void __launch_bounds__(1024) perm_place_kernel(const int* __restrict__ ids, long long P, int E,
+                                                          const int* __restrict__ bbase, PermuteOut o) {
+  extern __shared__ int wc[];   // [32][E]
+  const int b = blockIdx.x, nb = gridDim.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const long long b0 = P * b / nb, b1 = P * (b + 1) / nb, nbp = b1 - b0;
+  const long long c0 = b0 + nbp * warp / 32, c1 = b0 + nbp * (warp + 1) / 32;
+  for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) wc[i] = 0;
+  __syncthreads();
+  for (long long base = c0; base < c1; base += 32) {          // per-warp counts
+    const long long idx = base + lane;
+    const bool valid = idx < c1;
+    const int e = valid ? ids[idx] : -1;
+    const unsigned mask = __match_any_sync(0xffffffffu, e);
+    if (valid && lane == __ffs(mask) - 1 && e >= 0 && e < E) wc[warp * E + e] += __popc(mask);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = bbase[(size_t)b * E + e];
+    for (int w = 0; w < 32; ++w) {
+      const int c = wc[w * E + e];
+      wc[w * E + e] = run;
+      run += c;
     }
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    *o.n_jobs1 = misc[1];
-    *o.n_jobs2 = misc[2];
-    *o.n_dense = misc[3];
-    o.dense_ntoff[misc[3]] = misc[4];
-    o.dense_ntoff[E + 1 + misc[3]] = misc[6];
-    *o.dense_pad_total = misc[5];
-    if (misc[3] > 0 && !dense_supported) set_error(o.err, kErrUnsupported);
+  const unsigned lt = (1u << lane) - 1u;
+  for (long long base = c0; base < c1; base += 32) {          // positions
+    const long long idx = base + lane;
+    const bool valid = idx < c1;
+    const int e = valid ? ids[idx] : -1;
+    const unsigned mask = __match_any_sync(0xffffffffu, e);
+    const bool ok = valid && e >= 0 && e < E;
+    if (ok) {
+      const int pos = wc[warp * E + e] + __popc(mask & lt);
+      o.perm[pos] = (int)idx;
+      o.inv[idx] = pos;
+    }
+    __syncwarp();
+    if (ok && lane == __ffs(mask) - 1) wc[warp * E + e] += __popc(mask);
+    __syncwarp();
   }
-}
-
-__global__ void __launch_bounds__(1024) permute_kernel(const int* __restrict__ ids, int T, int k,
-                                                       int E, int thr, int dense_supported,
-                                                       PermuteOut o) {
-  extern __shared__ int sm[];
-  build_permutation(ids, T, k, E, thr, dense_supported, o, sm);
 }
 
 // Small-T routing in one launch.  Block e (1024 threads) computes the fp32
