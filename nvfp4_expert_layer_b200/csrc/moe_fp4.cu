@@ -157,20 +157,21 @@ EncodeTiledFn encode_fn() {
 // the 128-byte swizzle the tcgen05 K-major shared-memory descriptors expect.
 // Rows past `rows` read as zeros.
 bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint32_t elem_bytes,
-                 uint64_t row_bytes, uint64_t rows, uint32_t box_rows) {
+                 uint64_t row_bytes, uint64_t rows, uint32_t box_rows, uint32_t box_bytes = 128) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {row_bytes / elem_bytes, rows};
   const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {128 / elem_bytes, box_rows};
+  const cuuint32_t box[2] = {box_bytes / elem_bytes, box_rows};
   const cuuint32_t es[2] = {1, 1};
-  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            box_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Byte operand of the dense GEMMs: rows of kDenseRowBytes per pipeline stage.
 bool make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows, uint32_t box_rows) {
-  return make_map_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, row_bytes, rows, box_rows);
+  return make_map_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, row_bytes, rows, box_rows, moe::kDenseRowBytes);
 }
 
 size_t workspace_bytes(const moe_fp4* h, int Tm) {
@@ -397,7 +398,7 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
     dp.ntoff = w.dense_ntoff;
     dp.wt_per_expert = 2 * f / moe::kDenseN;
     dp.rows_per_expert = 2 * f;
-    dp.kstages = d / 256;
+    dp.kstages = d / moe::kDenseKStage;
     dp.kb64 = d / 64;
     dp.d = d;
     dp.f = f;
@@ -423,7 +424,7 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
     dp2.ntoff = w.dense_ntoff + (E + 1);
     dp2.wt_per_expert = d / 128;
     dp2.rows_per_expert = d;
-    dp2.kstages = f / 256;
+    dp2.kstages = f / moe::kDenseKStage;
     dp2.kb64 = f / 64;
     MOE_CUDA(launch(moe::dense_gemm_kernel<moe::kDenseDown>, dim3(h->sm_count * kDenseGridPerSm),
                     dim3(moe::kDenseThreads), moe::dense_smem_size<moe::kDenseDown>(E), st, pdl, dp2));

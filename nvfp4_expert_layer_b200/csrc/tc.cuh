@@ -73,6 +73,20 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
   d |= (uint64_t)2 << 61;                           // layout: SWIZZLE_128B
   return d;
 }
+// K-major operand with rows of ROW_BYTES (128: 128-byte swizzle; 64: 64-byte
+// swizzle), 8-row atoms of 8 * ROW_BYTES bytes.
+template <int ROW_BYTES>
+__device__ __forceinline__ uint64_t smem_desc_kmajor(uint32_t saddr) {
+  static_assert(ROW_BYTES == 128 || ROW_BYTES == 64, "row bytes");
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)((8 * ROW_BYTES) >> 4) << 32;      // stride byte offset: next 8-row group
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)(ROW_BYTES == 128 ? 2 : 4) << 61;  // SWIZZLE_128B / SWIZZLE_64B
+  return d;
+}
+
 // Scale-factor copy source: 128 rows x 32 bytes, no swizzle, as core matrices
 // of 8 rows x 16 bytes; the two 16-byte halves of a row group are 128 bytes
 // apart (leading byte offset), row groups 256 bytes apart (stride byte offset).
