@@ -301,8 +301,15 @@ cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, c
 
 size_t permute_smem_bytes(int E) { return moe::permute_smem_ints(E) * 4; }
 
-size_t route_smem_bytes(int E, int d, int P) {
-  return std::max((size_t)d * 4 + 32 * 32 * 4, (moe::permute_smem_ints(E) + (size_t)P) * 4);
+size_t route_smem_bytes(int E, int d, int T, int k) {
+  const size_t P = (size_t)T * k;
+  const size_t tail = P <= 32 ? moe::route_small_ids_offset(E, T, k) + 32 : moe::permute_smem_ints(E) + P;
+  return std::max((size_t)d * 4 + 32 * 32 * 4, tail * 4);
+}
+
+// Largest route_kernel shared memory over every T <= kSmallT.
+size_t route_smem_max(int E, int d, int k) {
+  return std::max(route_smem_bytes(E, d, kSmallT, k), route_smem_bytes(E, d, std::max(1, 32 / k), k));
 }
 
 cudaError_t mark(moe_fp4* h, int i, cudaStream_t st) {
@@ -338,7 +345,7 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
   const bool run_dense = h->dense_ok && T >= h->thr;
   if (T <= kSmallT) {
     // 1-3. router logits, x staging, top-k and permutation in one launch
-    MOE_CUDA(launch(moe::route_kernel, dim3(E), dim3(1024), route_smem_bytes(E, d, T * k), st, false,
+    MOE_CUDA(launch(moe::route_kernel, dim3(E), dim3(1024), route_smem_bytes(E, d, T, k), st, false,
                     xb, rw, T, d, E, k, thr, dense_ok, w.logits, w.x16, w.xscale, w.ids, w.wts, ticket, po));
     MOE_CUDA(mark(h, 1, st));
     MOE_CUDA(mark(h, 2, st));
@@ -542,7 +549,7 @@ int moe_fp4_create(int E, int top_k, int d, int f, moe_fp4_t** out) {
         smem_attr((const void*)moe::expert_kernel<2>, kExpSmem) != cudaSuccess ||
         smem_attr((const void*)moe::perm_scan_kernel, permute_smem_bytes(E)) != cudaSuccess ||
         smem_attr((const void*)moe::perm_place_kernel, (size_t)32 * E * 4) != cudaSuccess ||
-        smem_attr((const void*)moe::route_kernel, route_smem_bytes(E, d, kSmallT * top_k)) != cudaSuccess ||
+        smem_attr((const void*)moe::route_kernel, route_smem_max(E, d, top_k)) != cudaSuccess ||
         smem_attr((const void*)moe::dense_gemm_kernel<moe::kDenseGateUp>,
                   moe::dense_smem_size<moe::kDenseGateUp>(E)) != cudaSuccess ||
         smem_attr((const void*)moe::dense_gemm_kernel<moe::kDenseDown>,

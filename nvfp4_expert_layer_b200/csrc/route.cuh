@@ -9,6 +9,7 @@
 // Ultra-Large Sparse Models", section II, Index Pipeline) and sorts a step's
 // experts by row count (Muse Spark page, section 5).
 #pragma once
+#include <climits>
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -142,43 +143,50 @@ __global__ void __launch_bounds__(256) router_tiled_kernel(
 // Warp top-k over v[i] = logit of expert lane + 32 i (-inf beyond E).
 // Lane j < k receives the j-th selected expert and its renormalised weight.
 // PER = logits per lane rounded up to a power of two.  Each lane keeps its
-// best untaken (logit, expert); a round takes the warp arg-max and only the
-// winning lane rescans its PER values.  Within a lane experts increase with
-// i, so a strict comparison keeps the lower expert on ties.
+// best untaken (logit, expert) as an order-preserving 32-bit key; a round is
+// two warp reductions (the largest key, then the lowest expert among the
+// lanes holding it) and only the winning lane rescans its PER values.
+// Within a lane experts increase with i, so a strict comparison keeps the
+// lower expert on ties.
+// Order-preserving key of a logit: a > b as floats <=> key(a) > key(b); -0 and
+// +0 share one key (they compare equal, so the lower expert wins), and every
+// non-NaN logit has a key above 0.
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if ((u << 1) == 0u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float order_key_value(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
 template <int PER>
 __device__ __forceinline__ void topk_warp_t(const float (&v)[32], int E, int k, int lane, int& my_e,
                                             float& my_w) {
   float sel_l0 = 0.f, sum = 0.f, my_p = 0.f;
   my_e = 0;
   unsigned taken = 0u;            // bit i: element lane + 32 i already selected
-  float lv = -INFINITY;
-  int le = 0x7fffffff;
+  uint32_t lk = 0u;               // 0: no candidate left in this lane
+  int le = 0;
   auto lane_best = [&]() {
-    lv = -INFINITY;
-    le = 0x7fffffff;
+    lk = 0u;
+    le = 0;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
       const int e = lane + 32 * i;
-      const bool cand = e < E && !((taken >> i) & 1u);
-      if (cand && (le == 0x7fffffff || v[i] > lv)) { lv = v[i]; le = e; }
+      const uint32_t key = (e < E && !((taken >> i) & 1u)) ? order_key(v[i]) : 0u;
+      if (key > lk) { lk = key; le = e; }
     }
   };
   lane_best();
   for (int j = 0; j < k; ++j) {
-    float bv = lv;
-    int be = le;
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      const bool better = (oe != 0x7fffffff) &&
-                          (be == 0x7fffffff || ov > bv || (ov == bv && oe < be));
-      if (better) { bv = ov; be = oe; }
-    }
-    if (be == 0x7fffffff) be = 0;       // unreachable for k <= E
+    const uint32_t mk = __reduce_max_sync(0xffffffffu, lk);
+    const int be = (int)__reduce_min_sync(0xffffffffu, lk == mk ? (uint32_t)le : 0xffffffffu);
     if ((be & 31) == lane) {
       taken |= 1u << (be >> 5);
       lane_best();
     }
+    const float bv = order_key_value(mk);
     if (j == 0) sel_l0 = bv;
     const float p = expf(bv - sel_l0);
     sum += p;
@@ -322,52 +330,6 @@ __device__ void build_permutation(const int* ids, int T, int k, int E, int thr, 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const long long P = (long long)T * k;
   const long long c0 = P * warp / 32, c1 = P * (warp + 1) / 32;
-  if (P <= 32) {
-    // Small batches (decode): one warp ranks the <= 32 pairs by (expert, pair);
-    // every thread derives count and offset of its experts from the pair list.
-    int* pe = wc;                                   // [32] expert of each pair, -1 if none
-    if (threadIdx.x < 32) {
-      const int e = threadIdx.x < P ? ids[threadIdx.x] : -1;
-      pe[threadIdx.x] = (e >= 0 && e < E) ? e : -1;
-    }
-    if (threadIdx.x < 8) misc[threadIdx.x] = 0;
-    __syncthreads();
-    for (int e = threadIdx.x; e <= E; e += blockDim.x) {
-      int cn = 0, before = 0;
-      for (int q = 0; q < (int)P; ++q) {
-        const int pq = pe[q];
-        cn += pq == e;
-        before += pq >= 0 && pq < e;
-      }
-      if (e < E) { cnt[e] = cn; o.counts[e] = cn; }
-      off[e] = before;
-      o.offsets[e] = before;
-    }
-    if (warp == 0) {
-      const int e = pe[lane];
-      const bool ok = e >= 0;
-      int rank = 0, arank = 0;
-      bool first = ok;
-      for (int m = 0; m < 32; ++m) {
-        const int em = pe[m];
-        rank += em >= 0 && (em < e || (em == e && m < lane));
-        if (m < lane && em == e) first = false;
-      }
-      for (int m = 0; m < 32; ++m) {
-        const bool fm = __shfl_sync(0xffffffffu, first, m);
-        const int em = __shfl_sync(0xffffffffu, e, m);
-        arank += fm && em < e;
-      }
-      if (ok) {
-        o.perm[rank] = lane;
-        o.inv[lane] = rank;
-      }
-      if (first) act[arank] = e;
-      const int A = __popc(__ballot_sync(0xffffffffu, first));
-      if (lane == 0) misc[0] = A;
-    }
-    __syncthreads();
-  } else {
   for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) wc[i] = 0;
   if (threadIdx.x < 8) misc[threadIdx.x] = 0;
   __syncthreads();
@@ -432,8 +394,196 @@ __device__ void build_permutation(const int* ids, int T, int k, int E, int thr, 
     if (ok && lane == __ffs(mask) - 1) wc[warp * E + e] += __popc(mask);
     __syncwarp();
   }
-  }
   perm_classes(E, thr, dense_supported, o, sm);
+}
+
+// ---------------------------------------------------------------------------
+// Small batches (T * k <= 32 pairs, decode): top-k and permutation in the one
+// block of 1024 threads, built from independent comparisons instead of k
+// sequential arg-max rounds, so the latency is a few short phases.
+// ---------------------------------------------------------------------------
+// Shared-memory ints used by topk_small_block.
+__host__ __device__ constexpr size_t topk_small_ints(int E, int T, int k) {
+  const size_t G = (size_t)(E + 31) / 32, kk = (size_t)(k < 32 ? k : 32);
+  return (size_t)T * G * 32 + 2 * (size_t)T * G * kk + 2 * (size_t)T * k;
+}
+
+// Pair experts of the small path sit after the top-k scratch (and after the
+// 64 ints the permutation exchanges through shared memory).
+__host__ __device__ constexpr size_t route_small_ids_offset(int E, int T, int k) {
+  return topk_small_ints(E, T, k) > 64 ? topk_small_ints(E, T, k) : 64;
+}
+
+// Top-k of T tokens (T <= 32) over the logits [T][E] with the order and the
+// weights of topk_warp_t: (logit desc, expert asc), weights the softmax of the
+// selected logits accumulated in selection order.  Phase 1 ranks every
+// logit inside its group of 32 experts and keeps the best min(k, 32) of each
+// group as candidates (a global top-k member has fewer than k better experts
+// in its group); phase 2 ranks the candidates of a token against each other.
+__device__ void topk_small_block(const float* logits, int T, int E, int k, int* ids_s, int* ids_out,
+                                 float* wts, uint32_t* scratch) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int tp = 1;
+  while (tp < T) tp <<= 1;
+  const int wpt = (int)(blockDim.x >> 5) / tp;       // warps per token (>= 1)
+  const int t = warp / wpt, wt = warp - t * wpt;
+  const int G = (E + 31) / 32, kk = min(k, 32), C = G * kk;
+  uint32_t* s_key = scratch;                          // [T][G*32] keys, 0 beyond E
+  uint32_t* c_key = s_key + (size_t)T * G * 32;       // [T][C]
+  int* c_e = reinterpret_cast<int*>(c_key + (size_t)T * C);
+  uint32_t* sel_key = reinterpret_cast<uint32_t*>(c_e + (size_t)T * C);   // [T][k]
+  int* sel_e = reinterpret_cast<int*>(sel_key + (size_t)T * k);
+  for (int i = tid; i < T * G * 32; i += blockDim.x) {
+    const int tt = i / (G * 32), e = i - tt * G * 32;
+    float l = 0.f;
+    if (e < E) asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(l) : "l"(logits + (size_t)tt * E + e));
+    s_key[i] = e < E ? order_key(l) : 0u;
+  }
+  __syncthreads();
+  if (t < T) {
+    for (int g = wt; g < G; g += wpt) {
+      const uint32_t* gk = s_key + ((size_t)t * G + g) * 32;
+      const uint32_t mine = gk[lane];
+      int r = 0;
+#pragma unroll
+      for (int m = 0; m < 32; ++m) {
+        const uint32_t o = gk[m];
+        r += (o > mine || (o == mine && m < lane)) ? 1 : 0;
+      }
+      if (r < kk) {
+        c_key[(size_t)t * C + g * kk + r] = mine;
+        c_e[(size_t)t * C + g * kk + r] = g * 32 + lane;
+      }
+    }
+  }
+  __syncthreads();
+  if (t < T) {
+    const uint32_t* ck = c_key + (size_t)t * C;
+    const int* ce = c_e + (size_t)t * C;
+    for (int c = wt * 32 + lane; c < C; c += wpt * 32) {
+      const uint32_t mine = ck[c];
+      const int me = ce[c];
+      int r = 0;
+#pragma unroll 8
+      for (int m = 0; m < C; ++m) {
+        const uint32_t o = ck[m];
+        r += (o > mine || (o == mine && ce[m] < me)) ? 1 : 0;
+      }
+      if (r < k) {
+        sel_key[(size_t)t * k + r] = mine;
+        sel_e[(size_t)t * k + r] = me;
+      }
+    }
+  }
+  __syncthreads();
+  if (t < T && wt == 0 && lane < k) {
+    const uint32_t* sk = sel_key + (size_t)t * k;
+    const float l0 = order_key_value(sk[0]);
+    float sum = 0.f, my_p = 0.f;
+    for (int j = 0; j < k; ++j) {
+      const float p = expf(order_key_value(sk[j]) - l0);
+      sum += p;
+      if (j == lane) my_p = p;
+    }
+    const int e = sel_e[(size_t)t * k + lane];
+    ids_s[t * k + lane] = e;
+    ids_out[(size_t)t * k + lane] = e;
+    wts[(size_t)t * k + lane] = my_p / sum;
+  }
+}
+
+// Permutation and classes of at most 32 pairs (ids in shared memory), with
+// the results of build_permutation + perm_classes.  Threads 32.. write the
+// count and offset of every expert; warp 0 holds pair l in lane l, ranks it in
+// (expert, pair) order and classes the active experts one lane each.
+__device__ void perm_small(const int* ids, int P, int E, int thr, int dense_supported, const PermuteOut& o,
+                           int* s_n, int* s_e) {
+  const unsigned FULL = 0xffffffffu;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int x = tid - 32; x >= 0 && x <= E; x += (int)blockDim.x - 32) {
+    int cn = 0, before = 0;
+#pragma unroll
+    for (int q = 0; q < 32; ++q) {
+      if (q < P) {
+        const int eq = ids[q];
+        const bool okq = eq >= 0 && eq < E;
+        cn += (okq && eq == x) ? 1 : 0;
+        before += (okq && eq < x) ? 1 : 0;
+      }
+    }
+    if (x < E) o.counts[x] = cn;
+    o.offsets[x] = before;
+  }
+  if (warp != 0) return;
+  const int e0 = lane < P ? ids[lane] : -1;
+  const bool ok = e0 >= 0 && e0 < E;
+  const int e = ok ? e0 : INT_MAX;
+  int rank = 0, n = 0, nless = 0;
+  bool first = ok;
+#pragma unroll
+  for (int m = 0; m < 32; ++m) {
+    int em = m < P ? ids[m] : -1;
+    em = (em >= 0 && em < E) ? em : INT_MAX;
+    rank += (em < e || (em == e && m < lane)) ? 1 : 0;
+    n += em == e ? 1 : 0;
+    nless += em < e ? 1 : 0;
+    if (m < lane && em == e) first = false;
+  }
+  if (ok) {
+    o.perm[rank] = lane;
+    o.inv[lane] = rank;
+  }
+  s_n[lane] = first ? n : -1;
+  s_e[lane] = e;
+  __syncwarp();
+  const bool light = n < thr;
+  int crank = 0, s1 = 0, s2 = 0, pad0 = 0, nt0 = 0, nt1 = 0;
+  if (first) {
+#pragma unroll
+    for (int m = 0; m < 32; ++m) {
+      const int n2 = s_n[m], em = s_e[m];
+      if (n2 >= 0 && ((n2 < thr) == light) && (n2 > n || (n2 == n && em < e))) {
+        ++crank;
+        const int r2 = n2 % kJobRows;
+        s1 += (r2 > 0 && r2 <= 8) ? 1 : 0;
+        s2 += n2 / kJobRows + (r2 > 8 ? 1 : 0);
+        pad0 += (n2 + 255) & ~255;
+        nt0 += (n2 + 127) >> 7;
+        nt1 += (n2 + 255) >> 8;
+      }
+    }
+  }
+  const int r = n % kJobRows;
+  int c_j1 = 0, c_j2 = 0, c_d = 0, c_nt0 = 0, c_pad = 0, c_nt1 = 0;
+  if (first && light) {
+    for (int r0 = 0; r0 < n; r0 += kJobRows) {
+      const int nr = min(kJobRows, n - r0);
+      const int4 jb = make_int4(e, nless + r0, nr, 0);
+      if (nr <= 8) o.jobs1[s1] = jb; else o.jobs2[s2++] = jb;
+    }
+    c_j1 = (r > 0 && r <= 8) ? 1 : 0;
+    c_j2 = n / kJobRows + (r > 8 ? 1 : 0);
+  } else if (first) {
+    o.dense_list[crank] = make_int4(e, nless, n, pad0);
+    o.dense_ntoff[crank] = nt0;
+    o.dense_ntoff[E + 1 + crank] = nt1;
+    c_d = 1;
+    c_nt0 = (n + 127) >> 7;
+    c_pad = (n + 255) & ~255;
+    c_nt1 = (n + 255) >> 8;
+  }
+  const int n_j1 = __reduce_add_sync(FULL, c_j1), n_j2 = __reduce_add_sync(FULL, c_j2);
+  const int n_d = __reduce_add_sync(FULL, c_d), t_nt0 = __reduce_add_sync(FULL, c_nt0);
+  const int t_pad = __reduce_add_sync(FULL, c_pad), t_nt1 = __reduce_add_sync(FULL, c_nt1);
+  if (lane == 0) {
+    *o.n_jobs1 = n_j1;
+    *o.n_jobs2 = n_j2;
+    *o.n_dense = n_d;
+    o.dense_ntoff[n_d] = t_nt0;
+    o.dense_ntoff[E + 1 + n_d] = t_nt1;
+    *o.dense_pad_total = t_pad;
+    if (n_d > 0 && !dense_supported) set_error(o.err, kErrUnsupported);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -558,9 +708,11 @@ __global__ void __launch_bounds__(1024) perm_place_kernel(const int* __restrict_
 // logits of expert e for every token (its router row is staged in shared
 // memory, one warp per token) and stages x rows t = e, e + E, ... in fp16.
 // The last block to finish (an atomic ticket; no grid barrier) runs the
-// routing tail: top-k for every token (warp per token) and the permutation,
-// then clears the ticket for the next launch.  Dynamic shared memory:
-// max(d floats, permute_smem_ints(E) + T*k ints).
+// routing tail: top-k and the permutation (at most 32 pairs: the ranked
+// top-k and perm_small; otherwise a warp per token and build_permutation),
+// then clears the ticket for the next launch.  Dynamic shared memory: the
+// largest of d + 1024 floats (router row and warp partials), the small path's
+// route_small_ids_offset + 32 ints, or permute_smem_ints(E) + T*k ints.
 __global__ void __launch_bounds__(1024) route_kernel(
     const uint16_t* __restrict__ x, const float* __restrict__ rw, int T, int d, int E, int k,
     int thr, int dense_supported, float* __restrict__ logits, __half* __restrict__ x16,
@@ -641,6 +793,16 @@ __global__ void __launch_bounds__(1024) route_kernel(
   }
   __syncthreads();
   if (!s_last) return;
+  if ((long long)T * k <= 32) {
+    // decode: ranked top-k (scratch from the start of shared memory, the pair
+    // experts after it), then the small permutation
+    int* ids_small = sm + route_small_ids_offset(E, T, k);
+    topk_small_block(logits, T, E, k, ids_small, ids_out, wts, reinterpret_cast<uint32_t*>(sm));
+    __syncthreads();
+    perm_small(ids_small, T * k, E, thr, dense_supported, o, sm, sm + 32);
+    if (threadIdx.x == 0) *ticket = 0;
+    return;
+  }
   int* ids_s = sm + permute_smem_ints(E);
   for (int t = warp; t < T; t += 32) {
     float v[32];

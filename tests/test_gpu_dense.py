@@ -27,6 +27,15 @@ def test_dense_tiny_every_expert_dense():
     assert c.n_dense_rows == c.cfg.T * c.cfg.k
 
 
+def test_dense_and_light_classes_small_batch():
+    # 32 pairs (the small-batch routing path): experts with >= 3 rows dense, the rest light
+    cfg = W.custom_config(T=4, d=512, E=16, k=8, f=256, seed=56, router="unit")
+    c = _run(cfg, thr=3)
+    counts = c.o["counts"]
+    assert np.any(counts >= 3) and np.any((counts > 0) & (counts < 3)), counts
+    assert 0 < c.n_dense_rows < cfg.T * cfg.k
+
+
 def test_dense_ragged_multi_tile_experts():
     # ~175 rows per expert: two 128-token tiles, the second ragged
     cfg = W.custom_config(T=700, d=512, E=8, k=2, f=512, seed=51, router="unit")
