@@ -405,7 +405,7 @@ __device__ void build_permutation(const int* ids, int T, int k, int E, int thr, 
 // Shared-memory ints used by topk_small_block.
 __host__ __device__ constexpr size_t topk_small_ints(int E, int T, int k) {
   const size_t G = (size_t)(E + 31) / 32, kk = (size_t)(k < 32 ? k : 32);
-  return (size_t)T * G * 32 + 2 * (size_t)T * G * kk + 2 * (size_t)T * k;
+  return (size_t)T * G * 32 + 2 * (size_t)T * G * kk + 2 * (size_t)T * k + 2;
 }
 
 // Pair experts of the small path sit after the top-k scratch (and after the
@@ -414,31 +414,35 @@ __host__ __device__ constexpr size_t route_small_ids_offset(int E, int T, int k)
   return topk_small_ints(E, T, k) > 64 ? topk_small_ints(E, T, k) : 64;
 }
 
-// Top-k of T tokens (T <= 32) over the logits [T][E] with the order and the
+// Top-k of T tokens (T <= 32; a block of 1024 threads) over the logits [T][E] with the order and the
 // weights of topk_warp_t: (logit desc, expert asc), weights the softmax of the
 // selected logits accumulated in selection order.  Phase 1 ranks every
 // logit inside its group of 32 experts and keeps the best min(k, 32) of each
 // group as candidates (a global top-k member has fewer than k better experts
-// in its group); phase 2 ranks the candidates of a token against each other.
+// in its group); phase 2 ranks the candidates of a token against each other,
+// several threads per candidate.  Candidates carry one 64-bit key, logit key
+// above the complemented expert, so one comparison orders (logit, expert).
+// Every loop has independent iterations (no load behind a branch): the
+// phases are latency-bound, not issue-bound.
 __device__ void topk_small_block(const float* logits, int T, int E, int k, int* ids_s, int* ids_out,
                                  float* wts, uint32_t* scratch) {
+  const unsigned FULL = 0xffffffffu;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int tp = 1;
-  while (tp < T) tp <<= 1;
-  const int wpt = (int)(blockDim.x >> 5) / tp;       // warps per token (>= 1)
-  const int t = warp / wpt, wt = warp - t * wpt;
+  int ltp = 0;                                        // tokens rounded up to 2^ltp
+  while ((1 << ltp) < T) ++ltp;
+  const int ltpt = 10 - ltp;                          // threads per token 2^ltpt (>= 32)
+  const int tpt = 1 << ltpt, wpt = tpt >> 5;
+  const int t = tid >> ltpt, u = tid & (tpt - 1), wt = u >> 5;
   const int G = (E + 31) / 32, kk = min(k, 32), C = G * kk;
   uint32_t* s_key = scratch;                          // [T][G*32] keys, 0 beyond E
-  uint32_t* c_key = s_key + (size_t)T * G * 32;       // [T][C]
-  int* c_e = reinterpret_cast<int*>(c_key + (size_t)T * C);
-  uint32_t* sel_key = reinterpret_cast<uint32_t*>(c_e + (size_t)T * C);   // [T][k]
-  int* sel_e = reinterpret_cast<int*>(sel_key + (size_t)T * k);
-  for (int i = tid; i < T * G * 32; i += blockDim.x) {
-    const int tt = i / (G * 32), e = i - tt * G * 32;
-    float l = 0.f;
-    if (e < E) asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(l) : "l"(logits + (size_t)tt * E + e));
-    s_key[i] = e < E ? order_key(l) : 0u;
-  }
+  uint64_t* c_key = reinterpret_cast<uint64_t*>(s_key + (((size_t)T * G * 32 + 1) & ~(size_t)1));   // [T][C]
+  uint64_t* sel = c_key + (size_t)T * C;              // [T][k]
+  for (int tt = 0; tt < T; ++tt)
+    for (int e = tid; e < G * 32; e += blockDim.x) {
+      float l = 0.f;
+      if (e < E) asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(l) : "l"(logits + (size_t)tt * E + e));
+      s_key[(size_t)tt * G * 32 + e] = e < E ? order_key(l) : 0u;
+    }
   __syncthreads();
   if (t < T) {
     for (int g = wt; g < G; g += wpt) {
@@ -450,139 +454,162 @@ __device__ void topk_small_block(const float* logits, int T, int E, int k, int* 
         const uint32_t o = gk[m];
         r += (o > mine || (o == mine && m < lane)) ? 1 : 0;
       }
-      if (r < kk) {
-        c_key[(size_t)t * C + g * kk + r] = mine;
-        c_e[(size_t)t * C + g * kk + r] = g * 32 + lane;
-      }
+      if (r < kk)
+        c_key[(size_t)t * C + g * kk + r] = ((uint64_t)mine << 32) | (uint32_t)~(uint32_t)(g * 32 + lane);
     }
   }
   __syncthreads();
   if (t < T) {
-    const uint32_t* ck = c_key + (size_t)t * C;
-    const int* ce = c_e + (size_t)t * C;
-    for (int c = wt * 32 + lane; c < C; c += wpt * 32) {
-      const uint32_t mine = ck[c];
-      const int me = ce[c];
+    // 2^ls threads per candidate (at most 32), uniform trip counts per warp
+    int ls = 0;
+    while (ls < 5 && (C << (ls + 1)) <= tpt) ++ls;
+    const int s = 1 << ls;
+    const int per = tpt >> ls;                        // candidates per round
+    const int q = u & (s - 1);
+    const uint64_t* ck = c_key + (size_t)t * C;
+    const int nm = (C + s - 1) >> ls;
+    for (int c0 = 0; c0 < C; c0 += per) {
+      const int c = c0 + (u >> ls);
+      const uint64_t mine = c < C ? ck[c] : 0ull;
       int r = 0;
 #pragma unroll 8
-      for (int m = 0; m < C; ++m) {
-        const uint32_t o = ck[m];
-        r += (o > mine || (o == mine && ce[m] < me)) ? 1 : 0;
+      for (int i = 0; i < nm; ++i) {
+        const int m = q + i * s;
+        const uint64_t o = m < C ? ck[m] : 0ull;
+        r += o > mine ? 1 : 0;
       }
-      if (r < k) {
-        sel_key[(size_t)t * k + r] = mine;
-        sel_e[(size_t)t * k + r] = me;
-      }
+      for (int o = 1; o < s; o <<= 1) r += __shfl_xor_sync(FULL, r, o);
+      if (c < C && q == 0 && r < k) sel[(size_t)t * k + r] = mine;
     }
   }
   __syncthreads();
   if (t < T && wt == 0 && lane < k) {
-    const uint32_t* sk = sel_key + (size_t)t * k;
-    const float l0 = order_key_value(sk[0]);
+    const uint64_t* sk = sel + (size_t)t * k;
+    const float l0 = order_key_value((uint32_t)(sk[0] >> 32));
     float sum = 0.f, my_p = 0.f;
     for (int j = 0; j < k; ++j) {
-      const float p = expf(order_key_value(sk[j]) - l0);
+      const float p = expf(order_key_value((uint32_t)(sk[j] >> 32)) - l0);
       sum += p;
       if (j == lane) my_p = p;
     }
-    const int e = sel_e[(size_t)t * k + lane];
+    const int e = (int)~(uint32_t)sk[lane];
     ids_s[t * k + lane] = e;
     ids_out[(size_t)t * k + lane] = e;
     wts[(size_t)t * k + lane] = my_p / sum;
   }
 }
 
-// Permutation and classes of at most 32 pairs (ids in shared memory), with
-// the results of build_permutation + perm_classes.  Threads 32.. write the
-// count and offset of every expert; warp 0 holds pair l in lane l, ranks it in
-// (expert, pair) order and classes the active experts one lane each.
-__device__ void perm_small(const int* ids, int P, int E, int thr, int dense_supported, const PermuteOut& o,
-                           int* s_n, int* s_e) {
+// Ascending bitonic sort of one 32-bit key per lane across a warp.
+__device__ __forceinline__ uint32_t warp_sort_u32(uint32_t key, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const uint32_t other = __shfl_xor_sync(0xffffffffu, key, j);
+      const bool keep_min = ((lane & j) == 0) == ((lane & k) == 0);
+      key = keep_min ? min(key, other) : max(key, other);
+    }
+  }
+  return key;
+}
+
+// Inclusive warp scan.
+__device__ __forceinline__ uint32_t warp_scan_u32(uint32_t v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  return v;
+}
+
+// Permutation and classes of at most 32 pairs (ids in shared memory, padded
+// with -1 to 32 entries), with the results of build_permutation +
+// perm_classes (E <= 1024, so an expert fits 10 bits).  Threads 32.. write
+// the count and offset of every expert.  Warp 0 sorts the pair keys
+// (expert, pair): lane i then holds permuted row i, so perm and inv follow
+// directly, and the runs of equal experts give each active expert its row
+// count n and offset.  A second sort orders the active experts by class
+// (light before dense), n descending, expert ascending; exclusive warp scans
+// over that order give every expert's job-list slots and dense-tile prefixes.
+// A single warp runs at about one dependent instruction per several cycles,
+// so this path is built from log-depth shuffle networks, not loops over 32.
+__device__ void perm_small(const int* ids, int E, int thr, int dense_supported, const PermuteOut& o) {
   const unsigned FULL = 0xffffffffu;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int x = tid - 32; x >= 0 && x <= E; x += (int)blockDim.x - 32) {
     int cn = 0, before = 0;
 #pragma unroll
     for (int q = 0; q < 32; ++q) {
-      if (q < P) {
-        const int eq = ids[q];
-        const bool okq = eq >= 0 && eq < E;
-        cn += (okq && eq == x) ? 1 : 0;
-        before += (okq && eq < x) ? 1 : 0;
-      }
+      const int eq = ids[q];
+      const bool okq = eq >= 0 && eq < E;
+      cn += (okq && eq == x) ? 1 : 0;
+      before += (okq && eq < x) ? 1 : 0;
     }
     if (x < E) o.counts[x] = cn;
     o.offsets[x] = before;
   }
   if (warp != 0) return;
-  const int e0 = lane < P ? ids[lane] : -1;
+  const int e0 = ids[lane];
   const bool ok = e0 >= 0 && e0 < E;
-  const int e = ok ? e0 : INT_MAX;
-  int rank = 0, n = 0, nless = 0;
-  bool first = ok;
-#pragma unroll
-  for (int m = 0; m < 32; ++m) {
-    int em = m < P ? ids[m] : -1;
-    em = (em >= 0 && em < E) ? em : INT_MAX;
-    rank += (em < e || (em == e && m < lane)) ? 1 : 0;
-    n += em == e ? 1 : 0;
-    nless += em < e ? 1 : 0;
-    if (m < lane && em == e) first = false;
+  // 1. pairs in (expert, pair) order
+  const uint32_t pk = warp_sort_u32(ok ? ((uint32_t)e0 << 5) | (uint32_t)lane : 0xffffffffu, lane);
+  const bool valid = pk != 0xffffffffu;
+  const int e = (int)(pk >> 5), pair = (int)(pk & 31u);
+  if (valid) {
+    o.perm[lane] = pair;
+    o.inv[pair] = lane;
   }
-  if (ok) {
-    o.perm[rank] = lane;
-    o.inv[lane] = rank;
-  }
-  s_n[lane] = first ? n : -1;
-  s_e[lane] = e;
-  __syncwarp();
-  const bool light = n < thr;
-  int crank = 0, s1 = 0, s2 = 0, pad0 = 0, nt0 = 0, nt1 = 0;
-  if (first) {
-#pragma unroll
-    for (int m = 0; m < 32; ++m) {
-      const int n2 = s_n[m], em = s_e[m];
-      if (n2 >= 0 && ((n2 < thr) == light) && (n2 > n || (n2 == n && em < e))) {
-        ++crank;
-        const int r2 = n2 % kJobRows;
-        s1 += (r2 > 0 && r2 <= 8) ? 1 : 0;
-        s2 += n2 / kJobRows + (r2 > 8 ? 1 : 0);
-        pad0 += (n2 + 255) & ~255;
-        nt0 += (n2 + 127) >> 7;
-        nt1 += (n2 + 255) >> 8;
-      }
-    }
-  }
-  const int r = n % kJobRows;
-  int c_j1 = 0, c_j2 = 0, c_d = 0, c_nt0 = 0, c_pad = 0, c_nt1 = 0;
-  if (first && light) {
-    for (int r0 = 0; r0 < n; r0 += kJobRows) {
-      const int nr = min(kJobRows, n - r0);
-      const int4 jb = make_int4(e, nless + r0, nr, 0);
+  // 2. runs of equal experts: the first row of each run is the expert's offset
+  const int e_prev = __shfl_up_sync(FULL, e, 1);
+  const bool first = valid && (lane == 0 || e_prev != e);
+  const unsigned fm = __ballot_sync(FULL, first);
+  const int nvalid = __popc(__ballot_sync(FULL, valid));
+  const unsigned later = fm & ~((2u << lane) - 1u);          // run starts after this lane
+  const int n = first ? (later ? __ffs(later) - 1 : nvalid) - lane : 0;
+  // 3. active experts by (class, n desc, expert asc); the row offset rides along
+  const uint32_t cls = (first && n >= thr) ? 1u : 0u;
+  const uint32_t ck = first ? (cls << 21) | ((uint32_t)(63 - n) << 15) | ((uint32_t)e << 5) | (uint32_t)lane
+                            : 0xffffffffu;
+  const uint32_t sk = warp_sort_u32(ck, lane);
+  const bool act = sk != 0xffffffffu;
+  const bool dense = act && ((sk >> 21) & 1u);
+  const int ae = (int)((sk >> 5) & 1023u), an = act ? 63 - (int)((sk >> 15) & 63u) : 0;
+  const int aoff = (int)(sk & 31u);
+  // 4. exclusive scans over the class order: list-1 jobs, list-2 jobs, 128- and
+  // 256-row tiles (one byte each; at most 64 per byte), padded rows / 256
+  const int r = an % kJobRows;
+  const uint32_t c1 = (act && !dense && r > 0 && r <= 8) ? 1u : 0u;
+  const uint32_t c2 = (act && !dense) ? (uint32_t)(an / kJobRows + (r > 8 ? 1 : 0)) : 0u;
+  const uint32_t t0 = dense ? (uint32_t)((an + 127) >> 7) : 0u;
+  const uint32_t t1 = dense ? (uint32_t)((an + 255) >> 8) : 0u;
+  const uint32_t packed = c1 | (c2 << 8) | (t0 << 16) | (t1 << 24);
+  const uint32_t inc = warp_scan_u32(packed, lane);
+  const uint32_t exc = inc - packed;
+  const uint32_t tot = __shfl_sync(FULL, inc, 31);
+  const int nlight = __popc(__ballot_sync(FULL, act && !dense));
+  if (act && !dense) {
+    int s1 = (int)(exc & 0xffu), s2 = (int)((exc >> 8) & 0xffu);
+    for (int r0 = 0; r0 < an; r0 += kJobRows) {
+      const int nr = min(kJobRows, an - r0);
+      const int4 jb = make_int4(ae, aoff + r0, nr, 0);
       if (nr <= 8) o.jobs1[s1] = jb; else o.jobs2[s2++] = jb;
     }
-    c_j1 = (r > 0 && r <= 8) ? 1 : 0;
-    c_j2 = n / kJobRows + (r > 8 ? 1 : 0);
-  } else if (first) {
-    o.dense_list[crank] = make_int4(e, nless, n, pad0);
-    o.dense_ntoff[crank] = nt0;
-    o.dense_ntoff[E + 1 + crank] = nt1;
-    c_d = 1;
-    c_nt0 = (n + 127) >> 7;
-    c_pad = (n + 255) & ~255;
-    c_nt1 = (n + 255) >> 8;
+  } else if (dense) {
+    const int crank = lane - nlight;
+    o.dense_list[crank] = make_int4(ae, aoff, an, (int)((exc >> 24) & 0xffu) * 256);
+    o.dense_ntoff[crank] = (int)((exc >> 16) & 0xffu);
+    o.dense_ntoff[E + 1 + crank] = (int)((exc >> 24) & 0xffu);
   }
-  const int n_j1 = __reduce_add_sync(FULL, c_j1), n_j2 = __reduce_add_sync(FULL, c_j2);
-  const int n_d = __reduce_add_sync(FULL, c_d), t_nt0 = __reduce_add_sync(FULL, c_nt0);
-  const int t_pad = __reduce_add_sync(FULL, c_pad), t_nt1 = __reduce_add_sync(FULL, c_nt1);
+  const int n_dense = __popc(__ballot_sync(FULL, dense));
   if (lane == 0) {
-    *o.n_jobs1 = n_j1;
-    *o.n_jobs2 = n_j2;
-    *o.n_dense = n_d;
-    o.dense_ntoff[n_d] = t_nt0;
-    o.dense_ntoff[E + 1 + n_d] = t_nt1;
-    *o.dense_pad_total = t_pad;
-    if (n_d > 0 && !dense_supported) set_error(o.err, kErrUnsupported);
+    *o.n_jobs1 = (int)(tot & 0xffu);
+    *o.n_jobs2 = (int)((tot >> 8) & 0xffu);
+    *o.n_dense = n_dense;
+    o.dense_ntoff[n_dense] = (int)((tot >> 16) & 0xffu);
+    o.dense_ntoff[E + 1 + n_dense] = (int)((tot >> 24) & 0xffu);
+    *o.dense_pad_total = (int)((tot >> 24) & 0xffu) * 256;
+    if (n_dense > 0 && !dense_supported) set_error(o.err, kErrUnsupported);
   }
 }
 
@@ -798,8 +825,9 @@ __global__ void __launch_bounds__(1024) route_kernel(
     // experts after it), then the small permutation
     int* ids_small = sm + route_small_ids_offset(E, T, k);
     topk_small_block(logits, T, E, k, ids_small, ids_out, wts, reinterpret_cast<uint32_t*>(sm));
+    if (threadIdx.x >= T * k && threadIdx.x < 32) ids_small[threadIdx.x] = -1;
     __syncthreads();
-    perm_small(ids_small, T * k, E, thr, dense_supported, o, sm, sm + 32);
+    perm_small(ids_small, E, thr, dense_supported, o);
     if (threadIdx.x == 0) *ticket = 0;
     return;
   }
