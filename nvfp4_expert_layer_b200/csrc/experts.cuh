@@ -168,39 +168,70 @@ __device__ __forceinline__ uint32_t e4m3_dup_f16x2(uint32_t four, int k) {
 }
 constexpr float kScaleUndo = 256.f;
 
+// The same for two scales at once: {a_k, b_k} * 2^-8 as f16x2 (byte k of `a`
+// in the low half, byte k of `b` in the high half).  One byte permute puts the
+// two bytes in the low byte of each half (the other bytes come from the
+// sign-replicate mode of a byte whose top bit is clear, i.e. zero), one shift
+// moves them to f16 bit 7.
+// (The PTX prmt default mode honours the selector's sign-replicate bit;
+// __byte_perm keeps only the low three bits of each selector nibble.)
+template <int K>
+__device__ __forceinline__ uint32_t e4m3_pair_f16x2(uint32_t a, uint32_t b) {
+  constexpr uint32_t sel = (uint32_t)K | ((8u | K) << 4) | ((4u + K) << 8) | ((12u + K) << 12);
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "n"(sel));
+  return r << 7;
+}
+
+// a * {lo(s), lo(s)} and a * {hi(s), hi(s)}: the half broadcast is an operand
+// modifier of the f16x2 multiply.
+__device__ __forceinline__ uint32_t hmul2_bcast_lo(uint32_t a, uint32_t s) {
+  const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&a), __low2half2(*reinterpret_cast<const __half2*>(&s)));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t hmul2_bcast_hi(uint32_t a, uint32_t s) {
+  const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&a), __high2half2(*reinterpret_cast<const __half2*>(&s)));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
 // One stage of shared-memory weights times the lane's activation fragments.
+// The codes and scales of the next (chunk, row tile) are loaded before the
+// current one is converted, so the shared-memory latency overlaps the math.
 template <int NT, int RT>
 __device__ __forceinline__ void mma_stage(uint32_t st, int nch, int lane, int g, const BFrag<NT>& b,
                                           int nrows, float (&acc)[RT][4][NT][4]) {
+  constexpr int NU = kExpSC * RT;                   // (chunk, row tile) units, chunk-major
+  auto unit_addr = [&](int u) { return st + (u % RT) * kExpSB + (u / RT) * kChunkBytes; };
+  uint4 codes_n = ld_shared_v4(unit_addr(0) + lane * 16);
+  uint2 sc_n = ld_shared_v2(unit_addr(0) + kChunkCodeBytes + g * 8);
 #pragma unroll
-  for (int ch = 0; ch < kExpSC; ++ch) {
+  for (int u = 0; u < NU; ++u) {
+    const int ch = u / RT, rt = u % RT;
+    if (ch >= nch) break;
+    const uint4 codes = codes_n;
+    const uint2 sc = sc_n;
+    if (u + 1 < NU && (u + 1) / RT < nch) {
+      codes_n = ld_shared_v4(unit_addr(u + 1) + lane * 16);
+      sc_n = ld_shared_v2(unit_addr(u + 1) + kChunkCodeBytes + g * 8);
+    }
+    const uint32_t cw[4] = {codes.x, codes.y, codes.z, codes.w};
+    const uint32_t sAB[4] = {e4m3_pair_f16x2<0>(sc.x, sc.y), e4m3_pair_f16x2<1>(sc.x, sc.y),
+                             e4m3_pair_f16x2<2>(sc.x, sc.y), e4m3_pair_f16x2<3>(sc.x, sc.y)};
 #pragma unroll
-    for (int rt = 0; rt < RT; ++rt)
-    if (ch < nch) {
-      const uint32_t sr = st + rt * kExpSB;
-      const uint4 codes = ld_shared_v4(sr + ch * kChunkBytes + lane * 16);
-      const uint2 sc = ld_shared_v2(sr + ch * kChunkBytes + kChunkCodeBytes + g * 8);
-      const uint32_t cw[4] = {codes.x, codes.y, codes.z, codes.w};
-      // scales: sc.x = row A(g) for K steps 0..3, sc.y = row B(g); non-negative
-      // e4m3 bytes (signs are folded into the codes), see e4m3_dup_f16x2
+    for (int ks = 0; ks < 4; ++ks) {
+      uint32_t a[4];
+      e2m1x8_to_f16x2x4(cw[ks], a);
+      a[0] = hmul2_bcast_lo(a[0], sAB[ks]);
+      a[1] = hmul2_bcast_hi(a[1], sAB[ks]);
+      a[2] = hmul2_bcast_lo(a[2], sAB[ks]);
+      a[3] = hmul2_bcast_hi(a[3], sAB[ks]);
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        const uint32_t sA = e4m3_dup_f16x2(sc.x, ks);
-        const uint32_t sB = e4m3_dup_f16x2(sc.y, ks);
-        uint32_t a[4];
-        e2m1x8_to_f16x2x4(cw[ks], a);
-        a[0] = hmul2_u32(a[0], sA);
-        a[1] = hmul2_u32(a[1], sB);
-        a[2] = hmul2_u32(a[2], sA);
-        a[3] = hmul2_u32(a[3], sB);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const uint4& lo = b.v[nt][ch][0];
-          const uint4& hi = b.v[nt][ch][1];
-          const uint32_t b0 = ks == 0 ? lo.x : ks == 1 ? lo.z : ks == 2 ? hi.x : hi.z;
-          const uint32_t b1 = ks == 0 ? lo.y : ks == 1 ? lo.w : ks == 2 ? hi.y : hi.w;
-          if (NT == 1 || nt * 8 < nrows) mma_16816_f16(acc[rt][ks][nt], a, b0, b1);
-        }
+      for (int nt = 0; nt < NT; ++nt) {
+        const uint4& lo = b.v[nt][ch][0];
+        const uint4& hi = b.v[nt][ch][1];
+        const uint32_t b0 = ks == 0 ? lo.x : ks == 1 ? lo.z : ks == 2 ? hi.x : hi.z;
+        const uint32_t b1 = ks == 0 ? lo.y : ks == 1 ? lo.w : ks == 2 ? hi.y : hi.w;
+        if (NT == 1 || nt * 8 < nrows) mma_16816_f16(acc[rt][ks][nt], a, b0, b1);
       }
     }
   }

@@ -151,10 +151,12 @@ __device__ __forceinline__ uint32_t dup_lo(uint32_t v) { return __byte_perm(v, 0
 __device__ __forceinline__ uint32_t dup_hi(uint32_t v) { return __byte_perm(v, 0, 0x3232); }
 
 // ---------------------------------------------------------------- mma.sync
-// D (16x8 fp32) += A (16x16 f16, row) * B (16x8 f16, col).
+// D (16x8 fp32) += A (16x16 f16, row) * B (16x8 f16, col).  Not volatile: a
+// register-only operation the compiler may schedule freely (its inputs were
+// loaded before any later reuse of their shared-memory slot).
 __device__ __forceinline__ void mma_16816_f16(float (&d)[4], const uint32_t (&a)[4],
                                               uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
       "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
