@@ -300,6 +300,8 @@ def run_native(args, rank, world, local):
         c = dbg["counts"].cpu().numpy()
         experts_per_input.append(int((c > 0).sum()))
         dense_rows.append(int(c[c >= 128].sum()) if dense else 0)
+    # T >= thr only allows the dense class; it runs when some expert reaches thr rows
+    dense = dense and sum(dense_rows) > 0
     stream = torch.cuda.Stream()
     graphs = []
     with torch.cuda.stream(stream):

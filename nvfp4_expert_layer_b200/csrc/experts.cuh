@@ -46,7 +46,7 @@ namespace moe {
 constexpr int kExpWarps = 4;
 constexpr int kExpThreads = kExpWarps * 32;
 constexpr int kExpSC = 4;          // 64-wide K chunks per bulk-copy stage (2304 bytes)
-constexpr int kExpRing = 6;        // stages in flight per warp
+constexpr int kExpRing = 4;        // bulk-copy stage slots per warp (RT row tiles share RT slots)
 constexpr int kExpSB = kExpSC * kChunkBytes;
 constexpr int kExpSmemJobs = 512;  // job table copied to shared memory when it fits
 
@@ -238,12 +238,57 @@ __device__ __forceinline__ void mma_stage(uint32_t st, int nch, int lane, int g,
 }
 
 
+// One stage of a one-n-tile work tile (NT = 1, RT row tiles sharing the
+// activation fragments).  The activation fragments are loaded per chunk, not
+// a stage ahead: 8 registers instead of 64, which lets four blocks share an
+// SM; their latency (an L1 hit for x, L2 for h) is covered by the other warps.
+template <int RT, bool COHERENT>
+__device__ __forceinline__ void mma_stage_jit(uint32_t st, int nch, int lane, int g, const __half* brow,
+                                              int chunk0, int c, float (&acc)[RT][4][1][4]) {
+  constexpr int NU = kExpSC * RT;
+  auto unit_addr = [&](int u) { return st + (u % RT) * kExpSB + (u / RT) * kChunkBytes; };
+  uint4 codes_n = ld_shared_v4(unit_addr(0) + lane * 16);
+  uint2 sc_n = ld_shared_v2(unit_addr(0) + kChunkCodeBytes + g * 8);
+  uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int u = 0; u < NU; ++u) {
+    const int ch = u / RT, rt = u % RT;
+    if (ch >= nch) break;
+    if (rt == 0 && brow != nullptr) {
+      const __half* bp = brow + (size_t)(chunk0 + ch) * kChunkK + c * 16;
+      lo = COHERENT ? ldg_cg_v4(bp) : ldg_nc_v4(bp);
+      hi = COHERENT ? ldg_cg_v4(bp + 8) : ldg_nc_v4(bp + 8);
+    }
+    const uint4 codes = codes_n;
+    const uint2 sc = sc_n;
+    if (u + 1 < NU && (u + 1) / RT < nch) {
+      codes_n = ld_shared_v4(unit_addr(u + 1) + lane * 16);
+      sc_n = ld_shared_v2(unit_addr(u + 1) + kChunkCodeBytes + g * 8);
+    }
+    const uint32_t cw[4] = {codes.x, codes.y, codes.z, codes.w};
+    const uint32_t sAB[4] = {e4m3_pair_f16x2<0>(sc.x, sc.y), e4m3_pair_f16x2<1>(sc.x, sc.y),
+                             e4m3_pair_f16x2<2>(sc.x, sc.y), e4m3_pair_f16x2<3>(sc.x, sc.y)};
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      uint32_t a[4];
+      e2m1x8_to_f16x2x4(cw[ks], a);
+      a[0] = hmul2_bcast_lo(a[0], sAB[ks]);
+      a[1] = hmul2_bcast_hi(a[1], sAB[ks]);
+      a[2] = hmul2_bcast_lo(a[2], sAB[ks]);
+      a[3] = hmul2_bcast_hi(a[3], sAB[ks]);
+      const uint32_t b0 = ks == 0 ? lo.x : ks == 1 ? lo.z : ks == 2 ? hi.x : hi.z;
+      const uint32_t b1 = ks == 0 ? lo.y : ks == 1 ? lo.w : ks == 2 ? hi.y : hi.w;
+      mma_16816_f16(acc[rt][ks][0], a, b0, b1);
+    }
+  }
+}
+
 // NT = 8-wide n-tiles per job: expert_kernel<1> runs jobs of <= 8 rows,
 // expert_kernel<2> jobs of 9..16 rows; each has its own job list and counters.
 // With one n-tile a work tile is two 16-row tiles (RT = 2) that share the
 // activation fragments, the loop control and the epilogue barrier.
 template <int NT>
-__global__ void __launch_bounds__(kExpThreads, 3) expert_kernel(ExpertParams p) {
+__global__ void __launch_bounds__(kExpThreads, NT == 1 ? 4 : 3) expert_kernel(ExpertParams p) {
   constexpr int RT = NT == 1 ? 2 : 1;
   constexpr int RING = kExpRing / RT;          // stages in flight per warp (same bytes)
   constexpr int SLOT = RT * kExpSB;
@@ -314,7 +359,6 @@ __global__ void __launch_bounds__(kExpThreads, 3) expert_kernel(ExpertParams p) 
 
   bool failed = false;
   int consumed = 0;
-  BFrag<1> b1cur, b1nxt;
   BFrag<2> b2;
 
   // B rows of this lane (row n = nt*8 + g of the job), resolved one tile ahead
@@ -363,7 +407,7 @@ __global__ void __launch_bounds__(kExpThreads, 3) expert_kernel(ExpertParams p) 
 
     float part[2][4];                    // this warp's partial sums, per unit u = rt * NT + nt
     if constexpr (NT == 1) {
-      // one n-tile, two row tiles: activation fragments double-buffered one stage ahead
+      // one n-tile, two row tiles
       float acc[RT][4][1][4];
 #pragma unroll
       for (int rt = 0; rt < RT; ++rt)
@@ -371,32 +415,22 @@ __global__ void __launch_bounds__(kExpThreads, 3) expert_kernel(ExpertParams p) 
         for (int a = 0; a < 4; ++a)
 #pragma unroll
           for (int q = 0; q < 4; ++q) acc[rt][a][0][q] = 0.f;
-      auto load1 = [&](BFrag<1>& bf, int s) {
-        const int n1 = min(kExpSC, ti.cpt - kExpSC * s);
-        if (ti.down) load_bfrag<1, true>(bf, row, kExpSC * s, n1, c);
-        else load_bfrag<1, false>(bf, row, kExpSC * s, n1, c);
-      };
-      auto step1 = [&](const BFrag<1>& bf, int s) {
+      for (int ss = 0; ss < ti.nw; ++ss) {
+        const int s = ti.slo + ss;
         const int nch = min(kExpSC, ti.cpt - kExpSC * s);
         const int slot = consumed % RING;
         if (!failed && !mbar_wait_until(bars_s + 8 * slot, (consumed / RING) & 1, deadline)) {
           failed = true;
           set_error(p.err, kErrTimeout);
         }
-        if (!failed) mma_stage<1, RT>(ring_s + slot * SLOT, nch, lane, g, bf, ti.nrows, acc);
+        if (!failed) {
+          if (ti.down) mma_stage_jit<RT, true>(ring_s + slot * SLOT, nch, lane, g, row[0], kExpSC * s, c, acc);
+          else mma_stage_jit<RT, false>(ring_s + slot * SLOT, nch, lane, g, row[0], kExpSC * s, c, acc);
+        }
         __syncwarp();
         ++consumed;
         if (lane == 0 && !failed) produce(consumed);
-      };
-      if (ti.nw > 0) load1(b1cur, ti.slo);
-      int ss = 0;
-      for (; ss + 1 < ti.nw; ss += 2) {
-        load1(b1nxt, ti.slo + ss + 1);
-        step1(b1cur, ti.slo + ss);
-        if (ss + 2 < ti.nw) load1(b1cur, ti.slo + ss + 2);
-        step1(b1nxt, ti.slo + ss + 1);
       }
-      if (ss < ti.nw) step1(b1cur, ti.slo + ss);
 #pragma unroll
       for (int rt = 0; rt < 2; ++rt)
 #pragma unroll

@@ -781,25 +781,42 @@ __global__ void __launch_bounds__(1024) route_kernel(
   }
   for (int t0 = 0; t0 < T; t0 += 32) {
     const int tn = min(32, T - t0);
-    for (int tt = 0; tt < tn; ++tt) {
-      const uint16_t* xr = x + (size_t)(t0 + tt) * d;
-      float acc = 0.f;
+    // four tokens per pass: their x loads are in flight together (the loop is
+    // latency-bound, not issue-bound); each token's sum keeps the same order
+    for (int tt = 0; tt < tn; tt += 4) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
         if (has[q]) {
-          const uint4 xv = *reinterpret_cast<const uint4*>(xr + 8 * (threadIdx.x + q * blockDim.x));
-          acc = fmaf(__uint_as_float(xv.x << 16), wa[q].x, acc);
-          acc = fmaf(__uint_as_float(xv.x & 0xffff0000u), wa[q].y, acc);
-          acc = fmaf(__uint_as_float(xv.y << 16), wa[q].z, acc);
-          acc = fmaf(__uint_as_float(xv.y & 0xffff0000u), wa[q].w, acc);
-          acc = fmaf(__uint_as_float(xv.z << 16), wb[q].x, acc);
-          acc = fmaf(__uint_as_float(xv.z & 0xffff0000u), wb[q].y, acc);
-          acc = fmaf(__uint_as_float(xv.w << 16), wb[q].z, acc);
-          acc = fmaf(__uint_as_float(xv.w & 0xffff0000u), wb[q].w, acc);
+          uint4 xv[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            xv[j] = tt + j < tn ? *reinterpret_cast<const uint4*>(x + (size_t)(t0 + tt + j) * d +
+                                                                  8 * (threadIdx.x + q * blockDim.x))
+                                : make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            float a = acc[j];
+            a = fmaf(__uint_as_float(xv[j].x << 16), wa[q].x, a);
+            a = fmaf(__uint_as_float(xv[j].x & 0xffff0000u), wa[q].y, a);
+            a = fmaf(__uint_as_float(xv[j].y << 16), wa[q].z, a);
+            a = fmaf(__uint_as_float(xv[j].y & 0xffff0000u), wa[q].w, a);
+            a = fmaf(__uint_as_float(xv[j].z << 16), wb[q].x, a);
+            a = fmaf(__uint_as_float(xv[j].z & 0xffff0000u), wb[q].y, a);
+            a = fmaf(__uint_as_float(xv[j].w << 16), wb[q].z, a);
+            a = fmaf(__uint_as_float(xv[j].w & 0xffff0000u), wb[q].w, a);
+            acc[j] = a;
+          }
         }
       }
-      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-      if (lane == 0) s_part[tt * 32 + warp] = acc;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        for (int off = 16; off > 0; off >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
+      if (lane == 0) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (tt + j < tn) s_part[(tt + j) * 32 + warp] = acc[j];
+      }
     }
     __syncthreads();
     if (warp < tn) {                       // warp tt sums the 32 warp partials of token t0 + tt
