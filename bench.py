@@ -385,11 +385,15 @@ def run_native(args, rank, world, local):
     layer(xs[0], rw, out=out)
     torch.cuda.synchronize()
     gpu_out0 = out.view(torch.int16).cpu().numpy().view(np.uint16).copy()
-    # kernels per step: routing (1 fused launch up to 256 tokens, else the
-    # weight split, router, x staging, top-k, 3 permutation kernels), the dense class
+    # kernels per step: routing (up to 256 tokens the router kernel, which for
+    # at most 32 pairs also runs top-k and the permutation, else top-k and 3
+    # permutation kernels follow it; above 256 tokens the weight split, router,
+    # x staging, top-k and 3 permutation kernels), the dense class
     # (quantiser, gather, 2 GEMMs) when T >= thr, the light-class expert
     # kernels (the 9..16-row one only when T >= 9) and the combine
-    launches = (1 if cfg.T <= 256 else 7) + (4 if cfg.T >= 128 else 0) + (2 if cfg.T >= 9 else 1) + 1
+    pairs = cfg.T * cfg.k
+    routing = (1 if pairs <= 32 else 5) if cfg.T <= 256 else 7
+    launches = routing + (4 if cfg.T >= 128 else 0) + (2 if cfg.T >= 9 else 1) + 1
     return dict(cfg=cfg, ms=ms, clk=clk, err=err, stage_ms=stage_ms, dom_ms=dom_ms / n,
                 dom_work=dom_work / n, dense=dense, e2e_ms=e2e_ms, xs_np=xs_np, rw_np=rw_np,
                 gpu_out0=gpu_out0, launches_per_step=launches, stages=layer.STAGES,

@@ -301,10 +301,13 @@ cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, c
 
 size_t permute_smem_bytes(int E) { return moe::permute_smem_ints(E) * 4; }
 
+// Experts per routing block: two when one K group of 8 per thread covers d.
+int route_epb(int d) { return d <= 8192 ? 2 : 1; }
+
 size_t route_smem_bytes(int E, int d, int T, int k) {
   const size_t P = (size_t)T * k;
-  const size_t tail = P <= 32 ? moe::route_small_ids_offset(E, T, k) + 32 : moe::permute_smem_ints(E) + P;
-  return std::max((size_t)d * 4 + 32 * 32 * 4, tail * 4);
+  const size_t tail = P <= 32 ? moe::route_small_ids_offset(E, T, k) + 32 : 0;
+  return std::max((size_t)route_epb(d) * (d + 32 * 32) * 4, tail * 4);
 }
 
 // Largest route_kernel shared memory over every T <= kSmallT.
@@ -343,12 +346,20 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
   const int dense_ok = h->dense_ok ? 1 : 0;
   const int thr = h->dense_ok ? h->thr : INT_MAX;
   const bool run_dense = h->dense_ok && T >= h->thr;
+  const long long P = (long long)T * k;
   if (T <= kSmallT) {
-    // 1-3. router logits, x staging, top-k and permutation in one launch
-    MOE_CUDA(launch(moe::route_kernel, dim3(E), dim3(1024), route_smem_bytes(E, d, T, k), st, false,
-                    xb, rw, T, d, E, k, thr, dense_ok, w.logits, w.x16, w.xscale, w.ids, w.wts, ticket, po));
+    // 1. router logits and x staging; at most 32 pairs: top-k and the
+    // permutation in the same launch
+    const int epb = route_epb(d), tail = P <= 32 ? 1 : 0;
+    const dim3 rgrid((E + epb - 1) / epb);
+    const size_t rsm = route_smem_bytes(E, d, T, k);
+    if (epb == 2)
+      MOE_CUDA(launch(moe::route_kernel<2>, rgrid, dim3(1024), rsm, st, false, xb, rw, T, d, E, k, thr,
+                      dense_ok, tail, w.logits, w.x16, w.xscale, w.ids, w.wts, ticket, po));
+    else
+      MOE_CUDA(launch(moe::route_kernel<1>, rgrid, dim3(1024), rsm, st, false, xb, rw, T, d, E, k, thr,
+                      dense_ok, tail, w.logits, w.x16, w.xscale, w.ids, w.wts, ticket, po));
     MOE_CUDA(mark(h, 1, st));
-    MOE_CUDA(mark(h, 2, st));
   } else {
     // 1. router logits: fp32 weights split into three exact bf16 parts, then
     // the tensor-core GEMM (x bf16 exact products, fp32 accumulation)
@@ -373,11 +384,15 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
     MOE_CUDA(launch(moe::stage_x_kernel, dim3(std::min(T, 8 * h->sm_count)), dim3(256), 0, st, false,
                     xb, T, d, w.x16, w.xscale, h->err));
     MOE_CUDA(mark(h, 1, st));
+  }
+  if (P <= 32 && T <= kSmallT) {
+    MOE_CUDA(mark(h, 2, st));
+  } else {
+    // 2. top-k, a warp per token
     MOE_CUDA(launch(moe::topk_kernel, dim3((T + 7) / 8), dim3(256), 0, st, false,
                     (const float*)w.logits, T, E, k, w.ids, w.wts));
     MOE_CUDA(mark(h, 2, st));
     // 3. permutation: per-block counts, one-block scan and classes, placement
-    const long long P = (long long)T * k;
     const int nb = (int)std::min<long long>(kPermMaxBlocks, std::max<long long>(1, (P + 1023) / 1024));
     MOE_CUDA(launch(moe::perm_hist_kernel, dim3(nb), dim3(1024), (size_t)E * 4, st, false,
                     (const int*)w.ids, P, E, w.perm_bcnt));
@@ -549,7 +564,8 @@ int moe_fp4_create(int E, int top_k, int d, int f, moe_fp4_t** out) {
         smem_attr((const void*)moe::expert_kernel<2>, kExpSmem) != cudaSuccess ||
         smem_attr((const void*)moe::perm_scan_kernel, permute_smem_bytes(E)) != cudaSuccess ||
         smem_attr((const void*)moe::perm_place_kernel, (size_t)32 * E * 4) != cudaSuccess ||
-        smem_attr((const void*)moe::route_kernel, route_smem_max(E, d, top_k)) != cudaSuccess ||
+        smem_attr((const void*)moe::route_kernel<1>, route_smem_max(E, d, top_k)) != cudaSuccess ||
+        smem_attr((const void*)moe::route_kernel<2>, route_smem_max(E, d, top_k)) != cudaSuccess ||
         smem_attr((const void*)moe::dense_gemm_kernel<moe::kDenseGateUp>,
                   moe::dense_smem_size<moe::kDenseGateUp>(E)) != cudaSuccess ||
         smem_attr((const void*)moe::dense_gemm_kernel<moe::kDenseDown>,

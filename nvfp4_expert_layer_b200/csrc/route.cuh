@@ -229,18 +229,17 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 }
 
 // ---------------------------------------------------------------------------
-// Permutation, built by one block of 1024 threads (32 warps).
-// Pairs p = t*k + j in [0, P) are cut into 32 contiguous warp chunks.  Each
-// warp counts its chunk per expert (match_any groups equal experts inside a
-// 32-pair step, so no atomics), the counts are scanned, and a second walk
-// assigns positions in (expert, pair) order -- deterministic and stable.
-// Then the active experts are classed by row count n:
+// Permutation: pairs p = t*k + j in [0, P) are placed in (expert, pair) order
+// -- deterministic and stable -- and the active experts are classed by row
+// count n:
 //   light (n < thr): cut into jobs of 16 rows plus one remainder job; jobs of
 //     <= 8 rows go to list 1 (one 8-wide MMA n-tile), jobs of 9..16 rows to
 //     list 2 (two n-tiles); each list is ordered heavy expert first;
 //   dense (n >= thr): listed by n descending.
-// Shared memory (ints): 32*E (warp counts) + 4*E + 1 (counts, offsets,
-// active list) + 8 scalars.
+// At most 32 pairs: perm_small inside the routing kernel; otherwise three
+// launches (perm_hist_kernel, perm_scan_kernel, perm_place_kernel).
+// Shared memory of the scan (ints): 32*E + 4*E + 1 (counts, offsets, active
+// list) + 8 scalars.
 // ---------------------------------------------------------------------------
 struct PermuteOut {
   int* counts;       // [E]
@@ -262,8 +261,8 @@ struct PermuteOut {
 __host__ __device__ constexpr size_t permute_smem_ints(int E) { return (size_t)36 * E + 1 + 8; }
 
 // Expert classes over the active experts (light jobs, dense list) from the
-// counts, offsets and active list in shared memory (layout of
-// build_permutation); writes the job lists, the dense list and the scalars.
+// counts, offsets and active list in shared memory (the layout of
+// permute_smem_ints); writes the job lists, the dense list and the scalars.
 __device__ void perm_classes(int E, int thr, int dense_supported, const PermuteOut& o, int* sm) {
   int* cnt = sm + 32 * E;
   int* off = cnt + E;
@@ -318,83 +317,6 @@ __device__ void perm_classes(int E, int thr, int dense_supported, const PermuteO
     *o.dense_pad_total = misc[5];
     if (misc[3] > 0 && !dense_supported) set_error(o.err, kErrUnsupported);
   }
-}
-
-__device__ void build_permutation(const int* ids, int T, int k, int E, int thr, int dense_supported,
-                                  const PermuteOut& o, int* sm) {
-  int* wc = sm;                 // [32][E]
-  int* cnt = wc + 32 * E;       // [E]
-  int* off = cnt + E;           // [E+1]
-  int* act = off + E + 1;       // [E]  active experts, ascending
-  int* misc = act + E;          // [8]  0: n_active 1: n_jobs1 2: n_jobs2 3: n_dense
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const long long P = (long long)T * k;
-  const long long c0 = P * warp / 32, c1 = P * (warp + 1) / 32;
-  for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) wc[i] = 0;
-  if (threadIdx.x < 8) misc[threadIdx.x] = 0;
-  __syncthreads();
-  for (long long base = c0; base < c1; base += 32) {          // pass 1: counts
-    const long long idx = base + lane;
-    const bool valid = idx < c1;
-    const int e = valid ? ids[idx] : -1;
-    const unsigned mask = __match_any_sync(0xffffffffu, e);
-    if (valid && lane == __ffs(mask) - 1 && e >= 0 && e < E) wc[warp * E + e] += __popc(mask);
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int s = 0;
-    for (int w = 0; w < 32; ++w) s += wc[w * E + e];
-    cnt[e] = s;
-  }
-  __syncthreads();
-  if (warp == 0) {              // exclusive scan of the counts; compaction of active experts
-    int carry = 0, acarry = 0;
-    for (int b = 0; b < E; b += 32) {
-      const int e = b + lane;
-      const int v = e < E ? cnt[e] : 0;
-      int incl = v;
-      for (int d = 1; d < 32; d <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, incl, d);
-        if (lane >= d) incl += n;
-      }
-      if (e < E) off[e] = carry + incl - v;
-      carry += __shfl_sync(0xffffffffu, incl, 31);
-      const unsigned am = __ballot_sync(0xffffffffu, v > 0);
-      if (v > 0) act[acarry + __popc(am & ((1u << lane) - 1u))] = e;
-      acarry += __popc(am);
-    }
-    if (lane == 0) { off[E] = carry; misc[0] = acarry; }
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int run = off[e];
-    for (int w = 0; w < 32; ++w) {
-      const int c = wc[w * E + e];
-      wc[w * E + e] = run;
-      run += c;
-    }
-    o.counts[e] = cnt[e];
-    o.offsets[e] = off[e];
-  }
-  if (threadIdx.x == 0) o.offsets[E] = off[E];
-  __syncthreads();
-  const unsigned lt = (1u << lane) - 1u;
-  for (long long base = c0; base < c1; base += 32) {          // pass 2: positions
-    const long long idx = base + lane;
-    const bool valid = idx < c1;
-    const int e = valid ? ids[idx] : -1;
-    const unsigned mask = __match_any_sync(0xffffffffu, e);
-    const bool ok = valid && e >= 0 && e < E;
-    if (ok) {
-      const int pos = wc[warp * E + e] + __popc(mask & lt);
-      o.perm[pos] = (int)idx;
-      o.inv[idx] = pos;
-    }
-    __syncwarp();
-    if (ok && lane == __ffs(mask) - 1) wc[warp * E + e] += __popc(mask);
-    __syncwarp();
-  }
-  perm_classes(E, thr, dense_supported, o, sm);
 }
 
 // ---------------------------------------------------------------------------
@@ -524,8 +446,8 @@ __device__ __forceinline__ uint32_t warp_scan_u32(uint32_t v, int lane) {
 }
 
 // Permutation and classes of at most 32 pairs (ids in shared memory, padded
-// with -1 to 32 entries), with the results of build_permutation +
-// perm_classes (E <= 1024, so an expert fits 10 bits).  Threads 32.. write
+// with -1 to 32 entries), with the results of the three-launch permutation
+// and perm_classes (E <= 1024, so an expert fits 10 bits).  Threads 32.. write
 // the count and offset of every expert.  Warp 0 sorts the pair keys
 // (expert, pair): lane i then holds permuted row i, so perm and inv follow
 // directly, and the runs of equal experts give each active expert its row
@@ -621,8 +543,8 @@ __device__ void perm_small(const int* ids, int E, int thr, int dense_supported, 
 //                      classes, and bcnt turned into per-block bases
 //                      off[e] + sum over earlier blocks;
 //   perm_place_kernel: per block, per-warp counts on top of the block base,
-//                      then positions in (expert, pair) order as in
-//                      build_permutation -- the same stable order.
+//                      then positions in (expert, pair) order (match_any
+//                      groups equal experts inside a 32-pair step).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) perm_hist_kernel(const int* __restrict__ ids, long long P, int E,
                                                          int* __restrict__ bcnt) {
@@ -731,29 +653,35 @@ __global__ void __launch_bounds__(1024) perm_place_kernel(const int* __restrict_
   }
 }
 
-// Small-T routing in one launch.  Block e (1024 threads) computes the fp32
-// logits of expert e for every token (its router row is staged in shared
-// memory, one warp per token) and stages x rows t = e, e + E, ... in fp16.
-// The last block to finish (an atomic ticket; no grid barrier) runs the
-// routing tail: top-k and the permutation (at most 32 pairs: the ranked
-// top-k and perm_small; otherwise a warp per token and build_permutation),
-// then clears the ticket for the next launch.  Dynamic shared memory: the
-// largest of d + 1024 floats (router row and warp partials), the small path's
-// route_small_ids_offset + 32 ints, or permute_smem_ints(E) + T*k ints.
+// Small-T router logits (T <= 256) and x staging in one launch, plus the
+// routing tail for at most 32 (token, expert) pairs.  Block b (1024 threads)
+// computes the fp32 logits of experts EPB*b .. EPB*b + EPB-1 for every token:
+// the router rows are staged in shared memory, thread i owns K = [8i, 8i+8)
+// (and [8(i+1024), ...) when d > 8192, EPB = 1), so one x load feeds EPB
+// experts; per token the 32 warp sums meet in shared memory.  Blocks also
+// stage x rows t = b, b + grid, ... in fp16.  With tail != 0 the last block
+// to finish (an atomic ticket; no grid barrier) runs the ranked top-k and the
+// small permutation, then clears the ticket for the next launch.  Dynamic
+// shared memory: the larger of EPB * (d + 1024) floats and, with the tail,
+// route_small_ids_offset + 32 ints.
+template <int EPB>
 __global__ void __launch_bounds__(1024) route_kernel(
     const uint16_t* __restrict__ x, const float* __restrict__ rw, int T, int d, int E, int k,
-    int thr, int dense_supported, float* __restrict__ logits, __half* __restrict__ x16,
+    int thr, int dense_supported, int tail, float* __restrict__ logits, __half* __restrict__ x16,
     float* __restrict__ xscale, int* __restrict__ ids_out, float* __restrict__ wts,
     int* __restrict__ ticket, PermuteOut o) {
+  constexpr int NG = 2 / EPB;                           // K groups of 8 per thread
   extern __shared__ __align__(16) int sm[];
   __shared__ float red[33];
   __shared__ int s_last;
-  const int e = blockIdx.x;
+  const int e0 = blockIdx.x * EPB;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  float* s_w = reinterpret_cast<float*>(sm);
-  {
+  float* s_w = reinterpret_cast<float*>(sm);            // [EPB][d]
+#pragma unroll
+  for (int j = 0; j < EPB; ++j) {
+    if (e0 + j >= E) break;
     // d <= 16384: at most 4 float4 per thread, all loads issued before the stores
-    const float4* src = reinterpret_cast<const float4*>(rw + (size_t)e * d);
+    const float4* src = reinterpret_cast<const float4*>(rw + (size_t)(e0 + j) * d);
     float4 v[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -763,72 +691,92 @@ __global__ void __launch_bounds__(1024) route_kernel(
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int i = threadIdx.x + q * blockDim.x;
-      if (i < d / 4) reinterpret_cast<float4*>(s_w)[i] = v[q];
+      if (i < d / 4) reinterpret_cast<float4*>(s_w + (size_t)j * d)[i] = v[q];
     }
   }
   __syncthreads();
-  // every thread owns up to 2 groups of 8 consecutive K (d <= 16384); per token
-  // the 32 warp sums meet in shared memory (tokens in batches of 32)
-  float* s_part = reinterpret_cast<float*>(sm) + d;     // [32 tokens][32 warps]
-  float4 wa[2], wb[2];
-  bool has[2];
+  float* s_part = s_w + (size_t)EPB * d;                // [EPB][32 tokens][32 warps]
+  float4 wa[EPB][NG], wb[EPB][NG];
+  bool has[NG];
 #pragma unroll
-  for (int q = 0; q < 2; ++q) {
+  for (int q = 0; q < NG; ++q) {
     const int kk = 8 * (threadIdx.x + q * blockDim.x);
     has[q] = kk < d;
-    wa[q] = has[q] ? *reinterpret_cast<const float4*>(s_w + kk) : make_float4(0, 0, 0, 0);
-    wb[q] = has[q] ? *reinterpret_cast<const float4*>(s_w + kk + 4) : make_float4(0, 0, 0, 0);
+#pragma unroll
+    for (int j = 0; j < EPB; ++j) {
+      const bool ok = has[q] && e0 + j < E;
+      wa[j][q] = ok ? *reinterpret_cast<const float4*>(s_w + (size_t)j * d + kk) : make_float4(0, 0, 0, 0);
+      wb[j][q] = ok ? *reinterpret_cast<const float4*>(s_w + (size_t)j * d + kk + 4) : make_float4(0, 0, 0, 0);
+    }
   }
   for (int t0 = 0; t0 < T; t0 += 32) {
     const int tn = min(32, T - t0);
     // four tokens per pass: their x loads are in flight together (the loop is
     // latency-bound, not issue-bound); each token's sum keeps the same order
     for (int tt = 0; tt < tn; tt += 4) {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      float acc[EPB][4];
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
+      for (int j = 0; j < EPB; ++j)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) acc[j][u] = 0.f;
+#pragma unroll
+      for (int q = 0; q < NG; ++q) {
         if (has[q]) {
           uint4 xv[4];
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            xv[j] = tt + j < tn ? *reinterpret_cast<const uint4*>(x + (size_t)(t0 + tt + j) * d +
+          for (int u = 0; u < 4; ++u)
+            xv[u] = tt + u < tn ? *reinterpret_cast<const uint4*>(x + (size_t)(t0 + tt + u) * d +
                                                                   8 * (threadIdx.x + q * blockDim.x))
                                 : make_uint4(0, 0, 0, 0);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            float a = acc[j];
-            a = fmaf(__uint_as_float(xv[j].x << 16), wa[q].x, a);
-            a = fmaf(__uint_as_float(xv[j].x & 0xffff0000u), wa[q].y, a);
-            a = fmaf(__uint_as_float(xv[j].y << 16), wa[q].z, a);
-            a = fmaf(__uint_as_float(xv[j].y & 0xffff0000u), wa[q].w, a);
-            a = fmaf(__uint_as_float(xv[j].z << 16), wb[q].x, a);
-            a = fmaf(__uint_as_float(xv[j].z & 0xffff0000u), wb[q].y, a);
-            a = fmaf(__uint_as_float(xv[j].w << 16), wb[q].z, a);
-            a = fmaf(__uint_as_float(xv[j].w & 0xffff0000u), wb[q].w, a);
-            acc[j] = a;
+          for (int u = 0; u < 4; ++u) {
+#pragma unroll
+            for (int j = 0; j < EPB; ++j) {
+              float a = acc[j][u];
+              a = fmaf(__uint_as_float(xv[u].x << 16), wa[j][q].x, a);
+              a = fmaf(__uint_as_float(xv[u].x & 0xffff0000u), wa[j][q].y, a);
+              a = fmaf(__uint_as_float(xv[u].y << 16), wa[j][q].z, a);
+              a = fmaf(__uint_as_float(xv[u].y & 0xffff0000u), wa[j][q].w, a);
+              a = fmaf(__uint_as_float(xv[u].z << 16), wb[j][q].x, a);
+              a = fmaf(__uint_as_float(xv[u].z & 0xffff0000u), wb[j][q].y, a);
+              a = fmaf(__uint_as_float(xv[u].w << 16), wb[j][q].z, a);
+              a = fmaf(__uint_as_float(xv[u].w & 0xffff0000u), wb[j][q].w, a);
+              acc[j][u] = a;
+            }
           }
         }
       }
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        for (int off = 16; off > 0; off >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
+      for (int j = 0; j < EPB; ++j)
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          for (int off = 16; off > 0; off >>= 1) acc[j][u] += __shfl_xor_sync(0xffffffffu, acc[j][u], off);
       if (lane == 0) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (tt + j < tn) s_part[(tt + j) * 32 + warp] = acc[j];
+        for (int j = 0; j < EPB; ++j)
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (tt + u < tn) s_part[((size_t)j * 32 + tt + u) * 32 + warp] = acc[j][u];
       }
     }
     __syncthreads();
     if (warp < tn) {                       // warp tt sums the 32 warp partials of token t0 + tt
-      float v = s_part[warp * 32 + lane];
-      for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-      if (lane == 0) logits[(size_t)(t0 + warp) * E + e] = v;
+#pragma unroll
+      for (int j = 0; j < EPB; ++j) {
+        float v = s_part[((size_t)j * 32 + warp) * 32 + lane];
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (lane == 0 && e0 + j < E) logits[(size_t)(t0 + warp) * E + e0 + j] = v;
+      }
     }
     __syncthreads();
   }
-  for (int t = e; t < T; t += gridDim.x)
+  for (int t = blockIdx.x; t < T; t += gridDim.x)
     stage_x_row(x + (size_t)t * d, d, x16 + (size_t)t * d, xscale + t, o.err, red);
-  // ---- last block: routing tail
+  if (!tail) {
+    pdl_launch_dependents();
+    return;
+  }
+  // ---- last block: routing tail (at most 32 pairs)
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
@@ -837,38 +785,13 @@ __global__ void __launch_bounds__(1024) route_kernel(
   }
   __syncthreads();
   if (!s_last) return;
-  if ((long long)T * k <= 32) {
-    // decode: ranked top-k (scratch from the start of shared memory, the pair
-    // experts after it), then the small permutation
-    int* ids_small = sm + route_small_ids_offset(E, T, k);
-    topk_small_block(logits, T, E, k, ids_small, ids_out, wts, reinterpret_cast<uint32_t*>(sm));
-    if (threadIdx.x >= T * k && threadIdx.x < 32) ids_small[threadIdx.x] = -1;
-    __syncthreads();
-    perm_small(ids_small, E, thr, dense_supported, o);
-    if (threadIdx.x == 0) *ticket = 0;
-    return;
-  }
-  int* ids_s = sm + permute_smem_ints(E);
-  for (int t = warp; t < T; t += 32) {
-    float v[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int ee = lane + 32 * i;
-      float l = -INFINITY;
-      if (ee < E) asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(l) : "l"(logits + (size_t)t * E + ee));
-      v[i] = l;
-    }
-    int my_e;
-    float my_w;
-    topk_warp(v, E, k, lane, my_e, my_w);
-    if (lane < k) {
-      ids_s[t * k + lane] = my_e;
-      ids_out[(size_t)t * k + lane] = my_e;
-      wts[(size_t)t * k + lane] = my_w;
-    }
-  }
+  // ranked top-k (scratch from the start of shared memory, the pair experts
+  // after it), then the small permutation
+  int* ids_small = sm + route_small_ids_offset(E, T, k);
+  topk_small_block(logits, T, E, k, ids_small, ids_out, wts, reinterpret_cast<uint32_t*>(sm));
+  if (threadIdx.x >= T * k && threadIdx.x < 32) ids_small[threadIdx.x] = -1;
   __syncthreads();
-  build_permutation(ids_s, T, k, E, thr, dense_supported, o, sm);
+  perm_small(ids_small, E, thr, dense_supported, o);
   if (threadIdx.x == 0) *ticket = 0;
 }
 
