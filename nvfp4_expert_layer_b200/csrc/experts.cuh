@@ -238,26 +238,41 @@ __device__ __forceinline__ void mma_stage(uint32_t st, int nch, int lane, int g,
 }
 
 
+// Activation fragment (two 16-byte halves) of one 64-wide chunk for lane c.
+template <bool COHERENT>
+__device__ __forceinline__ void load_bchunk(const __half* brow, int chunk, int c, uint4& lo, uint4& hi) {
+  if (brow == nullptr) {
+    lo = make_uint4(0, 0, 0, 0);
+    hi = lo;
+    return;
+  }
+  const __half* bp = brow + (size_t)chunk * kChunkK + c * 16;
+  lo = COHERENT ? ldg_cg_v4(bp) : ldg_nc_v4(bp);
+  hi = COHERENT ? ldg_cg_v4(bp + 8) : ldg_nc_v4(bp + 8);
+}
+
 // One stage of a one-n-tile work tile (NT = 1, RT row tiles sharing the
-// activation fragments).  The activation fragments are loaded per chunk, not
-// a stage ahead: 8 registers instead of 64, which lets four blocks share an
-// SM; their latency (an L1 hit for x, L2 for h) is covered by the other warps.
+// activation fragments).  The activation fragments are not held a stage
+// ahead (64 registers) but one chunk ahead (8): (blo, bhi) holds chunk0's on
+// entry and the next chunk's on exit when `more` says the warp's next stage
+// of this tile follows; that lets four blocks share an SM.
 template <int RT, bool COHERENT>
 __device__ __forceinline__ void mma_stage_jit(uint32_t st, int nch, int lane, int g, const __half* brow,
-                                              int chunk0, int c, float (&acc)[RT][4][1][4]) {
+                                              int chunk0, int c, bool more, uint4& blo, uint4& bhi,
+                                              float (&acc)[RT][4][1][4]) {
   constexpr int NU = kExpSC * RT;
   auto unit_addr = [&](int u) { return st + (u % RT) * kExpSB + (u / RT) * kChunkBytes; };
   uint4 codes_n = ld_shared_v4(unit_addr(0) + lane * 16);
   uint2 sc_n = ld_shared_v2(unit_addr(0) + kChunkCodeBytes + g * 8);
-  uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
+  uint4 lo = blo, hi = bhi;
 #pragma unroll
   for (int u = 0; u < NU; ++u) {
     const int ch = u / RT, rt = u % RT;
     if (ch >= nch) break;
-    if (rt == 0 && brow != nullptr) {
-      const __half* bp = brow + (size_t)(chunk0 + ch) * kChunkK + c * 16;
-      lo = COHERENT ? ldg_cg_v4(bp) : ldg_nc_v4(bp);
-      hi = COHERENT ? ldg_cg_v4(bp + 8) : ldg_nc_v4(bp + 8);
+    if (rt == 0) {
+      lo = blo;
+      hi = bhi;
+      if (ch + 1 < nch || more) load_bchunk<COHERENT>(brow, chunk0 + ch + 1, c, blo, bhi);
     }
     const uint4 codes = codes_n;
     const uint2 sc = sc_n;
@@ -415,17 +430,25 @@ __global__ void __launch_bounds__(kExpThreads, NT == 1 ? 4 : 3) expert_kernel(Ex
         for (int a = 0; a < 4; ++a)
 #pragma unroll
           for (int q = 0; q < 4; ++q) acc[rt][a][0][q] = 0.f;
+      uint4 blo, bhi;
+      if (ti.nw > 0) {
+        if (ti.down) load_bchunk<true>(row[0], kExpSC * ti.slo, c, blo, bhi);
+        else load_bchunk<false>(row[0], kExpSC * ti.slo, c, blo, bhi);
+      }
       for (int ss = 0; ss < ti.nw; ++ss) {
         const int s = ti.slo + ss;
         const int nch = min(kExpSC, ti.cpt - kExpSC * s);
+        const bool more = ss + 1 < ti.nw;
         const int slot = consumed % RING;
         if (!failed && !mbar_wait_until(bars_s + 8 * slot, (consumed / RING) & 1, deadline)) {
           failed = true;
           set_error(p.err, kErrTimeout);
         }
         if (!failed) {
-          if (ti.down) mma_stage_jit<RT, true>(ring_s + slot * SLOT, nch, lane, g, row[0], kExpSC * s, c, acc);
-          else mma_stage_jit<RT, false>(ring_s + slot * SLOT, nch, lane, g, row[0], kExpSC * s, c, acc);
+          if (ti.down)
+            mma_stage_jit<RT, true>(ring_s + slot * SLOT, nch, lane, g, row[0], kExpSC * s, c, more, blo, bhi, acc);
+          else
+            mma_stage_jit<RT, false>(ring_s + slot * SLOT, nch, lane, g, row[0], kExpSC * s, c, more, blo, bhi, acc);
         }
         __syncwarp();
         ++consumed;
