@@ -197,7 +197,7 @@ __device__ __forceinline__ uint32_t hmul2_bcast_hi(uint32_t a, uint32_t s) {
 // One stage of shared-memory weights times the lane's activation fragments.
 // The codes and scales of the next (chunk, row tile) are loaded before the
 // current one is converted, so the shared-memory latency overlaps the math.
-template <int NT, int RT>
+template <int NT, int RT, bool FULL>
 __device__ __forceinline__ void mma_stage(uint32_t st, int nch, int lane, int g, const BFrag<NT>& b,
                                           int nrows, float (&acc)[RT][4][NT][4]) {
   constexpr int NU = kExpSC * RT;                   // (chunk, row tile) units, chunk-major
@@ -207,10 +207,10 @@ __device__ __forceinline__ void mma_stage(uint32_t st, int nch, int lane, int g,
 #pragma unroll
   for (int u = 0; u < NU; ++u) {
     const int ch = u / RT, rt = u % RT;
-    if (ch >= nch) break;
+    if (!FULL && ch >= nch) break;
     const uint4 codes = codes_n;
     const uint2 sc = sc_n;
-    if (u + 1 < NU && (u + 1) / RT < nch) {
+    if (u + 1 < NU && (FULL || (u + 1) / RT < nch)) {
       codes_n = ld_shared_v4(unit_addr(u + 1) + lane * 16);
       sc_n = ld_shared_v2(unit_addr(u + 1) + kChunkCodeBytes + g * 8);
     }
@@ -256,27 +256,35 @@ __device__ __forceinline__ void load_bchunk(const __half* brow, int chunk, int c
 // ahead (64 registers) but one chunk ahead (8): (blo, bhi) holds chunk0's on
 // entry and the next chunk's on exit when `more` says the warp's next stage
 // of this tile follows; that lets four blocks share an SM.
-template <int RT, bool COHERENT>
+template <int RT, bool COHERENT, bool FULL>
 __device__ __forceinline__ void mma_stage_jit(uint32_t st, int nch, int lane, int g, const __half* brow,
                                               int chunk0, int c, bool more, uint4& blo, uint4& bhi,
                                               float (&acc)[RT][4][1][4]) {
+  // FULL: all kExpSC chunks present (no per-chunk bounds).  The fragments of
+  // even chunks live in (blo, bhi), those of odd chunks in (olo, ohi): each
+  // chunk prefetches the next one into the other pair, so a full stage ends
+  // with the next stage's first chunk in (blo, bhi) and nothing is copied.
   constexpr int NU = kExpSC * RT;
   auto unit_addr = [&](int u) { return st + (u % RT) * kExpSB + (u / RT) * kChunkBytes; };
   uint4 codes_n = ld_shared_v4(unit_addr(0) + lane * 16);
   uint2 sc_n = ld_shared_v2(unit_addr(0) + kChunkCodeBytes + g * 8);
-  uint4 lo = blo, hi = bhi;
+  uint4 olo = make_uint4(0, 0, 0, 0), ohi = olo;
 #pragma unroll
   for (int u = 0; u < NU; ++u) {
     const int ch = u / RT, rt = u % RT;
-    if (ch >= nch) break;
+    if (!FULL && ch >= nch) break;
     if (rt == 0) {
-      lo = blo;
-      hi = bhi;
-      if (ch + 1 < nch || more) load_bchunk<COHERENT>(brow, chunk0 + ch + 1, c, blo, bhi);
+      const bool pf = FULL ? (ch + 1 < kExpSC || more) : (ch + 1 < nch || more);
+      if (pf) {
+        if (ch & 1) load_bchunk<COHERENT>(brow, chunk0 + ch + 1, c, blo, bhi);
+        else load_bchunk<COHERENT>(brow, chunk0 + ch + 1, c, olo, ohi);
+      }
     }
+    const uint4& lo = (ch & 1) ? olo : blo;
+    const uint4& hi = (ch & 1) ? ohi : bhi;
     const uint4 codes = codes_n;
     const uint2 sc = sc_n;
-    if (u + 1 < NU && (u + 1) / RT < nch) {
+    if (u + 1 < NU && (FULL || (u + 1) / RT < nch)) {
       codes_n = ld_shared_v4(unit_addr(u + 1) + lane * 16);
       sc_n = ld_shared_v2(unit_addr(u + 1) + kChunkCodeBytes + g * 8);
     }
@@ -338,35 +346,37 @@ __global__ void __launch_bounds__(kExpThreads, NT == 1 ? 4 : 3) expert_kernel(Ex
   }
   __syncwarp();
 
-  // ---- producer state (lane 0 of each warp): walks this warp's stages in order
-  int c_it = 0, c_s = 0, issued = 0;
-  bool c_valid = false;
-  TileInfo c_ti{};
+  // ---- producer state (lane 0 of each warp): walks this warp's stages in order.
+  // Per tile: the source of the warp's next stage (row tile 0), the distance
+  // between row tiles, the stages left and the chunk count of the last one.
+  static_assert((RING & (RING - 1)) == 0, "ring slots: a power of two");
+  int c_it = 0, c_left = 0, c_nch_last = 0, issued = 0;
+  const uint8_t* c_src = nullptr;
+  size_t c_rt_stride = 0;
   auto cursor_ready = [&]() -> bool {
-    while (true) {
-      if (!c_valid) {
-        if (c_it >= my_tiles) return false;
-        c_ti = tile_info<RT>(p, jobs, b + c_it * G, ngu, warp);
-        c_s = 0;
-        c_valid = true;
-      }
-      if (c_s < c_ti.nw) return true;
-      c_valid = false;
+    while (c_left == 0) {
+      if (c_it >= my_tiles) return false;
+      const TileInfo t = tile_info<RT>(p, jobs, b + c_it * G, ngu, warp);
       ++c_it;
+      c_left = t.nw;
+      c_src = t.base + (size_t)kExpSC * t.slo * kChunkBytes;
+      c_rt_stride = (size_t)t.cpt * kChunkBytes;
+      c_nch_last = t.cpt - kExpSC * (t.slo + t.nw - 1);
+      if (c_nch_last > kExpSC) c_nch_last = kExpSC;
     }
+    return true;
   };
   auto produce = [&](int consumed) {          // keep RING stages in flight
     while (issued < consumed + RING && cursor_ready()) {
-      const int s = c_ti.slo + c_s;
-      const int nch = min(kExpSC, c_ti.cpt - kExpSC * s);
-      const int slot = issued % RING;
+      const int nch = c_left == 1 ? c_nch_last : kExpSC;
+      const int slot = issued & (RING - 1);
       mbar_arrive_expect_tx(bars_s + 8 * slot, RT * nch * kChunkBytes);
 #pragma unroll
       for (int rt = 0; rt < RT; ++rt)
-        bulk_g2s(ring_s + slot * SLOT + rt * kExpSB,
-                 c_ti.base + ((size_t)rt * c_ti.cpt + (size_t)kExpSC * s) * kChunkBytes, nch * kChunkBytes,
+        bulk_g2s(ring_s + slot * SLOT + rt * kExpSB, c_src + rt * c_rt_stride, nch * kChunkBytes,
                  bars_s + 8 * slot, pol);
-      ++c_s;
+      c_src += kExpSC * kChunkBytes;
+      --c_left;
       ++issued;
     }
   };
@@ -439,16 +449,20 @@ __global__ void __launch_bounds__(kExpThreads, NT == 1 ? 4 : 3) expert_kernel(Ex
         const int s = ti.slo + ss;
         const int nch = min(kExpSC, ti.cpt - kExpSC * s);
         const bool more = ss + 1 < ti.nw;
-        const int slot = consumed % RING;
-        if (!failed && !mbar_wait_until(bars_s + 8 * slot, (consumed / RING) & 1, deadline)) {
+        const int slot = consumed & (RING - 1);
+        if (!failed && !mbar_wait_until(bars_s + 8 * slot, ((unsigned)consumed / RING) & 1u, deadline)) {
           failed = true;
           set_error(p.err, kErrTimeout);
         }
         if (!failed) {
-          if (ti.down)
-            mma_stage_jit<RT, true>(ring_s + slot * SLOT, nch, lane, g, row[0], kExpSC * s, c, more, blo, bhi, acc);
-          else
-            mma_stage_jit<RT, false>(ring_s + slot * SLOT, nch, lane, g, row[0], kExpSC * s, c, more, blo, bhi, acc);
+          const uint32_t sp = ring_s + slot * SLOT;
+          if (nch == kExpSC) {
+            if (ti.down) mma_stage_jit<RT, true, true>(sp, nch, lane, g, row[0], kExpSC * s, c, more, blo, bhi, acc);
+            else mma_stage_jit<RT, false, true>(sp, nch, lane, g, row[0], kExpSC * s, c, more, blo, bhi, acc);
+          } else {
+            if (ti.down) mma_stage_jit<RT, true, false>(sp, nch, lane, g, row[0], kExpSC * s, c, more, blo, bhi, acc);
+            else mma_stage_jit<RT, false, false>(sp, nch, lane, g, row[0], kExpSC * s, c, more, blo, bhi, acc);
+          }
         }
         __syncwarp();
         ++consumed;
@@ -472,12 +486,15 @@ __global__ void __launch_bounds__(kExpThreads, NT == 1 ? 4 : 3) expert_kernel(Ex
         const int nch = min(kExpSC, ti.cpt - kExpSC * s);
         if (ti.down) load_bfrag<2, true>(b2, row, kExpSC * s, nch, c);
         else load_bfrag<2, false>(b2, row, kExpSC * s, nch, c);
-        const int slot = consumed % RING;
-        if (!failed && !mbar_wait_until(bars_s + 8 * slot, (consumed / RING) & 1, deadline)) {
+        const int slot = consumed & (RING - 1);
+        if (!failed && !mbar_wait_until(bars_s + 8 * slot, ((unsigned)consumed / RING) & 1u, deadline)) {
           failed = true;
           set_error(p.err, kErrTimeout);
         }
-        if (!failed) mma_stage<2, 1>(ring_s + slot * SLOT, nch, lane, g, b2, ti.nrows, acc);
+        if (!failed) {
+          if (nch == kExpSC) mma_stage<2, 1, true>(ring_s + slot * SLOT, nch, lane, g, b2, ti.nrows, acc);
+          else mma_stage<2, 1, false>(ring_s + slot * SLOT, nch, lane, g, b2, ti.nrows, acc);
+        }
         __syncwarp();
         ++consumed;
         if (lane == 0 && !failed) produce(consumed);
@@ -552,7 +569,7 @@ __global__ void __launch_bounds__(kExpThreads, NT == 1 ? 4 : 3) expert_kernel(Ex
   if (failed && lane == 0) {
     const uint64_t drain = globaltimer_ns() + (uint64_t)p.wait_timeout_ns;
     for (int jj = consumed; jj < issued; ++jj)
-      if (!mbar_wait_until(bars_s + 8 * (jj % RING), (jj / RING) & 1, drain)) break;
+      if (!mbar_wait_until(bars_s + 8 * (jj & (RING - 1)), ((unsigned)jj / RING) & 1u, drain)) break;
   }
   // ---- exit protocol: the last block clears the per-job counters
   __syncthreads();
