@@ -49,6 +49,9 @@ constexpr int kExpSC = 4;          // 64-wide K chunks per bulk-copy stage (2304
 constexpr int kExpRing = 4;        // bulk-copy stage slots per warp (RT row tiles share RT slots)
 constexpr int kExpSB = kExpSC * kChunkBytes;
 constexpr int kExpSmemJobs = 512;  // job table copied to shared memory when it fits
+// fp32 MMA accumulators per (row tile, n-tile): the four K steps of a chunk
+// chain into one (the chains of the row tiles and n-tiles interleave).
+constexpr int kAccK = 1;
 
 struct ExpertParams {
   const uint8_t* gu_frag;     // gate/up fragment layout [E][f/8 tiles][d/64 chunks]
@@ -199,7 +202,7 @@ __device__ __forceinline__ uint32_t hmul2_bcast_hi(uint32_t a, uint32_t s) {
 // current one is converted, so the shared-memory latency overlaps the math.
 template <int NT, int RT, bool FULL>
 __device__ __forceinline__ void mma_stage(uint32_t st, int nch, int lane, int g, const BFrag<NT>& b,
-                                          int nrows, float (&acc)[RT][4][NT][4]) {
+                                          int nrows, float (&acc)[RT][kAccK][NT][4]) {
   constexpr int NU = kExpSC * RT;                   // (chunk, row tile) units, chunk-major
   auto unit_addr = [&](int u) { return st + (u % RT) * kExpSB + (u / RT) * kChunkBytes; };
   uint4 codes_n = ld_shared_v4(unit_addr(0) + lane * 16);
@@ -231,7 +234,7 @@ __device__ __forceinline__ void mma_stage(uint32_t st, int nch, int lane, int g,
         const uint4& hi = b.v[nt][ch][1];
         const uint32_t b0 = ks == 0 ? lo.x : ks == 1 ? lo.z : ks == 2 ? hi.x : hi.z;
         const uint32_t b1 = ks == 0 ? lo.y : ks == 1 ? lo.w : ks == 2 ? hi.y : hi.w;
-        if (NT == 1 || nt * 8 < nrows) mma_16816_f16(acc[rt][ks][nt], a, b0, b1);
+        if (NT == 1 || nt * 8 < nrows) mma_16816_f16(acc[rt][ks % kAccK][nt], a, b0, b1);
       }
     }
   }
@@ -259,7 +262,7 @@ __device__ __forceinline__ void load_bchunk(const __half* brow, int chunk, int c
 template <int RT, bool COHERENT, bool FULL>
 __device__ __forceinline__ void mma_stage_jit(uint32_t st, int nch, int lane, int g, const __half* brow,
                                               int chunk0, int c, bool more, uint4& blo, uint4& bhi,
-                                              float (&acc)[RT][4][1][4]) {
+                                              float (&acc)[RT][kAccK][1][4]) {
   // FULL: all kExpSC chunks present (no per-chunk bounds).  The fragments of
   // even chunks live in (blo, bhi), those of odd chunks in (olo, ohi): each
   // chunk prefetches the next one into the other pair, so a full stage ends
@@ -301,7 +304,7 @@ __device__ __forceinline__ void mma_stage_jit(uint32_t st, int nch, int lane, in
       a[3] = hmul2_bcast_hi(a[3], sAB[ks]);
       const uint32_t b0 = ks == 0 ? lo.x : ks == 1 ? lo.z : ks == 2 ? hi.x : hi.z;
       const uint32_t b1 = ks == 0 ? lo.y : ks == 1 ? lo.w : ks == 2 ? hi.y : hi.w;
-      mma_16816_f16(acc[rt][ks][0], a, b0, b1);
+      mma_16816_f16(acc[rt][ks % kAccK][0], a, b0, b1);
     }
   }
 }
@@ -433,11 +436,11 @@ __global__ void __launch_bounds__(kExpThreads, NT == 1 ? 4 : 3) expert_kernel(Ex
     float part[2][4];                    // this warp's partial sums, per unit u = rt * NT + nt
     if constexpr (NT == 1) {
       // one n-tile, two row tiles
-      float acc[RT][4][1][4];
+      float acc[RT][kAccK][1][4];
 #pragma unroll
       for (int rt = 0; rt < RT; ++rt)
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int a = 0; a < kAccK; ++a)
 #pragma unroll
           for (int q = 0; q < 4; ++q) acc[rt][a][0][q] = 0.f;
       uint4 blo, bhi;
@@ -471,12 +474,16 @@ __global__ void __launch_bounds__(kExpThreads, NT == 1 ? 4 : 3) expert_kernel(Ex
 #pragma unroll
       for (int rt = 0; rt < 2; ++rt)
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          part[rt][q] = (acc[rt][0][0][q] + acc[rt][1][0][q]) + (acc[rt][2][0][q] + acc[rt][3][0][q]);
-    } else {
-      float acc[1][4][2][4];
+        for (int q = 0; q < 4; ++q) {
+          float v = acc[rt][0][0][q];
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+          for (int a = 1; a < kAccK; ++a) v += acc[rt][a][0][q];
+          part[rt][q] = v;
+        }
+    } else {
+      float acc[1][kAccK][2][4];
+#pragma unroll
+      for (int a = 0; a < kAccK; ++a)
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -502,8 +509,12 @@ __global__ void __launch_bounds__(kExpThreads, NT == 1 ? 4 : 3) expert_kernel(Ex
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          part[nt][q] = (acc[0][0][nt][q] + acc[0][1][nt][q]) + (acc[0][2][nt][q] + acc[0][3][nt][q]);
+        for (int q = 0; q < 4; ++q) {
+          float v = acc[0][0][nt][q];
+#pragma unroll
+          for (int a = 1; a < kAccK; ++a) v += acc[0][a][nt][q];
+          part[nt][q] = v;
+        }
     }
 
     // ---- cross-warp reduction of the tile (buffer alternates by tile parity)
