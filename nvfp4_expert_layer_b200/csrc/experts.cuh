@@ -1,6 +1,7 @@
-// Light-class expert phase as one persistent kernel: gate/up + SwiGLU, down
-// (x routing weight) and the combine / unpermute, for every job whose expert
-// received fewer rows than the dense threshold.
+// Light-class expert phase as one persistent kernel: gate/up + SwiGLU and
+// down (x routing weight) into per-pair fp32 partials, for every job whose
+// expert received fewer rows than the dense threshold (the combine /
+// unpermute is the next kernel).
 //
 // The weights stay 4-bit in HBM and shared memory; each warp unpacks e2m1
 // codes and their e4m3 block scales in registers into exact fp16 MMA operands
@@ -25,15 +26,9 @@
 // rows 8t+g, so one accumulator holds g and u of the same f and the SwiGLU
 // epilogue stays in registers.
 //
-// Combine (section 8 of the Muse Spark page: a one-pass combine; every output
-// row written once, no zero fill): every down tile adds its row count to the
-// counter of its 16-row output slice; the block that completes a slice sums
-// the k partials of every token in slot order and writes bf16 once.
-//
-// Counters reset themselves: the combining block clears its slice counter and
-// the last block to leave clears the per-job counters, so a CUDA graph can
-// replay the kernel without a memset.  The permutation kernel guarantees that
-// every job has 1..16 rows.
+// Counters reset themselves: the last block to leave clears the per-job
+// counters, so a CUDA graph can replay the kernel without a memset.  The
+// permutation guarantees that every job has 1..16 rows.
 #pragma once
 #include <cstdint>
 #include <cuda_fp16.h>
@@ -60,7 +55,6 @@ struct ExpertParams {
   int tpe_dn, cpt_dn;         // d/16, f/64
   const int4* jobs;           // {expert, row0, nrows, 0}, 1 <= nrows <= 16
   const int* njobs;
-  const int* n_dense;         // dense experts present -> combine is left to a later kernel
   const int* perm;            // pair index per permuted row
   const int* inv;             // permuted row per pair
   int topk, T, d, f, E;
@@ -71,9 +65,7 @@ struct ExpertParams {
   const float* gs;            // [3][E] gate, up, down tensor scales
   const float* wts;           // [P] routing weight per pair
   float* partial;             // [P][d]
-  uint16_t* out;              // [T][d] bf16
   int* gu_done;               // [max jobs] gate/up tiles finished per job
-  int* dn_done;               // [d/16] pairs finished per output slice
   int* exit_cnt;              // blocks that left
   int* err;
   int64_t wait_timeout_ns;

@@ -51,7 +51,7 @@ struct Workspace {
   int* n_jobs1 = nullptr;
   int4* jobs2 = nullptr;
   int* n_jobs2 = nullptr;
-  int* counters = nullptr;     // gu_done [max jobs] | dn_done [d/16] | exit | ticket
+  int* counters = nullptr;     // gu_done [max jobs] | exit | ticket
   size_t counter_bytes = 0;
   int4* dense_list = nullptr;
   int* n_dense = nullptr;
@@ -122,9 +122,9 @@ T* carve(uint8_t*& cur, size_t count) {
 }
 
 // completion counters: gu_done of list 1 [E] | gu_done of list 2 [E + P/16 + 1] |
-// dn_done [d/16] | exit 1 | exit 2 | routing ticket
+// exit 1 | exit 2 | routing ticket
 size_t counter_ints(const moe_fp4* h, int Tm) {
-  return (size_t)h->E + ((size_t)h->E + (size_t)Tm * h->k / moe::kJobRows + 1) + h->d / 16 + 3;
+  return (size_t)h->E + ((size_t)h->E + (size_t)Tm * h->k / moe::kJobRows + 1) + 3;
 }
 
 // rows of the dense-class operand buffers: every pair plus up to 127 padding
@@ -334,8 +334,7 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
   const size_t max_jobs2 = (size_t)E + (size_t)w.max_T * k / moe::kJobRows + 1;   // counter layout
   int* gu_done1 = w.counters;
   int* gu_done2 = gu_done1 + E;
-  int* dn_done = gu_done2 + max_jobs2;
-  int* exit1 = dn_done + d / 16;
+  int* exit1 = gu_done2 + max_jobs2;
   int* exit2 = exit1 + 1;
   int* ticket = exit2 + 1;
   moe::PermuteOut po{w.counts, w.offsets, w.perm, w.inv, w.jobs1, w.n_jobs1, w.jobs2, w.n_jobs2,
@@ -463,7 +462,6 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
   ep.cpt_gu = d / moe::kChunkK;
   ep.tpe_dn = d / 16;
   ep.cpt_dn = f / moe::kChunkK;
-  ep.n_dense = w.n_dense;
   ep.perm = w.perm;
   ep.inv = w.inv;
   ep.topk = k;
@@ -478,8 +476,6 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
   ep.gs = h->gs;
   ep.wts = w.wts;
   ep.partial = w.partial;
-  ep.out = static_cast<uint16_t*>(out);
-  ep.dn_done = dn_done;
   ep.err = h->err;
   ep.wait_timeout_ns = h->wait_timeout_ns;
   moe::ExpertParams ep1 = ep, ep2 = ep;
