@@ -129,30 +129,6 @@ __device__ __forceinline__ TileInfo tile_info(const ExpertParams& p, const int4*
   return ti;
 }
 
-// Activation fragments of one stage for this lane (NT n-tiles x 4 chunks).
-template <int NT>
-struct BFrag {
-  uint4 v[NT][kExpSC][2];
-};
-
-template <int NT, bool COHERENT>
-__device__ __forceinline__ void load_bfrag(BFrag<NT>& b, const __half* const (&row)[2], int chunk0,
-                                           int nch, int c) {
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-    for (int ch = 0; ch < kExpSC; ++ch) {
-      if (row[nt] != nullptr && ch < nch) {
-        const __half* bp = row[nt] + (size_t)(chunk0 + ch) * kChunkK + c * 16;
-        b.v[nt][ch][0] = COHERENT ? ldg_cg_v4(bp) : ldg_nc_v4(bp);
-        b.v[nt][ch][1] = COHERENT ? ldg_cg_v4(bp + 8) : ldg_nc_v4(bp + 8);
-      } else {
-        b.v[nt][ch][0] = make_uint4(0, 0, 0, 0);
-        b.v[nt][ch][1] = make_uint4(0, 0, 0, 0);
-      }
-    }
-}
-
 // {s, s} * 2^-8 as f16x2 for the non-negative e4m3 byte k of `four`, on the
 // integer pipes: the byte's 7 bits placed at f16 bit 7 give 2^(E-15) (1 + M/8)
 // for exponent field E >= 1 and 2^-14 M/8 for E = 0, i.e. exactly 2^-8 times
@@ -189,20 +165,60 @@ __device__ __forceinline__ uint32_t hmul2_bcast_hi(uint32_t a, uint32_t s) {
   return *reinterpret_cast<const uint32_t*>(&r);
 }
 
-// One stage of shared-memory weights times the lane's activation fragments.
-// The codes and scales of the next (chunk, row tile) are loaded before the
-// current one is converted, so the shared-memory latency overlaps the math.
-template <int NT, int RT, bool FULL>
-__device__ __forceinline__ void mma_stage(uint32_t st, int nch, int lane, int g, const BFrag<NT>& b,
-                                          int nrows, float (&acc)[RT][kAccK][NT][4]) {
-  constexpr int NU = kExpSC * RT;                   // (chunk, row tile) units, chunk-major
+// Activation fragment of one 64-wide chunk for lane c and one n-tile: the two
+// 16-byte halves holding b0, b1 of the chunk's four K steps (zero beyond the
+// job's rows).
+struct BPair {
+  uint4 lo, hi;
+};
+
+template <int NT, bool COHERENT>
+__device__ __forceinline__ void load_bchunk(const __half* const (&brow)[2], int chunk, int c, BPair (&b)[NT]) {
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    if (brow[nt] == nullptr) {
+      b[nt].lo = make_uint4(0, 0, 0, 0);
+      b[nt].hi = b[nt].lo;
+    } else {
+      const __half* bp = brow[nt] + (size_t)chunk * kChunkK + c * 16;
+      b[nt].lo = COHERENT ? ldg_cg_v4(bp) : ldg_nc_v4(bp);
+      b[nt].hi = COHERENT ? ldg_cg_v4(bp + 8) : ldg_nc_v4(bp + 8);
+    }
+  }
+}
+
+// One stage of a work tile: RT row tiles x NT n-tiles.  The activation
+// fragments are not held a stage ahead (64 NT registers) but one chunk ahead:
+// `be` holds chunk0's on entry and the next chunk's on exit when `more` says
+// the warp's next stage of this tile follows.  FULL: all kExpSC chunks
+// present (no per-chunk bounds).  The fragments of even chunks live in `be`,
+// those of odd chunks in `bo`: each chunk prefetches the next one into the
+// other set, so a full stage ends with the next stage's first chunk in `be`
+// and nothing is copied.  The codes and scales of the next (chunk, row tile)
+// unit are loaded before the current one is converted.
+template <int NT, int RT, bool COHERENT, bool FULL>
+__device__ __forceinline__ void mma_stage_jit(uint32_t st, int nch, int lane, int g, const __half* const (&brow)[2],
+                                              int chunk0, int c, bool more, int nrows, BPair (&be)[NT],
+                                              float (&acc)[RT][kAccK][NT][4]) {
+  constexpr int NU = kExpSC * RT;
   auto unit_addr = [&](int u) { return st + (u % RT) * kExpSB + (u / RT) * kChunkBytes; };
   uint4 codes_n = ld_shared_v4(unit_addr(0) + lane * 16);
   uint2 sc_n = ld_shared_v2(unit_addr(0) + kChunkCodeBytes + g * 8);
+  BPair bo[NT];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) { bo[nt].lo = make_uint4(0, 0, 0, 0); bo[nt].hi = bo[nt].lo; }
 #pragma unroll
   for (int u = 0; u < NU; ++u) {
     const int ch = u / RT, rt = u % RT;
     if (!FULL && ch >= nch) break;
+    if (rt == 0) {
+      const bool pf = FULL ? (ch + 1 < kExpSC || more) : (ch + 1 < nch || more);
+      if (pf) {
+        if (ch & 1) load_bchunk<NT, COHERENT>(brow, chunk0 + ch + 1, c, be);
+        else load_bchunk<NT, COHERENT>(brow, chunk0 + ch + 1, c, bo);
+      }
+    }
+    const BPair (&bb)[NT] = (ch & 1) ? bo : be;
     const uint4 codes = codes_n;
     const uint2 sc = sc_n;
     if (u + 1 < NU && (FULL || (u + 1) / RT < nch)) {
@@ -210,6 +226,8 @@ __device__ __forceinline__ void mma_stage(uint32_t st, int nch, int lane, int g,
       sc_n = ld_shared_v2(unit_addr(u + 1) + kChunkCodeBytes + g * 8);
     }
     const uint32_t cw[4] = {codes.x, codes.y, codes.z, codes.w};
+    // scales: sc.x = row A(g) for K steps 0..3, sc.y = row B(g); non-negative
+    // e4m3 bytes (signs are folded into the codes)
     const uint32_t sAB[4] = {e4m3_pair_f16x2<0>(sc.x, sc.y), e4m3_pair_f16x2<1>(sc.x, sc.y),
                              e4m3_pair_f16x2<2>(sc.x, sc.y), e4m3_pair_f16x2<3>(sc.x, sc.y)};
 #pragma unroll
@@ -222,81 +240,12 @@ __device__ __forceinline__ void mma_stage(uint32_t st, int nch, int lane, int g,
       a[3] = hmul2_bcast_hi(a[3], sAB[ks]);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const uint4& lo = b.v[nt][ch][0];
-        const uint4& hi = b.v[nt][ch][1];
+        const uint4& lo = bb[nt].lo;
+        const uint4& hi = bb[nt].hi;
         const uint32_t b0 = ks == 0 ? lo.x : ks == 1 ? lo.z : ks == 2 ? hi.x : hi.z;
         const uint32_t b1 = ks == 0 ? lo.y : ks == 1 ? lo.w : ks == 2 ? hi.y : hi.w;
         if (NT == 1 || nt * 8 < nrows) mma_16816_f16(acc[rt][ks % kAccK][nt], a, b0, b1);
       }
-    }
-  }
-}
-
-
-// Activation fragment (two 16-byte halves) of one 64-wide chunk for lane c.
-template <bool COHERENT>
-__device__ __forceinline__ void load_bchunk(const __half* brow, int chunk, int c, uint4& lo, uint4& hi) {
-  if (brow == nullptr) {
-    lo = make_uint4(0, 0, 0, 0);
-    hi = lo;
-    return;
-  }
-  const __half* bp = brow + (size_t)chunk * kChunkK + c * 16;
-  lo = COHERENT ? ldg_cg_v4(bp) : ldg_nc_v4(bp);
-  hi = COHERENT ? ldg_cg_v4(bp + 8) : ldg_nc_v4(bp + 8);
-}
-
-// One stage of a one-n-tile work tile (NT = 1, RT row tiles sharing the
-// activation fragments).  The activation fragments are not held a stage
-// ahead (64 registers) but one chunk ahead (8): (blo, bhi) holds chunk0's on
-// entry and the next chunk's on exit when `more` says the warp's next stage
-// of this tile follows; that lets four blocks share an SM.
-template <int RT, bool COHERENT, bool FULL>
-__device__ __forceinline__ void mma_stage_jit(uint32_t st, int nch, int lane, int g, const __half* brow,
-                                              int chunk0, int c, bool more, uint4& blo, uint4& bhi,
-                                              float (&acc)[RT][kAccK][1][4]) {
-  // FULL: all kExpSC chunks present (no per-chunk bounds).  The fragments of
-  // even chunks live in (blo, bhi), those of odd chunks in (olo, ohi): each
-  // chunk prefetches the next one into the other pair, so a full stage ends
-  // with the next stage's first chunk in (blo, bhi) and nothing is copied.
-  constexpr int NU = kExpSC * RT;
-  auto unit_addr = [&](int u) { return st + (u % RT) * kExpSB + (u / RT) * kChunkBytes; };
-  uint4 codes_n = ld_shared_v4(unit_addr(0) + lane * 16);
-  uint2 sc_n = ld_shared_v2(unit_addr(0) + kChunkCodeBytes + g * 8);
-  uint4 olo = make_uint4(0, 0, 0, 0), ohi = olo;
-#pragma unroll
-  for (int u = 0; u < NU; ++u) {
-    const int ch = u / RT, rt = u % RT;
-    if (!FULL && ch >= nch) break;
-    if (rt == 0) {
-      const bool pf = FULL ? (ch + 1 < kExpSC || more) : (ch + 1 < nch || more);
-      if (pf) {
-        if (ch & 1) load_bchunk<COHERENT>(brow, chunk0 + ch + 1, c, blo, bhi);
-        else load_bchunk<COHERENT>(brow, chunk0 + ch + 1, c, olo, ohi);
-      }
-    }
-    const uint4& lo = (ch & 1) ? olo : blo;
-    const uint4& hi = (ch & 1) ? ohi : bhi;
-    const uint4 codes = codes_n;
-    const uint2 sc = sc_n;
-    if (u + 1 < NU && (FULL || (u + 1) / RT < nch)) {
-      codes_n = ld_shared_v4(unit_addr(u + 1) + lane * 16);
-      sc_n = ld_shared_v2(unit_addr(u + 1) + kChunkCodeBytes + g * 8);
-    }
-    const uint32_t cw[4] = {codes.x, codes.y, codes.z, codes.w};
-    const uint32_t sAB[4] = {e4m3_pair_f16x2<0>(sc.x, sc.y), e4m3_pair_f16x2<1>(sc.x, sc.y),
-                             e4m3_pair_f16x2<2>(sc.x, sc.y), e4m3_pair_f16x2<3>(sc.x, sc.y)};
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      uint32_t a[4];
-      e2m1x8_to_f16x2x4(cw[ks], a);
-      a[0] = hmul2_bcast_lo(a[0], sAB[ks]);
-      a[1] = hmul2_bcast_hi(a[1], sAB[ks]);
-      a[2] = hmul2_bcast_lo(a[2], sAB[ks]);
-      a[3] = hmul2_bcast_hi(a[3], sAB[ks]);
-      const uint32_t b0 = ks == 0 ? lo.x : ks == 1 ? lo.z : ks == 2 ? hi.x : hi.z;
-      const uint32_t b1 = ks == 0 ? lo.y : ks == 1 ? lo.w : ks == 2 ? hi.y : hi.w;
-      mma_16816_f16(acc[rt][ks % kAccK][0], a, b0, b1);
     }
   }
 }
@@ -306,7 +255,7 @@ __device__ __forceinline__ void mma_stage_jit(uint32_t st, int nch, int lane, in
 // With one n-tile a work tile is two 16-row tiles (RT = 2) that share the
 // activation fragments, the loop control and the epilogue barrier.
 template <int NT>
-__global__ void __launch_bounds__(kExpThreads, NT == 1 ? 4 : 3) expert_kernel(ExpertParams p) {
+__global__ void __launch_bounds__(kExpThreads, 4) expert_kernel(ExpertParams p) {
   constexpr int RT = NT == 1 ? 2 : 1;
   constexpr int RING = kExpRing / RT;          // stages in flight per warp (same bytes)
   constexpr int SLOT = RT * kExpSB;
@@ -379,7 +328,6 @@ __global__ void __launch_bounds__(kExpThreads, NT == 1 ? 4 : 3) expert_kernel(Ex
 
   bool failed = false;
   int consumed = 0;
-  BFrag<2> b2;
 
   // B rows of this lane (row n = nt*8 + g of the job), resolved one tile ahead
   auto tile_rows = [&](const TileInfo& t, const __half* (&row)[2]) {
@@ -426,19 +374,20 @@ __global__ void __launch_bounds__(kExpThreads, NT == 1 ? 4 : 3) expert_kernel(Ex
     }
 
     float part[2][4];                    // this warp's partial sums, per unit u = rt * NT + nt
-    if constexpr (NT == 1) {
-      // one n-tile, two row tiles
-      float acc[RT][kAccK][1][4];
+    {
+      float acc[RT][kAccK][NT][4];
 #pragma unroll
       for (int rt = 0; rt < RT; ++rt)
 #pragma unroll
         for (int a = 0; a < kAccK; ++a)
 #pragma unroll
-          for (int q = 0; q < 4; ++q) acc[rt][a][0][q] = 0.f;
-      uint4 blo, bhi;
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[rt][a][nt][q] = 0.f;
+      BPair be[NT];
       if (ti.nw > 0) {
-        if (ti.down) load_bchunk<true>(row[0], kExpSC * ti.slo, c, blo, bhi);
-        else load_bchunk<false>(row[0], kExpSC * ti.slo, c, blo, bhi);
+        if (ti.down) load_bchunk<NT, true>(row, kExpSC * ti.slo, c, be);
+        else load_bchunk<NT, false>(row, kExpSC * ti.slo, c, be);
       }
       for (int ss = 0; ss < ti.nw; ++ss) {
         const int s = ti.slo + ss;
@@ -451,62 +400,31 @@ __global__ void __launch_bounds__(kExpThreads, NT == 1 ? 4 : 3) expert_kernel(Ex
         }
         if (!failed) {
           const uint32_t sp = ring_s + slot * SLOT;
+          const int k0 = kExpSC * s, nr = ti.nrows;
           if (nch == kExpSC) {
-            if (ti.down) mma_stage_jit<RT, true, true>(sp, nch, lane, g, row[0], kExpSC * s, c, more, blo, bhi, acc);
-            else mma_stage_jit<RT, false, true>(sp, nch, lane, g, row[0], kExpSC * s, c, more, blo, bhi, acc);
+            if (ti.down) mma_stage_jit<NT, RT, true, true>(sp, nch, lane, g, row, k0, c, more, nr, be, acc);
+            else mma_stage_jit<NT, RT, false, true>(sp, nch, lane, g, row, k0, c, more, nr, be, acc);
           } else {
-            if (ti.down) mma_stage_jit<RT, true, false>(sp, nch, lane, g, row[0], kExpSC * s, c, more, blo, bhi, acc);
-            else mma_stage_jit<RT, false, false>(sp, nch, lane, g, row[0], kExpSC * s, c, more, blo, bhi, acc);
+            if (ti.down) mma_stage_jit<NT, RT, true, false>(sp, nch, lane, g, row, k0, c, more, nr, be, acc);
+            else mma_stage_jit<NT, RT, false, false>(sp, nch, lane, g, row, k0, c, more, nr, be, acc);
           }
         }
         __syncwarp();
         ++consumed;
         if (lane == 0 && !failed) produce(consumed);
       }
+      // units: NT == 1 -> (row tile u, n-tile 0); NT == 2 -> (row tile 0, n-tile u)
 #pragma unroll
-      for (int rt = 0; rt < 2; ++rt)
+      for (int u = 0; u < 2; ++u) {
+        const int rt = NT == 1 ? u : 0, nt = NT == 1 ? 0 : u;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          float v = acc[rt][0][0][q];
+          float v = acc[rt][0][nt][q];
 #pragma unroll
-          for (int a = 1; a < kAccK; ++a) v += acc[rt][a][0][q];
-          part[rt][q] = v;
+          for (int a = 1; a < kAccK; ++a) v += acc[rt][a][nt][q];
+          part[u][q] = v;
         }
-    } else {
-      float acc[1][kAccK][2][4];
-#pragma unroll
-      for (int a = 0; a < kAccK; ++a)
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) acc[0][a][nt][q] = 0.f;
-      for (int ss = 0; ss < ti.nw; ++ss) {
-        const int s = ti.slo + ss;
-        const int nch = min(kExpSC, ti.cpt - kExpSC * s);
-        if (ti.down) load_bfrag<2, true>(b2, row, kExpSC * s, nch, c);
-        else load_bfrag<2, false>(b2, row, kExpSC * s, nch, c);
-        const int slot = consumed & (RING - 1);
-        if (!failed && !mbar_wait_until(bars_s + 8 * slot, ((unsigned)consumed / RING) & 1u, deadline)) {
-          failed = true;
-          set_error(p.err, kErrTimeout);
-        }
-        if (!failed) {
-          if (nch == kExpSC) mma_stage<2, 1, true>(ring_s + slot * SLOT, nch, lane, g, b2, ti.nrows, acc);
-          else mma_stage<2, 1, false>(ring_s + slot * SLOT, nch, lane, g, b2, ti.nrows, acc);
-        }
-        __syncwarp();
-        ++consumed;
-        if (lane == 0 && !failed) produce(consumed);
       }
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float v = acc[0][0][nt][q];
-#pragma unroll
-          for (int a = 1; a < kAccK; ++a) v += acc[0][a][nt][q];
-          part[nt][q] = v;
-        }
     }
 
     // ---- cross-warp reduction of the tile (buffer alternates by tile parity)
