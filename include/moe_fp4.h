@@ -172,7 +172,9 @@ MOE_FP4_API int moe_fp4_set_dense_threshold(moe_fp4_t* h, int thr);
  * router (and x staging), events[2] after top-k, events[3] after the
  * permutation, events[4] after the dense-class activation quantiser,
  * events[5] after the dense gate/up + SwiGLU GEMM, events[6] after the dense
- * down GEMM (4-6 follow 3 directly when T < thr and no expert can be dense),
+ * down GEMM (4-6 follow 3 directly when T < thr and no expert can be dense;
+ * with at most 32 (token, expert) pairs the router kernel also runs top-k and
+ * the permutation, so 2 and 3 follow 1 directly),
  * events[7] after the light-class expert kernels and events[8] after the
  * combine (as external event nodes when the stream is being captured into a
  * CUDA graph).  The events must be created with timing enabled; the caller
