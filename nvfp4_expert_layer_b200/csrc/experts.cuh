@@ -88,13 +88,6 @@ __device__ __forceinline__ uint4 ldg_cg_v4(const void* p) {
   return v;
 }
 
-__device__ __forceinline__ float4 ldg_cg_f4(const float* p) {
-  float4 v;
-  asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p));
-  return v;
-}
-
 // Everything a warp needs to know about one tile of the list.
 struct TileInfo {
   int down;       // 0 gate/up, 1 down
@@ -129,23 +122,19 @@ __device__ __forceinline__ TileInfo tile_info(const ExpertParams& p, const int4*
   return ti;
 }
 
-// {s, s} * 2^-8 as f16x2 for the non-negative e4m3 byte k of `four`, on the
-// integer pipes: the byte's 7 bits placed at f16 bit 7 give 2^(E-15) (1 + M/8)
+// Two non-negative e4m3 block scales as f16x2, each times 2^-8, on the
+// integer pipes: {a_k, b_k} (byte k of `a` in the low half, byte k of `b` in
+// the high half).  A byte's 7 bits placed at f16 bit 7 give 2^(E-15) (1 + M/8)
 // for exponent field E >= 1 and 2^-14 M/8 for E = 0, i.e. exactly 2^-8 times
-// the e4m3 value in both cases (f16 subnormals cover the e4m3 subnormals).
-// The 2^-8 is undone on the fp32 accumulators.
-__device__ __forceinline__ uint32_t e4m3_dup_f16x2(uint32_t four, int k) {
-  return __byte_perm(four, 0u, 0x4440u + k) * 0x00800080u;
-}
+// the e4m3 value in both cases (f16 subnormals cover the e4m3 subnormals);
+// the 2^-8 is undone on the fp32 accumulators.  One byte permute puts the two
+// bytes in the low byte of each half (the other bytes come from the
+// sign-replicate mode of a byte whose top bit is clear, i.e. zero), one shift
+// moves them to f16 bit 7.  (The PTX prmt default mode honours the selector's
+// sign-replicate bit; __byte_perm keeps only the low three bits of each
+// selector nibble.)
 constexpr float kScaleUndo = 256.f;
 
-// The same for two scales at once: {a_k, b_k} * 2^-8 as f16x2 (byte k of `a`
-// in the low half, byte k of `b` in the high half).  One byte permute puts the
-// two bytes in the low byte of each half (the other bytes come from the
-// sign-replicate mode of a byte whose top bit is clear, i.e. zero), one shift
-// moves them to f16 bit 7.
-// (The PTX prmt default mode honours the selector's sign-replicate bit;
-// __byte_perm keeps only the low three bits of each selector nibble.)
 template <int K>
 __device__ __forceinline__ uint32_t e4m3_pair_f16x2(uint32_t a, uint32_t b) {
   constexpr uint32_t sel = (uint32_t)K | ((8u | K) << 4) | ((4u + K) << 8) | ((12u + K) << 12);

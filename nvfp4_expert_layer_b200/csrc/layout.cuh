@@ -32,8 +32,6 @@ namespace moe {
 constexpr int kChunkK = 64;
 constexpr int kChunkBytes = 576;
 constexpr int kChunkCodeBytes = 512;
-constexpr int kStageChunks = 4;
-constexpr int kStageBytes = kChunkBytes * kStageChunks;
 
 __host__ __device__ __forceinline__ int bfrag_offset(int kidx) {
   const int chunk = kidx >> 6, kk = kidx & 63;

@@ -26,10 +26,6 @@ __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
                :: "r"(bar), "r"(bytes) : "memory");
@@ -113,14 +109,6 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
 }
 
 // ---------------------------------------------------------------- conversions
-// Two e2m1 codes (low nibble -> low half) to f16x2, exact.
-__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
-  uint32_t out;
-  asm("{\n .reg .b8 b;\n cvt.u8.u32 b, %1;\n cvt.rn.f16x2.e2m1x2 %0, b;\n}"
-      : "=r"(out) : "r"(byte));
-  return out;
-}
-
 // Four e2m1 pairs packed in a 32-bit word -> four f16x2 (byte i -> out[i]).
 __device__ __forceinline__ void e2m1x8_to_f16x2x4(uint32_t w, uint32_t (&o)[4]) {
   asm("{\n .reg .b8 b0, b1, b2, b3;\n"
@@ -139,16 +127,6 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
       : "=r"(out) : "r"(two_bytes));
   return out;
 }
-
-__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-
-// {lo, lo} and {hi, hi} from a packed pair.
-__device__ __forceinline__ uint32_t dup_lo(uint32_t v) { return __byte_perm(v, 0, 0x1010); }
-__device__ __forceinline__ uint32_t dup_hi(uint32_t v) { return __byte_perm(v, 0, 0x3232); }
 
 // ---------------------------------------------------------------- mma.sync
 // D (16x8 fp32) += A (16x16 f16, row) * B (16x8 f16, col).  Not volatile: a
