@@ -44,6 +44,8 @@ METRIC = "MoE-layer tokens/s; decode HBM GB/s and prefill FP4 TFLOP/s vs B200 ro
 EXPERT_BYTES = None   # set from the config: bytes of one expert (gate + up + down, NVFP4)
 POOL = 32
 FP4_OVER_BF16 = 4.0   # nominal dense FP4 / BF16 tensor throughput ratio on B200 (9 / 2.25 PFLOP/s)
+NOMINAL_HBM_GBS = 8000.0       # nominal B200 HBM3e bandwidth, for the second fraction
+NOMINAL_FP4_TFLOPS = 9000.0    # nominal dense FP4 tensor throughput
 
 
 def parse():
@@ -487,6 +489,7 @@ def main():
         roofline = {"bound": "tensor", "kernel": "dense_gemm_kernel<gate/up> (tcgen05 NVFP4, dense class)",
                     "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s", "frac": achieved / fp4_peak,
                     "peak_kind": f"{peak_kind} bf16 burst x {FP4_OVER_BF16:g} (nominal FP4/BF16 ratio)",
+                    "nominal_peak": NOMINAL_FP4_TFLOPS, "frac_nominal": achieved / NOMINAL_FP4_TFLOPS,
                     "traffic": recorded_traffic("dense_gemm_kernel_gate_up"),
                     "algorithmic_flops_per_launch": r["dom_work"], "avg_launch_ms": r["dom_ms"]}
         compute = ("x and h quantised to NVFP4 (e4m3 scale per 16), tcgen05 block-scaled FP4 MMA, "
@@ -496,6 +499,7 @@ def main():
         roofline = {"bound": "hbm", "kernel": "expert_kernel (gate/up + SwiGLU + down, light class)",
                     "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
                     "peak_kind": peak_kind, "traffic": recorded_traffic("expert_kernel"),
+                    "nominal_peak": NOMINAL_HBM_GBS, "frac_nominal": achieved / NOMINAL_HBM_GBS,
                     "algorithmic_bytes_per_launch": r["dom_work"], "avg_launch_ms": r["dom_ms"]}
         compute = "fp4 weights dequantised in registers to fp16, m16n8k16 MMA, fp32 accumulate"
     line = {
