@@ -43,6 +43,9 @@ Readings where the pages are silent (each is stated where it is used):
      (token, slot) pairs by (expert, token, slot).
   R6 a token whose k-th and (k+1)-th fp64 logits differ by less than 1e-6 is a
      near-tie and is excluded from id / output comparisons.
+  R7 the optional per-expert output normalisation ([P2-S8]) is an RMS norm
+     over the d outputs of each expert, y / sqrt(mean(y^2) + eps), with no
+     learned gain and eps chosen by the caller (the pages give neither).
 """
 from __future__ import annotations
 
@@ -84,15 +87,23 @@ def unpack_e2m1(q: np.ndarray) -> np.ndarray:
     return out
 
 
+# Both e2m1 values of every packed byte (R1: element 2i in the low nibble):
+# _BYTE_PAIRS[b] = (e2m1(b & 15), e2m1(b >> 4)).
+_BYTE_PAIRS = np.stack([e2m1_decode(np.arange(256) & 15), e2m1_decode(np.arange(256) >> 4)], axis=-1)
+
+
 def dequant_nvfp4(q: np.ndarray, sf: np.ndarray, gs) -> np.ndarray:
     """Exact NVFP4 dequantisation  W[n,k] = e2m1(q[n,k]) * e4m3(sf[n,k//16]) * gs.
 
     [P2-BG] 4-bit weights with one scale per 16 values; [P3-S2] e2m1 with a
     per-16 block scale; R3 fp32 per-tensor scale.  Float64 holds every product
-    exactly."""
-    vals = e2m1_decode(unpack_e2m1(q))
-    scale = np.repeat(e4m3fn_decode(sf), 16, axis=-1)
-    return vals * scale * np.float64(np.float32(gs))
+    exactly (at most 3 + 4 + 24 significant bits), so the order of the two
+    multiplications does not matter.  Each byte is decoded to its two values
+    by table (the same values as e2m1_decode(unpack_e2m1(q)))."""
+    q = np.asarray(q, dtype=np.uint8)
+    vals = _BYTE_PAIRS[q].reshape(q.shape[:-1] + (q.shape[-1] // 8, 16))   # [..., K/16, 16]
+    scale = e4m3fn_decode(sf)[..., None] * np.float64(np.float32(gs))      # [..., K/16, 1]
+    return (vals * scale).reshape(q.shape[:-1] + (q.shape[-1] * 2,))
 
 
 # ----------------------------------------------------------------------------
@@ -261,7 +272,9 @@ def expert_ffn(xrows: np.ndarray, Wg: np.ndarray, Wu: np.ndarray, Wd: np.ndarray
     first; h is rounded to float32 before its quantiser (the kernel holds h
     in float32).
     magnitudes=True also returns the absolute-value sums that bound rounding
-    errors element by element (|Wg||x|, |Wu||x|, |Wd||h|, and g, u)."""
+    errors element by element (|Wg||x|, |Wu||x|, |Wd||h|, and g, u), and per
+    row the largest row L1 norms of the expert's matrices (l1g, l1u, l1d:
+    max_c sum_k |W[c,k]|) and max |x| of the row (xmax)."""
     xin = quantize_act_nvfp4(xrows)[2] if quantized else xrows
     g = xin @ Wg.T
     u = xin @ Wu.T
@@ -271,21 +284,50 @@ def expert_ffn(xrows: np.ndarray, Wg: np.ndarray, Wu: np.ndarray, Wd: np.ndarray
     if not magnitudes:
         return h, y
     ax = np.abs(xin)
+    ones = np.ones((xrows.shape[0], 1))
     mag = dict(g=g, u=u, gabs=ax @ np.abs(Wg).T, uabs=ax @ np.abs(Wu).T,
-               yabs=np.abs(hin) @ np.abs(Wd).T)
+               yabs=np.abs(hin) @ np.abs(Wd).T,
+               l1g=ones * np.abs(Wg).sum(axis=1).max(), l1u=ones * np.abs(Wu).sum(axis=1).max(),
+               l1d=ones * np.abs(Wd).sum(axis=1).max(), xmax=np.abs(xrows).max(axis=1, keepdims=True))
     return h, y, mag
+
+
+def expert_rms_norm(y: np.ndarray, eps: float) -> np.ndarray:
+    """Per-expert output normalisation  y / sqrt(mean_i y_i^2 + eps) over the
+    d outputs of each row, with no learned gain ([P2-S8]: each expert's output
+    is normalised before the weighted sum; reading R7: an RMS norm, eps given
+    by the caller)."""
+    return y / np.sqrt(np.mean(y * y, axis=-1, keepdims=True) + eps)
+
+
+def _expert_rows(task):
+    """One expert on its selected rows (dequantise, then expert_ffn).
+    task = (experts, e, xrows, quantized, magnitudes); a top-level function so
+    that a process pool can run it."""
+    experts, e, xrows, quantized, magnitudes = task
+    mats = experts.expert(e)
+    Wg = dequant_nvfp4(*mats[0])
+    Wu = dequant_nvfp4(*mats[1])
+    Wd = dequant_nvfp4(*mats[2])
+    return expert_ffn(xrows, Wg, Wu, Wd, quantized=quantized, magnitudes=magnitudes)
 
 
 def forward(x_bits: np.ndarray, router_w: np.ndarray, experts, E: int, k: int,
             thr: int = 128, token_subset=None, want_pairs: bool = True,
-            magnitudes: bool = False):
+            magnitudes: bool = False, expert_norm_eps=None, map_fn=map):
     """The whole layer.  `experts.expert(e)` -> {0: (q,sf,gs) gate, 1: up, 2: down}.
 
     token_subset: if given, expert outputs are evaluated only for pairs of those
     tokens (routing and permutation are always computed for every token).
+    expert_norm_eps: None for the plain weighted sum; a number eps >= 0 applies
+    expert_rms_norm(y, eps) to every expert output before the weighted sum.
+    map_fn: how the independent per-expert evaluations are mapped (the builtin
+    map, or a process pool's map; results are assembled in expert order
+    either way, so the output does not depend on it).
     Returns a dict with logits, ids, w, gap, counts, offsets, perm, inv, the
-    per-pair h and partial (rows in perm order; NaN where not evaluated), out64
-    and the bf16 output bits (rows outside the subset are 0)."""
+    per-pair h, y (the expert output Wd h) and partial (its contribution to
+    the output; rows in perm order; NaN where not evaluated), out64 and the
+    bf16 output bits (rows outside the subset are 0)."""
     T, d = x_bits.shape
     logits = router_logits(x_bits, router_w)
     ids, w, gap = route(logits, k)
@@ -295,10 +337,8 @@ def forward(x_bits: np.ndarray, router_w: np.ndarray, experts, E: int, k: int,
     want = np.zeros(T, dtype=bool)
     want[tokens] = True
     P = T * k
-    f = None
-    h_all = partial_all = None
-    out64 = np.zeros((T, d), dtype=np.float64)
-    mags = None
+    # the (expert, rows) work list, in expert order
+    work = []
     for e in range(E):
         lo, hi = offsets[e], offsets[e + 1]
         if hi == lo:
@@ -309,30 +349,34 @@ def forward(x_bits: np.ndarray, router_w: np.ndarray, experts, E: int, k: int,
         keep = want[toks]
         if not keep.any():
             continue
-        pos, pairs, toks = pos[keep], pairs[keep], toks[keep]
-        mats = experts.expert(e)
-        Wg = dequant_nvfp4(*mats[0])
-        Wu = dequant_nvfp4(*mats[1])
-        Wd = dequant_nvfp4(*mats[2])
-        if f is None:
-            f = Wg.shape[0]
-            if want_pairs:
-                h_all = np.full((P, f), np.nan)
-                partial_all = np.full((P, d), np.nan)
-        res = expert_ffn(x[toks], Wg, Wu, Wd, quantized=(hi - lo) >= thr, magnitudes=magnitudes)
+        # R4: the expert's class follows its full row count in the call
+        work.append((e, pos[keep], pairs[keep], toks[keep], (hi - lo) >= thr))
+    results = list(map_fn(_expert_rows, [(experts, e, x[toks], q, magnitudes)
+                                         for e, _, _, toks, q in work]))
+    h_all = partial_all = y_all = None
+    out64 = np.zeros((T, d), dtype=np.float64)
+    mags = None
+    for (e, pos, pairs, toks, _), res in zip(work, results):
         h, y = res[0], res[1]
+        if want_pairs and h_all is None:
+            f = h.shape[1]
+            h_all = np.full((P, f), np.nan)
+            partial_all = np.full((P, d), np.nan)
+            y_all = np.full((P, d), np.nan)
         if magnitudes:
             if mags is None:
                 mags = {n: np.full((P, v.shape[1]), np.nan) for n, v in res[2].items()}
             for n, v in res[2].items():
                 mags[n][pos] = v
         wj = w.reshape(-1)[pairs]
-        contrib = wj[:, None] * y
+        yn = y if expert_norm_eps is None else expert_rms_norm(y, expert_norm_eps)
+        contrib = wj[:, None] * yn
         if want_pairs:
             h_all[pos] = h
+            y_all[pos] = y
             partial_all[pos] = contrib
         np.add.at(out64, toks, contrib)
     out_bits = f64_to_bf16_bits_rne(out64)
     return dict(logits=logits, ids=ids, w=w, gap=gap, counts=counts, offsets=offsets,
-                perm=perm, inv=inv, h=h_all, partial=partial_all, out64=out64,
+                perm=perm, inv=inv, h=h_all, y=y_all, partial=partial_all, out64=out64,
                 out_bits=out_bits, tokens=tokens, mags=mags)
