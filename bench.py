@@ -1,16 +1,24 @@
 """Benchmark of the NVFP4 sparse-MoE layer forward on B200 (one JSON line).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
-                    [--workload decode1|decode64|verify|prefill|tiny]
+                    [--workload all|decode1|decode64|verify|prefill|tiny]
 
 A step is one forward of the layer (routing, permutation, gate/up + SwiGLU,
-down, combine) over one batch of synthetic tokens.  The default workload is
-batch-1 decode (T=1, d=7168, E=256, top-8, f=2048, NVFP4 experts).  Inputs
-are seeded and synthetic; every step takes the next x of a pool of 32
-distinct token batches whose routing touches different experts, so the
-weights a step streams were evicted from L2 by the steps in between (the
-prefill workload, 16384 tokens, uses a pool of 2: one x alone is 235 MB,
-larger than L2, and every step touches all experts).
+down, combine) over one batch of synthetic tokens.  The default (`all`)
+measures the five workloads one after the other and prints one line whose
+headline fields are batch-1 decode (T=1, d=7168, E=256, top-8, f=2048,
+NVFP4 experts), with a record per workload under "workloads":
+  tiny      T=4, d=512, E=8, top-2, f=256
+  decode1   T=1 (the headline)
+  decode64  T=64, Zipf(1.1)-biased router
+  verify    32 requests x 4 draft tokens, correlated within a request
+  prefill   8 x 2048 tokens (every expert in the dense class, tcgen05 FP4)
+The four full-size workloads share one seeded expert set (6.3 GB, generated
+and loaded once); each has its own seeded tokens and router.  Every step
+takes the next x of a pool of 32 token batches whose routing touches
+different experts, so the weights a step streams were evicted from L2 by the
+steps in between (prefill: a pool of 2; one x is 235 MB, larger than L2, and
+every step reads all 6.3 GB of experts).
 
 Roofline of the dominant kernel: for decode shapes the light-class expert
 kernel against HBM bandwidth (algorithmic bytes = NVFP4 bytes of the experts
@@ -41,42 +49,74 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/s; decode HBM GB/s and prefill FP4 TFLOP/s vs B200 roofline"
-EXPERT_BYTES = None   # set from the config: bytes of one expert (gate + up + down, NVFP4)
 POOL = 32
 FP4_OVER_BF16 = 4.0   # nominal dense FP4 / BF16 tensor throughput ratio on B200 (9 / 2.25 PFLOP/s)
 NOMINAL_HBM_GBS = 8000.0       # nominal B200 HBM3e bandwidth, for the second fraction
 NOMINAL_FP4_TFLOPS = 9000.0    # nominal dense FP4 tensor throughput
+ALL = ("decode1", "tiny", "decode64", "verify", "prefill")
+FULL_SIZE = ("decode1", "decode64", "verify", "prefill")
+OUT_TOL = 1e-2
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--workload", default="decode1")
+    ap.add_argument("--workload", default="all")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--shape", default="",
-                    help="profiling sizes over the workload's recipe, e.g. T=4096,E=32 "
+                    help="profiling sizes over one workload's recipe, e.g. T=4096,E=32 "
                          "(the JSON line then names the changed sizes)")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
-def workload_config(args):
+def workload_names(args):
+    return ALL if args.workload == "all" else (args.workload,)
+
+
+def workload_config(name, shape=""):
     from nvfp4_expert_layer_b200 import workloads as W
-    cfg = W.CONFIGS[args.workload]
-    if args.shape:
-        kw = {k: int(v) for k, v in (item.split("=") for item in args.shape.split(","))}
-        cfg = W.LayerConfig(f"{cfg.name}[{args.shape}]", kw.get("T", cfg.T), kw.get("d", cfg.d),
+    cfg = W.CONFIGS[name]
+    if shape:
+        kw = {k: int(v) for k, v in (item.split("=") for item in shape.split(","))}
+        cfg = W.LayerConfig(f"{cfg.name}[{shape}]", kw.get("T", cfg.T), kw.get("d", cfg.d),
                             kw.get("E", cfg.E), kw.get("k", cfg.k), kw.get("f", cfg.f), cfg.seed,
                             cfg.router, cfg.requests)
     return cfg
+
+
+def weights_config(cfg):
+    """The config whose seed generates the expert weights: the full-size
+    workloads share the batch-1 decode expert set."""
+    from nvfp4_expert_layer_b200 import workloads as W
+    base = cfg.name.split("[")[0]
+    if base in FULL_SIZE:
+        d1 = W.CONFIGS["decode1"]
+        return W.LayerConfig(cfg.name, cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, d1.seed, cfg.router, cfg.requests)
+    return cfg
+
+
+def pool_size(cfg) -> int:
+    return 2 if cfg.T * cfg.d * 2 > 126e6 else POOL
 
 
 def expert_bytes(cfg) -> int:
     """Algorithmic bytes of one expert: 3 matrices of f x d NVFP4 values
     (0.5 byte per value + one e4m3 byte per 16 values)."""
     return 3 * cfg.f * cfg.d // 2 + 3 * cfg.f * cfg.d // 16
+
+
+def config_dict(cfg, world: int) -> dict:
+    """The `config` of a line; the native and the reference arm print the same."""
+    pool = pool_size(cfg)
+    return {"workload": f"{cfg.name}: T={cfg.T} tokens, d={cfg.d}, E={cfg.E}, top-{cfg.k}, f={cfg.f}, "
+                        "NVFP4 experts (e2m1 + e4m3/16 + fp32 tensor scale)",
+            "global_batch": cfg.T * world, "parallelism": f"replicas x{world}",
+            "l2": f"inputs rotate over {pool} token batches of {cfg.T * cfg.d * 2 / 1e6:.1f} MB; "
+                  f"their experts span {cfg.E * expert_bytes(cfg) / 1e9:.2f} GB > 126 MB L2",
+            "timing": "CUDA graph replay per step, CUDA events on the launch stream, max over ranks"}
 
 
 def measured_peaks():
@@ -90,8 +130,8 @@ def measured_peaks():
 
 
 def is_dense(cfg, thr=128) -> bool:
-    """Whether the workload's experts run in the dense class (T >= thr and the
-    shapes the tensor-core path supports)."""
+    """Whether the workload's experts may run in the dense class (T >= thr and
+    the shapes the tensor-core path supports)."""
     return cfg.T >= thr and cfg.d % 256 == 0 and cfg.f % 256 == 0
 
 
@@ -105,17 +145,18 @@ def source_digest() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None
-    when the kernel sources changed since the counters were taken."""
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
+    summary, or None when the kernel sources changed since the counters were
+    taken (or none were taken for that workload)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as fh:
             rec = json.load(fh)
     except Exception:
         return None
-    ent = rec.get(kernel)
-    if not ent or ent.get("source_digest") != source_digest():
+    ent = rec.get(f"{kernel}@{workload}") or rec.get(kernel)
+    if not ent or ent.get("source_digest") != source_digest() or ent.get("workload", workload) != workload:
         return None
     return ent.get("dram_bytes_per_launch")
 
@@ -214,19 +255,34 @@ def barrier(world: int):
 # CPU baseline: the oracle on a bounded sample of the same workload
 # ----------------------------------------------------------------------------
 
-def oracle_sample(cfg, x, rw, n_tokens: int):
-    """Time the fp64 oracle on the first n_tokens of x (routing over all
-    experts, the selected experts dequantised exactly and evaluated).  Expert
-    weights are generated before the clock starts.  Returns (seconds, result)."""
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline_sample(cfg, x_np, rw_np):
+    """The oracle on a bounded sample of the first pool input: routing and the
+    permutation of the whole batch in fp64 (which decide the expert classes),
+    then the experts of its first min(T, 4) tokens (one token for the
+    full-size workloads) dequantised exactly and evaluated in fp64.  Expert
+    weights are generated before the clock starts.  Returns (seconds, tokens,
+    oracle result, description)."""
     from nvfp4_expert_layer_b200 import workloads as W
     from oracle import moe_oracle as O
-    lazy = W.LazyExperts(cfg)
-    ids, _, _ = O.route(O.router_logits(x[:n_tokens], rw), cfg.k)
+    n = 1 if cfg.name in FULL_SIZE else min(cfg.T, 4)
+    lazy = W.LazyExperts(weights_config(cfg))
+    ids, _, _ = O.route(O.router_logits(x_np[:n], rw_np), cfg.k)
     for e in np.unique(ids):
         lazy.expert(int(e))
     t0 = time.perf_counter()
-    res = O.forward(x[:n_tokens], rw, lazy, cfg.E, cfg.k, thr=128)
-    return time.perf_counter() - t0, res
+    res = O.forward(x_np, rw_np, lazy, cfg.E, cfg.k, thr=128, token_subset=list(range(n)))
+    secs = time.perf_counter() - t0
+    sample = (f"oracle on the {cfg.name} workload: routing and permutation of all {cfg.T} tokens "
+              f"(fp64 logits), then the experts of its first {n} token(s) dequantised exactly and "
+              f"evaluated in fp64; value = {n} token(s) / time")
+    return secs, n, res, sample
 
 
 REF_BLOCK = 128     # FFN channels per reference step
@@ -253,13 +309,6 @@ def reference_unit(cfg, x, rw, lazy, step):
     return w[0, j] * ((O.silu(g) * u) @ Wd.T)
 
 
-def cpu_cores() -> int:
-    try:
-        return len(os.sched_getaffinity(0))
-    except Exception:
-        return os.cpu_count() or 1
-
-
 # ----------------------------------------------------------------------------
 # native arm: the CUDA layer through its C ABI
 # ----------------------------------------------------------------------------
@@ -275,35 +324,100 @@ def pool_inputs(cfg, n):
     return xs, rw
 
 
-def run_native(args, rank, world, local):
+def launches_per_step(cfg) -> int:
+    """Kernels one forward launches: routing (up to 256 tokens the router
+    kernel, which for at most 32 pairs also runs top-k and the permutation,
+    else top-k and 3 permutation kernels follow it; above 256 tokens the
+    weight split, router, x staging, top-k and 3 permutation kernels), the
+    dense class (quantiser, gather, 2 GEMMs) when T >= thr, the light-class
+    expert kernels (the 9..16-row one only when T >= 9) and the combine."""
+    pairs = cfg.T * cfg.k
+    routing = (1 if pairs <= 32 else 5) if cfg.T <= 256 else 7
+    return routing + (4 if is_dense(cfg) else 0) + (2 if cfg.T >= 9 else 1) + 1
+
+
+def bf16_ulp_distance(a_bits, b_bits) -> int:
+    def line(b):
+        b = np.asarray(b, np.int64)
+        return np.where(b & 0x8000, -(b & 0x7FFF), b)
+    return int(np.abs(line(a_bits) - line(b_bits)).max()) if np.size(a_bits) else 0
+
+
+def parity_record(res, gpu) -> dict:
+    """Parity of the sampled tokens: the layer's pre-rounding output (the fp32
+    slot-order sum of its own partials) against the oracle's exact output,
+    relative to rms(out_oracle); the largest distance in bf16 ulps between
+    the layer's and the oracle's bf16 outputs; and the verdict (same expert
+    sets, no near tie, pre-rounding error <= 1e-2 rms, bf16 output within
+    1e-2 rms + half an ulp)."""
+    from oracle import moe_oracle as O
+    toks = np.asarray(res["tokens"])
+    ov = res["out64"][toks]
+    rms = float(np.sqrt(np.mean(ov ** 2)))
+    pre = gpu["pre32"].astype(np.float64)
+    gv = O.bf16_bits_to_f64(gpu["out_bits"])
+    half = np.exp2(np.floor(np.log2(np.maximum(np.abs(ov), 2.0 ** -126))) - 8)
+    err = float(np.abs(pre - ov).max())
+    same = bool(np.all(np.sort(gpu["ids"], axis=1) == np.sort(res["ids"][toks], axis=1)))
+    ties = bool(np.any(O.near_tie_flags(res["gap"])[toks]))
+    ok = same and not ties and err <= OUT_TOL * rms and bool(np.all(np.abs(gv - ov) <= OUT_TOL * rms + half))
+    return {"verdict": "pass" if ok else "fail", "pre_rounding_err_over_rms": err / rms if rms else err,
+            "bf16_ulp_max": bf16_ulp_distance(gpu["out_bits"], res["out_bits"][toks]),
+            "tokens": int(len(toks)), "same_expert_sets": same, "near_tie": ties,
+            "tolerance": "pre-rounding max|err| <= 1e-2 rms(oracle); bf16 output <= 1e-2 rms + half ulp"}
+
+
+class NativeLayers:
+    """One layer handle per (shape, expert seed); the full-size workloads
+    share one (6.3 GB of experts generated and loaded once)."""
+
+    def __init__(self):
+        self.layers = {}
+
+    def get(self, cfg, max_T):
+        import torch
+        from nvfp4_expert_layer_b200 import workloads as W
+        from nvfp4_expert_layer_b200.layer import MoeFp4Layer, experts_to_device
+        wc = weights_config(cfg)
+        key = (cfg.E, cfg.k, cfg.d, cfg.f, wc.seed)
+        if key not in self.layers:
+            ex = W.gen_experts(wc)
+            layer = MoeFp4Layer(cfg.E, cfg.k, cfg.d, cfg.f)
+            dev = experts_to_device(ex)
+            layer.load_experts(dev)
+            del dev, ex
+            torch.cuda.empty_cache()
+            self.layers[key] = layer
+        layer = self.layers[key]
+        layer.reserve(max_T)
+        return layer
+
+    def close(self):
+        for layer in self.layers.values():
+            layer.close()
+        self.layers = {}
+
+
+def run_workload(args, cfg, layer, rank, world, local):
+    """Time one workload: graphs of the pool inputs, K timed steps (headline
+    number), a stage-event pass for the dominant kernel, the end-to-end pass
+    through the host-buffer entry point, and the outputs for parity."""
     import torch
-    from nvfp4_expert_layer_b200 import workloads as W
-    from nvfp4_expert_layer_b200.layer import MoeFp4Layer, experts_to_device
-    torch.cuda.set_device(local)
-    cfg = workload_config(args)
-    ex = W.gen_experts(cfg)
-    layer = MoeFp4Layer(cfg.E, cfg.k, cfg.d, cfg.f)
-    dev = experts_to_device(ex)
-    layer.load_experts(dev)
-    del dev
-    torch.cuda.empty_cache()
-    layer.reserve(cfg.T)
-    pool = 2 if cfg.T * cfg.d * 2 > 126e6 else POOL
+    pool = pool_size(cfg)
     xs_np, rw_np = pool_inputs(cfg, pool)
     xs = [torch.from_numpy(x.view(np.int16).copy()).cuda().view(torch.bfloat16) for x in xs_np]
     rw = torch.from_numpy(rw_np).cuda()
     out = torch.empty_like(xs[0])
+    layer.set_dense_threshold(128)
     # units of work of one step, from the layer's own routing: distinct experts
     # touched (decode bytes) and rows of dense-class experts (prefill FLOPs)
-    dense = is_dense(cfg)
     experts_per_input, dense_rows = [], []
     for x in xs:
         _, dbg = layer.forward_ex(x, rw, want=("counts",))
         c = dbg["counts"].cpu().numpy()
         experts_per_input.append(int((c > 0).sum()))
-        dense_rows.append(int(c[c >= 128].sum()) if dense else 0)
-    # T >= thr only allows the dense class; it runs when some expert reaches thr rows
-    dense = dense and sum(dense_rows) > 0
+        dense_rows.append(int(c[c >= 128].sum()) if is_dense(cfg) else 0)
+    dense = is_dense(cfg) and sum(dense_rows) > 0
     stream = torch.cuda.Stream()
     graphs = []
     with torch.cuda.stream(stream):
@@ -321,7 +435,7 @@ def run_native(args, rank, world, local):
     for i in range(args.warmup):
         graphs[i % pool].replay()
     torch.cuda.synchronize()
-    # ---- timed region (headline)
+    # ---- timed region
     clocks = ClockSampler(local)
     barrier(world)
     torch.cuda.synchronize()
@@ -336,6 +450,7 @@ def run_native(args, rank, world, local):
     clk = clocks.stop()
     ms = allreduce_max(e0.elapsed_time(e1), world)
     err = layer.device_error()
+    del graphs
     # ---- per-stage pass: the same graphs with stage events (events between stages)
     nst = len(layer.STAGES)
     dom = layer.STAGES.index("dense_gate_up" if dense else "light")
@@ -370,6 +485,7 @@ def run_native(args, rank, world, local):
                 dom_work += experts_per_input[i] * expert_bytes(cfg)
             n += 1
     stage_ms /= n
+    del sgraphs
     # ---- end to end through the C ABI with host buffers
     xh = [torch.from_numpy(x.view(np.int16).copy()).view(torch.bfloat16).pin_memory() for x in xs_np]
     oh = torch.empty_like(xh[0]).pin_memory()
@@ -383,106 +499,29 @@ def run_native(args, rank, world, local):
     ee1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = allreduce_max(ee0.elapsed_time(ee1), world)
-    gpu_out0 = None
-    layer(xs[0], rw, out=out)
+    del xh, oh
+    # ---- outputs of pool input 0 for parity: bf16 out, ids, and the fp32
+    # slot-order sum of the partials of its first tokens (done on the device)
+    n_par = 1 if cfg.name.split("[")[0] in FULL_SIZE else min(cfg.T, 4)
+    o2, dbg = layer.forward_ex(xs[0], rw, want=("perm", "partial", "topk_ids"))
     torch.cuda.synchronize()
-    gpu_out0 = out.view(torch.int16).cpu().numpy().view(np.uint16).copy()
-    # kernels per step: routing (up to 256 tokens the router kernel, which for
-    # at most 32 pairs also runs top-k and the permutation, else top-k and 3
-    # permutation kernels follow it; above 256 tokens the weight split, router,
-    # x staging, top-k and 3 permutation kernels), the dense class
-    # (quantiser, gather, 2 GEMMs) when T >= thr, the light-class expert
-    # kernels (the 9..16-row one only when T >= 9) and the combine
-    pairs = cfg.T * cfg.k
-    routing = (1 if pairs <= 32 else 5) if cfg.T <= 256 else 7
-    launches = routing + (4 if cfg.T >= 128 else 0) + (2 if cfg.T >= 9 else 1) + 1
+    inv = torch.argsort(dbg["perm"].long())
+    pre = torch.zeros((n_par, cfg.d), dtype=torch.float32, device="cuda")
+    for j in range(cfg.k):
+        pre += dbg["partial"][inv[torch.arange(n_par, device="cuda") * cfg.k + j]]
+    gpu = {"out_bits": o2[:n_par].view(torch.int16).cpu().numpy().view(np.uint16).copy(),
+           "pre32": pre.cpu().numpy(), "ids": dbg["topk_ids"][:n_par].cpu().numpy()}
+    del dbg, o2, pre, inv
+    torch.cuda.empty_cache()
     return dict(cfg=cfg, ms=ms, clk=clk, err=err, stage_ms=stage_ms, dom_ms=dom_ms / n,
                 dom_work=dom_work / n, dense=dense, e2e_ms=e2e_ms, xs_np=xs_np, rw_np=rw_np,
-                gpu_out0=gpu_out0, launches_per_step=launches, stages=layer.STAGES,
+                gpu=gpu, launches=launches_per_step(cfg), stages=layer.STAGES,
                 dense_rows=float(np.mean(dense_rows)), pool=pool)
 
 
-def parity_vs_oracle(res_oracle, gpu_bits, tol=1e-2):
-    """Output parity of one sampled token batch (bf16 output within 1e-2*rms
-    plus the final rounding's half ulp of the oracle's exact output)."""
-    from oracle import moe_oracle as O
-    toks = res_oracle["tokens"]
-    ov = res_oracle["out64"][toks]
-    gv = O.bf16_bits_to_f64(gpu_bits[toks])
-    rms = float(np.sqrt(np.mean(ov ** 2)))
-    half = np.exp2(np.floor(np.log2(np.maximum(np.abs(ov), 2.0 ** -126))) - 8)
-    ties = bool(np.any(O.near_tie_flags(res_oracle["gap"])[toks]))
-    ok = bool(np.all(np.abs(gv - ov) <= tol * rms + half)) and not ties
-    return ("pass" if ok else "fail"), float(np.abs(gv - ov).max() / rms)
-
-
-def cpu_baseline_sample(cfg, xs_np, rw_np):
-    """Oracle on a bounded sample of the first pool input: all of its tokens
-    when T <= 8, else its first 8 tokens as a batch of their own.  When the
-    workload's experts run in the dense class, the sample keeps the whole
-    batch's routing (which decides the class) and evaluates the experts of
-    its first token only."""
-    if is_dense(cfg):
-        from nvfp4_expert_layer_b200 import workloads as W
-        from oracle import moe_oracle as O
-        lazy = W.LazyExperts(cfg)
-        ids, _, _ = O.route(O.router_logits(xs_np[0][:1], rw_np), cfg.k)
-        for e in np.unique(ids):
-            lazy.expert(int(e))
-        t0 = time.perf_counter()
-        res = O.forward(xs_np[0], rw_np, lazy, cfg.E, cfg.k, thr=128, token_subset=[0])
-        secs = time.perf_counter() - t0
-        sample = (f"oracle on the {cfg.name} workload: routing and permutation of all {cfg.T} tokens "
-                  f"(fp64 logits), then the {cfg.k} experts of token 0 in the dense class (NVFP4 "
-                  f"activations) dequantised exactly and evaluated in fp64; value = 1 token / time")
-        return secs, 1, res, sample
-    n = min(cfg.T, 8)
-    secs, res = oracle_sample(cfg, xs_np[0], rw_np, n)
-    sample = (f"oracle on {n} token(s) of the {cfg.name} workload: routing over {cfg.E} experts, "
-              f"the selected experts dequantised exactly and evaluated in fp64")
-    return secs, n, res, sample
-
-
-def main():
-    args = parse()
-    rank, world, local = dist_setup(args)
-    from nvfp4_expert_layer_b200 import workloads as W
-    cfg = workload_config(args)
-    if args.impl == "reference":
-        # the reference arm is the oracle (plain fp64 CPU code) on bounded
-        # slices of the same workload; rank 0 only
-        if rank != 0:
-            return
-        xs_np, rw_np = pool_inputs(cfg, 1)
-        lazy = W.LazyExperts(cfg)
-        from oracle import moe_oracle as O
-        ids, _, _ = O.route(O.router_logits(xs_np[0][:1], rw_np), cfg.k)
-        for e in ids[0]:
-            lazy.expert(int(e))                     # generated before timing
-        for i in range(args.warmup):
-            reference_unit(cfg, xs_np[0], rw_np, lazy, i)
-        t0 = time.perf_counter()
-        for i in range(args.steps):
-            reference_unit(cfg, xs_np[0], rw_np, lazy, i)
-        secs = time.perf_counter() - t0
-        per_step_tokens = 1.0 / (cfg.k * (cfg.f // REF_BLOCK))
-        value = per_step_tokens * args.steps / secs
-        sample = (f"per step: one routed (token, expert) pair of the {cfg.name} workload restricted to "
-                  f"{REF_BLOCK} of the f={cfg.f} FFN channels ({per_step_tokens:.6f} token)")
-        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
-                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": f"{cfg.name}: T={cfg.T}, d={cfg.d}, E={cfg.E}, top-{cfg.k}, f={cfg.f}"},
-                "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
-                                 "sample": sample},
-                "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-        print(json.dumps(line), flush=True)
-        return
-
-    r = run_native(args, rank, world, local)
+def workload_record(args, r, world) -> dict:
+    cfg = r["cfg"]
     tokens = cfg.T * args.steps * world
-    value = tokens / (r["ms"] * 1e-3)
     hbm_peak, fp4_peak, peak_kind = measured_peaks()
     if r["dense"]:
         achieved = r["dom_work"] / (r["dom_ms"] * 1e-3) / 1e12
@@ -490,45 +529,110 @@ def main():
                     "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s", "frac": achieved / fp4_peak,
                     "peak_kind": f"{peak_kind} bf16 burst x {FP4_OVER_BF16:g} (nominal FP4/BF16 ratio)",
                     "nominal_peak": NOMINAL_FP4_TFLOPS, "frac_nominal": achieved / NOMINAL_FP4_TFLOPS,
-                    "traffic": recorded_traffic("dense_gemm_kernel_gate_up"),
+                    "traffic": recorded_traffic("dense_gemm_kernel_gate_up", cfg.name),
                     "algorithmic_flops_per_launch": r["dom_work"], "avg_launch_ms": r["dom_ms"]}
         compute = ("x and h quantised to NVFP4 (e4m3 scale per 16), tcgen05 block-scaled FP4 MMA, "
                    "fp32 accumulate in TMEM")
+        dtype = "fp4"
     else:
         achieved = r["dom_work"] / (r["dom_ms"] * 1e-3) / 1e9
         roofline = {"bound": "hbm", "kernel": "expert_kernel (gate/up + SwiGLU + down, light class)",
                     "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
-                    "peak_kind": peak_kind, "traffic": recorded_traffic("expert_kernel"),
+                    "peak_kind": peak_kind, "traffic": recorded_traffic("expert_kernel", cfg.name),
                     "nominal_peak": NOMINAL_HBM_GBS, "frac_nominal": achieved / NOMINAL_HBM_GBS,
                     "algorithmic_bytes_per_launch": r["dom_work"], "avg_launch_ms": r["dom_ms"]}
         compute = "fp4 weights dequantised in registers to fp16, m16n8k16 MMA, fp32 accumulate"
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": r["ms"] / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "fp4" if r["dense"] else "f16",
+        dtype = "f16"
+    conf = config_dict(cfg, world)
+    return {
+        "metric": METRIC, "value": tokens / (r["ms"] * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms"] / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype,
         "data": "synthetic (seeded; NVFP4 experts from N(0,0.02), x ~ N(0,1) bf16)",
-        "config": {"workload": f"{cfg.name}: T={cfg.T} tokens, d={cfg.d}, E={cfg.E}, top-{cfg.k}, f={cfg.f}, "
-                               "NVFP4 experts (e2m1 + e4m3/16 + fp32 tensor scale)",
-                   "global_batch": cfg.T * world, "parallelism": f"replicas x{world}",
-                   "l2": f"inputs rotate over {r['pool']} token batches of {cfg.T * cfg.d * 2 / 1e6:.1f} MB; "
-                         f"their experts span {cfg.E * expert_bytes(cfg) / 1e9:.2f} GB > 126 MB L2",
-                   "timing": "CUDA graph replay per step, CUDA events on the launch stream, max over ranks",
-                   "compute": compute},
-        "roofline": roofline,
+        "config": conf, "compute": compute, "roofline": roofline,
         "stage_us": {n: round(float(v) * 1e3, 2) for n, v in zip(r["stages"], r["stage_ms"])},
         "clocks": r["clk"],
         "e2e": {"value": tokens / (r["e2e_ms"] * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 2},
-        "gpu_launches": r["launches_per_step"] * args.steps,
+        "gpu_launches": r["launches"] * args.steps,
         "device_error": r["err"],
     }
+
+
+def run_reference(args, rank):
+    """The reference arm: the oracle (plain fp64 CPU code) on bounded slices of
+    the headline workload; rank 0 only."""
+    from nvfp4_expert_layer_b200 import workloads as W
+    from oracle import moe_oracle as O
+    if rank != 0:
+        return
+    name = workload_names(args)[0]
+    cfg = workload_config(name, args.shape)
+    xs_np, rw_np = pool_inputs(cfg, 1)
+    lazy = W.LazyExperts(weights_config(cfg))
+    ids, _, _ = O.route(O.router_logits(xs_np[0][:1], rw_np), cfg.k)
+    for e in ids[0]:
+        lazy.expert(int(e))                     # generated before timing
+    for i in range(args.warmup):
+        reference_unit(cfg, xs_np[0], rw_np, lazy, i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        reference_unit(cfg, xs_np[0], rw_np, lazy, i)
+    secs = time.perf_counter() - t0
+    per_step_tokens = 1.0 / (cfg.k * (cfg.f // REF_BLOCK))
+    value = per_step_tokens * args.steps / secs
+    sample = (f"per step: one routed (token, expert) pair of the {cfg.name} workload restricted to "
+              f"{REF_BLOCK} of the f={cfg.f} FFN channels ({per_step_tokens:.6f} token)")
+    conf = config_dict(cfg, args.gpus)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": conf, "compute": "fp64 numpy oracle on the host cores",
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_setup(args)
+    if args.impl == "reference":
+        run_reference(args, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    import torch
+    torch.cuda.set_device(local)
+    names = workload_names(args)
+    cfgs = [workload_config(n, args.shape) for n in names]
+    layers = NativeLayers()
+    runs = []
+    for cfg in cfgs:
+        max_T = max(c.T for c in cfgs if weights_config(c).seed == weights_config(cfg).seed
+                    and (c.E, c.d, c.f) == (cfg.E, cfg.d, cfg.f))
+        layer = layers.get(cfg, max_T)
+        runs.append(run_workload(args, cfg, layer, rank, world, local))
+    layers.close()
+    records = {r["cfg"].name: workload_record(args, r, world) for r in runs}
+    # CPU baseline and parity after all GPU timing (rank 0 at N = 1 only)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        secs, n, res, sample = cpu_baseline_sample(cfg, r["xs_np"], r["rw_np"])
-        line["cpu_baseline"] = {"value": n / secs, "unit": "tokens/s", "cores": cpu_cores(),
-                                "kind": "oracle", "sample": sample}
-        line["parity"], line["parity_max_err_over_rms"] = parity_vs_oracle(res, r["gpu_out0"])
+        for r in runs:
+            cfg = r["cfg"]
+            secs, n, res, sample = cpu_baseline_sample(cfg, r["xs_np"], r["rw_np"])
+            rec = records[cfg.name]
+            rec["cpu_baseline"] = {"value": n / secs, "unit": "tokens/s", "cores": cpu_cores(),
+                                   "kind": "oracle", "sample": sample}
+            rec["parity"] = parity_record(res, r["gpu"])
+    head = dict(records[cfgs[0].name])
+    if len(cfgs) > 1:
+        keep = ("value", "unit", "steps", "ms_per_step", "dtype", "config", "compute", "roofline", "stage_us",
+                "clocks", "e2e", "gpu_launches", "device_error", "cpu_baseline", "parity")
+        head["workloads"] = {n: {k: v for k, v in rec.items() if k in keep} for n, rec in records.items()}
     if rank == 0:
-        print(json.dumps(line), flush=True)
+        print(json.dumps(head), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

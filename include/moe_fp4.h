@@ -90,6 +90,10 @@ typedef enum {
 } moe_fp4_status;
 
 /* Create a layer handle on the current device.
+ * Defines the layer's shape: E experts, top_k routed per token, model width
+ * d, expert FFN width f ("Optimizing Muse Spark Open on TPU v7 with
+ * SGLang-TorchTPU", Background: each token goes to 8 of 256 experts; the
+ * "Mixture of Experts" topic page: 256 experts, 8 selected).
  *   E       experts, 1..1024
  *   top_k   experts per token, 1..min(E, 32)
  *   d, f    model width and expert FFN width; multiples of 128, 128..16384
@@ -114,24 +118,62 @@ typedef struct {
 
 /* Copy and repack the experts into library-owned device buffers (the
  * register-dequant GEMV layout and the tensor-core block-scaled layout).
- * Synchronous; may be called again to replace the weights. */
+ * The weights are NVFP4 as defined on "Optimizing Models to Be Fast at
+ * Codegen", section 2 (e2m1 values, one scale per 16 along K) and the Muse
+ * Spark page's Background (4-bit experts with a per-16 block scale); each
+ * (expert, matrix) carries one fp32 tensor scale.  Also derives, per expert,
+ * the largest row L1 norm of the gate and up matrices, which bounds the
+ * light class's intermediates.  Synchronous; may be called again to replace
+ * the weights.  Errors: MOE_FP4_ERR_INVALID_ARG (null handle, struct or
+ * member), MOE_FP4_ERR_OOM, MOE_FP4_ERR_CUDA. */
 MOE_FP4_API int moe_fp4_load_experts(moe_fp4_t* h, const moe_fp4_experts* w);
+
+/* Which resident weight copies the next moe_fp4_load_experts keeps (each
+ * copy holds exactly the canonical NVFP4 bytes: E * 3 * f * d * (1/2 + 1/16)):
+ *   light = 1, dense = 1  both (the default): few-row experts stream the
+ *                         register-dequant copy, many-row experts the
+ *                         tensor-core copy;
+ *   light = 1, dense = 0  only the register-dequant copy: every expert runs
+ *                         in the light class;
+ *   light = 0, dense = 1  only the tensor-core copy: every expert runs in the
+ *                         dense class (NVFP4 activations), whatever its row
+ *                         count; needs d and f multiples of 256.
+ * The weights stay 4-bit in every copy ("Optimizing Models to Be Fast at
+ * Codegen", section 2).  The choice takes effect at the next load, which
+ * frees copies no longer kept; until then forwards report
+ * MOE_FP4_ERR_NOT_LOADED.  Errors: MOE_FP4_ERR_INVALID_ARG (null handle, a
+ * value other than 0/1, both 0), MOE_FP4_ERR_UNSUPPORTED (dense only with d
+ * or f not a multiple of 256). */
+MOE_FP4_API int moe_fp4_set_resident_classes(moe_fp4_t* h, int light, int dense);
+
+/* Device bytes the handle holds: *weights for the resident weight copies,
+ * *workspace for the forward's workspace.  Errors: MOE_FP4_ERR_INVALID_ARG. */
+MOE_FP4_API int moe_fp4_device_bytes(moe_fp4_t* h, size_t* weights, size_t* workspace);
 
 /* Pre-size the workspace for up to max_T tokens per forward (allocates).
  * After this, moe_fp4_forward with T <= max_T allocates nothing. */
 MOE_FP4_API int moe_fp4_reserve(moe_fp4_t* h, int max_T);
 
-/* The layer forward.
+/* The layer forward: router logits, softmax and top-k, the token -> expert
+ * permutation, gate/up + SwiGLU, down x routing weight and the combine, as
+ * stated at the top of this file (Muse Spark page, Background and section 8:
+ * gate/up, SwiGLU, down, a single combine pass writing each output row
+ * once; "Day-0 Inference Adaptation for Ultra-Large Sparse Models", section
+ * II: routing indexes built on the device without a host round trip).
  *   x_bf16    device, bf16 [T][d] row-major
  *   T         tokens, >= 0 (T = 0 is a no-op)
  *   router_w  device, fp32 [E][d] row-major
  *   out_bf16  device, bf16 [T][d]; written completely, must not overlap x
  *   stream    CUDA stream (0 = legacy default stream)
- * Asynchronous on `stream`. */
+ * Asynchronous on `stream`.  Errors: MOE_FP4_ERR_INVALID_ARG (null handle or
+ * pointer, T < 0, a pointer not 16-byte aligned, out overlapping x),
+ * MOE_FP4_ERR_UNSUPPORTED (T * top_k >= 2^30), MOE_FP4_ERR_NOT_LOADED,
+ * MOE_FP4_ERR_OOM / MOE_FP4_ERR_CAPTURE (workspace growth), MOE_FP4_ERR_CUDA. */
 MOE_FP4_API int moe_fp4_forward(moe_fp4_t* h, const void* x_bf16, int T, const float* router_w,
                     void* out_bf16, cudaStream_t stream);
 
-/* Intermediates of a forward, for layer-by-layer comparison.  Every member
+/* Intermediates of a forward, for layer-by-layer comparison (the steps of
+ * the layer as moe_fp4_forward states them).  Every member
  * may be NULL; non-NULL members are device buffers the caller owns:
  *   logits   fp32  [T][E]
  *   topk_ids int32 [T][top_k]   listed by (logit desc, expert asc)
@@ -141,6 +183,8 @@ MOE_FP4_API int moe_fp4_forward(moe_fp4_t* h, const void* x_bf16, int T, const f
  *   perm     int32 [T*top_k]    perm[pos] = t*top_k + j, pairs sorted by (expert, t, j)
  *   h        fp32  [T*top_k][f] SiLU(g)*u per pair, rows in perm order
  *   partial  fp32  [T*top_k][d] w * (Wd h) per pair, rows in perm order
+ *                               (Wd h, unweighted, while the per-expert norm
+ *                               is on)
  * Copies are enqueued on `stream` after the forward. */
 typedef struct {
   float*   logits;
@@ -164,8 +208,97 @@ MOE_FP4_API int moe_fp4_forward_ex(moe_fp4_t* h, const void* x_bf16, int T, cons
 MOE_FP4_API int moe_fp4_forward_host(moe_fp4_t* h, const void* x_host, int T, const float* router_w,
                          void* out_host, cudaStream_t stream);
 
-/* Activation-precision threshold (see the top of this file); thr >= 1. */
+/* ---------------------------------------------------------------------------
+ * Expert parallelism: the layer split over G ranks (one GPU each), rank r
+ * owning the contiguous experts [r E/G, (r+1) E/G).  The pages run the MoE
+ * layer with its experts sharded across devices and the token rows exchanged
+ * through an all-to-all ("Optimizing Muse Spark Open on TPU v7 with
+ * SGLang-TorchTPU", section 8, "Sequence-parallel prefill": routing ids and
+ * weights travel with the tokens, the MoE output returns through an
+ * all-to-all; "Day-0 Inference Adaptation for Ultra-Large Sparse Models":
+ * expert-parallel deployment).  These calls are the device-side pieces; the
+ * exchange between them is the caller's (NCCL all-to-all of device buffers).
+ * Because the permutation orders pairs by expert, the rows bound for one rank
+ * form one contiguous run of the permuted order.
+ * ------------------------------------------------------------------------ */
+
+/* Routing of a forward without the experts: fp32 logits, top-k, weights,
+ * counts, offsets, the permutation and its inverse (layouts as in
+ * moe_fp4_debug; inv[t*top_k + j] = position of pair (t, j) in perm).  Any
+ * member may be NULL; non-NULL members are caller-owned device buffers.
+ * Needs no moe_fp4_load_experts.  Asynchronous on `stream`.  Errors as
+ * moe_fp4_forward (without MOE_FP4_ERR_NOT_LOADED). */
+typedef struct {
+  float*   logits;
+  int32_t* topk_ids;
+  float*   topk_w;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* perm;
+  int32_t* inv;
+} moe_fp4_routing;
+MOE_FP4_API int moe_fp4_route(moe_fp4_t* h, const void* x_bf16, int T, const float* router_w,
+                              moe_fp4_routing* r, cudaStream_t stream);
+
+/* rows[i] = x[perm[i] / top_k] for i < P: the token row of every pair in
+ * permutation order (bf16 [P][d]; x bf16 [T][d]).  No handle.  d a multiple
+ * of 8, x and rows 16-byte aligned, P <= T * top_k, every perm[i] in
+ * [0, T * top_k) (not checked).  Errors: MOE_FP4_ERR_INVALID_ARG,
+ * MOE_FP4_ERR_CUDA. */
+MOE_FP4_API int moe_fp4_gather_rows(const void* x_bf16, int T, int d, const int32_t* perm, int P,
+                                    int top_k, void* rows_bf16, cudaStream_t stream);
+
+/* The experts of this handle on rows the caller routed: row i (bf16 [n][d])
+ * goes to expert expert_ids[i] (0 <= id < E of this handle) with weight 1,
+ * and y_rows[i] (fp32 [n][d]) receives Wd (SiLU(Wg x) * (Wu x)) of that
+ * expert, unweighted.  The expert classes follow each expert's row count in
+ * the call, as in moe_fp4_forward.  The handle must have top_k = 1.  An id
+ * out of range records MOE_FP4_ERR_INVALID_ARG in the device error word and
+ * leaves that row's output undefined.  Errors: MOE_FP4_ERR_INVALID_ARG,
+ * MOE_FP4_ERR_UNSUPPORTED (top_k != 1), MOE_FP4_ERR_NOT_LOADED, as
+ * moe_fp4_forward otherwise. */
+MOE_FP4_API int moe_fp4_forward_routed(moe_fp4_t* h, const void* rows_bf16, int n, const int32_t* expert_ids,
+                                       float* y_rows, cudaStream_t stream);
+
+/* out[t] = bf16_rn( sum_j fl(topk_w[t][j] * y_rows[inv[t*top_k + j]]) ),
+ * slots j = 0..top_k-1 in order, fp32: the routing-weighted combine of
+ * expert outputs that came back in permutation order (y_rows fp32 [P][d],
+ * out bf16 [T][d]).  No handle.  Errors: MOE_FP4_ERR_INVALID_ARG,
+ * MOE_FP4_ERR_CUDA. */
+MOE_FP4_API int moe_fp4_combine_rows(const float* y_rows, const int32_t* inv, const float* topk_w, int T,
+                                     int top_k, int d, void* out_bf16, cudaStream_t stream);
+
+/* Activation-precision threshold (see the top of this file); thr >= 1.
+ * The split of a step's experts into a loop for few-row experts and one for
+ * many-row experts follows the Muse Spark page, section 5 (two expert loops
+ * chosen by per-expert row count).  Errors: MOE_FP4_ERR_INVALID_ARG. */
 MOE_FP4_API int moe_fp4_set_dense_threshold(moe_fp4_t* h, int thr);
+
+/* Per-expert output normalisation before the weighted sum (Muse Spark page,
+ * section 8: each expert's output is normalised before the routing-weighted
+ * sum, in the one fused combine pass).  With enable = 1 every later forward
+ * computes
+ *   out[t] = bf16( sum_j w[t,j] * y_j / sqrt(mean_i y_j[i]^2 + eps) ),
+ *   y_j = Wd[S_j] (SiLU(Wg[S_j] x) * (Wu[S_j] x)),
+ * an RMS norm over the d outputs of each expert with no learned gain;
+ * enable = 0 (the default) restores the plain weighted sum.  eps >= 0 and
+ * finite (ignored when enable = 0).  Errors: MOE_FP4_ERR_INVALID_ARG. */
+MOE_FP4_API int moe_fp4_set_expert_norm(moe_fp4_t* h, int enable, float eps);
+
+/* Bound of every device-side wait of this handle's kernels, in milliseconds
+ * (default 2000, or MOE_FP4_WAIT_TIMEOUT_MS at create time); ms >= 1.  A
+ * wait that exceeds it records MOE_FP4_ERR_DEVICE_TIMEOUT in the device error
+ * word and the kernel returns.  Errors: MOE_FP4_ERR_INVALID_ARG. */
+MOE_FP4_API int moe_fp4_set_wait_timeout_ms(moe_fp4_t* h, int ms);
+
+/* Test hook for the failure path (no counterpart on the pages): with
+ * enable = 1 the light-class down tiles wait for a completion count that is
+ * never reached, so each such wait runs out after the wait bound, records
+ * MOE_FP4_ERR_DEVICE_TIMEOUT and the kernel drains the copies it issued and
+ * returns; the forward's output is then undefined.  enable = 0 (default)
+ * restores normal operation.  After moe_fp4_get_device_error has read the
+ * error, the handle is usable again.  Errors: MOE_FP4_ERR_INVALID_ARG. */
+MOE_FP4_API int moe_fp4_set_unreachable_wait(moe_fp4_t* h, int enable);
 
 /* Stage timing (profiling hook).  With n = 9, every later forward records,
  * on the forward's stream, events[0] before the router, events[1] after the
@@ -183,8 +316,12 @@ MOE_FP4_API int moe_fp4_set_dense_threshold(moe_fp4_t* h, int thr);
  * would otherwise overlap through programmatic dependent launch. */
 MOE_FP4_API int moe_fp4_set_stage_events(moe_fp4_t* h, cudaEvent_t* events, int n);
 
-/* Read and clear the device error word (synchronises the handle's device).
- * *code receives MOE_FP4_OK or the first MOE_FP4_ERR_* a kernel recorded. */
+/* Read and clear the device error word (synchronises the handle's whole
+ * device, not only one stream, so it waits for other work on that device
+ * too).  *code receives MOE_FP4_OK or the first MOE_FP4_ERR_* a kernel
+ * recorded; after an error the handle's completion counters are reset so
+ * the next forward runs normally.  Errors: MOE_FP4_ERR_INVALID_ARG,
+ * MOE_FP4_ERR_CUDA. */
 MOE_FP4_API int moe_fp4_get_device_error(moe_fp4_t* h, int* code);
 
 /* Allocation-free routing: fp32 router logits, top-k (ties to the lower
@@ -204,7 +341,9 @@ MOE_FP4_API int moe_fp4_get_device_error(moe_fp4_t* h, int* code);
  *   MOE_FP4_ERR_UNSUPPORTED), E, top_k, d as in moe_fp4_create; pointers
  *   16-byte aligned (else MOE_FP4_ERR_INVALID_ARG).
  * The first call on each device looks the scratch array up on that device
- * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * (cudaGetSymbolAddress) and keeps the address for the life of the process;
+ * make that first call before any stream capture.  The kept address does not
+ * survive cudaDeviceReset: no call may follow a reset of that device.
  * Asynchronous on `stream`.  All calls share the one scratch array per
  * device: calls whose executions overlap on the GPU (different streams
  * without ordering) race and give undefined results. */
@@ -212,6 +351,12 @@ MOE_FP4_API int moe_fp4_get_device_error(moe_fp4_t* h, int* code);
 MOE_FP4_API int moe_fp4_route_topk_static(const void* x_bf16, int T, int d, const float* router_w,
                                           int E, int top_k, int32_t* topk_ids, float* topk_w,
                                           cudaStream_t stream);
+
+/* The CUDA runtime error behind the last MOE_FP4_ERR_CUDA returned to the
+ * calling thread (error name, text and the library source line), or "" if
+ * there was none.  The string is owned by the library and stays valid until
+ * the thread's next failing call. */
+MOE_FP4_API const char* moe_fp4_last_error_detail(void);
 
 /* Static text for a status code. */
 MOE_FP4_API const char* moe_fp4_status_string(int status);

@@ -25,6 +25,10 @@ class Experts(ctypes.Structure):
                                    "down_q", "down_sf", "down_gs")]
 
 
+class Routing(ctypes.Structure):
+    _fields_ = [(n, _vp) for n in ("logits", "topk_ids", "topk_w", "counts", "offsets", "perm", "inv")]
+
+
 class Debug(ctypes.Structure):
     _fields_ = [(n, _vp) for n in ("logits", "topk_ids", "topk_w", "counts", "offsets", "perm",
                                    "h", "partial")]
@@ -39,10 +43,20 @@ SIGNATURES = {
     "moe_fp4_forward_ex": (_i, [_vp, _vp, _i, _vp, _vp, _vp, ctypes.POINTER(Debug)]),
     "moe_fp4_forward_host": (_i, [_vp, _vp, _i, _vp, _vp, _vp]),
     "moe_fp4_set_dense_threshold": (_i, [_vp, _i]),
+    "moe_fp4_set_expert_norm": (_i, [_vp, _i, ctypes.c_float]),
+    "moe_fp4_route": (_i, [_vp, _vp, _i, _vp, ctypes.POINTER(Routing), _vp]),
+    "moe_fp4_gather_rows": (_i, [_vp, _i, _i, _vp, _i, _i, _vp, _vp]),
+    "moe_fp4_forward_routed": (_i, [_vp, _vp, _i, _vp, _vp, _vp]),
+    "moe_fp4_combine_rows": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
+    "moe_fp4_set_resident_classes": (_i, [_vp, _i, _i]),
+    "moe_fp4_device_bytes": (_i, [_vp, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]),
+    "moe_fp4_set_wait_timeout_ms": (_i, [_vp, _i]),
+    "moe_fp4_set_unreachable_wait": (_i, [_vp, _i]),
     "moe_fp4_get_device_error": (_i, [_vp, ctypes.POINTER(_i)]),
     "moe_fp4_set_stage_events": (_i, [_vp, ctypes.POINTER(_vp), _i]),
     "moe_fp4_route_topk_static": (_i, [_vp, _i, _i, _vp, _i, _i, _vp, _vp, _vp]),
     "moe_fp4_status_string": (ctypes.c_char_p, [_i]),
+    "moe_fp4_last_error_detail": (ctypes.c_char_p, []),
     "moe_fp4_destroy": (None, [_vp]),
 }
 
@@ -76,4 +90,6 @@ class MoeFp4Error(RuntimeError):
 
 def check(status: int, where: str) -> None:
     if status != 0:
+        if status == STATUS_CODE["MOE_FP4_ERR_CUDA"] and _lib is not None:
+            where = f"{where} [{_lib.moe_fp4_last_error_detail().decode()}]"
         raise MoeFp4Error(status, where)

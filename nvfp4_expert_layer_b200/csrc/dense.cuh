@@ -47,8 +47,10 @@ constexpr int kDenseStages = kDenseKStage == 128 ? 6 : 3;
 constexpr int kDenseN = 256;               // weight rows per tile (MMA N)
 constexpr int kDenseABytes = 128 * kDenseRowBytes;       // 128 rows of the M operand
 constexpr int kDenseBBytes = kDenseN * kDenseRowBytes;   // 256 rows of the N operand
-constexpr int kDenseSfaBytes = kDenseMmaPerStage / 2 * 4096;   // M-side K-pair units (sf_pair_offset)
-constexpr int kDenseSfbBytes = kDenseMmaPerStage * 4096;       // N-side 256-row units (sf_rowpair_offset)
+// Scale units in shared memory: each 1 KB unit of device memory four times in a row
+constexpr int kSfSmemUnit = kSfReplicas * kSfUnitBytes;
+constexpr int kDenseSfaBytes = kDenseMmaPerStage / 2 * kSfSmemUnit;   // M-side K-pair units (sf_pair_offset)
+constexpr int kDenseSfbBytes = kDenseMmaPerStage * kSfSmemUnit;       // N-side 256-row units (sf_rowpair_offset)
 constexpr int kDenseStageBytes = kDenseABytes + kDenseBBytes + kDenseSfaBytes + kDenseSfbBytes;
 constexpr uint32_t kDenseTmemCols = 512;
 constexpr uint32_t kDenseSfCols = kDenseMmaPerStage * (4 + 8);   // per stage: 4 M-side + 8 N-side columns per MMA
@@ -75,7 +77,7 @@ struct DenseParams {
   const float* gs;       // [3][E]
   int E;
   const int* perm;
-  const float* wts;
+  const float* wts;      // routing weight per pair; null: partials unweighted
   // gate/up outputs
   uint8_t* hq;           // [P_pad][f/2]
   uint8_t* hsf;          // scales of hq (sf_rowpair_offset layout, K = f)
@@ -93,7 +95,7 @@ struct DenseParams {
 // gather_x_dense_kernel: one block per 128-row tile of the padded dense
 //   rows: the codes and scales of token perm[row0 + i] / topk copied into the
 //   padded permutation order (scales assembled into whole sf_pair_offset
-//   units, written as four replicas with coalesced 16-byte stores).
+//   units, written with coalesced 16-byte stores).
 //   Rows past an expert's count up to its next multiple of 128 -- the rows a
 //   128-token tile reads -- are zeros; rows beyond are never read.
 // Each token is quantised once, however many dense experts it is routed to.
@@ -190,9 +192,8 @@ __global__ void __launch_bounds__(256) gather_x_dense_kernel(
         w[m] = t >= 0 ? reinterpret_cast<const uint32_t*>(xsf_tok + (size_t)t * (d / 16))[g] : 0u;
       }
       const uint4 v = make_uint4(w[0], w[1], w[2], w[3]);
-      uint8_t* unit = xsf + ((size_t)tile * npairs + pr) * (1024 * kSfReplicas);
-#pragma unroll
-      for (int rep = 0; rep < kSfReplicas; ++rep) reinterpret_cast<uint4*>(unit + 1024 * rep)[q] = v;
+      uint8_t* unit = xsf + ((size_t)tile * npairs + pr) * kSfUnitBytes;
+      reinterpret_cast<uint4*>(unit)[q] = v;
     }
   }
   pdl_launch_dependents();
@@ -284,8 +285,8 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
         const int trow = tl.de.w + tl.tt * (MODE == kDenseGateUp ? 128 : kDenseN);   // padded token row
         const int arow = MODE == kDenseGateUp ? trow : wrow;
         const int brow = MODE == kDenseGateUp ? wrow : trow;
-        const uint8_t* sfa = p.sfA + (size_t)(arow >> 7) * (p.kb64 >> 1) * 4096;
-        const uint8_t* sfb = p.sfB + (size_t)(brow >> 8) * p.kb64 * 4096;
+        const uint8_t* sfa = p.sfA + (size_t)(arow >> 7) * (p.kb64 >> 1) * kSfUnitBytes;
+        const uint8_t* sfb = p.sfB + (size_t)(brow >> 8) * p.kb64 * kSfUnitBytes;
         for (int ks = 0; ks < p.kstages; ++ks, ++k) {
           const int s = k % kDenseStages;
           if (!mbar_wait_spin(empty_b(s), ((k / kDenseStages) & 1) ^ 1, deadline)) {
@@ -295,10 +296,24 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
           mbar_arrive_expect_tx(full_b(s), kDenseStageBytes);
           tma_load_2d(st, &p.tmA, ks * kDenseRowBytes, arow, full_b(s), pol_a);
           tma_load_2d(st + kDenseABytes, &p.tmB, ks * kDenseRowBytes, brow, full_b(s), pol_w);
-          bulk_g2s(st + kDenseABytes + kDenseBBytes, sfa + (size_t)(kDenseMmaPerStage / 2) * ks * 4096,
-                   kDenseSfaBytes, full_b(s), pol_a);
-          bulk_g2s(st + kDenseABytes + kDenseBBytes + kDenseSfaBytes, sfb + (size_t)kDenseMmaPerStage * ks * 4096,
-                   kDenseSfbBytes, full_b(s), pol_w);
+          // scale units: each 1 KB unit is read from device memory once (its
+          // other three copies come from L2) into four consecutive 1 KB
+          // replicas, the source of one 128x256b copy
+          const uint8_t* sa = sfa + (size_t)(kDenseMmaPerStage / 2) * ks * kSfUnitBytes;
+          const uint8_t* sb = sfb + (size_t)kDenseMmaPerStage * ks * kSfUnitBytes;
+          const uint32_t da = st + kDenseABytes + kDenseBBytes, db = da + kDenseSfaBytes;
+#pragma unroll
+          for (int u = 0; u < kDenseMmaPerStage / 2; ++u)
+#pragma unroll
+            for (int rep = 0; rep < kSfReplicas; ++rep)
+              bulk_g2s(da + u * kSfSmemUnit + rep * kSfUnitBytes, sa + (size_t)u * kSfUnitBytes, kSfUnitBytes,
+                       full_b(s), pol_a);
+#pragma unroll
+          for (int u = 0; u < kDenseMmaPerStage; ++u)
+#pragma unroll
+            for (int rep = 0; rep < kSfReplicas; ++rep)
+              bulk_g2s(db + u * kSfSmemUnit + rep * kSfUnitBytes, sb + (size_t)u * kSfUnitBytes, kSfUnitBytes,
+                       full_b(s), pol_w);
         }
       }
       // drain: every issued stage must land before the block exits
@@ -334,10 +349,10 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
           const uint32_t sfa_t = sf_t0 + kDenseSfCols * s, sfb_t = sfa_t + 4 * kDenseMmaPerStage;
 #pragma unroll
           for (int pr = 0; pr < kDenseMmaPerStage / 2; ++pr)
-            tc_cp_128x256b(sfa_t + 8 * pr, smem_desc_sf256(sfa_s + 4096 * pr));
+            tc_cp_128x256b(sfa_t + 8 * pr, smem_desc_sf256(sfa_s + kSfSmemUnit * pr));
 #pragma unroll
           for (int kb = 0; kb < kDenseMmaPerStage; ++kb)
-            tc_cp_128x256b(sfb_t + 8 * kb, smem_desc_sf256(sfb_s + 4096 * kb));
+            tc_cp_128x256b(sfb_t + 8 * kb, smem_desc_sf256(sfb_s + kSfSmemUnit * kb));
           const uint64_t adesc = smem_desc_kmajor<kDenseRowBytes>(st);
           const uint64_t bdesc = smem_desc_kmajor<kDenseRowBytes>(st + kDenseABytes);
 #pragma unroll
@@ -401,7 +416,8 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
         for (int c32 = 0; c32 < 4; ++c32) {
           if (32 * c32 >= nrows) break;                              // warp-uniform
           // routing weight x tensor scale of column 32 c32 + lane, broadcast below
-          const float wl = 32 * c32 + lane < nrows ? p.wts[p.perm[prow0 + 32 * c32 + lane]] * gsd : 0.f;
+          const float wl = 32 * c32 + lane < nrows
+                               ? (p.wts ? p.wts[p.perm[prow0 + 32 * c32 + lane]] : 1.f) * gsd : 0.f;
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             const float wv = __shfl_sync(0xffffffffu, wl, c);
@@ -456,8 +472,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
         dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
         // the four blocks share one 64-wide K group: four consecutive scale bytes
         const size_t so = sf_rowpair_offset(hrow, chb >> 4, p.f / 64);
-#pragma unroll
-        for (int c = 0; c < kSfReplicas; ++c) *reinterpret_cast<uint32_t*>(p.hsf + so + 1024 * c) = sfw;
+        *reinterpret_cast<uint32_t*>(p.hsf + so) = sfw;
       }
     }
   }

@@ -63,12 +63,14 @@ struct ExpertParams {
   __half* h16;                // [P][f] B-fragment layout
   float* h32;                 // [P][f]
   const float* gs;            // [3][E] gate, up, down tensor scales
-  const float* wts;           // [P] routing weight per pair
+  const int* hexp;            // [E] exponent bound of |g| * |u| per expert (light_h_exp)
+  const float* wts;           // [P] routing weight per pair; null: partials unweighted
   float* partial;             // [P][d]
   int* gu_done;               // [max jobs] gate/up tiles finished per job
   int* exit_cnt;              // blocks that left
   int* err;
   int64_t wait_timeout_ns;
+  int wait_extra;             // test hook: added to every down tile's completion target (0)
 };
 
 __device__ __forceinline__ int ld_acquire(const int* p) {
@@ -80,6 +82,26 @@ __device__ __forceinline__ int ld_acquire(const int* p) {
 __device__ __forceinline__ void red_release_add(int* p, int v) {
   asm volatile("red.release.gpu.global.add.s32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
 }
+
+// fp16 staging exponent of h for one (token, expert) row of the light class.
+// h enters the down projection as fp16, so it is held as h * 2^e_h with e_h
+// chosen before any gate/up tile of the row runs, from a bound that every
+// tile can compute alike:
+//   the staged x row has max |x * 2^s| < 2^15, xs = 2^-s (stage_x_row), so
+//   max |x| < 2^(15 - s);  |g| <= |gs_g| * L1_g * max|x| < 2^(Eg + 15 - s) and
+//   |u| < 2^(Eu + 15 - s) (hexp = Eg + Eu, expert_hexp_kernel);  |SiLU(g)| <= |g|,
+//   so |h| < 2^(Eg + Eu + 30 - 2s).
+// e_h = 2s - 15 - hexp keeps |h| * 2^e_h below 2^15 (half of the fp16 range,
+// room for the fp32 rounding of g and u) whatever the magnitudes of x and the
+// weights, so h never overflows fp16, and values far below the bound lose
+// only absolute precision 2^-25 * 2^-e_h.  The exponent is clamped to +-120
+// (fp32 range); beyond that the overflow check still reports
+// MOE_FP4_ERR_NUMERIC.
+__device__ __forceinline__ int light_h_exp(float xs, int hexp_e) {
+  const int s = 127 - (int)((__float_as_uint(xs) >> 23) & 0xffu);   // xs = 2^-s, a normal float
+  return max(-120, min(120, 2 * s - 15 - hexp_e));
+}
+__device__ __forceinline__ float exp2i(int e) { return __int_as_float((e + 127) << 23); }
 
 __device__ __forceinline__ uint4 ldg_cg_v4(const void* p) {
   uint4 v;
@@ -350,7 +372,7 @@ __global__ void __launch_bounds__(kExpThreads, 4) expert_kernel(ExpertParams p) 
       if (lane == 0) {
         uint32_t n = 0;
         // every gate/up tile of the job is published once per writer warp (n-tile)
-        const int target = p.tpe_gu * ((ti.nrows + 7) >> 3);
+        const int target = p.tpe_gu * ((ti.nrows + 7) >> 3) + p.wait_extra;
         while (ld_acquire(p.gu_done + ti.job) < target) {
           __nanosleep(128);
           if ((++n & 15u) == 0 && globaltimer_ns() > deadline) { ok = 0; break; }
@@ -450,8 +472,9 @@ __global__ void __launch_bounds__(kExpThreads, 4) expert_kernel(ExpertParams p) 
             const float uv = v[2 + q] * gsu * xs;
             const float hv = gv / (1.f + expf(-gv)) * uv;
             p.h32[(size_t)r * p.f + fidx] = hv;
-            if (!(fabsf(hv) <= 65504.f)) set_error(p.err, kErrNumeric);
-            p.h16[(size_t)r * p.f + bfrag_offset(fidx)] = __float2half_rn(hv);
+            const float hs = hv * exp2i(light_h_exp(xs, p.hexp[ti.e]));
+            if (!(fabsf(hs) <= 65504.f)) set_error(p.err, kErrNumeric);
+            p.h16[(size_t)r * p.f + bfrag_offset(fidx)] = __float2half_rn(hs);
           }
         }
       } else {
@@ -462,7 +485,9 @@ __global__ void __launch_bounds__(kExpThreads, 4) expert_kernel(ExpertParams p) 
           const int n = nt * 8 + 2 * c + q;
           if (n < ti.nrows) {
             const int r = ti.row0 + n;
-            const float wv = p.wts[p.perm[r]] * gsd * kScaleUndo;
+            const int pr = p.perm[r];
+            const float hinv = exp2i(-light_h_exp(p.xscale[pr / p.topk], p.hexp[ti.e]));
+            const float wv = (p.wts ? p.wts[pr] : 1.f) * gsd * kScaleUndo * hinv;
             p.partial[(size_t)r * p.d + drow] = v[q] * wv;
             p.partial[(size_t)r * p.d + drow + 8] = v[2 + q] * wv;
           }

@@ -14,6 +14,7 @@
 #include <cstdint>
 #include <climits>
 #include <cstdlib>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 #include <new>
@@ -91,12 +92,20 @@ struct moe_fp4 {
   uint8_t* gu_frag = nullptr;     // gate/up fragment layout, all experts
   uint8_t* dn_frag = nullptr;     // down fragment layout, all experts
   float* gs = nullptr;            // [3][E]: gate, up, down
+  float* l1 = nullptr;            // [2][E]: largest gate / up row L1 norm (expert_l1_kernel)
+  int* hexp = nullptr;            // [E]: light-class h staging exponent bound (expert_hexp_kernel)
+  bool expert_norm = false;       // RMS-normalise each expert's output before the weighted sum
+  float norm_eps = 1e-6f;
+  int wait_extra = 0;             // test hook: unreachable down-tile completion target
   uint8_t* dq_gu = nullptr;       // dense class: gate/up codes, rows interleaved by 16, signs folded [E*2f][d/2]
   uint8_t* dq_down = nullptr;     // [E*d][f/2]
   uint8_t* dsf_gu = nullptr;      // weight scales, 256-row tile layout (sf_rowpair_offset), rows E*2f, K = d
   uint8_t* dsf_dn = nullptr;      // 128-row tile layout (sf_pair_offset), rows E*d, K = f
   CUtensorMap tm_gu{}, tm_down{};
   bool dense_ok = false;          // d, f multiples of 256 and tensor maps available
+  bool want_light = true;         // resident weight copies kept by the next load
+  bool want_dense = true;
+  size_t weight_bytes = 0;        // device bytes of the resident weight copies
   bool dense_h32 = false;         // write fp32 h of the dense class (debug copies)
   int* err = nullptr;             // device error word
   cudaEvent_t stage_ev[kStageEvents] = {};   // optional stage-timing events (caller-owned)
@@ -106,10 +115,21 @@ struct moe_fp4 {
 
 namespace {
 
+// The CUDA error behind the last MOE_FP4_ERR_CUDA of this thread, with the
+// source line that met it (moe_fp4_last_error_detail).
+thread_local char g_err_detail[256] = "";
+
+int cuda_fail(cudaError_t e, int line) {
+  snprintf(g_err_detail, sizeof(g_err_detail), "%s (%s) at moe_fp4.cu:%d", cudaGetErrorName(e),
+           cudaGetErrorString(e), line);
+  (void)cudaGetLastError();
+  return MOE_FP4_ERR_CUDA;
+}
+
 #define MOE_CUDA(call)                                  \
   do {                                                  \
     cudaError_t e_ = (call);                            \
-    if (e_ != cudaSuccess) { (void)cudaGetLastError(); return MOE_FP4_ERR_CUDA; } \
+    if (e_ != cudaSuccess) return cuda_fail(e_, __LINE__); \
   } while (0)
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -325,7 +345,17 @@ cudaError_t mark(moe_fp4* h, int i, cudaStream_t st) {
                                                                       : cudaEventRecordDefault);
 }
 
-int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cudaStream_t st) {
+// What a call runs besides the plain forward: routing only (stops after the
+// permutation), or rows the caller routed (pre_ids, one expert per row,
+// weight 1) whose unweighted expert outputs go to y_rows in row order.
+struct RunMode {
+  bool route_only = false;
+  const int* pre_ids = nullptr;
+  float* y_rows = nullptr;
+};
+
+int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cudaStream_t st,
+                const RunMode& mode = RunMode()) {
   Workspace& w = h->ws;
   const int E = h->E, k = h->k, d = h->d, f = h->f;
   const uint16_t* xb = static_cast<const uint16_t*>(x);
@@ -342,11 +372,23 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
   // Without the dense class (shape or tensor-map support missing) every
   // expert runs in the light class.  An expert holds at most T rows (one per
   // token), so below T = thr no expert can be dense and its kernels are skipped.
+  // with only the dense copy resident every expert runs in the dense class
+  const bool light_ok = h->gu_frag != nullptr;
   const int dense_ok = h->dense_ok ? 1 : 0;
-  const int thr = h->dense_ok ? h->thr : INT_MAX;
-  const bool run_dense = h->dense_ok && T >= h->thr;
+  // (routing alone needs no expert classes: every active expert counts as light)
+  const int thr = mode.route_only ? INT_MAX : !light_ok ? 1 : h->dense_ok ? h->thr : INT_MAX;
+  if (!light_ok && !h->dense_ok && !mode.route_only) return MOE_FP4_ERR_UNSUPPORTED;
+  const bool run_dense = h->dense_ok && T >= thr;
   const long long P = (long long)T * k;
-  if (T <= kSmallT) {
+  const bool small_path = T <= kSmallT && P <= 32 && !mode.pre_ids;
+  if (mode.pre_ids) {
+    // 1. rows routed by the caller: ids and unit weights, x staging
+    MOE_CUDA(launch(moe::preroute_kernel, dim3(std::min<long long>((P + 255) / 256, 8 * h->sm_count)), dim3(256), 0,
+                    st, false, mode.pre_ids, (int)P, E, w.ids, w.wts, w.inv, h->err));
+    MOE_CUDA(launch(moe::stage_x_kernel, dim3(std::min(T, 8 * h->sm_count)), dim3(256), 0, st, false,
+                    xb, T, d, w.x16, w.xscale, h->err));
+    MOE_CUDA(mark(h, 1, st));
+  } else if (T <= kSmallT) {
     // 1. router logits and x staging; at most 32 pairs: top-k and the
     // permutation in the same launch
     const int epb = route_epb(d), tail = P <= 32 ? 1 : 0;
@@ -384,12 +426,13 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
                     xb, T, d, w.x16, w.xscale, h->err));
     MOE_CUDA(mark(h, 1, st));
   }
-  if (P <= 32 && T <= kSmallT) {
+  if (small_path) {
     MOE_CUDA(mark(h, 2, st));
   } else {
     // 2. top-k, a warp per token
-    MOE_CUDA(launch(moe::topk_kernel, dim3((T + 7) / 8), dim3(256), 0, st, false,
-                    (const float*)w.logits, T, E, k, w.ids, w.wts));
+    if (!mode.pre_ids)
+      MOE_CUDA(launch(moe::topk_kernel, dim3((T + 7) / 8), dim3(256), 0, st, false,
+                      (const float*)w.logits, T, E, k, w.ids, w.wts));
     MOE_CUDA(mark(h, 2, st));
     // 3. permutation: per-block counts, one-block scan and classes, placement
     const int nb = (int)std::min<long long>(kPermMaxBlocks, std::max<long long>(1, (P + 1023) / 1024));
@@ -401,6 +444,9 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
                     (const int*)w.ids, P, E, (const int*)w.perm_bcnt, po));
   }
   MOE_CUDA(mark(h, 3, st));
+  if (mode.route_only) return MOE_FP4_OK;
+  // the norm and caller-routed rows need the unweighted expert outputs
+  const float* wts_epi = (h->expert_norm || mode.pre_ids) ? nullptr : w.wts;
   // 4-5 (dense class). NVFP4 activations, then the two tensor-core GEMMs
   if (run_dense) {
     MOE_CUDA(launch(moe::quant_tok_kernel, dim3(std::min((T + 7) / 8, 8 * h->sm_count)), dim3(256), 0, st,
@@ -427,7 +473,7 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
     dp.gs = h->gs;
     dp.E = E;
     dp.perm = w.perm;
-    dp.wts = w.wts;
+    dp.wts = wts_epi;
     dp.hq = w.hq;
     dp.hsf = w.hsf;
     dp.h32 = h->dense_h32 ? w.h32 : nullptr;
@@ -474,23 +520,37 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
   ep.h16 = w.h16;
   ep.h32 = w.h32;
   ep.gs = h->gs;
-  ep.wts = w.wts;
+  ep.hexp = h->hexp;
+  ep.wts = wts_epi;
+  ep.wait_extra = h->wait_extra;
   ep.partial = w.partial;
   ep.err = h->err;
   ep.wait_timeout_ns = h->wait_timeout_ns;
   moe::ExpertParams ep1 = ep, ep2 = ep;
   ep1.jobs = w.jobs1; ep1.njobs = w.n_jobs1; ep1.gu_done = gu_done1; ep1.exit_cnt = exit1;
   ep2.jobs = w.jobs2; ep2.njobs = w.n_jobs2; ep2.gu_done = gu_done2; ep2.exit_cnt = exit2;
-  MOE_CUDA(launch(moe::expert_kernel<1>, dim3(h->sm_count * h->exp_bps1), dim3(moe::kExpThreads),
-                  kExpSmem, st, pdl, ep1));
-  // jobs of 9..16 rows need an expert with at least 9 rows, i.e. T >= 9
-  if (T >= 9)
-    MOE_CUDA(launch(moe::expert_kernel<2>, dim3(h->sm_count * h->exp_bps2), dim3(moe::kExpThreads),
-                    kExpSmem, st, pdl, ep2));
+  if (light_ok) {
+    MOE_CUDA(launch(moe::expert_kernel<1>, dim3(h->sm_count * h->exp_bps1), dim3(moe::kExpThreads),
+                    kExpSmem, st, pdl, ep1));
+    // jobs of 9..16 rows need an expert with at least 9 rows, i.e. T >= 9
+    if (T >= 9)
+      MOE_CUDA(launch(moe::expert_kernel<2>, dim3(h->sm_count * h->exp_bps2), dim3(moe::kExpThreads),
+                      kExpSmem, st, pdl, ep2));
+  }
   MOE_CUDA(mark(h, 7, st));
-  // 7. combine / unpermute: out[t] = bf16(sum_j partial[inv[t,j]])
-  MOE_CUDA(launch(moe::combine_kernel, dim3((d + 1023) / 1024, T), dim3(128), 0, st, pdl,
-                  (const float*)w.partial, (const int*)w.inv, T, k, d, static_cast<uint16_t*>(out)));
+  // 7. combine / unpermute: out[t] = bf16(sum_j partial[inv[t,j]]), or with
+  // the per-expert norm bf16(sum_j w[t,j] * rmsnorm(partial[inv[t,j]]))
+  if (mode.pre_ids)
+    MOE_CUDA(launch(moe::unpermute_rows_kernel, dim3(std::min<long long>(((long long)T * d / 4 + 255) / 256,
+                                                                          8 * h->sm_count)),
+                    dim3(256), 0, st, pdl, (const float*)w.partial, (const int*)w.inv, T, d, mode.y_rows));
+  else if (h->expert_norm)
+    MOE_CUDA(launch(moe::combine_norm_kernel, dim3(std::min(T, 8 * h->sm_count)), dim3(moe::kNormThreads), 0,
+                    st, pdl, (const float*)w.partial, (const int*)w.inv, (const float*)w.wts, T, k, d,
+                    h->norm_eps, static_cast<uint16_t*>(out)));
+  else
+    MOE_CUDA(launch(moe::combine_kernel, dim3(std::min(T, 65535), (d + 1023) / 1024), dim3(128), 0, st, pdl,
+                    (const float*)w.partial, (const int*)w.inv, T, k, d, static_cast<uint16_t*>(out)));
   MOE_CUDA(mark(h, 8, st));
   return MOE_FP4_OK;
 }
@@ -513,6 +573,8 @@ int check_forward_args(moe_fp4* h, const void* x, int T, const float* rw, const 
 }  // namespace
 
 extern "C" {
+
+const char* moe_fp4_last_error_detail(void) { return g_err_detail; }
 
 const char* moe_fp4_status_string(int s) {
   switch (s) {
@@ -581,6 +643,8 @@ int moe_fp4_create(int E, int top_k, int d, int f, moe_fp4_t** out) {
     if (cudaMalloc(&h->err, sizeof(int)) != cudaSuccess) { rc = MOE_FP4_ERR_OOM; break; }
     if (cudaMemset(h->err, 0, sizeof(int)) != cudaSuccess) { rc = MOE_FP4_ERR_CUDA; break; }
     if (cudaMalloc(&h->gs, sizeof(float) * 3 * E) != cudaSuccess) { rc = MOE_FP4_ERR_OOM; break; }
+    if (cudaMalloc(&h->l1, sizeof(float) * 2 * E) != cudaSuccess) { rc = MOE_FP4_ERR_OOM; break; }
+    if (cudaMalloc(&h->hexp, sizeof(int) * E) != cudaSuccess) { rc = MOE_FP4_ERR_OOM; break; }
   } while (0);
   if (rc != MOE_FP4_OK) {
     (void)cudaGetLastError();
@@ -597,6 +661,8 @@ void moe_fp4_destroy(moe_fp4_t* h) {
   cudaFree(h->gu_frag);
   cudaFree(h->dn_frag);
   cudaFree(h->gs);
+  cudaFree(h->l1);
+  cudaFree(h->hexp);
   cudaFree(h->dq_gu);
   cudaFree(h->dq_down);
   cudaFree(h->dsf_gu);
@@ -613,17 +679,33 @@ int moe_fp4_load_experts(moe_fp4_t* h, const moe_fp4_experts* w) {
       !w->down_q || !w->down_sf || !w->down_gs)
     return MOE_FP4_ERR_INVALID_ARG;
   const int E = h->E, d = h->d, f = h->f;
+  const bool dense_shape = (d % 256 == 0) && (f % 256 == 0);
+  if (!h->want_light && !dense_shape) return MOE_FP4_ERR_UNSUPPORTED;
   const size_t gu_bytes = (size_t)E * (f / 8) * (d / moe::kChunkK) * moe::kChunkBytes;
   const size_t dn_bytes = (size_t)E * (d / 16) * (f / moe::kChunkK) * moe::kChunkBytes;
-  if (!h->gu_frag) {
-    if (cudaMalloc(&h->gu_frag, gu_bytes) != cudaSuccess) { (void)cudaGetLastError(); return MOE_FP4_ERR_OOM; }
-  }
-  if (!h->dn_frag) {
-    if (cudaMalloc(&h->dn_frag, dn_bytes) != cudaSuccess) { (void)cudaGetLastError(); return MOE_FP4_ERR_OOM; }
-  }
+  const size_t gu_codes = (size_t)E * f * d / 2, dn_codes = (size_t)E * d * f / 2;
+  const size_t gu_atoms = moe::sf_rowpair_bytes((long long)E * 2 * f, d);
+  const size_t dn_atoms = moe::sf_pair_bytes((long long)E * d, f);
   h->loaded = false;
   MOE_CUDA(cudaDeviceSynchronize());
-  {
+  // copies the caller does not keep are released before anything is allocated
+  auto release = [](uint8_t** p) { cudaFree(*p); *p = nullptr; };
+  if (!h->want_light) { release(&h->gu_frag); release(&h->dn_frag); }
+  if (!h->want_dense || !dense_shape) {
+    release(&h->dq_gu); release(&h->dq_down); release(&h->dsf_gu); release(&h->dsf_dn);
+    h->dense_ok = false;
+  }
+  auto alloc = [](uint8_t** p, size_t n) {
+    if (*p) return true;
+    if (cudaMalloc(p, n) != cudaSuccess) { (void)cudaGetLastError(); *p = nullptr; return false; }
+    return true;
+  };
+  h->weight_bytes = 0;
+  if (h->want_light) {
+    if (!alloc(&h->gu_frag, gu_bytes) || !alloc(&h->dn_frag, dn_bytes)) return MOE_FP4_ERR_OOM;
+    h->weight_bytes += gu_bytes + dn_bytes;
+  }
+  if (h->want_light) {
     const long long thr = (long long)E * (f / 8) * (d / moe::kChunkK) * 32;
     const int blocks = (int)std::min<long long>((thr + 255) / 256, 65535LL * 16);
     moe::repack_fragment_kernel<moe::kGateUp><<<blocks, 256>>>(w->gate_q, w->gate_sf, w->up_q, w->up_sf,
@@ -638,25 +720,18 @@ int moe_fp4_load_experts(moe_fp4_t* h, const moe_fp4_experts* w) {
     MOE_CUDA(cudaGetLastError());
   }
   // dense class: codes with block-scale signs folded, scale atoms, tensor maps
-  {
-    const size_t gu_codes = (size_t)E * f * d / 2, dn_codes = (size_t)E * d * f / 2;
-    const size_t gu_atoms = moe::sf_rowpair_bytes((long long)E * 2 * f, d);
-    const size_t dn_atoms = moe::sf_pair_bytes((long long)E * d, f);
-    auto alloc = [](uint8_t** p, size_t n) {
-      if (*p) return true;
-      if (cudaMalloc(p, n) != cudaSuccess) { (void)cudaGetLastError(); *p = nullptr; return false; }
-      return true;
-    };
+  if (h->want_dense && dense_shape) {
     if (!alloc(&h->dq_gu, 2 * gu_codes) || !alloc(&h->dq_down, dn_codes) ||
         !alloc(&h->dsf_gu, gu_atoms) || !alloc(&h->dsf_dn, dn_atoms))
       return MOE_FP4_ERR_OOM;
+    h->weight_bytes += 2 * gu_codes + dn_codes + gu_atoms + dn_atoms;
     const int blocks = h->sm_count * 8;
     moe::dense_gu_codes_kernel<<<blocks, 256>>>(w->gate_q, w->gate_sf, w->up_q, w->up_sf, E, f, d, h->dq_gu);
     moe::dense_codes_kernel<<<blocks, 256>>>(w->down_q, w->down_sf, (long long)E * d, f, h->dq_down);
     moe::dense_sf_atoms_kernel<moe::kGateUp><<<blocks, 256>>>(w->gate_sf, w->up_sf, E, f, d, h->dsf_gu);
     moe::dense_sf_atoms_kernel<moe::kDown><<<blocks, 256>>>(w->down_sf, nullptr, E, d, f, h->dsf_dn);
     MOE_CUDA(cudaGetLastError());
-    h->dense_ok = (d % 256 == 0) && (f % 256 == 0) &&
+    h->dense_ok = dense_shape &&
                   make_map(&h->tm_gu, h->dq_gu, d / 2, (uint64_t)E * 2 * f, moe::kDenseN) &&
                   make_map(&h->tm_down, h->dq_down, f / 2, (uint64_t)E * d, 128);
     if (h->ws.base && (!make_map(&h->ws.tm_x, h->ws.xq, d / 2, h->ws.pad_rows, 128) ||
@@ -666,8 +741,31 @@ int moe_fp4_load_experts(moe_fp4_t* h, const moe_fp4_experts* w) {
   MOE_CUDA(cudaMemcpy(h->gs, w->gate_gs, sizeof(float) * E, cudaMemcpyDeviceToDevice));
   MOE_CUDA(cudaMemcpy(h->gs + E, w->up_gs, sizeof(float) * E, cudaMemcpyDeviceToDevice));
   MOE_CUDA(cudaMemcpy(h->gs + 2 * E, w->down_gs, sizeof(float) * E, cudaMemcpyDeviceToDevice));
+  // light class: exponent bound of |g| * |u| per expert (h's fp16 staging scale)
+  MOE_CUDA(cudaMemset(h->l1, 0, sizeof(float) * 2 * E));
+  moe::expert_l1_kernel<<<h->sm_count * 8, 256>>>(w->gate_q, w->gate_sf, w->up_q, w->up_sf, E, f, d, h->l1);
+  moe::expert_hexp_kernel<<<(E + 255) / 256, 256>>>(h->l1, h->gs, E, h->hexp);
+  MOE_CUDA(cudaGetLastError());
   MOE_CUDA(cudaDeviceSynchronize());
+  if (!h->want_light && !h->dense_ok) return MOE_FP4_ERR_UNSUPPORTED;   // tensor maps unavailable
   h->loaded = true;
+  return MOE_FP4_OK;
+}
+
+int moe_fp4_set_resident_classes(moe_fp4_t* h, int light, int dense) {
+  if (!h || (light != 0 && light != 1) || (dense != 0 && dense != 1) || (!light && !dense))
+    return MOE_FP4_ERR_INVALID_ARG;
+  if (!light && (h->d % 256 || h->f % 256)) return MOE_FP4_ERR_UNSUPPORTED;
+  h->want_light = light != 0;
+  h->want_dense = dense != 0;
+  h->loaded = false;                       // takes effect at the next load
+  return MOE_FP4_OK;
+}
+
+int moe_fp4_device_bytes(moe_fp4_t* h, size_t* weights, size_t* workspace) {
+  if (!h || !weights || !workspace) return MOE_FP4_ERR_INVALID_ARG;
+  *weights = h->weight_bytes;
+  *workspace = h->ws.bytes;
   return MOE_FP4_OK;
 }
 
@@ -680,6 +778,27 @@ int moe_fp4_reserve(moe_fp4_t* h, int max_T) {
 int moe_fp4_set_dense_threshold(moe_fp4_t* h, int thr) {
   if (!h || thr < 1) return MOE_FP4_ERR_INVALID_ARG;
   h->thr = thr;
+  return MOE_FP4_OK;
+}
+
+int moe_fp4_set_expert_norm(moe_fp4_t* h, int enable, float eps) {
+  if (!h || (enable != 0 && enable != 1)) return MOE_FP4_ERR_INVALID_ARG;
+  if (enable && !(eps >= 0.f && eps < INFINITY)) return MOE_FP4_ERR_INVALID_ARG;
+  if (enable && h->k > moe::kNormMaxK) return MOE_FP4_ERR_UNSUPPORTED;
+  h->expert_norm = enable != 0;
+  if (enable) h->norm_eps = eps;
+  return MOE_FP4_OK;
+}
+
+int moe_fp4_set_wait_timeout_ms(moe_fp4_t* h, int ms) {
+  if (!h || ms < 1) return MOE_FP4_ERR_INVALID_ARG;
+  h->wait_timeout_ns = (int64_t)ms * 1000000LL;
+  return MOE_FP4_OK;
+}
+
+int moe_fp4_set_unreachable_wait(moe_fp4_t* h, int enable) {
+  if (!h || (enable != 0 && enable != 1)) return MOE_FP4_ERR_INVALID_ARG;
+  h->wait_extra = enable ? (1 << 30) : 0;
   return MOE_FP4_OK;
 }
 
@@ -713,6 +832,81 @@ int moe_fp4_forward_ex(moe_fp4_t* h, const void* x, int T, const float* rw, void
   if ((rc = cp(dbg->perm, w.perm, P * 4))) return rc;
   if ((rc = cp(dbg->h, w.h32, P * h->f * 4))) return rc;
   if ((rc = cp(dbg->partial, w.partial, P * h->d * 4))) return rc;
+  return MOE_FP4_OK;
+}
+
+int moe_fp4_route(moe_fp4_t* h, const void* x, int T, const float* rw, moe_fp4_routing* r,
+                  cudaStream_t stream) {
+  if (!h || T < 0 || !r) return MOE_FP4_ERR_INVALID_ARG;
+  if (T == 0) return MOE_FP4_OK;
+  if (!x || !rw) return MOE_FP4_ERR_INVALID_ARG;
+  if ((long long)T * h->k >= (1LL << 30)) return MOE_FP4_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(rw)) & 15) return MOE_FP4_ERR_INVALID_ARG;
+  int rc = ensure_workspace(h, T, stream);
+  if (rc != MOE_FP4_OK) return rc;
+  RunMode mode;
+  mode.route_only = true;
+  rc = run_forward(h, x, T, rw, nullptr, stream, mode);
+  if (rc != MOE_FP4_OK) return rc;
+  const Workspace& w = h->ws;
+  const size_t P = (size_t)T * h->k;
+  auto cp = [&](void* dst, const void* src, size_t bytes) -> int {
+    if (!dst) return MOE_FP4_OK;
+    MOE_CUDA(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, stream));
+    return MOE_FP4_OK;
+  };
+  if ((rc = cp(r->logits, w.logits, (size_t)T * h->E * 4))) return rc;
+  if ((rc = cp(r->topk_ids, w.ids, P * 4))) return rc;
+  if ((rc = cp(r->topk_w, w.wts, P * 4))) return rc;
+  if ((rc = cp(r->counts, w.counts, (size_t)h->E * 4))) return rc;
+  if ((rc = cp(r->offsets, w.offsets, (size_t)(h->E + 1) * 4))) return rc;
+  if ((rc = cp(r->perm, w.perm, P * 4))) return rc;
+  if ((rc = cp(r->inv, w.inv, P * 4))) return rc;
+  return MOE_FP4_OK;
+}
+
+int moe_fp4_forward_routed(moe_fp4_t* h, const void* rows, int n, const int32_t* expert_ids, float* y_rows,
+                           cudaStream_t stream) {
+  if (!h || n < 0) return MOE_FP4_ERR_INVALID_ARG;
+  if (h->k != 1) return MOE_FP4_ERR_UNSUPPORTED;
+  if (n == 0) return MOE_FP4_OK;
+  if (!rows || !expert_ids || !y_rows) return MOE_FP4_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(rows) | reinterpret_cast<uintptr_t>(y_rows)) & 15) return MOE_FP4_ERR_INVALID_ARG;
+  if (ranges_overlap(rows, (size_t)n * h->d * 2, y_rows, (size_t)n * h->d * 4)) return MOE_FP4_ERR_INVALID_ARG;
+  if (!h->loaded) return MOE_FP4_ERR_NOT_LOADED;
+  int rc = ensure_workspace(h, n, stream);
+  if (rc != MOE_FP4_OK) return rc;
+  RunMode mode;
+  mode.pre_ids = expert_ids;
+  mode.y_rows = y_rows;
+  return run_forward(h, rows, n, nullptr, nullptr, stream, mode);
+}
+
+int moe_fp4_gather_rows(const void* x, int T, int d, const int32_t* perm, int P, int top_k, void* rows,
+                        cudaStream_t stream) {
+  if (T < 0 || P < 0 || top_k < 1 || d < 8 || d % 8) return MOE_FP4_ERR_INVALID_ARG;
+  if (P == 0) return MOE_FP4_OK;
+  if (!x || !perm || !rows || (long long)P > (long long)T * top_k) return MOE_FP4_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(rows)) & 15) return MOE_FP4_ERR_INVALID_ARG;
+  int sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  (void)cudaGetLastError();
+  const long long chunks = (long long)P * (d / 8);
+  MOE_CUDA(launch(moe::gather_rows_kernel, dim3((unsigned)std::min<long long>((chunks + 255) / 256, 8LL * sms)),
+                  dim3(256), 0, stream, false, static_cast<const uint16_t*>(x), (const int*)perm, P, top_k, d,
+                  static_cast<uint16_t*>(rows)));
+  return MOE_FP4_OK;
+}
+
+int moe_fp4_combine_rows(const float* y_rows, const int32_t* inv, const float* topk_w, int T, int top_k, int d,
+                         void* out, cudaStream_t stream) {
+  if (T < 0 || top_k < 1 || d < 8 || d % 8) return MOE_FP4_ERR_INVALID_ARG;
+  if (T == 0) return MOE_FP4_OK;
+  if (!y_rows || !inv || !topk_w || !out) return MOE_FP4_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(y_rows) | reinterpret_cast<uintptr_t>(out)) & 15) return MOE_FP4_ERR_INVALID_ARG;
+  MOE_CUDA(launch(moe::combine_rows_kernel, dim3(std::min(T, 65535), (d + 1023) / 1024), dim3(128), 0, stream,
+                  false, y_rows, (const int*)inv, topk_w, T, top_k, d, static_cast<uint16_t*>(out)));
   return MOE_FP4_OK;
 }
 

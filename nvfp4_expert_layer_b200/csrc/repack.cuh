@@ -75,6 +75,59 @@ __global__ void repack_fragment_kernel(const uint8_t* __restrict__ qa, const uin
 
 
 // ---------------------------------------------------------------------------
+// Largest row L1 norm of each expert's gate and up matrices, in units of
+// e2m1 value x e4m3 block scale (the fp32 tensor scale is applied later):
+//   l1[m * E + e] = max over rows c of sum_k |e2m1(q[c,k])| * |e4m3(sf[c,k/16])|
+// for m = 0 (gate), 1 (up).  One warp per row; the per-expert maximum is taken
+// with an integer atomicMax on the bits of the non-negative fp32 sums (order
+// independent, so the result is deterministic).  l1 must be zero on entry.
+// The light class uses it to bound |g| and |u| before any row is computed
+// (see light_h_exp in experts.cuh).
+// ---------------------------------------------------------------------------
+__global__ void expert_l1_kernel(const uint8_t* __restrict__ gq, const uint8_t* __restrict__ gsf,
+                                 const uint8_t* __restrict__ uq, const uint8_t* __restrict__ usf,
+                                 int E, int f, int d, float* __restrict__ l1) {
+  // twice the e2m1 magnitude of codes 0..7 (0, 1, 2, 3, 4, 6, 8, 12), one per nibble
+  constexpr uint32_t kTwiceMag = 0xC8643210u;
+  const int lane = threadIdx.x & 31;
+  const long long rows = 2LL * E * f;
+  const int nb = d / 16;
+  for (long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < rows;
+       w += ((long long)gridDim.x * blockDim.x) >> 5) {
+    const int m = (int)(w / ((long long)E * f));
+    const long long r = w - (long long)m * E * f;      // row of the [E*f] matrix
+    const uint8_t* q = (m ? uq : gq) + r * (d / 2);
+    const uint8_t* sf = (m ? usf : gsf) + r * nb;
+    float acc = 0.f;
+    for (int b = lane; b < nb; b += 32) {
+      const uint2 v = *reinterpret_cast<const uint2*>(q + b * 8);
+      uint32_t s = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t byte = ((i < 4 ? v.x : v.y) >> (8 * (i & 3))) & 0xffu;
+        s += ((kTwiceMag >> (4 * (byte & 7u))) & 15u) + ((kTwiceMag >> (4 * ((byte >> 4) & 7u))) & 15u);
+      }
+      acc += fabsf(e4m3_to_f32(sf[b])) * (0.5f * (float)s);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) atomicMax(reinterpret_cast<int*>(l1) + (size_t)m * E + r / f, __float_as_int(acc));
+  }
+}
+
+// hexp[e] = Eg + Eu with |gs_g| * l1_g < 2^Eg and |gs_u| * l1_u < 2^Eu
+// (frexp exponents; 0 for a zero matrix).  gs: [3][E] tensor scales.
+__global__ void expert_hexp_kernel(const float* __restrict__ l1, const float* __restrict__ gs, int E,
+                                   int* __restrict__ hexp) {
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < E; e += gridDim.x * blockDim.x) {
+    int eg = 0, eu = 0;
+    frexpf(fabsf(gs[e]) * l1[e], &eg);
+    frexpf(fabsf(gs[E + e]) * l1[E + e], &eu);
+    hexp[e] = eg + eu;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Dense-class weight copies for the tensor cores.  The block-scaled MMA reads
 // unsigned e4m3 scales, so a negative block scale is folded into the codes:
 // the 16 codes of that block change sign and the scale's sign bit is cleared
@@ -148,8 +201,7 @@ __global__ void dense_sf_atoms_kernel(const uint8_t* __restrict__ sfa, const uin
     const uint8_t v = src[row * nb + kb] & 0x7Fu;
     // gate/up weights are the N = 256 operand, down weights the M = 128 one
     const size_t o = MODE == kGateUp ? sf_rowpair_offset(R, kb, K / 64) : sf_pair_offset(R, kb, K / 64);
-#pragma unroll
-    for (int c = 0; c < kSfReplicas; ++c) out[o + 1024 * c] = v;
+    out[o] = v;
   }
 }
 

@@ -135,6 +135,25 @@ __global__ void __launch_bounds__(256) router_tiled_kernel(
     }
 }
 
+// Rows routed by the caller (one expert per row, weight 1): the ids are
+// copied into the workspace, the weights set to 1 and inv cleared to -1; an
+// id outside [0, E) records MOE_FP4_ERR_INVALID_ARG in the device error word
+// and is replaced by -1, which the permutation kernels skip (its inv stays -1).
+__global__ void __launch_bounds__(256) preroute_kernel(const int* __restrict__ in_ids, int n, int E,
+                                                       int* __restrict__ ids, float* __restrict__ wts,
+                                                       int* __restrict__ inv, int* err) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    int e = in_ids[i];
+    if (e < 0 || e >= E) {
+      set_error(err, 1);
+      e = -1;
+    }
+    ids[i] = e;
+    wts[i] = 1.f;
+    inv[i] = -1;            // the permutation writes the position of every valid row
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Top-k: one warp per token.  Lane l holds logits e = l + 32 i.  k rounds of a
 // warp arg-max ordered by (logit desc, expert asc); weights are the softmax of

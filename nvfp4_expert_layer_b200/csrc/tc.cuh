@@ -134,41 +134,43 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
 
 // Byte offset of the scale of (row r, K block kb of 16) in the scale layout of
 // the tensor-core operands.  Rows are grouped by 128 (one MMA tile) and K by
-// pairs of 64-wide groups (two MMAs); each (row tile, pair) is a 4 KB unit:
-// four identical 1 KB replicas, each holding 32 row slots l = r % 32 as 8-row
-// core matrices at
+// pairs of 64-wide groups (two MMAs); each (row tile, pair) is a 1 KB unit
+// holding 32 row slots l = r % 32 as 8-row core matrices at
 //   (l / 8) * 256 + h * 128 + (l % 8) * 16 + (r % 128 / 32) * 4 + kb % 4,
-// h = which 64-group of the pair.  The unit is the 128-row source of one
-// tcgen05.cp .128x256b, which gives every TMEM lane quarter the same 32 x 8
-// columns: column 4h + (r % 128) / 32 of lane r % 32 holds the four scales of
-// row r for the MMA of 64-group h.  Writers store the byte at this offset and
-// at +1024, +2048, +3072.  Size: rows / 128 * (K / 128) * 4096 bytes.
+// h = which 64-group of the pair.  Device memory holds each unit once; the
+// GEMMs place it four times in a row in shared memory (kSfReplicas), which
+// makes the 4 KB, 128-row source of one tcgen05.cp .128x256b that gives
+// every TMEM lane quarter the same 32 x 8 columns: column 4h + (r % 128) / 32
+// of lane r % 32 holds the four scales of row r for the MMA of 64-group h.
+// Size in device memory: rows / 128 * (K / 128) * 1024 bytes.
 constexpr int kSfReplicas = 4;
+constexpr int kSfUnitBytes = 1024;
 __host__ __device__ __forceinline__ size_t sf_pair_offset(long long r, int kb, int kblocks64) {
   const long long tile = r >> 7;
   const int rr = (int)(r & 127), l = rr & 31, kg = kb >> 2;
-  return ((size_t)tile * (kblocks64 >> 1) + (kg >> 1)) * (1024 * kSfReplicas) +
+  return ((size_t)tile * (kblocks64 >> 1) + (kg >> 1)) * kSfUnitBytes +
          (size_t)((l >> 3) * 256 + (kg & 1) * 128 + (l & 7) * 16 + (rr >> 5) * 4 + (kb & 3));
 }
 __host__ __device__ constexpr size_t sf_pair_bytes(long long rows, int K) {
-  return (size_t)(rows / 128) * (K / 128) * 1024 * kSfReplicas;
+  return (size_t)(rows / 128) * (K / 128) * kSfUnitBytes;
 }
 
-// Scale layout of an operand read as 256-row MMA tiles (N = 256): 4 KB units
-// per (256-row group, 64-wide K group), four identical 1 KB replicas with 32
-// row slots l = r % 32 as core matrices at
+// Scale layout of an operand read as 256-row MMA tiles (N = 256): 1 KB units
+// per (256-row group, 64-wide K group) with 32 row slots l = r % 32 as core
+// matrices at
 //   (l / 8) * 256 + h * 128 + (l % 8) * 16 + (r % 128 / 32) * 4 + kb % 4,
-// h = (r % 256) / 128.  One tcgen05.cp .128x256b of a unit fills the 8 scale
-// columns one N = 256 MMA reads: column (r % 256) / 32 of lane r % 32, in
-// every lane quarter.  Size: rows / 256 * (K / 64) * 4096 bytes.
+// h = (r % 256) / 128.  Stored once in device memory and four times in a row
+// in shared memory, where one tcgen05.cp .128x256b of the 4 KB fills the 8
+// scale columns one N = 256 MMA reads: column (r % 256) / 32 of lane r % 32,
+// in every lane quarter.  Size: rows / 256 * (K / 64) * 1024 bytes.
 __host__ __device__ __forceinline__ size_t sf_rowpair_offset(long long r, int kb, int kblocks64) {
   const long long g = r >> 8;
   const int rr = (int)(r & 255), h = rr >> 7, r128 = rr & 127, l = r128 & 31;
-  return ((size_t)g * kblocks64 + (kb >> 2)) * (1024 * kSfReplicas) +
+  return ((size_t)g * kblocks64 + (kb >> 2)) * kSfUnitBytes +
          (size_t)((l >> 3) * 256 + h * 128 + (l & 7) * 16 + (r128 >> 5) * 4 + (kb & 3));
 }
 __host__ __device__ constexpr size_t sf_rowpair_bytes(long long rows, int K) {
-  return (size_t)(rows / 256) * (K / 64) * 1024 * kSfReplicas;
+  return (size_t)(rows / 256) * (K / 64) * kSfUnitBytes;
 }
 
 }  // namespace moe

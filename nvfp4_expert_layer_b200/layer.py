@@ -50,6 +50,31 @@ class MoeFp4Layer:
     def set_dense_threshold(self, thr: int) -> None:
         _lib.check(self.lib.moe_fp4_set_dense_threshold(self._h, thr), "moe_fp4_set_dense_threshold")
 
+    def set_resident_classes(self, light: bool = True, dense: bool = True) -> None:
+        """Weight copies the next load_experts keeps (see moe_fp4.h)."""
+        _lib.check(self.lib.moe_fp4_set_resident_classes(self._h, int(light), int(dense)),
+                   "moe_fp4_set_resident_classes")
+
+    def device_bytes(self) -> tuple:
+        """(weight bytes, workspace bytes) the handle holds on the device."""
+        wb, sb = ctypes.c_size_t(0), ctypes.c_size_t(0)
+        _lib.check(self.lib.moe_fp4_device_bytes(self._h, ctypes.byref(wb), ctypes.byref(sb)),
+                   "moe_fp4_device_bytes")
+        return wb.value, sb.value
+
+    def set_expert_norm(self, enable: bool, eps: float = 1e-6) -> None:
+        """RMS-normalise each expert's output before the weighted sum (see moe_fp4.h)."""
+        _lib.check(self.lib.moe_fp4_set_expert_norm(self._h, 1 if enable else 0, eps),
+                   "moe_fp4_set_expert_norm")
+
+    def set_wait_timeout_ms(self, ms: int) -> None:
+        _lib.check(self.lib.moe_fp4_set_wait_timeout_ms(self._h, ms), "moe_fp4_set_wait_timeout_ms")
+
+    def set_unreachable_wait(self, enable: bool) -> None:
+        """Test hook: light-class down tiles wait for a count that is never reached."""
+        _lib.check(self.lib.moe_fp4_set_unreachable_wait(self._h, 1 if enable else 0),
+                   "moe_fp4_set_unreachable_wait")
+
     STAGES = ("router", "topk", "permute", "dense_quant", "dense_gate_up", "dense_down", "light", "combine")
 
     def set_stage_events(self, events) -> None:

@@ -43,7 +43,7 @@ Readings where the pages are silent (each is stated where it is used):
      (token, slot) pairs by (expert, token, slot).
   R6 a token whose k-th and (k+1)-th fp64 logits differ by less than 1e-6 is a
      near-tie and is excluded from id / output comparisons.
-  R7 the optional per-expert output normalisation ([P2-S8]) is an RMS norm
+  R12 the optional per-expert output normalisation ([P2-S8]) is an RMS norm
      over the d outputs of each expert, y / sqrt(mean(y^2) + eps), with no
      learned gain and eps chosen by the caller (the pages give neither).
 """
@@ -295,9 +295,38 @@ def expert_ffn(xrows: np.ndarray, Wg: np.ndarray, Wu: np.ndarray, Wd: np.ndarray
 def expert_rms_norm(y: np.ndarray, eps: float) -> np.ndarray:
     """Per-expert output normalisation  y / sqrt(mean_i y_i^2 + eps) over the
     d outputs of each row, with no learned gain ([P2-S8]: each expert's output
-    is normalised before the weighted sum; reading R7: an RMS norm, eps given
+    is normalised before the weighted sum; reading R12: an RMS norm, eps given
     by the caller)."""
     return y / np.sqrt(np.mean(y * y, axis=-1, keepdims=True) + eps)
+
+
+class PairRows:
+    """Per-pair values of a forward, stored only for the pairs evaluated.
+
+    Indexed like a [P, cols] array by permutation row (an int, an int array,
+    or (rows, cols)); rows that were not evaluated read as NaN."""
+
+    def __init__(self, P: int, cols: int):
+        self.shape = (P, cols)
+        self._index = np.full(P, -1, dtype=np.int64)
+        self._blocks = []
+        self._data = None
+
+    def _put(self, pos: np.ndarray, values: np.ndarray):
+        n0 = sum(b.shape[0] for b in self._blocks)
+        self._index[pos] = n0 + np.arange(len(pos))
+        self._blocks.append(np.asarray(values, dtype=np.float64))
+        self._data = None
+
+    def _rows(self, r):
+        if self._data is None:
+            self._data = np.concatenate(self._blocks + [np.full((1, self.shape[1]), np.nan)])
+        return self._data[self._index[r]]          # index -1 -> the NaN row
+
+    def __getitem__(self, key):
+        if isinstance(key, tuple):
+            return self._rows(key[0])[(Ellipsis,) + key[1:]]
+        return self._rows(key)
 
 
 def _expert_rows(task):
@@ -326,8 +355,8 @@ def forward(x_bits: np.ndarray, router_w: np.ndarray, experts, E: int, k: int,
     either way, so the output does not depend on it).
     Returns a dict with logits, ids, w, gap, counts, offsets, perm, inv, the
     per-pair h, y (the expert output Wd h) and partial (its contribution to
-    the output; rows in perm order; NaN where not evaluated), out64 and the
-    bf16 output bits (rows outside the subset are 0)."""
+    the output; PairRows indexed by permutation row, NaN where not
+    evaluated), out64 and the bf16 output bits (rows outside the subset are 0)."""
     T, d = x_bits.shape
     logits = router_logits(x_bits, router_w)
     ids, w, gap = route(logits, k)
@@ -359,22 +388,19 @@ def forward(x_bits: np.ndarray, router_w: np.ndarray, experts, E: int, k: int,
     for (e, pos, pairs, toks, _), res in zip(work, results):
         h, y = res[0], res[1]
         if want_pairs and h_all is None:
-            f = h.shape[1]
-            h_all = np.full((P, f), np.nan)
-            partial_all = np.full((P, d), np.nan)
-            y_all = np.full((P, d), np.nan)
+            h_all, partial_all, y_all = PairRows(P, h.shape[1]), PairRows(P, d), PairRows(P, d)
         if magnitudes:
             if mags is None:
-                mags = {n: np.full((P, v.shape[1]), np.nan) for n, v in res[2].items()}
+                mags = {n: PairRows(P, v.shape[1]) for n, v in res[2].items()}
             for n, v in res[2].items():
-                mags[n][pos] = v
+                mags[n]._put(pos, v)
         wj = w.reshape(-1)[pairs]
         yn = y if expert_norm_eps is None else expert_rms_norm(y, expert_norm_eps)
         contrib = wj[:, None] * yn
         if want_pairs:
-            h_all[pos] = h
-            y_all[pos] = y
-            partial_all[pos] = contrib
+            h_all._put(pos, h)
+            y_all._put(pos, y)
+            partial_all._put(pos, contrib)
         np.add.at(out64, toks, contrib)
     out_bits = f64_to_bf16_bits_rne(out64)
     return dict(logits=logits, ids=ids, w=w, gap=gap, counts=counts, offsets=offsets,

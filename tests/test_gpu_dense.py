@@ -4,12 +4,15 @@ Experts that receive at least `thr` rows quantise x and h to NVFP4 and run on
 the FP4 tensor cores; the oracle applies the same activation quantiser
 (reading R4) and the parity helpers bound the effect of quantiser decisions
 that may round the other way when h moves inside its accumulation bound."""
+import os
+
 import numpy as np
 import pytest
 import torch
 
 from nvfp4_expert_layer_b200 import workloads as W
 from nvfp4_expert_layer_b200.layer import MoeFp4Layer, experts_to_device
+from oracle import moe_oracle as O
 from tests.parity import Case, bf16_to_bits, to_dev_x
 
 pytestmark = pytest.mark.gpu
@@ -100,10 +103,53 @@ def test_dense_deterministic_and_graph_replay():
     assert np.array_equal(bf16_to_bits(out), a)
 
 
-def test_prefill_full_size_sampled_tokens():
-    # 8 x 2048 tokens, d = 7168, E = 256, k = 8, f = 2048: every expert dense
+def _cover_every_tile(ids, E, tile=128, seed=0):
+    """Tokens such that every (expert, 128-row tile of its permuted rows) holds
+    at least one of their pairs: walk the tiles, and for a tile no chosen
+    token covers yet, take a random token of it."""
+    rng = np.random.default_rng(seed)
+    T, k = ids.shape
+    counts, offsets, perm, _ = O.permute(ids, E)
+    tile_of = np.empty(T * k, np.int64)              # pair -> global tile id
+    tid = 0
+    starts = []
+    for e in range(E):
+        for r0 in range(offsets[e], offsets[e + 1], tile):
+            r1 = min(r0 + tile, offsets[e + 1])
+            tile_of[perm[r0:r1]] = tid
+            starts.append((r0, r1))
+            tid += 1
+    covered = np.zeros(tid, bool)
+    chosen = []
+    for t_id, (r0, r1) in enumerate(starts):
+        if covered[t_id]:
+            continue
+        tok = int(perm[rng.integers(r0, r1)] // k)
+        chosen.append(tok)
+        covered[tile_of[tok * k:(tok + 1) * k]] = True
+    return sorted(chosen), tid
+
+
+def test_prefill_full_size_every_expert_tile():
+    # 8 x 2048 tokens, d = 7168, E = 256, k = 8, f = 2048: every expert dense.
+    # One row or more of every (expert, 128-token tile) is compared element by
+    # element, so every expert and every tile position of the persistent
+    # schedulers is covered; the oracle's per-expert work runs in a spawned
+    # process pool (started before any work in it touches the GPU).
+    import multiprocessing as mp
     cfg = W.CONFIGS["prefill"]
-    c = Case(cfg, token_subset=[0, 8191, 16383]).run_gpu().run_oracle()
-    assert np.all(c.o["counts"] >= 128)
-    c.check_all()
-    assert c.n_dense_rows == len(c._rows()) > 0
+    x, rw = W.gen_x_router(cfg)
+    ids, _, _ = O.route(O.router_logits(x, rw), cfg.k)
+    toks, ntiles = _cover_every_tile(ids, cfg.E)
+    workers = max(1, min(16, (os.cpu_count() or 2) - 1))
+    with mp.get_context("spawn").Pool(workers) as pool:
+        c = Case(cfg, token_subset=toks, x=x, rw=rw, oracle_experts=W.LazyExperts(cfg),
+                 map_fn=pool.map).run_gpu().run_oracle()
+        assert np.all(c.o["counts"] >= 128)
+        c.check_all()
+    rows = c._rows()
+    assert c.n_dense_rows == len(rows) > 0
+    # every (expert, tile) position holds a compared row
+    e_of = np.searchsorted(c.o["offsets"], rows[:, 1], side="right") - 1
+    seen = set(zip(e_of.tolist(), ((rows[:, 1] - c.o["offsets"][e_of]) // 128).tolist()))
+    assert len(seen) >= ntiles - c.n_excluded * cfg.k, (len(seen), ntiles)

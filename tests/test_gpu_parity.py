@@ -6,7 +6,7 @@ import torch
 from nvfp4_expert_layer_b200 import workloads as W
 from nvfp4_expert_layer_b200.layer import MoeFp4Layer, experts_to_device
 from oracle import moe_oracle as O
-from tests.parity import Case, to_dev_x, bf16_to_bits
+from tests.parity import Case, bf16_to_bits, oracle_pool, to_dev_x
 
 pytestmark = pytest.mark.gpu
 
@@ -52,12 +52,14 @@ def test_decode1_full_size():
 
 def test_decode64_full_size():
     cfg = W.CONFIGS["decode64"]
-    Case(cfg).run_gpu().run_oracle().check_all()
+    with oracle_pool() as pool:
+        Case(cfg, oracle_experts=W.LazyExperts(cfg), map_fn=pool.map).run_gpu().run_oracle().check_all()
 
 
-def test_verify_sampled_tokens():
+def test_verify_full_size_every_token():
     cfg = W.CONFIGS["verify"]
-    Case(cfg, token_subset=[0, 1, 2, 3, 61, 127]).run_gpu().run_oracle().check_all()
+    with oracle_pool() as pool:
+        Case(cfg, oracle_experts=W.LazyExperts(cfg), map_fn=pool.map).run_gpu().run_oracle().check_all()
 
 
 def test_deterministic_repeat():

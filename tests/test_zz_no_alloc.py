@@ -7,12 +7,14 @@ up front.  For them the library offers routing (router logits, top-k and the
 renormalised weights) that needs no handle and allocates nothing; its logits
 scratch is a fixed-size array the library defines in device memory.
 
-These tests call it through the C ABI twice in a row, with different inputs,
-and check each result against the same values reported by the allocating
-entry point, moe_fp4_forward_ex, within the tolerances of the parity tests:
-ids bit-exact (the inputs are checked for near ties first) and weights within
-1e-5 relative.  This file is collected last so that a run which stops at the
-first failure has run every other test already."""
+These tests call it through the C ABI, twice in a row with different inputs,
+and check each result against the oracle's routing of the same inputs (ids
+bit-exact, near ties excluded; weights within the tolerance the parity tests
+derive from the fp32 logit bound) and against the allocating entry point
+moe_fp4_forward_ex (ids bit-exact, weights within 1e-5 relative).  One case
+fills the scratch array exactly (T * E = 65536).  This file is collected last
+so that a run which stops at the first failure has run every other test
+already."""
 import ctypes
 
 import numpy as np
@@ -27,6 +29,7 @@ from oracle import moe_oracle as O
 pytestmark = pytest.mark.gpu
 
 W_RTOL = 1e-5
+U32 = 2.0 ** -24
 
 
 def _static_route(lib, x, rw, E, k):
@@ -42,19 +45,27 @@ def _static_route(lib, x, rw, E, k):
     return ids.cpu().numpy(), w.cpu().numpy()
 
 
-def _case(T, seed):
-    cfg = W.custom_config(T=T, d=512, E=64, k=4, f=256, seed=seed, router="unit")
-    x, rw = W.gen_x_router(cfg)
-    _, _, gap = O.route(O.router_logits(x, rw), cfg.k)
-    assert np.all(gap > 1e-4), "seeded inputs must have no near-tie tokens"
-    return cfg, x, rw
+def _check_against_oracle(x, rw, k, ids, w):
+    """ids bit-exact on tokens without a near tie; weights within
+    max(1e-5, 2 delta + 4 delta^2 + (k + 8) 2^-24) relative, delta bounded by
+    the fp32 logit bound of the token's selected experts."""
+    logits = O.router_logits(x, rw)
+    oids, ow, gap = O.route(logits, k)
+    keep = ~O.near_tie_flags(gap)
+    assert keep.sum() >= len(keep) - 2 - len(keep) // 100
+    assert np.array_equal(ids[keep], oids[keep])
+    bound = O.fp32_logit_error_bound(x, rw)
+    delta = np.take_along_axis(bound, oids, axis=1).max(axis=1)
+    tol = np.maximum(W_RTOL, 2 * delta + 4 * delta ** 2 + (k + 8) * U32)[:, None]
+    assert np.all((np.abs(w.astype(np.float64) - ow) <= tol * ow + 1e-7)[keep])
 
 
-def test_static_routing_matches_forward_ex_twice():
+def test_static_routing_matches_oracle_and_forward_ex_twice():
     lib = _lib.load()
     results = []
     for T, seed in ((37, 101), (200, 102)):
-        cfg, x, rw = _case(T, seed)
+        cfg = W.custom_config(T=T, d=512, E=64, k=4, f=256, seed=seed, router="unit")
+        x, rw = W.gen_x_router(cfg)
         layer = MoeFp4Layer(cfg.E, cfg.k, cfg.d, cfg.f)
         layer.load_experts(experts_to_device(W.gen_experts(cfg)))
         xd = torch.from_numpy(x.view(np.int16).copy()).cuda().view(torch.bfloat16)
@@ -62,11 +73,25 @@ def test_static_routing_matches_forward_ex_twice():
         _, dbg = layer.forward_ex(xd, rwd, want=("topk_ids", "topk_w"))
         ref_ids, ref_w = dbg["topk_ids"].cpu().numpy(), dbg["topk_w"].cpu().numpy()
         ids, w = _static_route(lib, xd, rwd, cfg.E, cfg.k)
+        _check_against_oracle(x, rw, cfg.k, ids, w)
         assert np.array_equal(ids, ref_ids)
         np.testing.assert_allclose(w, ref_w, rtol=W_RTOL, atol=1e-7)
         results.append(ids)
         layer.close()
     assert results[0].shape != results[1].shape
+
+
+def test_static_routing_fills_the_scratch_exactly():
+    # T * E = 65536 logits, the largest call the scratch array holds
+    lib = _lib.load()
+    cfg = W.custom_config(T=256, d=512, E=256, k=8, f=256, seed=103, router="unit")
+    x, rw = W.gen_x_router(cfg)
+    assert cfg.T * cfg.E == 65536
+    xd = torch.from_numpy(x.view(np.int16).copy()).cuda().view(torch.bfloat16)
+    rwd = torch.from_numpy(rw).cuda()
+    for _ in range(2):
+        ids, w = _static_route(lib, xd, rwd, cfg.E, cfg.k)
+        _check_against_oracle(x, rw, cfg.k, ids, w)
 
 
 def test_static_routing_rejects_oversized_calls():
