@@ -621,7 +621,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         for r in runs:
             cfg = r["cfg"]
-            secs, n, res, sample = cpu_baseline_sample(cfg, r["xs_np"], r["rw_np"])
+            secs, n, res, sample = cpu_baseline_sample(cfg, r["xs_np"][0], r["rw_np"])
             rec = records[cfg.name]
             rec["cpu_baseline"] = {"value": n / secs, "unit": "tokens/s", "cores": cpu_cores(),
                                    "kind": "oracle", "sample": sample}

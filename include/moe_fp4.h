@@ -285,6 +285,44 @@ MOE_FP4_API int moe_fp4_set_dense_threshold(moe_fp4_t* h, int thr);
  * finite (ignored when enable = 0).  Errors: MOE_FP4_ERR_INVALID_ARG. */
 MOE_FP4_API int moe_fp4_set_expert_norm(moe_fp4_t* h, int enable, float eps);
 
+/* Activation tensor scale of the dense class (NVFP4 activations).
+ *   dynamic = 0 (default): tensor scale 1.0, as at the top of this file; a
+ *       16-block whose amax is below about 6 * 2^-10 quantises to zeros.
+ *   dynamic = 1: every forward scales x and h by powers of two chosen from
+ *       the call's own data: gs = 2^e, e the smallest integer with
+ *       max|a| <= 6 * 448 * 2^e, max over the whole tensor (x: all T tokens;
+ *       h: every dense-class row); a is quantised as a * 2^-e with the rule at
+ *       the top of this file and the results are multiplied by gs.  h's
+ *       maximum is known only after every gate/up tile, so in this mode the
+ *       gate/up GEMM writes h in fp32 and a separate pass quantises it.
+ * "Mixture of Experts" topic page and the Muse Spark page (Fig. 1 caption):
+ * low-precision activations beside NVFP4 experts; the scale rule is this
+ * library's.  Errors: MOE_FP4_ERR_INVALID_ARG. */
+MOE_FP4_API int moe_fp4_set_act_scale(moe_fp4_t* h, int dynamic);
+
+/* Residual add: with enable = 1 every later forward of this handle returns
+ * out[t] = bf16_rn( x[t] + sum_j ... ), the MoE block's output added to its
+ * input in the combine's fp32 sum (one rounding), as a decoder layer adds its
+ * MoE output to the residual stream.  enable = 0 (default): the plain layer.
+ * Not applied by moe_fp4_forward_routed.  Errors: MOE_FP4_ERR_INVALID_ARG. */
+MOE_FP4_API int moe_fp4_set_residual(moe_fp4_t* h, int enable);
+
+/* A stack of L layers on one stream: x_0 = x, x_{l+1} = forward of
+ * layers[l] on x_l with router_w[l] (each handle's own options: threshold,
+ * norm, residual, activation scale), out = x_L.  While layer l streams its
+ * experts, its expert kernel prefetches layer l+1's router weights into L2,
+ * so the next routing starts from L2 ("Optimizing Muse Spark Open on TPU v7
+ * with SGLang-TorchTPU", sections 1-2: one program over all layers, the next
+ * layer's weights fetched while the current layer computes).  Layer l < L-1
+ * writes into its own handle's staging buffer, so consecutive entries must be
+ * different handles; all on the same device with the same d.  Every argument
+ * and workspace is checked before anything runs.  Asynchronous on `stream`;
+ * capturable into one CUDA graph once every handle has reserved T tokens.
+ * Errors: as moe_fp4_forward, and MOE_FP4_ERR_INVALID_ARG for L < 1, a null
+ * entry, equal consecutive handles, or x overlapping out. */
+MOE_FP4_API int moe_fp4_forward_layers(moe_fp4_t* const* layers, int L, const void* x_bf16, int T,
+                                       const float* const* router_w, void* out_bf16, cudaStream_t stream);
+
 /* Bound of every device-side wait of this handle's kernels, in milliseconds
  * (default 2000, or MOE_FP4_WAIT_TIMEOUT_MS at create time); ms >= 1.  A
  * wait that exceeds it records MOE_FP4_ERR_DEVICE_TIMEOUT in the device error

@@ -44,6 +44,9 @@ SIGNATURES = {
     "moe_fp4_forward_host": (_i, [_vp, _vp, _i, _vp, _vp, _vp]),
     "moe_fp4_set_dense_threshold": (_i, [_vp, _i]),
     "moe_fp4_set_expert_norm": (_i, [_vp, _i, ctypes.c_float]),
+    "moe_fp4_set_act_scale": (_i, [_vp, _i]),
+    "moe_fp4_set_residual": (_i, [_vp, _i]),
+    "moe_fp4_forward_layers": (_i, [ctypes.POINTER(_vp), _i, _vp, _i, ctypes.POINTER(_vp), _vp, _vp]),
     "moe_fp4_route": (_i, [_vp, _vp, _i, _vp, ctypes.POINTER(Routing), _vp]),
     "moe_fp4_gather_rows": (_i, [_vp, _i, _i, _vp, _i, _i, _vp, _vp]),
     "moe_fp4_forward_routed": (_i, [_vp, _vp, _i, _vp, _vp, _vp]),

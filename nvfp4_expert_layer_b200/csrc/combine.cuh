@@ -1,7 +1,8 @@
 // Combine and unpermute in a single pass over the per-pair partials.
 //
 // combine_kernel:       out[t] = bf16_rn( sum_j partial[inv[t,j]] ), slots
-//                       j = 0..k-1 summed in order in fp32.
+//                       j = 0..k-1 summed in order in fp32 (after x[t] when
+//                       the residual add is on).
 // combine_norm_kernel:  out[t] = bf16_rn( sum_j w[t,j] * y_j / sqrt(mean_i y_j[i]^2 + eps) ),
 //                       y_j = partial[inv[t,j]] the unweighted expert output
 //                       (the down epilogues skip the routing weight in this
@@ -33,13 +34,32 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float (&s)[8]) {
 
 // grid (min(T, cap), ceil(d / (8 * blockDim.x))); tokens t = blockIdx.x,
 // blockIdx.x + gridDim.x, ...; each thread owns 8 consecutive columns.
+// resid (optional, bf16 [T][d]): the sum starts from resid[t] (a residual add
+// in the same fp32 sum, one rounding).
+__device__ __forceinline__ void load_resid8(const uint16_t* resid, size_t off, float (&s)[8]) {
+  if (!resid) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s[i] = 0.f;
+    return;
+  }
+  const uint4 r = *reinterpret_cast<const uint4*>(resid + off);
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    s[2 * i] = __uint_as_float(w[i] << 16);
+    s[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
 __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ partial,
                                                       const int* __restrict__ inv, int T, int k,
-                                                      int d, uint16_t* __restrict__ out) {
+                                                      int d, const uint16_t* __restrict__ resid,
+                                                      uint16_t* __restrict__ out) {
   pdl_wait();
   const int col = (blockIdx.y * blockDim.x + threadIdx.x) * 8;
   for (int t = blockIdx.x; t < T && col < d; t += gridDim.x) {
-    float s[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    float s[8];
+    load_resid8(resid, (size_t)t * d + col, s);
     // slots in groups of 8: all index loads, then all row loads, then the sums
     for (int j0 = 0; j0 < k; j0 += 8) {
       int pos[8];
@@ -76,7 +96,7 @@ constexpr int kNormMaxK = 32;
 // division), out = sum_j y_j * scale_j in slot order.  wts is [T][k].
 __global__ void __launch_bounds__(kNormThreads) combine_norm_kernel(
     const float* __restrict__ partial, const int* __restrict__ inv, const float* __restrict__ wts, int T,
-    int k, int d, float eps, uint16_t* __restrict__ out) {
+    int k, int d, float eps, const uint16_t* __restrict__ resid, uint16_t* __restrict__ out) {
   __shared__ float red[kNormThreads / 32][kNormMaxK];
   __shared__ float scale[kNormMaxK];
   pdl_wait();
@@ -115,7 +135,8 @@ __global__ void __launch_bounds__(kNormThreads) combine_norm_kernel(
     }
     __syncthreads();
     for (int col = threadIdx.x * 8; col < d; col += kNormThreads * 8) {
-      float s[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      float s[8];
+      load_resid8(resid, (size_t)t * d + col, s);
       for (int j = 0; j < k; ++j) {
         const float* src = partial + (size_t)inv[(size_t)t * k + j] * d + col;
         const float4 a = *reinterpret_cast<const float4*>(src);

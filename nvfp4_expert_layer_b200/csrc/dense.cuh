@@ -82,11 +82,31 @@ struct DenseParams {
   uint8_t* hq;           // [P_pad][f/2]
   uint8_t* hsf;          // scales of hq (sf_rowpair_offset layout, K = f)
   float* h32;            // [P][f] or null
+  // dynamic activation tensor scales (null: tensor scale 1):
+  const int* x_amax;     // bits of max|x| of the call: gate/up results times gs_x
+  int* h_amax;           // gate/up: write fp32 h to h32 and max|h| here, no NVFP4 h
+  const int* h_amax_in;  // down: results times gs_h
   // down output
   float* partial;        // [P][d]
   int* err;
   int64_t wait_timeout_ns;
 };
+
+// ---------------------------------------------------------------------------
+// Dynamic activation tensor scale (optional): gs = 2^e, e the smallest
+// integer with amax <= 6 * 448 * 2^e, so the block scales of the largest
+// block reach the top of the e4m3 range.  Found with exact comparisons
+// (2688 * 2^e is exact in fp32): amax < 2^E (frexp) gives e = E - 12 when
+// amax <= 2688 * 2^(E - 12) = 0.65625 * 2^E, else E - 11.  amax = 0 gives 0.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int pow2_tensor_exp(float amax) {
+  if (!(amax > 0.f)) return 0;
+  int E;
+  frexpf(amax, &E);
+  const int e = E - 12;
+  return max(-100, min(100, amax <= ldexpf(2688.f, e) ? e : e + 1));
+}
+__device__ __forceinline__ float exp2i_f(int e) { return __int_as_float((e + 127) << 23); }
 
 // ---------------------------------------------------------------------------
 // Activation quantiser of the dense class, in two passes.
@@ -111,11 +131,14 @@ __device__ __forceinline__ int dense_rank_of_padrow(const int4* dense, int nd, i
 
 __global__ void __launch_bounds__(256) quant_tok_kernel(const uint16_t* __restrict__ x, int T, int d,
                                                         const int* __restrict__ n_dense,
+                                                        const int* __restrict__ x_amax,
                                                         uint8_t* __restrict__ xq, uint8_t* __restrict__ xsf) {
   pdl_wait();
   if (*n_dense == 0) { pdl_launch_dependents(); return; }
   const int lane = threadIdx.x & 31;
   const int nblk = d / 16;
+  // dynamic tensor scale gs = 2^e: the values are quantised as v * 2^-e (exact)
+  const float inv_gs = x_amax ? exp2i_f(-pow2_tensor_exp(__int_as_float(*x_amax))) : 1.f;
   for (int t = blockIdx.x * 8 + (threadIdx.x >> 5); t < T; t += gridDim.x * 8) {
     const uint16_t* src = x + (size_t)t * d;
     for (int blk = lane; blk < nblk; blk += 32) {
@@ -125,8 +148,8 @@ __global__ void __launch_bounds__(256) quant_tok_kernel(const uint16_t* __restri
       float v[16];
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
-        v[2 * q] = __uint_as_float(wv[q] << 16);
-        v[2 * q + 1] = __uint_as_float(wv[q] & 0xffff0000u);
+        v[2 * q] = __uint_as_float(wv[q] << 16) * inv_gs;
+        v[2 * q + 1] = __uint_as_float(wv[q] & 0xffff0000u) * inv_gs;
       }
       float amax = 0.f;
 #pragma unroll
@@ -195,6 +218,77 @@ __global__ void __launch_bounds__(256) gather_x_dense_kernel(
       uint8_t* unit = xsf + ((size_t)tile * npairs + pr) * kSfUnitBytes;
       reinterpret_cast<uint4*>(unit)[q] = v;
     }
+  }
+  pdl_launch_dependents();
+}
+
+// max |x| of a bf16 tensor into *amax (int bits of a non-negative float;
+// atomicMax is order independent, so the result is deterministic)
+__global__ void __launch_bounds__(256) amax_bf16_kernel(const uint16_t* __restrict__ x, long long n,
+                                                        const int* __restrict__ n_dense, int* __restrict__ amax) {
+  pdl_wait();
+  if (*n_dense == 0) { pdl_launch_dependents(); return; }
+  float m = 0.f;
+  for (long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * 8; i < n;
+       i += (long long)gridDim.x * blockDim.x * 8) {
+    const uint4 v = *reinterpret_cast<const uint4*>(x + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      m = fmaxf(m, fmaxf(fabsf(__uint_as_float(w[q] << 16)), fabsf(__uint_as_float(w[q] & 0xffff0000u))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0 && m > 0.f) atomicMax(amax, __float_as_int(m));
+  pdl_launch_dependents();
+}
+
+// Dynamic h scale: the NVFP4 h of every padded dense row from the fp32 h the
+// gate/up GEMM wrote (permutation rows), quantised as h * 2^-e_h with the R4
+// rule; rows past an expert's count up to its next multiple of 128 are zeros.
+// One warp per (padded row, 8 blocks of 16): codes and sf_rowpair_offset scales.
+__global__ void __launch_bounds__(256) quant_h_dense_kernel(const float* __restrict__ h32, const int4* __restrict__ dense,
+                                                            const int* __restrict__ n_dense,
+                                                            const int* __restrict__ pad_total,
+                                                            const int* __restrict__ h_amax, int f,
+                                                            uint8_t* __restrict__ hq, uint8_t* __restrict__ hsf) {
+  pdl_wait();
+  const int nd = *n_dense;
+  if (nd == 0) { pdl_launch_dependents(); return; }
+  const float inv_gs = exp2i_f(-pow2_tensor_exp(__int_as_float(*h_amax)));
+  const int rows = *pad_total, nb = f / 16;
+  const long long units = (long long)rows * nb;
+  for (long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x; u < units;
+       u += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(u / nb), kb = (int)(u - (long long)r * nb);
+    const int4 de = dense[dense_rank_of_padrow(dense, nd, r)];
+    const int i = r - de.w;
+    if (i >= ((de.z + 127) & ~127)) continue;      // beyond the last 128-row tile: never read
+    uint32_t sfbyte = 0u;
+    uint2 codes = make_uint2(0, 0);
+    if (i < de.z) {
+      const float4* src = reinterpret_cast<const float4*>(h32 + (size_t)(de.y + i) * f + kb * 16);
+      float v[16];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 a = src[q];
+        v[4 * q] = a.x * inv_gs; v[4 * q + 1] = a.y * inv_gs; v[4 * q + 2] = a.z * inv_gs; v[4 * q + 3] = a.w * inv_gs;
+      }
+      float am = 0.f;
+#pragma unroll
+      for (int q = 0; q < 16; ++q) am = fmaxf(am, fabsf(v[q]));
+      sfbyte = f32x2_to_e4m3x2(0.f, am / 6.0f) & 0xffu;
+      const float sf = e4m3_to_f32(sfbyte);
+      if (sf > 0.f) {
+        uint32_t c[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) c[q] = f32x2_to_e2m1x2(v[2 * q + 1] / sf, v[2 * q] / sf);
+        codes.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
+        codes.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
+      }
+    }
+    *reinterpret_cast<uint2*>(hq + (size_t)r * (f / 2) + kb * 8) = codes;
+    hsf[sf_rowpair_offset(r, kb, f / 64)] = (uint8_t)sfbyte;
   }
   pdl_launch_dependents();
 }
@@ -411,7 +505,8 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
         const int drow = tl.wt * 128 + q * 32 + lane;
         const int nrows = min(kDenseN, tl.de.z - tl.tt * kDenseN) - hf * 128;
         const int prow0 = tl.de.y + tl.tt * kDenseN + hf * 128;      // permutation row of column 0
-        const float gsd = p.gs[2 * p.E + e];
+        const float gsd = p.gs[2 * p.E + e] *
+                          (p.h_amax_in ? exp2i_f(pow2_tensor_exp(__int_as_float(*p.h_amax_in))) : 1.f);
 #pragma unroll
         for (int c32 = 0; c32 < 4; ++c32) {
           if (32 * c32 >= nrows) break;                              // warp-uniform
@@ -432,7 +527,9 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
         const bool valid = tl.tt * 128 + tok < tl.de.z;
         const int prow = tl.de.y + tl.tt * 128 + tok;    // permutation row
         const int hrow = tl.de.w + tl.tt * 128 + tok;    // padded row
-        const float gsg = p.gs[e], gsu = p.gs[p.E + e];
+        const float gsx = p.x_amax ? exp2i_f(pow2_tensor_exp(__int_as_float(*p.x_amax))) : 1.f;
+        const float gsg = p.gs[e] * gsx, gsu = p.gs[p.E + e] * gsx;
+        float hmax = 0.f;
         const int chb = tl.wt * (kDenseN / 2) + hf * 64;
         uint32_t codes[8];
         uint32_t sfw = 0u;
@@ -452,6 +549,10 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
 #pragma unroll
             for (int i = 0; i < 4; ++i) dst[i] = make_float4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
           }
+          if (p.h_amax) {                 // dynamic h scale: quantised by quant_h_dense_kernel
+            if (valid) hmax = fmaxf(hmax, am);
+            continue;
+          }
           const uint32_t sfbyte = f32x2_to_e4m3x2(0.f, am / 6.0f) & 0xffu;
           const float sf = e4m3_to_f32(sfbyte);
           uint32_t w0 = 0u, w1 = 0u;                    // channel i -> nibble i % 8 of word i / 8
@@ -465,6 +566,12 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
           codes[2 * bl] = w0;
           codes[2 * bl + 1] = w1;
           sfw |= sfbyte << (8 * bl);
+        }
+        if (p.h_amax) {
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) hmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, o));
+          if (lane == 0 && hmax > 0.f) atomicMax(p.h_amax, __float_as_int(hmax));
+          continue;
         }
         // padding rows (accumulators of zero activations) are written too: zeros
         uint4* dst = reinterpret_cast<uint4*>(p.hq + (size_t)hrow * (p.f / 2) + (chb >> 1));

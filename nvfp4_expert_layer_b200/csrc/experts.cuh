@@ -71,6 +71,8 @@ struct ExpertParams {
   int* err;
   int64_t wait_timeout_ns;
   int wait_extra;             // test hook: added to every down tile's completion target (0)
+  const uint8_t* l2_next;     // bytes to prefetch into L2 (the next layer's router weights) or null
+  long long l2_next_bytes;    // a multiple of 16
 };
 
 __device__ __forceinline__ int ld_acquire(const int* p) {
@@ -183,8 +185,16 @@ struct BPair {
   uint4 lo, hi;
 };
 
-template <int NT, bool COHERENT>
-__device__ __forceinline__ void load_bchunk(const __half* const (&brow)[2], int chunk, int c, BPair (&b)[NT]) {
+// Units of a work tile: RT row tiles x NT n-tiles (two for NT = 1, 2; four for NT = 4).
+template <int NT>
+struct TileShape {
+  static constexpr int RT = NT == 1 ? 2 : 1;       // 16-row tiles per work tile
+  static constexpr int U = RT * NT;                // (row tile, n-tile) units, one per epilogue warp
+  static constexpr int NR = NT < 2 ? 2 : NT;       // B row pointers held per lane
+};
+
+template <int NT, int NR, bool COHERENT>
+__device__ __forceinline__ void load_bchunk(const __half* const (&brow)[NR], int chunk, int c, BPair (&b)[NT]) {
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     if (brow[nt] == nullptr) {
@@ -207,8 +217,8 @@ __device__ __forceinline__ void load_bchunk(const __half* const (&brow)[2], int 
 // other set, so a full stage ends with the next stage's first chunk in `be`
 // and nothing is copied.  The codes and scales of the next (chunk, row tile)
 // unit are loaded before the current one is converted.
-template <int NT, int RT, bool COHERENT, bool FULL>
-__device__ __forceinline__ void mma_stage_jit(uint32_t st, int nch, int lane, int g, const __half* const (&brow)[2],
+template <int NT, int RT, int NR, bool COHERENT, bool FULL>
+__device__ __forceinline__ void mma_stage_jit(uint32_t st, int nch, int lane, int g, const __half* const (&brow)[NR],
                                               int chunk0, int c, bool more, int nrows, BPair (&be)[NT],
                                               float (&acc)[RT][kAccK][NT][4]) {
   constexpr int NU = kExpSC * RT;
@@ -225,8 +235,8 @@ __device__ __forceinline__ void mma_stage_jit(uint32_t st, int nch, int lane, in
     if (rt == 0) {
       const bool pf = FULL ? (ch + 1 < kExpSC || more) : (ch + 1 < nch || more);
       if (pf) {
-        if (ch & 1) load_bchunk<NT, COHERENT>(brow, chunk0 + ch + 1, c, be);
-        else load_bchunk<NT, COHERENT>(brow, chunk0 + ch + 1, c, bo);
+        if (ch & 1) load_bchunk<NT, NR, COHERENT>(brow, chunk0 + ch + 1, c, be);
+        else load_bchunk<NT, NR, COHERENT>(brow, chunk0 + ch + 1, c, bo);
       }
     }
     const BPair (&bb)[NT] = (ch & 1) ? bo : be;
@@ -262,23 +272,35 @@ __device__ __forceinline__ void mma_stage_jit(uint32_t st, int nch, int lane, in
 }
 
 // NT = 8-wide n-tiles per job: expert_kernel<1> runs jobs of <= 8 rows,
-// expert_kernel<2> jobs of 9..16 rows; each has its own job list and counters.
-// With one n-tile a work tile is two 16-row tiles (RT = 2) that share the
-// activation fragments, the loop control and the epilogue barrier.
+// expert_kernel<2> jobs of 9..16 rows, expert_kernel<4> jobs of 17..32 rows;
+// each has its own job list and counters.  With one n-tile a work tile is
+// two 16-row tiles (RT = 2) that share the activation fragments, the loop
+// control and the epilogue barrier.  A job's weights are streamed once per
+// job, so the 32-row jobs stream an expert with up to 32 rows once.
 template <int NT>
-__global__ void __launch_bounds__(kExpThreads, 4) expert_kernel(ExpertParams p) {
-  constexpr int RT = NT == 1 ? 2 : 1;
+__global__ void __launch_bounds__(kExpThreads, NT == 4 ? 3 : 4) expert_kernel(ExpertParams p) {
+  constexpr int RT = TileShape<NT>::RT;
+  constexpr int U = TileShape<NT>::U;
+  constexpr int NR = TileShape<NT>::NR;
   constexpr int RING = kExpRing / RT;          // stages in flight per warp (same bytes)
   constexpr int SLOT = RT * kExpSB;
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* bars_all = reinterpret_cast<uint64_t*>(smem + kExpWarps * RING * SLOT);
-  float* red_all = reinterpret_cast<float*>(bars_all + kExpWarps * RING);   // [2][4][2][32][4]
+  float* red_all = reinterpret_cast<float*>(bars_all + kExpWarps * RING);   // [2][4 warps][U][32][4]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
   const int G = (int)gridDim.x, b = (int)blockIdx.x;
 
   pdl_wait();                                   // routing results of the previous kernel
+  // the next layer's router weights go to L2 while this layer streams its
+  // experts: each block asks for its slice (a hint; nothing waits on it)
+  if (p.l2_next && threadIdx.x == 0) {
+    const long long per = ((p.l2_next_bytes / G + 15) / 16) * 16;
+    const long long lo = per * b;
+    for (long long o = lo; o < lo + per && o < p.l2_next_bytes; o += 32768)
+      bulk_prefetch_l2(p.l2_next + o, (uint32_t)min(32768LL, min(lo + per, p.l2_next_bytes) - o));
+  }
   const int njobs = *p.njobs;
   const int ngu = njobs * (p.tpe_gu / RT);
   const int ntot = ngu + njobs * (p.tpe_dn / RT);
@@ -341,9 +363,9 @@ __global__ void __launch_bounds__(kExpThreads, 4) expert_kernel(ExpertParams p) 
   int consumed = 0;
 
   // B rows of this lane (row n = nt*8 + g of the job), resolved one tile ahead
-  auto tile_rows = [&](const TileInfo& t, const __half* (&row)[2]) {
+  auto tile_rows = [&](const TileInfo& t, const __half* (&row)[NR]) {
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
+    for (int nt = 0; nt < NR; ++nt) {
       const int n = nt * 8 + g;
       row[nt] = nullptr;
       if (n < t.nrows) {
@@ -353,7 +375,7 @@ __global__ void __launch_bounds__(kExpThreads, 4) expert_kernel(ExpertParams p) 
     }
   };
   TileInfo ti_next{};
-  const __half* row_next[2] = {nullptr, nullptr};
+  const __half* row_next[NR] = {};
   if (my_tiles > 0) {
     ti_next = tile_info<RT>(p, jobs, b, ngu, warp);
     tile_rows(ti_next, row_next);
@@ -362,7 +384,9 @@ __global__ void __launch_bounds__(kExpThreads, 4) expert_kernel(ExpertParams p) 
   for (int it = 0; it < my_tiles; ++it) {
     const TileInfo ti = ti_next;
     const int nt_used = (ti.nrows + 7) >> 3;
-    const __half* row[2] = {row_next[0], row_next[1]};
+    const __half* row[NR];
+#pragma unroll
+    for (int i = 0; i < NR; ++i) row[i] = row_next[i];
     if (it + 1 < my_tiles) {
       ti_next = tile_info<RT>(p, jobs, b + (it + 1) * G, ngu, warp);
       tile_rows(ti_next, row_next);
@@ -384,7 +408,7 @@ __global__ void __launch_bounds__(kExpThreads, 4) expert_kernel(ExpertParams p) 
       }
     }
 
-    float part[2][4];                    // this warp's partial sums, per unit u = rt * NT + nt
+    float part[U][4];                    // this warp's partial sums, per unit u = rt * NT + nt
     {
       float acc[RT][kAccK][NT][4];
 #pragma unroll
@@ -397,8 +421,8 @@ __global__ void __launch_bounds__(kExpThreads, 4) expert_kernel(ExpertParams p) 
             for (int q = 0; q < 4; ++q) acc[rt][a][nt][q] = 0.f;
       BPair be[NT];
       if (ti.nw > 0) {
-        if (ti.down) load_bchunk<NT, true>(row, kExpSC * ti.slo, c, be);
-        else load_bchunk<NT, false>(row, kExpSC * ti.slo, c, be);
+        if (ti.down) load_bchunk<NT, NR, true>(row, kExpSC * ti.slo, c, be);
+        else load_bchunk<NT, NR, false>(row, kExpSC * ti.slo, c, be);
       }
       for (int ss = 0; ss < ti.nw; ++ss) {
         const int s = ti.slo + ss;
@@ -413,20 +437,20 @@ __global__ void __launch_bounds__(kExpThreads, 4) expert_kernel(ExpertParams p) 
           const uint32_t sp = ring_s + slot * SLOT;
           const int k0 = kExpSC * s, nr = ti.nrows;
           if (nch == kExpSC) {
-            if (ti.down) mma_stage_jit<NT, RT, true, true>(sp, nch, lane, g, row, k0, c, more, nr, be, acc);
-            else mma_stage_jit<NT, RT, false, true>(sp, nch, lane, g, row, k0, c, more, nr, be, acc);
+            if (ti.down) mma_stage_jit<NT, RT, NR, true, true>(sp, nch, lane, g, row, k0, c, more, nr, be, acc);
+            else mma_stage_jit<NT, RT, NR, false, true>(sp, nch, lane, g, row, k0, c, more, nr, be, acc);
           } else {
-            if (ti.down) mma_stage_jit<NT, RT, true, false>(sp, nch, lane, g, row, k0, c, more, nr, be, acc);
-            else mma_stage_jit<NT, RT, false, false>(sp, nch, lane, g, row, k0, c, more, nr, be, acc);
+            if (ti.down) mma_stage_jit<NT, RT, NR, true, false>(sp, nch, lane, g, row, k0, c, more, nr, be, acc);
+            else mma_stage_jit<NT, RT, NR, false, false>(sp, nch, lane, g, row, k0, c, more, nr, be, acc);
           }
         }
         __syncwarp();
         ++consumed;
         if (lane == 0 && !failed) produce(consumed);
       }
-      // units: NT == 1 -> (row tile u, n-tile 0); NT == 2 -> (row tile 0, n-tile u)
+      // units: NT == 1 -> (row tile u, n-tile 0); NT >= 2 -> (row tile 0, n-tile u)
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
+      for (int u = 0; u < U; ++u) {
         const int rt = NT == 1 ? u : 0, nt = NT == 1 ? 0 : u;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -439,12 +463,12 @@ __global__ void __launch_bounds__(kExpThreads, 4) expert_kernel(ExpertParams p) 
     }
 
     // ---- cross-warp reduction of the tile (buffer alternates by tile parity)
-    float* red = red_all + (it & 1) * (kExpWarps * 2 * 32 * 4);
+    float* red = red_all + (it & 1) * (kExpWarps * U * 32 * 4);
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int u = 0; u < U; ++u)
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        red[((warp * 2 + nt) * 32 + lane) * 4 + q] = part[nt][q];
+        red[((warp * U + u) * 32 + lane) * 4 + q] = part[u][q];
     __syncthreads();
     const int units_used = RT * nt_used;
     if (warp < units_used) {
@@ -456,7 +480,7 @@ __global__ void __launch_bounds__(kExpThreads, 4) expert_kernel(ExpertParams p) 
       for (int q = 0; q < 4; ++q) {
         float sum = 0.f;
 #pragma unroll
-        for (int w = 0; w < kExpWarps; ++w) sum += red[((w * 2 + red_u) * 32 + lane) * 4 + q];
+        for (int w = 0; w < kExpWarps; ++w) sum += red[((w * U + red_u) * 32 + lane) * 4 + q];
         v[q] = sum;
       }
       if (!ti.down) {
@@ -520,9 +544,10 @@ __global__ void __launch_bounds__(kExpThreads, 4) expert_kernel(ExpertParams p) 
   pdl_launch_dependents();
 }
 
+template <int NT>
 constexpr size_t expert_smem_size() {
   return (size_t)kExpWarps * kExpRing * kExpSB + (size_t)kExpWarps * kExpRing * 8 +
-         (size_t)2 * kExpWarps * 2 * 32 * 4 * 4;
+         (size_t)2 * kExpWarps * TileShape<NT>::U * 32 * 4 * 4;
 }
 
 }  // namespace moe

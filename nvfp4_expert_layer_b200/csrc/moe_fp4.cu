@@ -32,7 +32,9 @@
 namespace {
 
 constexpr int kSmallT = 256;          // fused routing kernel up to this many tokens
-constexpr size_t kExpSmem = moe::expert_smem_size();
+constexpr size_t kExpSmem1 = moe::expert_smem_size<1>();
+constexpr size_t kExpSmem2 = moe::expert_smem_size<2>();
+constexpr size_t kExpSmem4 = moe::expert_smem_size<4>();
 constexpr int kDenseGridPerSm = 1;
 constexpr int kStageEvents = 9;
 constexpr int kPermMaxBlocks = 296;       // blocks of the large-batch permutation
@@ -52,13 +54,16 @@ struct Workspace {
   int* n_jobs1 = nullptr;
   int4* jobs2 = nullptr;
   int* n_jobs2 = nullptr;
-  int* counters = nullptr;     // gu_done [max jobs] | exit | ticket
+  int4* jobs4 = nullptr;
+  int* n_jobs4 = nullptr;
+  int* counters = nullptr;     // gu_done of the three job lists | exits | ticket
   size_t counter_bytes = 0;
   int4* dense_list = nullptr;
   int* n_dense = nullptr;
   int* dense_ntoff = nullptr;    // [2][E+1]: 128-row and 256-row tile prefixes
   int* perm_bcnt = nullptr;      // [kPermMaxBlocks][E] per-block expert counts / bases
   int* dense_pad_total = nullptr;
+  int* act_amax = nullptr;       // [2] max|x|, max|h| bits (dynamic activation scales)
   uint8_t* xq_tok = nullptr;     // dense class: NVFP4 x per token [T][d/2] and scales [T][d/16]
   uint8_t* xsf_tok = nullptr;
   uint8_t* xq = nullptr;         // dense class: NVFP4 activations [pad_rows][d/2]
@@ -86,7 +91,7 @@ struct moe_fp4 {
   int E = 0, k = 0, d = 0, f = 0;
   int thr = 128;
   int sm_count = 0;
-  int exp_bps1 = 1, exp_bps2 = 1; // resident blocks per SM of the expert kernels
+  int exp_bps1 = 1, exp_bps2 = 1, exp_bps4 = 1;  // resident blocks per SM of the expert kernels
   int64_t wait_timeout_ns = 2000000000LL;
   bool loaded = false;
   uint8_t* gu_frag = nullptr;     // gate/up fragment layout, all experts
@@ -95,6 +100,10 @@ struct moe_fp4 {
   float* l1 = nullptr;            // [2][E]: largest gate / up row L1 norm (expert_l1_kernel)
   int* hexp = nullptr;            // [E]: light-class h staging exponent bound (expert_hexp_kernel)
   bool expert_norm = false;       // RMS-normalise each expert's output before the weighted sum
+  bool act_dynamic = false;       // dense class: power-of-two activation tensor scales per call
+  bool residual = false;          // out = bf16(x + MoE(x)), the add fused in the combine
+  const uint8_t* l2_next = nullptr;   // (set by moe_fp4_forward_layers) prefetched during the experts
+  long long l2_next_bytes = 0;
   float norm_eps = 1e-6f;
   int wait_extra = 0;             // test hook: unreachable down-tile completion target
   uint8_t* dq_gu = nullptr;       // dense class: gate/up codes, rows interleaved by 16, signs folded [E*2f][d/2]
@@ -141,11 +150,13 @@ T* carve(uint8_t*& cur, size_t count) {
   return p;
 }
 
-// completion counters: gu_done of list 1 [E] | gu_done of list 2 [E + P/16 + 1] |
-// exit 1 | exit 2 | routing ticket
-size_t counter_ints(const moe_fp4* h, int Tm) {
-  return (size_t)h->E + ((size_t)h->E + (size_t)Tm * h->k / moe::kJobRows + 1) + 3;
-}
+// Largest job list of 17..32-row jobs: every light expert's full 32-row
+// jobs plus one remainder each.
+size_t max_jobs4(const moe_fp4* h, int Tm) { return (size_t)h->E + (size_t)Tm * h->k / moe::kJobRows + 1; }
+
+// completion counters: gu_done of list 1 [E] | of list 2 [E] | of list 4
+// [max_jobs4] | exit 1 | exit 2 | exit 4 | routing ticket
+size_t counter_ints(const moe_fp4* h, int Tm) { return (size_t)2 * h->E + max_jobs4(h, Tm) + 4; }
 
 // rows of the dense-class operand buffers: every pair plus up to 127 padding
 // rows per dense expert, in whole 128-row tiles
@@ -208,12 +219,15 @@ size_t workspace_bytes(const moe_fp4* h, int Tm) {
   add(P * 4);                       // inv
   add((size_t)h->E * 16);                              // light jobs, <= 8 rows
   add(4);
-  add(((size_t)h->E + P / moe::kJobRows + 1) * 16);   // light jobs, 9..16 rows
+  add((size_t)h->E * 16);                              // light jobs, 9..16 rows
+  add(4);
+  add(max_jobs4(h, Tm) * 16);                          // light jobs, 17..32 rows
   add(4);
   add(counter_ints(h, Tm) * 4);                        // counters
   add(((size_t)h->E + 1) * 8);                         // dense 128- and 256-row tile prefixes
   add((size_t)kPermMaxBlocks * h->E * 4);              // permutation block counts
   add(4);                                              // dense padded rows
+  add(8);                                              // activation amax slots
   const size_t pr = dense_pad_rows(h, Tm);
   add((size_t)Tm * h->d / 2);                          // xq_tok
   add((size_t)Tm * h->d / 16);                         // xsf_tok
@@ -264,8 +278,10 @@ int ensure_workspace(moe_fp4* h, int Tm, cudaStream_t stream) {
   w.inv = carve<int>(cur, P);
   w.jobs1 = carve<int4>(cur, h->E);
   w.n_jobs1 = carve<int>(cur, 1);
-  w.jobs2 = carve<int4>(cur, (size_t)h->E + P / moe::kJobRows + 1);
+  w.jobs2 = carve<int4>(cur, h->E);
   w.n_jobs2 = carve<int>(cur, 1);
+  w.jobs4 = carve<int4>(cur, max_jobs4(h, Tm));
+  w.n_jobs4 = carve<int>(cur, 1);
   w.counter_bytes = counter_ints(h, Tm) * 4;
   w.counters = carve<int>(cur, w.counter_bytes / 4);
   w.dense_list = carve<int4>(cur, h->E);
@@ -280,6 +296,7 @@ int ensure_workspace(moe_fp4* h, int Tm, cudaStream_t stream) {
   w.dense_ntoff = carve<int>(cur, 2 * (h->E + 1));
   w.perm_bcnt = carve<int>(cur, (size_t)kPermMaxBlocks * h->E);
   w.dense_pad_total = carve<int>(cur, 1);
+  w.act_amax = carve<int>(cur, 2);
   w.pad_rows = dense_pad_rows(h, Tm);
   w.xq_tok = carve<uint8_t>(cur, (size_t)Tm * h->d / 2);
   w.xsf_tok = carve<uint8_t>(cur, (size_t)Tm * h->d / 16);
@@ -361,14 +378,15 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
   const uint16_t* xb = static_cast<const uint16_t*>(x);
   const bool pdl = !h->stage_timing;
   MOE_CUDA(mark(h, 0, st));
-  const size_t max_jobs2 = (size_t)E + (size_t)w.max_T * k / moe::kJobRows + 1;   // counter layout
-  int* gu_done1 = w.counters;
+  int* gu_done1 = w.counters;                  // counter layout of counter_ints
   int* gu_done2 = gu_done1 + E;
-  int* exit1 = gu_done2 + max_jobs2;
+  int* gu_done4 = gu_done2 + E;
+  int* exit1 = gu_done4 + max_jobs4(h, w.max_T);
   int* exit2 = exit1 + 1;
-  int* ticket = exit2 + 1;
+  int* exit4 = exit2 + 1;
+  int* ticket = exit4 + 1;
   moe::PermuteOut po{w.counts, w.offsets, w.perm, w.inv, w.jobs1, w.n_jobs1, w.jobs2, w.n_jobs2,
-                     w.dense_list, w.n_dense, w.dense_ntoff, w.dense_pad_total, h->err};
+                     w.jobs4, w.n_jobs4, w.dense_list, w.n_dense, w.dense_ntoff, w.dense_pad_total, h->err};
   // Without the dense class (shape or tensor-map support missing) every
   // expert runs in the light class.  An expert holds at most T rows (one per
   // token), so below T = thr no expert can be dense and its kernels are skipped.
@@ -449,8 +467,16 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
   const float* wts_epi = (h->expert_norm || mode.pre_ids) ? nullptr : w.wts;
   // 4-5 (dense class). NVFP4 activations, then the two tensor-core GEMMs
   if (run_dense) {
+    const bool dyn = h->act_dynamic;
+    if (dyn) {       // max|x| of the call for the x tensor scale
+      MOE_CUDA(cudaMemsetAsync(w.act_amax, 0, 2 * sizeof(int), st));
+      MOE_CUDA(launch(moe::amax_bf16_kernel, dim3(std::min<long long>(((long long)T * d / 8 + 255) / 256,
+                                                                     8 * h->sm_count)),
+                      dim3(256), 0, st, false, xb, (long long)T * d, (const int*)w.n_dense, w.act_amax));
+    }
     MOE_CUDA(launch(moe::quant_tok_kernel, dim3(std::min((T + 7) / 8, 8 * h->sm_count)), dim3(256), 0, st,
-                    pdl, xb, T, d, (const int*)w.n_dense, w.xq_tok, w.xsf_tok));
+                    pdl && !dyn, xb, T, d, (const int*)w.n_dense, dyn ? (const int*)w.act_amax : nullptr,
+                    w.xq_tok, w.xsf_tok));
     MOE_CUDA(launch(moe::gather_x_dense_kernel, dim3(8 * h->sm_count), dim3(256), 0, st, pdl,
                     (const uint8_t*)w.xq_tok, (const uint8_t*)w.xsf_tok, (const int4*)w.dense_list,
                     (const int*)w.n_dense, (const int*)w.dense_pad_total, (const int*)w.perm, k, d, w.xq, w.xsf));
@@ -476,14 +502,23 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
     dp.wts = wts_epi;
     dp.hq = w.hq;
     dp.hsf = w.hsf;
-    dp.h32 = h->dense_h32 ? w.h32 : nullptr;
+    dp.h32 = (h->dense_h32 || dyn) ? w.h32 : nullptr;
+    dp.x_amax = dyn ? w.act_amax : nullptr;
+    dp.h_amax = dyn ? w.act_amax + 1 : nullptr;
     dp.partial = w.partial;
     dp.err = h->err;
     dp.wait_timeout_ns = h->wait_timeout_ns;
     MOE_CUDA(launch(moe::dense_gemm_kernel<moe::kDenseGateUp>, dim3(h->sm_count * kDenseGridPerSm),
                     dim3(moe::kDenseThreads), moe::dense_smem_size<moe::kDenseGateUp>(E), st, pdl, dp));
     MOE_CUDA(mark(h, 5, st));
+    if (dyn)         // NVFP4 h with the h tensor scale, once every gate/up tile is done
+      MOE_CUDA(launch(moe::quant_h_dense_kernel, dim3(8 * h->sm_count), dim3(256), 0, st, pdl,
+                      (const float*)w.h32, (const int4*)w.dense_list, (const int*)w.n_dense,
+                      (const int*)w.dense_pad_total, (const int*)(w.act_amax + 1), f, w.hq, w.hsf));
     moe::DenseParams dp2 = dp;
+    dp2.x_amax = nullptr;
+    dp2.h_amax = nullptr;
+    dp2.h_amax_in = dyn ? w.act_amax + 1 : nullptr;
     dp2.tmA = h->tm_down;       // weights: 128-row M tiles
     dp2.tmB = w.tm_h;           // tokens: 256-row N tiles
     dp2.sfA = h->dsf_dn;
@@ -523,19 +558,27 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
   ep.hexp = h->hexp;
   ep.wts = wts_epi;
   ep.wait_extra = h->wait_extra;
+  ep.l2_next = h->l2_next;
+  ep.l2_next_bytes = h->l2_next_bytes;
   ep.partial = w.partial;
   ep.err = h->err;
   ep.wait_timeout_ns = h->wait_timeout_ns;
-  moe::ExpertParams ep1 = ep, ep2 = ep;
+  moe::ExpertParams ep1 = ep, ep2 = ep, ep4 = ep;
   ep1.jobs = w.jobs1; ep1.njobs = w.n_jobs1; ep1.gu_done = gu_done1; ep1.exit_cnt = exit1;
   ep2.jobs = w.jobs2; ep2.njobs = w.n_jobs2; ep2.gu_done = gu_done2; ep2.exit_cnt = exit2;
+  ep4.jobs = w.jobs4; ep4.njobs = w.n_jobs4; ep4.gu_done = gu_done4; ep4.exit_cnt = exit4;
+  ep2.l2_next = ep4.l2_next = nullptr;      // the first light kernel issues the prefetch
   if (light_ok) {
     MOE_CUDA(launch(moe::expert_kernel<1>, dim3(h->sm_count * h->exp_bps1), dim3(moe::kExpThreads),
-                    kExpSmem, st, pdl, ep1));
-    // jobs of 9..16 rows need an expert with at least 9 rows, i.e. T >= 9
+                    kExpSmem1, st, pdl, ep1));
+    // jobs of 9..16 (17..32) rows need an expert with at least 9 (17) rows,
+    // i.e. T >= 9 (T >= 17)
     if (T >= 9)
       MOE_CUDA(launch(moe::expert_kernel<2>, dim3(h->sm_count * h->exp_bps2), dim3(moe::kExpThreads),
-                      kExpSmem, st, pdl, ep2));
+                      kExpSmem2, st, pdl, ep2));
+    if (T >= 17)
+      MOE_CUDA(launch(moe::expert_kernel<4>, dim3(h->sm_count * h->exp_bps4), dim3(moe::kExpThreads),
+                      kExpSmem4, st, pdl, ep4));
   }
   MOE_CUDA(mark(h, 7, st));
   // 7. combine / unpermute: out[t] = bf16(sum_j partial[inv[t,j]]), or with
@@ -547,10 +590,11 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
   else if (h->expert_norm)
     MOE_CUDA(launch(moe::combine_norm_kernel, dim3(std::min(T, 8 * h->sm_count)), dim3(moe::kNormThreads), 0,
                     st, pdl, (const float*)w.partial, (const int*)w.inv, (const float*)w.wts, T, k, d,
-                    h->norm_eps, static_cast<uint16_t*>(out)));
+                    h->norm_eps, h->residual ? xb : nullptr, static_cast<uint16_t*>(out)));
   else
     MOE_CUDA(launch(moe::combine_kernel, dim3(std::min(T, 65535), (d + 1023) / 1024), dim3(128), 0, st, pdl,
-                    (const float*)w.partial, (const int*)w.inv, T, k, d, static_cast<uint16_t*>(out)));
+                    (const float*)w.partial, (const int*)w.inv, T, k, d, h->residual ? xb : nullptr,
+                    static_cast<uint16_t*>(out)));
   MOE_CUDA(mark(h, 8, st));
   return MOE_FP4_OK;
 }
@@ -615,11 +659,21 @@ int moe_fp4_create(int E, int top_k, int d, int f, moe_fp4_t** out) {
     if (cudaDeviceGetAttribute(&h->sm_count, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess) {
       rc = MOE_FP4_ERR_CUDA; break;
     }
+    // The dynamic shared-memory limit is an attribute of the kernel, shared by
+    // every handle in the process: only ever raise it, so a handle created
+    // later with a smaller shape cannot lower what an earlier one launches.
     auto smem_attr = [](const void* fn, size_t bytes) {
+      static std::mutex mu;
+      std::lock_guard<std::mutex> lock(mu);
+      cudaFuncAttributes fa{};
+      cudaError_t e = cudaFuncGetAttributes(&fa, fn);
+      if (e != cudaSuccess) return e;
+      if ((size_t)fa.maxDynamicSharedSizeBytes >= bytes) return cudaSuccess;
       return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     };
-    if (smem_attr((const void*)moe::expert_kernel<1>, kExpSmem) != cudaSuccess ||
-        smem_attr((const void*)moe::expert_kernel<2>, kExpSmem) != cudaSuccess ||
+    if (smem_attr((const void*)moe::expert_kernel<1>, kExpSmem1) != cudaSuccess ||
+        smem_attr((const void*)moe::expert_kernel<2>, kExpSmem2) != cudaSuccess ||
+        smem_attr((const void*)moe::expert_kernel<4>, kExpSmem4) != cudaSuccess ||
         smem_attr((const void*)moe::perm_scan_kernel, permute_smem_bytes(E)) != cudaSuccess ||
         smem_attr((const void*)moe::perm_place_kernel, (size_t)32 * E * 4) != cudaSuccess ||
         smem_attr((const void*)moe::route_kernel<1>, route_smem_max(E, d, top_k)) != cudaSuccess ||
@@ -631,15 +685,18 @@ int moe_fp4_create(int E, int top_k, int d, int f, moe_fp4_t** out) {
         smem_attr((const void*)moe::router_tc_kernel, moe::router_tc_smem_size()) != cudaSuccess) {
       rc = MOE_FP4_ERR_CUDA; break;
     }
-    int nb1 = 0, nb2 = 0;
+    int nb1 = 0, nb2 = 0, nb4 = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb1, moe::expert_kernel<1>, moe::kExpThreads,
-                                                      kExpSmem) != cudaSuccess ||
+                                                      kExpSmem1) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb2, moe::expert_kernel<2>, moe::kExpThreads,
-                                                      kExpSmem) != cudaSuccess) {
+                                                      kExpSmem2) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb4, moe::expert_kernel<4>, moe::kExpThreads,
+                                                      kExpSmem4) != cudaSuccess) {
       rc = MOE_FP4_ERR_CUDA; break;
     }
     h->exp_bps1 = std::max(1, nb1);
     h->exp_bps2 = std::max(1, nb2);
+    h->exp_bps4 = std::max(1, nb4);
     if (cudaMalloc(&h->err, sizeof(int)) != cudaSuccess) { rc = MOE_FP4_ERR_OOM; break; }
     if (cudaMemset(h->err, 0, sizeof(int)) != cudaSuccess) { rc = MOE_FP4_ERR_CUDA; break; }
     if (cudaMalloc(&h->gs, sizeof(float) * 3 * E) != cudaSuccess) { rc = MOE_FP4_ERR_OOM; break; }
@@ -705,18 +762,15 @@ int moe_fp4_load_experts(moe_fp4_t* h, const moe_fp4_experts* w) {
     if (!alloc(&h->gu_frag, gu_bytes) || !alloc(&h->dn_frag, dn_bytes)) return MOE_FP4_ERR_OOM;
     h->weight_bytes += gu_bytes + dn_bytes;
   }
-  if (h->want_light) {
-    const long long thr = (long long)E * (f / 8) * (d / moe::kChunkK) * 32;
-    const int blocks = (int)std::min<long long>((thr + 255) / 256, 65535LL * 16);
-    moe::repack_fragment_kernel<moe::kGateUp><<<blocks, 256>>>(w->gate_q, w->gate_sf, w->up_q, w->up_sf,
-                                                              E, f, d, h->gu_frag);
-    MOE_CUDA(cudaGetLastError());
-  }
-  {
-    const long long thr = (long long)E * (d / 16) * (f / moe::kChunkK) * 32;
-    const int blocks = (int)std::min<long long>((thr + 255) / 256, 65535LL * 16);
-    moe::repack_fragment_kernel<moe::kDown><<<blocks, 256>>>(w->down_q, w->down_sf, nullptr, nullptr,
-                                                            E, d, f, h->dn_frag);
+  if (h->want_light) {       // both fragment copies exist only when the light class is kept
+    const long long thr_gu = (long long)E * (f / 8) * (d / moe::kChunkK) * 32;
+    const int blocks_gu = (int)std::min<long long>((thr_gu + 255) / 256, 65535LL * 16);
+    moe::repack_fragment_kernel<moe::kGateUp><<<blocks_gu, 256>>>(w->gate_q, w->gate_sf, w->up_q, w->up_sf,
+                                                                 E, f, d, h->gu_frag);
+    const long long thr_dn = (long long)E * (d / 16) * (f / moe::kChunkK) * 32;
+    const int blocks_dn = (int)std::min<long long>((thr_dn + 255) / 256, 65535LL * 16);
+    moe::repack_fragment_kernel<moe::kDown><<<blocks_dn, 256>>>(w->down_q, w->down_sf, nullptr, nullptr,
+                                                               E, d, f, h->dn_frag);
     MOE_CUDA(cudaGetLastError());
   }
   // dense class: codes with block-scale signs folded, scale atoms, tensor maps
@@ -787,6 +841,53 @@ int moe_fp4_set_expert_norm(moe_fp4_t* h, int enable, float eps) {
   if (enable && h->k > moe::kNormMaxK) return MOE_FP4_ERR_UNSUPPORTED;
   h->expert_norm = enable != 0;
   if (enable) h->norm_eps = eps;
+  return MOE_FP4_OK;
+}
+
+int moe_fp4_set_residual(moe_fp4_t* h, int enable) {
+  if (!h || (enable != 0 && enable != 1)) return MOE_FP4_ERR_INVALID_ARG;
+  h->residual = enable != 0;
+  return MOE_FP4_OK;
+}
+
+int moe_fp4_forward_layers(moe_fp4_t* const* layers, int L, const void* x, int T, const float* const* router_w,
+                           void* out, cudaStream_t stream) {
+  if (!layers || L < 1 || !router_w || T < 0) return MOE_FP4_ERR_INVALID_ARG;
+  for (int l = 0; l < L; ++l) {
+    if (!layers[l] || !router_w[l]) return MOE_FP4_ERR_INVALID_ARG;
+    if (l > 0 && (layers[l] == layers[l - 1] || layers[l]->d != layers[0]->d ||
+                  layers[l]->device != layers[0]->device))
+      return MOE_FP4_ERR_INVALID_ARG;
+  }
+  if (T == 0) return MOE_FP4_OK;
+  // every check and every workspace first, so nothing runs unless all layers can
+  // (x against out for every layer: pointers, alignment, no overlap, loaded)
+  for (int l = 0; l < L; ++l) {
+    int rc = check_forward_args(layers[l], x, T, router_w[l], out);
+    if (rc != MOE_FP4_OK) return rc;
+    if ((rc = ensure_workspace(layers[l], T, stream)) != MOE_FP4_OK) return rc;
+  }
+  // layer l reads layer l-1's output from that handle's staging buffer
+  const void* in = x;
+  for (int l = 0; l < L; ++l) {
+    moe_fp4* h = layers[l];
+    void* dst = l == L - 1 ? out : h->ws.xout;
+    if (l + 1 < L) {
+      h->l2_next = reinterpret_cast<const uint8_t*>(router_w[l + 1]);
+      h->l2_next_bytes = (long long)layers[l + 1]->E * layers[l + 1]->d * 4;
+    }
+    const int rc = run_forward(h, in, T, router_w[l], dst, stream);
+    h->l2_next = nullptr;
+    h->l2_next_bytes = 0;
+    if (rc != MOE_FP4_OK) return rc;
+    in = dst;
+  }
+  return MOE_FP4_OK;
+}
+
+int moe_fp4_set_act_scale(moe_fp4_t* h, int dynamic) {
+  if (!h || (dynamic != 0 && dynamic != 1)) return MOE_FP4_ERR_INVALID_ARG;
+  h->act_dynamic = dynamic != 0;
   return MOE_FP4_OK;
 }
 

@@ -18,7 +18,7 @@
 
 namespace moe {
 
-constexpr int kJobRows = 16;   // rows per light job (two 8-wide MMA n-tiles)
+constexpr int kJobRows = 32;   // rows per light job (up to four 8-wide MMA n-tiles)
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);
@@ -251,9 +251,10 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 // Permutation: pairs p = t*k + j in [0, P) are placed in (expert, pair) order
 // -- deterministic and stable -- and the active experts are classed by row
 // count n:
-//   light (n < thr): cut into jobs of 16 rows plus one remainder job; jobs of
+//   light (n < thr): cut into jobs of 32 rows plus one remainder job; jobs of
 //     <= 8 rows go to list 1 (one 8-wide MMA n-tile), jobs of 9..16 rows to
-//     list 2 (two n-tiles); each list is ordered heavy expert first;
+//     list 2 (two n-tiles), jobs of 17..32 rows to list 4 (four n-tiles);
+//     each list is ordered heavy expert first;
 //   dense (n >= thr): listed by n descending.
 // At most 32 pairs: perm_small inside the routing kernel; otherwise three
 // launches (perm_hist_kernel, perm_scan_kernel, perm_place_kernel).
@@ -267,8 +268,10 @@ struct PermuteOut {
   int* inv;          // [P]
   int4* jobs1;       // [E]            {expert, row0, nrows, 0}, 1 <= nrows <= 8
   int* n_jobs1;
-  int4* jobs2;       // [E + P/16 + 1] {expert, row0, nrows, 0}, 9 <= nrows <= 16
+  int4* jobs2;       // [E]            {expert, row0, nrows, 0}, 9 <= nrows <= 16
   int* n_jobs2;
+  int4* jobs4;       // [E + P/32 + 1] {expert, row0, nrows, 0}, 17 <= nrows <= 32
+  int* n_jobs4;
   int4* dense_list;  // [E]            {expert, row0, nrows, padded row0}
   int* n_dense;
   int* dense_ntoff;  // [2][E+1]       exclusive prefixes of ceil(nrows / 128) and ceil(nrows / 256)
@@ -293,7 +296,7 @@ __device__ void perm_classes(int E, int thr, int dense_supported, const PermuteO
     const int e = act[a];
     const int n = cnt[e];
     const bool light = n < thr;
-    int rank = 0, s1 = 0, s2 = 0, pad0 = 0, nt0 = 0, nt1 = 0;
+    int rank = 0, s1 = 0, s2 = 0, s4 = 0, pad0 = 0, nt0 = 0, nt1 = 0;
     for (int b = 0; b < A; ++b) {
       const int e2 = act[b], n2 = cnt[e2];
       if ((n2 < thr) != light) continue;
@@ -301,7 +304,8 @@ __device__ void perm_classes(int E, int thr, int dense_supported, const PermuteO
         ++rank;
         const int r2 = n2 % kJobRows;
         s1 += (r2 > 0 && r2 <= 8) ? 1 : 0;
-        s2 += n2 / kJobRows + (r2 > 8 ? 1 : 0);
+        s2 += (r2 > 8 && r2 <= 16) ? 1 : 0;
+        s4 += n2 / kJobRows + (r2 > 16 ? 1 : 0);
         pad0 += (n2 + 255) & ~255;
         nt0 += (n2 + 127) >> 7;
         nt1 += (n2 + 255) >> 8;
@@ -311,11 +315,12 @@ __device__ void perm_classes(int E, int thr, int dense_supported, const PermuteO
       for (int r0 = 0; r0 < n; r0 += kJobRows) {
         const int nr = min(kJobRows, n - r0);
         const int4 jb = make_int4(e, off[e] + r0, nr, 0);
-        if (nr <= 8) o.jobs1[s1] = jb; else o.jobs2[s2++] = jb;
+        if (nr <= 8) o.jobs1[s1] = jb; else if (nr <= 16) o.jobs2[s2] = jb; else o.jobs4[s4++] = jb;
       }
       const int r = n % kJobRows;
       atomicAdd(&misc[1], (r > 0 && r <= 8) ? 1 : 0);
-      atomicAdd(&misc[2], n / kJobRows + (r > 8 ? 1 : 0));
+      atomicAdd(&misc[2], (r > 8 && r <= 16) ? 1 : 0);
+      atomicAdd(&misc[7], n / kJobRows + (r > 16 ? 1 : 0));
     } else {
       o.dense_list[rank] = make_int4(e, off[e], n, pad0);
       o.dense_ntoff[rank] = nt0;
@@ -330,6 +335,7 @@ __device__ void perm_classes(int E, int thr, int dense_supported, const PermuteO
   if (threadIdx.x == 0) {
     *o.n_jobs1 = misc[1];
     *o.n_jobs2 = misc[2];
+    *o.n_jobs4 = misc[7];
     *o.n_dense = misc[3];
     o.dense_ntoff[misc[3]] = misc[4];
     o.dense_ntoff[E + 1 + misc[3]] = misc[6];
@@ -517,39 +523,41 @@ __device__ void perm_small(const int* ids, int E, int thr, int dense_supported, 
   const bool dense = act && ((sk >> 21) & 1u);
   const int ae = (int)((sk >> 5) & 1023u), an = act ? 63 - (int)((sk >> 15) & 63u) : 0;
   const int aoff = (int)(sk & 31u);
-  // 4. exclusive scans over the class order: list-1 jobs, list-2 jobs, 128- and
-  // 256-row tiles (one byte each; at most 64 per byte), padded rows / 256
-  const int r = an % kJobRows;
-  const uint32_t c1 = (act && !dense && r > 0 && r <= 8) ? 1u : 0u;
-  const uint32_t c2 = (act && !dense) ? (uint32_t)(an / kJobRows + (r > 8 ? 1 : 0)) : 0u;
+  // 4. exclusive scans over the class order: list-1, list-2 and list-4 jobs
+  // (10 bits each), 128- and 256-row tiles (one byte each; at most 64 per
+  // byte), padded rows / 256.  At most 32 pairs: an expert has at most 32
+  // rows, so one job.
+  const uint32_t c1 = (act && !dense && an <= 8) ? 1u : 0u;
+  const uint32_t c2 = (act && !dense && an > 8 && an <= 16) ? 1u : 0u;
+  const uint32_t c4 = (act && !dense && an > 16) ? 1u : 0u;
   const uint32_t t0 = dense ? (uint32_t)((an + 127) >> 7) : 0u;
   const uint32_t t1 = dense ? (uint32_t)((an + 255) >> 8) : 0u;
-  const uint32_t packed = c1 | (c2 << 8) | (t0 << 16) | (t1 << 24);
-  const uint32_t inc = warp_scan_u32(packed, lane);
-  const uint32_t exc = inc - packed;
-  const uint32_t tot = __shfl_sync(FULL, inc, 31);
+  const uint32_t packed = t0 | (t1 << 8);
+  const uint32_t jpacked = c1 | (c2 << 10) | (c4 << 20);
+  const uint32_t inc = warp_scan_u32(packed, lane), jinc = warp_scan_u32(jpacked, lane);
+  const uint32_t exc = inc - packed, jexc = jinc - jpacked;
+  const uint32_t tot = __shfl_sync(FULL, inc, 31), jtot = __shfl_sync(FULL, jinc, 31);
   const int nlight = __popc(__ballot_sync(FULL, act && !dense));
   if (act && !dense) {
-    int s1 = (int)(exc & 0xffu), s2 = (int)((exc >> 8) & 0xffu);
-    for (int r0 = 0; r0 < an; r0 += kJobRows) {
-      const int nr = min(kJobRows, an - r0);
-      const int4 jb = make_int4(ae, aoff + r0, nr, 0);
-      if (nr <= 8) o.jobs1[s1] = jb; else o.jobs2[s2++] = jb;
-    }
+    const int4 jb = make_int4(ae, aoff, an, 0);
+    if (an <= 8) o.jobs1[jexc & 0x3ffu] = jb;
+    else if (an <= 16) o.jobs2[(jexc >> 10) & 0x3ffu] = jb;
+    else o.jobs4[(jexc >> 20) & 0x3ffu] = jb;
   } else if (dense) {
     const int crank = lane - nlight;
-    o.dense_list[crank] = make_int4(ae, aoff, an, (int)((exc >> 24) & 0xffu) * 256);
-    o.dense_ntoff[crank] = (int)((exc >> 16) & 0xffu);
-    o.dense_ntoff[E + 1 + crank] = (int)((exc >> 24) & 0xffu);
+    o.dense_list[crank] = make_int4(ae, aoff, an, (int)((exc >> 8) & 0xffu) * 256);
+    o.dense_ntoff[crank] = (int)(exc & 0xffu);
+    o.dense_ntoff[E + 1 + crank] = (int)((exc >> 8) & 0xffu);
   }
   const int n_dense = __popc(__ballot_sync(FULL, dense));
   if (lane == 0) {
-    *o.n_jobs1 = (int)(tot & 0xffu);
-    *o.n_jobs2 = (int)((tot >> 8) & 0xffu);
+    *o.n_jobs1 = (int)(jtot & 0x3ffu);
+    *o.n_jobs2 = (int)((jtot >> 10) & 0x3ffu);
+    *o.n_jobs4 = (int)((jtot >> 20) & 0x3ffu);
     *o.n_dense = n_dense;
-    o.dense_ntoff[n_dense] = (int)((tot >> 16) & 0xffu);
-    o.dense_ntoff[E + 1 + n_dense] = (int)((tot >> 24) & 0xffu);
-    *o.dense_pad_total = (int)((tot >> 24) & 0xffu) * 256;
+    o.dense_ntoff[n_dense] = (int)(tot & 0xffu);
+    o.dense_ntoff[E + 1 + n_dense] = (int)((tot >> 8) & 0xffu);
+    *o.dense_pad_total = (int)((tot >> 8) & 0xffu) * 256;
     if (n_dense > 0 && !dense_supported) set_error(o.err, kErrUnsupported);
   }
 }

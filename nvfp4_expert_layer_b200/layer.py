@@ -67,6 +67,14 @@ class MoeFp4Layer:
         _lib.check(self.lib.moe_fp4_set_expert_norm(self._h, 1 if enable else 0, eps),
                    "moe_fp4_set_expert_norm")
 
+    def set_act_scale(self, dynamic: bool) -> None:
+        """Dense class: power-of-two activation tensor scales per call (see moe_fp4.h)."""
+        _lib.check(self.lib.moe_fp4_set_act_scale(self._h, 1 if dynamic else 0), "moe_fp4_set_act_scale")
+
+    def set_residual(self, enable: bool) -> None:
+        """out = bf16(x + MoE(x)) (see moe_fp4.h)."""
+        _lib.check(self.lib.moe_fp4_set_residual(self._h, 1 if enable else 0), "moe_fp4_set_residual")
+
     def set_wait_timeout_ms(self, ms: int) -> None:
         _lib.check(self.lib.moe_fp4_set_wait_timeout_ms(self._h, ms), "moe_fp4_set_wait_timeout_ms")
 
@@ -164,4 +172,19 @@ def experts_to_device(ex, device="cuda") -> dict:
     for n in EXPERT_FIELDS:
         a = getattr(ex, n)
         out[n] = torch.from_numpy(a).to(device)
+    return out
+
+
+def forward_layers(layers, x: torch.Tensor, router_ws, out=None, stream=None) -> torch.Tensor:
+    """A stack of MoeFp4Layer handles applied in order on one stream (see
+    moe_fp4_forward_layers): x_{l+1} = layers[l](x_l, router_ws[l])."""
+    lib = _lib.load()
+    L = len(layers)
+    if out is None:
+        out = torch.empty_like(x)
+    hs = (ctypes.c_void_p * L)(*[l._h.value for l in layers])
+    rws = (ctypes.c_void_p * L)(*[r.data_ptr() for r in router_ws])
+    T = x.shape[0] if x.dim() == 2 else 0
+    _lib.check(lib.moe_fp4_forward_layers(hs, L, _ptr(x), T, rws, _ptr(out), _stream_ptr(stream)),
+               "moe_fp4_forward_layers")
     return out

@@ -43,6 +43,12 @@ Readings where the pages are silent (each is stated where it is used):
      (token, slot) pairs by (expert, token, slot).
   R6 a token whose k-th and (k+1)-th fp64 logits differ by less than 1e-6 is a
      near-tie and is excluded from id / output comparisons.
+  R13 the optional dynamic activation tensor scale of the dense class: a
+     power of two, gs = 2^e with e the smallest integer such that
+     max|a| <= 6 * 448 * 2^e over the whole tensor of the call; a is quantised
+     as a / gs by R4's rule and dequantised times gs.
+  R14 the optional residual add: the block's input x joins the same fp64 sum
+     as the expert outputs, out = bf16(x + sum_j w_j y_j), one rounding.
   R12 the optional per-expert output normalisation ([P2-S8]) is an RMS norm
      over the d outputs of each expert, y / sqrt(mean(y^2) + eps), with no
      learned gain and eps chosen by the caller (the pages give neither).
@@ -160,6 +166,23 @@ def quantize_act_nvfp4(v: np.ndarray):
     return (codes.reshape(v32.shape), sf, deq.reshape(v32.shape))
 
 
+def pow2_tensor_scale(amax: float) -> float:
+    """Dynamic activation tensor scale (reading R13): 2^e for the smallest
+    integer e with amax <= 6 * 448 * 2^e, so the largest 16-block's scale lands
+    at the top of the e4m3 range; 1.0 when amax is 0.  Exact: amax <= 2^E
+    for E = frexp exponent, and 2688 * 2^e is exact in binary floating point."""
+    amax = float(amax)
+    if not amax > 0:
+        return 1.0
+    _, E = np.frexp(amax)                       # amax = m 2^E, 0.5 <= m < 1
+    e = int(E) - 12
+    while amax > 2688.0 * 2.0 ** e:             # at most two steps
+        e += 1
+    while e > -1074 and amax <= 2688.0 * 2.0 ** (e - 1):
+        e -= 1
+    return 2.0 ** e
+
+
 # ----------------------------------------------------------------------------
 # bf16
 # ----------------------------------------------------------------------------
@@ -264,22 +287,24 @@ def silu(z: np.ndarray) -> np.ndarray:
 
 
 def expert_ffn(xrows: np.ndarray, Wg: np.ndarray, Wu: np.ndarray, Wd: np.ndarray,
-               quantized: bool, magnitudes: bool = False):
+               quantized: bool, magnitudes: bool = False, scales=(1.0, 1.0)):
     """One expert on its rows.  Returns (h, y) in float64.
 
     quantized=False (R4, n_e < thr): h = SiLU(Wg x) * (Wu x); y = Wd h.
     quantized=True  (R4, n_e >= thr): x and h pass through quantize_act_nvfp4
     first; h is rounded to float32 before its quantiser (the kernel holds h
-    in float32).
+    in float32).  scales = (gs_x, gs_h): the activation tensor scales (R13;
+    1.0 by default): a is quantised as a / gs and dequantised times gs.
     magnitudes=True also returns the absolute-value sums that bound rounding
     errors element by element (|Wg||x|, |Wu||x|, |Wd||h|, and g, u), and per
     row the largest row L1 norms of the expert's matrices (l1g, l1u, l1d:
     max_c sum_k |W[c,k]|) and max |x| of the row (xmax)."""
-    xin = quantize_act_nvfp4(xrows)[2] if quantized else xrows
+    gx, gh = scales
+    xin = quantize_act_nvfp4(xrows / gx)[2] * gx if quantized else xrows
     g = xin @ Wg.T
     u = xin @ Wu.T
     h = silu(g) * u
-    hin = quantize_act_nvfp4(h.astype(np.float32))[2] if quantized else h
+    hin = quantize_act_nvfp4(h.astype(np.float32) / np.float32(gh))[2] * gh if quantized else h
     y = hin @ Wd.T
     if not magnitudes:
         return h, y
@@ -331,19 +356,30 @@ class PairRows:
 
 def _expert_rows(task):
     """One expert on its selected rows (dequantise, then expert_ffn).
-    task = (experts, e, xrows, quantized, magnitudes); a top-level function so
-    that a process pool can run it."""
-    experts, e, xrows, quantized, magnitudes = task
+    task = (experts, e, xrows, quantized, magnitudes, scales); a top-level
+    function so that a process pool can run it."""
+    experts, e, xrows, quantized, magnitudes, scales = task
     mats = experts.expert(e)
     Wg = dequant_nvfp4(*mats[0])
     Wu = dequant_nvfp4(*mats[1])
     Wd = dequant_nvfp4(*mats[2])
-    return expert_ffn(xrows, Wg, Wu, Wd, quantized=quantized, magnitudes=magnitudes)
+    return expert_ffn(xrows, Wg, Wu, Wd, quantized=quantized, magnitudes=magnitudes, scales=scales)
+
+
+def _expert_h_amax(task):
+    """max |fp32(h)| of one dense-class expert over all its rows (R13's first
+    pass).  task = (experts, e, xrows, gs_x)."""
+    experts, e, xrows, gx = task
+    mats = experts.expert(e)
+    xin = quantize_act_nvfp4(xrows / gx)[2] * gx
+    h = silu(xin @ dequant_nvfp4(*mats[0]).T) * (xin @ dequant_nvfp4(*mats[1]).T)
+    return float(np.max(np.abs(h.astype(np.float32)))) if h.size else 0.0
 
 
 def forward(x_bits: np.ndarray, router_w: np.ndarray, experts, E: int, k: int,
             thr: int = 128, token_subset=None, want_pairs: bool = True,
-            magnitudes: bool = False, expert_norm_eps=None, map_fn=map):
+            magnitudes: bool = False, expert_norm_eps=None, map_fn=map, act_scale: str = "fixed",
+            residual: bool = False):
     """The whole layer.  `experts.expert(e)` -> {0: (q,sf,gs) gate, 1: up, 2: down}.
 
     token_subset: if given, expert outputs are evaluated only for pairs of those
@@ -353,6 +389,13 @@ def forward(x_bits: np.ndarray, router_w: np.ndarray, experts, E: int, k: int,
     map_fn: how the independent per-expert evaluations are mapped (the builtin
     map, or a process pool's map; results are assembled in expert order
     either way, so the output does not depend on it).
+    residual: the block's input is added to its output before the one bf16
+    rounding (R14: out = bf16(x + sum_j w_j y_j), a decoder layer's residual
+    stream; rows outside token_subset then hold x).
+    act_scale: "fixed" (R4: activation tensor scale 1.0) or "dynamic" (R13:
+    gs_x from max|x| over all T tokens, gs_h from max|h| over every pair of
+    every dense-class expert, each pow2_tensor_scale; h is evaluated for all
+    dense pairs first, whatever token_subset is).
     Returns a dict with logits, ids, w, gap, counts, offsets, perm, inv, the
     per-pair h, y (the expert output Wd h) and partial (its contribution to
     the output; PairRows indexed by permutation row, NaN where not
@@ -380,7 +423,17 @@ def forward(x_bits: np.ndarray, router_w: np.ndarray, experts, E: int, k: int,
             continue
         # R4: the expert's class follows its full row count in the call
         work.append((e, pos[keep], pairs[keep], toks[keep], (hi - lo) >= thr))
-    results = list(map_fn(_expert_rows, [(experts, e, x[toks], q, magnitudes)
+    gs_x = gs_h = 1.0
+    h_amax = None
+    if act_scale == "dynamic":
+        gs_x = pow2_tensor_scale(np.max(np.abs(x)) if x.size else 0.0)
+        dense_all = [(experts, e, x[perm[offsets[e]:offsets[e + 1]] // k], gs_x) for e in range(E)
+                     if offsets[e + 1] - offsets[e] >= thr and offsets[e + 1] > offsets[e]]
+        h_amax = max(list(map_fn(_expert_h_amax, dense_all)) + [0.0])
+        gs_h = pow2_tensor_scale(h_amax)
+    elif act_scale != "fixed":
+        raise ValueError(act_scale)
+    results = list(map_fn(_expert_rows, [(experts, e, x[toks], q, magnitudes, (gs_x, gs_h))
                                          for e, _, _, toks, q in work]))
     h_all = partial_all = y_all = None
     out64 = np.zeros((T, d), dtype=np.float64)
@@ -402,7 +455,9 @@ def forward(x_bits: np.ndarray, router_w: np.ndarray, experts, E: int, k: int,
             y_all._put(pos, y)
             partial_all._put(pos, contrib)
         np.add.at(out64, toks, contrib)
+    if residual:
+        out64 = out64 + x
     out_bits = f64_to_bf16_bits_rne(out64)
     return dict(logits=logits, ids=ids, w=w, gap=gap, counts=counts, offsets=offsets,
                 perm=perm, inv=inv, h=h_all, y=y_all, partial=partial_all, out64=out64,
-                out_bits=out_bits, tokens=tokens, mags=mags)
+                out_bits=out_bits, tokens=tokens, mags=mags, gs_x=gs_x, gs_h=gs_h, h_amax=h_amax)

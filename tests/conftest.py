@@ -7,9 +7,6 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-# Parity summaries of the cases checked in this session (tests.parity.Case.check_all
-# appends one per case); printed at the end of the run.
-PARITY_REPORT = []
 
 
 def pytest_configure(config):
@@ -18,6 +15,9 @@ def pytest_configure(config):
 
 
 def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    # the parity summaries tests.parity.Case.check_all collected in this session
+    mod = sys.modules.get("tests.parity")
+    PARITY_REPORT = getattr(mod, "PARITY_REPORT", None)
     if not PARITY_REPORT:
         return
     tr = terminalreporter

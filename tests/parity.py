@@ -23,6 +23,8 @@ Parity contract, applied per compared token:
   - h element-wise within the propagated fp32 accumulation bound
     (d+2) 2^-24 (|Wg||x|, |Wu||x|) through SiLU(g)*u, times 2 for second
     order terms;
+  - every partial additionally within (w_rtol |w| + 2^-149) |Wd||h|: the
+    layer's fp32 routing weight carries the weight tolerance above;
   - light-class partial element-wise within |w| (2^-10 |Wd||h| + 2 L1d hfl):
     h enters the down projection as fp16 after a power-of-two scale 2^e_h
     (relative rounding 2^-11, doubled for the fp32 accumulation and the
@@ -62,6 +64,8 @@ from oracle import moe_oracle as O
 from tests._oracle_tasks import abs_wd_times
 
 OUT_TOL = 1e-2
+# one summary per checked case of this session (printed by tests/conftest.py)
+PARITY_REPORT = []
 W_RTOL = 1e-5
 U32 = 2.0 ** -24
 
@@ -152,7 +156,8 @@ class Case:
     """Inputs, the CUDA layer's results and the oracle's for one config."""
 
     def __init__(self, cfg, thr=128, layer=None, experts=None, token_subset=None, x=None, rw=None,
-                 norm_eps=None, oracle_experts=None, map_fn=map, oracle_thr=None):
+                 norm_eps=None, oracle_experts=None, map_fn=map, oracle_thr=None, act_dynamic=False,
+                 residual=False):
         self.cfg = cfg
         self.thr = thr
         # the class threshold the oracle applies (by default the layer's)
@@ -167,6 +172,8 @@ class Case:
         self.token_subset = token_subset
         self.norm_eps = norm_eps
         self.map_fn = map_fn
+        self.act_dynamic = act_dynamic
+        self.residual = residual
 
     def run_gpu(self):
         if self.layer is None:
@@ -174,6 +181,8 @@ class Case:
             self.layer.load_experts(experts_to_device(self.experts))
         self.layer.set_dense_threshold(self.thr)
         self.layer.set_expert_norm(self.norm_eps is not None, 0.0 if self.norm_eps is None else self.norm_eps)
+        self.layer.set_act_scale(self.act_dynamic)
+        self.layer.set_residual(self.residual)
         xd = to_dev_x(self.x)
         rwd = torch.from_numpy(self.rw).cuda()
         out, dbg = self.layer.forward_ex(xd, rwd)
@@ -190,7 +199,13 @@ class Case:
             thr = self.oracle_thr
         self.o = O.forward(self.x, self.rw, self.oracle_experts, self.cfg.E, self.cfg.k, thr=thr,
                            token_subset=self.token_subset, magnitudes=True,
-                           expert_norm_eps=self.norm_eps, map_fn=self.map_fn)
+                           expert_norm_eps=self.norm_eps, map_fn=self.map_fn,
+                           act_scale="dynamic" if self.act_dynamic else "fixed", residual=self.residual)
+        if self.act_dynamic and self.o["h_amax"]:
+            # the two sides pick the same power of two for h unless max|h| sits
+            # within h's fp32 error of a boundary 6 * 448 * 2^e (checked here)
+            r = math.log2(self.o["h_amax"] / 2688.0)
+            assert abs(r - round(r)) > 1e-4, "seeded input has max|h| on a tensor-scale boundary"
         return self
 
     # ------------------------------------------------------------- checks
@@ -238,6 +253,7 @@ class Case:
         wo = np.take_along_axis(o["w"], order_o, axis=1)
         delta = np.take_along_axis(dl, oi, axis=1).max(axis=1)
         w_rtol = np.maximum(W_RTOL, 2 * delta + 4 * delta ** 2 + (k + 8) * U32)[:, None]
+        self.w_rtol_tok = w_rtol[:, 0]          # the weights' own error enters every partial
         bad = (np.abs(wg - wo) > w_rtol * np.abs(wo) + 1e-7) & keep[:, None]
         assert not bad.any(), f"routing weights: {int(bad.sum())} outside the derived tolerance"
         # permutation
@@ -302,8 +318,13 @@ class Case:
         # partial = w * (Wd h16) (light); with the norm the partial is the unweighted y
         wpair = np.abs(o["w"].reshape(-1)[o["perm"][ro]])
         wscale = np.ones_like(wpair) if self.norm_eps is not None else wpair
+        # the layer's fp32 routing weight is within w_rtol |w| (+ 2^-149 below
+        # fp32's range) of the oracle's; that error scales the whole partial
+        wrt = np.zeros_like(wpair) if self.norm_eps is not None else \
+            self.w_rtol_tok[o["perm"][ro] // self.cfg.k] * wpair + 2.0 ** -149
         hfl = 2.0 ** -35 * m["l1g"][ro, 0] * m["l1u"][ro, 0] * m["xmax"][ro, 0] ** 2
-        pb = wscale[:, None] * ((2.0 ** -10) * m["yabs"][ro] + (2 * hfl * m["l1d"][ro, 0])[:, None]) + 1e-30
+        pb = wscale[:, None] * ((2.0 ** -10) * m["yabs"][ro] + (2 * hfl * m["l1d"][ro, 0])[:, None]) + \
+            wrt[:, None] * m["yabs"][ro] + 1e-30
         dense = self.dense_rows(ro)
         self.n_dense_rows = int(dense.sum())
         self.flip_rows = {}      # GPU row -> |Wd| dev: effect of h codes that may round either way
@@ -313,11 +334,13 @@ class Case:
             tasks, sels = [], []
             for e in np.unique(e_of[dense]):
                 sel = np.nonzero(dense & (e_of == e))[0]
-                dev, _ = quant_deviation(o["h"][ro[sel]], hb[sel])
-                tasks.append((self.oracle_experts, int(e), dev))
+                gh = o["gs_h"]                  # h quantised as h / gs_h (1 unless dynamic)
+                dev, _ = quant_deviation(o["h"][ro[sel]] / gh, hb[sel] / gh)
+                tasks.append((self.oracle_experts, int(e), dev * gh))
                 sels.append(sel)
             for sel, flip in zip(sels, self.map_fn(abs_wd_times, tasks)):
-                pb[sel] = wscale[sel, None] * (flip + gam * (m["yabs"][ro[sel]] + flip)) + 1e-30
+                pb[sel] = wscale[sel, None] * (flip + gam * (m["yabs"][ro[sel]] + flip)) + \
+                    wrt[sel, None] * (m["yabs"][ro[sel]] + flip) + 1e-30
                 for n_i, r in enumerate(rg[sel]):
                     self.flip_rows[int(r)] = flip[n_i]
         ref = o["y"][ro] if self.norm_eps is not None else o["partial"][ro]
@@ -340,13 +363,13 @@ class Case:
         if self.norm_eps is not None:
             # the GPU's own partials (unweighted y), normalised and weighted in fp64
             wg = self.g["topk_w"].astype(np.float64)
-            pre = np.zeros((len(toks), self.cfg.d))
+            pre = O.bf16_bits_to_f64(self.x[toks]) if self.residual else np.zeros((len(toks), self.cfg.d))
             for j in range(k):
                 y = self.g["partial"][inv_g[toks * k + j]].astype(np.float64)
                 pre += wg[toks, j][:, None] * O.expert_rms_norm(y, self.norm_eps)
             hu = np.exp2(np.floor(np.log2(np.maximum(np.abs(pre), 2.0 ** -126))) - 8)
             # fp32 combine: the norm factors and a sum of k terms, relative to the terms' magnitudes
-            mag = np.zeros_like(pre)
+            mag = np.abs(O.bf16_bits_to_f64(self.x[toks])) if self.residual else np.zeros_like(pre)
             for j in range(k):
                 y = self.g["partial"][inv_g[toks * k + j]].astype(np.float64)
                 mag += np.abs(wg[toks, j][:, None] * O.expert_rms_norm(y, self.norm_eps))
@@ -354,7 +377,8 @@ class Case:
                 "out is not bf16 of its combine"
         else:
             # the combine: fp32 sum of the k partials in slot order, then bf16_rn
-            s32 = np.zeros((len(toks), self.cfg.d), np.float32)
+            s32 = (O.bf16_bits_to_f64(self.x[toks]).astype(np.float32) if self.residual
+                   else np.zeros((len(toks), self.cfg.d), np.float32))
             for j in range(k):
                 s32 = (s32 + self.g["partial"][inv_g[toks * k + j]].astype(np.float32)).astype(np.float32)
             assert np.array_equal(O.f64_to_bf16_bits_rne(s32.astype(np.float64)), self.g["out_bits"][toks]), \
@@ -392,12 +416,8 @@ class Case:
     def check_all(self):
         assert self.err == 0, f"device error word {self.err}"
         self.check_routing().check_intermediates().check_out()
-        try:
-            from tests.conftest import PARITY_REPORT
-            name = os.environ.get("PYTEST_CURRENT_TEST", self.cfg.name).split(" ")[0]
-            PARITY_REPORT.append((name, self.summary()))
-        except ImportError:
-            pass
+        name = os.environ.get("PYTEST_CURRENT_TEST", self.cfg.name).split(" ")[0]
+        PARITY_REPORT.append((name, self.summary()))
         return self
 
     def summary(self) -> dict:

@@ -76,3 +76,25 @@ def test_create_without_a_device_reports_cuda_error(lib):
         pytest.skip("a GPU is present")
     h = ctypes.c_void_p()
     assert lib.moe_fp4_create(8, 2, 512, 256, ctypes.byref(h)) == _lib.STATUS_CODE["MOE_FP4_ERR_CUDA"]
+
+
+def test_new_calls_reject_null_handles_and_bad_values(lib):
+    inv = _lib.STATUS_CODE["MOE_FP4_ERR_INVALID_ARG"]
+    assert lib.moe_fp4_set_expert_norm(None, 1, 1e-6) == inv
+    assert lib.moe_fp4_set_act_scale(None, 1) == inv
+    assert lib.moe_fp4_set_residual(None, 1) == inv
+    assert lib.moe_fp4_set_resident_classes(None, 1, 1) == inv
+    assert lib.moe_fp4_set_wait_timeout_ms(None, 5) == inv
+    assert lib.moe_fp4_set_unreachable_wait(None, 1) == inv
+    assert lib.moe_fp4_route(None, None, 1, None, None, None) == inv
+    assert lib.moe_fp4_forward_routed(None, None, 1, None, None, None) == inv
+    assert lib.moe_fp4_forward_layers(None, 1, None, 1, None, None, None) == inv
+    # handle-free calls check their sizes before touching any pointer
+    assert lib.moe_fp4_gather_rows(None, 4, 100, None, 4, 1, None, None) == inv      # d % 8
+    assert lib.moe_fp4_gather_rows(None, 0, 128, None, 0, 1, None, None) == 0        # nothing to do
+    assert lib.moe_fp4_combine_rows(None, None, None, -1, 1, 128, None, None) == inv
+    assert lib.moe_fp4_combine_rows(None, None, None, 0, 1, 128, None, None) == 0
+    import ctypes as C
+    wb, sb = C.c_size_t(1), C.c_size_t(1)
+    assert lib.moe_fp4_device_bytes(None, C.byref(wb), C.byref(sb)) == inv
+    assert lib.moe_fp4_last_error_detail() is not None

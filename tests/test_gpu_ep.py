@@ -2,9 +2,9 @@
 of nvfp4_expert_layer_b200.ep.  G ranks are held in one process on one GPU
 (the all-to-alls become slices), each with its own handle for its E/G
 experts; the sharded forward must match the single-device layer (bf16
-outputs within one ulp: the routing weight is applied in the combine instead
-of the down epilogue, a different fp32 rounding) and the oracle (1e-2 rms +
-half an ulp).  A one-rank NCCL process group runs the torch.distributed path
+outputs within one ulp or 1e-5 rms: the routing weight is applied in the
+combine instead of the down epilogue, a different fp32 rounding) and the
+oracle (1e-2 rms + half an ulp).  A one-rank NCCL process group runs the torch.distributed path
 (all-to-all through NCCL) on the same GPU.  Not measured across GPUs: this
 pool gives one GPU per run."""
 import os
@@ -20,10 +20,20 @@ from nvfp4_expert_layer_b200 import workloads as W
 from nvfp4_expert_layer_b200.ep import CudaEpBackend, ep_forward_local, shard_experts
 from nvfp4_expert_layer_b200.layer import MoeFp4Layer, experts_to_device
 from oracle import moe_oracle as O
-from tests.parity import bf16_to_bits, bf16_ulp_distance, to_dev_x
+from tests.parity import bf16_to_bits, to_dev_x
 
 pytestmark = pytest.mark.gpu
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _close_to_single_device(got, ref):
+    """Within one bf16 ulp of the single-device output, or 1e-5 rms absolutely
+    (the weight enters in the combine instead of the down epilogue, an fp32
+    rounding apart; near zero a sum may change sign by that much)."""
+    a, b = O.bf16_bits_to_f64(got), O.bf16_bits_to_f64(ref)
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(b), 2.0 ** -126))) - 7)
+    rms = np.sqrt(np.mean(b ** 2))
+    assert np.all(np.abs(a - b) <= ulp + 1e-5 * rms)
 
 
 def _oracle_check(x, rw, ex, cfg, thr, out_bits):
@@ -56,7 +66,7 @@ def test_virtual_ranks_match_single_device_and_oracle(G, T, thr):
     torch.cuda.synchronize()
     assert all(b.device_error() == 0 for b in backends)
     got = np.concatenate([bf16_to_bits(o) for o in outs])
-    assert bf16_ulp_distance(got, ref) <= 1
+    _close_to_single_device(got, ref)
     _oracle_check(x, rw, ex, cfg, thr, got)
     for b in backends:
         b.close()
@@ -97,12 +107,14 @@ ref = single(xd, rwd).view(torch.int16).cpu().numpy()
 b = CudaEpBackend(cfg.E, cfg.k, cfg.d, cfg.f, 0, 1, dev, rwd)
 out = ep_forward(b, xd).view(torch.int16).cpu().numpy()
 torch.cuda.synchronize()
-line = lambda v: np.where(v & 0x8000, -(v & 0x7FFF), v).astype(np.int64)
-diff = int(np.abs(line(out.view(np.uint16).astype(np.int64)) - line(ref.view(np.uint16).astype(np.int64))).max())
-print("ulp", diff, "err", b.device_error(), flush=True)
+f = lambda v: (v.view(np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+a, r = f(out), f(ref)
+ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(r), 2.0 ** -126))) - 7)
+ok = bool(np.all(np.abs(a - r) <= ulp + 1e-5 * np.sqrt(np.mean(r ** 2))))
+print("close", ok, "err", b.device_error(), flush=True)
 b.close()
 dist.destroy_process_group()
-sys.exit(0 if diff <= 1 else 3)
+sys.exit(0 if ok else 3)
 '''
 
 

@@ -142,3 +142,14 @@ def test_tensor_core_router_shapes(T, E, k, d):
     # a multiple of 128, a single expert
     cfg = W.custom_config(T=T, d=d, E=E, k=k, f=128, seed=60 + E, router="unit")
     Case(cfg).run_gpu().run_oracle().check_all()
+
+
+@pytest.mark.parametrize("T,E", [(20, 1), (32, 1), (33, 1), (64, 2), (97, 3)])
+def test_thirty_two_row_jobs(T, E):
+    # an expert with 17..32 rows is one job of the four-n-tile kernel; with
+    # more it splits into 32-row jobs plus a remainder (33 = 32 + 1).  T * k
+    # <= 32 takes the small-batch permutation, larger T the three-launch one.
+    cfg = W.custom_config(T=T, d=256, E=E, k=1, f=128, seed=200 + T, router="unit")
+    c = Case(cfg).run_gpu().run_oracle()
+    assert c.o["counts"].max() >= 17
+    c.check_all()

@@ -214,3 +214,56 @@ def test_expert_norm_keeps_the_routing_weights():
     np.testing.assert_allclose(rms, 1.0, rtol=1e-9)
     yn = O.expert_rms_norm(res["y"][res["inv"][0]][None], 0.0)[0]
     np.testing.assert_allclose(res["out64"][0], yn, rtol=1e-9, atol=1e-12)
+
+
+# ----------------------------------------------------------------- dynamic activation scale (R13)
+
+def test_pow2_tensor_scale_is_the_smallest_power_of_two():
+    rng = np.random.default_rng(9)
+    for a in list(np.exp(rng.uniform(-60, 60, size=200))) + [2688.0, 1344.0, 2688 * 2.0 ** -20, 1.0]:
+        g = O.pow2_tensor_scale(a)
+        e = int(round(math.log2(g)))
+        assert g == 2.0 ** e and a <= 2688.0 * g and not a <= 2688.0 * g / 2
+    assert O.pow2_tensor_scale(0.0) == 1.0
+
+
+def test_dynamic_scale_makes_the_dense_class_homogeneous_in_the_up_scale():
+    # h = SiLU(g) u is linear in u: scaling the up tensor scale by 2^-12
+    # scales h, the dynamic h scale, and so the output, by exactly 2^-12.  With
+    # the fixed scale 1 the small h underflows the e4m3 block scales instead.
+    cfg = W.custom_config(T=6, d=64, E=4, k=2, f=32, seed=29, router="unit")
+    x, rw, ex = W.gen_all(cfg)
+    a = O.forward(x, rw, ex, cfg.E, cfg.k, thr=1, act_scale="dynamic")
+    ex.up_gs = (ex.up_gs * np.float32(2.0 ** -12)).astype(np.float32)
+    b = O.forward(x, rw, ex, cfg.E, cfg.k, thr=1, act_scale="dynamic")
+    np.testing.assert_array_equal(b["out64"], a["out64"] * 2.0 ** -12)
+    assert b["gs_h"] == a["gs_h"] * 2.0 ** -12
+    fixed = O.forward(x, rw, ex, cfg.E, cfg.k, thr=1)
+    assert not np.allclose(fixed["out64"], b["out64"], rtol=1e-3, atol=0)
+
+
+def test_dynamic_scale_quantises_x_independently_of_its_magnitude():
+    # x * 2^-12 quantises to the same codes and block scales as x under the
+    # dynamic scale: the gate and up values scale by exactly 2^-12
+    cfg = W.custom_config(T=5, d=64, E=4, k=2, f=32, seed=31, router="unit")
+    x, rw, ex = W.gen_all(cfg)
+    xs = W.f32_to_bf16_bits_trunc(W.bf16_bits_to_f32(x) * np.float32(2.0 ** -12))
+    a = O.forward(x, rw, ex, cfg.E, cfg.k, thr=1, act_scale="dynamic", magnitudes=True)
+    b = O.forward(xs, rw, ex, cfg.E, cfg.k, thr=1, act_scale="dynamic", magnitudes=True)
+    rows = np.arange(cfg.T * cfg.k)
+    np.testing.assert_array_equal(b["mags"]["g"][rows], a["mags"]["g"][rows] * 2.0 ** -12)
+    np.testing.assert_array_equal(b["mags"]["u"][rows], a["mags"]["u"][rows] * 2.0 ** -12)
+    assert b["gs_x"] == a["gs_x"] * 2.0 ** -12
+
+
+# ----------------------------------------------------------------- residual add (R14)
+
+def test_residual_of_a_zero_expert_is_the_identity():
+    # down weights all zero: the block adds nothing, out = x exactly
+    cfg = W.custom_config(T=4, d=64, E=2, k=1, f=32, seed=37, router="unit")
+    x, rw, ex = W.gen_all(cfg)
+    ex.down_q[:] = 0
+    res = O.forward(x, rw, ex, cfg.E, cfg.k, residual=True)
+    assert np.array_equal(res["out_bits"], x)
+    plain = O.forward(x, rw, ex, cfg.E, cfg.k)
+    assert not np.any(plain["out64"])
