@@ -337,10 +337,17 @@ def launches_per_step(cfg) -> int:
 
 
 def bf16_ulp_distance(a_bits, b_bits) -> int:
-    def line(b):
-        b = np.asarray(b, np.int64)
-        return np.where(b & 0x8000, -(b & 0x7FFF), b)
-    return int(np.abs(line(a_bits) - line(b_bits)).max()) if np.size(a_bits) else 0
+    """Largest distance, in bf16 ulps of the reference b, over the elements
+    with |b| >= rms(b) / 64 (near zero the absolute tolerance governs)."""
+    f = lambda v: (np.asarray(v, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    a, b = f(a_bits), f(b_bits)
+    if not b.size:
+        return 0
+    big = (np.abs(b) >= np.sqrt(np.mean(b * b)) / 64) & (b != 0)
+    if not big.any():
+        return 0
+    ulp = np.exp2(np.floor(np.log2(np.abs(b[big]))) - 7)
+    return int(np.round(np.abs(a[big] - b[big]) / ulp).max())
 
 
 def parity_record(res, gpu) -> dict:

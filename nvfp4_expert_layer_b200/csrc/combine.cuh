@@ -32,8 +32,8 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float (&s)[8]) {
   return o;
 }
 
-// grid (min(T, cap), ceil(d / (8 * blockDim.x))); tokens t = blockIdx.x,
-// blockIdx.x + gridDim.x, ...; each thread owns 8 consecutive columns.
+// grid (ceil(d / (8 * blockDim.x)), min(T, 65535)); tokens t = blockIdx.y,
+// blockIdx.y + gridDim.y, ...; each thread owns 8 consecutive columns.
 // resid (optional, bf16 [T][d]): the sum starts from resid[t] (a residual add
 // in the same fp32 sum, one rounding).
 __device__ __forceinline__ void load_resid8(const uint16_t* resid, size_t off, float (&s)[8]) {
@@ -56,8 +56,8 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
                                                       int d, const uint16_t* __restrict__ resid,
                                                       uint16_t* __restrict__ out) {
   pdl_wait();
-  const int col = (blockIdx.y * blockDim.x + threadIdx.x) * 8;
-  for (int t = blockIdx.x; t < T && col < d; t += gridDim.x) {
+  const int col = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  for (int t = blockIdx.y; t < T && col < d; t += gridDim.y) {
     float s[8];
     load_resid8(resid, (size_t)t * d + col, s);
     // slots in groups of 8: all index loads, then all row loads, then the sums
@@ -189,13 +189,13 @@ __global__ void __launch_bounds__(256) unpermute_rows_kernel(const float* __rest
   }
 }
 
-// grid (min(T, cap), ceil(d / (8 * blockDim.x))), as combine_kernel
+// grid (ceil(d / (8 * blockDim.x)), min(T, 65535)), as combine_kernel
 __global__ void __launch_bounds__(128) combine_rows_kernel(const float* __restrict__ y,
                                                            const int* __restrict__ inv,
                                                            const float* __restrict__ wts, int T, int k,
                                                            int d, uint16_t* __restrict__ out) {
-  const int col = (blockIdx.y * blockDim.x + threadIdx.x) * 8;
-  for (int t = blockIdx.x; t < T && col < d; t += gridDim.x) {
+  const int col = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  for (int t = blockIdx.y; t < T && col < d; t += gridDim.y) {
     float s[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     for (int j = 0; j < k; ++j) {
       const float w = wts[(size_t)t * k + j];

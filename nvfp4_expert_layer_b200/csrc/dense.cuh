@@ -47,10 +47,13 @@ constexpr int kDenseStages = kDenseKStage == 128 ? 6 : 3;
 constexpr int kDenseN = 256;               // weight rows per tile (MMA N)
 constexpr int kDenseABytes = 128 * kDenseRowBytes;       // 128 rows of the M operand
 constexpr int kDenseBBytes = kDenseN * kDenseRowBytes;   // 256 rows of the N operand
-// Scale units in shared memory: each 1 KB unit of device memory four times in a row
-constexpr int kSfSmemUnit = kSfReplicas * kSfUnitBytes;
-constexpr int kDenseSfaBytes = kDenseMmaPerStage / 2 * kSfSmemUnit;   // M-side K-pair units (sf_pair_offset)
-constexpr int kDenseSfbBytes = kDenseMmaPerStage * kSfSmemUnit;       // N-side 256-row units (sf_rowpair_offset)
+// Scale blocks of a stage: one (tile, stage) block of device memory (2 KB M
+// side, 4 KB N side), placed four times in a row in shared memory
+constexpr int kSfaBlock = kSfPairUnitsPerStage * 4 * kSfGroupBytes;
+constexpr int kSfbBlock = kSfRowpairUnitsPerStage * 4 * kSfGroupBytes;
+constexpr int kDenseSfaBytes = kSfReplicas * kSfaBlock;   // M-side pair layout
+constexpr int kDenseSfbBytes = kSfReplicas * kSfbBlock;   // N-side rowpair layout
+static_assert(kDenseMmaPerStage == 4, "scale blocks assume four MMAs (K = 256) per stage");
 constexpr int kDenseStageBytes = kDenseABytes + kDenseBBytes + kDenseSfaBytes + kDenseSfbBytes;
 constexpr uint32_t kDenseTmemCols = 512;
 constexpr uint32_t kDenseSfCols = kDenseMmaPerStage * (4 + 8);   // per stage: 4 M-side + 8 N-side columns per MMA
@@ -201,12 +204,12 @@ __global__ void __launch_bounds__(256) gather_x_dense_kernel(
                              : make_uint4(0, 0, 0, 0);
       reinterpret_cast<uint4*>(xq + (size_t)(tile * 128 + r) * (d / 2))[ch] = v;
     }
-    // scales: 16-byte chunk q of unit p holds, for row slot l and 64-group
-    // 2p + h, the 4 scale bytes of rows l, l + 32, l + 64, l + 96 (see
-    // sf_pair_offset); consecutive threads write consecutive chunks
+    // scales: the 16 bytes of row slot l and 64-group g hold the 4 scale
+    // bytes of rows l, l + 32, l + 64, l + 96 (see sf_pair_offset), one 16-byte
+    // store per (pair, row slot, half)
     for (int c = threadIdx.x; c < npairs * 64; c += blockDim.x) {
       const int pr = c >> 6, q = c & 63;
-      const int l = (q >> 4) * 8 + (q & 7), h = (q >> 3) & 1;
+      const int l = q >> 1, h = q & 1;
       const int g = 2 * pr + h;                  // 64-wide K group
       uint32_t w[4];
 #pragma unroll
@@ -214,9 +217,8 @@ __global__ void __launch_bounds__(256) gather_x_dense_kernel(
         const int t = s_tok[l + 32 * m];
         w[m] = t >= 0 ? reinterpret_cast<const uint32_t*>(xsf_tok + (size_t)t * (d / 16))[g] : 0u;
       }
-      const uint4 v = make_uint4(w[0], w[1], w[2], w[3]);
-      uint8_t* unit = xsf + ((size_t)tile * npairs + pr) * kSfUnitBytes;
-      reinterpret_cast<uint4*>(unit)[q] = v;
+      *reinterpret_cast<uint4*>(xsf + sf_pair_offset((long long)tile * 128 + l, 4 * g, d / 64)) =
+          make_uint4(w[0], w[1], w[2], w[3]);
     }
   }
   pdl_launch_dependents();
@@ -379,8 +381,8 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
         const int trow = tl.de.w + tl.tt * (MODE == kDenseGateUp ? 128 : kDenseN);   // padded token row
         const int arow = MODE == kDenseGateUp ? trow : wrow;
         const int brow = MODE == kDenseGateUp ? wrow : trow;
-        const uint8_t* sfa = p.sfA + (size_t)(arow >> 7) * (p.kb64 >> 1) * kSfUnitBytes;
-        const uint8_t* sfb = p.sfB + (size_t)(brow >> 8) * p.kb64 * kSfUnitBytes;
+        const uint8_t* sfa = p.sfA + (size_t)(arow >> 7) * p.kstages * kSfaBlock;
+        const uint8_t* sfb = p.sfB + (size_t)(brow >> 8) * p.kstages * kSfbBlock;
         for (int ks = 0; ks < p.kstages; ++ks, ++k) {
           const int s = k % kDenseStages;
           if (!mbar_wait_spin(empty_b(s), ((k / kDenseStages) & 1) ^ 1, deadline)) {
@@ -390,24 +392,16 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
           mbar_arrive_expect_tx(full_b(s), kDenseStageBytes);
           tma_load_2d(st, &p.tmA, ks * kDenseRowBytes, arow, full_b(s), pol_a);
           tma_load_2d(st + kDenseABytes, &p.tmB, ks * kDenseRowBytes, brow, full_b(s), pol_w);
-          // scale units: each 1 KB unit is read from device memory once (its
-          // other three copies come from L2) into four consecutive 1 KB
-          // replicas, the source of one 128x256b copy
-          const uint8_t* sa = sfa + (size_t)(kDenseMmaPerStage / 2) * ks * kSfUnitBytes;
-          const uint8_t* sb = sfb + (size_t)kDenseMmaPerStage * ks * kSfUnitBytes;
+          // scale blocks: each read from device memory once (the other three
+          // copies come from L2) into four consecutive replicas
+          const uint8_t* sa = sfa + (size_t)ks * kSfaBlock;
+          const uint8_t* sb = sfb + (size_t)ks * kSfbBlock;
           const uint32_t da = st + kDenseABytes + kDenseBBytes, db = da + kDenseSfaBytes;
 #pragma unroll
-          for (int u = 0; u < kDenseMmaPerStage / 2; ++u)
-#pragma unroll
-            for (int rep = 0; rep < kSfReplicas; ++rep)
-              bulk_g2s(da + u * kSfSmemUnit + rep * kSfUnitBytes, sa + (size_t)u * kSfUnitBytes, kSfUnitBytes,
-                       full_b(s), pol_a);
-#pragma unroll
-          for (int u = 0; u < kDenseMmaPerStage; ++u)
-#pragma unroll
-            for (int rep = 0; rep < kSfReplicas; ++rep)
-              bulk_g2s(db + u * kSfSmemUnit + rep * kSfUnitBytes, sb + (size_t)u * kSfUnitBytes, kSfUnitBytes,
-                       full_b(s), pol_w);
+          for (int rep = 0; rep < kSfReplicas; ++rep) {
+            bulk_g2s(da + rep * kSfaBlock, sa, kSfaBlock, full_b(s), pol_a);
+            bulk_g2s(db + rep * kSfbBlock, sb, kSfbBlock, full_b(s), pol_w);
+          }
         }
       }
       // drain: every issued stage must land before the block exits
@@ -443,10 +437,12 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
           const uint32_t sfa_t = sf_t0 + kDenseSfCols * s, sfb_t = sfa_t + 4 * kDenseMmaPerStage;
 #pragma unroll
           for (int pr = 0; pr < kDenseMmaPerStage / 2; ++pr)
-            tc_cp_128x256b(sfa_t + 8 * pr, smem_desc_sf256(sfa_s + kSfSmemUnit * pr));
+            tc_cp_128x256b(sfa_t + 8 * pr, smem_desc_sf256(sfa_s + kSfGroupBytes * pr,
+                                                           kSfPairUnitsPerStage * kSfGroupBytes));
 #pragma unroll
           for (int kb = 0; kb < kDenseMmaPerStage; ++kb)
-            tc_cp_128x256b(sfb_t + 8 * kb, smem_desc_sf256(sfb_s + kSfSmemUnit * kb));
+            tc_cp_128x256b(sfb_t + 8 * kb, smem_desc_sf256(sfb_s + kSfGroupBytes * kb,
+                                                           kSfRowpairUnitsPerStage * kSfGroupBytes));
           const uint64_t adesc = smem_desc_kmajor<kDenseRowBytes>(st);
           const uint64_t bdesc = smem_desc_kmajor<kDenseRowBytes>(st + kDenseABytes);
 #pragma unroll

@@ -410,7 +410,10 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
     // 1. router logits and x staging; at most 32 pairs: top-k and the
     // permutation in the same launch
     const int epb = route_epb(d), tail = P <= 32 ? 1 : 0;
-    const dim3 rgrid((E + epb - 1) / epb);
+    // x staging blocks on the SMs the logit blocks leave free (one
+    // 1024-thread block fills an SM), for small batches
+    const int nlb = (E + epb - 1) / epb;
+    const dim3 rgrid(nlb + (T <= 32 ? std::min(T, std::max(0, h->sm_count - nlb)) : 0));
     const size_t rsm = route_smem_bytes(E, d, T, k);
     if (epb == 2)
       MOE_CUDA(launch(moe::route_kernel<2>, rgrid, dim3(1024), rsm, st, false, xb, rw, T, d, E, k, thr,
@@ -592,7 +595,7 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
                     st, pdl, (const float*)w.partial, (const int*)w.inv, (const float*)w.wts, T, k, d,
                     h->norm_eps, h->residual ? xb : nullptr, static_cast<uint16_t*>(out)));
   else
-    MOE_CUDA(launch(moe::combine_kernel, dim3(std::min(T, 65535), (d + 1023) / 1024), dim3(128), 0, st, pdl,
+    MOE_CUDA(launch(moe::combine_kernel, dim3((d + 1023) / 1024, std::min(T, 65535)), dim3(128), 0, st, pdl,
                     (const float*)w.partial, (const int*)w.inv, T, k, d, h->residual ? xb : nullptr,
                     static_cast<uint16_t*>(out)));
   MOE_CUDA(mark(h, 8, st));
@@ -1006,7 +1009,7 @@ int moe_fp4_combine_rows(const float* y_rows, const int32_t* inv, const float* t
   if (T == 0) return MOE_FP4_OK;
   if (!y_rows || !inv || !topk_w || !out) return MOE_FP4_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(y_rows) | reinterpret_cast<uintptr_t>(out)) & 15) return MOE_FP4_ERR_INVALID_ARG;
-  MOE_CUDA(launch(moe::combine_rows_kernel, dim3(std::min(T, 65535), (d + 1023) / 1024), dim3(128), 0, stream,
+  MOE_CUDA(launch(moe::combine_rows_kernel, dim3((d + 1023) / 1024, std::min(T, 65535)), dim3(128), 0, stream,
                   false, y_rows, (const int*)inv, topk_w, T, top_k, d, static_cast<uint16_t*>(out)));
   return MOE_FP4_OK;
 }

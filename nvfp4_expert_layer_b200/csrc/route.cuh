@@ -681,7 +681,9 @@ __global__ void __launch_bounds__(1024) perm_place_kernel(const int* __restrict_
 }
 
 // Small-T router logits (T <= 256) and x staging in one launch, plus the
-// routing tail for at most 32 (token, expert) pairs.  Block b (1024 threads)
+// routing tail for at most 32 (token, expert) pairs.  With T <= 32 the grid
+// may have extra blocks (on SMs the logit blocks leave free) that only stage
+// x, in parallel with the logits.  Block b (1024 threads)
 // computes the fp32 logits of experts EPB*b .. EPB*b + EPB-1 for every token:
 // the router rows are staged in shared memory, thread i owns K = [8i, 8i+8)
 // (and [8(i+1024), ...) when d > 8192, EPB = 1), so one x load feeds EPB
@@ -701,28 +703,17 @@ __global__ void __launch_bounds__(1024) route_kernel(
   extern __shared__ __align__(16) int sm[];
   __shared__ float red[33];
   __shared__ int s_last;
-  const int e0 = blockIdx.x * EPB;
+  // blocks [0, nlb) compute logits; extra blocks, if any, only stage x (in
+  // parallel with the logits); without them the logit blocks stage x
+  const int nlb = (E + EPB - 1) / EPB;
+  const bool stage_only = blockIdx.x >= nlb;
+  const int e0 = stage_only ? E : blockIdx.x * EPB;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  float* s_w = reinterpret_cast<float*>(sm);            // [EPB][d]
-#pragma unroll
-  for (int j = 0; j < EPB; ++j) {
-    if (e0 + j >= E) break;
-    // d <= 16384: at most 4 float4 per thread, all loads issued before the stores
-    const float4* src = reinterpret_cast<const float4*>(rw + (size_t)(e0 + j) * d);
-    float4 v[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int i = threadIdx.x + q * blockDim.x;
-      if (i < d / 4) v[q] = src[i];
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int i = threadIdx.x + q * blockDim.x;
-      if (i < d / 4) reinterpret_cast<float4*>(s_w + (size_t)j * d)[i] = v[q];
-    }
-  }
-  __syncthreads();
+  float* s_w = reinterpret_cast<float*>(sm);
   float* s_part = s_w + (size_t)EPB * d;                // [EPB][32 tokens][32 warps]
+  // each thread's router weights straight into registers: thread i owns
+  // K = [8 i, 8 i + 8) (and [8 (i + 1024), ...) when NG = 2); every weight
+  // is used from registers for all tokens, so no shared-memory staging
   float4 wa[EPB][NG], wb[EPB][NG];
   bool has[NG];
 #pragma unroll
@@ -732,11 +723,12 @@ __global__ void __launch_bounds__(1024) route_kernel(
 #pragma unroll
     for (int j = 0; j < EPB; ++j) {
       const bool ok = has[q] && e0 + j < E;
-      wa[j][q] = ok ? *reinterpret_cast<const float4*>(s_w + (size_t)j * d + kk) : make_float4(0, 0, 0, 0);
-      wb[j][q] = ok ? *reinterpret_cast<const float4*>(s_w + (size_t)j * d + kk + 4) : make_float4(0, 0, 0, 0);
+      const float4* src = reinterpret_cast<const float4*>(rw + (size_t)(e0 + j) * d + kk);
+      wa[j][q] = ok ? __ldg(src) : make_float4(0, 0, 0, 0);
+      wb[j][q] = ok ? __ldg(src + 1) : make_float4(0, 0, 0, 0);
     }
   }
-  for (int t0 = 0; t0 < T; t0 += 32) {
+  for (int t0 = 0; t0 < (stage_only ? 0 : T); t0 += 32) {
     const int tn = min(32, T - t0);
     // four tokens per pass: their x loads are in flight together (the loop is
     // latency-bound, not issue-bound); each token's sum keeps the same order
@@ -797,8 +789,14 @@ __global__ void __launch_bounds__(1024) route_kernel(
     }
     __syncthreads();
   }
-  for (int t = blockIdx.x; t < T; t += gridDim.x)
-    stage_x_row(x + (size_t)t * d, d, x16 + (size_t)t * d, xscale + t, o.err, red);
+  if (gridDim.x > nlb) {
+    if (stage_only)
+      for (int t = blockIdx.x - nlb; t < T; t += gridDim.x - nlb)
+        stage_x_row(x + (size_t)t * d, d, x16 + (size_t)t * d, xscale + t, o.err, red);
+  } else {
+    for (int t = blockIdx.x; t < T; t += gridDim.x)
+      stage_x_row(x + (size_t)t * d, d, x16 + (size_t)t * d, xscale + t, o.err, red);
+  }
   if (!tail) {
     pdl_launch_dependents();
     return;

@@ -89,12 +89,13 @@ __device__ __forceinline__ uint64_t smem_desc_kmajor(uint32_t saddr) {
 
 // Scale-factor copy source: 128 rows x 32 bytes, no swizzle, as core matrices
 // of 8 rows x 16 bytes; the two 16-byte halves of a row group are 128 bytes
-// apart (leading byte offset), row groups 256 bytes apart (stride byte offset).
-__device__ __forceinline__ uint64_t smem_desc_sf256(uint32_t saddr) {
+// apart (leading byte offset), row groups `sbo` bytes apart (stride byte
+// offset: 256 times the units per stage of the interleaved scale layouts).
+__device__ __forceinline__ uint64_t smem_desc_sf256(uint32_t saddr, uint32_t sbo) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFF);
   d |= (uint64_t)(128 >> 4) << 16;
-  d |= (uint64_t)(256 >> 4) << 32;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
   d |= (uint64_t)1 << 46;
   return d;                                         // layout: SWIZZLE_NONE
 }
@@ -132,45 +133,53 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
   return __half2float(__ushort_as_half((unsigned short)(h2 & 0xffffu)));
 }
 
-// Byte offset of the scale of (row r, K block kb of 16) in the scale layout of
-// the tensor-core operands.  Rows are grouped by 128 (one MMA tile) and K by
-// pairs of 64-wide groups (two MMAs); each (row tile, pair) is a 1 KB unit
-// holding 32 row slots l = r % 32 as 8-row core matrices at
-//   (l / 8) * 256 + h * 128 + (l % 8) * 16 + (r % 128 / 32) * 4 + kb % 4,
-// h = which 64-group of the pair.  Device memory holds each unit once; the
-// GEMMs place it four times in a row in shared memory (kSfReplicas), which
-// makes the 4 KB, 128-row source of one tcgen05.cp .128x256b that gives
-// every TMEM lane quarter the same 32 x 8 columns: column 4h + (r % 128) / 32
-// of lane r % 32 holds the four scales of row r for the MMA of 64-group h.
-// Size in device memory: rows / 128 * (K / 128) * 1024 bytes.
+// Scale layouts of the tensor-core operands.  The scale bytes of one MMA
+// (K = 64, four 16-blocks) for 128 rows form a "unit" of 32 row slots
+// l = r % 32 in four 8-row groups g = l / 8, a group being 256 bytes:
+//   h * 128 + (l % 8) * 16 + (r % 128 / 32) * 4 + kb % 4,
+// where h picks one of two 16-byte columns.  A tcgen05.cp .128x256b copies
+// 128 rows x 32 bytes (16 groups, the two 16-byte columns 128 bytes apart)
+// and fills every TMEM lane quarter with the same 32 x 8 columns when its
+// source is a unit four times over (groups 4i..4i+3 = replica i).  So that
+// one bulk copy moves one replica of all the units of a K-stage (K = 256),
+// the units of a (row tile, stage) are interleaved by group in memory:
+//   block (tile, stage) = [group g (4)][unit j (U)][256 bytes],  U units per stage,
+// and the copy of unit j reads groups at j * 256 + g * U * 256 (the
+// descriptor's stride).  Device memory holds each block once; shared memory
+// holds it four times in a row (kSfReplicas).
 constexpr int kSfReplicas = 4;
-constexpr int kSfUnitBytes = 1024;
+constexpr int kSfGroupBytes = 256;
+
+// M side, 128-row tiles (pair layout): a unit covers two 64-wide K groups
+// (h = which one), two units per stage; column 4h + (r % 128) / 32 of lane
+// r % 32 holds the four scales of row r for the MMA of 64-group h.
+// Size: rows / 128 * (K / 128) * 1024 bytes.
+constexpr int kSfPairUnitsPerStage = 2;
 __host__ __device__ __forceinline__ size_t sf_pair_offset(long long r, int kb, int kblocks64) {
   const long long tile = r >> 7;
-  const int rr = (int)(r & 127), l = rr & 31, kg = kb >> 2;
-  return ((size_t)tile * (kblocks64 >> 1) + (kg >> 1)) * kSfUnitBytes +
-         (size_t)((l >> 3) * 256 + (kg & 1) * 128 + (l & 7) * 16 + (rr >> 5) * 4 + (kb & 3));
+  const int rr = (int)(r & 127), l = rr & 31, kg = kb >> 2, pr = kg >> 1;
+  const int stage = pr >> 1, j = pr & 1, nstages = kblocks64 >> 2;
+  return (((size_t)tile * nstages + stage) * 4 + (l >> 3)) * (kSfPairUnitsPerStage * kSfGroupBytes) +
+         (size_t)(j * kSfGroupBytes + (kg & 1) * 128 + (l & 7) * 16 + (rr >> 5) * 4 + (kb & 3));
 }
 __host__ __device__ constexpr size_t sf_pair_bytes(long long rows, int K) {
-  return (size_t)(rows / 128) * (K / 128) * kSfUnitBytes;
+  return (size_t)(rows / 128) * (K / 128) * 1024;
 }
 
-// Scale layout of an operand read as 256-row MMA tiles (N = 256): 1 KB units
-// per (256-row group, 64-wide K group) with 32 row slots l = r % 32 as core
-// matrices at
-//   (l / 8) * 256 + h * 128 + (l % 8) * 16 + (r % 128 / 32) * 4 + kb % 4,
-// h = (r % 256) / 128.  Stored once in device memory and four times in a row
-// in shared memory, where one tcgen05.cp .128x256b of the 4 KB fills the 8
-// scale columns one N = 256 MMA reads: column (r % 256) / 32 of lane r % 32,
-// in every lane quarter.  Size: rows / 256 * (K / 64) * 1024 bytes.
+// N side, 256-row groups (rowpair layout): a unit covers one 64-wide K group
+// for 256 rows (h = (r % 256) / 128), four units per stage; one copy fills
+// the 8 scale columns one N = 256 MMA reads: column (r % 256) / 32 of lane
+// r % 32.  Size: rows / 256 * (K / 64) * 1024 bytes.
+constexpr int kSfRowpairUnitsPerStage = 4;
 __host__ __device__ __forceinline__ size_t sf_rowpair_offset(long long r, int kb, int kblocks64) {
-  const long long g = r >> 8;
-  const int rr = (int)(r & 255), h = rr >> 7, r128 = rr & 127, l = r128 & 31;
-  return ((size_t)g * kblocks64 + (kb >> 2)) * kSfUnitBytes +
-         (size_t)((l >> 3) * 256 + h * 128 + (l & 7) * 16 + (r128 >> 5) * 4 + (kb & 3));
+  const long long grp = r >> 8;
+  const int rr = (int)(r & 255), h = rr >> 7, r128 = rr & 127, l = r128 & 31, kg = kb >> 2;
+  const int stage = kg >> 2, j = kg & 3, nstages = kblocks64 >> 2;
+  return (((size_t)grp * nstages + stage) * 4 + (l >> 3)) * (kSfRowpairUnitsPerStage * kSfGroupBytes) +
+         (size_t)(j * kSfGroupBytes + h * 128 + (l & 7) * 16 + (r128 >> 5) * 4 + (kb & 3));
 }
 __host__ __device__ constexpr size_t sf_rowpair_bytes(long long rows, int K) {
-  return (size_t)(rows / 256) * (K / 64) * kSfUnitBytes;
+  return (size_t)(rows / 256) * (K / 64) * 1024;
 }
 
 }  // namespace moe

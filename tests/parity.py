@@ -137,12 +137,18 @@ def bf16_to_bits(t: torch.Tensor) -> np.ndarray:
 
 
 def bf16_ulp_distance(a_bits: np.ndarray, b_bits: np.ndarray) -> int:
-    """Largest distance in bf16 ulps between two arrays of bf16 bit patterns
-    (the patterns mapped to a monotone integer line, -0 and +0 equal)."""
-    def line(b):
-        b = np.asarray(b, np.int64)
-        return np.where(b & 0x8000, -(b & 0x7FFF), b)
-    return int(np.abs(line(a_bits) - line(b_bits)).max()) if np.size(a_bits) else 0
+    """Largest distance, in bf16 ulps of the reference value b, between two
+    arrays of bf16 bit patterns, over the elements with |b| >= rms(b) / 64
+    (near zero an ulp is tiny and the absolute tolerance governs)."""
+    a = O.bf16_bits_to_f64(np.asarray(a_bits))
+    b = O.bf16_bits_to_f64(np.asarray(b_bits))
+    if not b.size:
+        return 0
+    big = (np.abs(b) >= np.sqrt(np.mean(b * b)) / 64) & (b != 0)
+    if not big.any():
+        return 0
+    ulp = np.exp2(np.floor(np.log2(np.abs(b[big]))) - 7)
+    return int(np.round(np.abs(a[big] - b[big]) / ulp).max())
 
 
 def oracle_pool(workers: int = 16):
