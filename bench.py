@@ -66,6 +66,8 @@ def parse(argv=None):
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="all")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--thr", type=int, default=DENSE_THR,
+                    help="dense-class row threshold (experts with at least thr rows run on tcgen05)")
     ap.add_argument("--shape", default="",
                     help="profiling sizes over one workload's recipe, e.g. T=4096,E=32 "
                          "(the JSON line then names the changed sizes)")
@@ -73,7 +75,8 @@ def parse(argv=None):
 
 
 def workload_names(args):
-    return ALL if args.workload == "all" else (args.workload,)
+    """`all`, one workload, or a comma-separated list of them."""
+    return ALL if args.workload == "all" else tuple(args.workload.split(","))
 
 
 def workload_config(name, shape=""):
@@ -129,7 +132,12 @@ def measured_peaks():
         return 6650.0, 1590.0 * FP4_OVER_BF16, "fallback"
 
 
-def is_dense(cfg, thr=128) -> bool:
+# Row count from which an expert runs in the dense (tensor-core) class: the
+# library's default, chosen from the measurements in the design notes.
+DENSE_THR = 128
+
+
+def is_dense(cfg, thr=DENSE_THR) -> bool:
     """Whether the workload's experts may run in the dense class (T >= thr and
     the shapes the tensor-core path supports)."""
     return cfg.T >= thr and cfg.d % 256 == 0 and cfg.f % 256 == 0
@@ -262,7 +270,7 @@ def cpu_cores() -> int:
         return os.cpu_count() or 1
 
 
-def cpu_baseline_sample(cfg, x_np, rw_np):
+def cpu_baseline_sample(cfg, x_np, rw_np, thr=DENSE_THR):
     """The oracle on a bounded sample of the first pool input: routing and the
     permutation of the whole batch in fp64 (which decide the expert classes),
     then the experts of its first min(T, 4) tokens (one token for the
@@ -277,7 +285,7 @@ def cpu_baseline_sample(cfg, x_np, rw_np):
     for e in np.unique(ids):
         lazy.expert(int(e))
     t0 = time.perf_counter()
-    res = O.forward(x_np, rw_np, lazy, cfg.E, cfg.k, thr=128, token_subset=list(range(n)))
+    res = O.forward(x_np, rw_np, lazy, cfg.E, cfg.k, thr=thr, token_subset=list(range(n)))
     secs = time.perf_counter() - t0
     sample = (f"oracle on the {cfg.name} workload: routing and permutation of all {cfg.T} tokens "
               f"(fp64 logits), then the experts of its first {n} token(s) dequantised exactly and "
@@ -324,16 +332,18 @@ def pool_inputs(cfg, n):
     return xs, rw
 
 
-def launches_per_step(cfg) -> int:
+def launches_per_step(cfg, thr=DENSE_THR) -> int:
     """Kernels one forward launches: routing (up to 256 tokens the router
     kernel, which for at most 32 pairs also runs top-k and the permutation,
     else top-k and 3 permutation kernels follow it; above 256 tokens the
     weight split, router, x staging, top-k and 3 permutation kernels), the
     dense class (quantiser, gather, 2 GEMMs) when T >= thr, the light-class
-    expert kernels (the 9..16-row one only when T >= 9) and the combine."""
+    expert kernels (the 9..16-row one when T >= 9, the 17..32-row one when
+    T >= 17) and the combine."""
     pairs = cfg.T * cfg.k
     routing = (1 if pairs <= 32 else 5) if cfg.T <= 256 else 7
-    return routing + (4 if is_dense(cfg) else 0) + (2 if cfg.T >= 9 else 1) + 1
+    light = 1 + (1 if cfg.T >= 9 else 0) + (1 if cfg.T >= 17 else 0)
+    return routing + (4 if is_dense(cfg, thr) else 0) + light + 1
 
 
 def bf16_ulp_distance(a_bits, b_bits) -> int:
@@ -415,7 +425,8 @@ def run_workload(args, cfg, layer, rank, world, local):
     xs = [torch.from_numpy(x.view(np.int16).copy()).cuda().view(torch.bfloat16) for x in xs_np]
     rw = torch.from_numpy(rw_np).cuda()
     out = torch.empty_like(xs[0])
-    layer.set_dense_threshold(128)
+    thr = args.thr
+    layer.set_dense_threshold(thr)
     # units of work of one step, from the layer's own routing: distinct experts
     # touched (decode bytes) and rows of dense-class experts (prefill FLOPs)
     experts_per_input, dense_rows = [], []
@@ -423,8 +434,13 @@ def run_workload(args, cfg, layer, rank, world, local):
         _, dbg = layer.forward_ex(x, rw, want=("counts",))
         c = dbg["counts"].cpu().numpy()
         experts_per_input.append(int((c > 0).sum()))
-        dense_rows.append(int(c[c >= 128].sum()) if is_dense(cfg) else 0)
-    dense = is_dense(cfg) and sum(dense_rows) > 0
+        dense_rows.append(int(c[c >= thr].sum()) if is_dense(cfg, thr) else 0)
+    any_dense = is_dense(cfg, thr) and sum(dense_rows) > 0
+    # tensor-bound roofline when most routed rows are in the dense class
+    # (prefill); otherwise the HBM roofline of the whole expert phase (every
+    # kernel that streams expert weights: the light kernels and, for experts
+    # with at least thr rows, the dense class)
+    dense = any_dense and np.mean(dense_rows) >= 0.5 * cfg.T * cfg.k
     stream = torch.cuda.Stream()
     graphs = []
     with torch.cuda.stream(stream):
@@ -460,7 +476,12 @@ def run_workload(args, cfg, layer, rank, world, local):
     del graphs
     # ---- per-stage pass: the same graphs with stage events (events between stages)
     nst = len(layer.STAGES)
-    dom = layer.STAGES.index("dense_gate_up" if dense else "light")
+    if dense:
+        dom = [layer.STAGES.index("dense_gate_up")]
+    else:
+        dom = [layer.STAGES.index("light")] + ([layer.STAGES.index(n) for n in
+                                                ("dense_quant", "dense_gate_up", "dense_down")]
+                                               if any_dense else [])
     stage_ms = np.zeros(nst)
     sgraphs, sevents = [], []
     with torch.cuda.stream(stream):
@@ -485,7 +506,7 @@ def run_workload(args, cfg, layer, rank, world, local):
         for i in range(pool):
             d = [sevents[i][j].elapsed_time(sevents[i][j + 1]) for j in range(nst)]
             stage_ms += d
-            dom_ms += d[dom]
+            dom_ms += sum(d[j] for j in dom)
             if dense:   # gate and up GEMMs over the routed rows: 2 * rows * d * 2f
                 dom_work += 2.0 * dense_rows[i] * cfg.d * 2 * cfg.f
             else:
@@ -522,8 +543,8 @@ def run_workload(args, cfg, layer, rank, world, local):
     torch.cuda.empty_cache()
     return dict(cfg=cfg, ms=ms, clk=clk, err=err, stage_ms=stage_ms, dom_ms=dom_ms / n,
                 dom_work=dom_work / n, dense=dense, e2e_ms=e2e_ms, xs_np=xs_np, rw_np=rw_np,
-                gpu=gpu, launches=launches_per_step(cfg), stages=layer.STAGES,
-                dense_rows=float(np.mean(dense_rows)), pool=pool)
+                gpu=gpu, launches=launches_per_step(cfg, thr), stages=layer.STAGES,
+                dense_rows=float(np.mean(dense_rows)), any_dense=any_dense, thr=thr, pool=pool)
 
 
 def workload_record(args, r, world) -> dict:
@@ -543,7 +564,11 @@ def workload_record(args, r, world) -> dict:
         dtype = "fp4"
     else:
         achieved = r["dom_work"] / (r["dom_ms"] * 1e-3) / 1e9
-        roofline = {"bound": "hbm", "kernel": "expert_kernel (gate/up + SwiGLU + down, light class)",
+        kern = "expert_kernel (gate/up + SwiGLU + down, light class)"
+        if r["any_dense"]:
+            kern = (f"expert phase: expert_kernel (light class) + quantiser and dense_gemm_kernel "
+                    f"gate/up, down (experts with >= {r['thr']} rows)")
+        roofline = {"bound": "hbm", "kernel": kern,
                     "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
                     "peak_kind": peak_kind, "traffic": recorded_traffic("expert_kernel", cfg.name),
                     "nominal_peak": NOMINAL_HBM_GBS, "frac_nominal": achieved / NOMINAL_HBM_GBS,
@@ -551,6 +576,7 @@ def workload_record(args, r, world) -> dict:
         compute = "fp4 weights dequantised in registers to fp16, m16n8k16 MMA, fp32 accumulate"
         dtype = "f16"
     conf = config_dict(cfg, world)
+    conf["dense_threshold"] = r["thr"]
     return {
         "metric": METRIC, "value": tokens / (r["ms"] * 1e-3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms"] / args.steps,
@@ -628,7 +654,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         for r in runs:
             cfg = r["cfg"]
-            secs, n, res, sample = cpu_baseline_sample(cfg, r["xs_np"][0], r["rw_np"])
+            secs, n, res, sample = cpu_baseline_sample(cfg, r["xs_np"][0], r["rw_np"], r["thr"])
             rec = records[cfg.name]
             rec["cpu_baseline"] = {"value": n / secs, "unit": "tokens/s", "cores": cpu_cores(),
                                    "kind": "oracle", "sample": sample}

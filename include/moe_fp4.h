@@ -39,6 +39,10 @@
  *   and f to be multiples of 256 (one 256-element K stage of the tensor-core
  *   pipeline); for other shapes, or if the driver's tensor-map encoder is not
  *   available, every expert runs in the light class whatever its row count.
+ *   The dense GEMMs run on CTA pairs (clusters of two SMs, 256 x 256 tiles)
+ *   when the device fits them, else on single CTAs (128-row tiles); the
+ *   environment variable MOE_FP4_DENSE_PAIRS set to "0" at create time
+ *   selects the single-CTA kernels.  Both give results within the same bounds.
  *
  * Conventions
  *   - Every call returns a moe_fp4_status and never aborts the process.

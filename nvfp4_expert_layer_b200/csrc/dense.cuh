@@ -43,29 +43,48 @@ constexpr int kDenseThreads = 64 + 32 * kDenseEpiWarps;   // warp 0 TMA, warp 1 
 constexpr int kDenseKStage = 256;
 constexpr int kDenseRowBytes = kDenseKStage / 2;
 constexpr int kDenseMmaPerStage = kDenseKStage / 64;
-constexpr int kDenseStages = kDenseKStage == 128 ? 6 : 3;
+// Scale copies into TMEM, per GEMM (DenseStageCfg): a broadcast copy
+// (tcgen05.cp .32x128b.warpx4) fills all four TMEM lane quarters from one
+// 512-byte source, so shared memory holds every scale block once (6 KB a
+// stage) and four stages fit; a .128x256b copy reads four replicas of a
+// block (24 KB a stage, three stages) with half the copy instructions.  On
+// B200 the down GEMM (8 stages per tile) gains from the fourth stage and the
+// gate/up GEMM (28 stages per tile) from the fewer copies.
 constexpr int kDenseN = 256;               // weight rows per tile (MMA N)
 constexpr int kDenseABytes = 128 * kDenseRowBytes;       // 128 rows of the M operand
 constexpr int kDenseBBytes = kDenseN * kDenseRowBytes;   // 256 rows of the N operand
 // Scale blocks of a stage: one (tile, stage) block of device memory (2 KB M
-// side, 4 KB N side), placed four times in a row in shared memory
+// side, 4 KB N side), placed kDenseSfCopies times in a row in shared memory
 constexpr int kSfaBlock = kSfPairUnitsPerStage * 4 * kSfGroupBytes;
 constexpr int kSfbBlock = kSfRowpairUnitsPerStage * 4 * kSfGroupBytes;
-constexpr int kDenseSfaBytes = kSfReplicas * kSfaBlock;   // M-side pair layout
-constexpr int kDenseSfbBytes = kSfReplicas * kSfbBlock;   // N-side rowpair layout
-static_assert(kDenseMmaPerStage == 4, "scale blocks assume four MMAs (K = 256) per stage");
-constexpr int kDenseStageBytes = kDenseABytes + kDenseBBytes + kDenseSfaBytes + kDenseSfbBytes;
 constexpr uint32_t kDenseTmemCols = 512;
 constexpr uint32_t kDenseSfCols = kDenseMmaPerStage * (4 + 8);   // per stage: 4 M-side + 8 N-side columns per MMA
-static_assert(kDenseN + kDenseSfCols * kDenseStages <= kDenseTmemCols, "accumulator + scales exceed TMEM");
-constexpr int kDenseBarBytes = (2 * kDenseStages + 3) * 8 + 8;   // full[S] empty[S] accf acce done, padded
 
 enum DenseMode { kDenseGateUp = 0, kDenseDown = 1 };
+
+template <int MODE>
+struct DenseStageCfg {
+  static constexpr bool kBcast = MODE == kDenseDown;
+  static constexpr int kCopies = kBcast ? 1 : kSfReplicas;        // copies of each scale block in shared memory
+  static constexpr int kStages = kBcast ? 4 : 3;
+  static constexpr int kSfaBytes = kCopies * kSfaBlock;           // M-side pair layout
+  static constexpr int kSfbBytes = kCopies * kSfbBlock;           // N-side rowpair layout
+  static constexpr int kStageBytes = kDenseABytes + kDenseBBytes + kSfaBytes + kSfbBytes;
+  static constexpr int kBarBytes = (2 * kStages + 3) * 8 + 8;     // full[S] empty[S] accf acce done, padded
+  static_assert(kDenseN + kDenseSfCols * kStages <= kDenseTmemCols, "accumulator + scales exceed TMEM");
+  static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled tiles");
+};
 
 // Dense list entry: {expert, row0 (permutation rows), rows, padded row0}.
 struct DenseParams {
   CUtensorMap tmA;       // M side, box 128 B x 128 rows: gate/up x codes [pad rows][d/2]; down Wd [E*d][f/2]
   CUtensorMap tmB;       // N side, box 128 B x 256 rows: gate/up combined W [E*2f][d/2]; down h codes [pad rows][f/2]
+  // CTA pairs (dense_gemm_pair_kernel): the N side in boxes of 128 rows, and
+  // the scale blocks as 2-D byte tensors of 256-byte rows (a stage's M-side
+  // block is 8 rows, its N-side block 16 rows)
+  CUtensorMap tmB2;
+  CUtensorMap tmSfa;
+  CUtensorMap tmSfb;
   const uint8_t* sfA;    // M-side scales (sf_pair_offset layout)
   const uint8_t* sfB;    // N-side scales (sf_rowpair_offset layout)
   const int4* dense;     // dense list, ranked by rows descending
@@ -119,8 +138,9 @@ __device__ __forceinline__ float exp2i_f(int e) { return __int_as_float((e + 127
 //   rows: the codes and scales of token perm[row0 + i] / topk copied into the
 //   padded permutation order (scales assembled into whole sf_pair_offset
 //   units, written with coalesced 16-byte stores).
-//   Rows past an expert's count up to its next multiple of 128 -- the rows a
-//   128-token tile reads -- are zeros; rows beyond are never read.
+//   Rows past an expert's count up to its next multiple of tile_rows -- the
+//   rows a token tile of the gate/up GEMM reads (128, or 256 for CTA pairs)
+//   -- are zeros; rows beyond are never read.
 // Each token is quantised once, however many dense experts it is routed to.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ int dense_rank_of_padrow(const int4* dense, int nd, int prow) {
@@ -177,7 +197,7 @@ __global__ void __launch_bounds__(256) quant_tok_kernel(const uint16_t* __restri
 __global__ void __launch_bounds__(256) gather_x_dense_kernel(
     const uint8_t* __restrict__ xq_tok, const uint8_t* __restrict__ xsf_tok, const int4* __restrict__ dense,
     const int* __restrict__ n_dense, const int* __restrict__ pad_total, const int* __restrict__ perm, int topk,
-    int d, uint8_t* __restrict__ xq, uint8_t* __restrict__ xsf) {
+    int d, int tile_rows, uint8_t* __restrict__ xq, uint8_t* __restrict__ xsf) {
   __shared__ int s_tok[128];                     // token of each row of the tile, -1 for padding
   pdl_wait();
   const int nd = *n_dense;
@@ -189,7 +209,7 @@ __global__ void __launch_bounds__(256) gather_x_dense_kernel(
     // a 128-row tile lies inside one expert: padding is to 256 rows
     const int4 de = dense[dense_rank_of_padrow(dense, nd, tile * 128)];
     const int i0 = tile * 128 - de.w;
-    if (i0 >= ((de.z + 127) & ~127)) continue;   // beyond the last 128-token tile: never read
+    if (i0 >= (de.z + tile_rows - 1) / tile_rows * tile_rows) continue;   // beyond the last token tile: never read
     __syncthreads();                             // s_tok of the previous tile consumed
     if (threadIdx.x < 128) {
       const int i = i0 + threadIdx.x;
@@ -247,12 +267,13 @@ __global__ void __launch_bounds__(256) amax_bf16_kernel(const uint16_t* __restri
 
 // Dynamic h scale: the NVFP4 h of every padded dense row from the fp32 h the
 // gate/up GEMM wrote (permutation rows), quantised as h * 2^-e_h with the R4
-// rule; rows past an expert's count up to its next multiple of 128 are zeros.
+// rule; rows past an expert's count up to its next multiple of tile_rows
+// (the token tile of the down GEMM: 128, or 256 for CTA pairs) are zeros.
 // One warp per (padded row, 8 blocks of 16): codes and sf_rowpair_offset scales.
 __global__ void __launch_bounds__(256) quant_h_dense_kernel(const float* __restrict__ h32, const int4* __restrict__ dense,
                                                             const int* __restrict__ n_dense,
                                                             const int* __restrict__ pad_total,
-                                                            const int* __restrict__ h_amax, int f,
+                                                            const int* __restrict__ h_amax, int f, int tile_rows,
                                                             uint8_t* __restrict__ hq, uint8_t* __restrict__ hsf) {
   pdl_wait();
   const int nd = *n_dense;
@@ -265,7 +286,7 @@ __global__ void __launch_bounds__(256) quant_h_dense_kernel(const float* __restr
     const int r = (int)(u / nb), kb = (int)(u - (long long)r * nb);
     const int4 de = dense[dense_rank_of_padrow(dense, nd, r)];
     const int i = r - de.w;
-    if (i >= ((de.z + 127) & ~127)) continue;      // beyond the last 128-row tile: never read
+    if (i >= (de.z + tile_rows - 1) / tile_rows * tile_rows) continue;   // beyond the last token tile: never read
     uint32_t sfbyte = 0u;
     uint2 codes = make_uint2(0, 0);
     if (i < de.z) {
@@ -323,15 +344,107 @@ __device__ __forceinline__ DenseTile dense_tile(const int4* __restrict__ dl, con
   return t;
 }
 
+// One epilogue warp's share of a drained accumulator: this lane's M-side
+// row (m_row: an output dimension for down, a token index within the expert
+// for gate/up) x the 128 accumulator columns 128 hf .. 128 hf + 127.  For
+// down the columns are the tokens n_tok0 + 128 hf + c of the expert.
+template <int MODE>
+__device__ __forceinline__ void dense_epilogue(const DenseParams& p, const DenseTile& tl, const uint32_t (&r)[128],
+                                               int m_row, int n_tok0, int hf, int lane) {
+  const int e = tl.de.x;
+  if (MODE == kDenseDown) {
+    // lane = output dimension drow; columns = tokens 128 hf .. 128 hf + 127 of the tile
+    const int drow = m_row;
+    const int nrows = min(kDenseN, tl.de.z - n_tok0) - hf * 128;
+    const int prow0 = tl.de.y + n_tok0 + hf * 128;               // permutation row of column 0
+    const float gsd = p.gs[2 * p.E + e] *
+                      (p.h_amax_in ? exp2i_f(pow2_tensor_exp(__int_as_float(*p.h_amax_in))) : 1.f);
+#pragma unroll
+    for (int c32 = 0; c32 < 4; ++c32) {
+      if (32 * c32 >= nrows) break;                              // warp-uniform
+      // routing weight x tensor scale of column 32 c32 + lane, broadcast below
+      const float wl = 32 * c32 + lane < nrows
+                           ? (p.wts ? p.wts[p.perm[prow0 + 32 * c32 + lane]] : 1.f) * gsd : 0.f;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const float wv = __shfl_sync(0xffffffffu, wl, c);
+        if (32 * c32 + c < nrows)
+          p.partial[(size_t)(prow0 + 32 * c32 + c) * p.d + drow] = __uint_as_float(r[32 * c32 + c]) * wv;
+      }
+    }
+  } else {
+    // columns 32 bl .. 32 bl + 31: gate (first 16) and up (last 16) of the
+    // channels chb + 16 bl .. chb + 16 bl + 15, one NVFP4 block of h each
+    const int tok = m_row;                           // token of this lane within the expert
+    const bool valid = tok < tl.de.z;
+    const int prow = tl.de.y + tok;                  // permutation row
+    const int hrow = tl.de.w + tok;                  // padded row
+    const float gsx = p.x_amax ? exp2i_f(pow2_tensor_exp(__int_as_float(*p.x_amax))) : 1.f;
+    const float gsg = p.gs[e] * gsx, gsu = p.gs[p.E + e] * gsx;
+    float hmax = 0.f;
+    const int chb = tl.wt * (kDenseN / 2) + hf * 64;
+    uint32_t codes[8];
+    uint32_t sfw = 0u;
+#pragma unroll
+    for (int bl = 0; bl < 4; ++bl) {
+      float hv[16];
+      float am = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float gv = __uint_as_float(r[32 * bl + i]) * gsg;
+        const float uv = __uint_as_float(r[32 * bl + 16 + i]) * gsu;
+        hv[i] = gv / (1.f + expf(-gv)) * uv;
+        am = fmaxf(am, fabsf(hv[i]));
+      }
+      if (p.h32 && valid) {
+        float4* dst = reinterpret_cast<float4*>(p.h32 + (size_t)prow * p.f + chb + 16 * bl);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[i] = make_float4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
+      }
+      if (p.h_amax) {                 // dynamic h scale: quantised by quant_h_dense_kernel
+        if (valid) hmax = fmaxf(hmax, am);
+        continue;
+      }
+      const uint32_t sfbyte = f32x2_to_e4m3x2(0.f, am / 6.0f) & 0xffu;
+      const float sf = e4m3_to_f32(sfbyte);
+      uint32_t w0 = 0u, w1 = 0u;                    // channel i -> nibble i % 8 of word i / 8
+      if (sf > 0.f) {
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) {
+          w0 |= f32x2_to_e2m1x2(hv[i + 1] / sf, hv[i] / sf) << (4 * i);
+          w1 |= f32x2_to_e2m1x2(hv[i + 9] / sf, hv[i + 8] / sf) << (4 * i);
+        }
+      }
+      codes[2 * bl] = w0;
+      codes[2 * bl + 1] = w1;
+      sfw |= sfbyte << (8 * bl);
+    }
+    if (p.h_amax) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) hmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, o));
+      if (lane == 0 && hmax > 0.f) atomicMax(p.h_amax, __float_as_int(hmax));
+      return;
+    }
+    // padding rows (accumulators of zero activations) are written too: zeros
+    uint4* dst = reinterpret_cast<uint4*>(p.hq + (size_t)hrow * (p.f / 2) + (chb >> 1));
+    dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+    dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+    // the four blocks share one 64-wide K group: four consecutive scale bytes
+    const size_t so = sf_rowpair_offset(hrow, chb >> 4, p.f / 64);
+    *reinterpret_cast<uint32_t*>(p.hsf + so) = sfw;
+  }
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __grid_constant__ DenseParams p) {
+  using C = DenseStageCfg<MODE>;
   extern __shared__ __align__(1024) uint8_t dsm_raw[];
   // 1024-byte alignment (shared-window offset) for the 128-byte-swizzled tiles
   uint8_t* dsm = dsm_raw + ((1024u - (smem_u32(dsm_raw) & 1023u)) & 1023u);
-  uint8_t* meta = dsm + kDenseStages * kDenseStageBytes;
+  uint8_t* meta = dsm + C::kStages * C::kStageBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(meta);                 // full[S] empty[S] accf acce done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(meta + kDenseBarBytes);
-  int* svote = reinterpret_cast<int*>(meta + kDenseBarBytes + 16);    // [8] epilogue wait outcomes
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(meta + C::kBarBytes);
+  int* svote = reinterpret_cast<int*>(meta + C::kBarBytes + 16);    // [8] epilogue wait outcomes
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_wait();
@@ -339,12 +452,12 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
   if (nd == 0) { pdl_launch_dependents(); return; }
   const uint32_t bars_s = smem_u32(bars);
   auto full_b = [&](int s) { return bars_s + 8 * s; };
-  auto empty_b = [&](int s) { return bars_s + 8 * (kDenseStages + s); };
-  const uint32_t accf_b = bars_s + 8 * (2 * kDenseStages);
+  auto empty_b = [&](int s) { return bars_s + 8 * (C::kStages + s); };
+  const uint32_t accf_b = bars_s + 8 * (2 * C::kStages);
   const uint32_t acce_b = accf_b + 8;
   const uint32_t done_b = accf_b + 16;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kDenseStages; ++s) { mbar_init(full_b(s), 1); mbar_init(empty_b(s), 1); }
+    for (int s = 0; s < C::kStages; ++s) { mbar_init(full_b(s), 1); mbar_init(empty_b(s), 1); }
     mbar_init(accf_b, 1);
     mbar_init(acce_b, kDenseEpiWarps);
     mbar_init(done_b, 1);
@@ -384,29 +497,29 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
         const uint8_t* sfa = p.sfA + (size_t)(arow >> 7) * p.kstages * kSfaBlock;
         const uint8_t* sfb = p.sfB + (size_t)(brow >> 8) * p.kstages * kSfbBlock;
         for (int ks = 0; ks < p.kstages; ++ks, ++k) {
-          const int s = k % kDenseStages;
-          if (!mbar_wait_spin(empty_b(s), ((k / kDenseStages) & 1) ^ 1, deadline)) {
+          const int s = k % C::kStages;
+          if (!mbar_wait_spin(empty_b(s), ((k / C::kStages) & 1) ^ 1, deadline)) {
             failed = true; set_error(p.err, kErrTimeout); break;
           }
-          const uint32_t st = stage0 + s * kDenseStageBytes;
-          mbar_arrive_expect_tx(full_b(s), kDenseStageBytes);
+          const uint32_t st = stage0 + s * C::kStageBytes;
+          mbar_arrive_expect_tx(full_b(s), C::kStageBytes);
           tma_load_2d(st, &p.tmA, ks * kDenseRowBytes, arow, full_b(s), pol_a);
           tma_load_2d(st + kDenseABytes, &p.tmB, ks * kDenseRowBytes, brow, full_b(s), pol_w);
-          // scale blocks: each read from device memory once (the other three
-          // copies come from L2) into four consecutive replicas
+          // scale blocks: each read from device memory once (replicas, if
+          // any, come from L2)
           const uint8_t* sa = sfa + (size_t)ks * kSfaBlock;
           const uint8_t* sb = sfb + (size_t)ks * kSfbBlock;
-          const uint32_t da = st + kDenseABytes + kDenseBBytes, db = da + kDenseSfaBytes;
+          const uint32_t da = st + kDenseABytes + kDenseBBytes, db = da + C::kSfaBytes;
 #pragma unroll
-          for (int rep = 0; rep < kSfReplicas; ++rep) {
+          for (int rep = 0; rep < C::kCopies; ++rep) {
             bulk_g2s(da + rep * kSfaBlock, sa, kSfaBlock, full_b(s), pol_a);
             bulk_g2s(db + rep * kSfbBlock, sb, kSfbBlock, full_b(s), pol_w);
           }
         }
       }
       // drain: every issued stage must land before the block exits
-      for (int kk = max(0, k - kDenseStages); kk < k; ++kk)
-        mbar_wait_spin(full_b(kk % kDenseStages), (kk / kDenseStages) & 1,
+      for (int kk = max(0, k - C::kStages); kk < k; ++kk)
+        mbar_wait_spin(full_b(kk % C::kStages), (kk / C::kStages) & 1,
                        globaltimer_ns() + (uint64_t)p.wait_timeout_ns);
     }
   } else if (warp == 1) {
@@ -427,22 +540,38 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
         }
         tc_fence_after();
         for (int ks = 0; ks < p.kstages; ++ks, ++k) {
-          const int s = k % kDenseStages;
-          if (!mbar_wait_spin(full_b(s), (k / kDenseStages) & 1, deadline)) {
+          const int s = k % C::kStages;
+          if (!mbar_wait_spin(full_b(s), (k / C::kStages) & 1, deadline)) {
             failed = true; set_error(p.err, kErrTimeout); break;
           }
           tc_fence_after();
-          const uint32_t st = stage0 + s * kDenseStageBytes;
-          const uint32_t sfa_s = st + kDenseABytes + kDenseBBytes, sfb_s = sfa_s + kDenseSfaBytes;
+          const uint32_t st = stage0 + s * C::kStageBytes;
+          const uint32_t sfa_s = st + kDenseABytes + kDenseBBytes, sfb_s = sfa_s + C::kSfaBytes;
           const uint32_t sfa_t = sf_t0 + kDenseSfCols * s, sfb_t = sfa_t + 4 * kDenseMmaPerStage;
+          if (C::kBcast) {
+            // MMA kb: M side unit kb / 2, 16-byte column kb % 2 -> 4 columns;
+            // N side unit kb, columns h = 0, 1 (rows 0..127, 128..255) -> 8 columns
 #pragma unroll
-          for (int pr = 0; pr < kDenseMmaPerStage / 2; ++pr)
-            tc_cp_128x256b(sfa_t + 8 * pr, smem_desc_sf256(sfa_s + kSfGroupBytes * pr,
-                                                           kSfPairUnitsPerStage * kSfGroupBytes));
+            for (int kb = 0; kb < kDenseMmaPerStage; ++kb) {
+              tc_cp_32x128b_warpx4(sfa_t + 4 * kb,
+                                   smem_desc_sf128(sfa_s + kSfGroupBytes * (kb >> 1) + 128 * (kb & 1),
+                                                   kSfPairUnitsPerStage * kSfGroupBytes));
 #pragma unroll
-          for (int kb = 0; kb < kDenseMmaPerStage; ++kb)
-            tc_cp_128x256b(sfb_t + 8 * kb, smem_desc_sf256(sfb_s + kSfGroupBytes * kb,
-                                                           kSfRowpairUnitsPerStage * kSfGroupBytes));
+              for (int h = 0; h < 2; ++h)
+                tc_cp_32x128b_warpx4(sfb_t + 8 * kb + 4 * h,
+                                     smem_desc_sf128(sfb_s + kSfGroupBytes * kb + 128 * h,
+                                                     kSfRowpairUnitsPerStage * kSfGroupBytes));
+            }
+          } else {
+#pragma unroll
+            for (int pr = 0; pr < kDenseMmaPerStage / 2; ++pr)
+              tc_cp_128x256b(sfa_t + 8 * pr, smem_desc_sf256(sfa_s + kSfGroupBytes * pr,
+                                                             kSfPairUnitsPerStage * kSfGroupBytes));
+#pragma unroll
+            for (int kb = 0; kb < kDenseMmaPerStage; ++kb)
+              tc_cp_128x256b(sfb_t + 8 * kb, smem_desc_sf256(sfb_s + kSfGroupBytes * kb,
+                                                             kSfRowpairUnitsPerStage * kSfGroupBytes));
+          }
           const uint64_t adesc = smem_desc_kmajor<kDenseRowBytes>(st);
           const uint64_t bdesc = smem_desc_kmajor<kDenseRowBytes>(st + kDenseABytes);
 #pragma unroll
@@ -495,88 +624,10 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acce_b);
-      const int e = tl.de.x;
-      if (MODE == kDenseDown) {
-        // lane = output dimension drow; columns = tokens 128 hf .. 128 hf + 127 of the tile
-        const int drow = tl.wt * 128 + q * 32 + lane;
-        const int nrows = min(kDenseN, tl.de.z - tl.tt * kDenseN) - hf * 128;
-        const int prow0 = tl.de.y + tl.tt * kDenseN + hf * 128;      // permutation row of column 0
-        const float gsd = p.gs[2 * p.E + e] *
-                          (p.h_amax_in ? exp2i_f(pow2_tensor_exp(__int_as_float(*p.h_amax_in))) : 1.f);
-#pragma unroll
-        for (int c32 = 0; c32 < 4; ++c32) {
-          if (32 * c32 >= nrows) break;                              // warp-uniform
-          // routing weight x tensor scale of column 32 c32 + lane, broadcast below
-          const float wl = 32 * c32 + lane < nrows
-                               ? (p.wts ? p.wts[p.perm[prow0 + 32 * c32 + lane]] : 1.f) * gsd : 0.f;
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float wv = __shfl_sync(0xffffffffu, wl, c);
-            if (32 * c32 + c < nrows)
-              p.partial[(size_t)(prow0 + 32 * c32 + c) * p.d + drow] = __uint_as_float(r[32 * c32 + c]) * wv;
-          }
-        }
-      } else {
-        // columns 32 bl .. 32 bl + 31: gate (first 16) and up (last 16) of the
-        // channels chb + 16 bl .. chb + 16 bl + 15, one NVFP4 block of h each
-        const int tok = q * 32 + lane;                   // token of this lane within the tile
-        const bool valid = tl.tt * 128 + tok < tl.de.z;
-        const int prow = tl.de.y + tl.tt * 128 + tok;    // permutation row
-        const int hrow = tl.de.w + tl.tt * 128 + tok;    // padded row
-        const float gsx = p.x_amax ? exp2i_f(pow2_tensor_exp(__int_as_float(*p.x_amax))) : 1.f;
-        const float gsg = p.gs[e] * gsx, gsu = p.gs[p.E + e] * gsx;
-        float hmax = 0.f;
-        const int chb = tl.wt * (kDenseN / 2) + hf * 64;
-        uint32_t codes[8];
-        uint32_t sfw = 0u;
-#pragma unroll
-        for (int bl = 0; bl < 4; ++bl) {
-          float hv[16];
-          float am = 0.f;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float gv = __uint_as_float(r[32 * bl + i]) * gsg;
-            const float uv = __uint_as_float(r[32 * bl + 16 + i]) * gsu;
-            hv[i] = gv / (1.f + expf(-gv)) * uv;
-            am = fmaxf(am, fabsf(hv[i]));
-          }
-          if (p.h32 && valid) {
-            float4* dst = reinterpret_cast<float4*>(p.h32 + (size_t)prow * p.f + chb + 16 * bl);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_float4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
-          }
-          if (p.h_amax) {                 // dynamic h scale: quantised by quant_h_dense_kernel
-            if (valid) hmax = fmaxf(hmax, am);
-            continue;
-          }
-          const uint32_t sfbyte = f32x2_to_e4m3x2(0.f, am / 6.0f) & 0xffu;
-          const float sf = e4m3_to_f32(sfbyte);
-          uint32_t w0 = 0u, w1 = 0u;                    // channel i -> nibble i % 8 of word i / 8
-          if (sf > 0.f) {
-#pragma unroll
-            for (int i = 0; i < 8; i += 2) {
-              w0 |= f32x2_to_e2m1x2(hv[i + 1] / sf, hv[i] / sf) << (4 * i);
-              w1 |= f32x2_to_e2m1x2(hv[i + 9] / sf, hv[i + 8] / sf) << (4 * i);
-            }
-          }
-          codes[2 * bl] = w0;
-          codes[2 * bl + 1] = w1;
-          sfw |= sfbyte << (8 * bl);
-        }
-        if (p.h_amax) {
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) hmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, o));
-          if (lane == 0 && hmax > 0.f) atomicMax(p.h_amax, __float_as_int(hmax));
-          continue;
-        }
-        // padding rows (accumulators of zero activations) are written too: zeros
-        uint4* dst = reinterpret_cast<uint4*>(p.hq + (size_t)hrow * (p.f / 2) + (chb >> 1));
-        dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-        dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
-        // the four blocks share one 64-wide K group: four consecutive scale bytes
-        const size_t so = sf_rowpair_offset(hrow, chb >> 4, p.f / 64);
-        *reinterpret_cast<uint32_t*>(p.hsf + so) = sfw;
-      }
+      // M side: an output dimension (down) or a token of the expert (gate/up)
+      const int mrow = tl.wt * 128 + q * 32 + lane;
+      const int mtok = tl.tt * 128 + q * 32 + lane;
+      dense_epilogue<MODE>(p, tl, r, MODE == kDenseDown ? mrow : mtok, tl.tt * kDenseN, hf, lane);
     }
   }
   tc_fence_before();
@@ -588,9 +639,218 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
   pdl_launch_dependents();
 }
 
+// ---------------------------------------------------------------------------
+// The same grouped GEMM on CTA pairs (clusters of two, tcgen05 cta_group::2).
+// A pair computes a 256 x 256 tile: M = 256 (128 rows in each CTA: tokens
+// for gate/up, rows of Wd for down), N = 256 (each CTA loads 128 of the B
+// rows; the pair's tensor cores read both halves), so each CTA streams half
+// of the B tile and the B operand bytes per MMA flop halve.  Each CTA loads
+// its own A half, its B half, the scale block of its 128 A rows and the
+// whole N-side scale block (every CTA's accumulator covers all 256 N
+// columns); all four loads of both CTAs complete on the even CTA's `full`
+// barrier.  The even CTA's single MMA thread copies the scales (warpx4
+// broadcast copies, both CTAs) and issues the MMAs; its commits arrive on
+// the `empty`, `accf` and `done` barriers of both CTAs.  Each CTA drains
+// its own TMEM; the 16 epilogue warps of the pair release the accumulator
+// on the even CTA's `acce` barrier.  Token tiles are 256 rows for both GEMMs
+// (the dense rows are padded to 256).
+// ---------------------------------------------------------------------------
+constexpr int kPairStages = 5;
+constexpr int kPairABytes = 128 * kDenseRowBytes;
+constexpr int kPairBBytes = 128 * kDenseRowBytes;
+constexpr int kPairStageBytes = kPairABytes + kPairBBytes + kSfaBlock + kSfbBlock;
+static_assert(kPairStageBytes % 1024 == 0, "pair stages keep the 1024-byte alignment of the swizzled tiles");
+static_assert(kDenseN + kDenseSfCols * kPairStages <= kDenseTmemCols, "pair accumulator + scales exceed TMEM");
+constexpr int kPairBarBytes = (2 * kPairStages + 3) * 8 + 8;
+
+template <int MODE>
+__global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_pair_kernel(const __grid_constant__ DenseParams p) {
+  extern __shared__ __align__(1024) uint8_t dsm_raw[];
+  uint8_t* dsm = dsm_raw + ((1024u - (smem_u32(dsm_raw) & 1023u)) & 1023u);
+  uint8_t* meta = dsm + kPairStages * kPairStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(meta);                 // full[S] empty[S] accf acce done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(meta + kPairBarBytes);
+  int* svote = reinterpret_cast<int*>(meta + kPairBarBytes + 16);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  pdl_wait();
+  const int nd = *p.n_dense;
+  if (nd == 0) { pdl_launch_dependents(); return; }      // both CTAs of a pair read the same nd
+  const uint32_t bars_s = smem_u32(bars);
+  auto full_b = [&](int s) { return bars_s + 8 * s; };
+  auto empty_b = [&](int s) { return bars_s + 8 * (kPairStages + s); };
+  const uint32_t accf_b = bars_s + 8 * (2 * kPairStages);
+  const uint32_t acce_b = accf_b + 8;
+  const uint32_t done_b = accf_b + 16;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPairStages; ++s) { mbar_init(full_b(s), 1); mbar_init(empty_b(s), 1); }
+    mbar_init(accf_b, 1);
+    mbar_init(acce_b, 2 * kDenseEpiWarps);
+    mbar_init(done_b, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc2(smem_u32(tmem_slot), kDenseTmemCols);
+    tmem_relinquish2();
+  }
+  tc_fence_before();
+  cluster_sync();                  // both CTAs' barriers initialised before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t sf_t0 = tmem + kDenseN;
+
+  const int ntiles = p.wt_per_expert * __ldg(p.ntoff + nd);
+  const int G = gridDim.x >> 1, c = blockIdx.x >> 1;
+  const int my_tiles = c < ntiles ? (ntiles - 1 - c) / G + 1 : 0;
+  const uint64_t deadline = globaltimer_ns() + (uint64_t)p.wait_timeout_ns;
+  const uint32_t stage0 = smem_u32(dsm);
+  bool failed = false;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_normal(), pol_a = policy_evict_last();
+      tma_prefetch_desc(&p.tmA);
+      tma_prefetch_desc(&p.tmB2);
+      tma_prefetch_desc(&p.tmSfa);
+      tma_prefetch_desc(&p.tmSfb);
+      int k = 0;
+      for (int it = 0; it < my_tiles && !failed; ++it) {
+        const DenseTile tl = dense_tile(p.dense, p.ntoff, nd, p.wt_per_expert, c + it * G);
+        const int wrow = tl.de.x * p.rows_per_expert + tl.wt * 256;      // weight rows of the tile
+        const int trow = tl.de.w + tl.tt * 256;                          // padded token rows
+        const int arow = (MODE == kDenseGateUp ? trow : wrow) + 128 * (int)rank;
+        const int brow = MODE == kDenseGateUp ? wrow : trow;
+        const int sfa_y = ((arow >> 7) * p.kstages) * 8;                 // + 8 per stage
+        const int sfb_y = ((brow >> 8) * p.kstages) * 16;                // + 16 per stage
+        const int brow_mine = brow + 128 * (int)rank;
+        for (int ks = 0; ks < p.kstages; ++ks, ++k) {
+          const int s = k % kPairStages;
+          if (!mbar_wait_spin(empty_b(s), ((k / kPairStages) & 1) ^ 1, deadline)) {
+            failed = true; set_error(p.err, kErrTimeout); break;
+          }
+          const uint32_t st = stage0 + s * kPairStageBytes;
+          const uint32_t fb = mapa_shared(full_b(s), 0);
+          if (leader) mbar_arrive_expect_tx(full_b(s), 2 * kPairStageBytes);
+          tma_load_2d_pair(st, &p.tmA, ks * kDenseRowBytes, arow, fb, pol_a);
+          tma_load_2d_pair(st + kPairABytes, &p.tmB2, ks * kDenseRowBytes, brow_mine, fb, pol_w);
+          tma_load_2d_pair(st + kPairABytes + kPairBBytes, &p.tmSfa, 0, sfa_y + 8 * ks, fb, pol_a);
+          tma_load_2d_pair(st + kPairABytes + kPairBBytes + kSfaBlock, &p.tmSfb, 0, sfb_y + 16 * ks, fb, pol_w);
+        }
+      }
+      // drain: the even CTA's full barriers count the loads of both CTAs
+      if (leader)
+        for (int kk = max(0, k - kPairStages); kk < k; ++kk)
+          mbar_wait_spin(full_b(kk % kPairStages), (kk / kPairStages) & 1,
+                         globaltimer_ns() + (uint64_t)p.wait_timeout_ns);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && leader) {
+      const uint32_t idesc = idesc_nvf4(kDenseN, 256);
+      int k = 0;
+      for (int it = 0; it < my_tiles && !failed; ++it) {
+        if (!mbar_wait_cluster(acce_b, (it & 1) ^ 1, deadline)) {
+          failed = true; set_error(p.err, kErrTimeout); break;
+        }
+        tc_fence_after();
+        for (int ks = 0; ks < p.kstages; ++ks, ++k) {
+          const int s = k % kPairStages;
+          if (!mbar_wait_spin(full_b(s), (k / kPairStages) & 1, deadline)) {
+            failed = true; set_error(p.err, kErrTimeout); break;
+          }
+          tc_fence_after();
+          const uint32_t st = stage0 + s * kPairStageBytes;
+          const uint32_t sfa_s = st + kPairABytes + kPairBBytes, sfb_s = sfa_s + kSfaBlock;
+          const uint32_t sfa_t = sf_t0 + kDenseSfCols * s, sfb_t = sfa_t + 4 * kDenseMmaPerStage;
+#pragma unroll
+          for (int kb = 0; kb < kDenseMmaPerStage; ++kb) {
+            tc_cp2_32x128b_warpx4(sfa_t + 4 * kb,
+                                  smem_desc_sf128(sfa_s + kSfGroupBytes * (kb >> 1) + 128 * (kb & 1),
+                                                  kSfPairUnitsPerStage * kSfGroupBytes));
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              tc_cp2_32x128b_warpx4(sfb_t + 8 * kb + 4 * h,
+                                    smem_desc_sf128(sfb_s + kSfGroupBytes * kb + 128 * h,
+                                                    kSfRowpairUnitsPerStage * kSfGroupBytes));
+          }
+          const uint64_t adesc = smem_desc_kmajor<kDenseRowBytes>(st);
+          const uint64_t bdesc = smem_desc_kmajor<kDenseRowBytes>(st + kPairABytes);
+#pragma unroll
+          for (int kb = 0; kb < kDenseMmaPerStage; ++kb)
+            tc_mma2_nvf4(tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc, sfa_t + 4 * kb, sfb_t + 8 * kb,
+                         (ks > 0 || kb > 0) ? 1u : 0u);
+          tc_commit2_mc(empty_b(s), 3);
+        }
+        if (failed) break;
+        tc_commit2_mc(accf_b, 3);
+      }
+      // both CTAs learn that every MMA issued (none, possibly) has completed
+      tc_commit2_mc(done_b, 3);
+    }
+    if (lane == 0) mbar_wait_spin(done_b, 0, globaltimer_ns() + (uint64_t)p.wait_timeout_ns);
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2.., both CTAs)
+    const int q = warp & 3;
+    const int ew = warp - 2;
+    const int hf = ew >> 2;
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    const uint32_t acce_leader = mapa_shared(acce_b, 0);
+    for (int it = 0; it < my_tiles && !failed; ++it) {
+      const DenseTile tl = dense_tile(p.dense, p.ntoff, nd, p.wt_per_expert, c + it * G);
+      const bool ok = mbar_wait_spin(accf_b, it & 1, deadline);
+      if (lane == 0) svote[ew] = ok ? 1 : 0;
+      named_bar_sync(2, 32 * kDenseEpiWarps);
+      bool all_ok = true;
+#pragma unroll
+      for (int i = 0; i < kDenseEpiWarps; ++i) all_ok = all_ok && svote[i];
+      named_bar_sync(2, 32 * kDenseEpiWarps);
+      if (!all_ok) {
+        failed = true;
+        if (lane == 0) set_error(p.err, kErrTimeout);
+        break;
+      }
+      tc_fence_after();
+      uint32_t r[128];
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t (&rc)[32] = *reinterpret_cast<uint32_t (*)[32]>(r + 32 * cc);
+        tmem_ld_32x32b_x32(tmem + lane_base + hf * 128 + 32 * cc, rc);
+      }
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acce_leader);
+      const int m_in_tile = 128 * (int)rank + q * 32 + lane;
+      const int mrow = tl.wt * 256 + m_in_tile;           // down: output dimension
+      const int mtok = tl.tt * 256 + m_in_tile;           // gate/up: token of the expert
+      dense_epilogue<MODE>(p, tl, r, MODE == kDenseDown ? mrow : mtok, tl.tt * 256, hf, lane);
+    }
+  }
+  // no CTA leaves (or frees TMEM) while the other may still reach its shared
+  // memory or TMEM: every MMA completed (done), both epilogues drained
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc2(tmem, kDenseTmemCols);
+  }
+  pdl_launch_dependents();
+}
+
+template <int MODE>
+constexpr size_t dense_pair_smem_size() {
+  return 1024 + (size_t)kPairStages * kPairStageBytes + kPairBarBytes + 48;
+}
+
 template <int MODE>
 constexpr size_t dense_smem_size(int) {
-  return 1024 + (size_t)kDenseStages * kDenseStageBytes + kDenseBarBytes + 48;
+  return 1024 + (size_t)DenseStageCfg<MODE>::kStages * DenseStageCfg<MODE>::kStageBytes +
+         DenseStageCfg<MODE>::kBarBytes + 48;
 }
 
 }  // namespace moe

@@ -193,6 +193,21 @@ struct TileShape {
   static constexpr int NR = NT < 2 ? 2 : NT;       // B row pointers held per lane
 };
 
+// h of a down tile is read with ordinary L1-allocating loads after each lane
+// acquired the job's completion counter (no line of a row is read before the
+// row is final, so L1 never holds a stale copy), or else with .cg loads.
+#ifndef MOE_LIGHT_H_L1
+#define MOE_LIGHT_H_L1 1
+#endif
+constexpr bool kLightHCached = MOE_LIGHT_H_L1 != 0;
+
+__device__ __forceinline__ uint4 ldg_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+
 template <int NT, int NR, bool COHERENT>
 __device__ __forceinline__ void load_bchunk(const __half* const (&brow)[NR], int chunk, int c, BPair (&b)[NT]) {
 #pragma unroll
@@ -202,8 +217,8 @@ __device__ __forceinline__ void load_bchunk(const __half* const (&brow)[NR], int
       b[nt].hi = b[nt].lo;
     } else {
       const __half* bp = brow[nt] + (size_t)chunk * kChunkK + c * 16;
-      b[nt].lo = COHERENT ? ldg_cg_v4(bp) : ldg_nc_v4(bp);
-      b[nt].hi = COHERENT ? ldg_cg_v4(bp + 8) : ldg_nc_v4(bp + 8);
+      b[nt].lo = !COHERENT ? ldg_nc_v4(bp) : kLightHCached ? ldg_v4(bp) : ldg_cg_v4(bp);
+      b[nt].hi = !COHERENT ? ldg_nc_v4(bp + 8) : kLightHCached ? ldg_v4(bp + 8) : ldg_cg_v4(bp + 8);
     }
   }
 }
@@ -292,6 +307,13 @@ __global__ void __launch_bounds__(kExpThreads, NT == 4 ? 3 : 4) expert_kernel(Ex
   const int g = lane >> 2, c = lane & 3;
   const int G = (int)gridDim.x, b = (int)blockIdx.x;
 
+  const uint32_t ring_s = smem_u32(smem + warp * RING * SLOT);
+  const uint32_t bars_s = smem_u32(bars_all + warp * RING);
+  const uint64_t pol = policy_evict_first();
+  if (lane == 0) {                              // before the wait: nothing here needs routing
+    for (int i = 0; i < RING; ++i) mbar_init(bars_s + 8 * i, 1);
+    fence_mbar_init();
+  }
   pdl_wait();                                   // routing results of the previous kernel
   // the next layer's router weights go to L2 while this layer streams its
   // experts: each block asks for its slice (a hint; nothing waits on it)
@@ -301,26 +323,20 @@ __global__ void __launch_bounds__(kExpThreads, NT == 4 ? 3 : 4) expert_kernel(Ex
     for (long long o = lo; o < lo + per && o < p.l2_next_bytes; o += 32768)
       bulk_prefetch_l2(p.l2_next + o, (uint32_t)min(32768LL, min(lo + per, p.l2_next_bytes) - o));
   }
-  const int njobs = *p.njobs;
-  const int ngu = njobs * (p.tpe_gu / RT);
-  const int ntot = ngu + njobs * (p.tpe_dn / RT);
-  const int my_tiles = b < ntot ? (ntot - 1 - b) / G + 1 : 0;
-  const uint64_t deadline = globaltimer_ns() + (uint64_t)p.wait_timeout_ns;
   __shared__ int4 s_jobs[kExpSmemJobs];
+  const int* perm = p.perm;
+  const float* wts = p.wts;
+  const int njobs = *p.njobs;
   const int4* jobs = p.jobs;
   if (njobs <= kExpSmemJobs) {
     for (int i = threadIdx.x; i < njobs; i += blockDim.x) s_jobs[i] = p.jobs[i];
     jobs = s_jobs;
   }
   __syncthreads();
-
-  const uint32_t ring_s = smem_u32(smem + warp * RING * SLOT);
-  const uint32_t bars_s = smem_u32(bars_all + warp * RING);
-  const uint64_t pol = policy_evict_first();
-  if (lane == 0) {
-    for (int i = 0; i < RING; ++i) mbar_init(bars_s + 8 * i, 1);
-    fence_mbar_init();
-  }
+  const int ngu = njobs * (p.tpe_gu / RT);
+  const int ntot = ngu + njobs * (p.tpe_dn / RT);
+  const int my_tiles = b < ntot ? (ntot - 1 - b) / G + 1 : 0;
+  const uint64_t deadline = globaltimer_ns() + (uint64_t)p.wait_timeout_ns;
   __syncwarp();
 
   // ---- producer state (lane 0 of each warp): walks this warp's stages in order.
@@ -370,7 +386,7 @@ __global__ void __launch_bounds__(kExpThreads, NT == 4 ? 3 : 4) expert_kernel(Ex
       row[nt] = nullptr;
       if (n < t.nrows) {
         const int r = t.row0 + n;
-        row[nt] = t.down ? p.h16 + (size_t)r * p.f : p.x16 + (size_t)(p.perm[r] / p.topk) * p.d;
+        row[nt] = t.down ? p.h16 + (size_t)r * p.f : p.x16 + (size_t)(perm[r] / p.topk) * p.d;
       }
     }
   };
@@ -405,6 +421,10 @@ __global__ void __launch_bounds__(kExpThreads, NT == 4 ? 3 : 4) expert_kernel(Ex
       if (!__shfl_sync(0xffffffffu, ok, 0)) {
         failed = true;
         if (lane == 0) set_error(p.err, kErrTimeout);
+      } else if (kLightHCached) {
+        // every lane acquires the counter itself, so its ordinary (L1-cached)
+        // loads of h below observe the gate/up tiles' writes
+        (void)ld_acquire(p.gu_done + ti.job);
       }
     }
 
@@ -491,7 +511,7 @@ __global__ void __launch_bounds__(kExpThreads, NT == 4 ? 3 : 4) expert_kernel(Ex
           const int n = nt * 8 + 2 * c + q;
           if (n < ti.nrows) {
             const int r = ti.row0 + n;
-            const float xs = p.xscale[p.perm[r] / p.topk];
+            const float xs = p.xscale[perm[r] / p.topk];
             const float gv = v[q] * gsg * xs;
             const float uv = v[2 + q] * gsu * xs;
             const float hv = gv / (1.f + expf(-gv)) * uv;
@@ -509,9 +529,9 @@ __global__ void __launch_bounds__(kExpThreads, NT == 4 ? 3 : 4) expert_kernel(Ex
           const int n = nt * 8 + 2 * c + q;
           if (n < ti.nrows) {
             const int r = ti.row0 + n;
-            const int pr = p.perm[r];
+            const int pr = perm[r];
             const float hinv = exp2i(-light_h_exp(p.xscale[pr / p.topk], p.hexp[ti.e]));
-            const float wv = (p.wts ? p.wts[pr] : 1.f) * gsd * kScaleUndo * hinv;
+            const float wv = (wts ? wts[pr] : 1.f) * gsd * kScaleUndo * hinv;
             p.partial[(size_t)r * p.d + drow] = v[q] * wv;
             p.partial[(size_t)r * p.d + drow + 8] = v[2 + q] * wv;
           }

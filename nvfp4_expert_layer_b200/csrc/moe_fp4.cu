@@ -72,6 +72,9 @@ struct Workspace {
   uint8_t* hsf = nullptr;
   size_t pad_rows = 0;
   CUtensorMap tm_x{}, tm_h{};    // B operands of the dense GEMMs
+  // CTA-pair GEMMs: h in 128-row boxes, the x and h scale blocks as byte tensors
+  CUtensorMap tm_h2{}, tm_sfx{}, tm_sfh{};
+  bool pair_maps = false;
   __nv_bfloat16* rw3 = nullptr;  // router weights split into three exact bf16 parts [3][E][d]
   CUtensorMap tm_rw3{};
   bool tc_router = false;        // tensor-core router available (tensor maps encoded)
@@ -111,6 +114,10 @@ struct moe_fp4 {
   uint8_t* dsf_gu = nullptr;      // weight scales, 256-row tile layout (sf_rowpair_offset), rows E*2f, K = d
   uint8_t* dsf_dn = nullptr;      // 128-row tile layout (sf_pair_offset), rows E*d, K = f
   CUtensorMap tm_gu{}, tm_down{};
+  // CTA-pair GEMMs: gate/up codes in 128-row boxes, the weight scale blocks as byte tensors
+  CUtensorMap tm_gu2{}, tm_sfgu{}, tm_sfdn{};
+  bool pair_maps = false;
+  int pair_clusters = 0;          // co-resident CTA pairs of the pair GEMM (0: one-CTA GEMMs)
   bool dense_ok = false;          // d, f multiples of 256 and tensor maps available
   bool want_light = true;         // resident weight copies kept by the next load
   bool want_dense = true;
@@ -200,6 +207,21 @@ bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint3
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Scale blocks of the dense GEMMs as a 2-D byte tensor of 256-byte rows,
+// boxes of box_rows rows (no swizzle): a (tile, stage) block of the M-side
+// layout is 8 rows, of the N-side layout 16.
+bool make_map_sf(CUtensorMap* m, const void* base, size_t bytes, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || bytes % 256) return false;
+  const cuuint64_t dims[2] = {256, bytes / 256};
+  const cuuint64_t strides[1] = {256};
+  const cuuint32_t box[2] = {256, box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Byte operand of the dense GEMMs: rows of kDenseRowBytes per pipeline stage.
 bool make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows, uint32_t box_rows) {
   return make_map_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, row_bytes, rows, box_rows, moe::kDenseRowBytes);
@@ -245,6 +267,12 @@ size_t workspace_bytes(const moe_fp4* h, int Tm) {
   add((size_t)Tm * h->d * 2);       // xin
   add((size_t)Tm * h->d * 2);       // xout
   return b;
+}
+
+bool make_ws_pair_maps(const moe_fp4* h, Workspace& w) {
+  return make_map(&w.tm_h2, w.hq, h->f / 2, w.pad_rows, 128) &&
+         make_map_sf(&w.tm_sfx, w.xsf, moe::sf_pair_bytes(w.pad_rows, h->d), 8) &&
+         make_map_sf(&w.tm_sfh, w.hsf, moe::sf_rowpair_bytes(w.pad_rows, h->f), 16);
 }
 
 int ensure_workspace(moe_fp4* h, int Tm, cudaStream_t stream) {
@@ -306,6 +334,7 @@ int ensure_workspace(moe_fp4* h, int Tm, cudaStream_t stream) {
   w.hsf = carve<uint8_t>(cur, moe::sf_rowpair_bytes(w.pad_rows, h->f));
   if (!make_map(&w.tm_x, w.xq, h->d / 2, w.pad_rows, 128) || !make_map(&w.tm_h, w.hq, h->f / 2, w.pad_rows, 256))
     h->dense_ok = false;
+  w.pair_maps = make_ws_pair_maps(h, w);
   if (cudaMemset(w.counters, 0, w.counter_bytes) != cudaSuccess) {
     (void)cudaGetLastError();
     cudaFree(base);
@@ -334,6 +363,48 @@ cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, c
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+// The same with thread-block clusters of cluster_x CTAs along x.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                           bool pdl, unsigned cluster_x, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cluster_x;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+// CTA pairs of a pair-GEMM kernel that fit on the device at once (one CTA per SM).
+int pair_clusters_resident(const void* fn, size_t smem, int sm_count) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (sm_count / 2));
+  cfg.blockDim = dim3(moe::kDenseThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  return std::min(n, sm_count / 2);
 }
 
 size_t permute_smem_bytes(int E) { return moe::permute_smem_ints(E) * 4; }
@@ -471,6 +542,9 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
   // 4-5 (dense class). NVFP4 activations, then the two tensor-core GEMMs
   if (run_dense) {
     const bool dyn = h->act_dynamic;
+    // CTA pairs (256 x 256 tiles on two SMs) when the device fits them
+    const bool pairs = h->pair_clusters > 0 && h->pair_maps && w.pair_maps;
+    const int tok_tile = pairs ? 256 : 128;
     if (dyn) {       // max|x| of the call for the x tensor scale
       MOE_CUDA(cudaMemsetAsync(w.act_amax, 0, 2 * sizeof(int), st));
       MOE_CUDA(launch(moe::amax_bf16_kernel, dim3(std::min<long long>(((long long)T * d / 8 + 255) / 256,
@@ -482,7 +556,8 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
                     w.xq_tok, w.xsf_tok));
     MOE_CUDA(launch(moe::gather_x_dense_kernel, dim3(8 * h->sm_count), dim3(256), 0, st, pdl,
                     (const uint8_t*)w.xq_tok, (const uint8_t*)w.xsf_tok, (const int4*)w.dense_list,
-                    (const int*)w.n_dense, (const int*)w.dense_pad_total, (const int*)w.perm, k, d, w.xq, w.xsf));
+                    (const int*)w.n_dense, (const int*)w.dense_pad_total, (const int*)w.perm, k, d, tok_tile,
+                    w.xq, w.xsf));
     MOE_CUDA(mark(h, 4, st));
     moe::DenseParams dp{};
     dp.tmA = w.tm_x;           // tokens: the M side of the MMA
@@ -511,13 +586,25 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
     dp.partial = w.partial;
     dp.err = h->err;
     dp.wait_timeout_ns = h->wait_timeout_ns;
-    MOE_CUDA(launch(moe::dense_gemm_kernel<moe::kDenseGateUp>, dim3(h->sm_count * kDenseGridPerSm),
-                    dim3(moe::kDenseThreads), moe::dense_smem_size<moe::kDenseGateUp>(E), st, pdl, dp));
+    if (pairs) {
+      moe::DenseParams dq = dp;
+      dq.tmB2 = h->tm_gu2;
+      dq.tmSfa = w.tm_sfx;
+      dq.tmSfb = h->tm_sfgu;
+      dq.ntoff = w.dense_ntoff + (E + 1);      // 256-row token tiles
+      dq.wt_per_expert = 2 * f / 256;
+      MOE_CUDA(launch_cluster(moe::dense_gemm_pair_kernel<moe::kDenseGateUp>, dim3(2 * h->pair_clusters),
+                              dim3(moe::kDenseThreads), moe::dense_pair_smem_size<moe::kDenseGateUp>(), st, pdl,
+                              2u, dq));
+    } else {
+      MOE_CUDA(launch(moe::dense_gemm_kernel<moe::kDenseGateUp>, dim3(h->sm_count * kDenseGridPerSm),
+                      dim3(moe::kDenseThreads), moe::dense_smem_size<moe::kDenseGateUp>(E), st, pdl, dp));
+    }
     MOE_CUDA(mark(h, 5, st));
     if (dyn)         // NVFP4 h with the h tensor scale, once every gate/up tile is done
       MOE_CUDA(launch(moe::quant_h_dense_kernel, dim3(8 * h->sm_count), dim3(256), 0, st, pdl,
                       (const float*)w.h32, (const int4*)w.dense_list, (const int*)w.n_dense,
-                      (const int*)w.dense_pad_total, (const int*)(w.act_amax + 1), f, w.hq, w.hsf));
+                      (const int*)w.dense_pad_total, (const int*)(w.act_amax + 1), f, tok_tile, w.hq, w.hsf));
     moe::DenseParams dp2 = dp;
     dp2.x_amax = nullptr;
     dp2.h_amax = nullptr;
@@ -531,8 +618,20 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
     dp2.rows_per_expert = d;
     dp2.kstages = f / moe::kDenseKStage;
     dp2.kb64 = f / 64;
-    MOE_CUDA(launch(moe::dense_gemm_kernel<moe::kDenseDown>, dim3(h->sm_count * kDenseGridPerSm),
-                    dim3(moe::kDenseThreads), moe::dense_smem_size<moe::kDenseDown>(E), st, pdl, dp2));
+    if (pairs) {
+      moe::DenseParams dq2 = dp2;
+      dq2.tmB2 = w.tm_h2;
+      dq2.tmSfa = h->tm_sfdn;
+      dq2.tmSfb = w.tm_sfh;
+      dq2.ntoff = w.dense_ntoff + (E + 1);
+      dq2.wt_per_expert = d / 256;
+      MOE_CUDA(launch_cluster(moe::dense_gemm_pair_kernel<moe::kDenseDown>, dim3(2 * h->pair_clusters),
+                              dim3(moe::kDenseThreads), moe::dense_pair_smem_size<moe::kDenseDown>(), st, pdl,
+                              2u, dq2));
+    } else {
+      MOE_CUDA(launch(moe::dense_gemm_kernel<moe::kDenseDown>, dim3(h->sm_count * kDenseGridPerSm),
+                      dim3(moe::kDenseThreads), moe::dense_smem_size<moe::kDenseDown>(E), st, pdl, dp2));
+    }
   } else {
     MOE_CUDA(mark(h, 4, st));
     MOE_CUDA(mark(h, 5, st));
@@ -685,8 +784,22 @@ int moe_fp4_create(int E, int top_k, int d, int f, moe_fp4_t** out) {
                   moe::dense_smem_size<moe::kDenseGateUp>(E)) != cudaSuccess ||
         smem_attr((const void*)moe::dense_gemm_kernel<moe::kDenseDown>,
                   moe::dense_smem_size<moe::kDenseDown>(E)) != cudaSuccess ||
+        smem_attr((const void*)moe::dense_gemm_pair_kernel<moe::kDenseGateUp>,
+                  moe::dense_pair_smem_size<moe::kDenseGateUp>()) != cudaSuccess ||
+        smem_attr((const void*)moe::dense_gemm_pair_kernel<moe::kDenseDown>,
+                  moe::dense_pair_smem_size<moe::kDenseDown>()) != cudaSuccess ||
         smem_attr((const void*)moe::router_tc_kernel, moe::router_tc_smem_size()) != cudaSuccess) {
       rc = MOE_FP4_ERR_CUDA; break;
+    }
+    // CTA pairs for the dense GEMMs (MOE_FP4_DENSE_PAIRS=0 keeps one-CTA tiles)
+    {
+      const char* ev = std::getenv("MOE_FP4_DENSE_PAIRS");
+      const bool want_pairs = !(ev && ev[0] == '0');
+      const int c1 = pair_clusters_resident((const void*)moe::dense_gemm_pair_kernel<moe::kDenseGateUp>,
+                                            moe::dense_pair_smem_size<moe::kDenseGateUp>(), h->sm_count);
+      const int c2 = pair_clusters_resident((const void*)moe::dense_gemm_pair_kernel<moe::kDenseDown>,
+                                            moe::dense_pair_smem_size<moe::kDenseDown>(), h->sm_count);
+      h->pair_clusters = want_pairs ? std::min(c1, c2) : 0;
     }
     int nb1 = 0, nb2 = 0, nb4 = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb1, moe::expert_kernel<1>, moe::kExpThreads,
@@ -794,6 +907,10 @@ int moe_fp4_load_experts(moe_fp4_t* h, const moe_fp4_experts* w) {
     if (h->ws.base && (!make_map(&h->ws.tm_x, h->ws.xq, d / 2, h->ws.pad_rows, 128) ||
                        !make_map(&h->ws.tm_h, h->ws.hq, f / 2, h->ws.pad_rows, 256)))
       h->dense_ok = false;
+    h->pair_maps = make_map(&h->tm_gu2, h->dq_gu, d / 2, (uint64_t)E * 2 * f, 128) &&
+                   make_map_sf(&h->tm_sfgu, h->dsf_gu, gu_atoms, 16) &&
+                   make_map_sf(&h->tm_sfdn, h->dsf_dn, dn_atoms, 8);
+    if (h->ws.base) h->ws.pair_maps = make_ws_pair_maps(h, h->ws);
   }
   MOE_CUDA(cudaMemcpy(h->gs, w->gate_gs, sizeof(float) * E, cudaMemcpyDeviceToDevice));
   MOE_CUDA(cudaMemcpy(h->gs + E, w->up_gs, sizeof(float) * E, cudaMemcpyDeviceToDevice));

@@ -33,6 +33,11 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
 __device__ __forceinline__ void tc_cp_128x256b(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" :: "r"(taddr), "l"(sdesc) : "memory");
 }
+// Shared memory (descriptor) -> TMEM: 32 rows x 128 bits (4 columns), row L
+// to lane L of every one of the four lane quarters.
+__device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(sdesc) : "memory");
+}
 // D[128 x N] (+)= A[128 x 64] * B[N x 64]^T, NVFP4 operands with e4m3 scales per 16 (in TMEM).
 __device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
@@ -99,9 +104,21 @@ __device__ __forceinline__ uint64_t smem_desc_sf256(uint32_t saddr, uint32_t sbo
   d |= (uint64_t)1 << 46;
   return d;                                         // layout: SWIZZLE_NONE
 }
-// Instruction descriptor: kind::mxf4nvf4, A/B e2m1, e4m3 scales, fp32 accumulate, M=128, K-major.
-__host__ __device__ constexpr uint32_t idesc_nvf4(int N) {
-  return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | (0u << 23) | ((uint32_t)(128 >> 4) << 24);
+// Scale-factor copy source of 32 rows x 16 bytes, no swizzle: four core
+// matrices of 8 rows x 16 bytes, `sbo` bytes apart (the leading byte offset
+// is unused with one 16-byte column).
+__device__ __forceinline__ uint64_t smem_desc_sf128(uint32_t saddr, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)(128 >> 4) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+  d |= (uint64_t)1 << 46;
+  return d;                                         // layout: SWIZZLE_NONE
+}
+// Instruction descriptor: kind::mxf4nvf4, A/B e2m1, e4m3 scales, fp32 accumulate, K-major;
+// M = 128 (one CTA) or 256 (a CTA pair).
+__host__ __device__ constexpr uint32_t idesc_nvf4(int N, int M = 128) {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | (0u << 23) | ((uint32_t)(M >> 4) << 24);
 }
 
 // ---------------------------------------------------------------- tensor TMA
@@ -114,6 +131,83 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 }
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" :: "l"(map) : "memory");
+}
+
+// ---------------------------------------------------------------- CTA pairs (cta_group::2)
+// A cluster of two CTAs runs one MMA of M = 256 (128 rows in each CTA's
+// TMEM and shared memory) x N (each CTA holding N / 2 rows of B); the even
+// CTA of the pair issues the MMAs and the scale copies for both.
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the same shared-memory offset in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+// every thread of both CTAs: release this CTA's prior work to the cluster, wait for the other CTA
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_alloc2(uint32_t smem_result, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+               :: "r"(smem_result), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish2() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" :: "r"(taddr), "r"(ncols) : "memory");
+}
+// arrive on the mbarrier at `bar` (a shared::cta offset) in every CTA of
+// `mask` once the MMAs issued so far complete
+__device__ __forceinline__ void tc_commit2_mc(uint32_t bar, uint16_t mask) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+               :: "r"(bar), "h"(mask) : "memory");
+}
+__device__ __forceinline__ void tc_cp2_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(sdesc) : "memory");
+}
+__device__ __forceinline__ void tc_mma2_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n}"
+      :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+// Tensor load into this CTA's shared memory whose completion is counted on
+// an mbarrier of either CTA of the pair (`bar` a shared::cluster address);
+// no multicast.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar,
+                                                 uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;"
+      :: "r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar), "l"(policy) : "memory");
+}
+// arrive (release, cluster scope) on an mbarrier of any CTA of the cluster
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" :: "r"(bar_cluster) : "memory");
+}
+// try_wait with acquire at cluster scope (arrivals from the other CTA)
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t phase) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok) : "r"(bar), "r"(phase) : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t phase, uint64_t deadline_ns) {
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait_cluster(bar, phase)) return true;
+    if ((i & 63u) == 0 && globaltimer_ns() > deadline_ns) return false;
+  }
 }
 
 // ---------------------------------------------------------------- NVFP4 conversions
@@ -145,8 +239,10 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
 // the units of a (row tile, stage) are interleaved by group in memory:
 //   block (tile, stage) = [group g (4)][unit j (U)][256 bytes],  U units per stage,
 // and the copy of unit j reads groups at j * 256 + g * U * 256 (the
-// descriptor's stride).  Device memory holds each block once; shared memory
-// holds it four times in a row (kSfReplicas).
+// descriptor's stride).  Device memory holds each block once; for the
+// .128x256b copies shared memory holds it four times in a row (kSfReplicas),
+// while a .32x128b.warpx4 copy reads one 16-byte column h of a unit's four
+// groups and broadcasts it to the four lane quarters itself.
 constexpr int kSfReplicas = 4;
 constexpr int kSfGroupBytes = 256;
 

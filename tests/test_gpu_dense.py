@@ -24,8 +24,16 @@ def _run(cfg, thr, **kw):
     return c
 
 
-def test_dense_tiny_every_expert_dense():
-    # thr = 1: every active expert is dense; each holds <= 4 rows of a 128-row tile
+@pytest.fixture(params=["pairs", "single"])
+def gemm_tiles(request, monkeypatch):
+    """The dense GEMMs on CTA pairs (256 x 256 tiles, the default) or on
+    single CTAs (128-row tiles); the choice is read when a layer is created."""
+    monkeypatch.setenv("MOE_FP4_DENSE_PAIRS", "1" if request.param == "pairs" else "0")
+    return request.param
+
+
+def test_dense_tiny_every_expert_dense(gemm_tiles):
+    # thr = 1: every active expert is dense; each holds <= 4 rows of a token tile
     c = _run(W.CONFIGS["tiny"], thr=1)
     assert c.n_dense_rows == c.cfg.T * c.cfg.k
 
@@ -39,8 +47,8 @@ def test_dense_and_light_classes_small_batch():
     assert 0 < c.n_dense_rows < cfg.T * cfg.k
 
 
-def test_dense_ragged_multi_tile_experts():
-    # ~175 rows per expert: two 128-token tiles, the second ragged
+def test_dense_ragged_multi_tile_experts(gemm_tiles):
+    # ~175 rows per expert: two 128-token tiles (one 256-token pair tile), the second ragged
     cfg = W.custom_config(T=700, d=512, E=8, k=2, f=512, seed=51, router="unit")
     c = _run(cfg, thr=64)
     counts = c.o["counts"]
@@ -48,7 +56,7 @@ def test_dense_ragged_multi_tile_experts():
     assert c.n_dense_rows > 0
 
 
-def test_dense_and_light_classes_in_one_call():
+def test_dense_and_light_classes_in_one_call(gemm_tiles):
     cfg = W.custom_config(T=600, d=1024, E=16, k=4, f=768, seed=52, router="unit")
     c = Case(cfg, thr=150).run_gpu().run_oracle()
     counts = c.o["counts"]
