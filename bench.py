@@ -134,7 +134,7 @@ def measured_peaks():
 
 # Row count from which an expert runs in the dense (tensor-core) class: the
 # library's default, chosen from the measurements in the design notes.
-DENSE_THR = 128
+DENSE_THR = 9
 
 
 def is_dense(cfg, thr=DENSE_THR) -> bool:
@@ -436,11 +436,17 @@ def run_workload(args, cfg, layer, rank, world, local):
         experts_per_input.append(int((c > 0).sum()))
         dense_rows.append(int(c[c >= thr].sum()) if is_dense(cfg, thr) else 0)
     any_dense = is_dense(cfg, thr) and sum(dense_rows) > 0
-    # tensor-bound roofline when most routed rows are in the dense class
-    # (prefill); otherwise the HBM roofline of the whole expert phase (every
-    # kernel that streams expert weights: the light kernels and, for experts
-    # with at least thr rows, the dense class)
-    dense = any_dense and np.mean(dense_rows) >= 0.5 * cfg.T * cfg.k
+    # Which roofline bounds the step: an expert with n routed rows does
+    # 2 * n flops per weight for 0.5625 bytes per weight, so it is tensor-bound
+    # when n exceeds the ridge point (FP4 peak / HBM peak) * 0.5625 / 2 (about
+    # 280 rows on B200).  Prefill (~512 rows per expert): the tensor roofline of
+    # the gate/up GEMM.  Decode workloads: the HBM roofline of the whole expert
+    # phase (every kernel that streams expert weights: the light kernels and,
+    # for experts with at least thr rows, the dense class).
+    hbm_peak, fp4_peak, _ = measured_peaks()
+    ridge_rows = fp4_peak * 1e12 / (hbm_peak * 1e9) * 0.5625 / 2
+    rows_per_expert = cfg.T * cfg.k / max(1.0, float(np.mean(experts_per_input)))
+    dense = any_dense and rows_per_expert >= ridge_rows
     stream = torch.cuda.Stream()
     graphs = []
     with torch.cuda.stream(stream):

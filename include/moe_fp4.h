@@ -34,15 +34,16 @@
  *                            tensor scale 1.0 (sf = e4m3_rn(amax/6),
  *                            q = e2m1_rn(v/sf), decisions in fp32) and the
  *                            expert runs on block-scaled FP4 tensor cores.
- *   The threshold defaults to 128 (environment MOE_FP4_DENSE_THRESHOLD at
- *   create time, or moe_fp4_set_dense_threshold).  The dense class needs d
+ *   The threshold defaults to 9 (environment MOE_FP4_DENSE_THRESHOLD at
+ *   create time, or moe_fp4_set_dense_threshold): an expert with 9 or more
+ *   rows streams its weights faster through the tensor-core class.  The dense class needs d
  *   and f to be multiples of 256 (one 256-element K stage of the tensor-core
  *   pipeline); for other shapes, or if the driver's tensor-map encoder is not
  *   available, every expert runs in the light class whatever its row count.
- *   The dense GEMMs run on CTA pairs (clusters of two SMs, 256 x 256 tiles)
- *   when the device fits them, else on single CTAs (128-row tiles); the
- *   environment variable MOE_FP4_DENSE_PAIRS set to "0" at create time
- *   selects the single-CTA kernels.  Both give results within the same bounds.
+ *   The dense GEMMs run on single CTAs (128-row tiles); the environment
+ *   variable MOE_FP4_DENSE_PAIRS set to "1" at create time selects CTA pairs
+ *   (clusters of two SMs, tcgen05 cta_group::2, 256 x 256 tiles) when the
+ *   device fits them.  Both give results within the same bounds.
  *
  * Conventions
  *   - Every call returns a moe_fp4_status and never aborts the process.

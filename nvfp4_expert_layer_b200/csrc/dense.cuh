@@ -132,12 +132,13 @@ __device__ __forceinline__ float exp2i_f(int e) { return __int_as_float((e + 127
 
 // ---------------------------------------------------------------------------
 // Activation quantiser of the dense class, in two passes.
-// quant_tok_kernel: one warp per token: the bf16 row -> NVFP4 codes
-//   [T][d/2] and one e4m3 scale byte per 16 values [T][d/16] (plain layout).
-// gather_x_dense_kernel: one block per 128-row tile of the padded dense
-//   rows: the codes and scales of token perm[row0 + i] / topk copied into the
-//   padded permutation order (scales assembled into whole sf_pair_offset
-//   units, written with coalesced 16-byte stores).
+// quant_tok_kernel: one thread per (token, 16-value block): the bf16 row ->
+//   NVFP4 codes [T][d/2] and one e4m3 scale byte per 16 values [T][d/16]
+//   (plain layout).
+// gather_x_dense_kernel: the codes and scales of token perm[row0 + i] / topk
+//   copied into the padded permutation order, codes a warp per row over the
+//   whole grid, scales a block per 128-row tile (assembled into whole
+//   sf_pair_offset units, written with coalesced 16-byte stores).
 //   Rows past an expert's count up to its next multiple of tile_rows -- the
 //   rows a token tile of the gate/up GEMM reads (128, or 256 for CTA pairs)
 //   -- are zeros; rows beyond are never read.
@@ -158,38 +159,40 @@ __global__ void __launch_bounds__(256) quant_tok_kernel(const uint16_t* __restri
                                                         uint8_t* __restrict__ xq, uint8_t* __restrict__ xsf) {
   pdl_wait();
   if (*n_dense == 0) { pdl_launch_dependents(); return; }
-  const int lane = threadIdx.x & 31;
   const int nblk = d / 16;
   // dynamic tensor scale gs = 2^e: the values are quantised as v * 2^-e (exact)
   const float inv_gs = x_amax ? exp2i_f(-pow2_tensor_exp(__int_as_float(*x_amax))) : 1.f;
-  for (int t = blockIdx.x * 8 + (threadIdx.x >> 5); t < T; t += gridDim.x * 8) {
-    const uint16_t* src = x + (size_t)t * d;
-    for (int blk = lane; blk < nblk; blk += 32) {
-      const uint4 a = *reinterpret_cast<const uint4*>(src + blk * 16);
-      const uint4 b = *reinterpret_cast<const uint4*>(src + blk * 16 + 8);
-      const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-      float v[16];
+  // one thread per (token, 16-value block); consecutive threads take
+  // consecutive blocks of a row (32-byte loads, 8-byte code stores)
+  const long long units = (long long)T * nblk;
+  for (long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x; u < units;
+       u += (long long)gridDim.x * blockDim.x) {
+    const int t = (int)(u / nblk), blk = (int)(u - (long long)t * nblk);
+    const uint16_t* src = x + (size_t)t * d + blk * 16;
+    const uint4 a = *reinterpret_cast<const uint4*>(src);
+    const uint4 b = *reinterpret_cast<const uint4*>(src + 8);
+    const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    float v[16];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        v[2 * q] = __uint_as_float(wv[q] << 16) * inv_gs;
-        v[2 * q + 1] = __uint_as_float(wv[q] & 0xffff0000u) * inv_gs;
-      }
-      float amax = 0.f;
-#pragma unroll
-      for (int q = 0; q < 16; ++q) amax = fmaxf(amax, fabsf(v[q]));
-      const uint32_t sfbyte = f32x2_to_e4m3x2(0.f, amax / 6.0f) & 0xffu;
-      const float sf = e4m3_to_f32(sfbyte);
-      uint2 codes = make_uint2(0, 0);
-      if (sf > 0.f) {
-        uint32_t c[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) c[q] = f32x2_to_e2m1x2(v[2 * q + 1] / sf, v[2 * q] / sf);
-        codes.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-        codes.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
-      }
-      *reinterpret_cast<uint2*>(xq + (size_t)t * (d / 2) + blk * 8) = codes;
-      xsf[(size_t)t * nblk + blk] = (uint8_t)sfbyte;
+    for (int q = 0; q < 8; ++q) {
+      v[2 * q] = __uint_as_float(wv[q] << 16) * inv_gs;
+      v[2 * q + 1] = __uint_as_float(wv[q] & 0xffff0000u) * inv_gs;
     }
+    float amax = 0.f;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) amax = fmaxf(amax, fabsf(v[q]));
+    const uint32_t sfbyte = f32x2_to_e4m3x2(0.f, amax / 6.0f) & 0xffu;
+    const float sf = e4m3_to_f32(sfbyte);
+    uint2 codes = make_uint2(0, 0);
+    if (sf > 0.f) {
+      uint32_t c[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) c[q] = f32x2_to_e2m1x2(v[2 * q + 1] / sf, v[2 * q] / sf);
+      codes.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
+      codes.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
+    }
+    *reinterpret_cast<uint2*>(xq + (size_t)t * (d / 2) + blk * 8) = codes;
+    xsf[(size_t)t * nblk + blk] = (uint8_t)sfbyte;
   }
   pdl_launch_dependents();
 }
@@ -198,35 +201,39 @@ __global__ void __launch_bounds__(256) gather_x_dense_kernel(
     const uint8_t* __restrict__ xq_tok, const uint8_t* __restrict__ xsf_tok, const int4* __restrict__ dense,
     const int* __restrict__ n_dense, const int* __restrict__ pad_total, const int* __restrict__ perm, int topk,
     int d, int tile_rows, uint8_t* __restrict__ xq, uint8_t* __restrict__ xsf) {
-  __shared__ int s_tok[128];                     // token of each row of the tile, -1 for padding
+  __shared__ int s_tok[128];                     // token of each row of a tile, -1 for padding
   pdl_wait();
   const int nd = *n_dense;
   if (nd == 0) { pdl_launch_dependents(); return; }
-  const int ntile = *pad_total / 128;
+  const int rows = *pad_total;
   const int n16 = d / 32;                        // 16-byte chunks of a code row
   const int npairs = d / 128;                    // scale units per 128-row tile
-  for (int tile = blockIdx.x; tile < ntile; tile += gridDim.x) {
-    // a 128-row tile lies inside one expert: padding is to 256 rows
-    const int4 de = dense[dense_rank_of_padrow(dense, nd, tile * 128)];
+  const int lane = threadIdx.x & 31;
+  // codes: a warp per padded row (every block takes part, however few the
+  // rows), its lanes on consecutive 16-byte chunks
+  const int nwarps = gridDim.x * (blockDim.x >> 5);
+  for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += nwarps) {
+    const int4 de = dense[dense_rank_of_padrow(dense, nd, r)];
+    const int i = r - de.w;
+    if (i >= (de.z + tile_rows - 1) / tile_rows * tile_rows) continue;   // past the last token tile: never read
+    const int t = i < de.z ? perm[de.y + i] / topk : -1;
+    const uint4* src = reinterpret_cast<const uint4*>(xq_tok + (size_t)max(t, 0) * (d / 2));
+    uint4* dst = reinterpret_cast<uint4*>(xq + (size_t)r * (d / 2));
+    for (int ch = lane; ch < n16; ch += 32) dst[ch] = t >= 0 ? src[ch] : make_uint4(0, 0, 0, 0);
+  }
+  // scales: a block per 128-row tile; the 16 bytes of row slot l and 64-group
+  // g hold the 4 scale bytes of rows l, l + 32, l + 64, l + 96 (see
+  // sf_pair_offset), one 16-byte store per (pair, row slot, half)
+  for (int tile = blockIdx.x; tile < rows / 128; tile += gridDim.x) {
+    const int4 de = dense[dense_rank_of_padrow(dense, nd, tile * 128)];   // a tile lies inside one expert
     const int i0 = tile * 128 - de.w;
-    if (i0 >= (de.z + tile_rows - 1) / tile_rows * tile_rows) continue;   // beyond the last token tile: never read
+    if (i0 >= (de.z + tile_rows - 1) / tile_rows * tile_rows) continue;
     __syncthreads();                             // s_tok of the previous tile consumed
     if (threadIdx.x < 128) {
       const int i = i0 + threadIdx.x;
       s_tok[threadIdx.x] = i < de.z ? perm[de.y + i] / topk : -1;
     }
     __syncthreads();
-    // codes: one 16-byte chunk per thread and step, rows in order
-    for (int c = threadIdx.x; c < 128 * n16; c += blockDim.x) {
-      const int r = c / n16, ch = c - r * n16;
-      const int t = s_tok[r];
-      const uint4 v = t >= 0 ? reinterpret_cast<const uint4*>(xq_tok + (size_t)t * (d / 2))[ch]
-                             : make_uint4(0, 0, 0, 0);
-      reinterpret_cast<uint4*>(xq + (size_t)(tile * 128 + r) * (d / 2))[ch] = v;
-    }
-    // scales: the 16 bytes of row slot l and 64-group g hold the 4 scale
-    // bytes of rows l, l + 32, l + 64, l + 96 (see sf_pair_offset), one 16-byte
-    // store per (pair, row slot, half)
     for (int c = threadIdx.x; c < npairs * 64; c += blockDim.x) {
       const int pr = c >> 6, q = c & 63;
       const int l = q >> 1, h = q & 1;
@@ -647,21 +654,38 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
 // of the B tile and the B operand bytes per MMA flop halve.  Each CTA loads
 // its own A half, its B half, the scale block of its 128 A rows and the
 // whole N-side scale block (every CTA's accumulator covers all 256 N
-// columns); all four loads of both CTAs complete on the even CTA's `full`
-// barrier.  The even CTA's single MMA thread copies the scales (warpx4
-// broadcast copies, both CTAs) and issues the MMAs; its commits arrive on
+// columns); all loads of both CTAs complete on the even CTA's `full`
+// barrier.  The even CTA's single MMA thread copies the scales into both
+// CTAs' TMEM (each from its own shared memory) and issues the MMAs; its commits arrive on
 // the `empty`, `accf` and `done` barriers of both CTAs.  Each CTA drains
 // its own TMEM; the 16 epilogue warps of the pair release the accumulator
 // on the even CTA's `acce` barrier.  Token tiles are 256 rows for both GEMMs
 // (the dense rows are padded to 256).
 // ---------------------------------------------------------------------------
-constexpr int kPairStages = 5;
 constexpr int kPairABytes = 128 * kDenseRowBytes;
 constexpr int kPairBBytes = 128 * kDenseRowBytes;
-constexpr int kPairStageBytes = kPairABytes + kPairBBytes + kSfaBlock + kSfbBlock;
-static_assert(kPairStageBytes % 1024 == 0, "pair stages keep the 1024-byte alignment of the swizzled tiles");
-static_assert(kDenseN + kDenseSfCols * kPairStages <= kDenseTmemCols, "pair accumulator + scales exceed TMEM");
-constexpr int kPairBarBytes = (2 * kPairStages + 3) * 8 + 8;
+// Scale copies of the pair kernel: four replicas of each block in shared
+// memory read by .128x256b copies (6 copy instructions a stage, 4 stages of
+// 56 KB), or one copy read by .32x128b.warpx4 broadcasts (12 a stage, 5
+// stages of 38 KB).  The tensor pipe spends about as long on a copy
+// instruction of either shape, so the fewer, larger copies win on B200.
+#ifndef MOE_PAIR_SF_BCAST
+#define MOE_PAIR_SF_BCAST 0
+#endif
+struct PairStageCfg {
+  static constexpr bool kBcast = MOE_PAIR_SF_BCAST != 0;
+  static constexpr int kCopies = kBcast ? 1 : kSfReplicas;
+  static constexpr int kStages = kBcast ? 5 : 4;
+  static constexpr int kSfaBytes = kCopies * kSfaBlock;
+  static constexpr int kSfbBytes = kCopies * kSfbBlock;
+  static constexpr int kStageBytes = kPairABytes + kPairBBytes + kSfaBytes + kSfbBytes;
+  static constexpr int kBarBytes = (2 * kStages + 3) * 8 + 8;
+  static_assert(kStageBytes % 1024 == 0, "pair stages keep the 1024-byte alignment of the swizzled tiles");
+  static_assert(kDenseN + kDenseSfCols * kStages <= kDenseTmemCols, "pair accumulator + scales exceed TMEM");
+};
+constexpr int kPairStages = PairStageCfg::kStages;
+constexpr int kPairStageBytes = PairStageCfg::kStageBytes;
+constexpr int kPairBarBytes = PairStageCfg::kBarBytes;
 
 template <int MODE>
 __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_pair_kernel(const __grid_constant__ DenseParams p) {
@@ -736,8 +760,13 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_pair_kernel(const
           if (leader) mbar_arrive_expect_tx(full_b(s), 2 * kPairStageBytes);
           tma_load_2d_pair(st, &p.tmA, ks * kDenseRowBytes, arow, fb, pol_a);
           tma_load_2d_pair(st + kPairABytes, &p.tmB2, ks * kDenseRowBytes, brow_mine, fb, pol_w);
-          tma_load_2d_pair(st + kPairABytes + kPairBBytes, &p.tmSfa, 0, sfa_y + 8 * ks, fb, pol_a);
-          tma_load_2d_pair(st + kPairABytes + kPairBBytes + kSfaBlock, &p.tmSfb, 0, sfb_y + 16 * ks, fb, pol_w);
+#pragma unroll
+          for (int rep = 0; rep < PairStageCfg::kCopies; ++rep) {   // replicas after the first come from L2
+            tma_load_2d_pair(st + kPairABytes + kPairBBytes + rep * kSfaBlock, &p.tmSfa, 0, sfa_y + 8 * ks, fb,
+                             pol_a);
+            tma_load_2d_pair(st + kPairABytes + kPairBBytes + PairStageCfg::kSfaBytes + rep * kSfbBlock, &p.tmSfb,
+                             0, sfb_y + 16 * ks, fb, pol_w);
+          }
         }
       }
       // drain: the even CTA's full barriers count the loads of both CTAs
@@ -763,18 +792,29 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_pair_kernel(const
           }
           tc_fence_after();
           const uint32_t st = stage0 + s * kPairStageBytes;
-          const uint32_t sfa_s = st + kPairABytes + kPairBBytes, sfb_s = sfa_s + kSfaBlock;
+          const uint32_t sfa_s = st + kPairABytes + kPairBBytes, sfb_s = sfa_s + PairStageCfg::kSfaBytes;
           const uint32_t sfa_t = sf_t0 + kDenseSfCols * s, sfb_t = sfa_t + 4 * kDenseMmaPerStage;
+          if (PairStageCfg::kBcast) {
 #pragma unroll
-          for (int kb = 0; kb < kDenseMmaPerStage; ++kb) {
-            tc_cp2_32x128b_warpx4(sfa_t + 4 * kb,
-                                  smem_desc_sf128(sfa_s + kSfGroupBytes * (kb >> 1) + 128 * (kb & 1),
-                                                  kSfPairUnitsPerStage * kSfGroupBytes));
+            for (int kb = 0; kb < kDenseMmaPerStage; ++kb) {
+              tc_cp2_32x128b_warpx4(sfa_t + 4 * kb,
+                                    smem_desc_sf128(sfa_s + kSfGroupBytes * (kb >> 1) + 128 * (kb & 1),
+                                                    kSfPairUnitsPerStage * kSfGroupBytes));
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
-              tc_cp2_32x128b_warpx4(sfb_t + 8 * kb + 4 * h,
-                                    smem_desc_sf128(sfb_s + kSfGroupBytes * kb + 128 * h,
-                                                    kSfRowpairUnitsPerStage * kSfGroupBytes));
+              for (int h = 0; h < 2; ++h)
+                tc_cp2_32x128b_warpx4(sfb_t + 8 * kb + 4 * h,
+                                      smem_desc_sf128(sfb_s + kSfGroupBytes * kb + 128 * h,
+                                                      kSfRowpairUnitsPerStage * kSfGroupBytes));
+            }
+          } else {
+#pragma unroll
+            for (int pr = 0; pr < kDenseMmaPerStage / 2; ++pr)
+              tc_cp2_128x256b(sfa_t + 8 * pr, smem_desc_sf256(sfa_s + kSfGroupBytes * pr,
+                                                              kSfPairUnitsPerStage * kSfGroupBytes));
+#pragma unroll
+            for (int kb = 0; kb < kDenseMmaPerStage; ++kb)
+              tc_cp2_128x256b(sfb_t + 8 * kb, smem_desc_sf256(sfb_s + kSfGroupBytes * kb,
+                                                              kSfRowpairUnitsPerStage * kSfGroupBytes));
           }
           const uint64_t adesc = smem_desc_kmajor<kDenseRowBytes>(st);
           const uint64_t bdesc = smem_desc_kmajor<kDenseRowBytes>(st + kPairABytes);

@@ -193,21 +193,6 @@ struct TileShape {
   static constexpr int NR = NT < 2 ? 2 : NT;       // B row pointers held per lane
 };
 
-// h of a down tile is read with ordinary L1-allocating loads after each lane
-// acquired the job's completion counter (no line of a row is read before the
-// row is final, so L1 never holds a stale copy), or else with .cg loads.
-#ifndef MOE_LIGHT_H_L1
-#define MOE_LIGHT_H_L1 1
-#endif
-constexpr bool kLightHCached = MOE_LIGHT_H_L1 != 0;
-
-__device__ __forceinline__ uint4 ldg_v4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-  return v;
-}
-
 template <int NT, int NR, bool COHERENT>
 __device__ __forceinline__ void load_bchunk(const __half* const (&brow)[NR], int chunk, int c, BPair (&b)[NT]) {
 #pragma unroll
@@ -217,8 +202,8 @@ __device__ __forceinline__ void load_bchunk(const __half* const (&brow)[NR], int
       b[nt].hi = b[nt].lo;
     } else {
       const __half* bp = brow[nt] + (size_t)chunk * kChunkK + c * 16;
-      b[nt].lo = !COHERENT ? ldg_nc_v4(bp) : kLightHCached ? ldg_v4(bp) : ldg_cg_v4(bp);
-      b[nt].hi = !COHERENT ? ldg_nc_v4(bp + 8) : kLightHCached ? ldg_v4(bp + 8) : ldg_cg_v4(bp + 8);
+      b[nt].lo = COHERENT ? ldg_cg_v4(bp) : ldg_nc_v4(bp);
+      b[nt].hi = COHERENT ? ldg_cg_v4(bp + 8) : ldg_nc_v4(bp + 8);
     }
   }
 }
@@ -421,10 +406,6 @@ __global__ void __launch_bounds__(kExpThreads, NT == 4 ? 3 : 4) expert_kernel(Ex
       if (!__shfl_sync(0xffffffffu, ok, 0)) {
         failed = true;
         if (lane == 0) set_error(p.err, kErrTimeout);
-      } else if (kLightHCached) {
-        // every lane acquires the counter itself, so its ordinary (L1-cached)
-        // loads of h below observe the gate/up tiles' writes
-        (void)ld_acquire(p.gu_done + ti.job);
       }
     }
 

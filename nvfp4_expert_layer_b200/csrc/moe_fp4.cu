@@ -92,7 +92,8 @@ struct Workspace {
 struct moe_fp4 {
   int device = 0;
   int E = 0, k = 0, d = 0, f = 0;
-  int thr = 128;
+  int thr = 9;                    // dense class from 9 rows (measured: the light kernels' 9..32-row jobs
+                                  // stream weights slower than the tensor-core class)
   int sm_count = 0;
   int exp_bps1 = 1, exp_bps2 = 1, exp_bps4 = 1;  // resident blocks per SM of the expert kernels
   int64_t wait_timeout_ns = 2000000000LL;
@@ -542,7 +543,7 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
   // 4-5 (dense class). NVFP4 activations, then the two tensor-core GEMMs
   if (run_dense) {
     const bool dyn = h->act_dynamic;
-    // CTA pairs (256 x 256 tiles on two SMs) when the device fits them
+    // CTA pairs (256 x 256 tiles on two SMs) when requested and the device fits them
     const bool pairs = h->pair_clusters > 0 && h->pair_maps && w.pair_maps;
     const int tok_tile = pairs ? 256 : 128;
     if (dyn) {       // max|x| of the call for the x tensor scale
@@ -551,7 +552,9 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
                                                                      8 * h->sm_count)),
                       dim3(256), 0, st, false, xb, (long long)T * d, (const int*)w.n_dense, w.act_amax));
     }
-    MOE_CUDA(launch(moe::quant_tok_kernel, dim3(std::min((T + 7) / 8, 8 * h->sm_count)), dim3(256), 0, st,
+    MOE_CUDA(launch(moe::quant_tok_kernel,
+                    dim3((unsigned)std::min<long long>(((long long)T * (d / 16) + 255) / 256, 8LL * h->sm_count)),
+                    dim3(256), 0, st,
                     pdl && !dyn, xb, T, d, (const int*)w.n_dense, dyn ? (const int*)w.act_amax : nullptr,
                     w.xq_tok, w.xsf_tok));
     MOE_CUDA(launch(moe::gather_x_dense_kernel, dim3(8 * h->sm_count), dim3(256), 0, st, pdl,
@@ -791,10 +794,11 @@ int moe_fp4_create(int E, int top_k, int d, int f, moe_fp4_t** out) {
         smem_attr((const void*)moe::router_tc_kernel, moe::router_tc_smem_size()) != cudaSuccess) {
       rc = MOE_FP4_ERR_CUDA; break;
     }
-    // CTA pairs for the dense GEMMs (MOE_FP4_DENSE_PAIRS=0 keeps one-CTA tiles)
+    // CTA pairs for the dense GEMMs on request (MOE_FP4_DENSE_PAIRS=1): on B200
+    // the one-CTA GEMMs measured faster, so they are the default
     {
       const char* ev = std::getenv("MOE_FP4_DENSE_PAIRS");
-      const bool want_pairs = !(ev && ev[0] == '0');
+      const bool want_pairs = ev && ev[0] == '1';
       const int c1 = pair_clusters_resident((const void*)moe::dense_gemm_pair_kernel<moe::kDenseGateUp>,
                                             moe::dense_pair_smem_size<moe::kDenseGateUp>(), h->sm_count);
       const int c2 = pair_clusters_resident((const void*)moe::dense_gemm_pair_kernel<moe::kDenseDown>,

@@ -26,8 +26,8 @@ def _run(cfg, thr, **kw):
 
 @pytest.fixture(params=["pairs", "single"])
 def gemm_tiles(request, monkeypatch):
-    """The dense GEMMs on CTA pairs (256 x 256 tiles, the default) or on
-    single CTAs (128-row tiles); the choice is read when a layer is created."""
+    """The dense GEMMs on CTA pairs (256 x 256 tiles) or on single CTAs
+    (128-row tiles, the default); the choice is read when a layer is created."""
     monkeypatch.setenv("MOE_FP4_DENSE_PAIRS", "1" if request.param == "pairs" else "0")
     return request.param
 

@@ -50,16 +50,23 @@ def test_decode1_full_size():
     Case(cfg).run_gpu().run_oracle().check_all()
 
 
-def test_decode64_full_size():
+# thr = 9 is the library's default (the benchmark's configuration: experts
+# with 9 or more rows in the tensor-core class); 128 keeps every expert light.
+@pytest.mark.parametrize("thr", [9, 128])
+def test_decode64_full_size(thr):
     cfg = W.CONFIGS["decode64"]
     with oracle_pool() as pool:
-        Case(cfg, oracle_experts=W.LazyExperts(cfg), map_fn=pool.map).run_gpu().run_oracle().check_all()
+        c = Case(cfg, thr=thr, oracle_experts=W.LazyExperts(cfg), map_fn=pool.map).run_gpu().run_oracle()
+        c.check_all()
+    if thr == 9:
+        assert 0 < c.n_dense_rows < cfg.T * cfg.k
 
 
-def test_verify_full_size_every_token():
+@pytest.mark.parametrize("thr", [9, 128])
+def test_verify_full_size_every_token(thr):
     cfg = W.CONFIGS["verify"]
     with oracle_pool() as pool:
-        Case(cfg, oracle_experts=W.LazyExperts(cfg), map_fn=pool.map).run_gpu().run_oracle().check_all()
+        Case(cfg, thr=thr, oracle_experts=W.LazyExperts(cfg), map_fn=pool.map).run_gpu().run_oracle().check_all()
 
 
 def test_deterministic_repeat():
