@@ -143,10 +143,18 @@ def is_dense(cfg, thr=DENSE_THR) -> bool:
     return cfg.T >= thr and cfg.d % 256 == 0 and cfg.f % 256 == 0
 
 
-def source_digest() -> str:
+# Sources each profiled kernel is compiled from: a recorded DRAM traffic
+# figure stays valid while these files are unchanged.
+KERNEL_SOURCES = {
+    "expert_kernel": ("experts.cuh", "layout.cuh", "ptx.cuh"),
+    "dense_gemm_kernel_gate_up": ("dense.cuh", "tc.cuh", "ptx.cuh"),
+}
+
+
+def source_digest(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "nvfp4_expert_layer_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
+    for fn in sorted(KERNEL_SOURCES[kernel]):
         with open(os.path.join(csrc, fn), "rb") as fh:
             h.update(fn.encode())
             h.update(fh.read())
@@ -163,8 +171,8 @@ def recorded_traffic(kernel: str, workload: str):
             rec = json.load(fh)
     except Exception:
         return None
-    ent = rec.get(f"{kernel}@{workload}") or rec.get(kernel)
-    if not ent or ent.get("source_digest") != source_digest() or ent.get("workload", workload) != workload:
+    ent = rec.get(f"{kernel}@{workload}")
+    if not ent or ent.get("source_digest") != source_digest(kernel) or ent.get("workload", workload) != workload:
         return None
     return ent.get("dram_bytes_per_launch")
 
@@ -339,11 +347,14 @@ def launches_per_step(cfg, thr=DENSE_THR) -> int:
     weight split, router, x staging, top-k and 3 permutation kernels), the
     dense class (quantiser, gather, 2 GEMMs) when T >= thr, the light-class
     expert kernels (the 9..16-row one when T >= 9, the 17..32-row one when
-    T >= 17) and the combine."""
+    T >= 17, each only if a light expert can have that many rows, i.e. the
+    dense class is off or thr is above 9 / 17) and the combine."""
     pairs = cfg.T * cfg.k
     routing = (1 if pairs <= 32 else 5) if cfg.T <= 256 else 7
-    light = 1 + (1 if cfg.T >= 9 else 0) + (1 if cfg.T >= 17 else 0)
-    return routing + (4 if is_dense(cfg, thr) else 0) + light + 1
+    dense = is_dense(cfg, thr)
+    light = 1 + (1 if cfg.T >= 9 and (not dense or thr > 9) else 0) + \
+        (1 if cfg.T >= 17 and (not dense or thr > 17) else 0)
+    return routing + (4 if dense else 0) + light + 1
 
 
 def bf16_ulp_distance(a_bits, b_bits) -> int:

@@ -292,13 +292,6 @@ __global__ void __launch_bounds__(kExpThreads, NT == 4 ? 3 : 4) expert_kernel(Ex
   const int g = lane >> 2, c = lane & 3;
   const int G = (int)gridDim.x, b = (int)blockIdx.x;
 
-  const uint32_t ring_s = smem_u32(smem + warp * RING * SLOT);
-  const uint32_t bars_s = smem_u32(bars_all + warp * RING);
-  const uint64_t pol = policy_evict_first();
-  if (lane == 0) {                              // before the wait: nothing here needs routing
-    for (int i = 0; i < RING; ++i) mbar_init(bars_s + 8 * i, 1);
-    fence_mbar_init();
-  }
   pdl_wait();                                   // routing results of the previous kernel
   // the next layer's router weights go to L2 while this layer streams its
   // experts: each block asks for its slice (a hint; nothing waits on it)
@@ -308,20 +301,26 @@ __global__ void __launch_bounds__(kExpThreads, NT == 4 ? 3 : 4) expert_kernel(Ex
     for (long long o = lo; o < lo + per && o < p.l2_next_bytes; o += 32768)
       bulk_prefetch_l2(p.l2_next + o, (uint32_t)min(32768LL, min(lo + per, p.l2_next_bytes) - o));
   }
-  __shared__ int4 s_jobs[kExpSmemJobs];
-  const int* perm = p.perm;
-  const float* wts = p.wts;
   const int njobs = *p.njobs;
+  const int ngu = njobs * (p.tpe_gu / RT);
+  const int ntot = ngu + njobs * (p.tpe_dn / RT);
+  const int my_tiles = b < ntot ? (ntot - 1 - b) / G + 1 : 0;
+  const uint64_t deadline = globaltimer_ns() + (uint64_t)p.wait_timeout_ns;
+  __shared__ int4 s_jobs[kExpSmemJobs];
   const int4* jobs = p.jobs;
   if (njobs <= kExpSmemJobs) {
     for (int i = threadIdx.x; i < njobs; i += blockDim.x) s_jobs[i] = p.jobs[i];
     jobs = s_jobs;
   }
   __syncthreads();
-  const int ngu = njobs * (p.tpe_gu / RT);
-  const int ntot = ngu + njobs * (p.tpe_dn / RT);
-  const int my_tiles = b < ntot ? (ntot - 1 - b) / G + 1 : 0;
-  const uint64_t deadline = globaltimer_ns() + (uint64_t)p.wait_timeout_ns;
+
+  const uint32_t ring_s = smem_u32(smem + warp * RING * SLOT);
+  const uint32_t bars_s = smem_u32(bars_all + warp * RING);
+  const uint64_t pol = policy_evict_first();
+  if (lane == 0) {
+    for (int i = 0; i < RING; ++i) mbar_init(bars_s + 8 * i, 1);
+    fence_mbar_init();
+  }
   __syncwarp();
 
   // ---- producer state (lane 0 of each warp): walks this warp's stages in order.
@@ -371,7 +370,7 @@ __global__ void __launch_bounds__(kExpThreads, NT == 4 ? 3 : 4) expert_kernel(Ex
       row[nt] = nullptr;
       if (n < t.nrows) {
         const int r = t.row0 + n;
-        row[nt] = t.down ? p.h16 + (size_t)r * p.f : p.x16 + (size_t)(perm[r] / p.topk) * p.d;
+        row[nt] = t.down ? p.h16 + (size_t)r * p.f : p.x16 + (size_t)(p.perm[r] / p.topk) * p.d;
       }
     }
   };
@@ -492,7 +491,7 @@ __global__ void __launch_bounds__(kExpThreads, NT == 4 ? 3 : 4) expert_kernel(Ex
           const int n = nt * 8 + 2 * c + q;
           if (n < ti.nrows) {
             const int r = ti.row0 + n;
-            const float xs = p.xscale[perm[r] / p.topk];
+            const float xs = p.xscale[p.perm[r] / p.topk];
             const float gv = v[q] * gsg * xs;
             const float uv = v[2 + q] * gsu * xs;
             const float hv = gv / (1.f + expf(-gv)) * uv;
@@ -510,9 +509,9 @@ __global__ void __launch_bounds__(kExpThreads, NT == 4 ? 3 : 4) expert_kernel(Ex
           const int n = nt * 8 + 2 * c + q;
           if (n < ti.nrows) {
             const int r = ti.row0 + n;
-            const int pr = perm[r];
+            const int pr = p.perm[r];
             const float hinv = exp2i(-light_h_exp(p.xscale[pr / p.topk], p.hexp[ti.e]));
-            const float wv = (wts ? wts[pr] : 1.f) * gsd * kScaleUndo * hinv;
+            const float wv = (p.wts ? p.wts[pr] : 1.f) * gsd * kScaleUndo * hinv;
             p.partial[(size_t)r * p.d + drow] = v[q] * wv;
             p.partial[(size_t)r * p.d + drow + 8] = v[2 + q] * wv;
           }

@@ -676,12 +676,13 @@ int run_forward(moe_fp4* h, const void* x, int T, const float* rw, void* out, cu
   if (light_ok) {
     MOE_CUDA(launch(moe::expert_kernel<1>, dim3(h->sm_count * h->exp_bps1), dim3(moe::kExpThreads),
                     kExpSmem1, st, pdl, ep1));
-    // jobs of 9..16 (17..32) rows need an expert with at least 9 (17) rows,
-    // i.e. T >= 9 (T >= 17)
-    if (T >= 9)
+    // jobs of 9..16 (17..32) rows need a light expert with at least 9 (17)
+    // rows: T >= 9 (T >= 17), and a dense threshold above 9 (17) when the
+    // dense class runs (every light expert has fewer than thr rows)
+    if (T >= 9 && (!run_dense || thr > 9))
       MOE_CUDA(launch(moe::expert_kernel<2>, dim3(h->sm_count * h->exp_bps2), dim3(moe::kExpThreads),
                       kExpSmem2, st, pdl, ep2));
-    if (T >= 17)
+    if (T >= 17 && (!run_dense || thr > 17))
       MOE_CUDA(launch(moe::expert_kernel<4>, dim3(h->sm_count * h->exp_bps4), dim3(moe::kExpThreads),
                       kExpSmem4, st, pdl, ep4));
   }
