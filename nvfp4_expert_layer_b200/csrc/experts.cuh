@@ -40,10 +40,25 @@ namespace moe {
 
 constexpr int kExpWarps = 4;
 constexpr int kExpThreads = kExpWarps * 32;
-constexpr int kExpSC = 4;          // 64-wide K chunks per bulk-copy stage (2304 bytes)
-constexpr int kExpRing = 4;        // bulk-copy stage slots per warp (RT row tiles share RT slots)
+#ifndef MOE_EXP_SC
+#define MOE_EXP_SC 4
+#endif
+#ifndef MOE_EXP_RING
+#define MOE_EXP_RING 4
+#endif
+constexpr int kExpSC = MOE_EXP_SC;      // 64-wide K chunks per bulk-copy stage (4: 2304 bytes)
+constexpr int kExpRing = MOE_EXP_RING;  // bulk-copy stage slots per warp (RT row tiles share RT slots)
+static_assert(kExpSC % 2 == 0 && (kExpRing & (kExpRing - 1)) == 0 && kExpRing >= 4, "ring shape");
 constexpr int kExpSB = kExpSC * kChunkBytes;
-constexpr int kExpSmemJobs = 512;  // job table copied to shared memory when it fits
+// Resident blocks per SM of the 1- and 2-n-tile kernels (registers capped by
+// __launch_bounds__); with 5 the job table and the reduction buffer shrink so
+// that five blocks' shared memory fits an SM.
+#ifndef MOE_EXP_BLOCKS
+#define MOE_EXP_BLOCKS 4
+#endif
+constexpr int kExpBlocks = MOE_EXP_BLOCKS;
+constexpr int kExpSmemJobs = kExpBlocks > 4 ? 64 : 512;  // job table copied to shared memory when it fits
+constexpr int kExpRedBufs = kExpBlocks > 4 ? 1 : 2;      // cross-warp reduction buffers (by tile parity)
 // fp32 MMA accumulators per (row tile, n-tile): the four K steps of a chunk
 // chain into one (the chains of the row tiles and n-tiles interleave).
 constexpr int kAccK = 1;
@@ -278,7 +293,7 @@ __device__ __forceinline__ void mma_stage_jit(uint32_t st, int nch, int lane, in
 // control and the epilogue barrier.  A job's weights are streamed once per
 // job, so the 32-row jobs stream an expert with up to 32 rows once.
 template <int NT>
-__global__ void __launch_bounds__(kExpThreads, NT == 4 ? 3 : 4) expert_kernel(ExpertParams p) {
+__global__ void __launch_bounds__(kExpThreads, NT == 4 ? 3 : kExpBlocks) expert_kernel(ExpertParams p) {
   constexpr int RT = TileShape<NT>::RT;
   constexpr int U = TileShape<NT>::U;
   constexpr int NR = TileShape<NT>::NR;
@@ -462,8 +477,10 @@ __global__ void __launch_bounds__(kExpThreads, NT == 4 ? 3 : 4) expert_kernel(Ex
       }
     }
 
-    // ---- cross-warp reduction of the tile (buffer alternates by tile parity)
-    float* red = red_all + (it & 1) * (kExpWarps * U * 32 * 4);
+    // ---- cross-warp reduction of the tile (buffer alternates by tile parity;
+    // with one buffer the previous tile's readers finish first)
+    if (kExpRedBufs == 1 && it > 0) __syncthreads();
+    float* red = red_all + (kExpRedBufs == 1 ? 0 : (it & 1)) * (kExpWarps * U * 32 * 4);
 #pragma unroll
     for (int u = 0; u < U; ++u)
 #pragma unroll
@@ -547,7 +564,7 @@ __global__ void __launch_bounds__(kExpThreads, NT == 4 ? 3 : 4) expert_kernel(Ex
 template <int NT>
 constexpr size_t expert_smem_size() {
   return (size_t)kExpWarps * kExpRing * kExpSB + (size_t)kExpWarps * kExpRing * 8 +
-         (size_t)2 * kExpWarps * TileShape<NT>::U * 32 * 4 * 4;
+         (size_t)kExpRedBufs * kExpWarps * TileShape<NT>::U * 32 * 4 * 4;
 }
 
 }  // namespace moe
