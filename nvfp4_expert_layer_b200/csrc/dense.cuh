@@ -822,13 +822,13 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_pair_kernel(const
           for (int kb = 0; kb < kDenseMmaPerStage; ++kb)
             tc_mma2_nvf4(tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc, sfa_t + 4 * kb, sfb_t + 8 * kb,
                          (ks > 0 || kb > 0) ? 1u : 0u);
-          tc_commit2_mc(empty_b(s), 3);
+          tc_commit2_both(empty_b(s));
         }
         if (failed) break;
-        tc_commit2_mc(accf_b, 3);
+        tc_commit2_both(accf_b);
       }
       // both CTAs learn that every MMA issued (none, possibly) has completed
-      tc_commit2_mc(done_b, 3);
+      tc_commit2_both(done_b);
     }
     if (lane == 0) mbar_wait_spin(done_b, 0, globaltimer_ns() + (uint64_t)p.wait_timeout_ns);
     __syncwarp();

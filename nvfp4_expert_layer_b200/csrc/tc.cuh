@@ -162,11 +162,16 @@ __device__ __forceinline__ void tmem_relinquish2() {
 __device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" :: "r"(taddr), "r"(ncols) : "memory");
 }
-// arrive on the mbarrier at `bar` (a shared::cta offset) in every CTA of
-// `mask` once the MMAs issued so far complete
-__device__ __forceinline__ void tc_commit2_mc(uint32_t bar, uint16_t mask) {
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
-               :: "r"(bar), "h"(mask) : "memory");
+// arrive on the mbarrier at `bar` (a shared::cluster address: this CTA's or
+// the other CTA's of the pair) once the MMAs issued so far complete
+__device__ __forceinline__ void tc_commit2(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+               :: "r"(bar) : "memory");
+}
+// the same arrival on the barrier at offset `bar` in both CTAs of the pair
+__device__ __forceinline__ void tc_commit2_both(uint32_t bar) {
+  tc_commit2(bar);
+  tc_commit2(mapa_shared(bar, 1));
 }
 __device__ __forceinline__ void tc_cp2_128x256b(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::2.128x256b [%0], %1;" :: "r"(taddr), "l"(sdesc) : "memory");
