@@ -634,6 +634,7 @@ def run_reference(args, rank):
     sample = (f"per step: one routed (token, expert) pair of the {cfg.name} workload restricted to "
               f"{REF_BLOCK} of the f={cfg.f} FFN channels ({per_step_tokens:.6f} token)")
     conf = config_dict(cfg, args.gpus)
+    conf["dense_threshold"] = args.thr
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
