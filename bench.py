@@ -137,6 +137,16 @@ def measured_peaks():
 DENSE_THR = 9
 
 
+def tensor_bound(cfg, experts_touched: float) -> bool:
+    """Whether the step is bound by the FP4 tensor cores rather than HBM: the
+    routed rows per touched expert reach the ridge point, (FP4 peak / HBM
+    peak) * 0.5625 bytes per weight / 2 flops per weight and row (about 280
+    rows with the measured B200 peaks)."""
+    hbm_peak, fp4_peak, _ = measured_peaks()
+    ridge_rows = fp4_peak * 1e12 / (hbm_peak * 1e9) * 0.5625 / 2
+    return cfg.T * cfg.k / max(1.0, experts_touched) >= ridge_rows
+
+
 def is_dense(cfg, thr=DENSE_THR) -> bool:
     """Whether the workload's experts may run in the dense class (T >= thr and
     the shapes the tensor-core path supports)."""
@@ -454,10 +464,7 @@ def run_workload(args, cfg, layer, rank, world, local):
     # the gate/up GEMM.  Decode workloads: the HBM roofline of the whole expert
     # phase (every kernel that streams expert weights: the light kernels and,
     # for experts with at least thr rows, the dense class).
-    hbm_peak, fp4_peak, _ = measured_peaks()
-    ridge_rows = fp4_peak * 1e12 / (hbm_peak * 1e9) * 0.5625 / 2
-    rows_per_expert = cfg.T * cfg.k / max(1.0, float(np.mean(experts_per_input)))
-    dense = any_dense and rows_per_expert >= ridge_rows
+    dense = any_dense and tensor_bound(cfg, float(np.mean(experts_per_input)))
     stream = torch.cuda.Stream()
     graphs = []
     with torch.cuda.stream(stream):
